@@ -1,0 +1,160 @@
+"""opt2s oracle: TEST INFRASTRUCTURE ONLY.
+
+A ctypes front end to ``opt2s_oracle.c``, the plain single-threaded CPU
+restatement of the 32-bit two-state optimizer update (Adam/AdamW, AdEMAMix).
+Only the tests, the entry module's ``smoke()`` and the benchmark's CPU
+baseline / reference legs may import this package; the library under
+``elementwise_optimizer_b200`` never does, and the two share no code.
+
+What it computes and where each step comes from is stated in the header of
+``opt2s_oracle.c`` (bitsandbytes issue "Investigate a 256-thread SM103 path
+for small 32-bit optimizer tensors", sections "Problem", "Scope" and
+"Correctness oracle"; Kingma & Ba 2015 Algorithm 1; Loshchilov & Hutter 2019
+Algorithm 2; Pagliardini et al. 2024 Algorithm 1).
+
+Every function here was pinned by ``tests/test_oracle_pins.py`` against
+values fixed by something other than the oracle itself (library optimizers in
+float64, closed forms, invariants, numpy/ml_dtypes conversions).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "opt2s_oracle.c")
+_LIB = os.path.join(_HERE, "libopt2s_oracle.so")
+
+# Strict IEEE fp32: no contraction into FMA, no fast-math, SSE scalar float.
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+          "-fno-fast-math", "-fexcess-precision=standard", "-mfpmath=sse",
+          "-msse2"]
+
+ALGO = {"adam": 0, "ademamix": 1}
+DTYPE = {"f32": 0, "f16": 1, "bf16": 2}
+_ITEMSIZE = {"f32": 4, "f16": 2, "bf16": 2}
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (if missing or older than its source).
+
+    ``OPT2S_ORACLE_LIB`` names a prebuilt library to load instead; the
+    mutation test uses it to check that the pins reject broken oracles."""
+    override = os.environ.get("OPT2S_ORACLE_LIB")
+    if override:
+        return override
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + ".tmp"
+    subprocess.run(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    i64, i32, f32, f64, vp = (ctypes.c_int64, ctypes.c_int, ctypes.c_float,
+                              ctypes.c_double, ctypes.c_void_p)
+    lib.oracle_step_f32.argtypes = [i32, i32, i32, f32, f32, f32, f32, f32,
+                                    f32, f32, i32, vp, vp, vp, vp, i64]
+    lib.oracle_step_f32.restype = i32
+    lib.oracle_step_f64.argtypes = [i32, i32, f64, f64, f64, f64, f64, f64,
+                                    f64, i32, vp, vp, vp, vp, vp, i64]
+    lib.oracle_step_f64.restype = i32
+    lib.oracle_bias_correction.argtypes = [f32, i32]
+    lib.oracle_bias_correction.restype = f32
+    lib.oracle_decay_factor.argtypes = [f32, f32]
+    lib.oracle_decay_factor.restype = f32
+    lib.oracle_narrow_array.argtypes = [i32, vp, vp, i64]
+    lib.oracle_narrow_array.restype = i32
+    lib.oracle_widen_array.argtypes = [i32, vp, vp, i64]
+    lib.oracle_widen_array.restype = i32
+    _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray | None) -> int | None:
+    if a is None:
+        return None
+    if not a.flags["C_CONTIGUOUS"]:
+        raise ValueError("oracle arrays must be C-contiguous")
+    return a.ctypes.data
+
+
+def step_f32(param: np.ndarray, grad: np.ndarray, state1: np.ndarray,
+             state2: np.ndarray, *, dtype: str, algo: str, step: int,
+             lr: float, beta1: float, beta2: float, eps: float,
+             beta3: float = 0.0, alpha: float = 0.0,
+             weight_decay: float = 0.0, skip_zeros: bool = False) -> None:
+    """One fp32 optimizer step over one tensor, in place.
+
+    ``param``/``grad`` hold the storage bits of ``dtype`` ('f32', 'f16',
+    'bf16'; any numpy dtype of the right item size); ``state1`` holds m
+    (Adam) or [m1 | m2] (AdEMAMix) as float32; ``state2`` holds v.
+    """
+    n = param.size
+    if grad.size != n or param.itemsize != _ITEMSIZE[dtype] or \
+            grad.itemsize != _ITEMSIZE[dtype]:
+        raise ValueError("param/grad size or item size mismatch")
+    want1 = 2 * n if algo == "ademamix" else n
+    if state1.dtype != np.float32 or state2.dtype != np.float32 or \
+            state1.size != want1 or state2.size != n:
+        raise ValueError("state arrays must be float32 of the right length")
+    rc = _load().oracle_step_f32(
+        ALGO[algo], DTYPE[dtype], int(bool(skip_zeros)), lr, beta1, beta2,
+        beta3, alpha, eps, weight_decay, int(step), _ptr(param), _ptr(grad),
+        _ptr(state1), _ptr(state2), n)
+    if rc != 0:
+        raise ValueError(f"oracle_step_f32 rejected its arguments ({rc})")
+
+
+def step_f64(param: np.ndarray, grad: np.ndarray, m: np.ndarray,
+             v: np.ndarray, m2: np.ndarray | None = None, *, algo: str,
+             step: int, lr: float, beta1: float, beta2: float, eps: float,
+             beta3: float = 0.0, alpha: float = 0.0,
+             weight_decay: float = 0.0, skip_zeros: bool = False) -> None:
+    """The float64 shadow of ``step_f32`` (same definitions, all in double)."""
+    arrs = [param, grad, m, v] + ([m2] if m2 is not None else [])
+    for a in arrs:
+        if a.dtype != np.float64 or a.size != param.size:
+            raise ValueError("shadow arrays must be float64 of equal size")
+    rc = _load().oracle_step_f64(
+        ALGO[algo], int(bool(skip_zeros)), lr, beta1, beta2, beta3, alpha,
+        eps, weight_decay, int(step), _ptr(param), _ptr(grad), _ptr(m),
+        _ptr(m2), _ptr(v), param.size)
+    if rc != 0:
+        raise ValueError(f"oracle_step_f64 rejected its arguments ({rc})")
+
+
+def bias_correction(beta: float, t: int) -> float:
+    return _load().oracle_bias_correction(beta, t)
+
+
+def decay_factor(lr: float, wd: float) -> float:
+    return _load().oracle_decay_factor(lr, wd)
+
+
+def narrow(x: np.ndarray, dtype: str) -> np.ndarray:
+    """float32 -> fp16/bf16 bit patterns (uint16), round-to-nearest-even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint16)
+    _load().oracle_narrow_array(DTYPE[dtype], _ptr(x), _ptr(out), x.size)
+    return out
+
+
+def widen(h: np.ndarray, dtype: str) -> np.ndarray:
+    """fp16/bf16 bit patterns (uint16) -> float32, exact."""
+    h = np.ascontiguousarray(h).view(np.uint16)
+    out = np.empty(h.shape, np.float32)
+    _load().oracle_widen_array(DTYPE[dtype], _ptr(h), _ptr(out), h.size)
+    return out

@@ -1,0 +1,310 @@
+/*
+ * opt2s oracle -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, single-threaded CPU restatement of the 32-bit two-state
+ * optimizer update (Adam/AdamW and AdEMAMix), used to check the CUDA path.
+ * Only the test suite, the smoke check of the entry module and the CPU
+ * baseline / reference legs of the benchmark may load it.  The product path
+ * never calls it, and it shares no code, header, table or constant with the
+ * CUDA library: every function below is written out here from the published
+ * definitions.
+ *
+ * Sources of what it computes:
+ *   [issue]    bitsandbytes issue "Investigate a 256-thread SM103 path for
+ *              small 32-bit optimizer tensors":
+ *                section "Problem"            -- the two-state 32-bit update,
+ *                                                32-bit (fp32) state;
+ *                section "Scope"              -- decoupled weight decay is
+ *                                                applied before the Adam /
+ *                                                AdEMAMix update;
+ *                section "Correctness oracle" -- variants ADAM/AdamW and
+ *                                                ADEMAMIX, FP16/BF16/FP32
+ *                                                param+grad storage, weight
+ *                                                decay and skip_zeros flags,
+ *                                                gradient left unchanged.
+ *   [Adam]     Kingma & Ba, "Adam: A Method for Stochastic Optimization",
+ *              ICLR 2015, Algorithm 1 (moments, bias correction, eps outside
+ *              the square root).
+ *   [AdamW]    Loshchilov & Hutter, "Decoupled Weight Decay Regularization",
+ *              ICLR 2019, Algorithm 2 (p <- p - lr*wd*p, decoupled from the
+ *              gradient moments).
+ *   [AdEMAMix] Pagliardini, Ablin & Grangier, "The AdEMAMix Optimizer:
+ *              Better, Faster, Older", 2024, Algorithm 1 (a second, slow EMA
+ *              m2 with rate beta3, not bias-corrected, mixed in with weight
+ *              alpha).
+ *   [IEEE754]  IEEE 754-2008, section 4.3.1 (roundTiesToEven) and 3.6
+ *              (binary16 format); bfloat16 is the upper half of binary32.
+ *
+ * Readings where the sources leave a step open (each one is also listed in
+ * the design notes of the repository):
+ *   - fp32 arithmetic, every operation rounded to fp32 in the order written
+ *     below, with no fused multiply-add (built with -ffp-contract=off) and no
+ *     flush-to-zero (the MXCSR FTZ/DAZ bits are cleared for the call).
+ *   - bias corrections bc1 = 1 - beta1^t, bc2 = 1 - beta2^t and the decay
+ *     factor 1 - lr*wd are evaluated in double and rounded to fp32 once.
+ *   - skip_zeros: an element whose gradient compares equal to zero (+0 or -0)
+ *     is left wholly unchanged: param, all moments, and no weight decay.
+ *   - AdEMAMix state1 holds [m1(0..n) | m2(0..n)], 2*n floats.
+ *   - fp16/bf16 params are widened exactly and narrowed with
+ *     round-to-nearest-even; state is always fp32.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <xmmintrin.h>
+
+#define OR_ADAM 0
+#define OR_ADEMAMIX 1
+#define OR_F32 0
+#define OR_F16 1
+#define OR_BF16 2
+
+/* ------------------------------------------------------------------------ */
+/* Storage conversions, written from the format definitions [IEEE754].       */
+/* ------------------------------------------------------------------------ */
+
+/* Split a finite, nonzero |x| (as binary32 bits without sign) into an exact
+ * integer significand M and exponent k with |x| = M * 2^k. */
+static void split_f32(uint32_t mag, uint64_t *M, int *k)
+{
+    uint32_t e = mag >> 23, f = mag & 0x7fffffu;
+    if (e == 0) { *M = f; *k = -149; }                  /* subnormal */
+    else        { *M = f | 0x800000u; *k = (int)e - 150; }
+}
+
+static int bit_length(uint64_t v)
+{
+    int n = 0;
+    while (v) { n++; v >>= 1; }
+    return n;
+}
+
+/* Round |x| = M*2^k to the nearest multiple of 2^Q, ties to an even multiple.
+ * Returns the multiple count. */
+static uint64_t round_to_quantum(uint64_t M, int k, int Q)
+{
+    int s = Q - k;
+    if (s <= 0) return M << (-s);                       /* already exact */
+    if (s >= 64) return 0;                              /* far below half a quantum */
+    uint64_t count = M >> s;
+    uint64_t rem = M & ((1ull << s) - 1);
+    uint64_t half = 1ull << (s - 1);
+    if (rem > half || (rem == half && (count & 1))) count++;
+    return count;
+}
+
+/* Narrow binary32 -> a smaller binary format with `fbits` fraction bits,
+ * exponent bias `bias`, round-to-nearest-even.  In that format a finite value
+ * is count * 2^Q with Q = max(floor(log2|x|) - fbits, 1 - bias - fbits), and
+ * its bit pattern (sign aside) is (Q - Qmin) * 2^fbits + count; the same
+ * formula covers subnormals, normals, the carry into the next binade, and the
+ * carry into the infinity pattern. */
+static uint32_t narrow_rne(float x, int fbits, int bias, uint32_t inf_bits,
+                           uint32_t qnan_bits, int total_bits)
+{
+    uint32_t u;
+    memcpy(&u, &x, sizeof u);
+    uint32_t sign = (u >> 31) << (total_bits - 1);
+    uint32_t mag = u & 0x7fffffffu;
+    if (mag > 0x7f800000u) return sign | qnan_bits;     /* NaN */
+    if (mag == 0x7f800000u) return sign | inf_bits;     /* infinity */
+    if (mag == 0) return sign;                          /* signed zero */
+    uint64_t M;
+    int k;
+    split_f32(mag, &M, &k);
+    int log2x = k + bit_length(M) - 1;                  /* floor(log2|x|) */
+    int Qmin = 1 - bias - fbits;
+    int Q = log2x - fbits;
+    if (Q < Qmin) Q = Qmin;
+    uint64_t count = round_to_quantum(M, k, Q);
+    uint64_t bits = (uint64_t)(Q - Qmin) * (1ull << fbits) + count;
+    if (bits >= inf_bits) return sign | inf_bits;       /* overflow */
+    return sign | (uint32_t)bits;
+}
+
+uint16_t oracle_f32_to_f16(float x)
+{
+    return (uint16_t)narrow_rne(x, 10, 15, 0x7c00u, 0x7e00u, 16);
+}
+
+uint16_t oracle_f32_to_bf16(float x)
+{
+    return (uint16_t)narrow_rne(x, 7, 127, 0x7f80u, 0x7fc0u, 16);
+}
+
+float oracle_f16_to_f32(uint16_t h)
+{
+    int sign = h >> 15, e = (h >> 10) & 0x1f, f = h & 0x3ff;
+    double mag;
+    if (e == 0x1f) mag = f ? NAN : INFINITY;
+    else if (e == 0) mag = ldexp((double)f, -24);       /* subnormal: f * 2^-24 */
+    else mag = ldexp((double)(1024 + f), e - 25);       /* (1.f) * 2^(e-15) */
+    return (float)(sign ? -mag : mag);                  /* exact in binary32 */
+}
+
+float oracle_bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;                     /* bf16 = top half of binary32 */
+    float x;
+    memcpy(&x, &u, sizeof x);
+    return x;
+}
+
+static float load_param(const void *p, int dtype, int64_t i)
+{
+    if (dtype == OR_F32) return ((const float *)p)[i];
+    if (dtype == OR_F16) return oracle_f16_to_f32(((const uint16_t *)p)[i]);
+    return oracle_bf16_to_f32(((const uint16_t *)p)[i]);
+}
+
+static void store_param(void *p, int dtype, int64_t i, float x)
+{
+    if (dtype == OR_F32) ((float *)p)[i] = x;
+    else if (dtype == OR_F16) ((uint16_t *)p)[i] = oracle_f32_to_f16(x);
+    else ((uint16_t *)p)[i] = oracle_f32_to_bf16(x);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Per-step scalars.                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* 1 - beta^t in double, rounded to fp32 once. [Adam] Algorithm 1. */
+float oracle_bias_correction(float beta, int t)
+{
+    return (float)(1.0 - pow((double)beta, (double)t));
+}
+
+/* 1 - lr*wd in double, rounded to fp32 once. [AdamW] Algorithm 2. */
+float oracle_decay_factor(float lr, float wd)
+{
+    return (float)(1.0 - (double)lr * (double)wd);
+}
+
+/* ------------------------------------------------------------------------ */
+/* The fp32 step.                                                            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * One optimizer step, in place, over one tensor of n elements.
+ *
+ * algo      0 = Adam (AdamW when wd != 0), 1 = AdEMAMix.
+ * dtype     storage of param and grad: 0 fp32, 1 fp16, 2 bf16.
+ * state1    Adam: m (n floats).  AdEMAMix: [m1 | m2] (2n floats).
+ * state2    v (n floats).
+ * step      t >= 1, the 1-based index of this update.
+ *
+ * Per element, every operation rounded to fp32 in this order:
+ *   m   = beta1*m + (1-beta1)*g                           [Adam]
+ *   v   = beta2*v + ((1-beta2)*g)*g                       [Adam]
+ *   num = m / bc1                                         [Adam]
+ *   AdEMAMix only:
+ *     m2  = beta3*m2 + (1-beta3)*g                        [AdEMAMix]
+ *     num = num + alpha*m2                                [AdEMAMix]
+ *   den = sqrt(v / bc2) + eps                             [Adam]
+ *   p   = p*decay - lr*(num/den)       decay first, [AdamW]; [issue] "Scope"
+ * Returns 0, or -1 on an argument the definitions do not cover.
+ */
+int oracle_step_f32(int algo, int dtype, int skip_zeros,
+                    float lr, float beta1, float beta2, float beta3,
+                    float alpha, float eps, float weight_decay, int step,
+                    void *param, const void *grad, float *state1,
+                    float *state2, int64_t n)
+{
+    if (step < 1 || n < 0) return -1;
+    if (algo != OR_ADAM && algo != OR_ADEMAMIX) return -1;
+    if (dtype != OR_F32 && dtype != OR_F16 && dtype != OR_BF16) return -1;
+
+    unsigned int csr = _mm_getcsr();
+    _mm_setcsr(csr & ~(0x8000u | 0x0040u));             /* FTZ and DAZ off */
+
+    const float bc1 = oracle_bias_correction(beta1, step);
+    const float bc2 = oracle_bias_correction(beta2, step);
+    const float decay = oracle_decay_factor(lr, weight_decay);
+    const float one_minus_b1 = 1.0f - beta1;
+    const float one_minus_b2 = 1.0f - beta2;
+    const float one_minus_b3 = 1.0f - beta3;
+
+    float *m = state1;
+    float *m2 = state1 + n;                             /* AdEMAMix only */
+    float *v = state2;
+
+    for (int64_t i = 0; i < n; i++) {
+        float g = load_param(grad, dtype, i);
+        if (skip_zeros && g == 0.0f) continue;
+        float p = load_param(param, dtype, i);
+
+        float mi = beta1 * m[i] + one_minus_b1 * g;
+        float vi = beta2 * v[i] + (one_minus_b2 * g) * g;
+        float num = mi / bc1;
+        if (algo == OR_ADEMAMIX) {
+            float m2i = beta3 * m2[i] + one_minus_b3 * g;
+            num = num + alpha * m2i;
+            m2[i] = m2i;
+        }
+        float den = sqrtf(vi / bc2) + eps;
+        p = p * decay - lr * (num / den);
+
+        m[i] = mi;
+        v[i] = vi;
+        store_param(param, dtype, i, p);
+    }
+
+    _mm_setcsr(csr);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* The fp64 shadow: the same definitions entirely in double, used to bound    */
+/* the rounding error of the fp32 oracle.  m2 may be NULL for Adam.           */
+/* ------------------------------------------------------------------------ */
+
+int oracle_step_f64(int algo, int skip_zeros, double lr, double beta1,
+                    double beta2, double beta3, double alpha, double eps,
+                    double weight_decay, int step, double *param,
+                    const double *grad, double *m, double *m2, double *v,
+                    int64_t n)
+{
+    if (step < 1 || n < 0) return -1;
+    if (algo != OR_ADAM && algo != OR_ADEMAMIX) return -1;
+    if (algo == OR_ADEMAMIX && m2 == NULL && n > 0) return -1;
+
+    const double bc1 = 1.0 - pow(beta1, (double)step);
+    const double bc2 = 1.0 - pow(beta2, (double)step);
+    const double decay = 1.0 - lr * weight_decay;
+
+    for (int64_t i = 0; i < n; i++) {
+        double g = grad[i];
+        if (skip_zeros && g == 0.0) continue;
+        m[i] = beta1 * m[i] + (1.0 - beta1) * g;
+        v[i] = beta2 * v[i] + (1.0 - beta2) * g * g;
+        double num = m[i] / bc1;
+        if (algo == OR_ADEMAMIX) {
+            m2[i] = beta3 * m2[i] + (1.0 - beta3) * g;
+            num += alpha * m2[i];
+        }
+        double den = sqrt(v[i] / bc2) + eps;
+        param[i] = param[i] * decay - lr * (num / den);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Array forms of the conversions, so the tests can sweep many values.        */
+/* dtype 1 = fp16, 2 = bf16.                                                  */
+/* ------------------------------------------------------------------------ */
+
+int oracle_narrow_array(int dtype, const float *x, uint16_t *out, int64_t n)
+{
+    if (dtype != OR_F16 && dtype != OR_BF16) return -1;
+    for (int64_t i = 0; i < n; i++)
+        out[i] = dtype == OR_F16 ? oracle_f32_to_f16(x[i]) : oracle_f32_to_bf16(x[i]);
+    return 0;
+}
+
+int oracle_widen_array(int dtype, const uint16_t *h, float *out, int64_t n)
+{
+    if (dtype != OR_F16 && dtype != OR_BF16) return -1;
+    for (int64_t i = 0; i < n; i++)
+        out[i] = dtype == OR_F16 ? oracle_f16_to_f32(h[i]) : oracle_bf16_to_f32(h[i]);
+    return 0;
+}

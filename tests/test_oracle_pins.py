@@ -1,0 +1,413 @@
+"""Pins for the CPU oracle: each check is fixed by something other than the
+oracle itself -- a library optimizer or conversion, a closed form, an
+invariant, or an exact special case -- so that a plausible slip in the oracle
+(a dropped term, a wrong index, a swapped operand or a wrong rounding) fails
+at least one of them.
+
+The method is the 32-bit two-state update of the bitsandbytes issue
+"Investigate a 256-thread SM103 path for small 32-bit optimizer tensors"
+(sections "Problem", "Scope", "Correctness oracle"), with the standard
+definitions of Adam (Kingma & Ba 2015, Algorithm 1), AdamW (Loshchilov &
+Hutter 2019, Algorithm 2) and AdEMAMix (Pagliardini et al. 2024, Algorithm 1).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from elementwise_optimizer_b200 import synth
+
+F32_EPS = 2.0 ** -23
+
+
+def ulp32(x):
+    """Spacing of float32 at |x| (at least the smallest subnormal)."""
+    x = np.abs(np.asarray(x, np.float32))
+    return np.spacing(x).astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# Storage conversions vs numpy / ml_dtypes / torch (IEEE 754 roundTiesToEven)
+# --------------------------------------------------------------------------
+
+def _conversion_probe(n=1 << 20, seed=7):
+    g = np.random.Generator(np.random.Philox(seed))
+    bits = g.integers(0, 1 << 32, n, dtype=np.uint64).astype(np.uint32)
+    x = bits.view(np.float32)
+    # values near the fp16/bf16 rounding boundaries, overflow and subnormals
+    special = np.array([0.0, -0.0, 1.0, -1.0, 65504.0, 65519.99, 65520.0,
+                        65536.0, 6.1035156e-05, 5.9604645e-08, 2.9802322e-08,
+                        2.9802326e-08, 1e-45, -1e-45, 3.4028235e38, np.inf,
+                        -np.inf, np.nan, 1.0 + 2 ** -11, 1.0 + 3 * 2 ** -11,
+                        1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.1754944e-38,
+                        1.1754942e-38], np.float32)
+    # exact ties: odd multiples of half a bf16/fp16 quantum around 1..2
+    k = np.arange(0, 4096, dtype=np.uint32)
+    ties_bf16 = ((np.uint32(0x3F800000) + (k << 16) + np.uint32(0x8000))).view(np.float32)
+    ties_f16 = ((np.uint32(0x3F800000) + (k << 13) + np.uint32(0x1000))).view(np.float32)
+    return np.concatenate([x, special, ties_bf16, ties_f16]).astype(np.float32)
+
+
+def _same_bits_or_both_nan(a_bits, b_bits, a_val, b_val):
+    nan = np.isnan(a_val) & np.isnan(b_val)
+    return np.all((a_bits == b_bits) | nan)
+
+
+def test_f16_narrowing_matches_numpy(oracle_mod):
+    x = _conversion_probe()
+    with np.errstate(over="ignore"):
+        ref = x.astype(np.float16)
+    got = oracle_mod.narrow(x, "f16")
+    assert _same_bits_or_both_nan(got, ref.view(np.uint16),
+                                  got.view(np.float16), ref)
+
+
+def test_bf16_narrowing_matches_ml_dtypes_and_torch(oracle_mod):
+    import ml_dtypes
+    x = _conversion_probe(seed=8)
+    ref = x.astype(ml_dtypes.bfloat16)
+    got = oracle_mod.narrow(x, "bf16")
+    assert _same_bits_or_both_nan(got, ref.view(np.uint16),
+                                  got.view(ml_dtypes.bfloat16).astype(np.float32),
+                                  ref.astype(np.float32))
+    tref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert _same_bits_or_both_nan(got, tref, x, x)
+
+
+def test_widening_exhaustive(oracle_mod):
+    import ml_dtypes
+    allbits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    f16 = oracle_mod.widen(allbits, "f16")
+    ref16 = allbits.view(np.float16).astype(np.float32)
+    assert np.array_equal(f16.view(np.uint32)[~np.isnan(ref16)],
+                          ref16.view(np.uint32)[~np.isnan(ref16)])
+    assert np.array_equal(np.isnan(f16), np.isnan(ref16))
+    bf = oracle_mod.widen(allbits, "bf16")
+    refb = allbits.view(ml_dtypes.bfloat16).astype(np.float32)
+    assert np.array_equal(np.isnan(bf), np.isnan(refb))
+    ok = ~np.isnan(refb)
+    assert np.array_equal(bf.view(np.uint32)[ok], refb.view(np.uint32)[ok])
+
+
+# --------------------------------------------------------------------------
+# The float64 shadow vs torch.optim (an independent library implementation)
+# --------------------------------------------------------------------------
+
+HYPERS = [
+    dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0),
+    dict(lr=1e-2, beta1=0.8, beta2=0.95, eps=1e-3, weight_decay=0.1),
+    dict(lr=3e-2, beta1=0.5, beta2=0.7, eps=1e-6, weight_decay=0.5),
+]
+
+
+def _torch_reference(p0, grads, hyper, cls=torch.optim.AdamW):
+    p = torch.tensor(p0, dtype=torch.float64, requires_grad=True)
+    opt = cls([p], lr=hyper["lr"], betas=(hyper["beta1"], hyper["beta2"]),
+              eps=hyper["eps"], weight_decay=hyper["weight_decay"],
+              foreach=False, fused=False)
+    for g in grads:
+        p.grad = torch.tensor(g, dtype=torch.float64)
+        opt.step()
+    st = opt.state[p]
+    return (p.detach().numpy(), st["exp_avg"].numpy(), st["exp_avg_sq"].numpy())
+
+
+@pytest.mark.parametrize("hyper", HYPERS)
+def test_shadow_adamw_matches_torch(oracle_mod, hyper):
+    n, steps = 4096, 12
+    g = np.random.Generator(np.random.Philox(11))
+    p0 = g.standard_normal(n)
+    grads = [g.standard_normal(n) * 10.0 ** g.uniform(-6, 1, n) for _ in range(steps)]
+    p, m, v = p0.copy(), np.zeros(n), np.zeros(n)
+    for t, gr in enumerate(grads, 1):
+        oracle_mod.step_f64(p, gr, m, v, algo="adam", step=t, **hyper)
+    tp, tm, tv = _torch_reference(p0, grads, hyper)
+    # m can cancel; bound its difference by the EMA of |g| (its magnitude scale)
+    scale = np.zeros(n)
+    for gr in grads:
+        scale = hyper["beta1"] * scale + (1 - hyper["beta1"]) * np.abs(gr)
+    assert np.all(np.abs(m - tm) <= 1e-14 * scale)
+    np.testing.assert_allclose(v, tv, rtol=1e-13, atol=1e-300)
+    np.testing.assert_allclose(p, tp, rtol=1e-12, atol=1e-15)
+
+
+def test_shadow_adam_without_decay_matches_torch_adam(oracle_mod):
+    hyper = dict(HYPERS[0])
+    n = 1000
+    g = np.random.Generator(np.random.Philox(12))
+    p0 = g.standard_normal(n)
+    grads = [g.standard_normal(n) * 1e-2 for _ in range(5)]
+    p, m, v = p0.copy(), np.zeros(n), np.zeros(n)
+    for t, gr in enumerate(grads, 1):
+        oracle_mod.step_f64(p, gr, m, v, algo="adam", step=t, **hyper)
+    tp, _, _ = _torch_reference(p0, grads, hyper, cls=torch.optim.Adam)
+    np.testing.assert_allclose(p, tp, rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("alpha,wd", [(5.0, 0.0), (2.0, 0.1), (0.5, 0.3)])
+def test_shadow_ademamix_reduces_to_torch_adam(oracle_mod, alpha, wd):
+    """With beta1 = beta3 = 0 the slow EMA is the gradient itself and the bias
+    correction of m1 is 1, so AdEMAMix(lr, alpha, wd) steps exactly like Adam
+    with beta1 = 0, learning rate lr*(1+alpha) and weight decay wd/(1+alpha)
+    (the decay factor 1 - lr*wd is unchanged)."""
+    n, steps, lr = 2048, 8, 1e-2
+    g = np.random.Generator(np.random.Philox(13))
+    p0 = g.standard_normal(n)
+    grads = [g.standard_normal(n) * 10.0 ** g.uniform(-4, 1, n) for _ in range(steps)]
+    p, m, v, m2 = p0.copy(), np.zeros(n), np.zeros(n), np.zeros(n)
+    for t, gr in enumerate(grads, 1):
+        oracle_mod.step_f64(p, gr, m, v, m2, algo="ademamix", step=t, lr=lr,
+                            beta1=0.0, beta2=0.99, beta3=0.0, alpha=alpha,
+                            eps=1e-8, weight_decay=wd)
+    lib = dict(lr=lr * (1 + alpha), beta1=0.0, beta2=0.99, eps=1e-8,
+               weight_decay=wd / (1 + alpha))
+    tp, _, _ = _torch_reference(p0, grads, lib)
+    np.testing.assert_allclose(p, tp, rtol=1e-12, atol=1e-14)
+    np.testing.assert_array_equal(m2, grads[-1])
+
+
+# --------------------------------------------------------------------------
+# The fp32 oracle vs the float64 shadow, one step from identical state
+# --------------------------------------------------------------------------
+
+def _random_state(seed, n, dtype, algo):
+    g = np.random.Generator(np.random.Philox(seed))
+    p = synth.to_storage(g.standard_normal(n).astype(np.float32), dtype)
+    gr = synth.to_storage((g.standard_normal(n) * 10.0 ** g.uniform(-5, 1, n)).astype(np.float32), dtype)
+    m = (g.standard_normal(n) * 1e-2).astype(np.float32)
+    m2 = (g.standard_normal(n) * 1e-2).astype(np.float32)
+    v = (g.random(n) * 1e-3).astype(np.float32)
+    s1 = np.concatenate([m, m2]) if algo == "ademamix" else m
+    return p, gr, s1, v
+
+
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("hi", range(len(HYPERS)))
+@pytest.mark.parametrize("t", [1, 2, 10, 1000])
+def test_f32_oracle_one_step_within_rounding_of_shadow(oracle_mod, algo, dtype, hi, t):
+    """From the same state and the same (fp32) hyper-parameters, the fp32
+    oracle stays within a rounding-error bound of the float64 shadow.  Each
+    fp32 operation errs by at most 2^-24 of its result, so every bound below
+    is a small multiple of 2^-24 times the magnitudes of the terms that feed
+    the result (which also covers cancellation in m and in p)."""
+    hyper = {k: float(np.float32(x)) for k, x in dict(HYPERS[hi], beta3=0.999, alpha=3.0).items()}
+    n = 20000
+    p, gr, s1, v = _random_state(100 + hi, n, dtype, algo)
+    pf = synth.from_storage(p, dtype).astype(np.float64)
+    gf = synth.from_storage(gr, dtype).astype(np.float64)
+    m_old = s1[:n].astype(np.float64)
+    m2_old = s1[n:].astype(np.float64) if algo == "ademamix" else None
+    v_old = v.astype(np.float64)
+    p64, m64, v64 = pf.copy(), m_old.copy(), v_old.copy()
+    m2_64 = m2_old.copy() if m2_old is not None else None
+    oracle_mod.step_f64(p64, gf, m64, v64, m2_64, algo=algo, step=t, **hyper)
+    p32, s1_32, v32 = p.copy(), s1.copy(), v.copy()
+    oracle_mod.step_f32(p32, gr, s1_32, v32, dtype=dtype, algo=algo, step=t, **hyper)
+
+    u = 2.0 ** -24
+    tiny = 1e-44
+    b1, b2, b3 = hyper["beta1"], hyper["beta2"], hyper["beta3"]
+    m_scale = np.abs(b1 * m_old) + np.abs((1 - b1) * gf)
+    assert np.all(np.abs(s1_32[:n] - m64) <= 4 * u * m_scale + tiny)
+    assert np.all(np.abs(v32 - v64) <= 8 * u * v64 + tiny)
+    num_scale = m_scale / (1 - b1 ** t)
+    if algo == "ademamix":
+        m2_scale = np.abs(b3 * m2_old) + np.abs((1 - b3) * gf)
+        assert np.all(np.abs(s1_32[n:] - m2_64) <= 4 * u * m2_scale + tiny)
+        num_scale = num_scale + hyper["alpha"] * m2_scale
+    den = np.sqrt(v64 / (1 - b2 ** t)) + hyper["eps"]
+    lr, wd = hyper["lr"], hyper["weight_decay"]
+    p_scale = np.abs(pf * (1 - lr * wd)) + lr * num_scale / den
+    got = synth.from_storage(p32, dtype).astype(np.float64)
+    bound = 24 * u * p_scale + tiny
+    if dtype == "f16":        # one more rounding, to binary16
+        bound = bound + 2.0 ** -11 * np.abs(p64) + 2.0 ** -25
+    elif dtype == "bf16":     # one more rounding, to bfloat16
+        bound = bound + 2.0 ** -8 * np.abs(p64) + 1e-40
+    assert np.all(np.abs(got - p64) <= bound)
+
+
+# --------------------------------------------------------------------------
+# Closed forms
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+def test_step_one_closed_form(oracle_mod, algo):
+    """At t = 1 from zero state m/bc1 = g and v/bc2 = g^2 exactly (real
+    arithmetic), and m2 = (1-beta3) g, so
+    p1 = p0*(1-lr*wd) - lr*(g + alpha*(1-beta3)*g)/(|g| + eps)."""
+    n = 50000
+    g = np.random.Generator(np.random.Philox(21))
+    p0 = g.standard_normal(n).astype(np.float32)
+    gr = (g.standard_normal(n) * 10.0 ** g.uniform(-9, 1, n)).astype(np.float32)
+    hyper = dict(lr=1e-2, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1,
+                 beta3=0.99, alpha=4.0)
+    p, s1 = p0.copy(), np.zeros(2 * n if algo == "ademamix" else n, np.float32)
+    v = np.zeros(n, np.float32)
+    oracle_mod.step_f32(p, gr, s1, v, dtype="f32", algo=algo, step=1, **hyper)
+    gd = gr.astype(np.float64)
+    num = gd + (hyper["alpha"] * (1 - hyper["beta3"]) * gd if algo == "ademamix" else 0)
+    exact = p0 * (1 - 1e-2 * 0.1) - 1e-2 * num / (np.abs(gd) + 1e-8)
+    step = 1e-2 * np.abs(num) / (np.abs(gd) + 1e-8)
+    assert np.all(np.abs(p - exact) <= 2 * ulp32(exact) + 16 * F32_EPS * step)
+
+
+def test_step_one_unit_gradient_is_exactly_minus_lr(oracle_mod):
+    """p0 = 0, g = 1: m/bc1 = v/bc2 = 1 exactly in fp32 (Sterbenz), and
+    1 + 1e-8 rounds to 1, so p1 is the fp32 value of -lr exactly."""
+    p = np.zeros(1, np.float32)
+    s1, v = np.zeros(1, np.float32), np.zeros(1, np.float32)
+    oracle_mod.step_f32(p, np.ones(1, np.float32), s1, v, dtype="f32",
+                        algo="adam", step=1, lr=1e-3, beta1=0.9, beta2=0.999,
+                        eps=1e-8)
+    assert p[0] == np.float32(-1e-3)
+
+
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+@pytest.mark.parametrize("wd", [0.0, 0.05])
+def test_constant_gradient_closed_form(oracle_mod, algo, wd):
+    """A constant gradient g keeps m/bc1 = g and v/bc2 = g^2 at every step,
+    while m2_k = g (1 - beta3^k), so with d = 1 - lr*wd
+    p_T = p0 d^T - lr * sum_k d^(T-k) (g + alpha g (1-beta3^k)) / (|g| + eps).
+    """
+    T, lr, b3, alpha, eps = 1000, 1e-3, 0.999, 5.0, 1e-8
+    gvals = np.array([0.5, -0.5, 2e-3, -7.0, 1e-6, 30.0], np.float32)
+    p0 = np.array([2.0, -2.0, 3.0, 5.0, -4.0, 3.0], np.float32)
+    n = gvals.size
+    p = p0.copy()
+    s1 = np.zeros(2 * n if algo == "ademamix" else n, np.float32)
+    v = np.zeros(n, np.float32)
+    for t in range(1, T + 1):
+        oracle_mod.step_f32(p, gvals, s1, v, dtype="f32", algo=algo, step=t,
+                            lr=lr, beta1=0.9, beta2=0.999, eps=eps, beta3=b3,
+                            alpha=alpha, weight_decay=wd)
+    gd = gvals.astype(np.float64)
+    d = 1 - lr * wd
+    k = np.arange(1, T + 1, dtype=np.float64)
+    mix = (alpha * (1 - b3 ** k)) if algo == "ademamix" else np.zeros(T)
+    w = d ** (T - k)
+    total = (w[None, :] * (1 + mix[None, :])).sum(axis=1)
+    exact = p0 * d ** T - lr * total * gd / (np.abs(gd) + eps)
+    # each step adds O(1) rounding of |p|; T steps -> T-ish ulps
+    np.testing.assert_allclose(p, exact, rtol=2e-4)
+    if algo == "ademamix":
+        np.testing.assert_allclose(s1[n:], gd * (1 - b3 ** T), rtol=1e-4)
+
+
+# --------------------------------------------------------------------------
+# Invariants and exact special cases
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_zero_gradient_fixed_point(oracle_mod, algo, dtype):
+    """g = 0 from zero state: nothing moves without decay; with decay only
+    p *= d each step (p_T = p0 d^T), moments stay zero."""
+    n = 513
+    p0 = synth.to_storage(np.linspace(-3, 3, n).astype(np.float32), dtype)
+    z = synth.to_storage(np.zeros(n, np.float32), dtype)
+    for wd in (0.0, 0.1):
+        p = p0.copy()
+        s1 = np.zeros(2 * n if algo == "ademamix" else n, np.float32)
+        v = np.zeros(n, np.float32)
+        for t in range(1, 11):
+            oracle_mod.step_f32(p, z, s1, v, dtype=dtype, algo=algo, step=t,
+                                lr=1e-2, beta1=0.9, beta2=0.999, eps=1e-8,
+                                beta3=0.999, alpha=5.0, weight_decay=wd)
+        assert not s1.any() and not v.any()
+        if wd == 0.0:
+            assert np.array_equal(p.view(np.uint8), p0.view(np.uint8))
+        else:
+            exact = synth.from_storage(p0, dtype).astype(np.float64) * (1 - 1e-3) ** 10
+            got = synth.from_storage(p, dtype).astype(np.float64)
+            tol = {"f32": 12 * F32_EPS, "f16": 12 * 2 ** -11, "bf16": 12 * 2 ** -8}[dtype]
+            assert np.all(np.abs(got - exact) <= tol * np.abs(exact) + 1e-30)
+
+
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_skip_zeros(oracle_mod, algo, dtype):
+    """skip_zeros leaves every zero-gradient element wholly untouched (also
+    without decay) and treats the others exactly as the plain step does."""
+    n = 4097
+    p, gr, s1, v = _random_state(31, n, dtype, algo)
+    gvals = synth.from_storage(gr, dtype)
+    zero = np.arange(n) % 3 == 0
+    gvals[zero] = 0.0
+    gvals[np.arange(n) % 6 == 0] = -0.0
+    gr = synth.to_storage(gvals, dtype)
+    kw = dict(dtype=dtype, algo=algo, step=5, lr=1e-2, beta1=0.9, beta2=0.999,
+              eps=1e-8, beta3=0.999, alpha=5.0, weight_decay=0.1)
+    a = [x.copy() for x in (p, s1, v)]
+    oracle_mod.step_f32(a[0], gr, a[1], a[2], skip_zeros=True, **kw)
+    b = [x.copy() for x in (p, s1, v)]
+    oracle_mod.step_f32(b[0], gr, b[1], b[2], skip_zeros=False, **kw)
+    zi = np.concatenate([zero, zero]) if algo == "ademamix" else zero
+    assert np.array_equal(a[0][zero].view(np.uint8), p[zero].view(np.uint8))
+    assert np.array_equal(a[1][zi], s1[zi]) and np.array_equal(a[2][zero], v[zero])
+    nz = ~zero
+    nzi = ~zi
+    assert np.array_equal(a[0][nz].view(np.uint8), b[0][nz].view(np.uint8))
+    assert np.array_equal(a[1][nzi], b[1][nzi]) and np.array_equal(a[2][nz], b[2][nz])
+    # and without skip_zeros the zero-gradient elements do decay
+    assert not np.array_equal(b[0][zero & (synth.from_storage(p, dtype) != 0)],
+                              p[zero & (synth.from_storage(p, dtype) != 0)])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_ademamix_alpha_zero_equals_adam_bitwise(oracle_mod, dtype):
+    """alpha = 0 adds an exact +0 to m/bc1, so param, m1 and v match Adam."""
+    n = 3000
+    p, gr, s1, v = _random_state(41, n, dtype, "ademamix")
+    kw = dict(dtype=dtype, step=7, lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8,
+              weight_decay=0.01)
+    pa, s1a, va = p.copy(), s1.copy(), v.copy()
+    oracle_mod.step_f32(pa, gr, s1a, va, algo="ademamix", beta3=0.9, alpha=0.0, **kw)
+    pb, mb, vb = p.copy(), s1[:n].copy(), v.copy()
+    oracle_mod.step_f32(pb, gr, mb, vb, algo="adam", **kw)
+    assert np.array_equal(pa.view(np.uint8), pb.view(np.uint8))
+    assert np.array_equal(s1a[:n], mb) and np.array_equal(va, vb)
+
+
+def test_gradient_is_never_written(oracle_mod):
+    n = 1025
+    for dtype in ("f32", "f16", "bf16"):
+        p, gr, s1, v = _random_state(51, n, dtype, "adam")
+        keep = gr.copy()
+        oracle_mod.step_f32(p, gr, s1, v, dtype=dtype, algo="adam", step=3,
+                            lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8)
+        assert np.array_equal(keep.view(np.uint8), gr.view(np.uint8))
+
+
+def test_rejects_step_zero(oracle_mod):
+    p = np.zeros(4, np.float32)
+    with pytest.raises(ValueError):
+        oracle_mod.step_f32(p, p.copy(), p.copy(), p.copy(), dtype="f32",
+                            algo="adam", step=0, lr=1e-3, beta1=0.9,
+                            beta2=0.999, eps=1e-8)
+
+
+def test_bias_correction_and_decay_round_once(oracle_mod):
+    """bc = 1 - beta^t and d = 1 - lr*wd are exact in double for these inputs
+    up to one double rounding, then rounded to fp32 once."""
+    assert oracle_mod.bias_correction(0.5, 3) == np.float32(0.875)
+    assert oracle_mod.bias_correction(0.0, 1) == np.float32(1.0)
+    assert oracle_mod.decay_factor(0.5, 0.25) == np.float32(0.875)
+    b = np.float32(0.9)
+    assert oracle_mod.bias_correction(float(b), 2) == np.float32(1 - float(b) ** 2)
+
+
+def test_golden_traces(oracle_mod):
+    """Single-element trajectories stored by tests/golden/make_golden.py; the
+    first seven agree with an independent hand computation (see the file)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "traces.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    assert rows
+    from tests.golden.make_golden import run_trace
+    for r in rows:
+        case, t, hexbits = r[0], int(r[1]), r[2]
+        got = run_trace(case)[t - 1]
+        assert got == hexbits, (case, t, got, hexbits)
