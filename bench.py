@@ -1,0 +1,506 @@
+"""Benchmark of the B200 two-state optimizer step (Adam/AdamW, AdEMAMix).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload large_f32|transformer_bf16|small_collection]
+
+One step is one optimizer update of the whole workload: one launch of the
+persistent multi-tensor kernel through the C ABI (opt2s_step).  The default
+workload is one fp32 tensor of 268,435,456 elements with Adam (28 algorithmic
+bytes per element: grad, param, m, v read; param, m, v written), the
+large-tensor case whose elements/s and HBM GB/s are the headline.  Its 7.5 GB
+per step is far larger than the 126 MB L2, so no L2 flush is needed between
+steps.  Gradients rotate through 4 pre-generated synthetic buffers.
+
+Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank steps its own
+full-size workload on its own GPU (the update is elementwise, so shards of a
+collection need no exchange): weak scaling, value = all ranks' elements per
+second over the slowest rank's time.
+
+--impl reference times the CPU oracle (the plain C restatement the tests check
+the kernel against) on the host cores, each step a bounded sample of the same
+workload; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = ("optimizer step: elements/s and HBM GB/s (% of B200 peak); "
+          "µs per small-tensor step")
+FALLBACK_HBM_GBS = 6650.0
+BYTES_PER_ELEM = {("adam", "f32"): 28, ("ademamix", "f32"): 36,
+                  ("adam", "f16"): 22, ("adam", "bf16"): 22,
+                  ("ademamix", "f16"): 30, ("ademamix", "bf16"): 30}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload(name, numel=0):
+    from elementwise_optimizer_b200 import synth
+    if name == "large_f32" and numel:
+        return synth.large_f32(numel)
+    return {"large_f32": synth.large_f32, "transformer_bf16": synth.transformer_bf16,
+            "small_collection": synth.small_collection}[name]()
+
+
+def algorithmic_bytes(w):
+    return sum(BYTES_PER_ELEM[(w.algo, d)] * n for n, d in zip(w.sizes, w.dtypes))
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling (nvidia-smi) during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for l in self.lines:
+            parts = [x.strip() for x in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), max=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hw_thermal=parts[6], sw_thermal=parts[7],
+                                 power_cap=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        loaded = [r for r in rows if r["power"] > 200] or rows
+        reasons = set()
+        for r in loaded:
+            for k, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                            ("sw_thermal", "sw_thermal_slowdown"), ("power_cap", "sw_power_cap")):
+                if r[k].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(loaded),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+def traffic_for(kernel_key):
+    """ncu DRAM bytes per launch, if the committed capture is of the kernel
+    source as it is now (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    src = os.path.join(ROOT, "elementwise_optimizer_b200", "csrc", "opt2s_kernel.cu")
+    try:
+        rec = json.load(open(path)).get(kernel_key)
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if rec and rec.get("kernel_source_sha256") == sha:
+            return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def make_device_workload(w, device, n_grad_buffers):
+    """Allocate param / grads / states for workload w on `device` and fill
+    them with seeded synthetic values (made on the device: this is bench
+    input, not a parity case)."""
+    import torch
+    from elementwise_optimizer_b200 import binding as B
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    params, s1, s2 = [], [], []
+    grads = [[] for _ in range(n_grad_buffers)]
+    for n, d in zip(w.sizes, w.dtypes):
+        p = torch.empty(n, dtype=torch.float32, device=device)
+        p.normal_(0.0, w.param_std, generator=gen)
+        params.append(p.to(tdt[d]))
+        del p
+        for k in range(n_grad_buffers):
+            g = torch.empty(n, dtype=torch.float32, device=device)
+            g.normal_(0.0, w.grad_std, generator=gen)
+            grads[k].append(g.to(tdt[d]))
+            del g
+        s1.append(torch.zeros(2 * n if w.algo == "ademamix" else n, device=device))
+        s2.append(torch.zeros(n, device=device))
+    lists = [B.TensorList.from_tensors(params, grads[k], s1, s2) for k in range(n_grad_buffers)]
+    hyper = B.make_hyper(w.algo, skip_zeros=w.skip_zeros, **w.hyper)
+    return dict(params=params, grads=grads, s1=s1, s2=s2, lists=lists, hyper=hyper)
+
+
+def small_collection_us(device, reps=200):
+    """µs per step of the 2,000-tensor collection (one launch per step),
+    L2 flushed before every step by writing a 256 MB buffer."""
+    import torch
+    from elementwise_optimizer_b200 import binding as B
+    w = workload("small_collection")
+    d = make_device_workload(w, device, 1)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+    for t in range(1, 6):
+        B.opt2s_step(d["lists"][0], d["hyper"], t)
+    torch.cuda.synchronize()
+    times = []
+    launches0 = B.launch_count()
+    for t in range(6, 6 + reps):
+        flush.fill_(float(t))
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        B.opt2s_step(d["lists"][0], d["hyper"], t)
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize()
+    us = sorted(a.elapsed_time(b) * 1e3 for a, b in times)
+    launches = B.launch_count() - launches0
+    q = lambda f: us[min(len(us) - 1, int(f * len(us)))]
+    return {"workload": w.name, "tensors": len(w.sizes), "numel": w.numel,
+            "us_per_step_median": q(0.5), "us_per_step_p10": q(0.1), "us_per_step_p90": q(0.9),
+            "launches_per_step": launches / reps, "l2": "flushed (256 MB write) before each step"}
+
+
+def e2e_measure(w, d, device, steps):
+    """Same metric through the public call with host buffers: every step
+    copies that step's gradient from pinned host memory to the device, runs
+    opt2s_step, and reads the updated param back into pinned host memory."""
+    import torch
+    from elementwise_optimizer_b200 import binding as B
+    host_g = [g.cpu().pin_memory() for g in d["grads"][0]]
+    host_p = [torch.empty(p.shape, dtype=p.dtype, pin_memory=True) for p in d["params"]]
+    stream = torch.cuda.current_stream()
+    h2d = sum(g.numel() * g.element_size() for g in host_g)
+    d2h = sum(p.numel() * p.element_size() for p in host_p)
+    t0 = 1000
+    def one(t):
+        for hg, dg in zip(host_g, d["grads"][0]):
+            dg.copy_(hg, non_blocking=True)
+        B.opt2s_step(d["lists"][0], d["hyper"], t)
+        for hp, dp in zip(host_p, d["params"]):
+            hp.copy_(dp, non_blocking=True)
+    for k in range(2):
+        one(t0 + k)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for k in range(steps):
+        one(t0 + 2 + k)
+    b.record(stream)
+    b.synchronize()
+    sec = a.elapsed_time(b) / 1e3
+    return {"value": w.numel * steps / sec, "unit": "elements/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": sec * 1e3 / steps,
+            "path": "pinned host grad -> device, opt2s_step, device param -> pinned host; one stream"}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from elementwise_optimizer_b200 import _build
+    from elementwise_optimizer_b200 import binding as B
+    if rank == 0 or not os.path.exists(B.LIB_PATH):
+        _build.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    w = workload(args.workload, args.numel)
+    d = make_device_workload(w, device, 4)
+    stream = torch.cuda.current_stream()
+    nbuf = len(d["lists"])
+
+    step = 0
+    for _ in range(args.warmup):
+        step += 1
+        B.opt2s_step(d["lists"][step % nbuf], d["hyper"], step)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    launches0 = B.launch_count()
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        events[0].record(stream)
+        for k in range(args.steps):
+            step += 1
+            B.opt2s_step(d["lists"][step % nbuf], d["hyper"], step)
+            events[k + 1].record(stream)
+        barrier()
+    launches = B.launch_count() - launches0
+    per_launch_ms = [events[k].elapsed_time(events[k + 1]) for k in range(args.steps)]
+    total_ms = events[0].elapsed_time(events[-1])
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    extras = {}
+    if rank == 0 and world == 1 and not args.no_extras:
+        extras["small_collection"] = small_collection_us(device)
+        extras["e2e"] = e2e_measure(w, d, device, args.e2e_steps)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    if rank != 0:
+        return None
+    sec = total_ms / 1e3
+    elems = w.numel * args.steps * world
+    algo_bytes = algorithmic_bytes(w)
+    mean_launch_s = statistics.mean(per_launch_ms) / 1e3
+    peak, peak_kind = measured_peak()
+    achieved = algo_bytes / mean_launch_s / 1e9
+    kernel_key = f"step_kernel/{w.name}"
+    traffic = traffic_for(kernel_key)
+    dtype = sorted(set(w.dtypes))
+    line = {
+        "metric": METRIC,
+        "value": elems / sec,
+        "unit": "elements/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32" if dtype == ["f32"] else f"{'+'.join(dtype)} storage, f32 math",
+        "data": "synthetic",
+        "config": {"workload": w.name, "numel_per_gpu": w.numel, "tensors": len(w.sizes),
+                   "algo": w.algo, "storage": dtype, "state": "f32",
+                   "bytes_per_element": algo_bytes / w.numel,
+                   "l2": f"inputs larger than L2 ({algo_bytes / 1e9:.2f} GB per step), no flush",
+                   "grad_buffers": nbuf,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "hbm_gbs": algo_bytes * args.steps * world / sec / 1e9 / world,
+        "hbm_frac_of_peak": algo_bytes * args.steps / sec / 1e9 / peak,
+        "launch_ms": {"median": statistics.median(per_launch_ms),
+                      "p10": float(np.percentile(per_launch_ms, 10)),
+                      "p90": float(np.percentile(per_launch_ms, 90)),
+                      "mean": statistics.mean(per_launch_ms)},
+        "clocks": clocks.summary(),
+        "gpu_launches": launches,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "kernel": "opt2s step_kernel", "algorithmic_bytes_per_launch": algo_bytes},
+    }
+    if "e2e" in extras:
+        line["e2e"] = extras.pop("e2e")
+    line.update(extras)
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return line
+
+
+# ---------------------------------------------------------------------------
+# The oracle on the host cores (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+
+def _oracle_sample(w, n_sample):
+    """A bounded sample of the workload's first tensor, as host arrays."""
+    from elementwise_optimizer_b200 import synth
+    d = w.dtypes[0]
+    p = synth.to_storage(synth.normal(w.seed, (11,), n_sample, w.param_std), d)
+    g = synth.to_storage(synth.normal(w.seed, (12,), n_sample, w.grad_std), d)
+    s1 = np.zeros(2 * n_sample if w.algo == "ademamix" else n_sample, np.float32)
+    s2 = np.zeros(n_sample, np.float32)
+    return d, p, g, s1, s2
+
+
+def _oracle_parallel_step(w, arrays, step, cores, pool):
+    import oracle
+    d, p, g, s1, s2 = arrays
+    n = p.size
+    bounds = np.linspace(0, n, cores + 1).astype(np.int64)
+
+    def part(k):
+        lo, hi = int(bounds[k]), int(bounds[k + 1])
+        if hi <= lo:
+            return
+        if w.algo == "ademamix":
+            # the oracle wants [m1 | m2] of its own slice contiguous
+            s1k = np.concatenate([s1[lo:hi], s1[n + lo:n + hi]])
+        else:
+            s1k = s1[lo:hi]
+        pk = p[lo:hi]
+        s2k = s2[lo:hi]
+        oracle.step_f32(pk, g[lo:hi], s1k, s2k, dtype=d, algo=w.algo, step=step,
+                        skip_zeros=w.skip_zeros, **w.hyper)
+        if w.algo == "ademamix":
+            s1[lo:hi] = s1k[:hi - lo]
+            s1[n + lo:n + hi] = s1k[hi - lo:]
+
+    list(pool.map(part, range(cores)))
+
+
+def cpu_baseline(w, seconds):
+    """The oracle as it stands, on all host cores (one single-threaded oracle
+    call per core on disjoint slices), on a bounded sample of the workload."""
+    import oracle
+    oracle.build()
+    cores = os.cpu_count() or 1
+    n_sample = 1 << 24
+    arrays = _oracle_sample(w, n_sample)
+    steps = 0
+    with cf.ThreadPoolExecutor(max_workers=cores) as pool:
+        _oracle_parallel_step(w, arrays, 1, cores, pool)           # warm-up
+        t0 = time.perf_counter()
+        while True:
+            steps += 1
+            _oracle_parallel_step(w, arrays, 1 + steps, cores, pool)
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+    return {"value": n_sample * steps / el, "unit": "elements/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"first {n_sample} elements of {w.name}, {steps} steps, "
+                      f"{el:.1f} s, {cores} threads x single-threaded oracle on disjoint slices"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    w = workload(args.workload, args.numel)
+    cores = os.cpu_count() or 1
+    n_sample = 1 << 22
+    arrays = _oracle_sample(w, n_sample)
+    with cf.ThreadPoolExecutor(max_workers=cores) as pool:
+        step = 0
+        for _ in range(args.warmup):
+            step += 1
+            _oracle_parallel_step(w, arrays, step, cores, pool)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            step += 1
+            _oracle_parallel_step(w, arrays, step, cores, pool)
+        sec = time.perf_counter() - t0
+    value = n_sample * args.steps / sec
+    sample = (f"each step: oracle over the first {n_sample} elements of {w.name} "
+              f"on {cores} threads (disjoint slices)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "elements/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "numel_per_gpu": w.numel, "algo": w.algo,
+                   "sample_elements_per_step": n_sample},
+        "cpu_baseline": {"value": value, "unit": "elements/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="large_f32",
+                    choices=["large_f32", "transformer_bf16", "small_collection"])
+    ap.add_argument("--numel", type=int, default=0,
+                    help="size of the large_f32 tensor (default 268,435,456)")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the small-collection, e2e and cpu_baseline legs")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"note: WORLD_SIZE={world}, --gpus={args.gpus}; using WORLD_SIZE")
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,268 @@
+"""Thin ctypes binding of libopt2s.so (include/opt2s.h).
+
+Argument marshalling only: every step of the optimizer update runs in the CUDA
+kernels of libopt2s.so.  There is no CPU fallback -- if the library is missing
+or cannot be loaded, every call raises.  PyTorch is used by callers only for
+device memory and streams; the binding takes raw device pointers or torch
+tensors (for which it reads ``data_ptr()``, ``numel()`` and ``dtype``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Iterable, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libopt2s.so")
+
+OPT2S_F32, OPT2S_F16, OPT2S_BF16 = 0, 1, 2
+OPT2S_ADAM, OPT2S_ADEMAMIX = 0, 1
+ALGOS = {"adam": OPT2S_ADAM, "adamw": OPT2S_ADAM, "ademamix": OPT2S_ADEMAMIX}
+DTYPES = {"f32": OPT2S_F32, "f16": OPT2S_F16, "bf16": OPT2S_BF16}
+
+OPT2S_OK = 0
+STATUS = {0: "OPT2S_OK", -1: "OPT2S_ERR_INVALID_ARG", -2: "OPT2S_ERR_ALIAS",
+          -3: "OPT2S_ERR_NO_MEMORY", -4: "OPT2S_ERR_CUDA",
+          -5: "OPT2S_ERR_DEVICE", -6: "OPT2S_ERR_TOO_LARGE"}
+
+
+class Opt2sError(RuntimeError):
+    def __init__(self, status: int, where: str, cuda_error: int = 0):
+        self.status = status
+        self.cuda_error = cuda_error
+        msg = f"{where}: {STATUS.get(status, status)} ({_error_string(status)})"
+        if status == -4:
+            msg += f", cudaError {cuda_error}"
+        super().__init__(msg)
+
+
+class opt2s_tensor(ctypes.Structure):
+    _fields_ = [("param", ctypes.c_void_p), ("grad", ctypes.c_void_p),
+                ("state1", ctypes.c_void_p), ("state2", ctypes.c_void_p),
+                ("numel", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+class TensorListDesc(ctypes.Structure):
+    _fields_ = [("tensors", ctypes.POINTER(opt2s_tensor)), ("count", ctypes.c_int32)]
+
+
+class Hyper(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float),
+                ("beta2", ctypes.c_float), ("beta3", ctypes.c_float),
+                ("alpha", ctypes.c_float), ("eps", ctypes.c_float),
+                ("weight_decay", ctypes.c_float), ("algo", ctypes.c_int32),
+                ("skip_zeros", ctypes.c_int32)]
+
+
+class opt2s_testing_chunk(ctypes.Structure):
+    _fields_ = [("tensor", ctypes.c_int64), ("start", ctypes.c_int64),
+                ("len", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+EXPORTS = {
+    # name: (restype, argtypes)
+    "opt2s_step": (ctypes.c_int, [ctypes.POINTER(TensorListDesc), ctypes.POINTER(Hyper),
+                                  ctypes.c_int, ctypes.c_void_p]),
+    "opt2s_plan_create": (ctypes.c_int, [ctypes.POINTER(TensorListDesc), ctypes.c_int32,
+                                         ctypes.POINTER(ctypes.c_void_p)]),
+    "opt2s_plan_step": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(Hyper), ctypes.c_int,
+                                       ctypes.c_void_p]),
+    "opt2s_plan_destroy": (ctypes.c_int, [ctypes.c_void_p]),
+    "opt2s_plan_num_chunks": (ctypes.c_int64, [ctypes.c_void_p]),
+    "opt2s_release_cache": (ctypes.c_int, []),
+    "opt2s_error_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "opt2s_last_cuda_error": (ctypes.c_int, []),
+    "opt2s_abi_version": (ctypes.c_int, []),
+    "opt2s_testing_build_chunks": (ctypes.c_int, [ctypes.POINTER(TensorListDesc), ctypes.c_int32,
+                                                  ctypes.c_int64,
+                                                  ctypes.POINTER(opt2s_testing_chunk),
+                                                  ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]),
+    "opt2s_testing_validate": (ctypes.c_int, [ctypes.POINTER(TensorListDesc),
+                                              ctypes.POINTER(Hyper), ctypes.c_int]),
+    "opt2s_testing_set_chunk_elems": (ctypes.c_int64, [ctypes.c_int64]),
+    "opt2s_testing_set_launch": (ctypes.c_int, [ctypes.c_int, ctypes.c_int]),
+    "opt2s_testing_default_chunk_elems": (ctypes.c_int64, []),
+    "opt2s_testing_launch_count": (ctypes.c_int64, []),
+    "opt2s_testing_max_block_threads": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libopt2s.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build the CUDA library first "
+                "(python -m elementwise_optimizer_b200._build); there is no CPU fallback")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in EXPORTS.items():
+            fn = getattr(L, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _error_string(status: int) -> str:
+    try:
+        return lib().opt2s_error_string(status).decode()
+    except Exception:  # pragma: no cover - only while formatting an error
+        return "?"
+
+
+def check(status: int, where: str) -> None:
+    if status != OPT2S_OK:
+        raise Opt2sError(status, where, lib().opt2s_last_cuda_error())
+
+
+# ---------------------------------------------------------------------------
+# Marshalling
+# ---------------------------------------------------------------------------
+
+def _torch_dtype_code(t) -> int:
+    import torch
+    code = {torch.float32: OPT2S_F32, torch.float16: OPT2S_F16,
+            torch.bfloat16: OPT2S_BF16}.get(t.dtype)
+    if code is None:
+        raise TypeError(f"unsupported param dtype {t.dtype}")
+    return code
+
+
+def _ptr(x) -> int:
+    return x if isinstance(x, int) else int(x.data_ptr())
+
+
+class TensorList:
+    """A marshalled collection: the ctypes descriptor a step is called with.
+
+    Build it once and reuse it: the records hold raw device pointers, so the
+    tensors must stay alive (and in place) while the list is used.
+    """
+
+    def __init__(self, records: Sequence[tuple]):
+        """records: (param, grad, state1, state2, numel, dtype_code) tuples,
+        the pointers as ints."""
+        n = len(records)
+        self._arr = (opt2s_tensor * max(n, 1))()
+        for i, (p, g, s1, s2, numel, dt) in enumerate(records):
+            self._arr[i] = opt2s_tensor(p, g, s1, s2, int(numel), int(dt), 0)
+        self.desc = TensorListDesc(ctypes.cast(self._arr, ctypes.POINTER(opt2s_tensor)), n)
+        self.count = n
+
+    @classmethod
+    def from_tensors(cls, params: Iterable, grads: Iterable, state1: Iterable,
+                     state2: Iterable) -> "TensorList":
+        """From torch tensors (contiguous, on the same CUDA device)."""
+        recs = []
+        for p, g, s1, s2 in zip(params, grads, state1, state2):
+            for t in (p, g, s1, s2):
+                if not t.is_contiguous():
+                    raise ValueError("tensors must be contiguous")
+            if g.dtype != p.dtype or g.numel() != p.numel():
+                raise ValueError("grad must match param in dtype and size")
+            recs.append((_ptr(p), _ptr(g), _ptr(s1), _ptr(s2), p.numel(),
+                         _torch_dtype_code(p)))
+        return cls(recs)
+
+
+def make_hyper(algo: str = "adam", lr: float = 1e-3, beta1: float = 0.9,
+               beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
+               beta3: float = 0.0, alpha: float = 0.0, skip_zeros: bool = False) -> Hyper:
+    return Hyper(lr, beta1, beta2, beta3, alpha, eps, weight_decay, ALGOS[algo],
+                 int(bool(skip_zeros)))
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+# ---------------------------------------------------------------------------
+# Entry points (same names as the C ABI)
+# ---------------------------------------------------------------------------
+
+def opt2s_step(tl: TensorList, hyper: Hyper, step: int, stream=None) -> None:
+    """One step of the whole collection in one launch (on torch's current
+    stream unless ``stream`` is given)."""
+    check(lib().opt2s_step(ctypes.byref(tl.desc), ctypes.byref(hyper), int(step),
+                           _stream_handle(stream)), "opt2s_step")
+
+
+class Plan:
+    """opt2s_plan_create / opt2s_plan_step / opt2s_plan_destroy."""
+
+    def __init__(self, tl: TensorList, algo: str):
+        self._h = ctypes.c_void_p()
+        self.tl = tl  # keep the descriptor alive with the plan
+        check(lib().opt2s_plan_create(ctypes.byref(tl.desc), ALGOS[algo],
+                                      ctypes.byref(self._h)), "opt2s_plan_create")
+
+    @property
+    def num_chunks(self) -> int:
+        return int(lib().opt2s_plan_num_chunks(self._h))
+
+    def step(self, hyper: Hyper, step: int, stream=None) -> None:
+        check(lib().opt2s_plan_step(self._h, ctypes.byref(hyper), int(step),
+                                    _stream_handle(stream)), "opt2s_plan_step")
+
+    def close(self) -> None:
+        if self._h:
+            check(lib().opt2s_plan_destroy(self._h), "opt2s_plan_destroy")
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def opt2s_release_cache() -> None:
+    check(lib().opt2s_release_cache(), "opt2s_release_cache")
+
+
+# ---------------------------------------------------------------------------
+# Validation scaffolding (include/opt2s_testing.h) -- tests only
+# ---------------------------------------------------------------------------
+
+def testing_build_chunks(tl: TensorList, algo: str, chunk_elems: int = 0) -> list:
+    L = lib()
+    n = ctypes.c_int64()
+    check(L.opt2s_testing_build_chunks(ctypes.byref(tl.desc), ALGOS[algo], chunk_elems,
+                                       None, 0, ctypes.byref(n)), "build_chunks")
+    arr = (opt2s_testing_chunk * max(n.value, 1))()
+    check(L.opt2s_testing_build_chunks(ctypes.byref(tl.desc), ALGOS[algo], chunk_elems,
+                                       arr, n.value, ctypes.byref(n)), "build_chunks")
+    return [(c.tensor, c.start, c.len, c.dtype) for c in arr[:n.value]]
+
+
+def testing_validate(tl: TensorList, hyper: Hyper, step: int) -> int:
+    return lib().opt2s_testing_validate(ctypes.byref(tl.desc), ctypes.byref(hyper), int(step))
+
+
+def testing_set_chunk_elems(n: int) -> int:
+    return int(lib().opt2s_testing_set_chunk_elems(int(n)))
+
+
+def testing_max_block_threads(algo: str, skip_zeros: bool) -> int:
+    r = int(lib().opt2s_testing_max_block_threads(ALGOS[algo], int(bool(skip_zeros))))
+    if r < 0:
+        check(r, "testing_max_block_threads")
+    return r
+
+
+def launch_count() -> int:
+    """Kernels launched by libopt2s.so so far in this process."""
+    return int(lib().opt2s_testing_launch_count())
+
+
+def testing_set_launch(block_threads: int = 0, max_blocks: int = 0) -> None:
+    check(lib().opt2s_testing_set_launch(int(block_threads), int(max_blocks)), "set_launch")

@@ -1,0 +1,457 @@
+// opt2s_api.cpp -- the C ABI of include/opt2s.h: argument validation, the
+// chunk-table builder, plans, and the per-device plan cache.
+//
+// The issue this library follows (bitsandbytes "Investigate a 256-thread
+// SM103 path for small 32-bit optimizer tensors") launches one kernel per
+// tensor (section "Problem"), so a model with thousands of bias / norm /
+// adapter tensors pays one launch each.  Here the host turns the whole
+// collection into a table of chunk records once, uploads it, and every later
+// step is a single launch that reads it.  The issue's section "Scope" asks
+// that per-device facts be cached per current device and that host dispatch
+// overhead stay small; both hold: plans are per device, and a repeated step
+// costs one descriptor comparison and one launch.
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <list>
+#include <mutex>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "opt2s.h"
+#include "opt2s_internal.h"
+#include "opt2s_testing.h"
+
+#define OPT2S_API extern "C" __attribute__((visibility("default")))
+
+using opt2s::ChunkRec;
+using opt2s::StepScalars;
+
+struct opt2s_plan {
+    int device;
+    int32_t algo;
+    int64_t nchunks;
+    ChunkRec* d_chunks;   // device copy of the chunk table
+};
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+int64_t g_chunk_elems = 0;     // testing override (0 = default)
+int g_block_threads = 0;       // testing override (0 = default)
+int g_max_blocks = 0;          // testing override (0 = occupancy cap)
+std::atomic<int64_t> g_launches{0};   // kernels launched by this library
+
+int cuda_fail(cudaError_t e)
+{
+    t_last_cuda_error = static_cast<int>(e);
+    return OPT2S_ERR_CUDA;
+}
+
+int64_t chunk_elems_now() { return g_chunk_elems > 0 ? g_chunk_elems : opt2s::kDefaultChunkElems; }
+int block_threads_now() { return g_block_threads > 0 ? g_block_threads : opt2s::kDefaultBlockThreads; }
+
+int elem_bytes(int32_t dtype) { return dtype == OPT2S_F32 ? 4 : 2; }
+
+// ---------------------------------------------------------------------------
+// Validation (host only, no CUDA call)
+// ---------------------------------------------------------------------------
+
+int validate_hyper(const Hyper* h, int step)
+{
+    if (!h) return OPT2S_ERR_INVALID_ARG;
+    if (h->algo != OPT2S_ADAM && h->algo != OPT2S_ADEMAMIX) return OPT2S_ERR_INVALID_ARG;
+    if (h->skip_zeros != 0 && h->skip_zeros != 1) return OPT2S_ERR_INVALID_ARG;
+    if (step < 1) return OPT2S_ERR_INVALID_ARG;
+    auto unit = [](float b) { return std::isfinite(b) && b >= 0.0f && b < 1.0f; };
+    if (!std::isfinite(h->lr) || !unit(h->beta1) || !unit(h->beta2)) return OPT2S_ERR_INVALID_ARG;
+    if (!std::isfinite(h->eps) || h->eps < 0.0f) return OPT2S_ERR_INVALID_ARG;
+    if (!std::isfinite(h->weight_decay)) return OPT2S_ERR_INVALID_ARG;
+    if (h->algo == OPT2S_ADEMAMIX && (!unit(h->beta3) || !std::isfinite(h->alpha)))
+        return OPT2S_ERR_INVALID_ARG;
+    return OPT2S_OK;
+}
+
+struct Range {
+    uintptr_t lo, hi;   // [lo, hi)
+    bool written;
+};
+
+// Every record well formed, and no buffer that is written overlaps any other
+// buffer (two gradients may share memory: both are only read).
+int validate_desc(const TensorListDesc* d, int32_t algo)
+{
+    if (!d) return OPT2S_ERR_INVALID_ARG;
+    if (algo != OPT2S_ADAM && algo != OPT2S_ADEMAMIX) return OPT2S_ERR_INVALID_ARG;
+    if (d->count < 0) return OPT2S_ERR_INVALID_ARG;
+    if (d->count > 0 && !d->tensors) return OPT2S_ERR_INVALID_ARG;
+    std::vector<Range> ranges;
+    for (int32_t i = 0; i < d->count; ++i) {
+        const opt2s_tensor& t = d->tensors[i];
+        if (t.numel < 0 || t.reserved != 0) return OPT2S_ERR_INVALID_ARG;
+        if (t.dtype != OPT2S_F32 && t.dtype != OPT2S_F16 && t.dtype != OPT2S_BF16)
+            return OPT2S_ERR_INVALID_ARG;
+        if (t.numel == 0) continue;
+        if (t.numel > (int64_t(1) << 40)) return OPT2S_ERR_INVALID_ARG;
+        if (!t.param || !t.grad || !t.state1 || !t.state2) return OPT2S_ERR_INVALID_ARG;
+        const int es = elem_bytes(t.dtype);
+        const auto p = reinterpret_cast<uintptr_t>(t.param);
+        const auto g = reinterpret_cast<uintptr_t>(t.grad);
+        const auto s1 = reinterpret_cast<uintptr_t>(t.state1);
+        const auto s2 = reinterpret_cast<uintptr_t>(t.state2);
+        if (p % es || g % es || s1 % 4 || s2 % 4) return OPT2S_ERR_INVALID_ARG;
+        const uintptr_t n = static_cast<uintptr_t>(t.numel);
+        const uintptr_t s1_elems = algo == OPT2S_ADEMAMIX ? 2 * n : n;
+        ranges.push_back({p, p + n * es, true});
+        ranges.push_back({g, g + n * es, false});
+        ranges.push_back({s1, s1 + s1_elems * 4, true});
+        ranges.push_back({s2, s2 + n * 4, true});
+    }
+    std::sort(ranges.begin(), ranges.end(),
+              [](const Range& a, const Range& b) { return a.lo < b.lo; });
+    // Sweep: compare each range with the furthest-reaching earlier range of
+    // each kind; any overlap involving a written range is an alias.
+    uintptr_t reach_w = 0, reach_any = 0;
+    bool have_w = false, have_any = false;
+    for (const Range& r : ranges) {
+        if (have_w && r.lo < reach_w) return OPT2S_ERR_ALIAS;
+        if (r.written && have_any && r.lo < reach_any) return OPT2S_ERR_ALIAS;
+        if (r.written) { reach_w = have_w ? std::max(reach_w, r.hi) : r.hi; have_w = true; }
+        reach_any = have_any ? std::max(reach_any, r.hi) : r.hi;
+        have_any = true;
+    }
+    return OPT2S_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Chunk-table builder
+// ---------------------------------------------------------------------------
+
+// Splits every tensor into chunks of at most `chunk_elems` elements, in
+// descriptor order.  Chunk starts are multiples of chunk_elems (a multiple of
+// 8), so a tensor whose arrays are 16-byte aligned keeps every chunk on the
+// 128-bit vector path.
+template <typename Emit>
+void for_each_chunk(const TensorListDesc* d, int64_t chunk_elems, Emit emit)
+{
+    for (int32_t i = 0; i < d->count; ++i) {
+        const opt2s_tensor& t = d->tensors[i];
+        for (int64_t s = 0; s < t.numel; s += chunk_elems)
+            emit(i, t, s, std::min(chunk_elems, t.numel - s));
+    }
+}
+
+int64_t count_chunks(const TensorListDesc* d, int64_t chunk_elems)
+{
+    int64_t n = 0;
+    for (int32_t i = 0; i < d->count; ++i)
+        n += (d->tensors[i].numel + chunk_elems - 1) / chunk_elems;
+    return n;
+}
+
+std::vector<ChunkRec> build_chunk_table(const TensorListDesc* d, int64_t chunk_elems)
+{
+    std::vector<ChunkRec> out;
+    out.reserve(static_cast<size_t>(count_chunks(d, chunk_elems)));
+    for_each_chunk(d, chunk_elems, [&](int32_t, const opt2s_tensor& t, int64_t s, int64_t len) {
+        const int es = elem_bytes(t.dtype);
+        ChunkRec r;
+        r.p = static_cast<char*>(t.param) + s * es;
+        r.g = static_cast<const char*>(t.grad) + s * es;
+        r.m = t.state1 + s;
+        r.v = t.state2 + s;
+        r.m2 = t.state1 + t.numel + s;
+        r.len = static_cast<uint32_t>(len);
+        r.dtype = t.dtype;
+        out.push_back(r);
+    });
+    return out;
+}
+
+int plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out)
+{
+    int st = validate_desc(desc, algo);
+    if (st != OPT2S_OK) return st;
+    const int64_t ce = chunk_elems_now();
+    if (count_chunks(desc, ce) > INT32_MAX) return OPT2S_ERR_TOO_LARGE;
+    std::vector<ChunkRec> table = build_chunk_table(desc, ce);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    auto* plan = new (std::nothrow) opt2s_plan{dev, algo, static_cast<int64_t>(table.size()), nullptr};
+    if (!plan) return OPT2S_ERR_NO_MEMORY;
+    if (!table.empty()) {
+        const size_t bytes = table.size() * sizeof(ChunkRec);
+        e = cudaMalloc(&plan->d_chunks, bytes);
+        if (e != cudaSuccess) {
+            delete plan;
+            if (e == cudaErrorMemoryAllocation) { t_last_cuda_error = e; return OPT2S_ERR_NO_MEMORY; }
+            return cuda_fail(e);
+        }
+        e = cudaMemcpy(plan->d_chunks, table.data(), bytes, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) {
+            cudaFree(plan->d_chunks);
+            delete plan;
+            return cuda_fail(e);
+        }
+    }
+    *out = plan;
+    return OPT2S_OK;
+}
+
+int plan_destroy(opt2s_plan* plan)
+{
+    if (!plan) return OPT2S_OK;
+    int st = OPT2S_OK;
+    if (plan->d_chunks) {
+        int cur = 0;
+        cudaError_t e = cudaGetDevice(&cur);
+        if (e == cudaSuccess && cur != plan->device) e = cudaSetDevice(plan->device);
+        if (e == cudaSuccess) e = cudaFree(plan->d_chunks);   // waits for the device
+        if (e != cudaSuccess) st = cuda_fail(e);
+        if (cur != plan->device) cudaSetDevice(cur);
+    }
+    delete plan;
+    return st;
+}
+
+StepScalars make_scalars(const Hyper* h, int step)
+{
+    StepScalars s;
+    s.lr = h->lr;
+    s.beta1 = h->beta1;
+    s.beta2 = h->beta2;
+    s.beta3 = h->beta3;
+    s.one_minus_beta1 = 1.0f - h->beta1;
+    s.one_minus_beta2 = 1.0f - h->beta2;
+    s.one_minus_beta3 = 1.0f - h->beta3;
+    s.alpha = h->alpha;
+    s.eps = h->eps;
+    s.bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(h->beta1), static_cast<double>(step)));
+    s.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(h->beta2), static_cast<double>(step)));
+    s.decay = static_cast<float>(1.0 - static_cast<double>(h->lr) * static_cast<double>(h->weight_decay));
+    return s;
+}
+
+int plan_step(const opt2s_plan* plan, const Hyper* h, int step, cudaStream_t stream)
+{
+    if (!plan) return OPT2S_ERR_INVALID_ARG;
+    int st = validate_hyper(h, step);
+    if (st != OPT2S_OK) return st;
+    if (h->algo != plan->algo) return OPT2S_ERR_INVALID_ARG;
+    if (plan->nchunks == 0) return OPT2S_OK;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev != plan->device) return OPT2S_ERR_DEVICE;
+    const int bt = block_threads_now();
+    if (bt != opt2s::kDefaultBlockThreads) {   // forced geometry: must fit the kernel
+        int widest = 0;
+        e = opt2s::max_block_threads(h->algo, h->skip_zeros, &widest);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (bt > widest) return OPT2S_ERR_INVALID_ARG;
+    }
+    e = opt2s::launch_step(plan->d_chunks, plan->nchunks, h->algo, h->skip_zeros,
+                           make_scalars(h, step), bt, g_max_blocks, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return OPT2S_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Per-device plan cache for opt2s_step, keyed by the descriptor's contents.
+// ---------------------------------------------------------------------------
+
+struct CacheEntry {
+    int device;
+    int32_t algo;
+    int64_t chunk_elems;
+    std::vector<opt2s_tensor> records;
+    opt2s_plan* plan;
+};
+
+constexpr size_t kCacheCapacity = 16;
+std::mutex g_cache_mu;
+std::list<CacheEntry> g_cache;   // most recently used first
+
+bool same_records(const CacheEntry& c, const TensorListDesc* d)
+{
+    return c.records.size() == static_cast<size_t>(d->count) &&
+           (d->count == 0 ||
+            std::memcmp(c.records.data(), d->tensors, sizeof(opt2s_tensor) * d->count) == 0);
+}
+
+bool all_empty(const TensorListDesc* d)
+{
+    for (int32_t i = 0; i < d->count; ++i)
+        if (d->tensors[i].numel != 0) return false;
+    return true;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Public entry points
+// ---------------------------------------------------------------------------
+
+OPT2S_API int opt2s_step(const TensorListDesc* desc, const Hyper* hyper, int step,
+                         cudaStream_t stream)
+{
+    int st = validate_hyper(hyper, step);
+    if (st != OPT2S_OK) return st;
+    if (!desc || desc->count < 0 || (desc->count > 0 && !desc->tensors))
+        return OPT2S_ERR_INVALID_ARG;
+    if (desc->count == 0) return OPT2S_OK;
+
+    int dev = 0;
+    const int64_t ce = chunk_elems_now();
+    std::unique_lock<std::mutex> lock(g_cache_mu);
+    const opt2s_plan* plan = nullptr;
+    {
+        // a cache hit needs no device query: compare on the device of the
+        // most recent entries first, then confirm the current device
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) {
+            // no usable device: still report argument errors first
+            int vs = validate_desc(desc, hyper->algo);
+            if (vs != OPT2S_OK) return vs;
+            if (all_empty(desc)) return OPT2S_OK;
+            return cuda_fail(e);
+        }
+        for (auto it = g_cache.begin(); it != g_cache.end(); ++it) {
+            if (it->device == dev && it->algo == hyper->algo && it->chunk_elems == ce &&
+                same_records(*it, desc)) {
+                if (it != g_cache.begin()) g_cache.splice(g_cache.begin(), g_cache, it);
+                plan = g_cache.front().plan;
+                break;
+            }
+        }
+    }
+    if (!plan) {
+        opt2s_plan* fresh = nullptr;
+        st = plan_create(desc, hyper->algo, &fresh);
+        if (st != OPT2S_OK) return st;
+        CacheEntry entry{dev, hyper->algo, ce,
+                         std::vector<opt2s_tensor>(desc->tensors, desc->tensors + desc->count), fresh};
+        g_cache.push_front(std::move(entry));
+        while (g_cache.size() > kCacheCapacity) {
+            plan_destroy(g_cache.back().plan);
+            g_cache.pop_back();
+        }
+        plan = fresh;
+    }
+    return plan_step(plan, hyper, step, stream);
+}
+
+OPT2S_API int opt2s_plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out_plan)
+{
+    if (!out_plan) return OPT2S_ERR_INVALID_ARG;
+    *out_plan = nullptr;
+    return plan_create(desc, algo, out_plan);
+}
+
+OPT2S_API int opt2s_plan_step(const opt2s_plan* plan, const Hyper* hyper, int step,
+                              cudaStream_t stream)
+{
+    return plan_step(plan, hyper, step, stream);
+}
+
+OPT2S_API int opt2s_plan_destroy(opt2s_plan* plan) { return plan_destroy(plan); }
+
+OPT2S_API int64_t opt2s_plan_num_chunks(const opt2s_plan* plan) { return plan ? plan->nchunks : -1; }
+
+OPT2S_API int opt2s_release_cache(void)
+{
+    std::lock_guard<std::mutex> lock(g_cache_mu);
+    int st = OPT2S_OK;
+    for (CacheEntry& c : g_cache) {
+        int s = plan_destroy(c.plan);
+        if (s != OPT2S_OK) st = s;
+    }
+    g_cache.clear();
+    return st;
+}
+
+OPT2S_API const char* opt2s_error_string(int status)
+{
+    switch (status) {
+    case OPT2S_OK: return "success";
+    case OPT2S_ERR_INVALID_ARG: return "invalid argument";
+    case OPT2S_ERR_ALIAS: return "a written buffer overlaps another buffer";
+    case OPT2S_ERR_NO_MEMORY: return "out of memory for the launch tables";
+    case OPT2S_ERR_CUDA: return "a CUDA call failed";
+    case OPT2S_ERR_DEVICE: return "plan used on another device than it was created on";
+    case OPT2S_ERR_TOO_LARGE: return "collection needs more chunks than a launch can index";
+    default: return "unknown status";
+    }
+}
+
+OPT2S_API int opt2s_last_cuda_error(void) { return t_last_cuda_error; }
+
+OPT2S_API int opt2s_abi_version(void) { return OPT2S_ABI_VERSION; }
+
+// ---------------------------------------------------------------------------
+// Validation scaffolding (include/opt2s_testing.h)
+// ---------------------------------------------------------------------------
+
+OPT2S_API int opt2s_testing_build_chunks(const TensorListDesc* desc, int32_t algo,
+                                         int64_t chunk_elems, opt2s_testing_chunk* out,
+                                         int64_t cap, int64_t* out_count)
+{
+    if (!out_count) return OPT2S_ERR_INVALID_ARG;
+    int st = validate_desc(desc, algo);
+    if (st != OPT2S_OK) return st;
+    const int64_t ce = chunk_elems > 0 ? chunk_elems : opt2s::kDefaultChunkElems;
+    const int64_t n = count_chunks(desc, ce);
+    *out_count = n;
+    if (!out) return OPT2S_OK;
+    if (cap < n) return OPT2S_ERR_INVALID_ARG;
+    int64_t k = 0;
+    for_each_chunk(desc, ce, [&](int32_t i, const opt2s_tensor& t, int64_t s, int64_t len) {
+        out[k++] = opt2s_testing_chunk{i, s, len, t.dtype, 0};
+    });
+    return OPT2S_OK;
+}
+
+OPT2S_API int opt2s_testing_validate(const TensorListDesc* desc, const Hyper* hyper, int step)
+{
+    int st = validate_hyper(hyper, step);
+    if (st != OPT2S_OK) return st;
+    return validate_desc(desc, hyper->algo);
+}
+
+OPT2S_API int64_t opt2s_testing_set_chunk_elems(int64_t chunk_elems)
+{
+    const int64_t prev = g_chunk_elems;
+    if (chunk_elems >= 0 && chunk_elems % 8 == 0 && chunk_elems <= (int64_t(1) << 31))
+        g_chunk_elems = chunk_elems;
+    return prev;
+}
+
+OPT2S_API int opt2s_testing_set_launch(int block_threads, int max_blocks)
+{
+    if (block_threads != 0 && (block_threads < 32 || block_threads > 1024 || block_threads % 32))
+        return OPT2S_ERR_INVALID_ARG;
+    if (max_blocks < 0) return OPT2S_ERR_INVALID_ARG;
+    g_block_threads = block_threads;
+    g_max_blocks = max_blocks;
+    return OPT2S_OK;
+}
+
+OPT2S_API int64_t opt2s_testing_default_chunk_elems(void) { return opt2s::kDefaultChunkElems; }
+
+OPT2S_API int opt2s_testing_max_block_threads(int32_t algo, int32_t skip_zeros)
+{
+    if ((algo != OPT2S_ADAM && algo != OPT2S_ADEMAMIX) || (skip_zeros != 0 && skip_zeros != 1))
+        return OPT2S_ERR_INVALID_ARG;
+    int widest = 0;
+    cudaError_t e = opt2s::max_block_threads(algo, skip_zeros, &widest);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return widest;
+}
+
+OPT2S_API int64_t opt2s_testing_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -1,0 +1,58 @@
+// Internal declarations shared by the host API (opt2s_api.cpp) and the
+// kernel translation unit (opt2s_kernel.cu).  Not installed, not public.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace opt2s {
+
+enum : int { kF32 = 0, kF16 = 1, kBF16 = 2 };
+enum : int { kAdam = 0, kAdEMAMix = 1 };
+
+// One work unit of a launch: a contiguous element range [0, len) of one
+// tensor, with every pointer already offset to the first element of the
+// range.  A warp processes one chunk at a time.
+struct alignas(16) ChunkRec {
+    void* p;          // param (storage dtype)
+    const void* g;    // grad  (storage dtype), read only
+    float* m;         // state1 (Adam m, AdEMAMix m1)
+    float* v;         // state2
+    float* m2;        // state1 + numel (AdEMAMix m2); not read by Adam
+    uint32_t len;     // elements in the chunk, >= 1
+    int32_t dtype;    // kF32 / kF16 / kBF16
+};
+static_assert(sizeof(ChunkRec) == 48, "ChunkRec layout");
+
+// Per-step scalars, all fp32 (the bias corrections and decay are evaluated in
+// double on the host and rounded once).
+struct StepScalars {
+    float lr;
+    float beta1, beta2, beta3;
+    float one_minus_beta1, one_minus_beta2, one_minus_beta3;
+    float alpha;
+    float eps;
+    float bc1, bc2;
+    float decay;
+};
+
+constexpr int kDefaultBlockThreads = 256;
+constexpr int64_t kDefaultChunkElems = 8192;
+
+// Launches one step over `nchunks` records at `d_chunks` (device memory) on
+// `stream`.  block_threads: multiple of 32; max_blocks <= 0: occupancy-based
+// cap (resident blocks per SM x SM count).  Returns the launch status.
+cudaError_t launch_step(const ChunkRec* d_chunks, int64_t nchunks, int algo,
+                        int skip_zeros, const StepScalars& s,
+                        int block_threads, int max_blocks,
+                        cudaStream_t stream);
+
+// Widest block (threads, a multiple of 32) the step kernel for (algo,
+// skip_zeros) can be launched with: its registers per thread limit it.
+cudaError_t max_block_threads(int algo, int skip_zeros, int* out);
+
+// Number of blocks a launch of `nchunks` chunks uses on the current device.
+cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros,
+                     int block_threads, int max_blocks, int* grid);
+
+}  // namespace opt2s

@@ -1,0 +1,361 @@
+// opt2s_kernel.cu -- the persistent multi-tensor optimizer-step kernel for
+// B200 (sm_100a).
+//
+// One launch steps a whole tensor collection.  The host splits every tensor
+// into chunks of at most a few thousand elements (opt2s_api.cpp); each warp
+// takes chunks c = warp, warp + total_warps, ... and streams through them with
+// 128-bit loads and stores, so 2,000 tiny bias/norm tensors cost one launch
+// and a multi-GB tensor is spread over every SM.  The path has no cross-
+// element reduction and no data reuse, so there is no shared-memory staging
+// and no tensor-core work: it is bound by HBM bandwidth (28 bytes per element
+// for fp32 Adam, 36 for fp32 AdEMAMix).
+//
+// Arithmetic: the 32-bit two-state update of bitsandbytes issue "Investigate
+// a 256-thread SM103 path for small 32-bit optimizer tensors" (sections
+// "Problem", "Scope", "Correctness oracle"), with the standard Adam (Kingma &
+// Ba 2015, Algorithm 1), decoupled weight decay (Loshchilov & Hutter 2019,
+// Algorithm 2) and AdEMAMix (Pagliardini et al. 2024, Algorithm 1)
+// definitions.  Every operation is an explicit round-to-nearest intrinsic
+// (__fmul_rn / __fadd_rn / __fdiv_rn / __fsqrt_rn), which the compiler may not
+// contract into FMA, so the result of an element never depends on which code
+// path (vector body, scalar head/tail), chunk, warp or block computed it: the
+// issue's "Correctness oracle" section requires that launch geometry must not
+// change optimizer arithmetic.
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "opt2s_internal.h"
+
+namespace opt2s {
+namespace {
+
+// ---------------------------------------------------------------------------
+// The per-element update.  With SKIP, an element whose gradient compares equal
+// to zero (+0 or -0) is left untouched (no decay either).
+// ---------------------------------------------------------------------------
+template <int ALGO, bool SKIP>
+__device__ __forceinline__ void update(float g, float& p, float& m, float& v,
+                                       float& m2, const StepScalars& s)
+{
+    if (SKIP && g == 0.0f) return;
+    m = __fadd_rn(__fmul_rn(s.beta1, m), __fmul_rn(s.one_minus_beta1, g));
+    v = __fadd_rn(__fmul_rn(s.beta2, v),
+                  __fmul_rn(__fmul_rn(s.one_minus_beta2, g), g));
+    float num = __fdiv_rn(m, s.bc1);
+    if (ALGO == kAdEMAMix) {
+        m2 = __fadd_rn(__fmul_rn(s.beta3, m2), __fmul_rn(s.one_minus_beta3, g));
+        num = __fadd_rn(num, __fmul_rn(s.alpha, m2));
+    }
+    const float den = __fadd_rn(__fsqrt_rn(__fdiv_rn(v, s.bc2)), s.eps);
+    p = __fsub_rn(__fmul_rn(p, s.decay), __fmul_rn(s.lr, __fdiv_rn(num, den)));
+}
+
+// ---------------------------------------------------------------------------
+// Storage traits of param / grad.  kVec elements make one 16-byte access.
+// Loads and stores use the streaming (evict-first) cache policy: every byte is
+// touched exactly once per step.
+// ---------------------------------------------------------------------------
+template <int DT> struct Param;
+
+template <> struct Param<kF32> {
+    static constexpr int kVec = 4;
+    static constexpr int kBytes = 4;
+    using Raw = float4;
+    __device__ static Raw load(const void* b, uint32_t i) {
+        return __ldcs(reinterpret_cast<const float4*>(static_cast<const float*>(b) + i));
+    }
+    __device__ static void store(void* b, uint32_t i, const Raw& r) {
+        __stcs(reinterpret_cast<float4*>(static_cast<float*>(b) + i), r);
+    }
+    __device__ static void widen(const Raw& r, float (&x)[4]) {
+        x[0] = r.x; x[1] = r.y; x[2] = r.z; x[3] = r.w;
+    }
+    __device__ static Raw narrow(const float (&x)[4], const Raw&, const float (&)[4], bool) {
+        // fp32: an untouched element already holds its loaded bits
+        return make_float4(x[0], x[1], x[2], x[3]);
+    }
+    __device__ static float load1(const void* b, uint32_t i) {
+        return __ldcs(static_cast<const float*>(b) + i);
+    }
+    __device__ static void store1(void* b, uint32_t i, float x) {
+        __stcs(static_cast<float*>(b) + i, x);
+    }
+};
+
+// Shared by the two 16-bit formats: only the conversions differ.
+template <typename H2, typename Cvt> struct Param16 {
+    static constexpr int kVec = 8;
+    static constexpr int kBytes = 2;
+    using Raw = uint4;
+    __device__ static Raw load(const void* b, uint32_t i) {
+        return __ldcs(reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(b) + i));
+    }
+    __device__ static void store(void* b, uint32_t i, const Raw& r) {
+        __stcs(reinterpret_cast<uint4*>(static_cast<unsigned short*>(b) + i), r);
+    }
+    __device__ static void widen(const Raw& r, float (&x)[8]) {
+        const H2* h = reinterpret_cast<const H2*>(&r);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = Cvt::to_float2(h[k]);
+            x[2 * k] = f.x;
+            x[2 * k + 1] = f.y;
+        }
+    }
+    // Round to nearest even; with `skip`, elements whose gradient is zero keep
+    // their original storage bits exactly (NaN payloads included).
+    __device__ static Raw narrow(const float (&x)[8], const Raw& orig,
+                                 const float (&g)[8], bool skip) {
+        Raw r;
+        H2* h = reinterpret_cast<H2*>(&r);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) h[k] = Cvt::from_float2(x[2 * k], x[2 * k + 1]);
+        if (skip) {
+            uint32_t* w = reinterpret_cast<uint32_t*>(&r);
+            const uint32_t* o = reinterpret_cast<const uint32_t*>(&orig);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t mask = 0xFFFFu << (16 * (j & 1));
+                if (g[j] == 0.0f) w[j >> 1] = (w[j >> 1] & ~mask) | (o[j >> 1] & mask);
+            }
+        }
+        return r;
+    }
+    __device__ static float load1(const void* b, uint32_t i) {
+        return Cvt::to_float(__ldcs(static_cast<const unsigned short*>(b) + i));
+    }
+    __device__ static void store1(void* b, uint32_t i, float x) {
+        __stcs(static_cast<unsigned short*>(b) + i, Cvt::from_float(x));
+    }
+};
+
+struct CvtF16 {
+    __device__ static float2 to_float2(__half2 h) { return __half22float2(h); }
+    __device__ static __half2 from_float2(float a, float b) { return __floats2half2_rn(a, b); }
+    __device__ static float to_float(unsigned short u) { return __half2float(__ushort_as_half(u)); }
+    __device__ static unsigned short from_float(float x) { return __half_as_ushort(__float2half_rn(x)); }
+};
+
+struct CvtBF16 {
+    __device__ static float2 to_float2(__nv_bfloat162 h) { return __bfloat1622float2(h); }
+    __device__ static __nv_bfloat162 from_float2(float a, float b) { return __floats2bfloat162_rn(a, b); }
+    __device__ static float to_float(unsigned short u) { return __bfloat162float(__ushort_as_bfloat16(u)); }
+    __device__ static unsigned short from_float(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+};
+
+template <> struct Param<kF16> : Param16<__half2, CvtF16> {};
+template <> struct Param<kBF16> : Param16<__nv_bfloat162, CvtBF16> {};
+
+// fp32 state: N elements as N/4 16-byte accesses.
+template <int N>
+__device__ __forceinline__ void load_state(const float* b, uint32_t i, float (&x)[N]) {
+#pragma unroll
+    for (int k = 0; k < N / 4; ++k) {
+        const float4 t = __ldcs(reinterpret_cast<const float4*>(b + i) + k);
+        x[4 * k] = t.x; x[4 * k + 1] = t.y; x[4 * k + 2] = t.z; x[4 * k + 3] = t.w;
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void store_state(float* b, uint32_t i, const float (&x)[N]) {
+#pragma unroll
+    for (int k = 0; k < N / 4; ++k)
+        __stcs(reinterpret_cast<float4*>(b + i) + k,
+               make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]));
+}
+
+// One element through the scalar path (chunk head, tail, or a chunk whose
+// arrays are not mutually 16-byte aligned).  A skipped element is not even
+// written back.
+template <int DT, int ALGO, bool SKIP>
+__device__ __forceinline__ void scalar_element(const ChunkRec& c, uint32_t i,
+                                               const StepScalars& s)
+{
+    using P = Param<DT>;
+    const float g = P::load1(c.g, i);
+    if (SKIP && g == 0.0f) return;
+    float p = P::load1(c.p, i);
+    float m = __ldcs(c.m + i);
+    float v = __ldcs(c.v + i);
+    float m2 = 0.0f;
+    if (ALGO == kAdEMAMix) m2 = __ldcs(c.m2 + i);
+    update<ALGO, false>(g, p, m, v, m2, s);
+    P::store1(c.p, i, p);
+    __stcs(c.m + i, m);
+    __stcs(c.v + i, v);
+    if (ALGO == kAdEMAMix) __stcs(c.m2 + i, m2);
+}
+
+__device__ __forceinline__ bool aligned16(const void* q, uint32_t head, int bytes) {
+    return ((reinterpret_cast<uintptr_t>(q) + static_cast<uintptr_t>(head) * bytes) & 15u) == 0;
+}
+
+// One chunk, processed by one warp.  Every lane moves 8 elements per
+// iteration (two 16-byte vectors of fp32, or one of fp16/bf16), so a warp
+// iteration covers 256 contiguous elements of each array.
+template <int DT, int ALGO, bool SKIP>
+__device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& s, int lane)
+{
+    using P = Param<DT>;
+    constexpr int V = P::kVec;
+    constexpr int U = 8 / V;
+    const uint32_t len = c.len;
+
+    // The first element at which param is 16-byte aligned; the vector path
+    // needs every array aligned at that same element.
+    uint32_t head = static_cast<uint32_t>(
+        ((16u - (reinterpret_cast<uintptr_t>(c.p) & 15u)) & 15u) / P::kBytes);
+    const bool vec_ok = aligned16(c.g, head, P::kBytes) && aligned16(c.m, head, 4) &&
+                        aligned16(c.v, head, 4) &&
+                        (ALGO != kAdEMAMix || aligned16(c.m2, head, 4));
+    if (!vec_ok || head > len) head = len;
+    const uint32_t nvec = (len - head) / V;
+    const uint32_t body_end = head + nvec * V;
+
+    for (uint32_t i = lane; i < head; i += 32) scalar_element<DT, ALGO, SKIP>(c, i, s);
+    for (uint32_t i = body_end + lane; i < len; i += 32) scalar_element<DT, ALGO, SKIP>(c, i, s);
+
+    for (uint32_t v0 = 0; v0 < nvec; v0 += 32 * U) {
+        typename P::Raw graw[U], praw[U];
+        float m[U][V], v[U][V], m2[U][V];
+        // all loads of the iteration first, so they are in flight together
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t vi = v0 + u * 32 + lane;
+            if (vi < nvec) {
+                const uint32_t e = head + vi * V;
+                graw[u] = P::load(c.g, e);
+                praw[u] = P::load(c.p, e);
+                load_state<V>(c.m, e, m[u]);
+                load_state<V>(c.v, e, v[u]);
+                if (ALGO == kAdEMAMix) load_state<V>(c.m2, e, m2[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t vi = v0 + u * 32 + lane;
+            if (vi < nvec) {
+                const uint32_t e = head + vi * V;
+                float g[V], p[V];
+                P::widen(graw[u], g);
+                P::widen(praw[u], p);
+#pragma unroll
+                for (int j = 0; j < V; ++j)
+                    update<ALGO, SKIP>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s);
+                P::store(c.p, e, P::narrow(p, praw[u], g, SKIP));
+                store_state<V>(c.m, e, m[u]);
+                store_state<V>(c.v, e, v[u]);
+                if (ALGO == kAdEMAMix) store_state<V>(c.m2, e, m2[u]);
+            }
+        }
+    }
+}
+
+template <int ALGO, bool SKIP>
+__global__ void step_kernel(const ChunkRec* __restrict__ chunks, int nchunks, StepScalars s)
+{
+    const int lane = threadIdx.x & 31;
+    const int warps_per_block = blockDim.x >> 5;
+    const int warp = blockIdx.x * warps_per_block + (threadIdx.x >> 5);
+    const int nwarps = gridDim.x * warps_per_block;
+    for (int c = warp; c < nchunks; c += nwarps) {
+        const ChunkRec rec = chunks[c];
+        switch (rec.dtype) {
+        case kF32: run_chunk<kF32, ALGO, SKIP>(rec, s, lane); break;
+        case kF16: run_chunk<kF16, ALGO, SKIP>(rec, s, lane); break;
+        default: run_chunk<kBF16, ALGO, SKIP>(rec, s, lane); break;
+        }
+    }
+}
+
+using KernelFn = void (*)(const ChunkRec*, int, StepScalars);
+
+KernelFn pick(int algo, int skip)
+{
+    if (algo == kAdEMAMix) return skip ? step_kernel<kAdEMAMix, true> : step_kernel<kAdEMAMix, false>;
+    return skip ? step_kernel<kAdam, true> : step_kernel<kAdam, false>;
+}
+
+// Resident blocks per SM and SM count, cached per device (and kernel / block
+// size): device attributes are per device, not per process.
+constexpr int kMaxDevices = 64;
+struct OccEntry { int block_threads; int blocks_per_sm; };
+struct DeviceInfo { int sms; OccEntry occ[4][6]; };
+DeviceInfo g_info[kMaxDevices];
+bool g_info_ok[kMaxDevices];
+
+cudaError_t device_info(int dev, DeviceInfo** out)
+{
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!g_info_ok[dev]) {
+        int sms = 0;
+        cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        g_info[dev].sms = sms;
+        for (auto& row : g_info[dev].occ)
+            for (auto& x : row) x = OccEntry{0, 0};
+        g_info_ok[dev] = true;
+    }
+    *out = &g_info[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros, int block_threads,
+                     int max_blocks, int* grid)
+{
+    const int warps_per_block = block_threads / 32;
+    const int64_t need = (nchunks + warps_per_block - 1) / warps_per_block;
+    int cap = max_blocks;
+    if (cap <= 0) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        DeviceInfo* info = nullptr;
+        if ((e = device_info(dev, &info)) != cudaSuccess) return e;
+        const int k = (algo == kAdEMAMix ? 2 : 0) + (skip_zeros ? 1 : 0);
+        int per_sm = 0;
+        for (auto& x : info->occ[k])
+            if (x.block_threads == block_threads) per_sm = x.blocks_per_sm;
+        if (per_sm == 0) {
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                &per_sm, pick(algo, skip_zeros), block_threads, 0);
+            if (e != cudaSuccess) return e;
+            if (per_sm < 1) per_sm = 1;
+            for (auto& x : info->occ[k])
+                if (x.block_threads == 0) { x = OccEntry{block_threads, per_sm}; break; }
+        }
+        cap = per_sm * info->sms;
+    }
+    *grid = static_cast<int>(need < cap ? need : cap);
+    return cudaSuccess;
+}
+
+cudaError_t max_block_threads(int algo, int skip_zeros, int* out)
+{
+    cudaFuncAttributes attr;
+    cudaError_t e = cudaFuncGetAttributes(&attr, pick(algo, skip_zeros));
+    if (e != cudaSuccess) return e;
+    *out = attr.maxThreadsPerBlock / 32 * 32;
+    return cudaSuccess;
+}
+
+cudaError_t launch_step(const ChunkRec* d_chunks, int64_t nchunks, int algo, int skip_zeros,
+                        const StepScalars& s, int block_threads, int max_blocks,
+                        cudaStream_t stream)
+{
+    if (nchunks <= 0) return cudaSuccess;
+    int grid = 0;
+    cudaError_t e = grid_for(nchunks, algo, skip_zeros, block_threads, max_blocks, &grid);
+    if (e != cudaSuccess) return e;
+    int n = static_cast<int>(nchunks);
+    StepScalars sc = s;
+    void* args[] = {const_cast<ChunkRec**>(&d_chunks), &n, &sc};
+    return cudaLaunchKernel(reinterpret_cast<const void*>(pick(algo, skip_zeros)),
+                            dim3(grid), dim3(block_threads), args, 0, stream);
+}
+
+}  // namespace opt2s

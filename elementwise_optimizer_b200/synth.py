@@ -90,7 +90,18 @@ def sparse_mixture(seed: int, stream: tuple, n: int, std: float,
 
 @dataclass
 class Workload:
-    """A tensor collection, its hyper-parameters and its gradient recipe."""
+    """A tensor collection, its hyper-parameters and its gradient recipe.
+
+    Two ways to draw values, both pure functions of (seed, tensor, step):
+      * direct (collections whose total size is below ``ring_threshold``):
+        every step draws fresh values for the whole collection from its own
+        Philox stream;
+      * ring (larger collections): one seeded pool of ``pool_len`` values per
+        quantity, and tensor i at step t reads the pool rotated by a seeded
+        offset, ``pool[(offset(i, t) + j) % pool_len]``.  Any element of any
+        step can then be rebuilt from its index alone, which lets the oracle
+        check a sample of a multi-GB step without regenerating it.
+    """
     name: str
     sizes: list
     dtypes: list
@@ -102,6 +113,7 @@ class Workload:
     grad_std: float = 1e-2
     param_std: float = 1.0
     skip_zeros: bool = False
+    ring_threshold: int = 1 << 24
     notes: str = ""
     extra: dict = field(default_factory=dict)
 
@@ -109,22 +121,79 @@ class Workload:
     def numel(self) -> int:
         return int(sum(self.sizes))
 
-    def param_init(self, i: int) -> np.ndarray:
-        """Initial values (float32) of tensor ``i``."""
-        return normal(self.seed, (1, i), self.sizes[i], self.param_std)
+    @property
+    def ring(self) -> bool:
+        return self.numel > self.ring_threshold
 
-    def grad(self, i: int, step: int) -> np.ndarray:
-        """Gradient values (float32) of tensor ``i`` at 1-based ``step``."""
-        n = self.sizes[i]
-        stream = (2 + step, i)
+    @property
+    def pool_len(self) -> int:
+        return int(max(max(self.sizes), 1 << 20))
+
+    # ---- direct mode ------------------------------------------------------
+    def _grad_values(self, g: np.random.Generator, n: int, std_per_elem=None) -> np.ndarray:
         if self.grad_kind == "normal":
-            return normal(self.seed, stream, n, self.grad_std)
+            return (g.standard_normal(n, dtype=np.float32) * np.float32(self.grad_std)).astype(np.float32)
         if self.grad_kind == "sparse_mixture":
-            std = 1e-3 if i % 2 == 0 else 10.0
-            return sparse_mixture(self.seed, stream, n, std, 0.10)
+            out = (g.standard_normal(n, dtype=np.float32) * std_per_elem).astype(np.float32)
+            out[g.random(n) < 0.10] = 0.0
+            return out
         if self.grad_kind == "mixed_magnitude":
-            return mixed_magnitude(self.seed, stream, n)
+            mag = np.exp(g.uniform(np.log(1e-6), np.log(1e2), n)).astype(np.float32)
+            sign = np.where(g.random(n) < 0.5, np.float32(-1), np.float32(1))
+            out = (mag * sign).astype(np.float32)
+            out[g.random(n) < 0.05] = 0.0
+            return out
         raise ValueError(self.grad_kind)
+
+    def _split(self, flat: np.ndarray) -> list:
+        return np.split(flat, np.cumsum(self.sizes)[:-1])
+
+    def _std_per_elem(self) -> np.ndarray:
+        """sparse_mixture: tensor i draws from N(0, 1e-3) if i is even, else
+        N(0, 10)."""
+        stds = np.where(np.arange(len(self.sizes)) % 2 == 0, np.float32(1e-3), np.float32(10.0))
+        return np.repeat(stds.astype(np.float32), self.sizes)
+
+    def params_init(self) -> list:
+        """Initial param values (float32, already representable in each
+        tensor's storage dtype) of every tensor, direct mode."""
+        flat = normal(self.seed, (1,), self.numel, self.param_std)
+        return [from_storage(to_storage(x, d), d) for x, d in zip(self._split(flat), self.dtypes)]
+
+    def grads(self, step: int) -> list:
+        """Gradient values (float32, representable in each storage dtype) of
+        every tensor at 1-based ``step``, direct mode."""
+        g = rng(self.seed, 2, step)
+        std = self._std_per_elem() if self.grad_kind == "sparse_mixture" else None
+        flat = self._grad_values(g, self.numel, std)
+        return [from_storage(to_storage(x, d), d) for x, d in zip(self._split(flat), self.dtypes)]
+
+    # ---- ring mode --------------------------------------------------------
+    def pool(self, which: str) -> np.ndarray:
+        """The seeded pool of float32 values for 'param' or 'grad'."""
+        key = "_pool_" + which
+        if key not in self.extra:
+            if which == "param":
+                vals = normal(self.seed, (5,), self.pool_len, self.param_std)
+            else:
+                std = np.full(self.pool_len, np.float32(self.grad_std), np.float32)
+                if self.grad_kind == "sparse_mixture":
+                    std = np.where(np.arange(self.pool_len) % 2 == 0, np.float32(1e-3),
+                                   np.float32(10.0)).astype(np.float32)
+                vals = self._grad_values(rng(self.seed, 6), self.pool_len, std)
+            self.extra[key] = vals
+        return self.extra[key]
+
+    def offset(self, i: int, step: int) -> int:
+        """Rotation of the pool for tensor i at ``step`` (step 0 = param init)."""
+        return int(rng(self.seed, 7, step, i).integers(0, self.pool_len))
+
+    def ring_values(self, which: str, i: int, step: int, idx: np.ndarray) -> np.ndarray:
+        """Values of tensor i at element indices ``idx`` (float32,
+        representable in the tensor's storage dtype)."""
+        pool = self.pool(which)
+        vals = pool[(self.offset(i, step) + idx) % self.pool_len]
+        return from_storage(to_storage(vals, self.dtypes[i]), self.dtypes[i])
 
 
 ADAM_HYPER = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, beta3=0.0,

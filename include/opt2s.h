@@ -1,0 +1,161 @@
+/*
+ * opt2s.h -- C ABI of the B200 (sm_100a) 32-bit two-state optimizer step.
+ *
+ * What is computed
+ * ----------------
+ * One in-place update of param, state1 and state2 from a gradient, element by
+ * element, with no cross-element reduction, over a collection of tensors in a
+ * single kernel launch.  The method is the "32-bit two-state" optimizer update
+ * of bitsandbytes issue "Investigate a 256-thread SM103 path for small 32-bit
+ * optimizer tensors" (section "Problem": the kOptimizer32bit2State update with
+ * fp32 state; section "Scope": decoupled weight decay applied before the
+ * update; section "Correctness oracle": ADAM/AdamW and ADEMAMIX, FP16/BF16/FP32
+ * param and grad storage, weight decay and skip_zeros, gradient unchanged,
+ * and launch geometry must not change the arithmetic).  The formulas are the
+ * standard ones: Adam (Kingma & Ba 2015, Algorithm 1), decoupled weight decay
+ * (Loshchilov & Hutter 2019, Algorithm 2) and AdEMAMix (Pagliardini et al.
+ * 2024, Algorithm 1).  Per element, at step t >= 1, every operation rounded
+ * to fp32 in this order (no fused multiply-add, no flush-to-zero):
+ *
+ *     if (skip_zeros && g == 0)  leave the element wholly unchanged
+ *     m   = beta1*m + (1-beta1)*g
+ *     v   = beta2*v + ((1-beta2)*g)*g
+ *     num = m / bc1                                   bc1 = 1 - beta1^t
+ *     AdEMAMix:  m2  = beta3*m2 + (1-beta3)*g
+ *                num = num + alpha*m2
+ *     den = sqrt(v / bc2) + eps                       bc2 = 1 - beta2^t
+ *     p   = p*decay - lr*(num/den)                    decay = 1 - lr*wd
+ *
+ * bc1, bc2 and decay are evaluated in double on the host and rounded to fp32
+ * once.  fp16/bf16 param and grad are widened exactly; the new param is
+ * narrowed with round-to-nearest-even.  State is always fp32.
+ *
+ * Memory layout and ownership
+ * ---------------------------
+ * All tensor buffers are DEVICE memory owned by the caller (e.g. allocated by
+ * PyTorch), contiguous, and must stay valid until the step's work on `stream`
+ * has finished.  Per tensor of `numel` elements:
+ *     param   numel elements of `dtype`           read and written
+ *     grad    numel elements of `dtype`           read only, never written
+ *     state1  Adam: m, numel floats               read and written
+ *             AdEMAMix: [m1 | m2], 2*numel floats (m2 starts at state1+numel)
+ *     state2  v, numel floats                     read and written
+ * State must be zero-filled by the caller before step 1.  Pointers need only
+ * element alignment (torch storage offsets are fine); 16-byte alignment of all
+ * arrays at the same element gives the 128-bit vector path, anything else
+ * takes a scalar path with bitwise identical results.
+ * The library owns only its launch tables (device memory plus host copies),
+ * held by a plan; opt2s_step keeps plans in a per-device cache that
+ * opt2s_release_cache() frees.
+ *
+ * Errors
+ * ------
+ * Every entry point returns OPT2S_OK (0) or a negative opt2s_status.  All
+ * arguments are validated before any launch, so an argument error never
+ * leaves a partial update.  OPT2S_ERR_CUDA means a CUDA call failed; the
+ * CUDA error is kept in opt2s_last_cuda_error().  Calls are asynchronous with
+ * respect to the host: execution errors of the kernel surface at the next
+ * synchronizing CUDA call.
+ */
+#ifndef OPT2S_H
+#define OPT2S_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define OPT2S_ABI_VERSION 1
+
+/* Storage type of param and grad.  State is always fp32. */
+typedef enum { OPT2S_F32 = 0, OPT2S_F16 = 1, OPT2S_BF16 = 2 } opt2s_dtype;
+
+/* OPT2S_ADAM is Adam, and AdamW when weight_decay != 0. */
+typedef enum { OPT2S_ADAM = 0, OPT2S_ADEMAMIX = 1 } opt2s_algo;
+
+typedef enum {
+    OPT2S_OK = 0,
+    OPT2S_ERR_INVALID_ARG = -1, /* null pointer, bad size/dtype/algo/step, non-finite or
+                                   out-of-range hyper-parameter, misaligned element */
+    OPT2S_ERR_ALIAS = -2,       /* a written buffer overlaps another buffer */
+    OPT2S_ERR_NO_MEMORY = -3,   /* the library could not allocate its tables */
+    OPT2S_ERR_CUDA = -4,        /* a CUDA call failed (see opt2s_last_cuda_error) */
+    OPT2S_ERR_DEVICE = -5,      /* plan used on another device than it was made on */
+    OPT2S_ERR_TOO_LARGE = -6    /* more chunks than the launch tables can index */
+} opt2s_status;
+
+/* One tensor of the collection (all pointers are device pointers). */
+typedef struct {
+    void *param;
+    const void *grad;
+    float *state1;
+    float *state2;
+    int64_t numel;      /* >= 0; 0 means "skip this record" */
+    int32_t dtype;      /* opt2s_dtype, for param and grad */
+    int32_t reserved;   /* must be 0 */
+} opt2s_tensor;
+
+/* The collection: a HOST array of `count` records (count >= 0). */
+typedef struct {
+    const opt2s_tensor *tensors;
+    int32_t count;
+} TensorListDesc;
+
+/* Hyper-parameters of one step.  beta1, beta2 (and beta3 for AdEMAMix) in
+ * [0, 1); eps >= 0; lr, alpha, weight_decay finite; skip_zeros 0 or 1.
+ * beta3 and alpha are ignored by Adam. */
+typedef struct {
+    float lr, beta1, beta2, beta3, alpha, eps, weight_decay;
+    int32_t algo;       /* opt2s_algo */
+    int32_t skip_zeros; /* 1: elements whose grad is +0 or -0 are left unchanged */
+} Hyper;
+
+/*
+ * One optimizer step over the whole collection, in ONE kernel launch on
+ * `stream` (0 = legacy default stream), on the current CUDA device.
+ * `step` is the 1-based index t of this update (t >= 1).
+ * The launch tables for `desc` come from a per-device cache keyed by the
+ * descriptor's contents and the algorithm; the first call with a new
+ * collection builds them (host work plus a synchronous upload), later calls
+ * only launch.  An empty collection (count == 0 or all numel == 0) is a no-op.
+ */
+int opt2s_step(const TensorListDesc *desc, const Hyper *hyper, int step,
+               cudaStream_t stream);
+
+/*
+ * Explicit plans, for callers that step the same collection many times and
+ * want no per-call descriptor lookup.  opt2s_plan_create validates `desc` for
+ * `algo`, builds the chunk table and uploads it to the current device
+ * (synchronously).  opt2s_plan_step launches the step (hyper->algo must equal
+ * the plan's algo; the current device must be the plan's device).
+ * opt2s_plan_destroy waits for the device and frees the plan; NULL is a no-op.
+ */
+typedef struct opt2s_plan opt2s_plan;
+int opt2s_plan_create(const TensorListDesc *desc, int32_t algo,
+                      opt2s_plan **out_plan);
+int opt2s_plan_step(const opt2s_plan *plan, const Hyper *hyper, int step,
+                    cudaStream_t stream);
+int opt2s_plan_destroy(opt2s_plan *plan);
+
+/* Number of chunk records in a plan (the work units of one launch). */
+int64_t opt2s_plan_num_chunks(const opt2s_plan *plan);
+
+/* Frees every cached plan of every device (waits for the devices first). */
+int opt2s_release_cache(void);
+
+/* Human-readable text for a status code (static storage). */
+const char *opt2s_error_string(int status);
+
+/* The cudaError_t of the last failed CUDA call in this thread (0 if none). */
+int opt2s_last_cuda_error(void);
+
+/* OPT2S_ABI_VERSION of the loaded library. */
+int opt2s_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OPT2S_H */

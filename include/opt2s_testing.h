@@ -1,0 +1,75 @@
+/*
+ * opt2s_testing.h -- validation scaffolding for the test suite.  NOT part of
+ * the public API.
+ *
+ * bitsandbytes issue "Investigate a 256-thread SM103 path for small 32-bit
+ * optimizer tensors", section "Scope", allows experimental forcing only in
+ * validation scaffolding, never as a public API; these entry points are that
+ * scaffolding.  They let the tests (a) run the host-side validation and
+ * chunk-table builder without a GPU and (b) force other launch geometries, to
+ * check the issue's "Correctness oracle" requirement that the launch geometry
+ * must not change the optimizer arithmetic (results must be bitwise equal).
+ *
+ * All knobs are process-wide, apply to plans created or launched afterwards,
+ * and are not thread-safe against concurrent steps.
+ */
+#ifndef OPT2S_TESTING_H
+#define OPT2S_TESTING_H
+
+#include "opt2s.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* One work unit of a launch as the host builder produced it. */
+typedef struct {
+    int64_t tensor;   /* index into the descriptor */
+    int64_t start;    /* first element of the chunk within the tensor */
+    int64_t len;      /* number of elements, 1..chunk_elems */
+    int32_t dtype;    /* opt2s_dtype of the tensor */
+    int32_t reserved;
+} opt2s_testing_chunk;
+
+/*
+ * Host only (no CUDA call): validate `desc` for `algo` exactly as
+ * opt2s_plan_create does and write its chunk list (in launch order) to `out`
+ * (capacity `cap` records; `out` may be NULL to query the count).
+ * chunk_elems <= 0 selects the library default.  *out_count receives the
+ * number of chunks.  Returns OPT2S_OK, a validation error, or
+ * OPT2S_ERR_INVALID_ARG when cap is too small.
+ */
+int opt2s_testing_build_chunks(const TensorListDesc *desc, int32_t algo,
+                               int64_t chunk_elems, opt2s_testing_chunk *out,
+                               int64_t cap, int64_t *out_count);
+
+/* Host only: the validation opt2s_step performs before any CUDA call. */
+int opt2s_testing_validate(const TensorListDesc *desc, const Hyper *hyper,
+                           int step);
+
+/* Chunk length (elements, a positive multiple of 8) for plans created
+ * afterwards; 0 restores the default.  Returns the previous value. */
+int64_t opt2s_testing_set_chunk_elems(int64_t chunk_elems);
+
+/* Threads per block (a multiple of 32 in [32, 1024]) and a cap on blocks per
+ * launch (>= 1) for later launches; 0 restores each default.  A step whose
+ * forced width exceeds opt2s_testing_max_block_threads() for its kernel
+ * returns OPT2S_ERR_INVALID_ARG without launching. */
+int opt2s_testing_set_launch(int block_threads, int max_blocks);
+
+/* Widest block (threads) the step kernel for (algo, skip_zeros) can launch
+ * with on the current device (its register use limits it), or a negative
+ * opt2s_status. */
+int opt2s_testing_max_block_threads(int32_t algo, int32_t skip_zeros);
+
+/* The library's default chunk length in elements. */
+int64_t opt2s_testing_default_chunk_elems(void);
+
+/* Number of kernels this library has launched in this process. */
+int64_t opt2s_testing_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OPT2S_TESTING_H */

@@ -1,0 +1,288 @@
+"""Host-side tests of the C ABI (no GPU needed).
+
+They check that libopt2s.so loads, that it exports exactly the entry points
+include/*.h declares, that the ctypes mirrors have the C layout, and the
+host logic every call runs before touching CUDA: argument validation (every
+record checked before any launch, so an argument error never leaves a partial
+update) and the chunk-table builder (every element covered exactly once).
+Pointers here are fake addresses: nothing is dereferenced on the host.
+"""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+from elementwise_optimizer_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+INCLUDE = os.path.join(ROOT, "include")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from elementwise_optimizer_b200 import _build
+    _build.build()
+    return B.lib()
+
+
+def declared_functions():
+    names = set()
+    for h in ("opt2s.h", "opt2s_testing.h"):
+        src = open(os.path.join(INCLUDE, h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"^[A-Za-z_][\w \t\*]*?\b(opt2s_\w+)\s*\(", src, flags=re.M))
+    return names
+
+
+def test_exports_match_headers(L):
+    decl = declared_functions()
+    assert "opt2s_step" in decl and "opt2s_plan_create" in decl
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], check=True,
+                         capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l and "opt2s_" in l}
+    assert exported == decl, (exported ^ decl)
+    for name in decl:
+        assert getattr(L, name) is not None
+    assert set(B.EXPORTS) == decl
+
+
+def test_struct_layout_matches_c(L):
+    prog = r"""
+    #include <stddef.h>
+    #include <stdio.h>
+    #include "opt2s_testing.h"
+    int main(void) {
+      printf("%zu %zu %zu %zu %zu %zu\n", sizeof(opt2s_tensor), offsetof(opt2s_tensor, numel),
+             offsetof(opt2s_tensor, dtype), sizeof(TensorListDesc), sizeof(Hyper),
+             offsetof(Hyper, skip_zeros));
+      printf("%zu %zu\n", sizeof(opt2s_testing_chunk), offsetof(opt2s_testing_chunk, dtype));
+      return 0;
+    }"""
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "p.c")
+        open(c, "w").write(prog)
+        exe = os.path.join(d, "p")
+        cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+        subprocess.run(["gcc", "-std=c11", "-I", INCLUDE, "-I", cuda_inc, "-o", exe, c], check=True)
+        lines = subprocess.run([exe], check=True, capture_output=True, text=True).stdout.split("\n")
+    a = list(map(int, lines[0].split()))
+    assert a == [ctypes.sizeof(B.opt2s_tensor), B.opt2s_tensor.numel.offset,
+                 B.opt2s_tensor.dtype.offset, ctypes.sizeof(B.TensorListDesc),
+                 ctypes.sizeof(B.Hyper), B.Hyper.skip_zeros.offset]
+    b = list(map(int, lines[1].split()))
+    assert b == [ctypes.sizeof(B.opt2s_testing_chunk), B.opt2s_testing_chunk.dtype.offset]
+
+
+def test_abi_version(L):
+    assert L.opt2s_abi_version() == 1
+
+
+def test_error_strings(L):
+    for code in B.STATUS:
+        s = L.opt2s_error_string(code).decode()
+        assert s and s != "unknown status"
+    assert L.opt2s_error_string(12345).decode() == "unknown status"
+
+
+# --------------------------------------------------------------------------
+# Fake device buffers: disjoint address ranges, 256-byte aligned
+# --------------------------------------------------------------------------
+
+class Arena:
+    def __init__(self, base=1 << 40):
+        self.next = base
+
+    def alloc(self, nbytes, align=256, offset=0):
+        a = (self.next + align - 1) // align * align + offset
+        self.next = a + nbytes + 4096
+        return a
+
+
+def records(sizes, dtypes=None, algo="adam", arena=None):
+    arena = arena or Arena()
+    dtypes = dtypes or ["f32"] * len(sizes)
+    recs = []
+    for n, dt in zip(sizes, dtypes):
+        es = 4 if dt == "f32" else 2
+        s1n = 2 * n if algo == "ademamix" else n
+        recs.append((arena.alloc(n * es), arena.alloc(n * es), arena.alloc(4 * s1n),
+                     arena.alloc(4 * n), n, B.DTYPES[dt]))
+    return recs
+
+
+H = B.make_hyper("adam")
+
+
+def validate(recs, hyper=H, step=1):
+    return B.testing_validate(B.TensorList(recs), hyper, step)
+
+
+def test_valid_collection_passes(L):
+    assert validate(records([1, 7, 4096, 100000], ["f32", "f16", "bf16", "f32"])) == 0
+    assert validate([]) == 0
+
+
+@pytest.mark.parametrize("field,value", [
+    ("algo", 2), ("algo", -1), ("skip_zeros", 2), ("lr", float("nan")),
+    ("lr", float("inf")), ("beta1", 1.0), ("beta1", -0.1), ("beta2", 1.5),
+    ("eps", -1e-8), ("eps", float("inf")), ("weight_decay", float("nan"))])
+def test_bad_hyper_rejected(L, field, value):
+    h = B.make_hyper("adam")
+    setattr(h, field, value)
+    assert validate(records([16]), h) == -1
+
+
+def test_ademamix_hyper_checked_only_for_ademamix(L):
+    h = B.make_hyper("adam", beta3=2.0, alpha=float("nan"))
+    assert validate(records([16]), h) == 0
+    h = B.make_hyper("ademamix", beta3=1.0, alpha=5.0)
+    assert validate(records([16], algo="ademamix"), h) == -1
+    h = B.make_hyper("ademamix", beta3=0.999, alpha=float("inf"))
+    assert validate(records([16], algo="ademamix"), h) == -1
+
+
+@pytest.mark.parametrize("step", [0, -1, -(2 ** 31)])
+def test_step_below_one_rejected(L, step):
+    assert validate(records([16]), step=step) == -1
+
+
+def test_bad_records_rejected(L):
+    good = records([64])
+    p, g, s1, s2, n, dt = good[0]
+    assert validate([(p, g, s1, s2, -1, dt)]) == -1            # negative numel
+    assert validate([(p, g, s1, s2, n, 7)]) == -1              # bad dtype
+    assert validate([(0, g, s1, s2, n, dt)]) == -1             # null param
+    assert validate([(p, 0, s1, s2, n, dt)]) == -1             # null grad
+    assert validate([(p, g, 0, s2, n, dt)]) == -1              # null state1
+    assert validate([(p, g, s1, 0, n, dt)]) == -1              # null state2
+    assert validate([(p + 2, g, s1, s2, n, dt)]) == -1         # fp32 param not 4-aligned
+    assert validate([(p, g, s1 + 1, s2, n, dt)]) == -1         # state not 4-aligned
+    assert validate([(0, 0, 0, 0, 0, dt)]) == 0                # empty record: skipped
+    tl = B.TensorList(good)
+    tl._arr[0].reserved = 1
+    assert B.testing_validate(tl, H, 1) == -1
+    null_desc = B.TensorListDesc(None, 3)
+    assert B.lib().opt2s_testing_validate(ctypes.byref(null_desc), ctypes.byref(H), 1) == -1
+    neg = B.TensorListDesc(None, -1)
+    assert B.lib().opt2s_testing_validate(ctypes.byref(neg), ctypes.byref(H), 1) == -1
+
+
+def test_half_storage_needs_only_2_byte_alignment(L):
+    p, g, s1, s2, n, _ = records([64], ["f16"])[0]
+    assert validate([(p + 2, g + 6, s1 + 4, s2 + 12, n, B.DTYPES["f16"])]) == 0
+    assert validate([(p + 1, g, s1, s2, n, B.DTYPES["f16"])]) == -1
+
+
+def test_aliasing_rejected(L):
+    p, g, s1, s2, n, dt = records([1024])[0]
+    assert validate([(p, p, s1, s2, n, dt)]) == -2                     # grad is param
+    assert validate([(p, g, s1, s1, n, dt)]) == -2                     # m is v
+    assert validate([(p, g, s1, s1 + 4 * 1023, n, dt)]) == -2          # partial overlap
+    assert validate([(p, g, p + 4 * 512, s2, n, dt)]) == -2            # state inside param
+    a, b = records([100, 100])
+    assert validate([a, (b[0], b[1], a[2], b[3], 100, dt)]) == -2      # states shared across tensors
+    # two tensors reading the same gradient is fine (it is never written)
+    assert validate([a, (b[0], a[1], b[2], b[3], 100, dt)]) == 0
+
+
+def test_ademamix_state1_is_twice_numel(L):
+    arena = Arena()
+    n = 256
+    p, g = arena.alloc(4 * n), arena.alloc(4 * n)
+    s1 = arena.alloc(4 * n, align=4096)      # room for n floats only ...
+    s2 = s1 + 4 * n                          # ... v starts right after m
+    adam_ok = validate([(p, g, s1, s2, n, 0)], B.make_hyper("adam"))
+    ademamix = validate([(p, g, s1, s2, n, 0)], B.make_hyper("ademamix", beta3=0.999, alpha=5))
+    assert adam_ok == 0 and ademamix == -2   # m2 = state1[n:2n] would overlap v
+
+
+# --------------------------------------------------------------------------
+# Chunk-table builder
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("chunk", [0, 8, 64, 4096, 8192])
+def test_chunks_cover_every_element_once(L, chunk):
+    sizes = [1, 2, 31, 32, 33, 255, 256, 257, 1023, 1024, 1025, 4095, 4096, 4097,
+             8191, 8192, 8193, 0, 100003]
+    dts = [("f32", "f16", "bf16")[i % 3] for i in range(len(sizes))]
+    tl = B.TensorList(records(sizes, dts))
+    chunks = B.testing_build_chunks(tl, "adam", chunk)
+    ce = chunk or B.lib().opt2s_testing_default_chunk_elems()
+    cover = {i: [] for i in range(len(sizes))}
+    for t, s, n, dt in chunks:
+        assert 1 <= n <= ce and s % ce == 0
+        assert dt == B.DTYPES[dts[t]]
+        cover[t].append((s, n))
+    for i, n in enumerate(sizes):
+        segs = cover[i]
+        assert sum(x[1] for x in segs) == n
+        pos = 0
+        for s, k in segs:                     # contiguous, in order, no overlap
+            assert s == pos
+            pos += k
+    # launch order follows descriptor order
+    assert [c[0] for c in chunks] == sorted(c[0] for c in chunks)
+
+
+def test_chunk_count_for_large_tensor(L):
+    tl = B.TensorList(records([268_435_456]))
+    ce = B.lib().opt2s_testing_default_chunk_elems()
+    assert len(B.testing_build_chunks(tl, "adam")) == 268_435_456 // ce
+
+
+def test_build_chunks_validates_first(L):
+    p, g, s1, s2, n, dt = records([64])[0]
+    with pytest.raises(B.Opt2sError) as e:
+        B.testing_build_chunks(B.TensorList([(p, p, s1, s2, n, dt)]), "adam")
+    assert e.value.status == -2
+
+
+def test_testing_knobs_validate(L):
+    with pytest.raises(B.Opt2sError):
+        B.testing_set_launch(33, 0)
+    with pytest.raises(B.Opt2sError):
+        B.testing_set_launch(2048, 0)
+    B.testing_set_launch(0, 0)
+    prev = B.testing_set_chunk_elems(0)
+    assert B.testing_set_chunk_elems(prev) == 0
+
+
+# --------------------------------------------------------------------------
+# The step entry point without a GPU: argument errors come first, no crash
+# --------------------------------------------------------------------------
+
+def _cuda_available():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+@pytest.mark.skipif(_cuda_available(), reason="checks the no-device path")
+def test_step_without_device(L):
+    tl = B.TensorList(records([64]))
+    with pytest.raises(B.Opt2sError) as e:
+        B.opt2s_step(tl, H, 1, stream=0)
+    assert e.value.status == -4                       # CUDA: no device
+    p, g, s1, s2, n, dt = records([64])[0]
+    with pytest.raises(B.Opt2sError) as e:            # argument errors still first
+        B.opt2s_step(B.TensorList([(p, p, s1, s2, n, dt)]), H, 1, stream=0)
+    assert e.value.status == -2
+    with pytest.raises(B.Opt2sError) as e:
+        B.opt2s_step(tl, H, 0, stream=0)
+    assert e.value.status == -1
+    B.opt2s_step(B.TensorList([]), H, 1, stream=0)    # empty collection: no-op
+    B.opt2s_step(B.TensorList([(0, 0, 0, 0, 0, 0)]), H, 1, stream=0)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    code = ("import elementwise_optimizer_b200.binding as b; b.LIB_PATH='/nonexistent/x.so'\n"
+            "try:\n  b.lib()\nexcept RuntimeError as e:\n  print('RAISED', e)\n")
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True,
+                         text=True, check=True).stdout
+    assert out.startswith("RAISED") and "no CPU fallback" in out
