@@ -184,8 +184,8 @@ def make_device_workload(w, device, n_grad_buffers):
 
 
 def small_collection_us(device, reps=200):
-    """µs per step of the 2,000-tensor collection (one launch per step),
-    L2 flushed before every step by writing a 256 MB buffer."""
+    """µs per step of the 2,000-tensor collection (one launch per step), L2
+    flushed before every step by writing and then reading a 256 MB buffer."""
     import torch
     from elementwise_optimizer_b200 import binding as B
     w = workload("small_collection")
@@ -198,7 +198,10 @@ def small_collection_us(device, reps=200):
     times = []
     launches0 = B.launch_count()
     for t in range(6, 6 + reps):
+        # write a buffer larger than L2, then read it back so the dirty lines
+        # drain before the timed launch rather than during it
         flush.fill_(float(t))
+        flush.sum()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -211,7 +214,7 @@ def small_collection_us(device, reps=200):
     q = lambda f: us[min(len(us) - 1, int(f * len(us)))]
     return {"workload": w.name, "tensors": len(w.sizes), "numel": w.numel,
             "us_per_step_median": q(0.5), "us_per_step_p10": q(0.1), "us_per_step_p90": q(0.9),
-            "launches_per_step": launches / reps, "l2": "flushed (256 MB write) before each step"}
+            "launches_per_step": launches / reps, "l2": "flushed before each step (256 MB written, then read)"}
 
 
 def e2e_measure(w, d, device, steps):
