@@ -71,6 +71,9 @@ EXPORTS = {
                                        ctypes.c_void_p]),
     "opt2s_plan_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "opt2s_plan_num_chunks": (ctypes.c_int64, [ctypes.c_void_p]),
+    "opt2s_step_noalloc": (ctypes.c_int, [ctypes.POINTER(TensorListDesc), ctypes.POINTER(Hyper),
+                                          ctypes.c_int, ctypes.c_void_p]),
+    "opt2s_noalloc_max_chunks": (ctypes.c_int64, []),
     "opt2s_release_cache": (ctypes.c_int, []),
     "opt2s_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "opt2s_last_cuda_error": (ctypes.c_int, []),
@@ -194,6 +197,21 @@ def opt2s_step(tl: TensorList, hyper: Hyper, step: int, stream=None) -> None:
     stream unless ``stream`` is given)."""
     check(lib().opt2s_step(ctypes.byref(tl.desc), ctypes.byref(hyper), int(step),
                            _stream_handle(stream)), "opt2s_step")
+
+
+def opt2s_step_noalloc(tl: TensorList, hyper: Hyper, step: int, stream=None) -> None:
+    """opt2s_step for callers that cannot let the library allocate device
+    memory (their runtime owns every byte through its own pool, or their
+    footprint is fixed at start-up): the launch table lives in a fixed
+    3 MiB device array instead of memory from cudaMalloc.  Collections that
+    need more than opt2s_noalloc_max_chunks() chunk records are rejected;
+    calls that overlap on the GPU race on the shared table."""
+    check(lib().opt2s_step_noalloc(ctypes.byref(tl.desc), ctypes.byref(hyper), int(step),
+                                   _stream_handle(stream)), "opt2s_step_noalloc")
+
+
+def noalloc_max_chunks() -> int:
+    return int(lib().opt2s_noalloc_max_chunks())
 
 
 class Plan:

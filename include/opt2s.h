@@ -142,6 +142,35 @@ int opt2s_plan_destroy(opt2s_plan *plan);
 /* Number of chunk records in a plan (the work units of one launch). */
 int64_t opt2s_plan_num_chunks(const opt2s_plan *plan);
 
+/*
+ * opt2s_step without any allocation by the library.  The paper this library
+ * follows has no counterpart to it: it exists for callers that cannot let a
+ * library allocate device memory -- runtimes that own all device memory
+ * through their own pool, deployments whose memory footprint is fixed at
+ * start-up, or code that must avoid the implicit synchronization of
+ * cudaMalloc/cudaFree.  Same arguments, arithmetic and results as opt2s_step.
+ *
+ * It calls no cudaMalloc, cudaFree or allocating library routine and keeps
+ * no plan.  Each call builds the chunk table in a fixed host array and
+ * uploads it (cudaMemcpyAsync on `stream`, from pageable memory, so the call
+ * waits for `stream`'s earlier work) into a fixed device array of
+ * opt2s_noalloc_max_chunks() records (65,536 records = 3 MiB), which every
+ * GPU that loads the library holds until the process exits.  A collection
+ * needing more chunk records (8,192 elements per chunk; at least one per
+ * non-empty tensor) returns OPT2S_ERR_TOO_LARGE before any work.
+ * All calls on a device share that array and leave the last call's table in
+ * it; every call rewrites what it reads, so nothing must start at zero.  Calls
+ * whose work overlaps on the GPU (unordered streams) race on the array.
+ * The first call on each device looks up the array's device address and
+ * caches it; make that first call before any stream capture begins.
+ * Calls from several host threads are serialized.
+ */
+int opt2s_step_noalloc(const TensorListDesc *desc, const Hyper *hyper, int step,
+                       cudaStream_t stream);
+
+/* Capacity of opt2s_step_noalloc's fixed chunk table, in records. */
+int64_t opt2s_noalloc_max_chunks(void);
+
 /* Frees every cached plan of every device (waits for the devices first). */
 int opt2s_release_cache(void);
 
