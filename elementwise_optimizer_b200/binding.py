@@ -88,6 +88,8 @@ EXPORTS = {
     "opt2s_testing_set_launch": (ctypes.c_int, [ctypes.c_int, ctypes.c_int]),
     "opt2s_testing_default_chunk_elems": (ctypes.c_int64, []),
     "opt2s_testing_launch_count": (ctypes.c_int64, []),
+    "opt2s_testing_check_division": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int32,
+                                                    ctypes.POINTER(ctypes.c_int64)]),
     "opt2s_testing_max_block_threads": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32]),
 }
 
@@ -275,6 +277,13 @@ def testing_max_block_threads(algo: str, skip_zeros: bool) -> int:
     if r < 0:
         check(r, "testing_max_block_threads")
     return r
+
+
+def testing_check_division(seed: int, n: int, mode: int) -> int:
+    """Mismatches between the kernel's constant division and __fdiv_rn."""
+    out = ctypes.c_int64()
+    check(lib().opt2s_testing_check_division(seed, n, mode, ctypes.byref(out)), "check_division")
+    return int(out.value)
 
 
 def launch_count() -> int:

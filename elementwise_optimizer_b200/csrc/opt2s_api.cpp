@@ -454,4 +454,21 @@ OPT2S_API int opt2s_testing_max_block_threads(int32_t algo, int32_t skip_zeros)
     return widest;
 }
 
+OPT2S_API int opt2s_testing_check_division(uint64_t seed, int64_t n, int32_t mode,
+                                           int64_t* mismatches)
+{
+    if (!mismatches || n < 0 || (mode != 0 && mode != 1)) return OPT2S_ERR_INVALID_ARG;
+    unsigned long long* d_count = nullptr;
+    cudaError_t e = cudaMalloc(&d_count, sizeof(*d_count));
+    if (e != cudaSuccess) return cuda_fail(e);
+    unsigned long long h = 0;
+    e = cudaMemset(d_count, 0, sizeof(*d_count));
+    if (e == cudaSuccess) e = opt2s::check_division(seed, n, mode, d_count, 0);
+    if (e == cudaSuccess) e = cudaMemcpy(&h, d_count, sizeof(h), cudaMemcpyDeviceToHost);
+    cudaFree(d_count);
+    if (e != cudaSuccess) return cuda_fail(e);
+    *mismatches = static_cast<int64_t>(h);
+    return OPT2S_OK;
+}
+
 OPT2S_API int64_t opt2s_testing_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -34,6 +34,10 @@ struct StepScalars {
     float eps;
     float bc1, bc2;
     float decay;
+    // RN64(1/bc1), RN64(1/bc2): filled in by launch_step from bc1/bc2 (both
+    // in (0, 1]); the kernel divides by bc1, bc2 exactly through them (see
+    // div_by_constant in opt2s_kernel.cu)
+    double inv_bc1, inv_bc2;
 };
 
 constexpr int kDefaultBlockThreads = 256;
@@ -50,6 +54,12 @@ cudaError_t launch_step(const ChunkRec* d_chunks, int64_t nchunks, int algo,
 // Widest block (threads, a multiple of 32) the step kernel for (algo,
 // skip_zeros) can be launched with: its registers per thread limit it.
 cudaError_t max_block_threads(int algo, int skip_zeros, int* out);
+
+// Validation scaffolding: counts into *d_count (device memory) the operands
+// among n seeded random ones for which the kernel's constant division differs
+// from __fdiv_rn (mode 0: any x; mode 1: x/d near a rounding boundary).
+cudaError_t check_division(uint64_t seed, int64_t n, int mode, unsigned long long* d_count,
+                           cudaStream_t stream);
 
 // Number of blocks a launch of `nchunks` chunks uses on the current device.
 cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros,

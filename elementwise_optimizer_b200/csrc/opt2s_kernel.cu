@@ -16,8 +16,10 @@
 // Ba 2015, Algorithm 1), decoupled weight decay (Loshchilov & Hutter 2019,
 // Algorithm 2) and AdEMAMix (Pagliardini et al. 2024, Algorithm 1)
 // definitions.  Every operation is an explicit round-to-nearest intrinsic
-// (__fmul_rn / __fadd_rn / __fdiv_rn / __fsqrt_rn), which the compiler may not
-// contract into FMA, so the result of an element never depends on which code
+// (__fmul_rn / __fadd_rn / __fdiv_rn / __fsqrt_rn) or the exact constant
+// division below, none of which the compiler may contract into FMA, so the
+// result of an element equals the plain IEEE evaluation of the documented
+// order and never depends on which code
 // path (vector body, scalar head/tail), chunk, warp or block computed it: the
 // issue's "Correctness oracle" section requires that launch geometry must not
 // change optimizer arithmetic.
@@ -32,8 +34,36 @@ namespace opt2s {
 namespace {
 
 // ---------------------------------------------------------------------------
+// Exact division by a per-launch constant.
+//
+// For every binary32 x and every binary32 d with 0 < |d| <= 1 (the bias
+// corrections bc1, bc2 lie in (0, 1]), with r = RN64(1/d) the correctly
+// rounded binary64 reciprocal computed once per launch on the host:
+//            RN32( RN64(x * r) ) == RN32(x / d).
+// Why: RN64(x*r) = (x/d)(1+e) with |e| <= 2^-52 + 2^-106, so it suffices that
+// x/d is never within 2^-49 (relative) of a binary32 rounding boundary
+// unless it is a binary32 number itself (then |e| < half an ulp keeps it).
+// A boundary is M = Mi*2^k with Mi odd; x - d*M is a multiple of the smaller
+// of the units of x's last bit and of d*M's last bit, and d*M spans fewer
+// than 2^49 of the latter, so if x != d*M then |x/d - M| >= 2^-49 |M|.
+// x == d*M cannot happen: for normal-range boundaries Mi has 25 significant
+// bits while x has 24, and a subnormal-range boundary (an odd multiple of
+// 2^-150) times |d| <= 1 is never a multiple of 2^-149 as every binary32 x
+// is.  binary64 neither overflows nor underflows here, and 0, +-Inf and NaN
+// pass through the product unchanged.  (The exclusion argument used in the
+// analysis of double rounding; see Muller et al., Handbook of Floating-Point
+// Arithmetic, 2nd ed., ch. 4.)  A GPU test checks it against __fdiv_rn on
+// random operands of every class.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float div_by_constant(float x, double r)
+{
+    return __double2float_rn(__dmul_rn(static_cast<double>(x), r));
+}
+
+// ---------------------------------------------------------------------------
 // The per-element update.  With SKIP, an element whose gradient compares equal
-// to zero (+0 or -0) is left untouched (no decay either).
+// to zero (+0 or -0) is left untouched (no decay either).  m/bc1 and v/bc2 use
+// the exact constant division above; num/den is an IEEE division.
 // ---------------------------------------------------------------------------
 template <int ALGO, bool SKIP>
 __device__ __forceinline__ void update(float g, float& p, float& m, float& v,
@@ -43,12 +73,12 @@ __device__ __forceinline__ void update(float g, float& p, float& m, float& v,
     m = __fadd_rn(__fmul_rn(s.beta1, m), __fmul_rn(s.one_minus_beta1, g));
     v = __fadd_rn(__fmul_rn(s.beta2, v),
                   __fmul_rn(__fmul_rn(s.one_minus_beta2, g), g));
-    float num = __fdiv_rn(m, s.bc1);
+    float num = div_by_constant(m, s.inv_bc1);
     if (ALGO == kAdEMAMix) {
         m2 = __fadd_rn(__fmul_rn(s.beta3, m2), __fmul_rn(s.one_minus_beta3, g));
         num = __fadd_rn(num, __fmul_rn(s.alpha, m2));
     }
-    const float den = __fadd_rn(__fsqrt_rn(__fdiv_rn(v, s.bc2)), s.eps);
+    const float den = __fadd_rn(__fsqrt_rn(div_by_constant(v, s.inv_bc2)), s.eps);
     p = __fsub_rn(__fmul_rn(p, s.decay), __fmul_rn(s.lr, __fdiv_rn(num, den)));
 }
 
@@ -302,7 +332,62 @@ cudaError_t device_info(int dev, DeviceInfo** out)
     return cudaSuccess;
 }
 
+// ---------------------------------------------------------------------------
+// Validation scaffolding: div_by_constant against __fdiv_rn on random operands.
+// Operands come from the SplitMix64 output function (Steele, Lea & Flood,
+// "Fast splittable pseudorandom number generators", OOPSLA 2014) applied to a
+// counter.  mode 0: x is a random bit pattern (every class: zeros, subnormals,
+// normals, infinities, NaNs).  mode 1: x = RN32(d * B) for B a random rounding
+// boundary, so x/d lies close to a boundary (the hard cases).  d is a random
+// binary32 in (0, 1] (subnormals included; d = 1 about once in 1,024 draws).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t splitmix64(uint64_t z)
+{
+    z += 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+__global__ void check_division_kernel(uint64_t seed, int64_t n, int mode,
+                                      unsigned long long* mismatches)
+{
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const uint64_t h1 = splitmix64(seed + 3 * static_cast<uint64_t>(i));
+        const uint64_t h2 = splitmix64(seed + 3 * static_cast<uint64_t>(i) + 1);
+        uint32_t dbits = (static_cast<uint32_t>(h2 >> 32) % 127u) << 23 |
+                         static_cast<uint32_t>(h2 & 0x7FFFFFu);
+        if (dbits == 0) dbits = 1;
+        if ((h2 >> 54) == 0) dbits = 0x3F800000u;          // d = 1
+        const float d = __uint_as_float(dbits);
+        float x;
+        if (mode == 0) {
+            x = __uint_as_float(static_cast<uint32_t>(h1));
+        } else {
+            // a rounding boundary: the midpoint just above a random finite float
+            const uint64_t h3 = splitmix64(seed + 3 * static_cast<uint64_t>(i) + 2);
+            const float f = __uint_as_float(static_cast<uint32_t>(h3) & 0x7F7FFFFFu);
+            const double mid = 0.5 * (static_cast<double>(f) +
+                                      static_cast<double>(__uint_as_float(__float_as_uint(f) + 1)));
+            x = __double2float_rn(__dmul_rn(mid, static_cast<double>(d)));
+            if (h1 & 1) x = -x;
+        }
+        const float a = div_by_constant(x, __drcp_rn(static_cast<double>(d)));
+        const float b = __fdiv_rn(x, d);
+        const bool same = __float_as_uint(a) == __float_as_uint(b) || (isnan(a) && isnan(b));
+        if (!same) atomicAdd(mismatches, 1ull);
+    }
+}
+
 }  // namespace
+
+cudaError_t check_division(uint64_t seed, int64_t n, int mode, unsigned long long* d_count,
+                           cudaStream_t stream)
+{
+    check_division_kernel<<<148 * 8, 256, 0, stream>>>(seed, n, mode, d_count);
+    return cudaGetLastError();
+}
 
 cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros, int block_threads,
                      int max_blocks, int* grid)
@@ -353,6 +438,8 @@ cudaError_t launch_step(const ChunkRec* d_chunks, int64_t nchunks, int algo, int
     if (e != cudaSuccess) return e;
     int n = static_cast<int>(nchunks);
     StepScalars sc = s;
+    sc.inv_bc1 = 1.0 / static_cast<double>(s.bc1);   // correctly rounded (IEEE)
+    sc.inv_bc2 = 1.0 / static_cast<double>(s.bc2);
     void* args[] = {const_cast<ChunkRec**>(&d_chunks), &n, &sc};
     return cudaLaunchKernel(reinterpret_cast<const void*>(pick(algo, skip_zeros)),
                             dim3(grid), dim3(block_threads), args, 0, stream);

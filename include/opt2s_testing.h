@@ -65,6 +65,13 @@ int opt2s_testing_max_block_threads(int32_t algo, int32_t skip_zeros);
 /* The library's default chunk length in elements. */
 int64_t opt2s_testing_default_chunk_elems(void);
 
+/* Runs the step kernel's exact division by a constant in (0, 1] and the IEEE
+ * division __fdiv_rn side by side on `n` seeded random operand pairs on the
+ * current device (mode 0: x of every class; mode 1: x/d next to a binary32
+ * rounding boundary) and writes how many results differ (NaN equals NaN) to
+ * *mismatches.  Synchronous; allocates a counter on the device. */
+int opt2s_testing_check_division(uint64_t seed, int64_t n, int32_t mode, int64_t *mismatches);
+
 /* Number of kernels this library has launched in this process. */
 int64_t opt2s_testing_launch_count(void);
 

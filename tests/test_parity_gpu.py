@@ -105,6 +105,15 @@ def test_boundary_sweep_1000_steps(algo, dtype, skip, wd):
     assert h.max_rel() <= 1e-5
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+def test_constant_division_is_exact(mode):
+    """The kernel divides by bc1, bc2 through a binary64 reciprocal; it must
+    equal IEEE division (__fdiv_rn) for every x and every divisor in (0, 1]:
+    2^32 random pairs of every class (mode 0) and near rounding boundaries
+    (mode 1)."""
+    assert B.testing_check_division(0x0E0A0000 + mode, 1 << 32, mode) == 0
+
+
 # --------------------------------------------------------------------------
 # Bitwise invariance of the launch geometry
 # --------------------------------------------------------------------------
