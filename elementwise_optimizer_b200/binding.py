@@ -55,6 +55,13 @@ class Hyper(ctypes.Structure):
                 ("skip_zeros", ctypes.c_int32)]
 
 
+class opt2s_step_scalars(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_float) for n in (
+        "lr", "beta1", "beta2", "beta3", "one_minus_beta1", "one_minus_beta2",
+        "one_minus_beta3", "alpha", "eps", "bc1", "bc2", "decay")] + [
+        ("inv_bc1", ctypes.c_double), ("inv_bc2", ctypes.c_double)]
+
+
 class opt2s_testing_chunk(ctypes.Structure):
     _fields_ = [("tensor", ctypes.c_int64), ("start", ctypes.c_int64),
                 ("len", ctypes.c_int64), ("dtype", ctypes.c_int32),
@@ -74,6 +81,10 @@ EXPORTS = {
     "opt2s_step_noalloc": (ctypes.c_int, [ctypes.POINTER(TensorListDesc), ctypes.POINTER(Hyper),
                                           ctypes.c_int, ctypes.c_void_p]),
     "opt2s_noalloc_max_chunks": (ctypes.c_int64, []),
+    "opt2s_fill_step_scalars": (ctypes.c_int, [ctypes.POINTER(Hyper), ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_void_p]),
+    "opt2s_plan_step_table": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                             ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
     "opt2s_release_cache": (ctypes.c_int, []),
     "opt2s_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "opt2s_last_cuda_error": (ctypes.c_int, []),
@@ -233,6 +244,13 @@ class Plan:
         check(lib().opt2s_plan_step(self._h, ctypes.byref(hyper), int(step),
                                     _stream_handle(stream)), "opt2s_plan_step")
 
+    def step_table(self, skip_zeros: bool, d_table: int, table_len: int, d_index: int,
+                   stream=None) -> None:
+        """opt2s_plan_step_table: the scalars come from d_table[*d_index]
+        (device pointers), which the call then advances; capturable."""
+        check(lib().opt2s_plan_step_table(self._h, int(bool(skip_zeros)), d_table, int(table_len),
+                                          d_index, _stream_handle(stream)), "opt2s_plan_step_table")
+
     def close(self) -> None:
         if self._h:
             check(lib().opt2s_plan_destroy(self._h), "opt2s_plan_destroy")
@@ -243,6 +261,15 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def fill_step_scalars(hyper: Hyper, first_step: int, count: int) -> bytes:
+    """opt2s_fill_step_scalars: the raw table of `count` steps (64 bytes each),
+    ready to be copied to device memory."""
+    arr = (opt2s_step_scalars * max(count, 1))()
+    check(lib().opt2s_fill_step_scalars(ctypes.byref(hyper), int(first_step), int(count),
+                                        ctypes.cast(arr, ctypes.c_void_p)), "opt2s_fill_step_scalars")
+    return bytes(arr)[:count * ctypes.sizeof(opt2s_step_scalars)]
 
 
 def opt2s_release_cache() -> None:

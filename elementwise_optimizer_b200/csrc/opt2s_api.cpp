@@ -14,6 +14,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <cstddef>
 #include <cstring>
 #include <list>
 #include <mutex>
@@ -363,6 +364,51 @@ OPT2S_API int opt2s_plan_step(const opt2s_plan* plan, const Hyper* hyper, int st
 OPT2S_API int opt2s_plan_destroy(opt2s_plan* plan) { return plan_destroy(plan); }
 
 OPT2S_API int64_t opt2s_plan_num_chunks(const opt2s_plan* plan) { return plan ? plan->nchunks : -1; }
+
+static_assert(sizeof(opt2s_step_scalars) == sizeof(StepScalars), "scalar table layout");
+static_assert(offsetof(opt2s_step_scalars, decay) == offsetof(StepScalars, decay), "scalar table layout");
+static_assert(offsetof(opt2s_step_scalars, inv_bc1) == offsetof(StepScalars, inv_bc1), "scalar table layout");
+static_assert(offsetof(opt2s_step_scalars, inv_bc2) == offsetof(StepScalars, inv_bc2), "scalar table layout");
+
+OPT2S_API int opt2s_fill_step_scalars(const Hyper* hyper, int first_step, int count,
+                                      opt2s_step_scalars* out)
+{
+    if (!out || count < 0) return OPT2S_ERR_INVALID_ARG;
+    if (count > 0 && first_step > INT32_MAX - (count - 1)) return OPT2S_ERR_INVALID_ARG;
+    int st = validate_hyper(hyper, first_step);
+    if (st != OPT2S_OK) return st;
+    for (int k = 0; k < count; ++k) {
+        StepScalars s = make_scalars(hyper, first_step + k);
+        opt2s::fill_reciprocals(&s);
+        std::memcpy(&out[k], &s, sizeof(s));
+    }
+    return OPT2S_OK;
+}
+
+OPT2S_API int opt2s_plan_step_table(const opt2s_plan* plan, int32_t skip_zeros,
+                                    const opt2s_step_scalars* d_table, int32_t table_len,
+                                    int32_t* d_index, cudaStream_t stream)
+{
+    if (!plan || !d_table || !d_index || table_len < 1) return OPT2S_ERR_INVALID_ARG;
+    if (skip_zeros != 0 && skip_zeros != 1) return OPT2S_ERR_INVALID_ARG;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev != plan->device) return OPT2S_ERR_DEVICE;
+    const int bt = block_threads_now();
+    if (bt != opt2s::kDefaultBlockThreads) {
+        int widest = 0;
+        e = opt2s::max_block_threads(plan->algo, skip_zeros, &widest);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (bt > widest) return OPT2S_ERR_INVALID_ARG;
+    }
+    e = opt2s::launch_step_table(plan->d_chunks, plan->nchunks, plan->algo, skip_zeros,
+                                 reinterpret_cast<const StepScalars*>(d_table), d_index, table_len,
+                                 bt, g_max_blocks, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_launches.fetch_add(plan->nchunks > 0 ? 2 : 1, std::memory_order_relaxed);
+    return OPT2S_OK;
+}
 
 OPT2S_API int opt2s_release_cache(void)
 {

@@ -51,6 +51,17 @@ cudaError_t launch_step(const ChunkRec* d_chunks, int64_t nchunks, int algo,
                         int block_threads, int max_blocks,
                         cudaStream_t stream);
 
+// Sets s->inv_bc1, s->inv_bc2 = RN64(1/bc1), RN64(1/bc2) (host).
+void fill_reciprocals(StepScalars* s);
+
+// Launches one step whose scalars are d_table[*d_index] (device memory),
+// followed by a one-thread launch that advances *d_index (to -1 after the
+// last entry).  Both launches may be captured in a CUDA graph.
+cudaError_t launch_step_table(const ChunkRec* d_chunks, int64_t nchunks, int algo,
+                              int skip_zeros, const StepScalars* d_table, int* d_index,
+                              int table_len, int block_threads, int max_blocks,
+                              cudaStream_t stream);
+
 // Widest block (threads, a multiple of 32) the step kernel for (algo,
 // skip_zeros) can be launched with: its registers per thread limit it.
 cudaError_t max_block_threads(int algo, int skip_zeros, int* out);

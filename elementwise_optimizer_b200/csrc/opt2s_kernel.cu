@@ -283,8 +283,10 @@ __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& 
     }
 }
 
+// The whole step: warp w takes chunks w, w + W, w + 2W, ... of the table.
 template <int ALGO, bool SKIP>
-__global__ void step_kernel(const ChunkRec* __restrict__ chunks, int nchunks, StepScalars s)
+__device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, int nchunks,
+                                          const StepScalars& s)
 {
     const int lane = threadIdx.x & 31;
     const int warps_per_block = blockDim.x >> 5;
@@ -300,12 +302,48 @@ __global__ void step_kernel(const ChunkRec* __restrict__ chunks, int nchunks, St
     }
 }
 
+// Per-step scalars passed by value (the host computes them for each call).
+template <int ALGO, bool SKIP>
+__global__ void step_kernel(const ChunkRec* __restrict__ chunks, int nchunks, StepScalars s)
+{
+    step_body<ALGO, SKIP>(chunks, nchunks, s);
+}
+
+// Per-step scalars read from a device table at a device-resident index, so a
+// captured CUDA graph performs the next step at every replay.  An index
+// outside [0, table_len) performs no update.
+template <int ALGO, bool SKIP>
+__global__ void step_kernel_table(const ChunkRec* __restrict__ chunks, int nchunks,
+                                  const StepScalars* __restrict__ table, const int* index,
+                                  int table_len)
+{
+    const int idx = *index;
+    if (idx < 0 || idx >= table_len) return;
+    const StepScalars s = table[idx];
+    step_body<ALGO, SKIP>(chunks, nchunks, s);
+}
+
+// Moves the index to the next table entry; -1 once the table is used up.
+__global__ void advance_index_kernel(int* index, int table_len)
+{
+    const int idx = *index;
+    *index = (idx >= 0 && idx + 1 < table_len) ? idx + 1 : -1;
+}
+
 using KernelFn = void (*)(const ChunkRec*, int, StepScalars);
+using TableKernelFn = void (*)(const ChunkRec*, int, const StepScalars*, const int*, int);
 
 KernelFn pick(int algo, int skip)
 {
     if (algo == kAdEMAMix) return skip ? step_kernel<kAdEMAMix, true> : step_kernel<kAdEMAMix, false>;
     return skip ? step_kernel<kAdam, true> : step_kernel<kAdam, false>;
+}
+
+TableKernelFn pick_table(int algo, int skip)
+{
+    if (algo == kAdEMAMix)
+        return skip ? step_kernel_table<kAdEMAMix, true> : step_kernel_table<kAdEMAMix, false>;
+    return skip ? step_kernel_table<kAdam, true> : step_kernel_table<kAdam, false>;
 }
 
 // Resident blocks per SM and SM count, cached per device (and kernel / block
@@ -438,11 +476,38 @@ cudaError_t launch_step(const ChunkRec* d_chunks, int64_t nchunks, int algo, int
     if (e != cudaSuccess) return e;
     int n = static_cast<int>(nchunks);
     StepScalars sc = s;
-    sc.inv_bc1 = 1.0 / static_cast<double>(s.bc1);   // correctly rounded (IEEE)
-    sc.inv_bc2 = 1.0 / static_cast<double>(s.bc2);
+    fill_reciprocals(&sc);   // correctly rounded binary64 reciprocals (IEEE)
     void* args[] = {const_cast<ChunkRec**>(&d_chunks), &n, &sc};
     return cudaLaunchKernel(reinterpret_cast<const void*>(pick(algo, skip_zeros)),
                             dim3(grid), dim3(block_threads), args, 0, stream);
+}
+
+void fill_reciprocals(StepScalars* s)
+{
+    s->inv_bc1 = 1.0 / static_cast<double>(s->bc1);
+    s->inv_bc2 = 1.0 / static_cast<double>(s->bc2);
+}
+
+cudaError_t launch_step_table(const ChunkRec* d_chunks, int64_t nchunks, int algo, int skip_zeros,
+                              const StepScalars* d_table, int* d_index, int table_len,
+                              int block_threads, int max_blocks, cudaStream_t stream)
+{
+    if (nchunks > 0) {
+        int grid = 0;
+        cudaError_t e = grid_for(nchunks, algo, skip_zeros, block_threads, max_blocks, &grid);
+        if (e != cudaSuccess) return e;
+        int n = static_cast<int>(nchunks);
+        const int* idx = d_index;
+        int len = table_len;
+        void* args[] = {const_cast<ChunkRec**>(&d_chunks), &n, const_cast<StepScalars**>(&d_table),
+                        const_cast<int**>(&idx), &len};
+        e = cudaLaunchKernel(reinterpret_cast<const void*>(pick_table(algo, skip_zeros)),
+                             dim3(grid), dim3(block_threads), args, 0, stream);
+        if (e != cudaSuccess) return e;
+    }
+    void* args2[] = {&d_index, &table_len};
+    return cudaLaunchKernel(reinterpret_cast<const void*>(advance_index_kernel), dim3(1), dim3(1),
+                            args2, 0, stream);
 }
 
 }  // namespace opt2s

@@ -1,0 +1,151 @@
+"""torch.optim-style front end over the C ABI.
+
+``TwoStateOptimizer`` keeps, for every parameter, the fp32 state of the
+32-bit two-state update (state1 = m, or [m1 | m2] for AdEMAMix; state2 = v)
+and steps each parameter group with ONE launch of the library's kernel,
+whatever the number, sizes and dtypes (fp32/fp16/bf16) of its tensors.  The
+classes mirror the optimizer families of the bitsandbytes issue "Investigate
+a 256-thread SM103 path for small 32-bit optimizer tensors" (section "B300
+benchmark and acceptance": AdamW32bit and AdEMAMix32bit).
+
+capturable=True routes every step through opt2s_plan_step_table: the per-step
+scalars live in a device table and the step index in device memory, so
+``step()`` may be captured in a CUDA graph and each replay performs the next
+step.  Make one eager ``step()`` before capturing (it builds the launch plan),
+and call ``refill_step_table()`` between replays at least once every
+``table_len`` steps (``steps_left()`` tells how many remain).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+
+class TwoStateOptimizer(torch.optim.Optimizer):
+    def __init__(self, params, algo: str = "adamw", lr: float = 1e-3,
+                 betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 0.0,
+                 beta3: float = 0.9999, alpha: float = 5.0, skip_zeros: bool = False,
+                 capturable: bool = False, table_len: int = 1024):
+        if algo not in B.ALGOS:
+            raise ValueError(f"algo must be one of {sorted(B.ALGOS)}")
+        defaults = dict(lr=lr, betas=tuple(betas), eps=eps, weight_decay=weight_decay,
+                        beta3=beta3, alpha=alpha, skip_zeros=skip_zeros)
+        self.algo = "ademamix" if algo == "ademamix" else "adam"
+        self.capturable = capturable
+        self.table_len = int(table_len)
+        super().__init__(params, defaults)
+        self._group_cache = {}
+
+    # ---- per-group launch data ------------------------------------------
+    def _hyper(self, group):
+        b1, b2 = group["betas"]
+        return B.make_hyper(self.algo, lr=group["lr"], beta1=b1, beta2=b2, eps=group["eps"],
+                            weight_decay=group["weight_decay"], beta3=group["beta3"],
+                            alpha=group["alpha"], skip_zeros=group["skip_zeros"])
+
+    def _state_of(self, p):
+        st = self.state[p]
+        if "state1" not in st:
+            n = p.numel()
+            st["state1"] = torch.zeros(2 * n if self.algo == "ademamix" else n,
+                                       dtype=torch.float32, device=p.device)
+            st["state2"] = torch.zeros(n, dtype=torch.float32, device=p.device)
+            st["step"] = 0
+        return st
+
+    def _launch_data(self, gi, group):
+        ps = [p for p in group["params"] if p.grad is not None]
+        for p in ps:
+            if not p.is_cuda or not p.is_contiguous() or not p.grad.is_contiguous():
+                raise ValueError("parameters and gradients must be contiguous CUDA tensors")
+        key = tuple((p.data_ptr(), p.grad.data_ptr(), p.numel()) for p in ps)
+        cached = self._group_cache.get(gi)
+        if cached is not None and cached["key"] == key:
+            return cached
+        states = [self._state_of(p) for p in ps]
+        tl = B.TensorList.from_tensors(ps, [p.grad for p in ps], [s["state1"] for s in states],
+                                       [s["state2"] for s in states])
+        data = {"key": key, "params": ps, "tl": tl, "states": states, "step": 0}
+        if cached is not None:
+            data["step"] = cached["step"]
+        elif states:
+            data["step"] = states[0]["step"]
+        if self.capturable:
+            data["plan"] = B.Plan(tl, self.algo)
+            dev = ps[0].device if ps else torch.device("cuda")
+            data["table"] = torch.empty(self.table_len * 64, dtype=torch.uint8, device=dev)
+            data["index"] = torch.zeros(1, dtype=torch.int32, device=dev)
+            self._refill(data, group)
+        self._group_cache[gi] = data
+        return data
+
+    def _refill(self, data, group):
+        first = data["step"] + 1
+        raw = B.fill_step_scalars(self._hyper(group), first, self.table_len)
+        host = torch.frombuffer(bytearray(raw), dtype=torch.uint8)
+        data["table"].copy_(host)
+        data["index"].zero_()
+        data["table_first"] = first
+
+    # ---- public API --------------------------------------------------------
+    @torch.no_grad()
+    def step(self, closure=None):
+        loss = None
+        if closure is not None:
+            with torch.enable_grad():
+                loss = closure()
+        for gi, group in enumerate(self.param_groups):
+            data = self._launch_data(gi, group)
+            if not data["params"]:
+                continue
+            if self.capturable:
+                data["plan"].step_table(group["skip_zeros"], data["table"].data_ptr(),
+                                        self.table_len, data["index"].data_ptr())
+            else:
+                B.opt2s_step(data["tl"], self._hyper(group), data["step"] + 1)
+            data["step"] += 1
+            for s in data["states"]:
+                s["step"] = data["step"]
+        return loss
+
+    def refill_step_table(self, next_step: int | None = None) -> None:
+        """Capturable mode: rewrite the device tables so that the next step
+        performed (eagerly or by a graph replay) is ``next_step`` (default:
+        one past the steps recorded by eager calls).  Call it only while no
+        replay is in flight."""
+        for gi, group in enumerate(self.param_groups):
+            data = self._group_cache.get(gi)
+            if data is None or "table" not in data:
+                continue
+            if next_step is not None:
+                data["step"] = next_step - 1
+            self._refill(data, group)
+
+    def steps_left(self) -> int:
+        """Capturable mode: table entries left before a refill is needed
+        (reads the device index; synchronizes)."""
+        left = []
+        for data in self._group_cache.values():
+            if "index" in data:
+                i = int(data["index"].item())
+                left.append(0 if i < 0 else self.table_len - i)
+        return min(left) if left else 0
+
+
+class AdamW32bit(TwoStateOptimizer):
+    def __init__(self, params, lr=1e-3, betas=(0.9, 0.999), eps=1e-8, weight_decay=1e-2, **kw):
+        super().__init__(params, "adamw", lr, betas, eps, weight_decay, **kw)
+
+
+class Adam32bit(TwoStateOptimizer):
+    def __init__(self, params, lr=1e-3, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0, **kw):
+        super().__init__(params, "adam", lr, betas, eps, weight_decay, **kw)
+
+
+class AdEMAMix32bit(TwoStateOptimizer):
+    def __init__(self, params, lr=1e-3, betas=(0.9, 0.999, 0.9999), alpha=5.0, eps=1e-8,
+                 weight_decay=1e-2, **kw):
+        b1, b2, b3 = betas
+        super().__init__(params, "ademamix", lr, (b1, b2), eps, weight_decay, beta3=b3,
+                         alpha=alpha, **kw)

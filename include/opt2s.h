@@ -143,6 +143,40 @@ int opt2s_plan_destroy(opt2s_plan *plan);
 int64_t opt2s_plan_num_chunks(const opt2s_plan *plan);
 
 /*
+ * Steps that a captured CUDA graph can replay.
+ *
+ * A captured launch keeps the arguments it was captured with, so a graph of
+ * opt2s_plan_step would repeat one step number.  Here the per-step scalars
+ * come from a DEVICE table instead: opt2s_fill_step_scalars computes, on the
+ * host and exactly as opt2s_step does, the scalars of steps first_step ..
+ * first_step+count-1; the caller uploads them to device memory.
+ * opt2s_plan_step_table then launches the step with the scalars
+ * d_table[*d_index] (d_index: one int32 in device memory) and a one-thread
+ * kernel that advances *d_index, to -1 after the last entry; an index outside
+ * [0, table_len) performs no update.  Both launches may be captured; each
+ * replay performs the next step.  Results are bitwise equal to opt2s_step.
+ * skip_zeros selects the kernel (0 or 1); the plan fixes the algorithm.
+ * The first call for a plan should come before capture starts (it may query
+ * device attributes).  Graph capture of this entry point is what the
+ * bitsandbytes issue "Investigate a 256-thread SM103 path for small 32-bit
+ * optimizer tensors" asks of its launch path (section "Scope": safe for CUDA
+ * graph capture; section "B300 benchmark and acceptance": a graph-compatible
+ * direct-call collection).
+ */
+typedef struct {
+    float lr, beta1, beta2, beta3;
+    float one_minus_beta1, one_minus_beta2, one_minus_beta3;
+    float alpha, eps, bc1, bc2, decay;
+    double inv_bc1, inv_bc2;    /* correctly rounded binary64 1/bc1, 1/bc2 */
+} opt2s_step_scalars;
+
+int opt2s_fill_step_scalars(const Hyper *hyper, int first_step, int count,
+                            opt2s_step_scalars *out);
+int opt2s_plan_step_table(const opt2s_plan *plan, int32_t skip_zeros,
+                          const opt2s_step_scalars *d_table, int32_t table_len,
+                          int32_t *d_index, cudaStream_t stream);
+
+/*
  * opt2s_step without any allocation by the library.  The paper this library
  * follows has no counterpart to it: it exists for callers that cannot let a
  * library allocate device memory -- runtimes that own all device memory

@@ -60,6 +60,8 @@ def test_struct_layout_matches_c(L):
              offsetof(opt2s_tensor, dtype), sizeof(TensorListDesc), sizeof(Hyper),
              offsetof(Hyper, skip_zeros));
       printf("%zu %zu\n", sizeof(opt2s_testing_chunk), offsetof(opt2s_testing_chunk, dtype));
+      printf("%zu %zu %zu\n", sizeof(opt2s_step_scalars), offsetof(opt2s_step_scalars, decay),
+             offsetof(opt2s_step_scalars, inv_bc2));
       return 0;
     }"""
     with tempfile.TemporaryDirectory() as d:
@@ -75,6 +77,9 @@ def test_struct_layout_matches_c(L):
                  ctypes.sizeof(B.Hyper), B.Hyper.skip_zeros.offset]
     b = list(map(int, lines[1].split()))
     assert b == [ctypes.sizeof(B.opt2s_testing_chunk), B.opt2s_testing_chunk.dtype.offset]
+    c = list(map(int, lines[2].split()))
+    assert c == [ctypes.sizeof(B.opt2s_step_scalars), B.opt2s_step_scalars.decay.offset,
+                 B.opt2s_step_scalars.inv_bc2.offset]
 
 
 def test_abi_version(L):
@@ -286,3 +291,41 @@ def test_missing_library_fails_loudly(tmp_path):
     out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True,
                          text=True, check=True).stdout
     assert out.startswith("RAISED") and "no CPU fallback" in out
+
+
+# --------------------------------------------------------------------------
+# Per-step scalar tables (host only)
+# --------------------------------------------------------------------------
+
+def test_step_scalar_table_matches_the_definitions(L, oracle_mod):
+    """The table a captured graph reads holds the same per-step scalars the
+    oracle computes: bc = 1 - beta^t and decay = 1 - lr*wd in double rounded
+    once, 1 - beta in fp32, and the binary64 reciprocals of bc1, bc2."""
+    import numpy as np
+    h = B.make_hyper("ademamix", lr=3e-3, beta1=0.9, beta2=0.999, eps=1e-8,
+                     weight_decay=0.1, beta3=0.9999, alpha=5.0)
+    raw = B.fill_step_scalars(h, 7, 20)
+    arr = (B.opt2s_step_scalars * 20).from_buffer_copy(raw)
+    f32 = np.float32
+    for k, s in enumerate(arr):
+        t = 7 + k
+        assert s.bc1 == oracle_mod.bias_correction(0.9, t)
+        assert s.bc2 == oracle_mod.bias_correction(0.999, t)
+        assert s.decay == oracle_mod.decay_factor(3e-3, 0.1)
+        assert s.one_minus_beta1 == f32(1) - f32(0.9)
+        assert s.one_minus_beta3 == f32(1) - f32(0.9999)
+        assert s.inv_bc1 == 1.0 / float(f32(s.bc1)) and s.inv_bc2 == 1.0 / float(f32(s.bc2))
+        assert (s.lr, s.alpha) == (f32(3e-3), f32(5.0))
+
+
+def test_step_scalar_table_rejects_bad_arguments(L):
+    h = B.make_hyper("adam")
+    out = (B.opt2s_step_scalars * 2)()
+    p = ctypes.cast(out, ctypes.c_void_p)
+    assert L.opt2s_fill_step_scalars(ctypes.byref(h), 0, 2, p) == -1        # step 0
+    assert L.opt2s_fill_step_scalars(ctypes.byref(h), 1, -1, p) == -1       # negative count
+    assert L.opt2s_fill_step_scalars(ctypes.byref(h), 2 ** 31 - 1, 2, p) == -1   # step overflow
+    assert L.opt2s_fill_step_scalars(ctypes.byref(h), 1, 2, None) == -1
+    h.beta1 = 1.0
+    assert L.opt2s_fill_step_scalars(ctypes.byref(h), 1, 2, p) == -1
+    assert L.opt2s_plan_step_table(None, 0, None, 1, None, None) == -1
