@@ -99,6 +99,8 @@ EXPORTS = {
     "opt2s_testing_set_launch": (ctypes.c_int, [ctypes.c_int, ctypes.c_int]),
     "opt2s_testing_default_chunk_elems": (ctypes.c_int64, []),
     "opt2s_testing_launch_count": (ctypes.c_int64, []),
+    "opt2s_testing_choose_chunk_elems": (ctypes.c_int64, [ctypes.POINTER(TensorListDesc),
+                                                          ctypes.c_int64]),
     "opt2s_testing_check_division": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int32,
                                                     ctypes.POINTER(ctypes.c_int64)]),
     "opt2s_testing_max_block_threads": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32]),
@@ -311,6 +313,10 @@ def testing_check_division(seed: int, n: int, mode: int) -> int:
     out = ctypes.c_int64()
     check(lib().opt2s_testing_check_division(seed, n, mode, ctypes.byref(out)), "check_division")
     return int(out.value)
+
+
+def testing_choose_chunk_elems(tl: TensorList, resident_warps: int) -> int:
+    return int(lib().opt2s_testing_choose_chunk_elems(ctypes.byref(tl.desc), int(resident_warps)))
 
 
 def launch_count() -> int:

@@ -53,8 +53,38 @@ int cuda_fail(cudaError_t e)
     return OPT2S_ERR_CUDA;
 }
 
-int64_t chunk_elems_now() { return g_chunk_elems > 0 ? g_chunk_elems : opt2s::kDefaultChunkElems; }
 int block_threads_now() { return g_block_threads > 0 ? g_block_threads : opt2s::kDefaultBlockThreads; }
+
+// Chunk length for a collection: the multiple of 256 elements in
+// [kMinChunkElems, kDefaultChunkElems] that minimizes the modelled time of the
+// slowest warp.  A warp handles ceil(chunks / resident_warps) chunks one after
+// the other; a chunk of c elements costs ceil(c / 256) dependent iterations
+// (256 elements per warp iteration) plus about one more for fetching its
+// record.  Large collections get long chunks (small table, few record
+// fetches); small ones get short chunks so every resident warp has work.
+int64_t choose_chunk_elems(const TensorListDesc* d, int64_t resident_warps)
+{
+    if (resident_warps < 1) return opt2s::kDefaultChunkElems;
+    int64_t best = opt2s::kDefaultChunkElems;
+    double best_cost = -1.0;
+    for (int64_t c = opt2s::kDefaultChunkElems; c >= opt2s::kMinChunkElems; c /= 2) {
+        int64_t chunks = 0;
+        for (int32_t i = 0; i < d->count; ++i) chunks += (d->tensors[i].numel + c - 1) / c;
+        const double waves = static_cast<double>((chunks + resident_warps - 1) / resident_warps);
+        const double cost = waves * static_cast<double>(c / opt2s::kMinChunkElems + 1);
+        if (best_cost < 0.0 || cost < best_cost) { best_cost = cost; best = c; }
+    }
+    return best;
+}
+
+int64_t chunk_elems_for(const TensorListDesc* d, int32_t algo)
+{
+    if (g_chunk_elems > 0) return g_chunk_elems;
+    int64_t warps = 0;
+    if (opt2s::resident_warps(algo, 0, block_threads_now(), &warps) != cudaSuccess)
+        return opt2s::kDefaultChunkElems;
+    return choose_chunk_elems(d, warps);
+}
 
 int elem_bytes(int32_t dtype) { return dtype == OPT2S_F32 ? 4 : 2; }
 
@@ -177,7 +207,7 @@ int plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out)
 {
     int st = validate_desc(desc, algo);
     if (st != OPT2S_OK) return st;
-    const int64_t ce = chunk_elems_now();
+    const int64_t ce = chunk_elems_for(desc, algo);
     if (count_chunks(desc, ce) > INT32_MAX) return OPT2S_ERR_TOO_LARGE;
     std::vector<ChunkRec> table = build_chunk_table(desc, ce);
     int dev = 0;
@@ -309,7 +339,7 @@ OPT2S_API int opt2s_step(const TensorListDesc* desc, const Hyper* hyper, int ste
     if (desc->count == 0) return OPT2S_OK;
 
     int dev = 0;
-    const int64_t ce = chunk_elems_now();
+    const int64_t ce = g_chunk_elems;   // part of the cache key: 0 = chosen per plan
     std::unique_lock<std::mutex> lock(g_cache_mu);
     const opt2s_plan* plan = nullptr;
     {
@@ -515,6 +545,12 @@ OPT2S_API int opt2s_testing_check_division(uint64_t seed, int64_t n, int32_t mod
     if (e != cudaSuccess) return cuda_fail(e);
     *mismatches = static_cast<int64_t>(h);
     return OPT2S_OK;
+}
+
+OPT2S_API int64_t opt2s_testing_choose_chunk_elems(const TensorListDesc* desc, int64_t resident_warps)
+{
+    if (!desc || desc->count < 0 || (desc->count > 0 && !desc->tensors)) return OPT2S_ERR_INVALID_ARG;
+    return choose_chunk_elems(desc, resident_warps);
 }
 
 OPT2S_API int64_t opt2s_testing_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

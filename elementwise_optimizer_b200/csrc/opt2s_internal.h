@@ -40,8 +40,9 @@ struct StepScalars {
     double inv_bc1, inv_bc2;
 };
 
-constexpr int kDefaultBlockThreads = 256;
-constexpr int64_t kDefaultChunkElems = 8192;
+constexpr int kDefaultBlockThreads = 128;
+constexpr int64_t kDefaultChunkElems = 4096;   // largest chunk the plan builder picks
+constexpr int64_t kMinChunkElems = 256;        // one warp iteration (8 elements per lane)
 
 // Launches one step over `nchunks` records at `d_chunks` (device memory) on
 // `stream`.  block_threads: multiple of 32; max_blocks <= 0: occupancy-based
@@ -61,6 +62,10 @@ cudaError_t launch_step_table(const ChunkRec* d_chunks, int64_t nchunks, int alg
                               int skip_zeros, const StepScalars* d_table, int* d_index,
                               int table_len, int block_threads, int max_blocks,
                               cudaStream_t stream);
+
+// Resident warps of the step kernel for (algo, skip_zeros) on the current
+// device at `block_threads` threads per block (blocks per SM x SMs x warps).
+cudaError_t resident_warps(int algo, int skip_zeros, int block_threads, int64_t* out);
 
 // Widest block (threads, a multiple of 32) the step kernel for (algo,
 // skip_zeros) can be launched with: its registers per thread limit it.

@@ -457,6 +457,16 @@ cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros, int block_thread
     return cudaSuccess;
 }
 
+cudaError_t resident_warps(int algo, int skip_zeros, int block_threads, int64_t* out)
+{
+    int grid = 0;
+    // the occupancy cap is what grid_for returns for an unbounded chunk count
+    cudaError_t e = grid_for(INT64_MAX / 2, algo, skip_zeros, block_threads, 0, &grid);
+    if (e != cudaSuccess) return e;
+    *out = static_cast<int64_t>(grid) * (block_threads / 32);
+    return cudaSuccess;
+}
+
 cudaError_t max_block_threads(int algo, int skip_zeros, int* out)
 {
     cudaFuncAttributes attr;

@@ -46,6 +46,7 @@ using opt2s::ChunkRec;
 using opt2s::StepScalars;
 
 constexpr int64_t kNoAllocMaxChunks = 65536;   // 48 B each: 3 MiB per device
+constexpr int64_t kNoAllocChunkElems = 8192;   // elements per chunk record
 constexpr int kMaxDevices = 64;
 
 // The device-side scratch: one fixed chunk table per GPU.  In host code this
@@ -148,7 +149,7 @@ OPT2S_API int opt2s_step_noalloc(const TensorListDesc* desc, const Hyper* hyper,
     int st = check_hyper(hyper, step);
     if (st != OPT2S_OK) return st;
     std::lock_guard<std::mutex> lock(g_mu);
-    const int64_t ce = opt2s::kDefaultChunkElems;
+    const int64_t ce = kNoAllocChunkElems;
     int64_t nchunks = 0;
     if ((st = check_desc(desc, hyper->algo, ce, &nchunks)) != OPT2S_OK) return st;
     if (nchunks == 0) return OPT2S_OK;

@@ -48,7 +48,7 @@ int opt2s_testing_validate(const TensorListDesc *desc, const Hyper *hyper,
                            int step);
 
 /* Chunk length (elements, a positive multiple of 8) for plans created
- * afterwards; 0 restores the default.  Returns the previous value. */
+ * afterwards; 0 restores the per-plan choice.  Returns the previous value. */
 int64_t opt2s_testing_set_chunk_elems(int64_t chunk_elems);
 
 /* Threads per block (a multiple of 32 in [32, 1024]) and a cap on blocks per
@@ -62,8 +62,15 @@ int opt2s_testing_set_launch(int block_threads, int max_blocks);
  * opt2s_status. */
 int opt2s_testing_max_block_threads(int32_t algo, int32_t skip_zeros);
 
-/* The library's default chunk length in elements. */
+/* The library's largest chunk length in elements (chunk_elems <= 0 in
+ * opt2s_testing_build_chunks means this length). */
 int64_t opt2s_testing_default_chunk_elems(void);
+
+/* Host only: the chunk length a plan for `desc` gets on a device with
+ * `resident_warps` resident warps of the step kernel: the multiple of 256 in
+ * [256, 4096] minimizing ceil(chunks / resident_warps) * (length / 256 + 1),
+ * the modelled time of the slowest warp. */
+int64_t opt2s_testing_choose_chunk_elems(const TensorListDesc *desc, int64_t resident_warps);
 
 /* Runs the step kernel's exact division by a constant in (0, 1] and the IEEE
  * division __fdiv_rn side by side on `n` seeded random operand pairs on the
