@@ -71,6 +71,11 @@ def _load():
     lib.oracle_step_f64.argtypes = [i32, i32, f64, f64, f64, f64, f64, f64,
                                     f64, i32, vp, vp, vp, vp, vp, i64]
     lib.oracle_step_f64.restype = i32
+    lib.oracle_step_f32_fgrad.argtypes = [i32, i32, i32, f32, f32, f32, f32, f32,
+                                          f32, f32, i32, vp, vp, vp, vp, i64]
+    lib.oracle_step_f32_fgrad.restype = i32
+    lib.oracle_average_grads.argtypes = [i32, i32, vp, vp, i64]
+    lib.oracle_average_grads.restype = i32
     lib.oracle_bias_correction.argtypes = [f32, i32]
     lib.oracle_bias_correction.restype = f32
     lib.oracle_decay_factor.argtypes = [f32, f32]
@@ -116,6 +121,44 @@ def step_f32(param: np.ndarray, grad: np.ndarray, state1: np.ndarray,
         _ptr(state1), _ptr(state2), n)
     if rc != 0:
         raise ValueError(f"oracle_step_f32 rejected its arguments ({rc})")
+
+
+def step_f32_fgrad(param: np.ndarray, grad: np.ndarray, state1: np.ndarray,
+                   state2: np.ndarray, *, dtype: str, algo: str, step: int,
+                   lr: float, beta1: float, beta2: float, eps: float,
+                   beta3: float = 0.0, alpha: float = 0.0,
+                   weight_decay: float = 0.0, skip_zeros: bool = False) -> None:
+    """``step_f32`` with a float32 gradient for a param of any storage dtype."""
+    n = param.size
+    if grad.dtype != np.float32 or grad.size != n or param.itemsize != _ITEMSIZE[dtype]:
+        raise ValueError("grad must be float32 of the param's size")
+    want1 = 2 * n if algo == "ademamix" else n
+    if state1.dtype != np.float32 or state2.dtype != np.float32 or \
+            state1.size != want1 or state2.size != n:
+        raise ValueError("state arrays must be float32 of the right length")
+    rc = _load().oracle_step_f32_fgrad(
+        ALGO[algo], DTYPE[dtype], int(bool(skip_zeros)), lr, beta1, beta2,
+        beta3, alpha, eps, weight_decay, int(step), _ptr(param), _ptr(grad),
+        _ptr(state1), _ptr(state2), n)
+    if rc != 0:
+        raise ValueError(f"oracle_step_f32_fgrad rejected its arguments ({rc})")
+
+
+def average_grads(grads: list, dtype: str) -> np.ndarray:
+    """The rank-order fp32 mean of several ranks' gradients (storage bits of
+    ``dtype``), as the sharded data-parallel step defines it."""
+    n = grads[0].size
+    arrs = [np.ascontiguousarray(g) for g in grads]
+    for a in arrs:
+        if a.size != n or a.itemsize != _ITEMSIZE[dtype]:
+            raise ValueError("gradients must share size and storage dtype")
+    ptrs = (ctypes.c_void_p * len(arrs))(*[a.ctypes.data for a in arrs])
+    out = np.empty(n, np.float32)
+    rc = _load().oracle_average_grads(DTYPE[dtype], len(arrs), ctypes.cast(ptrs, ctypes.c_void_p),
+                                      _ptr(out), n)
+    if rc != 0:
+        raise ValueError("oracle_average_grads rejected its arguments")
+    return out
 
 
 def step_f64(param: np.ndarray, grad: np.ndarray, m: np.ndarray,

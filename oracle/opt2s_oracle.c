@@ -204,11 +204,32 @@ float oracle_decay_factor(float lr, float wd)
  *   p   = p*decay - lr*(num/den)       decay first, [AdamW]; [issue] "Scope"
  * Returns 0, or -1 on an argument the definitions do not cover.
  */
-int oracle_step_f32(int algo, int dtype, int skip_zeros,
-                    float lr, float beta1, float beta2, float beta3,
-                    float alpha, float eps, float weight_decay, int step,
-                    void *param, const void *grad, float *state1,
-                    float *state2, int64_t n)
+/* The per-element update of one step (shared by both fp32 step entries). */
+static void update_element(int algo, float g, float *p, float *m, float *m2, float *v,
+                           float lr, float beta1, float beta2, float beta3, float alpha,
+                           float eps, float bc1, float bc2, float decay,
+                           float one_minus_b1, float one_minus_b2, float one_minus_b3)
+{
+    float mi = beta1 * *m + one_minus_b1 * g;
+    float vi = beta2 * *v + (one_minus_b2 * g) * g;
+    float num = mi / bc1;
+    if (algo == OR_ADEMAMIX) {
+        float m2i = beta3 * *m2 + one_minus_b3 * g;
+        num = num + alpha * m2i;
+        *m2 = m2i;
+    }
+    float den = sqrtf(vi / bc2) + eps;
+    *p = *p * decay - lr * (num / den);
+    *m = mi;
+    *v = vi;
+}
+
+/* One step over n elements whose gradient is read by get_grad(grad, i). */
+static int step_core(int algo, int dtype, int skip_zeros, float lr, float beta1,
+                     float beta2, float beta3, float alpha, float eps,
+                     float weight_decay, int step, void *param, const void *grad,
+                     float (*get_grad)(const void *, int, int64_t), int grad_dtype,
+                     float *state1, float *state2, int64_t n)
 {
     if (step < 1 || n < 0) return -1;
     if (algo != OR_ADAM && algo != OR_ADEMAMIX) return -1;
@@ -229,26 +250,95 @@ int oracle_step_f32(int algo, int dtype, int skip_zeros,
     float *v = state2;
 
     for (int64_t i = 0; i < n; i++) {
-        float g = load_param(grad, dtype, i);
+        float g = get_grad(grad, grad_dtype, i);
         if (skip_zeros && g == 0.0f) continue;
         float p = load_param(param, dtype, i);
-
-        float mi = beta1 * m[i] + one_minus_b1 * g;
-        float vi = beta2 * v[i] + (one_minus_b2 * g) * g;
-        float num = mi / bc1;
-        if (algo == OR_ADEMAMIX) {
-            float m2i = beta3 * m2[i] + one_minus_b3 * g;
-            num = num + alpha * m2i;
-            m2[i] = m2i;
-        }
-        float den = sqrtf(vi / bc2) + eps;
-        p = p * decay - lr * (num / den);
-
-        m[i] = mi;
-        v[i] = vi;
+        update_element(algo, g, &p, &m[i], &m2[i], &v[i], lr, beta1, beta2, beta3,
+                       alpha, eps, bc1, bc2, decay, one_minus_b1, one_minus_b2,
+                       one_minus_b3);
         store_param(param, dtype, i, p);
     }
 
+    _mm_setcsr(csr);
+    return 0;
+}
+
+static float grad_in_storage(const void *grad, int dtype, int64_t i)
+{
+    return load_param(grad, dtype, i);
+}
+
+static float grad_in_f32(const void *grad, int dtype, int64_t i)
+{
+    (void)dtype;
+    return ((const float *)grad)[i];
+}
+
+/*
+ * One optimizer step, in place, over one tensor of n elements.
+ *
+ * algo      0 = Adam (AdamW when wd != 0), 1 = AdEMAMix.
+ * dtype     storage of param and grad: 0 fp32, 1 fp16, 2 bf16.
+ * state1    Adam: m (n floats).  AdEMAMix: [m1 | m2] (2n floats).
+ * state2    v (n floats).
+ * step      t >= 1, the 1-based index of this update.
+ *
+ * Per element, every operation rounded to fp32 in this order:
+ *   m   = beta1*m + (1-beta1)*g                           [Adam]
+ *   v   = beta2*v + ((1-beta2)*g)*g                       [Adam]
+ *   num = m / bc1                                         [Adam]
+ *   AdEMAMix only:
+ *     m2  = beta3*m2 + (1-beta3)*g                        [AdEMAMix]
+ *     num = num + alpha*m2                                [AdEMAMix]
+ *   den = sqrt(v / bc2) + eps                             [Adam]
+ *   p   = p*decay - lr*(num/den)       decay first, [AdamW]; [issue] "Scope"
+ * Returns 0, or -1 on an argument the definitions do not cover.
+ */
+int oracle_step_f32(int algo, int dtype, int skip_zeros,
+                    float lr, float beta1, float beta2, float beta3,
+                    float alpha, float eps, float weight_decay, int step,
+                    void *param, const void *grad, float *state1,
+                    float *state2, int64_t n)
+{
+    return step_core(algo, dtype, skip_zeros, lr, beta1, beta2, beta3, alpha, eps,
+                     weight_decay, step, param, grad, grad_in_storage, dtype, state1,
+                     state2, n);
+}
+
+/* The same step with a gradient already in fp32 (whatever the param
+ * storage), e.g. the data-parallel average below. */
+int oracle_step_f32_fgrad(int algo, int dtype, int skip_zeros,
+                          float lr, float beta1, float beta2, float beta3,
+                          float alpha, float eps, float weight_decay, int step,
+                          void *param, const float *grad, float *state1,
+                          float *state2, int64_t n)
+{
+    return step_core(algo, dtype, skip_zeros, lr, beta1, beta2, beta3, alpha, eps,
+                     weight_decay, step, param, grad, grad_in_f32, OR_F32, state1,
+                     state2, n);
+}
+
+/*
+ * Data-parallel gradient: the mean of `world` ranks' gradients (storage
+ * dtype), widened exactly, summed in fp32 in rank order 0, 1, ..., world-1
+ * (each addition rounded), then divided by world (rounded).  This is the
+ * gradient the sharded step applies: the reduce-scatter of a ZeRO-style
+ * data-parallel optimizer, with the order fixed so every run gives the same
+ * bits.  Returns 0, or -1 on bad arguments.
+ */
+int oracle_average_grads(int dtype, int world, const void *const *grads,
+                         float *out, int64_t n)
+{
+    if (world < 1 || n < 0) return -1;
+    if (dtype != OR_F32 && dtype != OR_F16 && dtype != OR_BF16) return -1;
+    unsigned int csr = _mm_getcsr();
+    _mm_setcsr(csr & ~(0x8000u | 0x0040u));
+    for (int64_t i = 0; i < n; i++) {
+        float sum = load_param(grads[0], dtype, i);
+        for (int q = 1; q < world; q++)
+            sum = sum + load_param(grads[q], dtype, i);
+        out[i] = sum / (float)world;
+    }
     _mm_setcsr(csr);
     return 0;
 }

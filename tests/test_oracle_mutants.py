@@ -21,18 +21,22 @@ MUTANTS = {
     "eps_dropped": ("sqrtf(vi / bc2) + eps", "sqrtf(vi / bc2)"),
     "eps_inside_sqrt": ("sqrtf(vi / bc2) + eps", "sqrtf(vi / bc2 + eps)"),
     "bc1_for_v": ("sqrtf(vi / bc2)", "sqrtf(vi / bc1)"),
-    "decay_after_update": ("p = p * decay - lr * (num / den);",
-                           "p = (p - lr * (num / den)) * decay;"),
-    "update_sign": ("p = p * decay - lr * (num / den);",
-                    "p = p * decay + lr * (num / den);"),
+    "decay_after_update": ("*p = *p * decay - lr * (num / den);",
+                           "*p = (*p - lr * (num / den)) * decay;"),
+    "update_sign": ("*p = *p * decay - lr * (num / den);",
+                    "*p = *p * decay + lr * (num / den);"),
     "m2_bias_corrected": ("num = num + alpha * m2i;",
-                          "num = num + alpha * (m2i / oracle_bias_correction(beta3, step));"),
+                          "num = num + alpha * (m2i / bc1);"),
     "alpha_on_m1": ("num = num + alpha * m2i;", "num = alpha * num + m2i;"),
-    "one_minus_b3_dropped": ("beta3 * m2[i] + one_minus_b3 * g",
-                             "beta3 * m2[i] + g"),
+    "one_minus_b3_dropped": ("beta3 * *m2 + one_minus_b3 * g",
+                             "beta3 * *m2 + g"),
     "v_not_squared": ("(one_minus_b2 * g) * g", "(one_minus_b2 * g)"),
-    "m_uses_beta2": ("float mi = beta1 * m[i] + one_minus_b1 * g;",
-                     "float mi = beta2 * m[i] + one_minus_b1 * g;"),
+    "average_wrong_divisor": ("out[i] = sum / (float)world;",
+                              "out[i] = sum / (float)(world + 1);"),
+    "average_drops_last_rank": ("for (int q = 1; q < world; q++)",
+                                "for (int q = 1; q < world - 1; q++)"),
+    "m_uses_beta2": ("float mi = beta1 * *m + one_minus_b1 * g;",
+                     "float mi = beta2 * *m + one_minus_b1 * g;"),
     "bias_exponent_off_by_one": ("pow((double)beta, (double)t)",
                                  "pow((double)beta, (double)(t + 1))"),
     "decay_without_lr": ("1.0 - (double)lr * (double)wd", "1.0 - (double)wd"),

@@ -411,3 +411,53 @@ def test_golden_traces(oracle_mod):
         case, t, hexbits = r[0], int(r[1]), r[2]
         got = run_trace(case)[t - 1]
         assert got == hexbits, (case, t, got, hexbits)
+
+
+# --------------------------------------------------------------------------
+# Data-parallel pieces: rank-order mean of gradients, fp32-gradient step
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("world", [1, 2, 3, 5, 8])
+def test_average_grads_within_rounding_of_exact_mean(oracle_mod, dtype, world):
+    """Each of the world-1 additions and the division rounds once, so the
+    fp32 mean is within (world+1)*2^-24 * sum|g|/world of the exact mean."""
+    n = 20000
+    g = np.random.Generator(np.random.Philox(61))
+    grads = [synth.to_storage((g.standard_normal(n) * 10.0 ** g.uniform(-6, 2, n)).astype(np.float32), dtype)
+             for _ in range(world)]
+    avg = oracle_mod.average_grads(grads, dtype)
+    vals = np.stack([synth.from_storage(x, dtype).astype(np.float64) for x in grads])
+    exact = vals.mean(axis=0)
+    bound = (world + 1) * 2.0 ** -24 * np.abs(vals).sum(axis=0) / world + 1e-45
+    assert np.all(np.abs(avg - exact) <= bound)
+    if world == 1:
+        assert np.array_equal(avg, vals[0].astype(np.float32))
+
+
+@pytest.mark.parametrize("world", [2, 4, 8])
+def test_average_of_identical_grads_is_exact(oracle_mod, world):
+    """world identical copies (world a power of two) of values with at most
+    20 significant bits: every partial sum k*x (k <= 8) is exact, and so is
+    the division by world."""
+    g = np.random.Generator(np.random.Philox(62))
+    mant = g.integers(-(1 << 20) + 1, 1 << 20, 4096).astype(np.float64)
+    x = (mant * 2.0 ** g.integers(-60, 10, 4096)).astype(np.float32)
+    assert np.array_equal(oracle_mod.average_grads([x] * world, "f32"), x)
+
+
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_fp32_gradient_step_reduces_to_the_storage_step(oracle_mod, algo, dtype):
+    """A float32 gradient whose values are representable in the storage dtype
+    steps exactly like the storage-dtype gradient."""
+    n = 3001
+    p, gr, s1, v = _random_state(71, n, dtype, algo)
+    kw = dict(dtype=dtype, algo=algo, step=4, lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8,
+              beta3=0.99, alpha=5.0, weight_decay=0.01, skip_zeros=True)
+    a = [x.copy() for x in (p, s1, v)]
+    oracle_mod.step_f32(a[0], gr, a[1], a[2], **kw)
+    b = [x.copy() for x in (p, s1, v)]
+    oracle_mod.step_f32_fgrad(b[0], synth.from_storage(gr, dtype), b[1], b[2], **kw)
+    for x, y in zip(a, b):
+        assert np.array_equal(x.view(np.uint8), y.view(np.uint8))
