@@ -62,6 +62,16 @@ class opt2s_step_scalars(ctypes.Structure):
         ("inv_bc1", ctypes.c_double), ("inv_bc2", ctypes.c_double)]
 
 
+MAX_WORLD = 8
+
+
+class opt2s_shard_desc(ctypes.Structure):
+    _fields_ = [("world", ctypes.c_int32), ("rank", ctypes.c_int32), ("numel", ctypes.c_int64),
+                ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("params", ctypes.c_void_p * MAX_WORLD), ("grads", ctypes.c_void_p * MAX_WORLD),
+                ("state1", ctypes.c_void_p), ("state2", ctypes.c_void_p)]
+
+
 class opt2s_testing_chunk(ctypes.Structure):
     _fields_ = [("tensor", ctypes.c_int64), ("start", ctypes.c_int64),
                 ("len", ctypes.c_int64), ("dtype", ctypes.c_int32),
@@ -85,6 +95,11 @@ EXPORTS = {
                                                ctypes.c_void_p]),
     "opt2s_plan_step_table": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                              ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
+    "opt2s_shard_range": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                         ctypes.POINTER(ctypes.c_int64),
+                                         ctypes.POINTER(ctypes.c_int64)]),
+    "opt2s_shard_step": (ctypes.c_int, [ctypes.POINTER(opt2s_shard_desc), ctypes.POINTER(Hyper),
+                                        ctypes.c_int, ctypes.c_void_p]),
     "opt2s_release_cache": (ctypes.c_int, []),
     "opt2s_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "opt2s_last_cuda_error": (ctypes.c_int, []),
@@ -272,6 +287,31 @@ def fill_step_scalars(hyper: Hyper, first_step: int, count: int) -> bytes:
     check(lib().opt2s_fill_step_scalars(ctypes.byref(hyper), int(first_step), int(count),
                                         ctypes.cast(arr, ctypes.c_void_p)), "opt2s_fill_step_scalars")
     return bytes(arr)[:count * ctypes.sizeof(opt2s_step_scalars)]
+
+
+def opt2s_shard_range(numel: int, world: int, rank: int) -> tuple:
+    """(start, length) of rank's shard of a flat buffer of numel elements."""
+    a, n = ctypes.c_int64(), ctypes.c_int64()
+    check(lib().opt2s_shard_range(int(numel), int(world), int(rank), ctypes.byref(a),
+                                  ctypes.byref(n)), "opt2s_shard_range")
+    return a.value, n.value
+
+
+def make_shard_desc(world: int, rank: int, numel: int, dtype: int, params, grads,
+                    state1, state2) -> opt2s_shard_desc:
+    d = opt2s_shard_desc()
+    d.world, d.rank, d.numel, d.dtype, d.reserved = world, rank, numel, dtype, 0
+    for q in range(world):
+        d.params[q] = _ptr(params[q])
+        d.grads[q] = _ptr(grads[q])
+    d.state1 = _ptr(state1) if state1 is not None else None
+    d.state2 = _ptr(state2) if state2 is not None else None
+    return d
+
+
+def opt2s_shard_step(desc: opt2s_shard_desc, hyper: Hyper, step: int, stream=None) -> None:
+    check(lib().opt2s_shard_step(ctypes.byref(desc), ctypes.byref(hyper), int(step),
+                                 _stream_handle(stream)), "opt2s_shard_step")
 
 
 def opt2s_release_cache() -> None:

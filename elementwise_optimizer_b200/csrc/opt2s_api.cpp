@@ -440,6 +440,83 @@ OPT2S_API int opt2s_plan_step_table(const opt2s_plan* plan, int32_t skip_zeros,
     return OPT2S_OK;
 }
 
+static_assert(OPT2S_MAX_WORLD == opt2s::kMaxWorld, "world limit");
+
+OPT2S_API int opt2s_shard_range(int64_t numel, int32_t world, int32_t rank, int64_t* start,
+                                int64_t* len)
+{
+    if (!start || !len || numel < 0 || world < 1 || world > OPT2S_MAX_WORLD || rank < 0 ||
+        rank >= world)
+        return OPT2S_ERR_INVALID_ARG;
+    const int64_t units = (numel + 7) / 8;                 // 8-element units
+    const int64_t u0 = units * rank / world, u1 = units * (rank + 1) / world;
+    const int64_t a = std::min(u0 * 8, numel), b = std::min(u1 * 8, numel);
+    *start = a;
+    *len = b - a;
+    return OPT2S_OK;
+}
+
+OPT2S_API int opt2s_shard_step(const opt2s_shard_desc* d, const Hyper* hyper, int step,
+                               cudaStream_t stream)
+{
+    int st = validate_hyper(hyper, step);
+    if (st != OPT2S_OK) return st;
+    if (!d || d->reserved != 0) return OPT2S_ERR_INVALID_ARG;
+    int64_t start = 0, len = 0;
+    if ((st = opt2s_shard_range(d->numel, d->world, d->rank, &start, &len)) != OPT2S_OK) return st;
+    if (d->dtype != OPT2S_F32 && d->dtype != OPT2S_F16 && d->dtype != OPT2S_BF16)
+        return OPT2S_ERR_INVALID_ARG;
+    if (d->numel == 0) return OPT2S_OK;
+    const int es = elem_bytes(d->dtype);
+    std::vector<Range> ranges;
+    const uintptr_t n = static_cast<uintptr_t>(d->numel);
+    for (int q = 0; q < d->world; ++q) {
+        const auto p = reinterpret_cast<uintptr_t>(d->params[q]);
+        const auto g = reinterpret_cast<uintptr_t>(d->grads[q]);
+        if (!p || !g || p % es || g % es) return OPT2S_ERR_INVALID_ARG;
+        ranges.push_back({p, p + n * es, true});
+        ranges.push_back({g, g + n * es, false});
+    }
+    if (len > 0) {
+        const auto s1 = reinterpret_cast<uintptr_t>(d->state1);
+        const auto s2 = reinterpret_cast<uintptr_t>(d->state2);
+        if (!s1 || !s2 || s1 % 4 || s2 % 4) return OPT2S_ERR_INVALID_ARG;
+        const uintptr_t k = static_cast<uintptr_t>(len);
+        ranges.push_back({s1, s1 + (hyper->algo == OPT2S_ADEMAMIX ? 2 * k : k) * 4, true});
+        ranges.push_back({s2, s2 + k * 4, true});
+    }
+    std::sort(ranges.begin(), ranges.end(), [](const Range& a, const Range& b) { return a.lo < b.lo; });
+    uintptr_t reach_w = 0, reach_any = 0;
+    bool have_w = false, have_any = false;
+    for (const Range& r : ranges) {
+        if (have_w && r.lo < reach_w) return OPT2S_ERR_ALIAS;
+        if (r.written && have_any && r.lo < reach_any) return OPT2S_ERR_ALIAS;
+        if (r.written) { reach_w = have_w ? std::max(reach_w, r.hi) : r.hi; have_w = true; }
+        reach_any = have_any ? std::max(reach_any, r.hi) : r.hi;
+        have_any = true;
+    }
+    if (len == 0) return OPT2S_OK;
+    opt2s::ShardArgs a{};
+    for (int q = 0; q < d->world; ++q) {
+        a.params[q] = d->params[q];
+        a.grads[q] = d->grads[q];
+    }
+    a.m = d->state1;
+    a.v = d->state2;
+    a.m2 = d->state1 + len;
+    a.shard_start = start;
+    a.shard_len = len;
+    a.world = d->world;
+    a.rank = d->rank;
+    a.dtype = d->dtype;
+    a.chunk_elems = static_cast<int32_t>(g_chunk_elems > 0 ? g_chunk_elems : opt2s::kDefaultChunkElems);
+    cudaError_t e = opt2s::launch_shard_step(a, hyper->algo, hyper->skip_zeros, make_scalars(hyper, step),
+                                             block_threads_now(), stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return OPT2S_OK;
+}
+
 OPT2S_API int opt2s_release_cache(void)
 {
     std::lock_guard<std::mutex> lock(g_cache_mu);

@@ -44,6 +44,28 @@ constexpr int kDefaultBlockThreads = 128;
 constexpr int64_t kDefaultChunkElems = 4096;   // largest chunk the plan builder picks
 constexpr int64_t kMinChunkElems = 256;        // one warp iteration (8 elements per lane)
 
+// The sharded (ZeRO-style) step of one rank.  Every rank holds the whole flat
+// param and grad buffers (same layout); this rank updates the elements
+// [shard_start, shard_start + shard_len) with the rank-order mean of all
+// ranks' gradients and writes the new values into every rank's param buffer.
+constexpr int kMaxWorld = 8;
+struct ShardArgs {
+    void* params[kMaxWorld];        // rank q's flat param buffer, addressable here
+    const void* grads[kMaxWorld];   // rank q's flat grad buffer, addressable here
+    float* m;                       // this rank's shard state (shard-relative)
+    float* v;
+    float* m2;                      // AdEMAMix: m + shard_len
+    int64_t shard_start;
+    int64_t shard_len;
+    int32_t world;
+    int32_t rank;
+    int32_t dtype;
+    int32_t chunk_elems;
+};
+
+cudaError_t launch_shard_step(const ShardArgs& a, int algo, int skip_zeros, const StepScalars& s,
+                              int block_threads, cudaStream_t stream);
+
 // Launches one step over `nchunks` records at `d_chunks` (device memory) on
 // `stream`.  block_threads: multiple of 32; max_blocks <= 0: occupancy-based
 // cap (resident blocks per SM x SM count).  Returns the launch status.

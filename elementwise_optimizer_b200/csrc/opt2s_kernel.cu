@@ -283,6 +283,128 @@ __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& 
     }
 }
 
+// ---------------------------------------------------------------------------
+// The sharded step (reduce-scatter + update + all-gather in one kernel).
+//
+// Element e of this rank's shard gets g = (g_0[e] + g_1[e] + ... + g_{W-1}[e])
+// / W, widened exactly, summed in rank order and divided with IEEE fp32
+// operations, then the same update as the plain step; the new param is stored
+// into the param buffer of every rank.  Ranks touch disjoint shards, grads are
+// only read and state is local, so ranks never wait on one another inside the
+// kernel; the caller orders the step between two cross-rank barriers (grads
+// final before, params read after).  Peer buffers are reached with ordinary
+// loads and stores (NVLink on a multi-GPU node; no TMA, no multicast).
+// ---------------------------------------------------------------------------
+template <int DT, int ALGO, bool SKIP>
+__device__ __forceinline__ void shard_scalar(const ShardArgs& a, int64_t k, const StepScalars& s)
+{
+    using P = Param<DT>;
+    const int64_t e = a.shard_start + k;
+    constexpr int B = P::kBytes;
+    float g = P::load1(static_cast<const char*>(a.grads[0]) + e * B, 0);
+#pragma unroll
+    for (int q = 1; q < kMaxWorld; ++q)
+        if (q < a.world) g = __fadd_rn(g, P::load1(static_cast<const char*>(a.grads[q]) + e * B, 0));
+    g = __fdiv_rn(g, static_cast<float>(a.world));
+    if (SKIP && g == 0.0f) return;
+    float p = P::load1(static_cast<const char*>(a.params[a.rank]) + e * B, 0);
+    float m = __ldcs(a.m + k);
+    float v = __ldcs(a.v + k);
+    float m2 = 0.0f;
+    if (ALGO == kAdEMAMix) m2 = __ldcs(a.m2 + k);
+    update<ALGO, false>(g, p, m, v, m2, s);
+#pragma unroll
+    for (int q = 0; q < kMaxWorld; ++q)
+        if (q < a.world) P::store1(static_cast<char*>(a.params[q]) + e * B, 0, p);
+    __stcs(a.m + k, m);
+    __stcs(a.v + k, v);
+    if (ALGO == kAdEMAMix) __stcs(a.m2 + k, m2);
+}
+
+// Elements [k0, k0 + len) of the shard (shard-relative), one warp.
+template <int DT, int ALGO, bool SKIP>
+__device__ __forceinline__ void shard_chunk(const ShardArgs& a, int64_t k0, uint32_t len,
+                                            const StepScalars& s, int lane)
+{
+    using P = Param<DT>;
+    constexpr int V = P::kVec;
+    constexpr int B = P::kBytes;
+    const int64_t e0 = a.shard_start + k0;
+    const char* own = static_cast<const char*>(a.params[a.rank]) + e0 * B;
+    uint32_t head = static_cast<uint32_t>(((16u - (reinterpret_cast<uintptr_t>(own) & 15u)) & 15u) / B);
+    bool vec_ok = aligned16(a.m + k0, head, 4) && aligned16(a.v + k0, head, 4) &&
+                  (ALGO != kAdEMAMix || aligned16(a.m2 + k0, head, 4));
+#pragma unroll
+    for (int q = 0; q < kMaxWorld; ++q)
+        if (q < a.world)
+            vec_ok = vec_ok && aligned16(static_cast<const char*>(a.params[q]) + e0 * B, head, B) &&
+                     aligned16(static_cast<const char*>(a.grads[q]) + e0 * B, head, B);
+    if (!vec_ok || head > len) head = len;
+    const uint32_t nvec = (len - head) / V;
+    const uint32_t body_end = head + nvec * V;
+    for (uint32_t i = lane; i < head; i += 32) shard_scalar<DT, ALGO, SKIP>(a, k0 + i, s);
+    for (uint32_t i = body_end + lane; i < len; i += 32) shard_scalar<DT, ALGO, SKIP>(a, k0 + i, s);
+
+    const float world = static_cast<float>(a.world);
+    for (uint32_t vi = lane; vi < nvec; vi += 32) {
+        const uint32_t i = head + vi * V;          // chunk-relative element
+        const int64_t k = k0 + i;                  // shard-relative element
+        const int64_t e = e0 + i;                  // flat element
+        typename P::Raw graw[kMaxWorld];
+#pragma unroll
+        for (int q = 0; q < kMaxWorld; ++q)
+            if (q < a.world) graw[q] = P::load(static_cast<const char*>(a.grads[q]) + e * B, 0);
+        const typename P::Raw praw = P::load(static_cast<const char*>(a.params[a.rank]) + e * B, 0);
+        float m[V], v[V], m2[V], g[V], p[V];
+        P::widen(graw[0], g);
+        P::widen(praw, p);
+        load_state<V>(a.m + k, 0, m);
+        load_state<V>(a.v + k, 0, v);
+        if (ALGO == kAdEMAMix) load_state<V>(a.m2 + k, 0, m2);
+#pragma unroll
+        for (int q = 1; q < kMaxWorld; ++q) {
+            if (q < a.world) {
+                float x[V];
+                P::widen(graw[q], x);
+#pragma unroll
+                for (int j = 0; j < V; ++j) g[j] = __fadd_rn(g[j], x[j]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            g[j] = __fdiv_rn(g[j], world);
+            update<ALGO, SKIP>(g[j], p[j], m[j], v[j], m2[j], s);
+        }
+        const typename P::Raw out = P::narrow(p, praw, g, SKIP);
+#pragma unroll
+        for (int q = 0; q < kMaxWorld; ++q)
+            if (q < a.world) P::store(static_cast<char*>(a.params[q]) + e * B, 0, out);
+        store_state<V>(a.m + k, 0, m);
+        store_state<V>(a.v + k, 0, v);
+        if (ALGO == kAdEMAMix) store_state<V>(a.m2 + k, 0, m2);
+    }
+}
+
+template <int ALGO, bool SKIP>
+__global__ void shard_step_kernel(ShardArgs a, StepScalars s)
+{
+    const int lane = threadIdx.x & 31;
+    const int warps_per_block = blockDim.x >> 5;
+    const int64_t warp = static_cast<int64_t>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5);
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * warps_per_block;
+    const int64_t ce = a.chunk_elems;
+    const int64_t nchunks = (a.shard_len + ce - 1) / ce;
+    for (int64_t c = warp; c < nchunks; c += nwarps) {
+        const int64_t k0 = c * ce;
+        const uint32_t len = static_cast<uint32_t>(min(ce, a.shard_len - k0));
+        switch (a.dtype) {
+        case kF32: shard_chunk<kF32, ALGO, SKIP>(a, k0, len, s, lane); break;
+        case kF16: shard_chunk<kF16, ALGO, SKIP>(a, k0, len, s, lane); break;
+        default: shard_chunk<kBF16, ALGO, SKIP>(a, k0, len, s, lane); break;
+        }
+    }
+}
+
 // The whole step: warp w takes chunks w, w + W, w + 2W, ... of the table.
 template <int ALGO, bool SKIP>
 __device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, int nchunks,
@@ -490,6 +612,31 @@ cudaError_t launch_step(const ChunkRec* d_chunks, int64_t nchunks, int algo, int
     void* args[] = {const_cast<ChunkRec**>(&d_chunks), &n, &sc};
     return cudaLaunchKernel(reinterpret_cast<const void*>(pick(algo, skip_zeros)),
                             dim3(grid), dim3(block_threads), args, 0, stream);
+}
+
+cudaError_t launch_shard_step(const ShardArgs& a, int algo, int skip_zeros, const StepScalars& s,
+                              int block_threads, cudaStream_t stream)
+{
+    if (a.shard_len <= 0) return cudaSuccess;
+    using ShardFn = void (*)(ShardArgs, StepScalars);
+    ShardFn fn = algo == kAdEMAMix
+                     ? (skip_zeros ? shard_step_kernel<kAdEMAMix, true> : shard_step_kernel<kAdEMAMix, false>)
+                     : (skip_zeros ? shard_step_kernel<kAdam, true> : shard_step_kernel<kAdam, false>);
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, block_threads, 0);
+    if (e != cudaSuccess) return e;
+    const int64_t nchunks = (a.shard_len + a.chunk_elems - 1) / a.chunk_elems;
+    const int64_t need = (nchunks + block_threads / 32 - 1) / (block_threads / 32);
+    const int64_t cap = static_cast<int64_t>(per_sm < 1 ? 1 : per_sm) * sms;
+    const int grid = static_cast<int>(need < cap ? need : cap);
+    ShardArgs aa = a;
+    StepScalars sc = s;
+    fill_reciprocals(&sc);
+    void* args[] = {&aa, &sc};
+    return cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3(grid), dim3(block_threads), args, 0,
+                            stream);
 }
 
 void fill_reciprocals(StepScalars* s)

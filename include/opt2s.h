@@ -177,6 +177,48 @@ int opt2s_plan_step_table(const opt2s_plan *plan, int32_t skip_zeros,
                           int32_t *d_index, cudaStream_t stream);
 
 /*
+ * ZeRO-style sharded step: gradient reduce-scatter, update and parameter
+ * all-gather fused in one kernel over peer memory.
+ *
+ * `world` ranks (<= OPT2S_MAX_WORLD) each hold the whole flat param buffer and
+ * their own whole flat grad buffer (same length and storage dtype on every
+ * rank), and optimizer state only for their shard.  opt2s_shard_range gives
+ * rank r's shard: a contiguous range of the flat buffers, ranges disjoint and
+ * covering [0, numel), balanced to within 8 elements, starts multiples of 8.
+ * opt2s_shard_step, called by rank r (on its device, `stream`), updates every
+ * element e of its shard with
+ *     g = (g_0[e] + g_1[e] + ... + g_{world-1}[e]) / world
+ * (storage values widened exactly; fp32 additions in rank order, then an fp32
+ * division, each rounded once), then the plain step's update, and stores the
+ * new param into EVERY rank's param buffer.  params[q] and grads[q] are rank
+ * q's buffers as addressable from this rank's device (peer mappings: CUDA IPC,
+ * symmetric memory, or peer access between devices of one process); state1 /
+ * state2 hold this rank's shard (state1: m, or [m1 | m2] with 2 x shard
+ * length floats; state2: v), zero before step 1.  Ranks never wait for one
+ * another inside the kernel; the caller must order each step after every
+ * rank's gradient is complete and before any rank reads params again (e.g. a
+ * cross-rank barrier on both sides).  With world == 1 the result is bitwise
+ * that of opt2s_step.  No TMA and no multicast touch peer memory.
+ */
+#define OPT2S_MAX_WORLD 8
+typedef struct {
+    int32_t world;
+    int32_t rank;
+    int64_t numel;                           /* length of every flat buffer */
+    int32_t dtype;                           /* opt2s_dtype of params and grads */
+    int32_t reserved;                        /* must be 0 */
+    void *params[OPT2S_MAX_WORLD];           /* [q] rank q's param buffer */
+    const void *grads[OPT2S_MAX_WORLD];      /* [q] rank q's grad buffer */
+    float *state1;
+    float *state2;
+} opt2s_shard_desc;
+
+int opt2s_shard_range(int64_t numel, int32_t world, int32_t rank, int64_t *start,
+                      int64_t *len);
+int opt2s_shard_step(const opt2s_shard_desc *desc, const Hyper *hyper, int step,
+                     cudaStream_t stream);
+
+/*
  * opt2s_step without any allocation by the library.  The paper this library
  * follows has no counterpart to it: it exists for callers that cannot let a
  * library allocate device memory -- runtimes that own all device memory

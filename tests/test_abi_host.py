@@ -346,3 +346,55 @@ def test_chunk_length_follows_collection_size(L):
         c = B.testing_choose_chunk_elems(tl, W)
         assert c % 256 == 0 and 256 <= c <= 4096
     assert B.testing_choose_chunk_elems(B.TensorList([]), W) in (256, 512, 1024, 2048, 4096)
+
+
+# --------------------------------------------------------------------------
+# Sharded step: partition and validation (host only)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("numel", [0, 1, 7, 8, 9, 1000, 1000003, 268_435_456])
+@pytest.mark.parametrize("world", [1, 2, 3, 5, 8])
+def test_shard_ranges_partition_the_buffer(L, numel, world):
+    ranges = [B.opt2s_shard_range(numel, world, r) for r in range(world)]
+    pos = 0
+    for start, n in ranges:
+        assert start == pos and n >= 0 and start % 8 == 0 or n == 0
+        pos = start + n
+    assert pos == numel
+    sizes = [n for _, n in ranges]
+    assert max(sizes) - min(sizes) <= 8 + (numel % 8)
+
+
+def test_shard_range_rejects_bad_arguments(L):
+    for args in ((10, 0, 0), (10, 9, 0), (10, 2, 2), (10, 2, -1), (-1, 1, 0)):
+        with pytest.raises(B.Opt2sError):
+            B.opt2s_shard_range(*args)
+
+
+def test_shard_step_validation(L):
+    arena = Arena()
+    n, world = 4096, 2
+    params = [arena.alloc(4 * n) for _ in range(world)]
+    grads = [arena.alloc(4 * n) for _ in range(world)]
+    k = B.opt2s_shard_range(n, world, 0)[1]
+    s1, s2 = arena.alloc(4 * k), arena.alloc(4 * k)
+    h = B.make_hyper("adam")
+
+    def run(**kw):
+        d = B.make_shard_desc(world, 0, n, 0, params, grads, s1, s2)
+        for key, val in kw.items():
+            if key in ("params", "grads"):
+                for q, x in enumerate(val):
+                    getattr(d, key)[q] = x
+            else:
+                setattr(d, key, val)
+        return L.opt2s_shard_step(ctypes.byref(d), ctypes.byref(h), 1, None)
+
+    assert run(world=0) == -1 and run(world=9) == -1 and run(rank=2) == -1
+    assert run(dtype=5) == -1 and run(reserved=1) == -1
+    assert run(params=[params[0], 0]) == -1                        # missing peer buffer
+    assert run(grads=[grads[0], params[1]]) == -2                  # a grad is a param buffer
+    assert run(params=[params[0], params[0]]) == -2                # two ranks, one buffer
+    assert run(state1=params[0] + 64) == -2                        # state inside a param buffer
+    assert run(state2=0) == -1
+    assert L.opt2s_shard_step(None, ctypes.byref(h), 1, None) == -1
