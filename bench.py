@@ -500,6 +500,151 @@ def run_reference(args, rank, world):
     }
 
 
+# ---------------------------------------------------------------------------
+# Protocol of the bitsandbytes issue "Investigate a 256-thread SM103 path for
+# small 32-bit optimizer tensors" (section "B300 benchmark and acceptance"):
+# preallocated direct cells and eager collections, >= 20 warm-ups, 7
+# interleaved rounds, medians with p10/p90.
+# ---------------------------------------------------------------------------
+
+CELL_SIZES = [1, 32, 64, 128, 256, 512, 768, 1023, 1024, 1025, 2048, 4096]
+
+
+def _pct(xs, q):
+    xs = sorted(xs)
+    return xs[min(len(xs) - 1, int(q * len(xs)))]
+
+
+def run_direct_cells(rounds=7, samples=200, warmup=20):
+    """One tensor per call (opt2s_step), every (algo, dtype, n) cell; device
+    time per call from CUDA events, host dispatch time from the wall clock of
+    back-to-back calls.  torch.optim.AdamW(fused=True) on the same tensor is
+    timed alongside for context."""
+    import torch
+    from elementwise_optimizer_b200 import binding as B
+    dev = torch.device("cuda")
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+    cells = []
+    for algo in ("adam", "ademamix"):
+        for dt in ("f16", "bf16", "f32"):
+            for n in CELL_SIZES:
+                p = torch.randn(n, device=dev).to(tdt[dt])
+                g = (torch.randn(n, device=dev) * 1e-2).to(tdt[dt])
+                s1 = torch.zeros(2 * n if algo == "ademamix" else n, device=dev)
+                s2 = torch.zeros(n, device=dev)
+                h = B.make_hyper(algo, lr=1e-3, weight_decay=0.01, beta3=0.9999, alpha=5.0)
+                tl = B.TensorList.from_tensors([p], [g], [s1], [s2])
+                ref = None
+                if algo == "adam":
+                    rp = torch.nn.Parameter(p.clone())
+                    rp.grad = g.clone()
+                    ref = torch.optim.AdamW([rp], lr=1e-3, weight_decay=0.01, fused=True)
+                cells.append(dict(algo=algo, dtype=dt, n=n, tl=tl, h=h, ref=ref, step=0,
+                                  dev=[], host=[], torch_dev=[]))
+    stream = torch.cuda.current_stream()
+    for c in cells:
+        for _ in range(warmup):
+            c["step"] += 1
+            B.opt2s_step(c["tl"], c["h"], c["step"])
+            if c["ref"] is not None:
+                c["ref"].step()
+    torch.cuda.synchronize()
+    for _ in range(rounds):
+        for c in cells:                       # interleaved: every cell once per round
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(samples + 1)]
+            ev[0].record(stream)
+            for k in range(samples):
+                c["step"] += 1
+                B.opt2s_step(c["tl"], c["h"], c["step"])
+                ev[k + 1].record(stream)
+            torch.cuda.synchronize()
+            c["dev"] += [ev[k].elapsed_time(ev[k + 1]) * 1e3 for k in range(samples)]
+            t0 = time.perf_counter()
+            for k in range(samples):
+                c["step"] += 1
+                B.opt2s_step(c["tl"], c["h"], c["step"])
+            t1 = time.perf_counter()
+            torch.cuda.synchronize()
+            c["host"].append((t1 - t0) / samples * 1e6)
+            if c["ref"] is not None:
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(samples + 1)]
+                ev[0].record(stream)
+                for k in range(samples):
+                    c["ref"].step()
+                    ev[k + 1].record(stream)
+                torch.cuda.synchronize()
+                c["torch_dev"] += [ev[k].elapsed_time(ev[k + 1]) * 1e3 for k in range(samples)]
+    out = []
+    for c in cells:
+        row = {"algo": c["algo"], "dtype": c["dtype"], "n": c["n"],
+               "us_median": _pct(c["dev"], 0.5), "us_p10": _pct(c["dev"], 0.1),
+               "us_p90": _pct(c["dev"], 0.9), "host_dispatch_us_median": _pct(c["host"], 0.5)}
+        if c["torch_dev"]:
+            row["torch_fused_adamw_us_median"] = _pct(c["torch_dev"], 0.5)
+        out.append(row)
+    return {"mode": "direct-cells", "rounds": rounds, "samples_per_round": samples,
+            "warmup": warmup, "cells": out,
+            "note": "device time per call between CUDA events on the launching stream; "
+                    "host_dispatch_us is wall time per call of back-to-back calls (ctypes included)"}
+
+
+def run_eager_collection(rounds=7, steps=50, warmup=20):
+    """optimizer.step() on a fixed collection: the 2,000 bias/norm/LoRA-like
+    tensors (64..1,024 elements, fp32/bf16/fp16) plus 64 tensors of 4,096..
+    65,536 elements.  Wall time per step (host dispatch included, GPU drained
+    at the end of each batch); a captured CUDA graph of the same step as a
+    diagnostic control; torch.optim.AdamW(fused=True) for context."""
+    import torch
+    from elementwise_optimizer_b200 import optim, synth
+    dev = torch.device("cuda")
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+    w = synth.small_collection()
+    sizes = list(w.sizes) + [4096 * (1 << (i % 5)) for i in range(64)]
+    dtypes = list(w.dtypes) + [("f32", "bf16", "f16")[i % 3] for i in range(64)]
+    gen = torch.Generator(device=dev).manual_seed(1)
+
+    def make():
+        ps = []
+        for n, d in zip(sizes, dtypes):
+            p = torch.nn.Parameter(torch.randn(n, device=dev, generator=gen).to(tdt[d]))
+            p.grad = (torch.randn(n, device=dev, generator=gen) * 1e-2).to(tdt[d])
+            ps.append(p)
+        return ps
+
+    def timed(step_fn):
+        for _ in range(warmup):
+            step_fn()
+        torch.cuda.synchronize()
+        per = []
+        for _ in range(rounds):
+            t0 = time.perf_counter()
+            for _ in range(steps):
+                step_fn()
+            torch.cuda.synchronize()
+            per.append((time.perf_counter() - t0) / steps * 1e6)
+        return {"us_per_step_median": _pct(per, 0.5), "us_p10": _pct(per, 0.1), "us_p90": _pct(per, 0.9)}
+
+    res = {"mode": "eager-collection", "tensors": len(sizes), "numel": int(sum(sizes)),
+           "rounds": rounds, "steps_per_round": steps}
+    for name, cls, kw in (("AdamW32bit", optim.AdamW32bit, {}),
+                          ("AdEMAMix32bit", optim.AdEMAMix32bit, {}),
+                          ("AdamW32bit_flatten", optim.AdamW32bit, dict(flatten=True)),
+                          ("AdEMAMix32bit_flatten", optim.AdEMAMix32bit, dict(flatten=True))):
+        res[name] = timed(cls(make(), lr=1e-4, **kw).step)
+    # graph-compatible control: the AdamW32bit step captured once, replayed
+    opt = optim.AdamW32bit(make(), lr=1e-4, capturable=True, table_len=4096)
+    opt.step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        opt.step()
+    res["AdamW32bit_graph_replay"] = timed(graph.replay)
+    del graph
+    ref = torch.optim.AdamW(make(), lr=1e-4, fused=True)
+    res["torch_AdamW_fused_context"] = timed(ref.step)
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -514,6 +659,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the small-collection, e2e and cpu_baseline legs")
+    ap.add_argument("--mode", choices=["headline", "direct-cells", "eager-collection"],
+                    default="headline",
+                    help="headline: the one-line bench; the others follow the issue's "
+                         "direct-cell and eager-collection protocol and print their tables")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -523,6 +672,15 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         log(f"note: WORLD_SIZE={world}, --gpus={args.gpus}; using WORLD_SIZE")
+
+    if args.mode != "headline":
+        import torch
+        from elementwise_optimizer_b200 import _build
+        _build.build()
+        torch.cuda.set_device(local_rank)
+        res = run_direct_cells() if args.mode == "direct-cells" else run_eager_collection()
+        print(json.dumps(res), flush=True)
+        return
 
     if args.impl == "reference":
         line = run_reference(args, rank, world)

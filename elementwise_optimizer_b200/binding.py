@@ -209,10 +209,21 @@ def make_hyper(algo: str = "adam", lr: float = 1e-3, beta1: float = 0.9,
                  int(bool(skip_zeros)))
 
 
+def _current_stream_fast():
+    """Raw handle of torch's current stream on the current device.  Building
+    a torch.cuda.Stream object costs microseconds per call, so the private
+    raw-handle query is used when this torch build has it."""
+    import torch
+    get_raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    get_dev = getattr(torch._C, "_cuda_getDevice", None)
+    if get_raw is not None and get_dev is not None:
+        return int(get_raw(get_dev()))
+    return int(torch.cuda.current_stream().cuda_stream)
+
+
 def _stream_handle(stream) -> int:
     if stream is None:
-        import torch
-        return int(torch.cuda.current_stream().cuda_stream)
+        return _current_stream_fast()
     if isinstance(stream, int):
         return stream
     return int(stream.cuda_stream)

@@ -8,6 +8,14 @@ classes mirror the optimizer families of the bitsandbytes issue "Investigate
 a 256-thread SM103 path for small 32-bit optimizer tensors" (section "B300
 benchmark and acceptance": AdamW32bit and AdEMAMix32bit).
 
+flatten=True moves the parameters of each (param group, device, dtype) into
+one flat buffer (each parameter's .data becomes a view of it), points every
+.grad at a view of a matching flat gradient buffer, and keeps the state flat
+as well; step() is then one call per flat buffer with no per-parameter
+Python work, and zero_grad() zeroes the flat gradients in place (gradients
+must keep accumulating into those views: do not replace p.grad).  Results are
+the same bits as without flattening, since the update is elementwise.
+
 capturable=True routes every step through opt2s_plan_step_table: the per-step
 scalars live in a device table and the step index in device memory, so
 ``step()`` may be captured in a CUDA graph and each replay performs the next
@@ -26,7 +34,7 @@ class TwoStateOptimizer(torch.optim.Optimizer):
     def __init__(self, params, algo: str = "adamw", lr: float = 1e-3,
                  betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 0.0,
                  beta3: float = 0.9999, alpha: float = 5.0, skip_zeros: bool = False,
-                 capturable: bool = False, table_len: int = 1024):
+                 capturable: bool = False, table_len: int = 1024, flatten: bool = False):
         if algo not in B.ALGOS:
             raise ValueError(f"algo must be one of {sorted(B.ALGOS)}")
         defaults = dict(lr=lr, betas=tuple(betas), eps=eps, weight_decay=weight_decay,
@@ -36,6 +44,53 @@ class TwoStateOptimizer(torch.optim.Optimizer):
         self.table_len = int(table_len)
         super().__init__(params, defaults)
         self._group_cache = {}
+        self._flat = None
+        if flatten:
+            if capturable:
+                raise ValueError("flatten and capturable are not combined")
+            self._flatten()
+
+    # ---- flat layout ---------------------------------------------------------
+    def _flatten(self):
+        self._flat = []
+        two = self.algo == "ademamix"
+        for gi, group in enumerate(self.param_groups):
+            by_kind = {}
+            for p in group["params"]:
+                if not p.is_cuda:
+                    raise ValueError("parameters must be CUDA tensors")
+                by_kind.setdefault((p.device, p.dtype), []).append(p)
+            for (dev, dt), ps in by_kind.items():
+                n = sum(p.numel() for p in ps)
+                fp = torch.empty(n, dtype=dt, device=dev)
+                fg = torch.zeros(n, dtype=dt, device=dev)
+                fs1 = torch.zeros(2 * n if two else n, dtype=torch.float32, device=dev)
+                fs2 = torch.zeros(n, dtype=torch.float32, device=dev)
+                off = 0
+                with torch.no_grad():
+                    for p in ps:
+                        k = p.numel()
+                        fp[off:off + k].copy_(p.detach().reshape(-1))
+                        if p.grad is not None:
+                            fg[off:off + k].copy_(p.grad.detach().reshape(-1))
+                        p.data = fp[off:off + k].view_as(p)
+                        p.grad = fg[off:off + k].view_as(p)
+                        st = self.state[p]
+                        st["exp_avg"] = fs1[off:off + k].view_as(p)
+                        st["exp_avg_sq"] = fs2[off:off + k].view_as(p)
+                        if two:
+                            st["exp_avg_slow"] = fs1[n + off:n + off + k].view_as(p)
+                        st["step"] = 0
+                        off += k
+                tl = B.TensorList.from_tensors([fp], [fg], [fs1], [fs2])
+                self._flat.append(dict(group=gi, params=ps, param=fp, grad=fg, state1=fs1,
+                                       state2=fs2, plan=B.Plan(tl, self.algo), step=0))
+
+    def zero_grad(self, set_to_none: bool = True):
+        if self._flat is None:
+            return super().zero_grad(set_to_none)
+        for f in self._flat:           # keep the views: gradients accumulate into them
+            f["grad"].zero_()
 
     # ---- per-group launch data ------------------------------------------
     def _hyper(self, group):
@@ -95,6 +150,11 @@ class TwoStateOptimizer(torch.optim.Optimizer):
         if closure is not None:
             with torch.enable_grad():
                 loss = closure()
+        if self._flat is not None:
+            for f in self._flat:
+                f["plan"].step(self._hyper(self.param_groups[f["group"]]), f["step"] + 1)
+                f["step"] += 1
+            return loss
         for gi, group in enumerate(self.param_groups):
             data = self._launch_data(gi, group)
             if not data["params"]:

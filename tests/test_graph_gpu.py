@@ -189,3 +189,37 @@ def test_optimizer_capturable_graph_equals_eager():
         assert torch.equal(eager.state[a]["state1"], cap.state[b]["state1"])
         assert torch.equal(eager.state[a]["state2"], cap.state[b]["state2"])
     del graph
+
+
+@pytest.mark.parametrize("cls", [optim.AdamW32bit, optim.AdEMAMix32bit])
+def test_flattened_optimizer_equals_per_tensor_optimizer(cls):
+    """A small model trained a few steps with real backward passes: the flat
+    layout (params, grads and state in one buffer per dtype) gives the same
+    bits as the per-tensor layout."""
+    def model_params(seed):
+        gen = torch.Generator(device="cpu").manual_seed(seed)
+        shapes = [(64, 33), (33,), (33, 7), (7,), (1000,), (5, 200)]
+        dts = [torch.float32, torch.float32, torch.bfloat16, torch.bfloat16, torch.float16,
+               torch.float32]
+        return [torch.nn.Parameter(torch.randn(s, generator=gen).to(d).cuda()) for s, d in zip(shapes, dts)]
+
+    def loss_of(ps, x):
+        h = torch.tanh(x @ ps[0].float() + ps[1].float())
+        y = h @ ps[2].float() + ps[3].float()
+        return (y ** 2).mean() + (ps[4].float() ** 2).sum() * 1e-3 + ps[5].float().pow(2).mean()
+
+    pa, pb = model_params(7), model_params(7)
+    oa, ob = cls(pa, lr=1e-2), cls(pb, lr=1e-2, flatten=True)
+    gen = torch.Generator(device="cpu").manual_seed(8)
+    for _ in range(5):
+        x = torch.randn(16, 64, generator=gen).cuda()
+        for ps, o in ((pa, oa), (pb, ob)):
+            o.zero_grad()
+            loss_of(ps, x).backward()
+            o.step()
+    torch.cuda.synchronize()
+    for a, b in zip(pa, pb):
+        assert torch.equal(a.detach().view(torch.uint8), b.detach().view(torch.uint8))
+    # the flat layout really is flat: one plan per (group, dtype)
+    assert len(ob._flat) == 3
+    assert all(p.grad.data_ptr() >= f["grad"].data_ptr() for f in ob._flat for p in f["params"])
