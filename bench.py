@@ -540,7 +540,8 @@ def run_direct_cells(rounds=7, samples=200, warmup=20):
                     rp.grad = g.clone()
                     ref = torch.optim.AdamW([rp], lr=1e-3, weight_decay=0.01, fused=True)
                 cells.append(dict(algo=algo, dtype=dt, n=n, tl=tl, h=h, ref=ref, step=0,
-                                  dev=[], host=[], torch_dev=[]))
+                                  dev=[], host=[], torch_dev=[], graph=[],
+                                  plan=B.Plan(tl, algo)))
     stream = torch.cuda.current_stream()
     for c in cells:
         for _ in range(warmup):
@@ -574,9 +575,28 @@ def run_direct_cells(rounds=7, samples=200, warmup=20):
                     ev[k + 1].record(stream)
                 torch.cuda.synchronize()
                 c["torch_dev"] += [ev[k].elapsed_time(ev[k + 1]) * 1e3 for k in range(samples)]
+    # device-bound time per launch: 200 launches captured in a CUDA graph and
+    # replayed (no host dispatch between them)
+    for c in cells:
+        graph = torch.cuda.CUDAGraph()
+        c["plan"].step(c["h"], c["step"] + 1)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            for _ in range(samples):
+                c["plan"].step(c["h"], c["step"] + 1)
+        for _ in range(rounds):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+            b.synchronize()
+            c["graph"].append(a.elapsed_time(b) * 1e3 / samples)
+        del graph
     out = []
     for c in cells:
         row = {"algo": c["algo"], "dtype": c["dtype"], "n": c["n"],
+               "device_us_per_launch_graph": _pct(c["graph"], 0.5),
                "us_median": _pct(c["dev"], 0.5), "us_p10": _pct(c["dev"], 0.1),
                "us_p90": _pct(c["dev"], 0.9), "host_dispatch_us_median": _pct(c["host"], 0.5)}
         if c["torch_dev"]:
@@ -584,8 +604,10 @@ def run_direct_cells(rounds=7, samples=200, warmup=20):
         out.append(row)
     return {"mode": "direct-cells", "rounds": rounds, "samples_per_round": samples,
             "warmup": warmup, "cells": out,
-            "note": "device time per call between CUDA events on the launching stream; "
-                    "host_dispatch_us is wall time per call of back-to-back calls (ctypes included)"}
+            "note": "us_*: time per call between CUDA events around back-to-back opt2s_step "
+                    "calls from Python (bounded by host dispatch for small n); "
+                    "host_dispatch_us: wall time per call (ctypes included); "
+                    "device_us_per_launch_graph: 200 launches replayed from a CUDA graph"}
 
 
 def run_eager_collection(rounds=7, steps=50, warmup=20):

@@ -112,6 +112,11 @@ template <> struct Param<kF32> {
     __device__ static void store1(void* b, uint32_t i, float x) {
         __stcs(static_cast<float*>(b) + i, x);
     }
+    // kVec elements from an address that need not be 16-byte aligned
+    __device__ static Raw load_elems(const void* b, uint32_t i) {
+        const float* f = static_cast<const float*>(b) + i;
+        return make_float4(__ldcs(f), __ldcs(f + 1), __ldcs(f + 2), __ldcs(f + 3));
+    }
 };
 
 // Shared by the two 16-bit formats: only the conversions differ.
@@ -156,6 +161,16 @@ template <typename H2, typename Cvt> struct Param16 {
     __device__ static float load1(const void* b, uint32_t i) {
         return Cvt::to_float(__ldcs(static_cast<const unsigned short*>(b) + i));
     }
+    // kVec elements from an address that need not be 16-byte aligned
+    __device__ static Raw load_elems(const void* b, uint32_t i) {
+        const unsigned short* h = static_cast<const unsigned short*>(b) + i;
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[k] = static_cast<uint32_t>(__ldcs(h + 2 * k)) |
+                   (static_cast<uint32_t>(__ldcs(h + 2 * k + 1)) << 16);
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
     __device__ static void store1(void* b, uint32_t i, float x) {
         __stcs(static_cast<unsigned short*>(b) + i, Cvt::from_float(x));
     }
@@ -185,6 +200,30 @@ __device__ __forceinline__ void load_state(const float* b, uint32_t i, float (&x
     for (int k = 0; k < N / 4; ++k) {
         const float4 t = __ldcs(reinterpret_cast<const float4*>(b + i) + k);
         x[4 * k] = t.x; x[4 * k + 1] = t.y; x[4 * k + 2] = t.z; x[4 * k + 3] = t.w;
+    }
+}
+
+// fp32 state through 16-byte accesses when `vec`, else element by element.
+template <int N>
+__device__ __forceinline__ void load_state_any(const float* b, uint32_t i, bool vec, float (&x)[N]) {
+    if (vec) {
+        load_state<N>(b, i, x);
+    } else {
+#pragma unroll
+        for (int k = 0; k < N; ++k) x[k] = __ldcs(b + i + k);
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void store_state(float* b, uint32_t i, const float (&x)[N]);
+
+template <int N>
+__device__ __forceinline__ void store_state_any(float* b, uint32_t i, bool vec, const float (&x)[N]) {
+    if (vec) {
+        store_state<N>(b, i, x);
+    } else {
+#pragma unroll
+        for (int k = 0; k < N; ++k) __stcs(b + i + k, x[k]);
     }
 }
 
@@ -222,31 +261,26 @@ __device__ __forceinline__ bool aligned16(const void* q, uint32_t head, int byte
     return ((reinterpret_cast<uintptr_t>(q) + static_cast<uintptr_t>(head) * bytes) & 15u) == 0;
 }
 
-// One chunk, processed by one warp.  Every lane moves 8 elements per
-// iteration (two 16-byte vectors of fp32, or one of fp16/bf16), so a warp
-// iteration covers 256 contiguous elements of each array.
-template <int DT, int ALGO, bool SKIP>
-__device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& s, int lane)
+// Alignment of the arrays other than param at the vector body's start.
+struct Aligned {
+    bool g, m, v, m2;
+    __device__ bool all() const { return g && m && v && m2; }
+};
+
+// The vector body of a chunk: vectors [0, nvec) starting at element `head`,
+// at which param is 16-byte aligned.  ALL: every other array is aligned too
+// (the common case); otherwise each array uses 16-byte or element-wise
+// accesses according to its own flag.  In the aligned case every lane moves 8
+// elements per iteration (two 16-byte vectors of fp32, or one of fp16/bf16),
+// so a warp iteration covers 256 contiguous elements of each array; the mixed
+// case moves one vector per lane per iteration.
+template <int DT, int ALGO, bool SKIP, bool ALL>
+__device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars& s, int lane,
+                                            uint32_t head, uint32_t nvec, Aligned al)
 {
     using P = Param<DT>;
     constexpr int V = P::kVec;
-    constexpr int U = 8 / V;
-    const uint32_t len = c.len;
-
-    // The first element at which param is 16-byte aligned; the vector path
-    // needs every array aligned at that same element.
-    uint32_t head = static_cast<uint32_t>(
-        ((16u - (reinterpret_cast<uintptr_t>(c.p) & 15u)) & 15u) / P::kBytes);
-    const bool vec_ok = aligned16(c.g, head, P::kBytes) && aligned16(c.m, head, 4) &&
-                        aligned16(c.v, head, 4) &&
-                        (ALGO != kAdEMAMix || aligned16(c.m2, head, 4));
-    if (!vec_ok || head > len) head = len;
-    const uint32_t nvec = (len - head) / V;
-    const uint32_t body_end = head + nvec * V;
-
-    for (uint32_t i = lane; i < head; i += 32) scalar_element<DT, ALGO, SKIP>(c, i, s);
-    for (uint32_t i = body_end + lane; i < len; i += 32) scalar_element<DT, ALGO, SKIP>(c, i, s);
-
+    constexpr int U = ALL ? 8 / V : 1;   // the mixed path keeps fewer values live
     for (uint32_t v0 = 0; v0 < nvec; v0 += 32 * U) {
         typename P::Raw graw[U], praw[U];
         float m[U][V], v[U][V], m2[U][V];
@@ -256,11 +290,11 @@ __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& 
             const uint32_t vi = v0 + u * 32 + lane;
             if (vi < nvec) {
                 const uint32_t e = head + vi * V;
-                graw[u] = P::load(c.g, e);
+                graw[u] = (ALL || al.g) ? P::load(c.g, e) : P::load_elems(c.g, e);
                 praw[u] = P::load(c.p, e);
-                load_state<V>(c.m, e, m[u]);
-                load_state<V>(c.v, e, v[u]);
-                if (ALGO == kAdEMAMix) load_state<V>(c.m2, e, m2[u]);
+                load_state_any<V>(c.m, e, ALL || al.m, m[u]);
+                load_state_any<V>(c.v, e, ALL || al.v, v[u]);
+                if (ALGO == kAdEMAMix) load_state_any<V>(c.m2, e, ALL || al.m2, m2[u]);
             }
         }
 #pragma unroll
@@ -275,12 +309,37 @@ __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& 
                 for (int j = 0; j < V; ++j)
                     update<ALGO, SKIP>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s);
                 P::store(c.p, e, P::narrow(p, praw[u], g, SKIP));
-                store_state<V>(c.m, e, m[u]);
-                store_state<V>(c.v, e, v[u]);
-                if (ALGO == kAdEMAMix) store_state<V>(c.m2, e, m2[u]);
+                store_state_any<V>(c.m, e, ALL || al.m, m[u]);
+                store_state_any<V>(c.v, e, ALL || al.v, v[u]);
+                if (ALGO == kAdEMAMix) store_state_any<V>(c.m2, e, ALL || al.m2, m2[u]);
             }
         }
     }
+}
+
+// One chunk, processed by one warp: a scalar head up to the element at which
+// param is 16-byte aligned, the vector body, and a scalar tail.
+template <int DT, int ALGO, bool SKIP>
+__device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& s, int lane)
+{
+    using P = Param<DT>;
+    constexpr int V = P::kVec;
+    const uint32_t len = c.len;
+    uint32_t head = static_cast<uint32_t>(
+        ((16u - (reinterpret_cast<uintptr_t>(c.p) & 15u)) & 15u) / P::kBytes);
+    if (head > len) head = len;
+    const uint32_t nvec = (len - head) / V;
+    const uint32_t body_end = head + nvec * V;
+
+    for (uint32_t i = lane; i < head; i += 32) scalar_element<DT, ALGO, SKIP>(c, i, s);
+    for (uint32_t i = body_end + lane; i < len; i += 32) scalar_element<DT, ALGO, SKIP>(c, i, s);
+
+    const Aligned al{aligned16(c.g, head, P::kBytes), aligned16(c.m, head, 4),
+                     aligned16(c.v, head, 4), ALGO != kAdEMAMix || aligned16(c.m2, head, 4)};
+    if (al.all())
+        vector_body<DT, ALGO, SKIP, true>(c, s, lane, head, nvec, al);
+    else
+        vector_body<DT, ALGO, SKIP, false>(c, s, lane, head, nvec, al);
 }
 
 // ---------------------------------------------------------------------------

@@ -193,6 +193,55 @@ def test_misaligned_storage_is_bitwise_identical(layout, pad):
     _assert_same(ref, got)
 
 
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_arrays_at_different_alignments(algo, dtype):
+    """Param, grad, m and v each start at a different 16-byte phase (and
+    AdEMAMix sizes are odd, so m2 = state1 + n is misaligned too): the vector
+    body must still run, with the same bits as the aligned layout and the
+    oracle."""
+    import oracle
+    dev = torch.device("cuda")
+    sizes = [1, 7, 255, 1023, 1025, 4097, 100_003]
+    es = 4 if dtype == "f32" else 2
+    two = algo == "ademamix"
+    hyper = dict(synth.ADEMAMIX_HYPER if two else synth.ADAM_HYPER, weight_decay=0.01)
+    h = B.make_hyper(algo, **hyper)
+    for n in sizes:
+        pv = synth.normal(synth.SEED_BASE + 70, (n,), n, 1.0)
+        gv = synth.mixed_magnitude(synth.SEED_BASE + 71, (n,), n, zero_frac=0.0)
+        # misaligned buffers: element offsets 0 (p), 1 (g), 2 (m), 3 (v)
+        pb = to_device_storage(np.concatenate([np.zeros(0, np.float32), pv]), dtype, dev)
+        gb = to_device_storage(np.concatenate([np.zeros(1, np.float32), gv]), dtype, dev)
+        mb = torch.zeros((2 * n if two else n) + 2, device=dev)
+        vb = torch.zeros(n + 3, device=dev)
+        rec = [(pb.data_ptr(), gb.data_ptr() + es, mb.data_ptr() + 8, vb.data_ptr() + 12, n,
+                B.DTYPES[dtype])]
+        # aligned twin
+        pa = to_device_storage(pv, dtype, dev)
+        ga = to_device_storage(gv, dtype, dev)
+        ma = torch.zeros(2 * n if two else n, device=dev)
+        va = torch.zeros(n, device=dev)
+        twin = B.TensorList.from_tensors([pa], [ga], [ma], [va])
+        hp = synth.to_storage(pv, dtype)
+        hg = synth.to_storage(gv, dtype)
+        hs1 = np.zeros(2 * n if two else n, np.float32)
+        hs2 = np.zeros(n, np.float32)
+        for t in (1, 2, 3):
+            B.opt2s_step(B.TensorList(rec), h, t)
+            B.opt2s_step(twin, h, t)
+            oracle.step_f32(hp, hg, hs1, hs2, dtype=dtype, algo=algo, step=t, **hyper)
+        torch.cuda.synchronize()
+        got_p = storage_bits(pb)
+        got_m = storage_bits(mb)[2:]
+        got_v = storage_bits(vb)[3:]
+        assert np.array_equal(got_p, storage_bits(pa)), n
+        assert np.array_equal(got_m, storage_bits(ma)) and np.array_equal(got_v, storage_bits(va)), n
+        assert np.array_equal(got_p, hp.view(got_p.dtype)), n
+        assert np.array_equal(got_m, hs1.view(np.uint32)) and np.array_equal(got_v, hs2.view(np.uint32)), n
+        assert np.array_equal(storage_bits(gb)[1:], hg.view(got_p.dtype)), n
+
+
 def test_misaligned_storage_matches_oracle():
     h = Harness(_geometry_workload(), layout="padded", pad=3)
     run(h, 3, checkpoints=(1, 2, 3))
