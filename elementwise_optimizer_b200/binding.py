@@ -114,6 +114,7 @@ EXPORTS = {
     "opt2s_testing_set_launch": (ctypes.c_int, [ctypes.c_int, ctypes.c_int]),
     "opt2s_testing_default_chunk_elems": (ctypes.c_int64, []),
     "opt2s_testing_launch_count": (ctypes.c_int64, []),
+    "opt2s_testing_fail_allocs": (ctypes.c_int, [ctypes.c_int]),
     "opt2s_testing_choose_chunk_elems": (ctypes.c_int64, [ctypes.POINTER(TensorListDesc),
                                                           ctypes.c_int64]),
     "opt2s_testing_check_division": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int32,
@@ -368,6 +369,10 @@ def testing_check_division(seed: int, n: int, mode: int) -> int:
 
 def testing_choose_chunk_elems(tl: TensorList, resident_warps: int) -> int:
     return int(lib().opt2s_testing_choose_chunk_elems(ctypes.byref(tl.desc), int(resident_warps)))
+
+
+def testing_fail_allocs(count: int) -> None:
+    check(lib().opt2s_testing_fail_allocs(int(count)), "testing_fail_allocs")
 
 
 def launch_count() -> int:

@@ -46,6 +46,7 @@ int64_t g_chunk_elems = 0;     // testing override (0 = default)
 int g_block_threads = 0;       // testing override (0 = default)
 int g_max_blocks = 0;          // testing override (0 = occupancy cap)
 std::atomic<int64_t> g_launches{0};   // kernels launched by this library
+std::atomic<int> g_fail_allocs{0};    // testing: plan allocations to fail
 
 int cuda_fail(cudaError_t e)
 {
@@ -217,7 +218,10 @@ int plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out)
     if (!plan) return OPT2S_ERR_NO_MEMORY;
     if (!table.empty()) {
         const size_t bytes = table.size() * sizeof(ChunkRec);
-        e = cudaMalloc(&plan->d_chunks, bytes);
+        if (g_fail_allocs.load() > 0 && g_fail_allocs.fetch_sub(1) > 0)
+            e = cudaErrorMemoryAllocation;            // injected by the test scaffolding
+        else
+            e = cudaMalloc(&plan->d_chunks, bytes);
         if (e != cudaSuccess) {
             delete plan;
             if (e == cudaErrorMemoryAllocation) { t_last_cuda_error = e; return OPT2S_ERR_NO_MEMORY; }
@@ -628,6 +632,13 @@ OPT2S_API int64_t opt2s_testing_choose_chunk_elems(const TensorListDesc* desc, i
 {
     if (!desc || desc->count < 0 || (desc->count > 0 && !desc->tensors)) return OPT2S_ERR_INVALID_ARG;
     return choose_chunk_elems(desc, resident_warps);
+}
+
+OPT2S_API int opt2s_testing_fail_allocs(int count)
+{
+    if (count < 0) return OPT2S_ERR_INVALID_ARG;
+    g_fail_allocs.store(count);
+    return OPT2S_OK;
 }
 
 OPT2S_API int64_t opt2s_testing_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

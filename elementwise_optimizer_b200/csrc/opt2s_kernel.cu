@@ -33,6 +33,15 @@
 namespace opt2s {
 namespace {
 
+// Global loads and stores with the default cache policy.  Every byte of a
+// step is touched once, but measured on B200 the default (evict-normal)
+// policy streams this read-modify-write pattern about 1% faster than the
+// evict-first hints of ld/st.global.cs.
+template <typename T>
+__device__ __forceinline__ T ld_global(const T* p) { return *p; }
+template <typename T>
+__device__ __forceinline__ void st_global(T* p, const T& v) { *p = v; }
+
 // ---------------------------------------------------------------------------
 // Exact division by a per-launch constant.
 //
@@ -84,8 +93,6 @@ __device__ __forceinline__ void update(float g, float& p, float& m, float& v,
 
 // ---------------------------------------------------------------------------
 // Storage traits of param / grad.  kVec elements make one 16-byte access.
-// Loads and stores use the streaming (evict-first) cache policy: every byte is
-// touched exactly once per step.
 // ---------------------------------------------------------------------------
 template <int DT> struct Param;
 
@@ -94,10 +101,10 @@ template <> struct Param<kF32> {
     static constexpr int kBytes = 4;
     using Raw = float4;
     __device__ static Raw load(const void* b, uint32_t i) {
-        return __ldcs(reinterpret_cast<const float4*>(static_cast<const float*>(b) + i));
+        return ld_global(reinterpret_cast<const float4*>(static_cast<const float*>(b) + i));
     }
     __device__ static void store(void* b, uint32_t i, const Raw& r) {
-        __stcs(reinterpret_cast<float4*>(static_cast<float*>(b) + i), r);
+        st_global(reinterpret_cast<float4*>(static_cast<float*>(b) + i), r);
     }
     __device__ static void widen(const Raw& r, float (&x)[4]) {
         x[0] = r.x; x[1] = r.y; x[2] = r.z; x[3] = r.w;
@@ -107,15 +114,15 @@ template <> struct Param<kF32> {
         return make_float4(x[0], x[1], x[2], x[3]);
     }
     __device__ static float load1(const void* b, uint32_t i) {
-        return __ldcs(static_cast<const float*>(b) + i);
+        return ld_global(static_cast<const float*>(b) + i);
     }
     __device__ static void store1(void* b, uint32_t i, float x) {
-        __stcs(static_cast<float*>(b) + i, x);
+        st_global(static_cast<float*>(b) + i, x);
     }
     // kVec elements from an address that need not be 16-byte aligned
     __device__ static Raw load_elems(const void* b, uint32_t i) {
         const float* f = static_cast<const float*>(b) + i;
-        return make_float4(__ldcs(f), __ldcs(f + 1), __ldcs(f + 2), __ldcs(f + 3));
+        return make_float4(ld_global(f), ld_global(f + 1), ld_global(f + 2), ld_global(f + 3));
     }
 };
 
@@ -125,10 +132,10 @@ template <typename H2, typename Cvt> struct Param16 {
     static constexpr int kBytes = 2;
     using Raw = uint4;
     __device__ static Raw load(const void* b, uint32_t i) {
-        return __ldcs(reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(b) + i));
+        return ld_global(reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(b) + i));
     }
     __device__ static void store(void* b, uint32_t i, const Raw& r) {
-        __stcs(reinterpret_cast<uint4*>(static_cast<unsigned short*>(b) + i), r);
+        st_global(reinterpret_cast<uint4*>(static_cast<unsigned short*>(b) + i), r);
     }
     __device__ static void widen(const Raw& r, float (&x)[8]) {
         const H2* h = reinterpret_cast<const H2*>(&r);
@@ -159,7 +166,7 @@ template <typename H2, typename Cvt> struct Param16 {
         return r;
     }
     __device__ static float load1(const void* b, uint32_t i) {
-        return Cvt::to_float(__ldcs(static_cast<const unsigned short*>(b) + i));
+        return Cvt::to_float(ld_global(static_cast<const unsigned short*>(b) + i));
     }
     // kVec elements from an address that need not be 16-byte aligned
     __device__ static Raw load_elems(const void* b, uint32_t i) {
@@ -167,12 +174,12 @@ template <typename H2, typename Cvt> struct Param16 {
         uint32_t w[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            w[k] = static_cast<uint32_t>(__ldcs(h + 2 * k)) |
-                   (static_cast<uint32_t>(__ldcs(h + 2 * k + 1)) << 16);
+            w[k] = static_cast<uint32_t>(ld_global(h + 2 * k)) |
+                   (static_cast<uint32_t>(ld_global(h + 2 * k + 1)) << 16);
         return make_uint4(w[0], w[1], w[2], w[3]);
     }
     __device__ static void store1(void* b, uint32_t i, float x) {
-        __stcs(static_cast<unsigned short*>(b) + i, Cvt::from_float(x));
+        st_global(static_cast<unsigned short*>(b) + i, Cvt::from_float(x));
     }
 };
 
@@ -198,7 +205,7 @@ template <int N>
 __device__ __forceinline__ void load_state(const float* b, uint32_t i, float (&x)[N]) {
 #pragma unroll
     for (int k = 0; k < N / 4; ++k) {
-        const float4 t = __ldcs(reinterpret_cast<const float4*>(b + i) + k);
+        const float4 t = ld_global(reinterpret_cast<const float4*>(b + i) + k);
         x[4 * k] = t.x; x[4 * k + 1] = t.y; x[4 * k + 2] = t.z; x[4 * k + 3] = t.w;
     }
 }
@@ -210,7 +217,7 @@ __device__ __forceinline__ void load_state_any(const float* b, uint32_t i, bool 
         load_state<N>(b, i, x);
     } else {
 #pragma unroll
-        for (int k = 0; k < N; ++k) x[k] = __ldcs(b + i + k);
+        for (int k = 0; k < N; ++k) x[k] = ld_global(b + i + k);
     }
 }
 
@@ -223,7 +230,7 @@ __device__ __forceinline__ void store_state_any(float* b, uint32_t i, bool vec, 
         store_state<N>(b, i, x);
     } else {
 #pragma unroll
-        for (int k = 0; k < N; ++k) __stcs(b + i + k, x[k]);
+        for (int k = 0; k < N; ++k) st_global(b + i + k, x[k]);
     }
 }
 
@@ -231,7 +238,7 @@ template <int N>
 __device__ __forceinline__ void store_state(float* b, uint32_t i, const float (&x)[N]) {
 #pragma unroll
     for (int k = 0; k < N / 4; ++k)
-        __stcs(reinterpret_cast<float4*>(b + i) + k,
+        st_global(reinterpret_cast<float4*>(b + i) + k,
                make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]));
 }
 
@@ -246,15 +253,15 @@ __device__ __forceinline__ void scalar_element(const ChunkRec& c, uint32_t i,
     const float g = P::load1(c.g, i);
     if (SKIP && g == 0.0f) return;
     float p = P::load1(c.p, i);
-    float m = __ldcs(c.m + i);
-    float v = __ldcs(c.v + i);
+    float m = ld_global(c.m + i);
+    float v = ld_global(c.v + i);
     float m2 = 0.0f;
-    if (ALGO == kAdEMAMix) m2 = __ldcs(c.m2 + i);
+    if (ALGO == kAdEMAMix) m2 = ld_global(c.m2 + i);
     update<ALGO, false>(g, p, m, v, m2, s);
     P::store1(c.p, i, p);
-    __stcs(c.m + i, m);
-    __stcs(c.v + i, v);
-    if (ALGO == kAdEMAMix) __stcs(c.m2 + i, m2);
+    st_global(c.m + i, m);
+    st_global(c.v + i, v);
+    if (ALGO == kAdEMAMix) st_global(c.m2 + i, m2);
 }
 
 __device__ __forceinline__ bool aligned16(const void* q, uint32_t head, int bytes) {
@@ -367,17 +374,17 @@ __device__ __forceinline__ void shard_scalar(const ShardArgs& a, int64_t k, cons
     g = __fdiv_rn(g, static_cast<float>(a.world));
     if (SKIP && g == 0.0f) return;
     float p = P::load1(static_cast<const char*>(a.params[a.rank]) + e * B, 0);
-    float m = __ldcs(a.m + k);
-    float v = __ldcs(a.v + k);
+    float m = ld_global(a.m + k);
+    float v = ld_global(a.v + k);
     float m2 = 0.0f;
-    if (ALGO == kAdEMAMix) m2 = __ldcs(a.m2 + k);
+    if (ALGO == kAdEMAMix) m2 = ld_global(a.m2 + k);
     update<ALGO, false>(g, p, m, v, m2, s);
 #pragma unroll
     for (int q = 0; q < kMaxWorld; ++q)
         if (q < a.world) P::store1(static_cast<char*>(a.params[q]) + e * B, 0, p);
-    __stcs(a.m + k, m);
-    __stcs(a.v + k, v);
-    if (ALGO == kAdEMAMix) __stcs(a.m2 + k, m2);
+    st_global(a.m + k, m);
+    st_global(a.v + k, v);
+    if (ALGO == kAdEMAMix) st_global(a.m2 + k, m2);
 }
 
 // Elements [k0, k0 + len) of the shard (shard-relative), one warp.

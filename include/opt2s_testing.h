@@ -79,6 +79,10 @@ int64_t opt2s_testing_choose_chunk_elems(const TensorListDesc *desc, int64_t res
  * *mismatches.  Synchronous; allocates a counter on the device. */
 int opt2s_testing_check_division(uint64_t seed, int64_t n, int32_t mode, int64_t *mismatches);
 
+/* Fault injection on the host: the next `count` device allocations of plan
+ * creation fail as if the device were out of memory (OPT2S_ERR_NO_MEMORY). */
+int opt2s_testing_fail_allocs(int count);
+
 /* Number of kernels this library has launched in this process. */
 int64_t opt2s_testing_launch_count(void);
 
