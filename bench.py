@@ -667,6 +667,49 @@ def run_eager_collection(rounds=7, steps=50, warmup=20):
     return res
 
 
+def run_shard_emulated(numel=268_435_456, worlds=(1, 2, 4, 8), steps=20, warmup=5):
+    """The fused sharded step with `world` emulated ranks on one GPU: every
+    rank's param and grad buffer lives on this device, and one step is the
+    world ranks' launches one after another.  Per element of the collection
+    the step reads world gradients, the param and the fp32 state, and writes
+    world params and the state: (8*world + 20) bytes for fp32 Adam.  On a real
+    node the (world-1)/world remote share of those bytes crosses NVLink."""
+    import torch
+    from elementwise_optimizer_b200 import binding as B
+    from elementwise_optimizer_b200 import shard
+    dev = torch.device("cuda")
+    peak, _ = measured_peak()
+    res = {"mode": "shard-emulated", "numel": numel, "algo": "adam", "dtype": "f32", "rows": []}
+    h = B.make_hyper("adam")
+    for world in worlds:
+        params = [torch.randn(numel, device=dev) for _ in range(world)]
+        grads = [torch.randn(numel, device=dev) * 1e-2 for _ in range(world)]
+        steppers = [shard.ShardedStep(params, grads, r, "adam") for r in range(world)]
+        t = 0
+        for _ in range(warmup):
+            t += 1
+            for st in steppers:
+                st.step(h, t)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            t += 1
+            for st in steppers:
+                st.step(h, t)
+        b.record()
+        b.synchronize()
+        ms = a.elapsed_time(b) / steps
+        nbytes = (8 * world + 20) * numel
+        res["rows"].append({"world": world, "ms_per_step": ms, "algorithmic_bytes": nbytes,
+                            "gbs": nbytes / (ms / 1e3) / 1e9,
+                            "frac_of_hbm_peak": nbytes / (ms / 1e3) / 1e9 / peak})
+        del params, grads, steppers
+        torch.cuda.empty_cache()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -681,7 +724,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the small-collection, e2e and cpu_baseline legs")
-    ap.add_argument("--mode", choices=["headline", "direct-cells", "eager-collection"],
+    ap.add_argument("--mode", choices=["headline", "direct-cells", "eager-collection",
+                                       "shard-emulated"],
                     default="headline",
                     help="headline: the one-line bench; the others follow the issue's "
                          "direct-cell and eager-collection protocol and print their tables")
@@ -700,7 +744,8 @@ def main():
         from elementwise_optimizer_b200 import _build
         _build.build()
         torch.cuda.set_device(local_rank)
-        res = run_direct_cells() if args.mode == "direct-cells" else run_eager_collection()
+        res = {"direct-cells": run_direct_cells, "eager-collection": run_eager_collection,
+               "shard-emulated": run_shard_emulated}[args.mode]()
         print(json.dumps(res), flush=True)
         return
 
