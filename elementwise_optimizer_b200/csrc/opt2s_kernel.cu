@@ -361,7 +361,7 @@ __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& 
 // final before, params read after).  Peer buffers are reached with ordinary
 // loads and stores (NVLink on a multi-GPU node; no TMA, no multicast).
 // ---------------------------------------------------------------------------
-template <int DT, int ALGO, bool SKIP>
+template <int DT, int ALGO, bool SKIP, int W>
 __device__ __forceinline__ void shard_scalar(const ShardArgs& a, int64_t k, const StepScalars& s)
 {
     using P = Param<DT>;
@@ -369,9 +369,9 @@ __device__ __forceinline__ void shard_scalar(const ShardArgs& a, int64_t k, cons
     constexpr int B = P::kBytes;
     float g = P::load1(static_cast<const char*>(a.grads[0]) + e * B, 0);
 #pragma unroll
-    for (int q = 1; q < kMaxWorld; ++q)
-        if (q < a.world) g = __fadd_rn(g, P::load1(static_cast<const char*>(a.grads[q]) + e * B, 0));
-    g = __fdiv_rn(g, static_cast<float>(a.world));
+    for (int q = 1; q < W; ++q)
+        g = __fadd_rn(g, P::load1(static_cast<const char*>(a.grads[q]) + e * B, 0));
+    g = __fdiv_rn(g, static_cast<float>(W));
     if (SKIP && g == 0.0f) return;
     float p = P::load1(static_cast<const char*>(a.params[a.rank]) + e * B, 0);
     float m = ld_global(a.m + k);
@@ -380,20 +380,21 @@ __device__ __forceinline__ void shard_scalar(const ShardArgs& a, int64_t k, cons
     if (ALGO == kAdEMAMix) m2 = ld_global(a.m2 + k);
     update<ALGO, false>(g, p, m, v, m2, s);
 #pragma unroll
-    for (int q = 0; q < kMaxWorld; ++q)
-        if (q < a.world) P::store1(static_cast<char*>(a.params[q]) + e * B, 0, p);
+    for (int q = 0; q < W; ++q) P::store1(static_cast<char*>(a.params[q]) + e * B, 0, p);
     st_global(a.m + k, m);
     st_global(a.v + k, v);
     if (ALGO == kAdEMAMix) st_global(a.m2 + k, m2);
 }
 
-// Elements [k0, k0 + len) of the shard (shard-relative), one warp.
-template <int DT, int ALGO, bool SKIP>
+// Elements [k0, k0 + len) of the shard (shard-relative), one warp; W ranks.
+// Like the plain step's vector body, each lane moves 8 elements per iteration.
+template <int DT, int ALGO, bool SKIP, int W>
 __device__ __forceinline__ void shard_chunk(const ShardArgs& a, int64_t k0, uint32_t len,
                                             const StepScalars& s, int lane)
 {
     using P = Param<DT>;
     constexpr int V = P::kVec;
+    constexpr int U = 8 / V;
     constexpr int B = P::kBytes;
     const int64_t e0 = a.shard_start + k0;
     const char* own = static_cast<const char*>(a.params[a.rank]) + e0 * B;
@@ -401,57 +402,69 @@ __device__ __forceinline__ void shard_chunk(const ShardArgs& a, int64_t k0, uint
     bool vec_ok = aligned16(a.m + k0, head, 4) && aligned16(a.v + k0, head, 4) &&
                   (ALGO != kAdEMAMix || aligned16(a.m2 + k0, head, 4));
 #pragma unroll
-    for (int q = 0; q < kMaxWorld; ++q)
-        if (q < a.world)
-            vec_ok = vec_ok && aligned16(static_cast<const char*>(a.params[q]) + e0 * B, head, B) &&
-                     aligned16(static_cast<const char*>(a.grads[q]) + e0 * B, head, B);
+    for (int q = 0; q < W; ++q)
+        vec_ok = vec_ok && aligned16(static_cast<const char*>(a.params[q]) + e0 * B, head, B) &&
+                 aligned16(static_cast<const char*>(a.grads[q]) + e0 * B, head, B);
     if (!vec_ok || head > len) head = len;
     const uint32_t nvec = (len - head) / V;
     const uint32_t body_end = head + nvec * V;
-    for (uint32_t i = lane; i < head; i += 32) shard_scalar<DT, ALGO, SKIP>(a, k0 + i, s);
-    for (uint32_t i = body_end + lane; i < len; i += 32) shard_scalar<DT, ALGO, SKIP>(a, k0 + i, s);
+    for (uint32_t i = lane; i < head; i += 32) shard_scalar<DT, ALGO, SKIP, W>(a, k0 + i, s);
+    for (uint32_t i = body_end + lane; i < len; i += 32) shard_scalar<DT, ALGO, SKIP, W>(a, k0 + i, s);
 
-    const float world = static_cast<float>(a.world);
-    for (uint32_t vi = lane; vi < nvec; vi += 32) {
-        const uint32_t i = head + vi * V;          // chunk-relative element
-        const int64_t k = k0 + i;                  // shard-relative element
-        const int64_t e = e0 + i;                  // flat element
-        typename P::Raw graw[kMaxWorld];
+    for (uint32_t v0 = 0; v0 < nvec; v0 += 32 * U) {
+        typename P::Raw graw[U][W], praw[U];
+        float m[U][V], v[U][V], m2[U][V];
 #pragma unroll
-        for (int q = 0; q < kMaxWorld; ++q)
-            if (q < a.world) graw[q] = P::load(static_cast<const char*>(a.grads[q]) + e * B, 0);
-        const typename P::Raw praw = P::load(static_cast<const char*>(a.params[a.rank]) + e * B, 0);
-        float m[V], v[V], m2[V], g[V], p[V];
-        P::widen(graw[0], g);
-        P::widen(praw, p);
-        load_state<V>(a.m + k, 0, m);
-        load_state<V>(a.v + k, 0, v);
-        if (ALGO == kAdEMAMix) load_state<V>(a.m2 + k, 0, m2);
+        for (int u = 0; u < U; ++u) {
+            const uint32_t vi = v0 + u * 32 + lane;
+            if (vi < nvec) {
+                const uint32_t i = head + vi * V;      // chunk-relative element
+                const int64_t k = k0 + i;              // shard-relative element
+                const int64_t e = e0 + i;              // flat element
 #pragma unroll
-        for (int q = 1; q < kMaxWorld; ++q) {
-            if (q < a.world) {
-                float x[V];
-                P::widen(graw[q], x);
-#pragma unroll
-                for (int j = 0; j < V; ++j) g[j] = __fadd_rn(g[j], x[j]);
+                for (int q = 0; q < W; ++q)
+                    graw[u][q] = P::load(static_cast<const char*>(a.grads[q]) + e * B, 0);
+                praw[u] = P::load(static_cast<const char*>(a.params[a.rank]) + e * B, 0);
+                load_state<V>(a.m + k, 0, m[u]);
+                load_state<V>(a.v + k, 0, v[u]);
+                if (ALGO == kAdEMAMix) load_state<V>(a.m2 + k, 0, m2[u]);
             }
         }
 #pragma unroll
-        for (int j = 0; j < V; ++j) {
-            g[j] = __fdiv_rn(g[j], world);
-            update<ALGO, SKIP>(g[j], p[j], m[j], v[j], m2[j], s);
-        }
-        const typename P::Raw out = P::narrow(p, praw, g, SKIP);
+        for (int u = 0; u < U; ++u) {
+            const uint32_t vi = v0 + u * 32 + lane;
+            if (vi < nvec) {
+                const uint32_t i = head + vi * V;
+                const int64_t k = k0 + i;
+                const int64_t e = e0 + i;
+                float g[V], p[V];
+                P::widen(graw[u][0], g);
+                P::widen(praw[u], p);
 #pragma unroll
-        for (int q = 0; q < kMaxWorld; ++q)
-            if (q < a.world) P::store(static_cast<char*>(a.params[q]) + e * B, 0, out);
-        store_state<V>(a.m + k, 0, m);
-        store_state<V>(a.v + k, 0, v);
-        if (ALGO == kAdEMAMix) store_state<V>(a.m2 + k, 0, m2);
+                for (int q = 1; q < W; ++q) {
+                    float x[V];
+                    P::widen(graw[u][q], x);
+#pragma unroll
+                    for (int j = 0; j < V; ++j) g[j] = __fadd_rn(g[j], x[j]);
+                }
+#pragma unroll
+                for (int j = 0; j < V; ++j) {
+                    g[j] = __fdiv_rn(g[j], static_cast<float>(W));
+                    update<ALGO, SKIP>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s);
+                }
+                const typename P::Raw out = P::narrow(p, praw[u], g, SKIP);
+#pragma unroll
+                for (int q = 0; q < W; ++q)
+                    P::store(static_cast<char*>(a.params[q]) + e * B, 0, out);
+                store_state<V>(a.m + k, 0, m[u]);
+                store_state<V>(a.v + k, 0, v[u]);
+                if (ALGO == kAdEMAMix) store_state<V>(a.m2 + k, 0, m2[u]);
+            }
+        }
     }
 }
 
-template <int ALGO, bool SKIP>
+template <int ALGO, bool SKIP, int W>
 __global__ void shard_step_kernel(ShardArgs a, StepScalars s)
 {
     const int lane = threadIdx.x & 31;
@@ -464,11 +477,35 @@ __global__ void shard_step_kernel(ShardArgs a, StepScalars s)
         const int64_t k0 = c * ce;
         const uint32_t len = static_cast<uint32_t>(min(ce, a.shard_len - k0));
         switch (a.dtype) {
-        case kF32: shard_chunk<kF32, ALGO, SKIP>(a, k0, len, s, lane); break;
-        case kF16: shard_chunk<kF16, ALGO, SKIP>(a, k0, len, s, lane); break;
-        default: shard_chunk<kBF16, ALGO, SKIP>(a, k0, len, s, lane); break;
+        case kF32: shard_chunk<kF32, ALGO, SKIP, W>(a, k0, len, s, lane); break;
+        case kF16: shard_chunk<kF16, ALGO, SKIP, W>(a, k0, len, s, lane); break;
+        default: shard_chunk<kBF16, ALGO, SKIP, W>(a, k0, len, s, lane); break;
         }
     }
+}
+
+using ShardFn = void (*)(ShardArgs, StepScalars);
+
+template <int ALGO, bool SKIP>
+ShardFn pick_shard_w(int world)
+{
+    switch (world) {
+    case 1: return shard_step_kernel<ALGO, SKIP, 1>;
+    case 2: return shard_step_kernel<ALGO, SKIP, 2>;
+    case 3: return shard_step_kernel<ALGO, SKIP, 3>;
+    case 4: return shard_step_kernel<ALGO, SKIP, 4>;
+    case 5: return shard_step_kernel<ALGO, SKIP, 5>;
+    case 6: return shard_step_kernel<ALGO, SKIP, 6>;
+    case 7: return shard_step_kernel<ALGO, SKIP, 7>;
+    default: return shard_step_kernel<ALGO, SKIP, 8>;
+    }
+}
+
+ShardFn pick_shard(int algo, int skip, int world)
+{
+    if (algo == kAdEMAMix)
+        return skip ? pick_shard_w<kAdEMAMix, true>(world) : pick_shard_w<kAdEMAMix, false>(world);
+    return skip ? pick_shard_w<kAdam, true>(world) : pick_shard_w<kAdam, false>(world);
 }
 
 // The whole step: warp w takes chunks w, w + W, w + 2W, ... of the table.
@@ -684,10 +721,7 @@ cudaError_t launch_shard_step(const ShardArgs& a, int algo, int skip_zeros, cons
                               int block_threads, cudaStream_t stream)
 {
     if (a.shard_len <= 0) return cudaSuccess;
-    using ShardFn = void (*)(ShardArgs, StepScalars);
-    ShardFn fn = algo == kAdEMAMix
-                     ? (skip_zeros ? shard_step_kernel<kAdEMAMix, true> : shard_step_kernel<kAdEMAMix, false>)
-                     : (skip_zeros ? shard_step_kernel<kAdam, true> : shard_step_kernel<kAdam, false>);
+    ShardFn fn = pick_shard(algo, skip_zeros, a.world);
     int dev = 0, sms = 0, per_sm = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
