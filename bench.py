@@ -155,6 +155,17 @@ def traffic_for(kernel_key):
     return None
 
 
+def max_over_ranks(value, device=None):
+    """The largest `value` over all ranks of the default process group (the
+    slowest rank's time); one all-reduce of a scalar, no data-path traffic."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def make_device_workload(w, device, n_grad_buffers):
     """Allocate param / grads / states for workload w on `device` and fill
     them with seeded synthetic values (made on the device: this is bench
@@ -335,10 +346,7 @@ def run_ours(args, rank, world, local_rank):
     per_launch_ms = [events[k].elapsed_time(events[k + 1]) for k in range(args.steps)]
     total_ms = events[0].elapsed_time(events[-1])
     if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(total_ms, device)
 
     extras = {}
     if rank == 0 and world == 1 and not args.no_extras:
