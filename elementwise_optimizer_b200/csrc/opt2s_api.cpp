@@ -54,9 +54,12 @@ int cuda_fail(cudaError_t e)
     return OPT2S_ERR_CUDA;
 }
 
-int block_threads_now() { return g_block_threads > 0 ? g_block_threads : opt2s::kDefaultBlockThreads; }
+int block_threads_now(int algo)
+{
+    return g_block_threads > 0 ? g_block_threads : opt2s::default_block_threads(algo);
+}
 
-// Chunk length for a collection: the multiple of 256 elements in
+// Chunk length for a collection: the power-of-two multiple of 256 elements in
 // [kMinChunkElems, kDefaultChunkElems] that minimizes the modelled time of the
 // slowest warp.  A warp handles ceil(chunks / resident_warps) chunks one after
 // the other; a chunk of c elements costs ceil(c / 256) dependent iterations
@@ -82,7 +85,7 @@ int64_t chunk_elems_for(const TensorListDesc* d, int32_t algo)
 {
     if (g_chunk_elems > 0) return g_chunk_elems;
     int64_t warps = 0;
-    if (opt2s::resident_warps(algo, 0, block_threads_now(), &warps) != cudaSuccess)
+    if (opt2s::resident_warps(algo, 0, block_threads_now(algo), &warps) != cudaSuccess)
         return opt2s::kDefaultChunkElems;
     return choose_chunk_elems(d, warps);
 }
@@ -283,8 +286,8 @@ int plan_step(const opt2s_plan* plan, const Hyper* h, int step, cudaStream_t str
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev != plan->device) return OPT2S_ERR_DEVICE;
-    const int bt = block_threads_now();
-    if (bt != opt2s::kDefaultBlockThreads) {   // forced geometry: must fit the kernel
+    const int bt = block_threads_now(h->algo);
+    if (g_block_threads > 0) {   // forced geometry: must fit the kernel
         int widest = 0;
         e = opt2s::max_block_threads(h->algo, h->skip_zeros, &widest);
         if (e != cudaSuccess) return cuda_fail(e);
@@ -429,8 +432,8 @@ OPT2S_API int opt2s_plan_step_table(const opt2s_plan* plan, int32_t skip_zeros,
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev != plan->device) return OPT2S_ERR_DEVICE;
-    const int bt = block_threads_now();
-    if (bt != opt2s::kDefaultBlockThreads) {
+    const int bt = block_threads_now(plan->algo);
+    if (g_block_threads > 0) {
         int widest = 0;
         e = opt2s::max_block_threads(plan->algo, skip_zeros, &widest);
         if (e != cudaSuccess) return cuda_fail(e);
@@ -515,7 +518,8 @@ OPT2S_API int opt2s_shard_step(const opt2s_shard_desc* d, const Hyper* hyper, in
     a.dtype = d->dtype;
     a.chunk_elems = static_cast<int32_t>(g_chunk_elems > 0 ? g_chunk_elems : opt2s::kDefaultChunkElems);
     cudaError_t e = opt2s::launch_shard_step(a, hyper->algo, hyper->skip_zeros, make_scalars(hyper, step),
-                                             block_threads_now(), stream);
+                                             g_block_threads > 0 ? g_block_threads : opt2s::kAdamBlockThreads,
+                                             stream);
     if (e != cudaSuccess) return cuda_fail(e);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return OPT2S_OK;

@@ -40,8 +40,15 @@ struct StepScalars {
     double inv_bc1, inv_bc2;
 };
 
-constexpr int kDefaultBlockThreads = 128;
-constexpr int64_t kDefaultChunkElems = 4096;   // largest chunk the plan builder picks
+// Threads per block by algorithm.  Adam's kernel (96 registers) fits 20
+// resident warps per SM as 128-thread blocks (16 as 256-thread blocks);
+// AdEMAMix's (120 registers) fits 16 warps either way, and measured faster as
+// 256-thread blocks.
+constexpr int kAdamBlockThreads = 128;
+constexpr int kAdEMAMixBlockThreads = 256;
+constexpr int kDefaultBlockThreads = 128;      // the no-alloc entry point's width
+inline int default_block_threads(int algo) { return algo == kAdEMAMix ? kAdEMAMixBlockThreads : kAdamBlockThreads; }
+constexpr int64_t kDefaultChunkElems = 2048;   // largest chunk the plan builder picks
 constexpr int64_t kMinChunkElems = 256;        // one warp iteration (8 elements per lane)
 
 // The sharded (ZeRO-style) step of one rank.  Every rank holds the whole flat

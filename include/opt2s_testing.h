@@ -68,7 +68,7 @@ int64_t opt2s_testing_default_chunk_elems(void);
 
 /* Host only: the chunk length a plan for `desc` gets on a device with
  * `resident_warps` resident warps of the step kernel: the multiple of 256 in
- * [256, 4096] minimizing ceil(chunks / resident_warps) * (length / 256 + 1),
+ * [256, 2048] minimizing ceil(chunks / resident_warps) * (length / 256 + 1),
  * the modelled time of the slowest warp. */
 int64_t opt2s_testing_choose_chunk_elems(const TensorListDesc *desc, int64_t resident_warps);
 

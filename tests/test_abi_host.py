@@ -332,20 +332,20 @@ def test_step_scalar_table_rejects_bad_arguments(L):
 
 
 def test_chunk_length_follows_collection_size(L):
-    """Large collections get the longest chunk (4,096); a 2,000-tensor
+    """Large collections get the longest chunk (2,048); a 2,000-tensor
     collection of 64..1,024 elements gets 256-element chunks so that every
     resident warp has work and no warp walks a whole tensor alone."""
     from elementwise_optimizer_b200 import synth
     W = 148 * 20
     big = B.TensorList(records([268_435_456]))
-    assert B.testing_choose_chunk_elems(big, W) == 4096
+    assert B.testing_choose_chunk_elems(big, W) == 2048
     w = synth.small_collection()
     small = B.TensorList(records(w.sizes, w.dtypes))
     assert B.testing_choose_chunk_elems(small, W) == 256
     for tl in (big, small):
         c = B.testing_choose_chunk_elems(tl, W)
-        assert c % 256 == 0 and 256 <= c <= 4096
-    assert B.testing_choose_chunk_elems(B.TensorList([]), W) in (256, 512, 1024, 2048, 4096)
+        assert c % 256 == 0 and 256 <= c <= 2048
+    assert B.testing_choose_chunk_elems(B.TensorList([]), W) in (256, 512, 1024, 2048)
 
 
 # --------------------------------------------------------------------------
