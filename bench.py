@@ -140,15 +140,26 @@ class ClockSampler:
 # Our arm
 # ---------------------------------------------------------------------------
 
+KERNEL_SOURCES = ("opt2s_kernel.cu", "opt2s_internal.h", "opt2s_api.cpp")
+
+
+def kernel_source_sha256():
+    """Hash of the sources that define the step kernel and its launch
+    configuration (chunk length, block width)."""
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "elementwise_optimizer_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def traffic_for(kernel_key):
     """ncu DRAM bytes per launch, if the committed capture is of the kernel
-    source as it is now (else None)."""
+    sources as they are now (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    src = os.path.join(ROOT, "elementwise_optimizer_b200", "csrc", "opt2s_kernel.cu")
     try:
         rec = json.load(open(path)).get(kernel_key)
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        if rec and rec.get("kernel_source_sha256") == sha:
+        if rec and rec.get("kernel_source_sha256") == kernel_source_sha256():
             return float(rec["dram_bytes_per_launch"])
     except Exception:
         pass
