@@ -244,7 +244,7 @@ def e2e_measure(w, d, device, steps, slices=8):
     copies that step's gradient from pinned host memory to the device, runs
     the optimizer step, and reads the updated param back into pinned host
     memory.  The collection is cut into `slices` element ranges, each stepped
-    by its own opt2s_step call, so that host-to-device copies (one stream),
+    through its own plan, so that host-to-device copies (one stream),
     steps (the compute stream) and device-to-host copies (a third stream)
     overlap: slice i+1 arrives while slice i is stepped and slice i-1 leaves."""
     import torch
@@ -265,6 +265,7 @@ def e2e_measure(w, d, device, steps, slices=8):
             raise NotImplementedError("sliced e2e supports one-moment state1 layouts")
         lists.append(B.TensorList.from_tensors([params[i][a:a + n]], [grads[i][a:a + n]],
                                                [s1[i][a:a + n]], [s2[i][a:a + n]]))
+    plans = [B.Plan(tl, w.algo) for tl in lists]     # one explicit plan per slice
     compute = torch.cuda.current_stream()
     h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
     h2d_bytes = sum(g.numel() * g.element_size() for g in host_g)
@@ -284,7 +285,7 @@ def e2e_measure(w, d, device, steps, slices=8):
             arrived.append(ev)
         for k, (i, a, n) in enumerate(ranges):
             compute.wait_event(arrived[k])
-            B.opt2s_step(lists[k], d["hyper"], t, stream=compute)
+            plans[k].step(d["hyper"], t, stream=compute)
             done = torch.cuda.Event()
             done.record(compute)
             prev_done[k] = done
@@ -311,7 +312,7 @@ def e2e_measure(w, d, device, steps, slices=8):
     return {"value": w.numel * steps / sec, "unit": "elements/s", "h2d_bytes_per_step": h2d_bytes,
             "d2h_bytes_per_step": d2h_bytes, "steps": steps, "ms_per_step": sec * 1e3 / steps,
             "slices": len(ranges),
-            "path": "pinned host grad -> device (stream 1), opt2s_step per slice (stream 2), "
+            "path": "pinned host grad -> device (stream 1), opt2s_plan_step per slice (stream 2), "
                     "device param -> pinned host (stream 3), slices overlapped"}
 
 
