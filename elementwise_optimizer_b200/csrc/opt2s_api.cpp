@@ -34,6 +34,7 @@ using opt2s::StepScalars;
 struct opt2s_plan {
     int device;
     int32_t algo;
+    int32_t only;         // dtype all chunks share (specialised kernel), or -1
     int64_t nchunks;
     ChunkRec* d_chunks;   // device copy of the chunk table
 };
@@ -54,9 +55,21 @@ int cuda_fail(cudaError_t e)
     return OPT2S_ERR_CUDA;
 }
 
-int block_threads_now(int algo)
+int block_threads_now(int algo, int only)
 {
-    return g_block_threads > 0 ? g_block_threads : opt2s::default_block_threads(algo);
+    return g_block_threads > 0 ? g_block_threads : opt2s::default_block_threads(algo, only);
+}
+
+// The storage dtype every non-empty tensor of `d` shares, or -1.
+int uniform_dtype(const TensorListDesc* d)
+{
+    int u = -2;
+    for (int32_t i = 0; i < d->count; ++i) {
+        if (d->tensors[i].numel == 0) continue;
+        if (u == -2) u = d->tensors[i].dtype;
+        else if (u != d->tensors[i].dtype) return -1;
+    }
+    return u == -2 ? -1 : u;
 }
 
 // Chunk length for a collection: the power-of-two multiple of 256 elements in
@@ -81,11 +94,11 @@ int64_t choose_chunk_elems(const TensorListDesc* d, int64_t resident_warps)
     return best;
 }
 
-int64_t chunk_elems_for(const TensorListDesc* d, int32_t algo)
+int64_t chunk_elems_for(const TensorListDesc* d, int32_t algo, int only)
 {
     if (g_chunk_elems > 0) return g_chunk_elems;
     int64_t warps = 0;
-    if (opt2s::resident_warps(algo, 0, block_threads_now(algo), &warps) != cudaSuccess)
+    if (opt2s::resident_warps(algo, 0, only, block_threads_now(algo, only), &warps) != cudaSuccess)
         return opt2s::kDefaultChunkElems;
     return choose_chunk_elems(d, warps);
 }
@@ -211,13 +224,14 @@ int plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out)
 {
     int st = validate_desc(desc, algo);
     if (st != OPT2S_OK) return st;
-    const int64_t ce = chunk_elems_for(desc, algo);
+    const int only = opt2s::kernel_only(algo, uniform_dtype(desc));
+    const int64_t ce = chunk_elems_for(desc, algo, only);
     if (count_chunks(desc, ce) > INT32_MAX) return OPT2S_ERR_TOO_LARGE;
     std::vector<ChunkRec> table = build_chunk_table(desc, ce);
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
-    auto* plan = new (std::nothrow) opt2s_plan{dev, algo, static_cast<int64_t>(table.size()), nullptr};
+    auto* plan = new (std::nothrow) opt2s_plan{dev, algo, only, static_cast<int64_t>(table.size()), nullptr};
     if (!plan) return OPT2S_ERR_NO_MEMORY;
     if (!table.empty()) {
         const size_t bytes = table.size() * sizeof(ChunkRec);
@@ -286,14 +300,14 @@ int plan_step(const opt2s_plan* plan, const Hyper* h, int step, cudaStream_t str
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev != plan->device) return OPT2S_ERR_DEVICE;
-    const int bt = block_threads_now(h->algo);
+    const int bt = block_threads_now(h->algo, plan->only);
     if (g_block_threads > 0) {   // forced geometry: must fit the kernel
         int widest = 0;
-        e = opt2s::max_block_threads(h->algo, h->skip_zeros, &widest);
+        e = opt2s::max_block_threads(h->algo, h->skip_zeros, plan->only, &widest);
         if (e != cudaSuccess) return cuda_fail(e);
         if (bt > widest) return OPT2S_ERR_INVALID_ARG;
     }
-    e = opt2s::launch_step(plan->d_chunks, plan->nchunks, h->algo, h->skip_zeros,
+    e = opt2s::launch_step(plan->d_chunks, plan->nchunks, h->algo, h->skip_zeros, plan->only,
                            make_scalars(h, step), bt, g_max_blocks, stream);
     if (e != cudaSuccess) return cuda_fail(e);
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -432,14 +446,14 @@ OPT2S_API int opt2s_plan_step_table(const opt2s_plan* plan, int32_t skip_zeros,
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev != plan->device) return OPT2S_ERR_DEVICE;
-    const int bt = block_threads_now(plan->algo);
+    const int bt = block_threads_now(plan->algo, plan->only);
     if (g_block_threads > 0) {
         int widest = 0;
-        e = opt2s::max_block_threads(plan->algo, skip_zeros, &widest);
+        e = opt2s::max_block_threads(plan->algo, skip_zeros, plan->only, &widest);
         if (e != cudaSuccess) return cuda_fail(e);
         if (bt > widest) return OPT2S_ERR_INVALID_ARG;
     }
-    e = opt2s::launch_step_table(plan->d_chunks, plan->nchunks, plan->algo, skip_zeros,
+    e = opt2s::launch_step_table(plan->d_chunks, plan->nchunks, plan->algo, skip_zeros, plan->only,
                                  reinterpret_cast<const StepScalars*>(d_table), d_index, table_len,
                                  bt, g_max_blocks, stream);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -610,7 +624,7 @@ OPT2S_API int opt2s_testing_max_block_threads(int32_t algo, int32_t skip_zeros)
     if ((algo != OPT2S_ADAM && algo != OPT2S_ADEMAMIX) || (skip_zeros != 0 && skip_zeros != 1))
         return OPT2S_ERR_INVALID_ARG;
     int widest = 0;
-    cudaError_t e = opt2s::max_block_threads(algo, skip_zeros, &widest);
+    cudaError_t e = opt2s::max_block_threads(algo, skip_zeros, -1, &widest);
     if (e != cudaSuccess) return cuda_fail(e);
     return widest;
 }

@@ -40,14 +40,24 @@ struct StepScalars {
     double inv_bc1, inv_bc2;
 };
 
-// Threads per block by algorithm.  Adam's kernel (96 registers) fits 20
-// resident warps per SM as 128-thread blocks (16 as 256-thread blocks);
-// AdEMAMix's (120 registers) fits 16 warps either way, and measured faster as
-// 256-thread blocks.
+// Threads per block.  Adam's generic kernel (96 registers) fits 20 resident
+// warps per SM as 128-thread blocks (16 as 256-thread blocks); AdEMAMix's (120
+// registers) fits 16 warps either way and measured faster as 256-thread blocks;
+// Adam specialised to one 16-bit dtype (66-72 registers) measured fastest as
+// 256-thread blocks.  `only` is the dtype every chunk of a plan shares, or -1.
 constexpr int kAdamBlockThreads = 128;
 constexpr int kAdEMAMixBlockThreads = 256;
+constexpr int kSpecialisedBlockThreads = 256;
 constexpr int kDefaultBlockThreads = 128;      // the no-alloc entry point's width
-inline int default_block_threads(int algo) { return algo == kAdEMAMix ? kAdEMAMixBlockThreads : kAdamBlockThreads; }
+inline int kernel_only(int algo, int uniform_dtype)
+{
+    return (algo == kAdam && (uniform_dtype == kF16 || uniform_dtype == kBF16)) ? uniform_dtype : -1;
+}
+inline int default_block_threads(int algo, int only)
+{
+    if (only >= 0) return kSpecialisedBlockThreads;
+    return algo == kAdEMAMix ? kAdEMAMixBlockThreads : kAdamBlockThreads;
+}
 constexpr int64_t kDefaultChunkElems = 2048;   // largest chunk the plan builder picks
 constexpr int64_t kMinChunkElems = 256;        // one warp iteration (8 elements per lane)
 
@@ -77,7 +87,7 @@ cudaError_t launch_shard_step(const ShardArgs& a, int algo, int skip_zeros, cons
 // `stream`.  block_threads: multiple of 32; max_blocks <= 0: occupancy-based
 // cap (resident blocks per SM x SM count).  Returns the launch status.
 cudaError_t launch_step(const ChunkRec* d_chunks, int64_t nchunks, int algo,
-                        int skip_zeros, const StepScalars& s,
+                        int skip_zeros, int only, const StepScalars& s,
                         int block_threads, int max_blocks,
                         cudaStream_t stream);
 
@@ -88,17 +98,17 @@ void fill_reciprocals(StepScalars* s);
 // followed by a one-thread launch that advances *d_index (to -1 after the
 // last entry).  Both launches may be captured in a CUDA graph.
 cudaError_t launch_step_table(const ChunkRec* d_chunks, int64_t nchunks, int algo,
-                              int skip_zeros, const StepScalars* d_table, int* d_index,
+                              int skip_zeros, int only, const StepScalars* d_table, int* d_index,
                               int table_len, int block_threads, int max_blocks,
                               cudaStream_t stream);
 
 // Resident warps of the step kernel for (algo, skip_zeros) on the current
 // device at `block_threads` threads per block (blocks per SM x SMs x warps).
-cudaError_t resident_warps(int algo, int skip_zeros, int block_threads, int64_t* out);
+cudaError_t resident_warps(int algo, int skip_zeros, int only, int block_threads, int64_t* out);
 
 // Widest block (threads, a multiple of 32) the step kernel for (algo,
 // skip_zeros) can be launched with: its registers per thread limit it.
-cudaError_t max_block_threads(int algo, int skip_zeros, int* out);
+cudaError_t max_block_threads(int algo, int skip_zeros, int only, int* out);
 
 // Validation scaffolding: counts into *d_count (device memory) the operands
 // among n seeded random ones for which the kernel's constant division differs
@@ -107,7 +117,7 @@ cudaError_t check_division(uint64_t seed, int64_t n, int mode, unsigned long lon
                            cudaStream_t stream);
 
 // Number of blocks a launch of `nchunks` chunks uses on the current device.
-cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros,
+cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros, int only,
                      int block_threads, int max_blocks, int* grid);
 
 }  // namespace opt2s

@@ -509,7 +509,10 @@ ShardFn pick_shard(int algo, int skip, int world)
 }
 
 // The whole step: warp w takes chunks w, w + W, w + 2W, ... of the table.
-template <int ALGO, bool SKIP>
+// ONLY < 0: every chunk dispatches on its own dtype; ONLY >= 0: every chunk
+// of the plan has that dtype (the host guarantees it), so the kernel carries
+// only that body and fewer registers.
+template <int ALGO, bool SKIP, int ONLY>
 __device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, int nchunks,
                                           const StepScalars& s)
 {
@@ -519,25 +522,29 @@ __device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, i
     const int nwarps = gridDim.x * warps_per_block;
     for (int c = warp; c < nchunks; c += nwarps) {
         const ChunkRec rec = chunks[c];
-        switch (rec.dtype) {
-        case kF32: run_chunk<kF32, ALGO, SKIP>(rec, s, lane); break;
-        case kF16: run_chunk<kF16, ALGO, SKIP>(rec, s, lane); break;
-        default: run_chunk<kBF16, ALGO, SKIP>(rec, s, lane); break;
+        if (ONLY >= 0) {
+            run_chunk<(ONLY >= 0 ? ONLY : kF32), ALGO, SKIP>(rec, s, lane);
+        } else {
+            switch (rec.dtype) {
+            case kF32: run_chunk<kF32, ALGO, SKIP>(rec, s, lane); break;
+            case kF16: run_chunk<kF16, ALGO, SKIP>(rec, s, lane); break;
+            default: run_chunk<kBF16, ALGO, SKIP>(rec, s, lane); break;
+            }
         }
     }
 }
 
 // Per-step scalars passed by value (the host computes them for each call).
-template <int ALGO, bool SKIP>
+template <int ALGO, bool SKIP, int ONLY>
 __global__ void step_kernel(const ChunkRec* __restrict__ chunks, int nchunks, StepScalars s)
 {
-    step_body<ALGO, SKIP>(chunks, nchunks, s);
+    step_body<ALGO, SKIP, ONLY>(chunks, nchunks, s);
 }
 
 // Per-step scalars read from a device table at a device-resident index, so a
 // captured CUDA graph performs the next step at every replay.  An index
 // outside [0, table_len) performs no update.
-template <int ALGO, bool SKIP>
+template <int ALGO, bool SKIP, int ONLY>
 __global__ void step_kernel_table(const ChunkRec* __restrict__ chunks, int nchunks,
                                   const StepScalars* __restrict__ table, const int* index,
                                   int table_len)
@@ -545,7 +552,7 @@ __global__ void step_kernel_table(const ChunkRec* __restrict__ chunks, int nchun
     const int idx = *index;
     if (idx < 0 || idx >= table_len) return;
     const StepScalars s = table[idx];
-    step_body<ALGO, SKIP>(chunks, nchunks, s);
+    step_body<ALGO, SKIP, ONLY>(chunks, nchunks, s);
 }
 
 // Moves the index to the next table entry; -1 once the table is used up.
@@ -558,24 +565,48 @@ __global__ void advance_index_kernel(int* index, int table_len)
 using KernelFn = void (*)(const ChunkRec*, int, StepScalars);
 using TableKernelFn = void (*)(const ChunkRec*, int, const StepScalars*, const int*, int);
 
-KernelFn pick(int algo, int skip)
+template <int ALGO, bool SKIP>
+KernelFn pick_only(int only)
 {
-    if (algo == kAdEMAMix) return skip ? step_kernel<kAdEMAMix, true> : step_kernel<kAdEMAMix, false>;
-    return skip ? step_kernel<kAdam, true> : step_kernel<kAdam, false>;
+    if (only == kF16) return step_kernel<ALGO, SKIP, kF16>;
+    if (only == kBF16) return step_kernel<ALGO, SKIP, kBF16>;
+    return step_kernel<ALGO, SKIP, -1>;
 }
 
-TableKernelFn pick_table(int algo, int skip)
+// Specialised bodies exist for Adam over one 16-bit dtype (measured faster
+// there); every other combination uses the per-chunk dispatch.
+KernelFn pick(int algo, int skip, int only)
+{
+    if (algo == kAdEMAMix) return skip ? step_kernel<kAdEMAMix, true, -1> : step_kernel<kAdEMAMix, false, -1>;
+    return skip ? pick_only<kAdam, true>(only) : pick_only<kAdam, false>(only);
+}
+
+template <int ALGO, bool SKIP>
+TableKernelFn pick_table_only(int only)
+{
+    if (only == kF16) return step_kernel_table<ALGO, SKIP, kF16>;
+    if (only == kBF16) return step_kernel_table<ALGO, SKIP, kBF16>;
+    return step_kernel_table<ALGO, SKIP, -1>;
+}
+
+TableKernelFn pick_table(int algo, int skip, int only)
 {
     if (algo == kAdEMAMix)
-        return skip ? step_kernel_table<kAdEMAMix, true> : step_kernel_table<kAdEMAMix, false>;
-    return skip ? step_kernel_table<kAdam, true> : step_kernel_table<kAdam, false>;
+        return skip ? step_kernel_table<kAdEMAMix, true, -1> : step_kernel_table<kAdEMAMix, false, -1>;
+    return skip ? pick_table_only<kAdam, true>(only) : pick_table_only<kAdam, false>(only);
+}
+
+int only_class(int algo, int only)
+{
+    if (algo == kAdEMAMix) return 0;
+    return only == kF16 ? 1 : (only == kBF16 ? 2 : 0);
 }
 
 // Resident blocks per SM and SM count, cached per device (and kernel / block
 // size): device attributes are per device, not per process.
 constexpr int kMaxDevices = 64;
 struct OccEntry { int block_threads; int blocks_per_sm; };
-struct DeviceInfo { int sms; OccEntry occ[4][6]; };
+struct DeviceInfo { int sms; OccEntry occ[12][6]; };
 DeviceInfo g_info[kMaxDevices];
 bool g_info_ok[kMaxDevices];
 
@@ -652,7 +683,7 @@ cudaError_t check_division(uint64_t seed, int64_t n, int mode, unsigned long lon
     return cudaGetLastError();
 }
 
-cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros, int block_threads,
+cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros, int only, int block_threads,
                      int max_blocks, int* grid)
 {
     const int warps_per_block = block_threads / 32;
@@ -664,13 +695,13 @@ cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros, int block_thread
         if (e != cudaSuccess) return e;
         DeviceInfo* info = nullptr;
         if ((e = device_info(dev, &info)) != cudaSuccess) return e;
-        const int k = (algo == kAdEMAMix ? 2 : 0) + (skip_zeros ? 1 : 0);
+        const int k = ((algo == kAdEMAMix ? 2 : 0) + (skip_zeros ? 1 : 0)) * 3 + only_class(algo, only);
         int per_sm = 0;
         for (auto& x : info->occ[k])
             if (x.block_threads == block_threads) per_sm = x.blocks_per_sm;
         if (per_sm == 0) {
             e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                &per_sm, pick(algo, skip_zeros), block_threads, 0);
+                &per_sm, pick(algo, skip_zeros, only), block_threads, 0);
             if (e != cudaSuccess) return e;
             if (per_sm < 1) per_sm = 1;
             for (auto& x : info->occ[k])
@@ -682,38 +713,38 @@ cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros, int block_thread
     return cudaSuccess;
 }
 
-cudaError_t resident_warps(int algo, int skip_zeros, int block_threads, int64_t* out)
+cudaError_t resident_warps(int algo, int skip_zeros, int only, int block_threads, int64_t* out)
 {
     int grid = 0;
     // the occupancy cap is what grid_for returns for an unbounded chunk count
-    cudaError_t e = grid_for(INT64_MAX / 2, algo, skip_zeros, block_threads, 0, &grid);
+    cudaError_t e = grid_for(INT64_MAX / 2, algo, skip_zeros, only, block_threads, 0, &grid);
     if (e != cudaSuccess) return e;
     *out = static_cast<int64_t>(grid) * (block_threads / 32);
     return cudaSuccess;
 }
 
-cudaError_t max_block_threads(int algo, int skip_zeros, int* out)
+cudaError_t max_block_threads(int algo, int skip_zeros, int only, int* out)
 {
     cudaFuncAttributes attr;
-    cudaError_t e = cudaFuncGetAttributes(&attr, pick(algo, skip_zeros));
+    cudaError_t e = cudaFuncGetAttributes(&attr, pick(algo, skip_zeros, only));
     if (e != cudaSuccess) return e;
     *out = attr.maxThreadsPerBlock / 32 * 32;
     return cudaSuccess;
 }
 
 cudaError_t launch_step(const ChunkRec* d_chunks, int64_t nchunks, int algo, int skip_zeros,
-                        const StepScalars& s, int block_threads, int max_blocks,
+                        int only, const StepScalars& s, int block_threads, int max_blocks,
                         cudaStream_t stream)
 {
     if (nchunks <= 0) return cudaSuccess;
     int grid = 0;
-    cudaError_t e = grid_for(nchunks, algo, skip_zeros, block_threads, max_blocks, &grid);
+    cudaError_t e = grid_for(nchunks, algo, skip_zeros, only, block_threads, max_blocks, &grid);
     if (e != cudaSuccess) return e;
     int n = static_cast<int>(nchunks);
     StepScalars sc = s;
     fill_reciprocals(&sc);   // correctly rounded binary64 reciprocals (IEEE)
     void* args[] = {const_cast<ChunkRec**>(&d_chunks), &n, &sc};
-    return cudaLaunchKernel(reinterpret_cast<const void*>(pick(algo, skip_zeros)),
+    return cudaLaunchKernel(reinterpret_cast<const void*>(pick(algo, skip_zeros, only)),
                             dim3(grid), dim3(block_threads), args, 0, stream);
 }
 
@@ -746,19 +777,19 @@ void fill_reciprocals(StepScalars* s)
 }
 
 cudaError_t launch_step_table(const ChunkRec* d_chunks, int64_t nchunks, int algo, int skip_zeros,
-                              const StepScalars* d_table, int* d_index, int table_len,
+                              int only, const StepScalars* d_table, int* d_index, int table_len,
                               int block_threads, int max_blocks, cudaStream_t stream)
 {
     if (nchunks > 0) {
         int grid = 0;
-        cudaError_t e = grid_for(nchunks, algo, skip_zeros, block_threads, max_blocks, &grid);
+        cudaError_t e = grid_for(nchunks, algo, skip_zeros, only, block_threads, max_blocks, &grid);
         if (e != cudaSuccess) return e;
         int n = static_cast<int>(nchunks);
         const int* idx = d_index;
         int len = table_len;
         void* args[] = {const_cast<ChunkRec**>(&d_chunks), &n, const_cast<StepScalars**>(&d_table),
                         const_cast<int**>(&idx), &len};
-        e = cudaLaunchKernel(reinterpret_cast<const void*>(pick_table(algo, skip_zeros)),
+        e = cudaLaunchKernel(reinterpret_cast<const void*>(pick_table(algo, skip_zeros, only)),
                              dim3(grid), dim3(block_threads), args, 0, stream);
         if (e != cudaSuccess) return e;
     }

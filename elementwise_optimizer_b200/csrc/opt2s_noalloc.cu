@@ -182,7 +182,7 @@ OPT2S_API int opt2s_step_noalloc(const TensorListDesc* desc, const Hyper* hyper,
     if (cudaMemcpyAsync(table, g_host_table, sizeof(ChunkRec) * nchunks, cudaMemcpyHostToDevice,
                         stream) != cudaSuccess)
         return OPT2S_ERR_CUDA;
-    if (opt2s::launch_step(table, nchunks, hyper->algo, hyper->skip_zeros, scalars(hyper, step),
+    if (opt2s::launch_step(table, nchunks, hyper->algo, hyper->skip_zeros, -1, scalars(hyper, step),
                            opt2s::kDefaultBlockThreads, 0, stream) != cudaSuccess)
         return OPT2S_ERR_CUDA;
     return OPT2S_OK;

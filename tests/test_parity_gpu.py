@@ -184,6 +184,37 @@ def test_geometry_does_not_change_arithmetic(block_threads, max_blocks, chunk):
     _assert_same(ref, got)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_single_dtype_kernel_equals_the_generic_kernel(dtype):
+    """A collection whose tensors all share one 16-bit dtype runs Adam on a
+    kernel specialised to that dtype; the same tensors stepped inside a
+    mixed-dtype collection run on the generic kernel.  Same bits, and the
+    same under forced block widths and chunk lengths."""
+    sizes = [1, 33, 1000, 4097, 100_003, 1 << 20]
+    # "normal" gradients: one draw per step, so the first tensors of both
+    # collections receive the same values
+    w_uni = synth.Workload("uniform", sizes, [dtype] * len(sizes), "adam",
+                           dict(synth.ADAM_HYPER, weight_decay=0.01), 3, synth.SEED_BASE + 12,
+                           "normal", skip_zeros=True)
+    w_mix = synth.Workload("mixed", sizes + [4096], [dtype] * len(sizes) + ["f32"], "adam",
+                           dict(synth.ADAM_HYPER, weight_decay=0.01), 3, synth.SEED_BASE + 12,
+                           "normal", skip_zeros=True)
+    _, uni = _run_gpu_only(w_uni, 3)
+    _, mix = _run_gpu_only(w_mix, 3)
+    _assert_same(uni, mix[:len(sizes)])
+    for bt, chunk in ((128, 0), (64, 256), (512, 2048)):
+        B.opt2s_release_cache()
+        prev = B.testing_set_chunk_elems(chunk)
+        B.testing_set_launch(bt, 0)
+        try:
+            _, got = _run_gpu_only(w_uni, 3)
+        finally:
+            B.testing_set_launch(0, 0)
+            B.testing_set_chunk_elems(prev)
+            B.opt2s_release_cache()
+        _assert_same(uni, got)
+
+
 @pytest.mark.parametrize("layout,pad", [("packed", 0), ("padded", 1), ("padded", 2),
                                         ("padded", 3), ("padded", 5)])
 def test_misaligned_storage_is_bitwise_identical(layout, pad):
