@@ -260,12 +260,13 @@ int plan_destroy(opt2s_plan* plan)
     if (!plan) return OPT2S_OK;
     int st = OPT2S_OK;
     if (plan->d_chunks) {
-        int cur = 0;
+        int cur = -1;
         cudaError_t e = cudaGetDevice(&cur);
-        if (e == cudaSuccess && cur != plan->device) e = cudaSetDevice(plan->device);
+        const bool switched = e == cudaSuccess && cur != plan->device;
+        if (switched) e = cudaSetDevice(plan->device);
         if (e == cudaSuccess) e = cudaFree(plan->d_chunks);   // waits for the device
         if (e != cudaSuccess) st = cuda_fail(e);
-        if (cur != plan->device) cudaSetDevice(cur);
+        if (switched) cudaSetDevice(cur);
     }
     delete plan;
     return st;

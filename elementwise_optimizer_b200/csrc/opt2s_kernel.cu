@@ -24,6 +24,8 @@
 // issue's "Correctness oracle" section requires that launch geometry must not
 // change optimizer arithmetic.
 
+#include <mutex>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -609,6 +611,7 @@ struct OccEntry { int block_threads; int blocks_per_sm; };
 struct DeviceInfo { int sms; OccEntry occ[12][6]; };
 DeviceInfo g_info[kMaxDevices];
 bool g_info_ok[kMaxDevices];
+std::mutex g_info_mu;   // guards g_info / g_info_ok (host threads may launch concurrently)
 
 cudaError_t device_info(int dev, DeviceInfo** out)
 {
@@ -693,6 +696,7 @@ cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros, int only, int bl
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
+        std::lock_guard<std::mutex> lock(g_info_mu);
         DeviceInfo* info = nullptr;
         if ((e = device_info(dev, &info)) != cudaSuccess) return e;
         const int k = ((algo == kAdEMAMix ? 2 : 0) + (skip_zeros ? 1 : 0)) * 3 + only_class(algo, only);

@@ -105,3 +105,45 @@ def test_two_ranks_equal_one_process(tmp_path, dtype, algo):
         ref1 = np.concatenate([s1[a:a + n], s1[N + a:N + a + n]]) if algo == "ademamix" else s1[a:a + n]
         assert np.array_equal(np.load(tmp_path / f"s1_{r}.npy"), ref1)
         assert np.array_equal(np.load(tmp_path / f"s2_{r}.npy"), s2[a:a + n])
+
+
+def _leaving_rank_main(rank, world, port, out_dir):
+    """Rank 1 leaves after step 1 (between steps, nothing in flight); rank 0
+    must learn of it from its next collective, which fails within the
+    process group's short timeout instead of waiting forever."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=10))
+    status = "no failure seen"
+    try:
+        for t in (1, 2, 3):
+            if rank == 1 and t == 2:
+                os._exit(3)                  # leaves between steps
+            buf = [torch.empty(4) for _ in range(world)]
+            dist.all_gather(buf, torch.full((4,), float(t)))
+    except Exception as exc:                 # the detection this test is about
+        status = f"detected: {type(exc).__name__}"
+    with open(os.path.join(out_dir, f"status_{rank}.txt"), "w") as f:
+        f.write(status)
+    os._exit(0)
+
+
+def test_a_rank_leaving_between_steps_is_detected(tmp_path):
+    import time
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_leaving_rank_main, args=(r, world, port, str(tmp_path)))
+             for r in range(world)]
+    t0 = time.time()
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert procs[1].exitcode == 3
+    assert procs[0].exitcode == 0
+    assert (tmp_path / "status_0.txt").read_text().startswith("detected")
+    assert time.time() - t0 < 100
