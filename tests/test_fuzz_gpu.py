@@ -16,6 +16,7 @@ import pytest
 
 from elementwise_optimizer_b200 import binding as B
 from elementwise_optimizer_b200 import synth
+from tests.gpu_support import Harness
 
 pytestmark = pytest.mark.gpu
 
@@ -68,7 +69,6 @@ def draw_case(case):
 
 @pytest.mark.parametrize("case", range(CASES))
 def test_random_collection_matches_oracle(case):
-    from gpu_support import Harness
     w, layout, pad, first_step, steps, geometry = draw_case(case)
     if geometry is not None:
         B.opt2s_release_cache()
