@@ -72,24 +72,29 @@ int uniform_dtype(const TensorListDesc* d)
     return u == -2 ? -1 : u;
 }
 
-// Chunk length for a collection: the power-of-two multiple of 256 elements in
-// [kMinChunkElems, kDefaultChunkElems] that minimizes the modelled time of the
-// slowest warp.  A warp handles ceil(chunks / resident_warps) chunks one after
-// the other; a chunk of c elements costs ceil(c / 256) dependent iterations
-// (256 elements per warp iteration) plus about one more for fetching its
-// record.  Large collections get long chunks (small table, few record
-// fetches); small ones get short chunks so every resident warp has work.
+// Chunk length for a collection: the power of two in [kMinChunkElems,
+// kDefaultChunkElems] that minimizes the modelled time of the slowest warp.  A
+// warp handles ceil(chunks / resident_warps) chunks one after the other; in a
+// chunk of c elements each lane performs max(c / 32, V) element updates one
+// after the other (V = 4 when every tensor is fp32, else 8: a lane moves at
+// least one 16-byte vector of each array), plus about 8 more for fetching the
+// chunk's record.  Large collections get long chunks (small table, few record
+// fetches); small ones get short chunks so that every resident warp has work
+// and each lane's serial part is short.  Ties go to the longer chunk.
 int64_t choose_chunk_elems(const TensorListDesc* d, int64_t resident_warps)
 {
     if (resident_warps < 1) return opt2s::kDefaultChunkElems;
+    int64_t lane_min = 4;
+    for (int32_t i = 0; i < d->count; ++i)
+        if (d->tensors[i].numel > 0 && d->tensors[i].dtype != OPT2S_F32) lane_min = 8;
     int64_t best = opt2s::kDefaultChunkElems;
-    double best_cost = -1.0;
+    int64_t best_cost = -1;
     for (int64_t c = opt2s::kDefaultChunkElems; c >= opt2s::kMinChunkElems; c /= 2) {
         int64_t chunks = 0;
         for (int32_t i = 0; i < d->count; ++i) chunks += (d->tensors[i].numel + c - 1) / c;
-        const double waves = static_cast<double>((chunks + resident_warps - 1) / resident_warps);
-        const double cost = waves * static_cast<double>(c / opt2s::kMinChunkElems + 1);
-        if (best_cost < 0.0 || cost < best_cost) { best_cost = cost; best = c; }
+        const int64_t waves = (chunks + resident_warps - 1) / resident_warps;
+        const int64_t cost = waves * (std::max(c / 32, lane_min) + 8);
+        if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = c; }
     }
     return best;
 }

@@ -59,7 +59,7 @@ inline int default_block_threads(int algo, int only)
     return algo == kAdEMAMix ? kAdEMAMixBlockThreads : kAdamBlockThreads;
 }
 constexpr int64_t kDefaultChunkElems = 2048;   // largest chunk the plan builder picks
-constexpr int64_t kMinChunkElems = 256;        // one warp iteration (8 elements per lane)
+constexpr int64_t kMinChunkElems = 128;        // one 16-byte fp32 vector per lane
 
 // The sharded (ZeRO-style) step of one rank.  Every rank holds the whole flat
 // param and grad buffers (same layout); this rank updates the elements

@@ -334,7 +334,9 @@ def test_step_scalar_table_rejects_bad_arguments(L):
 def test_chunk_length_follows_collection_size(L):
     """Large collections get the longest chunk (2,048); a 2,000-tensor
     collection of 64..1,024 elements gets 256-element chunks so that every
-    resident warp has work and no warp walks a whole tensor alone."""
+    resident warp has work and no warp walks a whole tensor alone; a small
+    all-fp32 tensor gets 128-element chunks (4 elements per lane), while a
+    16-bit one keeps 256 (a lane moves 8 16-bit elements in one vector)."""
     from elementwise_optimizer_b200 import synth
     W = 148 * 20
     big = B.TensorList(records([268_435_456]))
@@ -342,10 +344,13 @@ def test_chunk_length_follows_collection_size(L):
     w = synth.small_collection()
     small = B.TensorList(records(w.sizes, w.dtypes))
     assert B.testing_choose_chunk_elems(small, W) == 256
+    assert B.testing_choose_chunk_elems(B.TensorList(records([1024])), W) == 128
+    assert B.testing_choose_chunk_elems(B.TensorList(records([1024], ["bf16"])), W) == 256
+    assert B.testing_choose_chunk_elems(B.TensorList(records([1024, 64], ["f32", "f16"])), W) == 256
     for tl in (big, small):
         c = B.testing_choose_chunk_elems(tl, W)
-        assert c % 256 == 0 and 256 <= c <= 2048
-    assert B.testing_choose_chunk_elems(B.TensorList([]), W) in (256, 512, 1024, 2048)
+        assert c in (128, 256, 512, 1024, 2048)
+    assert B.testing_choose_chunk_elems(B.TensorList([]), W) == 2048
 
 
 # --------------------------------------------------------------------------

@@ -10,9 +10,9 @@ against a plain restatement of its rule:
     since neither is written);
   * the chunk-table builder: every element of every tensor in exactly one
     chunk, chunks in descriptor order, none longer than the chunk length;
-  * the chunk-length chooser: the power-of-two multiple of 256 in
-    [256, 2048] that minimises (waves of chunks over the resident warps) x
-    (chunk length / 256 + 1), the longest on ties;
+  * the chunk-length chooser: the power of two c in [128, 2048] that
+    minimises (waves of chunks over the resident warps) x (max(c / 32, V) + 8)
+    with V = 4 for all-fp32 collections and 8 otherwise, the longest on ties;
   * the shard partition: consecutive, 8-element aligned, covering the buffer.
 
 Pointers are fake addresses: nothing is dereferenced.
@@ -134,11 +134,12 @@ def test_chunk_table_covers_each_element_once(coll, chunk):
         assert pos.get(i, 0) == n
 
 
-def chosen_by_brute_force(sizes, warps):
+def chosen_by_brute_force(sizes, dts, warps):
+    lane_min = 8 if any(n > 0 and dt != "f32" for n, dt in zip(sizes, dts)) else 4
     best, best_cost = None, None
-    for c in (2048, 1024, 512, 256):
+    for c in (2048, 1024, 512, 256, 128):
         chunks = sum(-(-n // c) for n in sizes)
-        cost = -(-chunks // warps) * (c // 256 + 1)
+        cost = -(-chunks // warps) * (max(c // 32, lane_min) + 8)
         if best_cost is None or cost < best_cost:
             best, best_cost = c, cost
     return best
@@ -147,9 +148,9 @@ def chosen_by_brute_force(sizes, warps):
 @SETTINGS
 @given(collections(), st.integers(1, 148 * 64))
 def test_chunk_length_minimises_the_wave_model(coll, warps):
-    sizes, _, recs = coll
+    sizes, dts, recs = coll
     got = B.testing_choose_chunk_elems(B.TensorList(recs), warps)
-    assert got == chosen_by_brute_force(sizes, warps)
+    assert got == chosen_by_brute_force(sizes, dts, warps)
 
 
 @SETTINGS
