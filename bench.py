@@ -153,6 +153,29 @@ def kernel_source_sha256():
     return h.hexdigest()
 
 
+def environment():
+    """What the numbers were measured on: GPU, driver, CUDA runtime, nvcc,
+    torch, the hash of the kernel sources and the command line."""
+    import subprocess
+    import torch
+    env = {"torch": torch.__version__, "cuda_runtime": torch.version.cuda,
+           "kernel_sources_sha256": kernel_source_sha256(), "command": " ".join(sys.argv)}
+    if torch.cuda.is_available():
+        env["gpu"] = torch.cuda.get_device_name()
+    try:
+        env["driver"] = subprocess.run(
+            ["nvidia-smi", "--query-gpu=driver_version", "--format=csv,noheader"],
+            capture_output=True, text=True, timeout=20).stdout.split("\n")[0].strip() or None
+    except (OSError, subprocess.SubprocessError):
+        env["driver"] = None
+    try:
+        out = subprocess.run(["nvcc", "--version"], capture_output=True, text=True, timeout=20).stdout
+        env["nvcc"] = out.strip().splitlines()[-1] if out.strip() else None
+    except (OSError, subprocess.SubprocessError):
+        env["nvcc"] = None
+    return env
+
+
 def traffic_for(kernel_key):
     """ncu DRAM bytes per launch, if the committed capture is of the kernel
     sources as they are now (else None)."""
@@ -430,6 +453,7 @@ def run_ours(args, rank, world, local_rank):
     if "e2e" in extras:
         line["e2e"] = extras.pop("e2e")
     line.update(extras)
+    line["env"] = environment()
     if cpu is not None:
         line["cpu_baseline"] = cpu
     return line
@@ -829,6 +853,7 @@ def main():
         res = {"direct-cells": run_direct_cells, "eager-collection": run_eager_collection,
                "shard-emulated": run_shard_emulated,
                "roofline-table": run_roofline_table}[args.mode]()
+        res["env"] = environment()
         print(json.dumps(res), flush=True)
         return
 
