@@ -72,28 +72,31 @@ int uniform_dtype(const TensorListDesc* d)
     return u == -2 ? -1 : u;
 }
 
-// Chunk length for a collection: the power of two in [kMinChunkElems,
-// kDefaultChunkElems] that minimizes the modelled time of the slowest warp.  A
-// warp handles ceil(chunks / resident_warps) chunks one after the other; in a
-// chunk of c elements each lane performs max(c / 32, V) element updates one
-// after the other (V = 4 when every tensor is fp32, else 8: a lane moves at
-// least one 16-byte vector of each array), plus about 8 more for fetching the
-// chunk's record.  Large collections get long chunks (small table, few record
+// Chunk length for a collection: the power of two c in [kMinChunkElems,
+// kDefaultChunkElems] that minimizes the modelled time of the slowest warp,
+// ceil(chunks / resident_warps) x (c / 32 + 8).  A warp handles its chunks one
+// after the other; in a chunk of c elements each lane makes c / 32 element
+// updates one after the other, plus about 8 more for fetching the chunk's
+// record.  Large collections get long chunks (small table, few record
 // fetches); small ones get short chunks so that every resident warp has work
-// and each lane's serial part is short.  Ties go to the longer chunk.
+// and each lane's serial part is short.  A 128-element chunk gives each lane
+// 4 elements: one 16-byte vector of fp32, or the short-chunk path for 16-bit
+// storage, which pays only when the whole plan fits in one wave of warps; so
+// a plan with 16-bit tensors takes 128 only then.  Ties go to the longer chunk.
 int64_t choose_chunk_elems(const TensorListDesc* d, int64_t resident_warps)
 {
     if (resident_warps < 1) return opt2s::kDefaultChunkElems;
-    int64_t lane_min = 4;
+    bool all_f32 = true;
     for (int32_t i = 0; i < d->count; ++i)
-        if (d->tensors[i].numel > 0 && d->tensors[i].dtype != OPT2S_F32) lane_min = 8;
+        if (d->tensors[i].numel > 0 && d->tensors[i].dtype != OPT2S_F32) all_f32 = false;
     int64_t best = opt2s::kDefaultChunkElems;
     int64_t best_cost = -1;
     for (int64_t c = opt2s::kDefaultChunkElems; c >= opt2s::kMinChunkElems; c /= 2) {
         int64_t chunks = 0;
         for (int32_t i = 0; i < d->count; ++i) chunks += (d->tensors[i].numel + c - 1) / c;
         const int64_t waves = (chunks + resident_warps - 1) / resident_warps;
-        const int64_t cost = waves * (std::max(c / 32, lane_min) + 8);
+        if (c <= static_cast<int64_t>(opt2s::kShortChunkElems) && !all_f32 && waves > 1) continue;
+        const int64_t cost = waves * (c / 32 + 8);
         if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = c; }
     }
     return best;
@@ -206,7 +209,9 @@ int64_t count_chunks(const TensorListDesc* d, int64_t chunk_elems)
     return n;
 }
 
-std::vector<ChunkRec> build_chunk_table(const TensorListDesc* d, int64_t chunk_elems)
+// With `short16`, 16-bit chunks of at most kShortChunkElems elements are
+// marked for the kernel's short-chunk path.
+std::vector<ChunkRec> build_chunk_table(const TensorListDesc* d, int64_t chunk_elems, bool short16)
 {
     std::vector<ChunkRec> out;
     out.reserve(static_cast<size_t>(count_chunks(d, chunk_elems)));
@@ -220,6 +225,8 @@ std::vector<ChunkRec> build_chunk_table(const TensorListDesc* d, int64_t chunk_e
         r.m2 = t.state1 + t.numel + s;
         r.len = static_cast<uint32_t>(len);
         r.dtype = t.dtype;
+        if (short16 && t.dtype != OPT2S_F32 && len <= static_cast<int64_t>(opt2s::kShortChunkElems))
+            r.dtype |= opt2s::kShortFlag;
         out.push_back(r);
     });
     return out;
@@ -232,7 +239,8 @@ int plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out)
     const int only = opt2s::kernel_only(algo, uniform_dtype(desc));
     const int64_t ce = chunk_elems_for(desc, algo, only);
     if (count_chunks(desc, ce) > INT32_MAX) return OPT2S_ERR_TOO_LARGE;
-    std::vector<ChunkRec> table = build_chunk_table(desc, ce);
+    std::vector<ChunkRec> table =
+        build_chunk_table(desc, ce, ce <= static_cast<int64_t>(opt2s::kShortChunkElems));
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);

@@ -20,7 +20,7 @@ struct alignas(16) ChunkRec {
     float* v;         // state2
     float* m2;        // state1 + numel (AdEMAMix m2); not read by Adam
     uint32_t len;     // elements in the chunk, >= 1
-    int32_t dtype;    // kF32 / kF16 / kBF16
+    int32_t dtype;    // kF32 / kF16 / kBF16, 16-bit ones possibly | kShortFlag
 };
 static_assert(sizeof(ChunkRec) == 48, "ChunkRec layout");
 
@@ -60,6 +60,14 @@ inline int default_block_threads(int algo, int only)
 }
 constexpr int64_t kDefaultChunkElems = 2048;   // largest chunk the plan builder picks
 constexpr int64_t kMinChunkElems = 128;        // one 16-byte fp32 vector per lane
+
+// A plan whose chunk length is at most kShortChunkElems marks its 16-bit
+// chunks (dtype | kShortFlag) for the short-chunk path: 4 elements per lane
+// with element-wise accesses instead of one 16-byte vector of 8.  The chunk
+// length chooser picks such a length for a plan with 16-bit tensors only when
+// the plan fits in one wave of warps, where each lane's serial work decides.
+constexpr uint32_t kShortChunkElems = 128;
+enum : int { kShortFlag = 8 };
 
 // The sharded (ZeRO-style) step of one rank.  Every rank holds the whole flat
 // param and grad buffers (same layout); this rank updates the elements

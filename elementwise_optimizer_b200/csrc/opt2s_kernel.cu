@@ -351,6 +351,46 @@ __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& 
         vector_body<DT, ALGO, SKIP, false>(c, s, lane, head, nvec, al);
 }
 
+// A short 16-bit chunk (its record's dtype carries kShortFlag), processed by
+// one warp with element-wise accesses: lane l takes elements l, l + 32, l + 64
+// and l + 96, so each access instruction is still contiguous across the warp,
+// and a lane updates at most 4 elements where one 16-byte vector would give it
+// 8.  All loads come first, then the updates and stores.  Same arithmetic as
+// the vector body; a skipped element is not written back.  Kept out of line,
+// with its arguments by value (no stack frame), so that the step kernel's
+// register count stays that of its vector path.
+template <int DT, int ALGO, bool SKIP>
+__device__ __noinline__ void short_chunk(const ChunkRec c, const StepScalars s, int lane)
+{
+    using P = Param<DT>;
+    constexpr int K = kShortChunkElems / 32;
+    const uint32_t len = c.len;
+    float g[K], p[K], m[K], v[K], m2[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        const uint32_t i = lane + 32 * k;
+        g[k] = p[k] = m[k] = v[k] = m2[k] = 0.0f;
+        if (i < len) {
+            g[k] = P::load1(c.g, i);
+            p[k] = P::load1(c.p, i);
+            m[k] = ld_global(c.m + i);
+            v[k] = ld_global(c.v + i);
+            if (ALGO == kAdEMAMix) m2[k] = ld_global(c.m2 + i);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        const uint32_t i = lane + 32 * k;
+        if (i < len && !(SKIP && g[k] == 0.0f)) {
+            update<ALGO, false>(g[k], p[k], m[k], v[k], m2[k], s);
+            P::store1(c.p, i, p[k]);
+            st_global(c.m + i, m[k]);
+            st_global(c.v + i, v[k]);
+            if (ALGO == kAdEMAMix) st_global(c.m2 + i, m2[k]);
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // The sharded step (reduce-scatter + update + all-gather in one kernel).
 //
@@ -513,8 +553,11 @@ ShardFn pick_shard(int algo, int skip, int world)
 // The whole step: warp w takes chunks w, w + W, w + 2W, ... of the table.
 // ONLY < 0: every chunk dispatches on its own dtype; ONLY >= 0: every chunk
 // of the plan has that dtype (the host guarantees it), so the kernel carries
-// only that body and fewer registers.
-template <int ALGO, bool SKIP, int ONLY>
+// only that body and fewer registers.  SHORT: chunks marked with kShortFlag
+// take the short-chunk path; otherwise they take the vector path, with the
+// same result (the table-driven kernel does so, which keeps its register
+// count at the plain kernel's).
+template <int ALGO, bool SKIP, int ONLY, bool SHORT>
 __device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, int nchunks,
                                           const StepScalars& s)
 {
@@ -524,13 +567,22 @@ __device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, i
     const int nwarps = gridDim.x * warps_per_block;
     for (int c = warp; c < nchunks; c += nwarps) {
         const ChunkRec rec = chunks[c];
+        const bool short16 = SHORT && (rec.dtype & kShortFlag) != 0;
         if (ONLY >= 0) {
-            run_chunk<(ONLY >= 0 ? ONLY : kF32), ALGO, SKIP>(rec, s, lane);
+            constexpr int D = ONLY >= 0 ? ONLY : kF16;
+            if (short16) short_chunk<D, ALGO, SKIP>(rec, s, lane);
+            else run_chunk<D, ALGO, SKIP>(rec, s, lane);
         } else {
-            switch (rec.dtype) {
+            switch (rec.dtype & ~kShortFlag) {
             case kF32: run_chunk<kF32, ALGO, SKIP>(rec, s, lane); break;
-            case kF16: run_chunk<kF16, ALGO, SKIP>(rec, s, lane); break;
-            default: run_chunk<kBF16, ALGO, SKIP>(rec, s, lane); break;
+            case kF16:
+                if (short16) short_chunk<kF16, ALGO, SKIP>(rec, s, lane);
+                else run_chunk<kF16, ALGO, SKIP>(rec, s, lane);
+                break;
+            default:
+                if (short16) short_chunk<kBF16, ALGO, SKIP>(rec, s, lane);
+                else run_chunk<kBF16, ALGO, SKIP>(rec, s, lane);
+                break;
             }
         }
     }
@@ -540,7 +592,7 @@ __device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, i
 template <int ALGO, bool SKIP, int ONLY>
 __global__ void step_kernel(const ChunkRec* __restrict__ chunks, int nchunks, StepScalars s)
 {
-    step_body<ALGO, SKIP, ONLY>(chunks, nchunks, s);
+    step_body<ALGO, SKIP, ONLY, true>(chunks, nchunks, s);
 }
 
 // Per-step scalars read from a device table at a device-resident index, so a
@@ -554,7 +606,7 @@ __global__ void step_kernel_table(const ChunkRec* __restrict__ chunks, int nchun
     const int idx = *index;
     if (idx < 0 || idx >= table_len) return;
     const StepScalars s = table[idx];
-    step_body<ALGO, SKIP, ONLY>(chunks, nchunks, s);
+    step_body<ALGO, SKIP, ONLY, false>(chunks, nchunks, s);
 }
 
 // Moves the index to the next table entry; -1 once the table is used up.

@@ -68,9 +68,10 @@ int64_t opt2s_testing_default_chunk_elems(void);
 
 /* Host only: the chunk length a plan for `desc` gets on a device with
  * `resident_warps` resident warps of the step kernel: the power of two c in
- * [128, 2048] minimizing ceil(chunks / resident_warps) * (max(c / 32, V) + 8),
- * the modelled time of the slowest warp, where V is 4 if every non-empty
- * tensor is fp32 and 8 otherwise; ties go to the longer chunk. */
+ * [128, 2048] minimizing ceil(chunks / resident_warps) * (c / 32 + 8), the
+ * modelled time of the slowest warp; ties go to the longer chunk.  A
+ * collection with a non-empty 16-bit tensor takes 128 only when its chunks
+ * fit in one wave (chunks <= resident_warps). */
 int64_t opt2s_testing_choose_chunk_elems(const TensorListDesc *desc, int64_t resident_warps);
 
 /* Runs the step kernel's exact division by a constant in (0, 1] and the IEEE

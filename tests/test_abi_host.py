@@ -335,8 +335,9 @@ def test_chunk_length_follows_collection_size(L):
     """Large collections get the longest chunk (2,048); a 2,000-tensor
     collection of 64..1,024 elements gets 256-element chunks so that every
     resident warp has work and no warp walks a whole tensor alone; a small
-    all-fp32 tensor gets 128-element chunks (4 elements per lane), while a
-    16-bit one keeps 256 (a lane moves 8 16-bit elements in one vector)."""
+    tensor gets 128-element chunks (4 elements per lane).  A plan with 16-bit
+    tensors takes 128 only when it fits in one wave of warps (the short-chunk
+    path pays only there); an all-fp32 one whenever the model says so."""
     from elementwise_optimizer_b200 import synth
     W = 148 * 20
     big = B.TensorList(records([268_435_456]))
@@ -345,8 +346,11 @@ def test_chunk_length_follows_collection_size(L):
     small = B.TensorList(records(w.sizes, w.dtypes))
     assert B.testing_choose_chunk_elems(small, W) == 256
     assert B.testing_choose_chunk_elems(B.TensorList(records([1024])), W) == 128
-    assert B.testing_choose_chunk_elems(B.TensorList(records([1024], ["bf16"])), W) == 256
-    assert B.testing_choose_chunk_elems(B.TensorList(records([1024, 64], ["f32", "f16"])), W) == 256
+    assert B.testing_choose_chunk_elems(B.TensorList(records([1024], ["bf16"])), W) == 128
+    assert B.testing_choose_chunk_elems(B.TensorList(records([1024, 64], ["f32", "f16"])), W) == 128
+    # ten 100-element tensors over 4 warps: three waves whatever the length
+    assert B.testing_choose_chunk_elems(B.TensorList(records([100] * 10)), 4) == 128
+    assert B.testing_choose_chunk_elems(B.TensorList(records([100] * 10, ["f16"] * 10)), 4) == 256
     for tl in (big, small):
         c = B.testing_choose_chunk_elems(tl, W)
         assert c in (128, 256, 512, 1024, 2048)

@@ -11,8 +11,9 @@ against a plain restatement of its rule:
   * the chunk-table builder: every element of every tensor in exactly one
     chunk, chunks in descriptor order, none longer than the chunk length;
   * the chunk-length chooser: the power of two c in [128, 2048] that
-    minimises (waves of chunks over the resident warps) x (max(c / 32, V) + 8)
-    with V = 4 for all-fp32 collections and 8 otherwise, the longest on ties;
+    minimises (waves of chunks over the resident warps) x (c / 32 + 8), the
+    longest on ties, where a plan with 16-bit tensors takes 128 only when it
+    fits in one wave;
   * the shard partition: consecutive, 8-element aligned, covering the buffer.
 
 Pointers are fake addresses: nothing is dereferenced.
@@ -135,11 +136,14 @@ def test_chunk_table_covers_each_element_once(coll, chunk):
 
 
 def chosen_by_brute_force(sizes, dts, warps):
-    lane_min = 8 if any(n > 0 and dt != "f32" for n, dt in zip(sizes, dts)) else 4
+    all_f32 = not any(n > 0 and dt != "f32" for n, dt in zip(sizes, dts))
     best, best_cost = None, None
     for c in (2048, 1024, 512, 256, 128):
         chunks = sum(-(-n // c) for n in sizes)
-        cost = -(-chunks // warps) * (max(c // 32, lane_min) + 8)
+        waves = -(-chunks // warps)
+        if c == 128 and not all_f32 and waves > 1:
+            continue
+        cost = waves * (c // 32 + 8)
         if best_cost is None or cost < best_cost:
             best, best_cost = c, cost
     return best

@@ -215,6 +215,39 @@ def test_single_dtype_kernel_equals_the_generic_kernel(dtype):
         _assert_same(uni, got)
 
 
+@pytest.mark.parametrize("skip", [False, True])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+def test_short_chunk_path_equals_vector_path_and_oracle(algo, dtype, skip):
+    """A one-wave plan of 16-bit tensors gets 128-element chunks, and its
+    chunks take the short-chunk path (element-wise accesses, 4 elements per
+    lane).  The same tensors with 2,048-element chunks take the 16-byte vector
+    path.  Both must hold the oracle's bits after every step."""
+    sizes = [1, 2, 31, 32, 33, 64, 100, 127, 128, 129, 255, 1000, 1024]
+    hy = dict(synth.ADEMAMIX_HYPER if algo == "ademamix" else synth.ADAM_HYPER, weight_decay=0.01)
+    w = synth.Workload("short16", sizes, [dtype] * len(sizes), algo, hy, 3,
+                       synth.SEED_BASE + 14, "mixed_magnitude", skip_zeros=skip)
+    half = [torch.empty(n, dtype=torch.bfloat16, device="cuda") for n in sizes]
+    state = [torch.empty(n, device="cuda") for n in sizes]
+    assert B.testing_choose_chunk_elems(B.TensorList.from_tensors(half, half, state, state),
+                                        148 * 16) == 128      # 29 chunks: one wave
+    results = []
+    for chunk in (0, 2048):
+        B.opt2s_release_cache()
+        prev = B.testing_set_chunk_elems(chunk)
+        try:
+            h = Harness(w)
+            for t in (1, 2, 3):
+                h.step_both(t)
+                assert h.max_ulps() == {"param": 0, "state1": 0, "state2": 0}, (chunk, t)
+                assert h.grads_unchanged()
+            results.append(_final_state(h))
+        finally:
+            B.testing_set_chunk_elems(prev)
+            B.opt2s_release_cache()
+    _assert_same(results[0], results[1])
+
+
 @pytest.mark.parametrize("layout,pad", [("packed", 0), ("padded", 1), ("padded", 2),
                                         ("padded", 3), ("padded", 5)])
 def test_misaligned_storage_is_bitwise_identical(layout, pad):
