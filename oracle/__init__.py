@@ -74,6 +74,9 @@ def _load():
     lib.oracle_step_f32_fgrad.argtypes = [i32, i32, i32, f32, f32, f32, f32, f32,
                                           f32, f32, i32, vp, vp, vp, vp, i64]
     lib.oracle_step_f32_fgrad.restype = i32
+    lib.oracle_step_f32_max_unorm.argtypes = [i32, i32, i32, f32, f32, f32, f32, f32,
+                                              f32, f32, f32, i32, vp, vp, vp, vp, i64, vp]
+    lib.oracle_step_f32_max_unorm.restype = i32
     lib.oracle_average_grads.argtypes = [i32, i32, vp, vp, i64]
     lib.oracle_average_grads.restype = i32
     lib.oracle_bias_correction.argtypes = [f32, i32]
@@ -121,6 +124,33 @@ def step_f32(param: np.ndarray, grad: np.ndarray, state1: np.ndarray,
         _ptr(state1), _ptr(state2), n)
     if rc != 0:
         raise ValueError(f"oracle_step_f32 rejected its arguments ({rc})")
+
+
+def step_f32_max_unorm(param: np.ndarray, grad: np.ndarray, state1: np.ndarray,
+                       state2: np.ndarray, *, dtype: str, algo: str, step: int,
+                       lr: float, beta1: float, beta2: float, eps: float,
+                       max_unorm: float, beta3: float = 0.0, alpha: float = 0.0,
+                       weight_decay: float = 0.0, skip_zeros: bool = False) -> float:
+    """One step over one tensor with its update norm clipped to
+    max_unorm x its weight norm (max_unorm > 0); arrays as in step_f32.
+    Returns the fp32 scale s the update was multiplied by (1 when the norm
+    is within the bound)."""
+    n = param.size
+    if grad.size != n or param.itemsize != _ITEMSIZE[dtype] or \
+            grad.itemsize != _ITEMSIZE[dtype]:
+        raise ValueError("param/grad size or item size mismatch")
+    want1 = 2 * n if algo == "ademamix" else n
+    if state1.dtype != np.float32 or state2.dtype != np.float32 or \
+            state1.size != want1 or state2.size != n:
+        raise ValueError("state arrays must be float32 of the right length")
+    scale = np.zeros(1, np.float32)
+    rc = _load().oracle_step_f32_max_unorm(
+        ALGO[algo], DTYPE[dtype], int(bool(skip_zeros)), lr, beta1, beta2,
+        beta3, alpha, eps, weight_decay, max_unorm, int(step), _ptr(param), _ptr(grad),
+        _ptr(state1), _ptr(state2), n, _ptr(scale))
+    if rc != 0:
+        raise ValueError(f"oracle_step_f32_max_unorm rejected its arguments ({rc})")
+    return float(scale[0])
 
 
 def step_f32_fgrad(param: np.ndarray, grad: np.ndarray, state1: np.ndarray,

@@ -204,24 +204,40 @@ float oracle_decay_factor(float lr, float wd)
  *   p   = p*decay - lr*(num/den)       decay first, [AdamW]; [issue] "Scope"
  * Returns 0, or -1 on an argument the definitions do not cover.
  */
+/* The new moments of one element and its update direction u = num/den
+ * (m2 is read and written only for AdEMAMix). */
+static void element_direction(int algo, float g, float m, float m2, float v,
+                              float beta1, float beta2, float beta3, float alpha,
+                              float eps, float bc1, float bc2, float one_minus_b1,
+                              float one_minus_b2, float one_minus_b3,
+                              float *mi, float *m2i, float *vi, float *u)
+{
+    *mi = beta1 * m + one_minus_b1 * g;
+    *vi = beta2 * v + (one_minus_b2 * g) * g;
+    float num = *mi / bc1;
+    *m2i = m2;
+    if (algo == OR_ADEMAMIX) {
+        *m2i = beta3 * m2 + one_minus_b3 * g;
+        num = num + alpha * *m2i;
+    }
+    float den = sqrtf(*vi / bc2) + eps;
+    *u = num / den;
+}
+
 /* The per-element update of one step (shared by both fp32 step entries). */
 static void update_element(int algo, float g, float *p, float *m, float *m2, float *v,
                            float lr, float beta1, float beta2, float beta3, float alpha,
                            float eps, float bc1, float bc2, float decay,
                            float one_minus_b1, float one_minus_b2, float one_minus_b3)
 {
-    float mi = beta1 * *m + one_minus_b1 * g;
-    float vi = beta2 * *v + (one_minus_b2 * g) * g;
-    float num = mi / bc1;
-    if (algo == OR_ADEMAMIX) {
-        float m2i = beta3 * *m2 + one_minus_b3 * g;
-        num = num + alpha * m2i;
-        *m2 = m2i;
-    }
-    float den = sqrtf(vi / bc2) + eps;
-    *p = *p * decay - lr * (num / den);
+    float mi, m2i, vi, u;
+    element_direction(algo, g, *m, algo == OR_ADEMAMIX ? *m2 : 0.0f, *v, beta1, beta2,
+                      beta3, alpha, eps, bc1, bc2, one_minus_b1, one_minus_b2,
+                      one_minus_b3, &mi, &m2i, &vi, &u);
+    *p = *p * decay - lr * u;
     *m = mi;
     *v = vi;
+    if (algo == OR_ADEMAMIX) *m2 = m2i;
 }
 
 /* One step over n elements whose gradient is read by get_grad(grad, i). */
@@ -316,6 +332,89 @@ int oracle_step_f32_fgrad(int algo, int dtype, int skip_zeros,
     return step_core(algo, dtype, skip_zeros, lr, beta1, beta2, beta3, alpha, eps,
                      weight_decay, step, param, grad, grad_in_f32, OR_F32, state1,
                      state2, n);
+}
+
+/*
+ * The step with the update norm of the tensor clipped: max_unorm > 0.
+ *
+ * [issue] "Scope" keeps the existing kernel for "max-unorm/LAMB use" and
+ * section "Correctness oracle" runs "max_unorm > 0" controls, so max_unorm
+ * is an option of this same two-state update, but the pages never write out
+ * its arithmetic.  Reading used here (the plainest one the name supports:
+ * max_unorm bounds the norm of the update relative to the norm of the
+ * weights, the tensor being the unit):
+ *   u_i = num_i / den_i, the update direction of element i exactly as in the
+ *         plain step (fp32); u_i = 0 for an element skip_zeros leaves alone;
+ *   U   = sqrt(sum_i u_i^2) and P = sqrt(sum_i p_i^2) over the tensor, p the
+ *         stored param before the step; squares, sums and roots in binary64,
+ *         summed in index order;
+ *   s   = max_unorm*P/U if U > max_unorm*P, else 1 (binary64, then rounded
+ *         to fp32 once);
+ *   p_i = p_i*decay - lr*(s*u_i) in fp32, with m, v (and m2) exactly as in
+ *         the plain step.  s = 1 gives the plain step's bits.
+ * The tensor is read twice: once for U and P, once for the update.
+ * Returns 0, or -1 on an argument the definitions do not cover.
+ */
+int oracle_step_f32_max_unorm(int algo, int dtype, int skip_zeros,
+                              float lr, float beta1, float beta2, float beta3,
+                              float alpha, float eps, float weight_decay,
+                              float max_unorm, int step, void *param,
+                              const void *grad, float *state1, float *state2,
+                              int64_t n, float *scale_out)
+{
+    if (step < 1 || n < 0 || !(max_unorm > 0.0f)) return -1;
+    if (algo != OR_ADAM && algo != OR_ADEMAMIX) return -1;
+    if (dtype != OR_F32 && dtype != OR_F16 && dtype != OR_BF16) return -1;
+
+    unsigned int csr = _mm_getcsr();
+    _mm_setcsr(csr & ~(0x8000u | 0x0040u));             /* FTZ and DAZ off */
+
+    const float bc1 = oracle_bias_correction(beta1, step);
+    const float bc2 = oracle_bias_correction(beta2, step);
+    const float decay = oracle_decay_factor(lr, weight_decay);
+    const float one_minus_b1 = 1.0f - beta1;
+    const float one_minus_b2 = 1.0f - beta2;
+    const float one_minus_b3 = 1.0f - beta3;
+    float *m = state1;
+    float *m2 = state1 + n;                             /* AdEMAMix only */
+    float *v = state2;
+
+    /* pass 1: the norms of the update and of the weights */
+    double su = 0.0, sp = 0.0;
+    for (int64_t i = 0; i < n; i++) {
+        float p = load_param(param, dtype, i);
+        sp += (double)p * (double)p;
+        float g = load_param(grad, dtype, i);
+        if (skip_zeros && g == 0.0f) continue;
+        float mi, m2i, vi, u;
+        element_direction(algo, g, m[i], algo == OR_ADEMAMIX ? m2[i] : 0.0f, v[i], beta1,
+                          beta2, beta3, alpha, eps, bc1, bc2, one_minus_b1, one_minus_b2,
+                          one_minus_b3, &mi, &m2i, &vi, &u);
+        su += (double)u * (double)u;
+    }
+    const double U = sqrt(su), P = sqrt(sp);
+    const double limit = (double)max_unorm * P;
+    const float scale = (float)(U > limit ? limit / U : 1.0);
+    if (scale_out) *scale_out = scale;
+
+    /* pass 2: the update, scaled */
+    for (int64_t i = 0; i < n; i++) {
+        float g = load_param(grad, dtype, i);
+        if (skip_zeros && g == 0.0f) continue;
+        float p = load_param(param, dtype, i);
+        float mi, m2i, vi, u;
+        element_direction(algo, g, m[i], algo == OR_ADEMAMIX ? m2[i] : 0.0f, v[i], beta1,
+                          beta2, beta3, alpha, eps, bc1, bc2, one_minus_b1, one_minus_b2,
+                          one_minus_b3, &mi, &m2i, &vi, &u);
+        p = p * decay - lr * (scale * u);
+        store_param(param, dtype, i, p);
+        m[i] = mi;
+        v[i] = vi;
+        if (algo == OR_ADEMAMIX) m2[i] = m2i;
+    }
+
+    _mm_setcsr(csr);
+    return 0;
 }
 
 /*

@@ -18,25 +18,21 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "opt2s_oracle.c")
 
 MUTANTS = {
-    "eps_dropped": ("sqrtf(vi / bc2) + eps", "sqrtf(vi / bc2)"),
-    "eps_inside_sqrt": ("sqrtf(vi / bc2) + eps", "sqrtf(vi / bc2 + eps)"),
-    "bc1_for_v": ("sqrtf(vi / bc2)", "sqrtf(vi / bc1)"),
-    "decay_after_update": ("*p = *p * decay - lr * (num / den);",
-                           "*p = (*p - lr * (num / den)) * decay;"),
-    "update_sign": ("*p = *p * decay - lr * (num / den);",
-                    "*p = *p * decay + lr * (num / den);"),
-    "m2_bias_corrected": ("num = num + alpha * m2i;",
-                          "num = num + alpha * (m2i / bc1);"),
-    "alpha_on_m1": ("num = num + alpha * m2i;", "num = alpha * num + m2i;"),
-    "one_minus_b3_dropped": ("beta3 * *m2 + one_minus_b3 * g",
-                             "beta3 * *m2 + g"),
+    "eps_dropped": ("sqrtf(*vi / bc2) + eps", "sqrtf(*vi / bc2)"),
+    "eps_inside_sqrt": ("sqrtf(*vi / bc2) + eps", "sqrtf(*vi / bc2 + eps)"),
+    "bc1_for_v": ("sqrtf(*vi / bc2)", "sqrtf(*vi / bc1)"),
+    "decay_after_update": ("*p = *p * decay - lr * u;", "*p = (*p - lr * u) * decay;"),
+    "update_sign": ("*p = *p * decay - lr * u;", "*p = *p * decay + lr * u;"),
+    "m2_bias_corrected": ("num = num + alpha * *m2i;", "num = num + alpha * (*m2i / bc1);"),
+    "alpha_on_m1": ("num = num + alpha * *m2i;", "num = alpha * num + *m2i;"),
+    "one_minus_b3_dropped": ("beta3 * m2 + one_minus_b3 * g", "beta3 * m2 + g"),
     "v_not_squared": ("(one_minus_b2 * g) * g", "(one_minus_b2 * g)"),
     "average_wrong_divisor": ("out[i] = sum / (float)world;",
                               "out[i] = sum / (float)(world + 1);"),
     "average_drops_last_rank": ("for (int q = 1; q < world; q++)",
                                 "for (int q = 1; q < world - 1; q++)"),
-    "m_uses_beta2": ("float mi = beta1 * *m + one_minus_b1 * g;",
-                     "float mi = beta2 * *m + one_minus_b1 * g;"),
+    "m_uses_beta2": ("*mi = beta1 * m + one_minus_b1 * g;",
+                     "*mi = beta2 * m + one_minus_b1 * g;"),
     "bias_exponent_off_by_one": ("pow((double)beta, (double)t)",
                                  "pow((double)beta, (double)(t + 1))"),
     "decay_without_lr": ("1.0 - (double)lr * (double)wd", "1.0 - (double)wd"),
@@ -51,6 +47,17 @@ MUTANTS = {
     "shadow_v_not_squared": ("(1.0 - beta2) * g * g;", "(1.0 - beta2) * g;"),
     "shadow_eps_inside_sqrt": ("sqrt(v[i] / bc2) + eps", "sqrt(v[i] / bc2 + eps)"),
     "shadow_m2_missing_rate": ("beta3 * m2[i] + (1.0 - beta3) * g", "beta3 * m2[i] + g"),
+    "unorm_of_grad": ("su += (double)u * (double)u;", "su += (double)g * (double)g;"),
+    "pnorm_after_decay": ("sp += (double)p * (double)p;",
+                          "sp += (double)(p * decay) * (double)(p * decay);"),
+    "unorm_ratio_inverted": ("U > limit ? limit / U : 1.0", "U > limit ? U / limit : 1.0"),
+    "unorm_scale_dropped": ("p = p * decay - lr * (scale * u);", "p = p * decay - lr * u;"),
+    "unorm_without_sqrt": ("const double U = sqrt(su), P = sqrt(sp);",
+                           "const double U = su, P = sp;"),
+    "unorm_counts_skipped": (
+        "sp += (double)p * (double)p;\n        float g = load_param(grad, dtype, i);\n"
+        "        if (skip_zeros && g == 0.0f) continue;\n",
+        "sp += (double)p * (double)p;\n        float g = load_param(grad, dtype, i);\n"),
 }
 
 

@@ -461,3 +461,103 @@ def test_fp32_gradient_step_reduces_to_the_storage_step(oracle_mod, algo, dtype)
     oracle_mod.step_f32_fgrad(b[0], synth.from_storage(gr, dtype), b[1], b[2], **kw)
     for x, y in zip(a, b):
         assert np.array_equal(x.view(np.uint8), y.view(np.uint8))
+
+
+# --------------------------------------------------------------------------
+# max_unorm: the update norm of a tensor clipped to max_unorm x its weight
+# norm (the reading the oracle states; the pages name the option only)
+# --------------------------------------------------------------------------
+
+UNORM_HYPER = dict(lr=0.1, beta1=0.9, beta2=0.999, eps=1e-8, beta3=0.999, alpha=3.0)
+
+
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("skip", [False, True])
+def test_max_unorm_above_the_norm_is_the_plain_step(oracle_mod, algo, dtype, skip):
+    """A bound no update reaches leaves every bit of the plain step."""
+    n = 5000
+    p, gr, s1, v = _random_state(300, n, dtype, algo)
+    gr[::7] = 0
+    a = (p.copy(), s1.copy(), v.copy())
+    b = (p.copy(), s1.copy(), v.copy())
+    h = dict(UNORM_HYPER, weight_decay=0.01)
+    oracle_mod.step_f32(a[0], gr, a[1], a[2], dtype=dtype, algo=algo, step=7, skip_zeros=skip, **h)
+    s = oracle_mod.step_f32_max_unorm(b[0], gr, b[1], b[2], dtype=dtype, algo=algo, step=7,
+                                      skip_zeros=skip, max_unorm=1e30, **h)
+    assert s == 1.0
+    for x, y in zip(a, b):
+        assert np.array_equal(x.view(np.uint8), y.view(np.uint8))
+
+
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+def test_max_unorm_step_one_closed_form(oracle_mod, algo):
+    """Every element equal: p0 = 0.5, g = 0.25.  At t = 1 every element has
+    the same update u (1 for Adam, 1 + alpha(1-beta3) for AdEMAMix, up to
+    eps), so |u| sqrt(n) against max_unorm * 0.5 sqrt(n) decides: a bound
+    below |u| / 0.5 clips every element to p1 = p0 - lr*max_unorm*p0, a bound
+    above it leaves p1 = p0 - lr*u."""
+    n = 4096
+    p0, g0 = 0.5, 0.25
+    u = 1.0 + (UNORM_HYPER["alpha"] * (1 - UNORM_HYPER["beta3"]) if algo == "ademamix" else 0.0)
+    for mu, want in ((0.1, p0 - UNORM_HYPER["lr"] * 0.1 * p0),
+                     (10.0, p0 - UNORM_HYPER["lr"] * u)):
+        p = np.full(n, p0, np.float32)
+        g = np.full(n, g0, np.float32)
+        s1 = np.zeros(2 * n if algo == "ademamix" else n, np.float32)
+        v = np.zeros(n, np.float32)
+        oracle_mod.step_f32_max_unorm(p, g, s1, v, dtype="f32", algo=algo, step=1,
+                                      max_unorm=mu, **UNORM_HYPER)
+        assert np.all(p == p[0])
+        assert abs(float(p[0]) - want) <= 8 * float(ulp32(want)), (mu, float(p[0]), want)
+
+
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+@pytest.mark.parametrize("wd", [0.0, 0.5])
+@pytest.mark.parametrize("t", [1, 10, 1000])
+def test_max_unorm_bounds_the_applied_update(oracle_mod, algo, wd, t):
+    """The update actually applied, p1 - p0*decay (one fp32 product rounded
+    as the step rounds it), has norm lr*max_unorm*||p0|| when the bound
+    binds, and the plain step's update otherwise; skipped elements add
+    nothing.  Checked on random states against norms taken in float64."""
+    n = 20000
+    for skip in (False, True):
+        p, gr, s1, v = _random_state(400 + t, n, "f32", algo)
+        if skip:
+            gr[::3] = 0
+        h = dict(UNORM_HYPER, weight_decay=wd)
+        decay = np.float32(oracle_mod.decay_factor(h["lr"], wd))
+        plain = (p.copy(), s1.copy(), v.copy())
+        oracle_mod.step_f32(plain[0], gr, plain[1], plain[2], dtype="f32", algo=algo, step=t,
+                            skip_zeros=skip, **h)
+        base = (p * decay).astype(np.float64)          # rounded to fp32 like the step
+        d_plain = plain[0].astype(np.float64) - base
+        if skip:
+            d_plain[gr == 0] = 0.0
+        pn = float(np.linalg.norm(p.astype(np.float64)))
+        free = float(np.linalg.norm(d_plain)) / (h["lr"] * pn)  # the unclipped ratio
+        for mu in (0.25 * free, 0.8 * free, 4.0 * free):
+            q, m_, v_ = p.copy(), s1.copy(), v.copy()
+            s = oracle_mod.step_f32_max_unorm(q, gr, m_, v_, dtype="f32", algo=algo, step=t,
+                                              skip_zeros=skip, max_unorm=float(np.float32(mu)), **h)
+            d = q.astype(np.float64) - base
+            if skip:
+                assert np.array_equal(q[gr == 0], p[gr == 0])
+                d[gr == 0] = 0.0
+            norm = float(np.linalg.norm(d))
+            if mu < free:
+                assert s < 1.0
+                assert norm == pytest.approx(h["lr"] * float(np.float32(mu)) * pn, rel=2e-4)
+            else:
+                assert s == 1.0
+                assert np.array_equal(q, plain[0])
+            # the moments never depend on the bound
+            assert np.array_equal(m_, plain[1]) and np.array_equal(v_, plain[2])
+
+
+def test_max_unorm_must_be_positive(oracle_mod):
+    p, gr, s1, v = _random_state(500, 16, "f32", "adam")
+    for mu in (0.0, -1.0, float("nan")):
+        with pytest.raises(ValueError):
+            oracle_mod.step_f32_max_unorm(p, gr, s1, v, dtype="f32", algo="adam", step=1,
+                                          max_unorm=mu, **UNORM_HYPER)
