@@ -816,6 +816,54 @@ def run_roofline_table(numel=268_435_456, steps=50, warmup=10):
             "rows": rows}
 
 
+def run_max_unorm(numel=268_435_456, steps=50, warmup=10, max_unorm=1.0):
+    """The bounded-update-norm step (opt2s_step_max_unorm: norm sums, scales,
+    scaled update) on one tensor of `numel` elements, timed beside the plain
+    step on the same buffers.  Its algorithmic bytes are the plain step's
+    plus one more read of every input (the norm pass reads g, p, m, v
+    [, m2] and writes nothing)."""
+    import torch
+    from elementwise_optimizer_b200 import binding as B
+    dev = torch.device("cuda")
+    peak, kind = measured_peak()
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+    read_bytes = {("adam", "f32"): 16, ("ademamix", "f32"): 20,
+                  ("adam", "bf16"): 12, ("ademamix", "bf16"): 16}
+    rows = []
+    for algo, dt in (("adam", "f32"), ("ademamix", "bf16")):
+        p = torch.randn(numel, device=dev).to(tdt[dt])
+        grads = [(torch.randn(numel, device=dev) * 1e-2).to(tdt[dt]) for _ in range(2)]
+        s1 = torch.zeros(2 * numel if algo == "ademamix" else numel, device=dev)
+        s2 = torch.zeros(numel, device=dev)
+        lists = [B.TensorList.from_tensors([p], [g], [s1], [s2]) for g in grads]
+        h = B.make_hyper(algo, weight_decay=0.01, beta3=0.9999, alpha=5.0)
+        row = {"algo": algo, "dtype": dt, "max_unorm": max_unorm}
+        for name, fn in (("plain", lambda k, t: B.opt2s_step(lists[k % 2], h, t)),
+                         ("max_unorm", lambda k, t: B.opt2s_step_max_unorm(lists[k % 2], h,
+                                                                            max_unorm, t))):
+            for t in range(1, warmup + 1):
+                fn(t, t)
+            torch.cuda.synchronize()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+            ev[0].record()
+            for k in range(steps):
+                fn(k, warmup + 1 + k)
+                ev[k + 1].record()
+            torch.cuda.synchronize()
+            ms = sum(ev[k].elapsed_time(ev[k + 1]) for k in range(steps)) / steps
+            per_elem = BYTES_PER_ELEM[(algo, dt)] + (read_bytes[(algo, dt)] if name == "max_unorm" else 0)
+            gbs = per_elem * numel / (ms / 1e3) / 1e9
+            row[name] = {"ms_mean": ms, "bytes_per_elem": per_elem, "gbs": gbs, "frac": gbs / peak}
+        row["time_ratio"] = row["max_unorm"]["ms_mean"] / row["plain"]["ms_mean"]
+        row["byte_ratio"] = row["max_unorm"]["bytes_per_elem"] / row["plain"]["bytes_per_elem"]
+        rows.append(row)
+        del p, grads, s1, s2, lists
+        B.opt2s_release_cache()
+        torch.cuda.empty_cache()
+    return {"mode": "max-unorm", "numel": numel, "peak_gbs": peak, "peak_source": kind,
+            "rows": rows}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -830,7 +878,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the small-collection, e2e and cpu_baseline legs")
-    ap.add_argument("--mode", choices=["headline", "direct-cells", "eager-collection",
+    ap.add_argument("--mode", choices=["headline", "direct-cells", "eager-collection", "max-unorm",
                                        "shard-emulated", "roofline-table"],
                     default="headline",
                     help="headline: the one-line bench; the others follow the issue's "
@@ -852,7 +900,7 @@ def main():
         torch.cuda.set_device(local_rank)
         res = {"direct-cells": run_direct_cells, "eager-collection": run_eager_collection,
                "shard-emulated": run_shard_emulated,
-               "roofline-table": run_roofline_table}[args.mode]()
+               "roofline-table": run_roofline_table, "max-unorm": run_max_unorm}[args.mode]()
         res["env"] = environment()
         print(json.dumps(res), flush=True)
         return

@@ -91,6 +91,8 @@ EXPORTS = {
     "opt2s_step_noalloc": (ctypes.c_int, [ctypes.POINTER(TensorListDesc), ctypes.POINTER(Hyper),
                                           ctypes.c_int, ctypes.c_void_p]),
     "opt2s_noalloc_max_chunks": (ctypes.c_int64, []),
+    "opt2s_step_max_unorm": (ctypes.c_int, [ctypes.POINTER(TensorListDesc), ctypes.POINTER(Hyper),
+                                            ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
     "opt2s_fill_step_scalars": (ctypes.c_int, [ctypes.POINTER(Hyper), ctypes.c_int, ctypes.c_int,
                                                ctypes.c_void_p]),
     "opt2s_plan_step_table": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
@@ -250,6 +252,15 @@ def opt2s_step_noalloc(tl: TensorList, hyper: Hyper, step: int, stream=None) -> 
     calls that overlap on the GPU race on the shared table."""
     check(lib().opt2s_step_noalloc(ctypes.byref(tl.desc), ctypes.byref(hyper), int(step),
                                    _stream_handle(stream)), "opt2s_step_noalloc")
+
+
+def opt2s_step_max_unorm(tl: TensorList, hyper: Hyper, max_unorm: float, step: int,
+                         stream=None) -> None:
+    """opt2s_step with each tensor's update norm bounded by max_unorm times
+    its weight norm (max_unorm > 0); three launches on `stream`."""
+    check(lib().opt2s_step_max_unorm(ctypes.byref(tl.desc), ctypes.byref(hyper),
+                                     float(max_unorm), int(step), _stream_handle(stream)),
+          "opt2s_step_max_unorm")
 
 
 def noalloc_max_chunks() -> int:

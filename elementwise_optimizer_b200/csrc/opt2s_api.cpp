@@ -37,6 +37,12 @@ struct opt2s_plan {
     int32_t only;         // dtype all chunks share (specialised kernel), or -1
     int64_t nchunks;
     ChunkRec* d_chunks;   // device copy of the chunk table
+    // Bounded-update-norm workspace (plans made for opt2s_step_max_unorm
+    // only): one device allocation holding the norm table, the per-block
+    // sums, the tensors' first blocks, the per-tensor scales and the
+    // chunk-to-tensor map.
+    void* d_unorm;
+    opt2s::UnormArgs unorm;
 };
 
 namespace {
@@ -232,7 +238,65 @@ std::vector<ChunkRec> build_chunk_table(const TensorListDesc* d, int64_t chunk_e
     return out;
 }
 
-int plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out)
+// Builds the bounded-update-norm workspace of `plan` for `desc` (host tables,
+// then one device allocation and three uploads).
+int unorm_workspace(const TensorListDesc* desc, int64_t chunk_elems, opt2s_plan* plan)
+{
+    using opt2s::kNormBlockElems;
+    if (count_chunks(desc, kNormBlockElems) > INT32_MAX) return OPT2S_ERR_TOO_LARGE;
+    std::vector<ChunkRec> blocks = build_chunk_table(desc, kNormBlockElems, false);
+    std::vector<uint32_t> first(static_cast<size_t>(desc->count) + 1, 0);
+    for (int32_t i = 0; i < desc->count; ++i)
+        first[i + 1] = first[i] + static_cast<uint32_t>(
+            (desc->tensors[i].numel + kNormBlockElems - 1) / kNormBlockElems);
+    std::vector<uint32_t> chunk_tensor;
+    chunk_tensor.reserve(static_cast<size_t>(plan->nchunks));
+    for_each_chunk(desc, chunk_elems, [&](int32_t i, const opt2s_tensor&, int64_t, int64_t) {
+        chunk_tensor.push_back(static_cast<uint32_t>(i));
+    });
+    // layout: blocks | partial (2 doubles each) | first | scale | chunk_tensor
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t b_bytes = up(blocks.size() * sizeof(ChunkRec));
+    const size_t p_bytes = up(blocks.size() * 2 * sizeof(double));
+    const size_t f_bytes = up(first.size() * sizeof(uint32_t));
+    const size_t s_bytes = up(static_cast<size_t>(desc->count) * sizeof(float));
+    const size_t c_bytes = up(chunk_tensor.size() * sizeof(uint32_t));
+    const size_t total = b_bytes + p_bytes + f_bytes + s_bytes + c_bytes;
+    cudaError_t e;
+    if (g_fail_allocs.load() > 0 && g_fail_allocs.fetch_sub(1) > 0)
+        e = cudaErrorMemoryAllocation;                // injected by the test scaffolding
+    else
+        e = cudaMalloc(&plan->d_unorm, total);
+    if (e != cudaSuccess) {
+        plan->d_unorm = nullptr;
+        if (e == cudaErrorMemoryAllocation) { t_last_cuda_error = e; return OPT2S_ERR_NO_MEMORY; }
+        return cuda_fail(e);
+    }
+    char* base = static_cast<char*>(plan->d_unorm);
+    opt2s::UnormArgs& u = plan->unorm;
+    u.blocks = reinterpret_cast<ChunkRec*>(base);
+    u.nblocks = static_cast<int64_t>(blocks.size());
+    u.partial = reinterpret_cast<double*>(base + b_bytes);
+    u.first_block = reinterpret_cast<uint32_t*>(base + b_bytes + p_bytes);
+    u.ntensors = desc->count;
+    u.scale = reinterpret_cast<float*>(base + b_bytes + p_bytes + f_bytes);
+    u.chunk_tensor = reinterpret_cast<uint32_t*>(base + b_bytes + p_bytes + f_bytes + s_bytes);
+    if (!blocks.empty())
+        e = cudaMemcpy(const_cast<ChunkRec*>(u.blocks), blocks.data(), blocks.size() * sizeof(ChunkRec),
+                       cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(const_cast<uint32_t*>(u.first_block), first.data(), first.size() * sizeof(uint32_t),
+                       cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !chunk_tensor.empty())
+        e = cudaMemcpy(const_cast<uint32_t*>(u.chunk_tensor), chunk_tensor.data(),
+                       chunk_tensor.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return OPT2S_OK;
+}
+
+int plan_destroy(opt2s_plan* plan);
+
+int plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out, bool unorm = false)
 {
     int st = validate_desc(desc, algo);
     if (st != OPT2S_OK) return st;
@@ -244,7 +308,8 @@ int plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out)
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
-    auto* plan = new (std::nothrow) opt2s_plan{dev, algo, only, static_cast<int64_t>(table.size()), nullptr};
+    auto* plan = new (std::nothrow) opt2s_plan{dev, algo, only, static_cast<int64_t>(table.size()), nullptr,
+                                               nullptr, opt2s::UnormArgs{}};
     if (!plan) return OPT2S_ERR_NO_MEMORY;
     if (!table.empty()) {
         const size_t bytes = table.size() * sizeof(ChunkRec);
@@ -264,6 +329,15 @@ int plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out)
             return cuda_fail(e);
         }
     }
+    if (unorm) {
+        st = unorm_workspace(desc, ce, plan);
+        if (st != OPT2S_OK) {
+            const int keep = t_last_cuda_error;
+            plan_destroy(plan);
+            t_last_cuda_error = keep;
+            return st;
+        }
+    }
     *out = plan;
     return OPT2S_OK;
 }
@@ -272,12 +346,13 @@ int plan_destroy(opt2s_plan* plan)
 {
     if (!plan) return OPT2S_OK;
     int st = OPT2S_OK;
-    if (plan->d_chunks) {
+    if (plan->d_chunks || plan->d_unorm) {
         int cur = -1;
         cudaError_t e = cudaGetDevice(&cur);
         const bool switched = e == cudaSuccess && cur != plan->device;
         if (switched) e = cudaSetDevice(plan->device);
-        if (e == cudaSuccess) e = cudaFree(plan->d_chunks);   // waits for the device
+        if (e == cudaSuccess && plan->d_chunks) e = cudaFree(plan->d_chunks);   // waits for the device
+        if (e == cudaSuccess && plan->d_unorm) e = cudaFree(plan->d_unorm);
         if (e != cudaSuccess) st = cuda_fail(e);
         if (switched) cudaSetDevice(cur);
     }
@@ -336,6 +411,7 @@ struct CacheEntry {
     int device;
     int32_t algo;
     int64_t chunk_elems;
+    bool unorm;                  // plan carries the bounded-update-norm workspace
     std::vector<opt2s_tensor> records;
     opt2s_plan* plan;
 };
@@ -364,6 +440,78 @@ bool all_empty(const TensorListDesc* d)
 // Public entry points
 // ---------------------------------------------------------------------------
 
+namespace {
+
+// The cached plan for `desc` on the current device (made on a miss); the
+// caller holds g_cache_mu.  Argument errors are reported before device errors.
+int cached_plan(const TensorListDesc* desc, int32_t algo, bool unorm, const opt2s_plan** out)
+{
+    int dev = 0;
+    const int64_t ce = g_chunk_elems;   // part of the cache key: 0 = chosen per plan
+    // a cache hit needs no device query: compare on the device of the most
+    // recent entries first, then confirm the current device
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        // no usable device: still report argument errors first
+        int vs = validate_desc(desc, algo);
+        if (vs != OPT2S_OK) return vs;
+        if (all_empty(desc)) { *out = nullptr; return OPT2S_OK; }
+        return cuda_fail(e);
+    }
+    for (auto it = g_cache.begin(); it != g_cache.end(); ++it) {
+        if (it->device == dev && it->algo == algo && it->chunk_elems == ce && it->unorm == unorm &&
+            same_records(*it, desc)) {
+            if (it != g_cache.begin()) g_cache.splice(g_cache.begin(), g_cache, it);
+            *out = g_cache.front().plan;
+            return OPT2S_OK;
+        }
+    }
+    opt2s_plan* fresh = nullptr;
+    int st = plan_create(desc, algo, &fresh, unorm);
+    if (st != OPT2S_OK) return st;
+    CacheEntry entry{dev, algo, ce, unorm,
+                     std::vector<opt2s_tensor>(desc->tensors, desc->tensors + desc->count), fresh};
+    g_cache.push_front(std::move(entry));
+    while (g_cache.size() > kCacheCapacity) {
+        plan_destroy(g_cache.back().plan);
+        g_cache.pop_back();
+    }
+    *out = fresh;
+    return OPT2S_OK;
+}
+
+int plan_step_max_unorm(const opt2s_plan* plan, const Hyper* h, float max_unorm, int step,
+                        cudaStream_t stream)
+{
+    if (!plan) return OPT2S_ERR_INVALID_ARG;
+    int st = validate_hyper(h, step);
+    if (st != OPT2S_OK) return st;
+    if (!std::isfinite(max_unorm) || !(max_unorm > 0.0f)) return OPT2S_ERR_INVALID_ARG;
+    if (h->algo != plan->algo) return OPT2S_ERR_INVALID_ARG;
+    if (plan->nchunks == 0) return OPT2S_OK;
+    if (!plan->d_unorm) return OPT2S_ERR_INVALID_ARG;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev != plan->device) return OPT2S_ERR_DEVICE;
+    const int bt = block_threads_now(h->algo, -1);
+    if (g_block_threads > 0) {   // forced geometry: must fit the kernel
+        int widest = 0;
+        e = opt2s::max_block_threads_scaled(h->algo, h->skip_zeros, &widest);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (bt > widest) return OPT2S_ERR_INVALID_ARG;
+    }
+    e = opt2s::launch_step_max_unorm(plan->d_chunks, plan->nchunks, h->algo, h->skip_zeros,
+                                     make_scalars(h, step), plan->unorm, max_unorm, bt,
+                                     g_max_blocks, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    const int launched = (plan->unorm.nblocks > 0) + (plan->unorm.ntensors > 0) + 1;
+    g_launches.fetch_add(launched, std::memory_order_relaxed);
+    return OPT2S_OK;
+}
+
+}  // namespace
+
 OPT2S_API int opt2s_step(const TensorListDesc* desc, const Hyper* hyper, int step,
                          cudaStream_t stream)
 {
@@ -372,45 +520,27 @@ OPT2S_API int opt2s_step(const TensorListDesc* desc, const Hyper* hyper, int ste
     if (!desc || desc->count < 0 || (desc->count > 0 && !desc->tensors))
         return OPT2S_ERR_INVALID_ARG;
     if (desc->count == 0) return OPT2S_OK;
-
-    int dev = 0;
-    const int64_t ce = g_chunk_elems;   // part of the cache key: 0 = chosen per plan
     std::unique_lock<std::mutex> lock(g_cache_mu);
     const opt2s_plan* plan = nullptr;
-    {
-        // a cache hit needs no device query: compare on the device of the
-        // most recent entries first, then confirm the current device
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e != cudaSuccess) {
-            // no usable device: still report argument errors first
-            int vs = validate_desc(desc, hyper->algo);
-            if (vs != OPT2S_OK) return vs;
-            if (all_empty(desc)) return OPT2S_OK;
-            return cuda_fail(e);
-        }
-        for (auto it = g_cache.begin(); it != g_cache.end(); ++it) {
-            if (it->device == dev && it->algo == hyper->algo && it->chunk_elems == ce &&
-                same_records(*it, desc)) {
-                if (it != g_cache.begin()) g_cache.splice(g_cache.begin(), g_cache, it);
-                plan = g_cache.front().plan;
-                break;
-            }
-        }
-    }
-    if (!plan) {
-        opt2s_plan* fresh = nullptr;
-        st = plan_create(desc, hyper->algo, &fresh);
-        if (st != OPT2S_OK) return st;
-        CacheEntry entry{dev, hyper->algo, ce,
-                         std::vector<opt2s_tensor>(desc->tensors, desc->tensors + desc->count), fresh};
-        g_cache.push_front(std::move(entry));
-        while (g_cache.size() > kCacheCapacity) {
-            plan_destroy(g_cache.back().plan);
-            g_cache.pop_back();
-        }
-        plan = fresh;
-    }
+    st = cached_plan(desc, hyper->algo, false, &plan);
+    if (st != OPT2S_OK || !plan) return st;
     return plan_step(plan, hyper, step, stream);
+}
+
+OPT2S_API int opt2s_step_max_unorm(const TensorListDesc* desc, const Hyper* hyper, float max_unorm,
+                                   int step, cudaStream_t stream)
+{
+    int st = validate_hyper(hyper, step);
+    if (st != OPT2S_OK) return st;
+    if (!std::isfinite(max_unorm) || !(max_unorm > 0.0f)) return OPT2S_ERR_INVALID_ARG;
+    if (!desc || desc->count < 0 || (desc->count > 0 && !desc->tensors))
+        return OPT2S_ERR_INVALID_ARG;
+    if (desc->count == 0) return OPT2S_OK;
+    std::unique_lock<std::mutex> lock(g_cache_mu);
+    const opt2s_plan* plan = nullptr;
+    st = cached_plan(desc, hyper->algo, true, &plan);
+    if (st != OPT2S_OK || !plan) return st;
+    return plan_step_max_unorm(plan, hyper, max_unorm, step, stream);
 }
 
 OPT2S_API int opt2s_plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out_plan)

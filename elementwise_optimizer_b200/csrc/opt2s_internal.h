@@ -99,6 +99,33 @@ cudaError_t launch_step(const ChunkRec* d_chunks, int64_t nchunks, int algo,
                         int block_threads, int max_blocks,
                         cudaStream_t stream);
 
+// The bounded-update-norm step (max_unorm > 0).  Device arrays, all owned
+// by the plan: `blocks` is the norm table (each tensor cut into blocks of
+// kNormBlockElems elements, in descriptor order), tensor t owns blocks
+// [first_block[t], first_block[t + 1]); `partial` holds two doubles per block,
+// `scale` one float per tensor, and chunk_tensor[c] is the tensor of the
+// plan's chunk c.
+constexpr int64_t kNormBlockElems = 2048;
+struct UnormArgs {
+    const ChunkRec* blocks;
+    int64_t nblocks;
+    const uint32_t* first_block;   // ntensors + 1 entries
+    int32_t ntensors;
+    double* partial;               // 2 * nblocks
+    float* scale;                  // ntensors
+    const uint32_t* chunk_tensor;  // one per chunk of the plan
+};
+
+// Launches the three kernels of the bounded-update-norm step on `stream`
+// (norm partials, per-tensor scales, the scaled step over the plan's chunks).
+cudaError_t launch_step_max_unorm(const ChunkRec* d_chunks, int64_t nchunks, int algo,
+                                  int skip_zeros, const StepScalars& s, const UnormArgs& u,
+                                  float max_unorm, int block_threads, int max_blocks,
+                                  cudaStream_t stream);
+
+// Widest block the scaled step kernel can launch with.
+cudaError_t max_block_threads_scaled(int algo, int skip_zeros, int* out);
+
 // Sets s->inv_bc1, s->inv_bc2 = RN64(1/bc1), RN64(1/bc2) (host).
 void fill_reciprocals(StepScalars* s);
 

@@ -72,15 +72,18 @@ __device__ __forceinline__ float div_by_constant(float x, double r)
 }
 
 // ---------------------------------------------------------------------------
-// The per-element update.  With SKIP, an element whose gradient compares equal
-// to zero (+0 or -0) is left untouched (no decay either).  m/bc1 and v/bc2 use
-// the exact constant division above; num/den is an IEEE division.
+// The per-element update.  direction() moves the moments of one element (in
+// place) and returns its update direction u = num/den; m/bc1 and v/bc2 use
+// the exact constant division above, num/den is an IEEE division.  update()
+// then applies p = p*decay - lr*u.  With SKIP, an element whose gradient
+// compares equal to zero (+0 or -0) is left untouched (no decay either).
+// SCALED (the bounded-update-norm step): p = p*decay - lr*(scale*u), which for
+// scale = 1 is the same value.
 // ---------------------------------------------------------------------------
-template <int ALGO, bool SKIP>
-__device__ __forceinline__ void update(float g, float& p, float& m, float& v,
-                                       float& m2, const StepScalars& s)
+template <int ALGO>
+__device__ __forceinline__ float direction(float g, float& m, float& v, float& m2,
+                                           const StepScalars& s)
 {
-    if (SKIP && g == 0.0f) return;
     m = __fadd_rn(__fmul_rn(s.beta1, m), __fmul_rn(s.one_minus_beta1, g));
     v = __fadd_rn(__fmul_rn(s.beta2, v),
                   __fmul_rn(__fmul_rn(s.one_minus_beta2, g), g));
@@ -90,7 +93,16 @@ __device__ __forceinline__ void update(float g, float& p, float& m, float& v,
         num = __fadd_rn(num, __fmul_rn(s.alpha, m2));
     }
     const float den = __fadd_rn(__fsqrt_rn(div_by_constant(v, s.inv_bc2)), s.eps);
-    p = __fsub_rn(__fmul_rn(p, s.decay), __fmul_rn(s.lr, __fdiv_rn(num, den)));
+    return __fdiv_rn(num, den);
+}
+
+template <int ALGO, bool SKIP, bool SCALED = false>
+__device__ __forceinline__ void update(float g, float& p, float& m, float& v,
+                                       float& m2, const StepScalars& s, float scale = 1.0f)
+{
+    if (SKIP && g == 0.0f) return;
+    const float u = direction<ALGO>(g, m, v, m2, s);
+    p = __fsub_rn(__fmul_rn(p, s.decay), __fmul_rn(s.lr, SCALED ? __fmul_rn(scale, u) : u));
 }
 
 // ---------------------------------------------------------------------------
@@ -247,9 +259,9 @@ __device__ __forceinline__ void store_state(float* b, uint32_t i, const float (&
 // One element through the scalar path (chunk head, tail, or a chunk whose
 // arrays are not mutually 16-byte aligned).  A skipped element is not even
 // written back.
-template <int DT, int ALGO, bool SKIP>
+template <int DT, int ALGO, bool SKIP, bool SCALED = false>
 __device__ __forceinline__ void scalar_element(const ChunkRec& c, uint32_t i,
-                                               const StepScalars& s)
+                                               const StepScalars& s, float scale = 1.0f)
 {
     using P = Param<DT>;
     const float g = P::load1(c.g, i);
@@ -259,7 +271,7 @@ __device__ __forceinline__ void scalar_element(const ChunkRec& c, uint32_t i,
     float v = ld_global(c.v + i);
     float m2 = 0.0f;
     if (ALGO == kAdEMAMix) m2 = ld_global(c.m2 + i);
-    update<ALGO, false>(g, p, m, v, m2, s);
+    update<ALGO, false, SCALED>(g, p, m, v, m2, s, scale);
     P::store1(c.p, i, p);
     st_global(c.m + i, m);
     st_global(c.v + i, v);
@@ -283,9 +295,10 @@ struct Aligned {
 // elements per iteration (two 16-byte vectors of fp32, or one of fp16/bf16),
 // so a warp iteration covers 256 contiguous elements of each array; the mixed
 // case moves one vector per lane per iteration.
-template <int DT, int ALGO, bool SKIP, bool ALL>
+template <int DT, int ALGO, bool SKIP, bool ALL, bool SCALED = false>
 __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars& s, int lane,
-                                            uint32_t head, uint32_t nvec, Aligned al)
+                                            uint32_t head, uint32_t nvec, Aligned al,
+                                            float scale = 1.0f)
 {
     using P = Param<DT>;
     constexpr int V = P::kVec;
@@ -316,7 +329,7 @@ __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars
                 P::widen(praw[u], p);
 #pragma unroll
                 for (int j = 0; j < V; ++j)
-                    update<ALGO, SKIP>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s);
+                    update<ALGO, SKIP, SCALED>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s, scale);
                 P::store(c.p, e, P::narrow(p, praw[u], g, SKIP));
                 store_state_any<V>(c.m, e, ALL || al.m, m[u]);
                 store_state_any<V>(c.v, e, ALL || al.v, v[u]);
@@ -328,8 +341,9 @@ __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars
 
 // One chunk, processed by one warp: a scalar head up to the element at which
 // param is 16-byte aligned, the vector body, and a scalar tail.
-template <int DT, int ALGO, bool SKIP>
-__device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& s, int lane)
+template <int DT, int ALGO, bool SKIP, bool SCALED = false>
+__device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& s, int lane,
+                                          float scale = 1.0f)
 {
     using P = Param<DT>;
     constexpr int V = P::kVec;
@@ -340,15 +354,17 @@ __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& 
     const uint32_t nvec = (len - head) / V;
     const uint32_t body_end = head + nvec * V;
 
-    for (uint32_t i = lane; i < head; i += 32) scalar_element<DT, ALGO, SKIP>(c, i, s);
-    for (uint32_t i = body_end + lane; i < len; i += 32) scalar_element<DT, ALGO, SKIP>(c, i, s);
+    for (uint32_t i = lane; i < head; i += 32)
+        scalar_element<DT, ALGO, SKIP, SCALED>(c, i, s, scale);
+    for (uint32_t i = body_end + lane; i < len; i += 32)
+        scalar_element<DT, ALGO, SKIP, SCALED>(c, i, s, scale);
 
     const Aligned al{aligned16(c.g, head, P::kBytes), aligned16(c.m, head, 4),
                      aligned16(c.v, head, 4), ALGO != kAdEMAMix || aligned16(c.m2, head, 4)};
     if (al.all())
-        vector_body<DT, ALGO, SKIP, true>(c, s, lane, head, nvec, al);
+        vector_body<DT, ALGO, SKIP, true, SCALED>(c, s, lane, head, nvec, al, scale);
     else
-        vector_body<DT, ALGO, SKIP, false>(c, s, lane, head, nvec, al);
+        vector_body<DT, ALGO, SKIP, false, SCALED>(c, s, lane, head, nvec, al, scale);
 }
 
 // A short 16-bit chunk (its record's dtype carries kShortFlag), processed by
@@ -616,6 +632,134 @@ __global__ void advance_index_kernel(int* index, int table_len)
     *index = (idx >= 0 && idx + 1 < table_len) ? idx + 1 : -1;
 }
 
+// ---------------------------------------------------------------------------
+// The step with bounded update norms (max_unorm > 0), three launches:
+//   1. unorm_partials_kernel: for every block of kNormBlockElems elements of
+//      a tensor (the host's norm table, fixed blocks whatever the plan's
+//      chunk length), the binary64 sums of u^2 (u = num/den, the update
+//      direction; 0 for an element skip_zeros leaves alone) and of p^2 (p
+//      the param before the step).  Nothing is written but the two sums;
+//   2. unorm_scale_kernel: per tensor, the sums of its blocks, U = sqrt(su),
+//      P = sqrt(sp), and scale = max_unorm*P/U if U > max_unorm*P, else 1
+//      (binary64, rounded to fp32 once);
+//   3. step_kernel_scaled: the step over the plan's chunks with
+//      p = p*decay - lr*(scale*u), scale read through the chunk's tensor.
+// The element arithmetic is direction(), as in the plain step.  Every sum
+// has a fixed order: lane l of the warp that owns a block adds the block's
+// elements l, l + 32, l + 64, ... one after the other, the 32 lanes then
+// combine in a fixed shuffle tree, and a tensor's blocks are combined the
+// same way; so the scale does not depend on the plan's chunk length, the
+// block width or the storage alignment.  Accesses are element-wise and
+// contiguous across the warp.
+// ---------------------------------------------------------------------------
+template <int DT, int ALGO, bool SKIP>
+__device__ __forceinline__ void norm_block(const ChunkRec& c, const StepScalars& s, int lane,
+                                           double& su, double& sp)
+{
+    using P = Param<DT>;
+    constexpr int K = 8;
+    const uint32_t len = c.len;
+    for (uint32_t base = 0; base < len; base += 32 * K) {
+        float g[K], p[K], m[K], v[K], m2[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            const uint32_t i = base + lane + 32 * k;
+            g[k] = p[k] = m[k] = v[k] = m2[k] = 0.0f;
+            if (i < len) {
+                g[k] = P::load1(c.g, i);
+                p[k] = P::load1(c.p, i);
+                m[k] = ld_global(c.m + i);
+                v[k] = ld_global(c.v + i);
+                if (ALGO == kAdEMAMix) m2[k] = ld_global(c.m2 + i);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            if (base + lane + 32 * k < len) {
+                sp = __dadd_rn(sp, __dmul_rn(static_cast<double>(p[k]), static_cast<double>(p[k])));
+                if (!(SKIP && g[k] == 0.0f)) {
+                    const float u = direction<ALGO>(g[k], m[k], v[k], m2[k], s);
+                    su = __dadd_rn(su, __dmul_rn(static_cast<double>(u), static_cast<double>(u)));
+                }
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void warp_tree_sum(double& a, double& b)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        a = __dadd_rn(a, __shfl_down_sync(0xffffffffu, a, off));
+        b = __dadd_rn(b, __shfl_down_sync(0xffffffffu, b, off));
+    }
+}
+
+template <int ALGO, bool SKIP>
+__global__ void unorm_partials_kernel(const ChunkRec* __restrict__ blocks, int nblocks,
+                                      StepScalars s, double2* __restrict__ partial)
+{
+    const int lane = threadIdx.x & 31;
+    const int warps_per_block = blockDim.x >> 5;
+    const int warp = blockIdx.x * warps_per_block + (threadIdx.x >> 5);
+    const int nwarps = gridDim.x * warps_per_block;
+    for (int b = warp; b < nblocks; b += nwarps) {
+        const ChunkRec rec = blocks[b];
+        double su = 0.0, sp = 0.0;
+        switch (rec.dtype & ~kShortFlag) {
+        case kF32: norm_block<kF32, ALGO, SKIP>(rec, s, lane, su, sp); break;
+        case kF16: norm_block<kF16, ALGO, SKIP>(rec, s, lane, su, sp); break;
+        default: norm_block<kBF16, ALGO, SKIP>(rec, s, lane, su, sp); break;
+        }
+        warp_tree_sum(su, sp);
+        if (lane == 0) partial[b] = make_double2(su, sp);
+    }
+}
+
+// One warp per tensor; tensor t owns blocks [first[t], first[t + 1]).
+__global__ void unorm_scale_kernel(const double2* __restrict__ partial,
+                                   const uint32_t* __restrict__ first, int ntensors,
+                                   float max_unorm, float* __restrict__ scale)
+{
+    const int lane = threadIdx.x & 31;
+    const int warps_per_block = blockDim.x >> 5;
+    const int nwarps = gridDim.x * warps_per_block;
+    for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < ntensors; t += nwarps) {
+        double su = 0.0, sp = 0.0;
+        for (uint32_t b = first[t] + lane; b < first[t + 1]; b += 32) {
+            const double2 x = partial[b];
+            su = __dadd_rn(su, x.x);
+            sp = __dadd_rn(sp, x.y);
+        }
+        warp_tree_sum(su, sp);
+        if (lane == 0) {
+            const double U = __dsqrt_rn(su), P = __dsqrt_rn(sp);
+            const double limit = __dmul_rn(static_cast<double>(max_unorm), P);
+            scale[t] = U > limit ? __double2float_rn(__ddiv_rn(limit, U)) : 1.0f;
+        }
+    }
+}
+
+template <int ALGO, bool SKIP>
+__global__ void step_kernel_scaled(const ChunkRec* __restrict__ chunks, int nchunks,
+                                   StepScalars s, const uint32_t* __restrict__ chunk_tensor,
+                                   const float* __restrict__ scale)
+{
+    const int lane = threadIdx.x & 31;
+    const int warps_per_block = blockDim.x >> 5;
+    const int warp = blockIdx.x * warps_per_block + (threadIdx.x >> 5);
+    const int nwarps = gridDim.x * warps_per_block;
+    for (int c = warp; c < nchunks; c += nwarps) {
+        const ChunkRec rec = chunks[c];
+        const float sc = scale[chunk_tensor[c]];
+        switch (rec.dtype & ~kShortFlag) {
+        case kF32: run_chunk<kF32, ALGO, SKIP, true>(rec, s, lane, sc); break;
+        case kF16: run_chunk<kF16, ALGO, SKIP, true>(rec, s, lane, sc); break;
+        default: run_chunk<kBF16, ALGO, SKIP, true>(rec, s, lane, sc); break;
+        }
+    }
+}
+
 using KernelFn = void (*)(const ChunkRec*, int, StepScalars);
 using TableKernelFn = void (*)(const ChunkRec*, int, const StepScalars*, const int*, int);
 
@@ -852,6 +996,110 @@ cudaError_t launch_step_table(const ChunkRec* d_chunks, int64_t nchunks, int alg
     void* args2[] = {&d_index, &table_len};
     return cudaLaunchKernel(reinterpret_cast<const void*>(advance_index_kernel), dim3(1), dim3(1),
                             args2, 0, stream);
+}
+
+namespace {
+
+// Resident blocks per SM of one of the max_unorm kernels at block_threads,
+// cached per device.
+struct UnormOcc { const void* fn; int block_threads; int per_sm; };
+UnormOcc g_unorm_occ[kMaxDevices][24];
+
+cudaError_t unorm_grid(const void* fn, int64_t warps_needed, int block_threads, int* grid)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(g_info_mu);
+    DeviceInfo* info = nullptr;
+    if ((e = device_info(dev, &info)) != cudaSuccess) return e;
+    int per_sm = 0;
+    for (auto& x : g_unorm_occ[dev])
+        if (x.fn == fn && x.block_threads == block_threads) per_sm = x.per_sm;
+    if (per_sm == 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, block_threads, 0);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) per_sm = 1;
+        for (auto& x : g_unorm_occ[dev])
+            if (x.fn == nullptr) { x = UnormOcc{fn, block_threads, per_sm}; break; }
+    }
+    const int64_t warps_per_block = block_threads / 32;
+    const int64_t need = (warps_needed + warps_per_block - 1) / warps_per_block;
+    const int64_t cap = static_cast<int64_t>(per_sm) * info->sms;
+    *grid = static_cast<int>(need < cap ? need : cap);
+    return cudaSuccess;
+}
+
+template <int ALGO, bool SKIP>
+cudaError_t launch_unorm_typed(const ChunkRec* d_chunks, int64_t nchunks, const StepScalars& sc,
+                               const UnormArgs& u, float max_unorm, int block_threads,
+                               int max_blocks, cudaStream_t stream)
+{
+    constexpr int kNormThreads = 256;
+    int grid = 0;
+    cudaError_t e = cudaSuccess;
+    if (u.nblocks > 0) {
+        const void* k1 = reinterpret_cast<const void*>(unorm_partials_kernel<ALGO, SKIP>);
+        if ((e = unorm_grid(k1, u.nblocks, kNormThreads, &grid)) != cudaSuccess) return e;
+        unorm_partials_kernel<ALGO, SKIP><<<grid, kNormThreads, 0, stream>>>(
+            u.blocks, static_cast<int>(u.nblocks), sc, reinterpret_cast<double2*>(u.partial));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (u.ntensors > 0) {
+        const void* k2 = reinterpret_cast<const void*>(unorm_scale_kernel);
+        if ((e = unorm_grid(k2, u.ntensors, kNormThreads, &grid)) != cudaSuccess) return e;
+        unorm_scale_kernel<<<grid, kNormThreads, 0, stream>>>(
+            reinterpret_cast<const double2*>(u.partial), u.first_block, u.ntensors, max_unorm,
+            u.scale);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (nchunks > 0) {
+        const void* k3 = reinterpret_cast<const void*>(step_kernel_scaled<ALGO, SKIP>);
+        if (max_blocks > 0) {
+            const int64_t need = (nchunks + block_threads / 32 - 1) / (block_threads / 32);
+            grid = static_cast<int>(need < max_blocks ? need : max_blocks);
+        } else if ((e = unorm_grid(k3, nchunks, block_threads, &grid)) != cudaSuccess) {
+            return e;
+        }
+        step_kernel_scaled<ALGO, SKIP><<<grid, block_threads, 0, stream>>>(
+            d_chunks, static_cast<int>(nchunks), sc, u.chunk_tensor, u.scale);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_step_max_unorm(const ChunkRec* d_chunks, int64_t nchunks, int algo,
+                                  int skip_zeros, const StepScalars& s, const UnormArgs& u,
+                                  float max_unorm, int block_threads, int max_blocks,
+                                  cudaStream_t stream)
+{
+    StepScalars sc = s;
+    fill_reciprocals(&sc);
+    if (algo == kAdEMAMix)
+        return skip_zeros ? launch_unorm_typed<kAdEMAMix, true>(d_chunks, nchunks, sc, u, max_unorm,
+                                                                block_threads, max_blocks, stream)
+                          : launch_unorm_typed<kAdEMAMix, false>(d_chunks, nchunks, sc, u, max_unorm,
+                                                                 block_threads, max_blocks, stream);
+    return skip_zeros ? launch_unorm_typed<kAdam, true>(d_chunks, nchunks, sc, u, max_unorm,
+                                                        block_threads, max_blocks, stream)
+                      : launch_unorm_typed<kAdam, false>(d_chunks, nchunks, sc, u, max_unorm,
+                                                         block_threads, max_blocks, stream);
+}
+
+cudaError_t max_block_threads_scaled(int algo, int skip_zeros, int* out)
+{
+    cudaFuncAttributes attr{};
+    const void* fn = algo == kAdEMAMix
+        ? (skip_zeros ? reinterpret_cast<const void*>(step_kernel_scaled<kAdEMAMix, true>)
+                      : reinterpret_cast<const void*>(step_kernel_scaled<kAdEMAMix, false>))
+        : (skip_zeros ? reinterpret_cast<const void*>(step_kernel_scaled<kAdam, true>)
+                      : reinterpret_cast<const void*>(step_kernel_scaled<kAdam, false>));
+    cudaError_t e = cudaFuncGetAttributes(&attr, fn);
+    if (e != cudaSuccess) return e;
+    *out = attr.maxThreadsPerBlock / 32 * 32;
+    return cudaSuccess;
 }
 
 }  // namespace opt2s

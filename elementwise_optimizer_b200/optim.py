@@ -16,6 +16,13 @@ Python work, and zero_grad() zeroes the flat gradients in place (gradients
 must keep accumulating into those views: do not replace p.grad).  Results are
 the same bits as without flattening, since the update is elementwise.
 
+max_unorm > 0 bounds each parameter's update norm by max_unorm times its
+weight norm (opt2s_step_max_unorm: three launches per group and step).  With
+flatten=True the bound still applies per parameter: the flat buffers are
+stepped through one record per parameter, and AdEMAMix keeps each
+parameter's [m1 | m2] together in the flat state.  It is not combined with
+capturable=True.
+
 capturable=True routes every step through opt2s_plan_step_table: the per-step
 scalars live in a device table and the step index in device memory, so
 ``step()`` may be captured in a CUDA graph and each replay performs the next
@@ -34,14 +41,20 @@ class TwoStateOptimizer(torch.optim.Optimizer):
     def __init__(self, params, algo: str = "adamw", lr: float = 1e-3,
                  betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 0.0,
                  beta3: float = 0.9999, alpha: float = 5.0, skip_zeros: bool = False,
-                 capturable: bool = False, table_len: int = 1024, flatten: bool = False):
+                 capturable: bool = False, table_len: int = 1024, flatten: bool = False,
+                 max_unorm: float = 0.0):
         if algo not in B.ALGOS:
             raise ValueError(f"algo must be one of {sorted(B.ALGOS)}")
+        if not (0.0 <= max_unorm < float("inf")):
+            raise ValueError("max_unorm must be finite and >= 0 (0 disables the bound)")
+        if max_unorm > 0.0 and capturable:
+            raise ValueError("max_unorm and capturable are not combined")
         defaults = dict(lr=lr, betas=tuple(betas), eps=eps, weight_decay=weight_decay,
                         beta3=beta3, alpha=alpha, skip_zeros=skip_zeros)
         self.algo = "ademamix" if algo == "ademamix" else "adam"
         self.capturable = capturable
         self.table_len = int(table_len)
+        self.max_unorm = float(max_unorm)
         super().__init__(params, defaults)
         self._group_cache = {}
         self._flat = None
@@ -66,7 +79,12 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                 fg = torch.zeros(n, dtype=dt, device=dev)
                 fs1 = torch.zeros(2 * n if two else n, dtype=torch.float32, device=dev)
                 fs2 = torch.zeros(n, dtype=torch.float32, device=dev)
+                # per_param: one record per parameter (needed by the per-
+                # parameter norms of max_unorm); AdEMAMix then keeps each
+                # parameter's [m1 | m2] together, else all m1 before all m2
+                per_param = self.max_unorm > 0.0
                 off = 0
+                views = ([], [], [], [])
                 with torch.no_grad():
                     for p in ps:
                         k = p.numel()
@@ -76,15 +94,25 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                         p.data = fp[off:off + k].view_as(p)
                         p.grad = fg[off:off + k].view_as(p)
                         st = self.state[p]
-                        st["exp_avg"] = fs1[off:off + k].view_as(p)
+                        m1_at = 2 * off if (two and per_param) else off
+                        st["exp_avg"] = fs1[m1_at:m1_at + k].view_as(p)
                         st["exp_avg_sq"] = fs2[off:off + k].view_as(p)
                         if two:
-                            st["exp_avg_slow"] = fs1[n + off:n + off + k].view_as(p)
+                            m2_at = m1_at + k if per_param else n + off
+                            st["exp_avg_slow"] = fs1[m2_at:m2_at + k].view_as(p)
                         st["step"] = 0
+                        views[0].append(fp[off:off + k])
+                        views[1].append(fg[off:off + k])
+                        views[2].append(fs1[m1_at:m1_at + (2 * k if two else k)])
+                        views[3].append(fs2[off:off + k])
                         off += k
-                tl = B.TensorList.from_tensors([fp], [fg], [fs1], [fs2])
-                self._flat.append(dict(group=gi, params=ps, param=fp, grad=fg, state1=fs1,
-                                       state2=fs2, plan=B.Plan(tl, self.algo), step=0))
+                entry = dict(group=gi, params=ps, param=fp, grad=fg, state1=fs1, state2=fs2, step=0)
+                if per_param:
+                    entry["records"] = B.TensorList.from_tensors(*views)
+                else:
+                    tl = B.TensorList.from_tensors([fp], [fg], [fs1], [fs2])
+                    entry["plan"] = B.Plan(tl, self.algo)
+                self._flat.append(entry)
 
     def zero_grad(self, set_to_none: bool = True):
         if self._flat is None:
@@ -152,7 +180,11 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                 loss = closure()
         if self._flat is not None:
             for f in self._flat:
-                f["plan"].step(self._hyper(self.param_groups[f["group"]]), f["step"] + 1)
+                hyper = self._hyper(self.param_groups[f["group"]])
+                if "records" in f:
+                    B.opt2s_step_max_unorm(f["records"], hyper, self.max_unorm, f["step"] + 1)
+                else:
+                    f["plan"].step(hyper, f["step"] + 1)
                 f["step"] += 1
             return loss
         for gi, group in enumerate(self.param_groups):
@@ -162,6 +194,9 @@ class TwoStateOptimizer(torch.optim.Optimizer):
             if self.capturable:
                 data["plan"].step_table(group["skip_zeros"], data["table"].data_ptr(),
                                         self.table_len, data["index"].data_ptr())
+            elif self.max_unorm > 0.0:
+                B.opt2s_step_max_unorm(data["tl"], self._hyper(group), self.max_unorm,
+                                       data["step"] + 1)
             else:
                 B.opt2s_step(data["tl"], self._hyper(group), data["step"] + 1)
             data["step"] += 1

@@ -247,6 +247,39 @@ int opt2s_step_noalloc(const TensorListDesc *desc, const Hyper *hyper, int step,
 /* Capacity of opt2s_step_noalloc's fixed chunk table, in records. */
 int64_t opt2s_noalloc_max_chunks(void);
 
+/*
+ * The step with each tensor's update norm bounded: bitsandbytes' max_unorm
+ * option of the same two-state update (the issue's section "Scope" keeps its
+ * kernel for "max-unorm/LAMB use", and section "Correctness oracle" runs
+ * "max_unorm > 0" controls).  The pages name the option without its
+ * arithmetic; this library reads it as a bound on the norm of a tensor's
+ * update relative to the norm of its weights:
+ *
+ *     u_i = num_i/den_i, the update direction of element i in the step above
+ *           (0 for an element skip_zeros leaves alone)
+ *     U   = sqrt(sum_i u_i^2),  P = sqrt(sum_i p_i^2), p before the step,
+ *           over each tensor of the collection; binary64 squares and sums
+ *     s   = max_unorm*P/U if U > max_unorm*P, else 1  (binary64, rounded to
+ *           fp32 once)
+ *     p_i = p_i*decay - lr*(s*u_i), with m, v (and m2) as in the step above.
+ *
+ * s = 1 gives exactly opt2s_step's bits.  The sums have a fixed order (lane
+ * l of a warp adds elements l, l+32, ... of a 2,048-element block, then a
+ * fixed tree over lanes and over a tensor's blocks), so s does not depend on
+ * launch geometry or storage alignment; against a plain sequential binary64
+ * sum it can differ only when the ratio lies within a few binary64 ulp of an
+ * fp32 rounding boundary.
+ *
+ * max_unorm: finite and > 0 (else OPT2S_ERR_INVALID_ARG).  Other arguments
+ * and validation as opt2s_step.  Three launches on `stream`: the norm sums,
+ * the per-tensor scales, and the scaled update.  The tensor is read twice
+ * (once for the sums, once for the update).  Plans are cached like
+ * opt2s_step's, each with a workspace of 64 bytes per 2,048 elements plus
+ * 4 bytes per tensor and per chunk, freed by opt2s_release_cache().
+ */
+int opt2s_step_max_unorm(const TensorListDesc *desc, const Hyper *hyper, float max_unorm,
+                         int step, cudaStream_t stream);
+
 /* Frees every cached plan of every device (waits for the devices first). */
 int opt2s_release_cache(void);
 

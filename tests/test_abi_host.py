@@ -285,6 +285,32 @@ def test_step_without_device(L):
     B.opt2s_step(B.TensorList([(0, 0, 0, 0, 0, 0)]), H, 1, stream=0)
 
 
+def test_max_unorm_argument_checks(L):
+    """The bound must be finite and positive; this is checked before any
+    CUDA call, so it holds with or without a device."""
+    tl = B.TensorList(records([64]))
+    for mu in (0.0, -1.0, float("nan"), float("inf"), float("-inf")):
+        with pytest.raises(B.Opt2sError) as e:
+            B.opt2s_step_max_unorm(tl, H, mu, 1, stream=0)
+        assert e.value.status == -1, mu
+    with pytest.raises(B.Opt2sError) as e:
+        B.opt2s_step_max_unorm(tl, H, 1.0, 0, stream=0)
+    assert e.value.status == -1
+    B.opt2s_step_max_unorm(B.TensorList([]), H, 1.0, 1, stream=0)   # empty: no-op
+
+
+@pytest.mark.skipif(_cuda_available(), reason="checks the no-device path")
+def test_max_unorm_step_without_device(L):
+    tl = B.TensorList(records([64, 3000], ["f32", "bf16"]))
+    with pytest.raises(B.Opt2sError) as e:
+        B.opt2s_step_max_unorm(tl, H, 1.0, 1, stream=0)
+    assert e.value.status == -4                       # CUDA: no device
+    p, g, s1, s2, n, dt = records([64])[0]
+    with pytest.raises(B.Opt2sError) as e:            # argument errors still first
+        B.opt2s_step_max_unorm(B.TensorList([(p, g, s1, s1, n, dt)]), H, 1.0, 1, stream=0)
+    assert e.value.status == -2
+
+
 def test_missing_library_fails_loudly(tmp_path):
     code = ("import elementwise_optimizer_b200.binding as b; b.LIB_PATH='/nonexistent/x.so'\n"
             "try:\n  b.lib()\nexcept RuntimeError as e:\n  print('RAISED', e)\n")
