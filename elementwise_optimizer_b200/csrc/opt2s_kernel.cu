@@ -647,9 +647,9 @@ __global__ void advance_index_kernel(int* index, int table_len)
 // The element arithmetic is direction(), as in the plain step.  Every sum
 // has a fixed order: lane l of the warp that owns a block adds the block's
 // elements l, l + 32, l + 64, ... one after the other, the 32 lanes then
-// combine in a fixed shuffle tree, and a tensor's blocks are combined the
-// same way; so the scale does not depend on the plan's chunk length, the
-// block width or the storage alignment.  Accesses are element-wise and
+// combine in a fixed shuffle tree, and one CTA combines a tensor's blocks in
+// a fixed order too; so the scale does not depend on the plan's chunk length,
+// the block width or the storage alignment.  Accesses are element-wise and
 // contiguous across the warp.
 // ---------------------------------------------------------------------------
 template <int DT, int ALGO, bool SKIP>
@@ -716,27 +716,52 @@ __global__ void unorm_partials_kernel(const ChunkRec* __restrict__ blocks, int n
     }
 }
 
-// One warp per tensor; tensor t owns blocks [first[t], first[t + 1]).
-__global__ void unorm_scale_kernel(const double2* __restrict__ partial,
-                                   const uint32_t* __restrict__ first, int ntensors,
-                                   float max_unorm, float* __restrict__ scale)
+// One CTA of kScaleThreads threads per tensor (tensor t owns blocks
+// [first[t], first[t + 1])): thread j keeps four running sums, sum k taking
+// blocks j + (4i + k)*kScaleThreads for i = 0, 1, ... in turn (four chains of
+// loads in flight), then (s0 + s1) + (s2 + s3), then a fixed tree over lanes
+// and over the CTA's warps.  The order depends only on the tensor, not on the
+// grid.
+constexpr int kScaleThreads = 1024;
+
+__global__ void __launch_bounds__(kScaleThreads)
+unorm_scale_kernel(const double2* __restrict__ partial, const uint32_t* __restrict__ first,
+                   int ntensors, float max_unorm, float* __restrict__ scale)
 {
+    constexpr int kWarps = kScaleThreads / 32;
+    __shared__ double su_w[kWarps], sp_w[kWarps];
     const int lane = threadIdx.x & 31;
-    const int warps_per_block = blockDim.x >> 5;
-    const int nwarps = gridDim.x * warps_per_block;
-    for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < ntensors; t += nwarps) {
-        double su = 0.0, sp = 0.0;
-        for (uint32_t b = first[t] + lane; b < first[t + 1]; b += 32) {
-            const double2 x = partial[b];
-            su = __dadd_rn(su, x.x);
-            sp = __dadd_rn(sp, x.y);
+    const int w = threadIdx.x >> 5;
+    for (int t = blockIdx.x; t < ntensors; t += gridDim.x) {   // the same t for the whole CTA
+        double au[4] = {0.0, 0.0, 0.0, 0.0}, ap[4] = {0.0, 0.0, 0.0, 0.0};
+        const uint32_t end = first[t + 1];
+        for (uint32_t b = first[t] + threadIdx.x; b < end; b += 4 * kScaleThreads) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t i = b + k * kScaleThreads;
+                if (i < end) {
+                    const double2 x = partial[i];
+                    au[k] = __dadd_rn(au[k], x.x);
+                    ap[k] = __dadd_rn(ap[k], x.y);
+                }
+            }
         }
+        double su = __dadd_rn(__dadd_rn(au[0], au[1]), __dadd_rn(au[2], au[3]));
+        double sp = __dadd_rn(__dadd_rn(ap[0], ap[1]), __dadd_rn(ap[2], ap[3]));
         warp_tree_sum(su, sp);
-        if (lane == 0) {
-            const double U = __dsqrt_rn(su), P = __dsqrt_rn(sp);
-            const double limit = __dmul_rn(static_cast<double>(max_unorm), P);
-            scale[t] = U > limit ? __double2float_rn(__ddiv_rn(limit, U)) : 1.0f;
+        if (lane == 0) { su_w[w] = su; sp_w[w] = sp; }
+        __syncthreads();
+        if (w == 0) {
+            su = lane < kWarps ? su_w[lane] : 0.0;
+            sp = lane < kWarps ? sp_w[lane] : 0.0;
+            warp_tree_sum(su, sp);
+            if (lane == 0) {
+                const double U = __dsqrt_rn(su), P = __dsqrt_rn(sp);
+                const double limit = __dmul_rn(static_cast<double>(max_unorm), P);
+                scale[t] = U > limit ? __double2float_rn(__ddiv_rn(limit, U)) : 1.0f;
+            }
         }
+        __syncthreads();   // the shared sums are reused by the next tensor
     }
 }
 
@@ -1047,8 +1072,11 @@ cudaError_t launch_unorm_typed(const ChunkRec* d_chunks, int64_t nchunks, const 
     }
     if (u.ntensors > 0) {
         const void* k2 = reinterpret_cast<const void*>(unorm_scale_kernel);
-        if ((e = unorm_grid(k2, u.ntensors, kNormThreads, &grid)) != cudaSuccess) return e;
-        unorm_scale_kernel<<<grid, kNormThreads, 0, stream>>>(
+        // one CTA per tensor, up to the resident CTAs of the device
+        if ((e = unorm_grid(k2, static_cast<int64_t>(u.ntensors) * (kScaleThreads / 32), kScaleThreads,
+                            &grid)) != cudaSuccess)
+            return e;
+        unorm_scale_kernel<<<grid, kScaleThreads, 0, stream>>>(
             reinterpret_cast<const double2*>(u.partial), u.first_block, u.ntensors, max_unorm,
             u.scale);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -265,10 +265,10 @@ int64_t opt2s_noalloc_max_chunks(void);
  *
  * s = 1 gives exactly opt2s_step's bits.  The sums have a fixed order (lane
  * l of a warp adds elements l, l+32, ... of a 2,048-element block, then a
- * fixed tree over lanes and over a tensor's blocks), so s does not depend on
- * launch geometry or storage alignment; against a plain sequential binary64
- * sum it can differ only when the ratio lies within a few binary64 ulp of an
- * fp32 rounding boundary.
+ * fixed tree over lanes; one CTA adds a tensor's blocks in a fixed order),
+ * so s does not depend on launch geometry or storage alignment; against a
+ * plain sequential binary64 sum it can differ only when the ratio lies
+ * within a few binary64 ulp of an fp32 rounding boundary.
  *
  * max_unorm: finite and > 0 (else OPT2S_ERR_INVALID_ARG).  Other arguments
  * and validation as opt2s_step.  Three launches on `stream`: the norm sums,
