@@ -257,7 +257,7 @@ def opt2s_step_noalloc(tl: TensorList, hyper: Hyper, step: int, stream=None) -> 
 def opt2s_step_max_unorm(tl: TensorList, hyper: Hyper, max_unorm: float, step: int,
                          stream=None) -> None:
     """opt2s_step with each tensor's update norm bounded by max_unorm times
-    its weight norm (max_unorm > 0); three launches on `stream`."""
+    its weight norm (max_unorm > 0); four launches on `stream`."""
     check(lib().opt2s_step_max_unorm(ctypes.byref(tl.desc), ctypes.byref(hyper),
                                      float(max_unorm), int(step), _stream_handle(stream)),
           "opt2s_step_max_unorm")

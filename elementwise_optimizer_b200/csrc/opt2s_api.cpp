@@ -243,25 +243,38 @@ std::vector<ChunkRec> build_chunk_table(const TensorListDesc* d, int64_t chunk_e
 int unorm_workspace(const TensorListDesc* desc, int64_t chunk_elems, opt2s_plan* plan)
 {
     using opt2s::kNormBlockElems;
+    using opt2s::kNormGroupBlocks;
     if (count_chunks(desc, kNormBlockElems) > INT32_MAX) return OPT2S_ERR_TOO_LARGE;
     std::vector<ChunkRec> blocks = build_chunk_table(desc, kNormBlockElems, false);
-    std::vector<uint32_t> first(static_cast<size_t>(desc->count) + 1, 0);
-    for (int32_t i = 0; i < desc->count; ++i)
-        first[i + 1] = first[i] + static_cast<uint32_t>(
+    // groups of kNormGroupBlocks consecutive blocks of one tensor
+    std::vector<uint32_t> ranges;
+    std::vector<uint32_t> first_group(static_cast<size_t>(desc->count) + 1, 0);
+    uint32_t block0 = 0;
+    for (int32_t i = 0; i < desc->count; ++i) {
+        const uint32_t nb = static_cast<uint32_t>(
             (desc->tensors[i].numel + kNormBlockElems - 1) / kNormBlockElems);
+        for (uint32_t b = 0; b < nb; b += kNormGroupBlocks) {
+            ranges.push_back(block0 + b);
+            ranges.push_back(block0 + std::min<uint32_t>(b + kNormGroupBlocks, nb));
+        }
+        block0 += nb;
+        first_group[i + 1] = static_cast<uint32_t>(ranges.size() / 2);
+    }
     std::vector<uint32_t> chunk_tensor;
     chunk_tensor.reserve(static_cast<size_t>(plan->nchunks));
     for_each_chunk(desc, chunk_elems, [&](int32_t i, const opt2s_tensor&, int64_t, int64_t) {
         chunk_tensor.push_back(static_cast<uint32_t>(i));
     });
-    // layout: blocks | partial (2 doubles each) | first | scale | chunk_tensor
+    const size_t ngroups = ranges.size() / 2;
+    // layout: blocks | partial | group ranges | group sums | first_group | scale | chunk_tensor
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t b_bytes = up(blocks.size() * sizeof(ChunkRec));
-    const size_t p_bytes = up(blocks.size() * 2 * sizeof(double));
-    const size_t f_bytes = up(first.size() * sizeof(uint32_t));
-    const size_t s_bytes = up(static_cast<size_t>(desc->count) * sizeof(float));
-    const size_t c_bytes = up(chunk_tensor.size() * sizeof(uint32_t));
-    const size_t total = b_bytes + p_bytes + f_bytes + s_bytes + c_bytes;
+    const size_t sizes[] = {up(blocks.size() * sizeof(ChunkRec)), up(blocks.size() * 2 * sizeof(double)),
+                            up(ranges.size() * sizeof(uint32_t)), up(ngroups * 2 * sizeof(double)),
+                            up(first_group.size() * sizeof(uint32_t)),
+                            up(static_cast<size_t>(desc->count) * sizeof(float)),
+                            up(chunk_tensor.size() * sizeof(uint32_t))};
+    size_t total = 0;
+    for (size_t x : sizes) total += x;
     cudaError_t e;
     if (g_fail_allocs.load() > 0 && g_fail_allocs.fetch_sub(1) > 0)
         e = cudaErrorMemoryAllocation;                // injected by the test scaffolding
@@ -272,24 +285,28 @@ int unorm_workspace(const TensorListDesc* desc, int64_t chunk_elems, opt2s_plan*
         if (e == cudaErrorMemoryAllocation) { t_last_cuda_error = e; return OPT2S_ERR_NO_MEMORY; }
         return cuda_fail(e);
     }
-    char* base = static_cast<char*>(plan->d_unorm);
+    char* at[7];
+    at[0] = static_cast<char*>(plan->d_unorm);
+    for (int k = 1; k < 7; ++k) at[k] = at[k - 1] + sizes[k - 1];
     opt2s::UnormArgs& u = plan->unorm;
-    u.blocks = reinterpret_cast<ChunkRec*>(base);
+    u.blocks = reinterpret_cast<ChunkRec*>(at[0]);
     u.nblocks = static_cast<int64_t>(blocks.size());
-    u.partial = reinterpret_cast<double*>(base + b_bytes);
-    u.first_block = reinterpret_cast<uint32_t*>(base + b_bytes + p_bytes);
+    u.partial = reinterpret_cast<double*>(at[1]);
+    u.group_range = reinterpret_cast<uint32_t*>(at[2]);
+    u.ngroups = static_cast<int64_t>(ngroups);
+    u.group_sum = reinterpret_cast<double*>(at[3]);
+    u.first_group = reinterpret_cast<uint32_t*>(at[4]);
     u.ntensors = desc->count;
-    u.scale = reinterpret_cast<float*>(base + b_bytes + p_bytes + f_bytes);
-    u.chunk_tensor = reinterpret_cast<uint32_t*>(base + b_bytes + p_bytes + f_bytes + s_bytes);
-    if (!blocks.empty())
-        e = cudaMemcpy(const_cast<ChunkRec*>(u.blocks), blocks.data(), blocks.size() * sizeof(ChunkRec),
-                       cudaMemcpyHostToDevice);
-    if (e == cudaSuccess)
-        e = cudaMemcpy(const_cast<uint32_t*>(u.first_block), first.data(), first.size() * sizeof(uint32_t),
-                       cudaMemcpyHostToDevice);
-    if (e == cudaSuccess && !chunk_tensor.empty())
-        e = cudaMemcpy(const_cast<uint32_t*>(u.chunk_tensor), chunk_tensor.data(),
-                       chunk_tensor.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
+    u.scale = reinterpret_cast<float*>(at[5]);
+    u.chunk_tensor = reinterpret_cast<uint32_t*>(at[6]);
+    auto put = [&](const void* dst, const void* src, size_t bytes) {
+        if (e == cudaSuccess && bytes > 0)
+            e = cudaMemcpy(const_cast<void*>(dst), src, bytes, cudaMemcpyHostToDevice);
+    };
+    put(u.blocks, blocks.data(), blocks.size() * sizeof(ChunkRec));
+    put(u.group_range, ranges.data(), ranges.size() * sizeof(uint32_t));
+    put(u.first_group, first_group.data(), first_group.size() * sizeof(uint32_t));
+    put(u.chunk_tensor, chunk_tensor.data(), chunk_tensor.size() * sizeof(uint32_t));
     if (e != cudaSuccess) return cuda_fail(e);
     return OPT2S_OK;
 }
@@ -505,7 +522,8 @@ int plan_step_max_unorm(const opt2s_plan* plan, const Hyper* h, float max_unorm,
                                      make_scalars(h, step), plan->unorm, max_unorm, bt,
                                      g_max_blocks, stream);
     if (e != cudaSuccess) return cuda_fail(e);
-    const int launched = (plan->unorm.nblocks > 0) + (plan->unorm.ntensors > 0) + 1;
+    const int launched = (plan->unorm.nblocks > 0) + (plan->unorm.ngroups > 0) +
+                         (plan->unorm.ntensors > 0) + 1;
     g_launches.fetch_add(launched, std::memory_order_relaxed);
     return OPT2S_OK;
 }

@@ -101,23 +101,30 @@ cudaError_t launch_step(const ChunkRec* d_chunks, int64_t nchunks, int algo,
 
 // The bounded-update-norm step (max_unorm > 0).  Device arrays, all owned
 // by the plan: `blocks` is the norm table (each tensor cut into blocks of
-// kNormBlockElems elements, in descriptor order), tensor t owns blocks
-// [first_block[t], first_block[t + 1]); `partial` holds two doubles per block,
-// `scale` one float per tensor, and chunk_tensor[c] is the tensor of the
-// plan's chunk c.
+// kNormBlockElems elements, in descriptor order) with two doubles of
+// `partial` per block; a tensor's blocks form groups of kNormGroupBlocks
+// consecutive blocks, group q spanning blocks [group_range[2q],
+// group_range[2q + 1]) with two doubles of `group_sum`; tensor t owns groups
+// [first_group[t], first_group[t + 1]); `scale` holds one float per tensor,
+// and chunk_tensor[c] is the tensor of the plan's chunk c.
 constexpr int64_t kNormBlockElems = 2048;
+constexpr int64_t kNormGroupBlocks = 64;
 struct UnormArgs {
     const ChunkRec* blocks;
     int64_t nblocks;
-    const uint32_t* first_block;   // ntensors + 1 entries
-    int32_t ntensors;
     double* partial;               // 2 * nblocks
+    const uint32_t* group_range;   // 2 * ngroups
+    int64_t ngroups;
+    double* group_sum;             // 2 * ngroups
+    const uint32_t* first_group;   // ntensors + 1 entries
+    int32_t ntensors;
     float* scale;                  // ntensors
     const uint32_t* chunk_tensor;  // one per chunk of the plan
 };
 
-// Launches the three kernels of the bounded-update-norm step on `stream`
-// (norm partials, per-tensor scales, the scaled step over the plan's chunks).
+// Launches the four kernels of the bounded-update-norm step on `stream`
+// (block sums, group sums, per-tensor scales, the scaled step over the plan's
+// chunks).
 cudaError_t launch_step_max_unorm(const ChunkRec* d_chunks, int64_t nchunks, int algo,
                                   int skip_zeros, const StepScalars& s, const UnormArgs& u,
                                   float max_unorm, int block_threads, int max_blocks,

@@ -639,7 +639,9 @@ __global__ void advance_index_kernel(int* index, int table_len)
 //      chunk length), the binary64 sums of u^2 (u = num/den, the update
 //      direction; 0 for an element skip_zeros leaves alone) and of p^2 (p
 //      the param before the step).  Nothing is written but the two sums;
-//   2. unorm_scale_kernel: per tensor, the sums of its blocks, U = sqrt(su),
+//   2. unorm_group_kernel: the sums of each group of kNormGroupBlocks
+//      consecutive blocks of a tensor (one warp per group);
+//      unorm_scale_kernel: per tensor, the sums of its groups, U = sqrt(su),
 //      P = sqrt(sp), and scale = max_unorm*P/U if U > max_unorm*P, else 1
 //      (binary64, rounded to fp32 once);
 //   3. step_kernel_scaled: the step over the plan's chunks with
@@ -647,10 +649,10 @@ __global__ void advance_index_kernel(int* index, int table_len)
 // The element arithmetic is direction(), as in the plain step.  Every sum
 // has a fixed order: lane l of the warp that owns a block adds the block's
 // elements l, l + 32, l + 64, ... one after the other, the 32 lanes then
-// combine in a fixed shuffle tree, and one CTA combines a tensor's blocks in
-// a fixed order too; so the scale does not depend on the plan's chunk length,
-// the block width or the storage alignment.  Accesses are element-wise and
-// contiguous across the warp.
+// combine in a fixed shuffle tree, a group's blocks and a tensor's groups are
+// combined in fixed orders too; so the scale does not depend on the plan's
+// chunk length, the block width or the storage alignment.  Accesses are
+// element-wise and contiguous across the warp.
 // ---------------------------------------------------------------------------
 template <int DT, int ALGO, bool SKIP>
 __device__ __forceinline__ void norm_block(const ChunkRec& c, const StepScalars& s, int lane,
@@ -716,16 +718,39 @@ __global__ void unorm_partials_kernel(const ChunkRec* __restrict__ blocks, int n
     }
 }
 
-// One CTA of kScaleThreads threads per tensor (tensor t owns blocks
+// One warp per group: group q holds blocks [range[q].x, range[q].y) of one
+// tensor (at most kNormGroupBlocks); lane l adds blocks x + l, x + l + 32 in
+// turn, then a fixed tree over lanes.
+__global__ void unorm_group_kernel(const double2* __restrict__ partial,
+                                   const uint2* __restrict__ range, int ngroups,
+                                   double2* __restrict__ group_sum)
+{
+    static_assert(kNormGroupBlocks <= 64, "two blocks per lane");
+    const int lane = threadIdx.x & 31;
+    const int warps_per_block = blockDim.x >> 5;
+    const int nwarps = gridDim.x * warps_per_block;
+    for (int q = blockIdx.x * warps_per_block + (threadIdx.x >> 5); q < ngroups; q += nwarps) {
+        const uint2 r = range[q];
+        double su = 0.0, sp = 0.0;
+        for (uint32_t b = r.x + lane; b < r.y; b += 32) {
+            const double2 x = partial[b];
+            su = __dadd_rn(su, x.x);
+            sp = __dadd_rn(sp, x.y);
+        }
+        warp_tree_sum(su, sp);
+        if (lane == 0) group_sum[q] = make_double2(su, sp);
+    }
+}
+
+// One CTA of kScaleThreads threads per tensor (tensor t owns groups
 // [first[t], first[t + 1])): thread j keeps four running sums, sum k taking
-// blocks j + (4i + k)*kScaleThreads for i = 0, 1, ... in turn (four chains of
-// loads in flight), then (s0 + s1) + (s2 + s3), then a fixed tree over lanes
-// and over the CTA's warps.  The order depends only on the tensor, not on the
-// grid.
+// groups j + (4i + k)*kScaleThreads for i = 0, 1, ... in turn, then
+// (s0 + s1) + (s2 + s3), then a fixed tree over lanes and over the CTA's
+// warps.  The order depends only on the tensor, not on the grid.
 constexpr int kScaleThreads = 1024;
 
 __global__ void __launch_bounds__(kScaleThreads)
-unorm_scale_kernel(const double2* __restrict__ partial, const uint32_t* __restrict__ first,
+unorm_scale_kernel(const double2* __restrict__ sums, const uint32_t* __restrict__ first,
                    int ntensors, float max_unorm, float* __restrict__ scale)
 {
     constexpr int kWarps = kScaleThreads / 32;
@@ -740,7 +765,7 @@ unorm_scale_kernel(const double2* __restrict__ partial, const uint32_t* __restri
             for (int k = 0; k < 4; ++k) {
                 const uint32_t i = b + k * kScaleThreads;
                 if (i < end) {
-                    const double2 x = partial[i];
+                    const double2 x = sums[i];
                     au[k] = __dadd_rn(au[k], x.x);
                     ap[k] = __dadd_rn(ap[k], x.y);
                 }
@@ -1070,6 +1095,14 @@ cudaError_t launch_unorm_typed(const ChunkRec* d_chunks, int64_t nchunks, const 
             u.blocks, static_cast<int>(u.nblocks), sc, reinterpret_cast<double2*>(u.partial));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    if (u.ngroups > 0) {
+        const void* kg = reinterpret_cast<const void*>(unorm_group_kernel);
+        if ((e = unorm_grid(kg, u.ngroups, kNormThreads, &grid)) != cudaSuccess) return e;
+        unorm_group_kernel<<<grid, kNormThreads, 0, stream>>>(
+            reinterpret_cast<const double2*>(u.partial), reinterpret_cast<const uint2*>(u.group_range),
+            static_cast<int>(u.ngroups), reinterpret_cast<double2*>(u.group_sum));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if (u.ntensors > 0) {
         const void* k2 = reinterpret_cast<const void*>(unorm_scale_kernel);
         // one CTA per tensor, up to the resident CTAs of the device
@@ -1077,7 +1110,7 @@ cudaError_t launch_unorm_typed(const ChunkRec* d_chunks, int64_t nchunks, const 
                             &grid)) != cudaSuccess)
             return e;
         unorm_scale_kernel<<<grid, kScaleThreads, 0, stream>>>(
-            reinterpret_cast<const double2*>(u.partial), u.first_block, u.ntensors, max_unorm,
+            reinterpret_cast<const double2*>(u.group_sum), u.first_group, u.ntensors, max_unorm,
             u.scale);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

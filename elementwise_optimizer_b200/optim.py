@@ -17,7 +17,7 @@ must keep accumulating into those views: do not replace p.grad).  Results are
 the same bits as without flattening, since the update is elementwise.
 
 max_unorm > 0 bounds each parameter's update norm by max_unorm times its
-weight norm (opt2s_step_max_unorm: three launches per group and step).  With
+weight norm (opt2s_step_max_unorm: four launches per group and step).  With
 flatten=True the bound still applies per parameter: the flat buffers are
 stepped through one record per parameter, and AdEMAMix keeps each
 parameter's [m1 | m2] together in the flat state.  It is not combined with

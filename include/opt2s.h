@@ -265,17 +265,19 @@ int64_t opt2s_noalloc_max_chunks(void);
  *
  * s = 1 gives exactly opt2s_step's bits.  The sums have a fixed order (lane
  * l of a warp adds elements l, l+32, ... of a 2,048-element block, then a
- * fixed tree over lanes; one CTA adds a tensor's blocks in a fixed order),
+ * fixed tree over lanes; a group's blocks and a tensor's groups are added
+ * in fixed orders too),
  * so s does not depend on launch geometry or storage alignment; against a
  * plain sequential binary64 sum it can differ only when the ratio lies
  * within a few binary64 ulp of an fp32 rounding boundary.
  *
  * max_unorm: finite and > 0 (else OPT2S_ERR_INVALID_ARG).  Other arguments
- * and validation as opt2s_step.  Three launches on `stream`: the norm sums,
- * the per-tensor scales, and the scaled update.  The tensor is read twice
- * (once for the sums, once for the update).  Plans are cached like
- * opt2s_step's, each with a workspace of 64 bytes per 2,048 elements plus
- * 4 bytes per tensor and per chunk, freed by opt2s_release_cache().
+ * and validation as opt2s_step.  Four launches on `stream`: the sums per
+ * 2,048-element block, the sums per group of 64 blocks, the per-tensor
+ * scales, and the scaled update.  The tensor is read twice (once for the
+ * sums, once for the update).  Plans are cached like opt2s_step's, each with
+ * a workspace of 64 bytes per 2,048 elements plus 24 bytes per group and
+ * 8 bytes per tensor and per chunk, freed by opt2s_release_cache().
  */
 int opt2s_step_max_unorm(const TensorListDesc *desc, const Hyper *hyper, float max_unorm,
                          int step, cudaStream_t stream);
