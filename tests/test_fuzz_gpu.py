@@ -7,13 +7,15 @@ specialised Adam kernel runs), the algorithm, skip_zeros, hyper-parameters
 (learning rate over four decades, beta1 including 0, weight decay on or off),
 the gradient recipe, the storage layout (separate allocations, packed back to
 back, or padded so that most tensors start misaligned), the starting step,
-and, for half the cases, a forced chunk length and launch shape.  After every
-step, param, state1 and state2 must hold the oracle's bits and the gradients
-must be untouched.
+for half the cases a forced chunk length and launch shape, and for a third of
+them a max_unorm bound (opt2s_step_max_unorm against the oracle's bounded
+step).  After every step, param, state1 and state2 must hold the oracle's
+bits and the gradients must be untouched.
 """
 import numpy as np
 import pytest
 
+import oracle
 from elementwise_optimizer_b200 import binding as B
 from elementwise_optimizer_b200 import synth
 from tests.gpu_support import Harness
@@ -64,12 +66,13 @@ def draw_case(case):
     if r.random() < 0.5:
         geometry = (int(r.choice([32, 64, 128, 256])), int(r.choice([0, 1, 3, 7])),
                     int(r.choice([0, 8, 256, 1000, 4096])))
-    return w, layout, pad, first_step, steps, geometry
+    max_unorm = float(np.float32(10 ** r.uniform(-2, 1))) if r.random() < 1 / 3 else 0.0
+    return w, layout, pad, first_step, steps, geometry, max_unorm
 
 
 @pytest.mark.parametrize("case", range(CASES))
 def test_random_collection_matches_oracle(case):
-    w, layout, pad, first_step, steps, geometry = draw_case(case)
+    w, layout, pad, first_step, steps, geometry, max_unorm = draw_case(case)
     if geometry is not None:
         B.opt2s_release_cache()
         prev = B.testing_set_chunk_elems(geometry[2])
@@ -77,7 +80,15 @@ def test_random_collection_matches_oracle(case):
     try:
         h = Harness(w, layout=layout, pad=pad)
         for t in range(first_step, first_step + steps):
-            h.step_both(t)
+            if max_unorm > 0.0:
+                h.load_grads(t)
+                B.opt2s_step_max_unorm(h.tl, h.hyper, max_unorm, t)
+                for i, dt in enumerate(w.dtypes):
+                    oracle.step_f32_max_unorm(h.h_p[i], h._h_g[i], h.h_s1[i], h.h_s2[i], dtype=dt,
+                                              algo=w.algo, step=t, skip_zeros=w.skip_zeros,
+                                              max_unorm=max_unorm, **w.hyper)
+            else:
+                h.step_both(t)
             worst = h.max_ulps()
             assert worst == {"param": 0, "state1": 0, "state2": 0}, (t, worst, w.sizes, w.dtypes)
             assert h.grads_unchanged()
