@@ -497,7 +497,11 @@ def _oracle_parallel_step(w, arrays, step, cores, pool):
             s1[lo:hi] = s1k[:hi - lo]
             s1[n + lo:n + hi] = s1k[hi - lo:]
 
-    list(pool.map(part, range(cores)))
+    if pool is None:
+        for k in range(cores):
+            part(k)
+    else:
+        list(pool.map(part, range(cores)))
 
 
 def cpu_baseline(w, seconds):
@@ -518,10 +522,25 @@ def cpu_baseline(w, seconds):
             el = time.perf_counter() - t0
             if el >= seconds:
                 break
+    # the same oracle on one core, on the first 1/cores of the sample, for about
+    # a fifth of the time: the single-threaded figure beside the all-core one
+    one = _oracle_sample(w, max(1, n_sample // cores))
+    steps1 = 0
+    t1 = time.perf_counter()
+    while True:
+        steps1 += 1
+        _oracle_parallel_step(w, one, 1 + steps1, 1, None)
+        el1 = time.perf_counter() - t1
+        if el1 >= seconds / 5:
+            break
+    n1 = max(1, n_sample // cores)
     return {"value": n_sample * steps / el, "unit": "elements/s", "cores": cores,
             "kind": "oracle",
+            "single_thread_value": n1 * steps1 / el1,
             "sample": f"first {n_sample} elements of {w.name}, {steps} steps, "
-                      f"{el:.1f} s, {cores} threads x single-threaded oracle on disjoint slices"}
+                      f"{el:.1f} s, {cores} threads x single-threaded oracle on disjoint slices; "
+                      f"single_thread_value: the first {n1} elements on one thread, {steps1} steps, "
+                      f"{el1:.1f} s"}
 
 
 def run_reference(args, rank, world):
