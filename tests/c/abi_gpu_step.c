@@ -1,8 +1,9 @@
 /* Uses the C ABI from plain C on a GPU (no Python, no PyTorch): cudaMalloc'd
- * buffers, three opt2s_step calls on a mixed fp32/fp16/bf16 AdEMAMix
- * collection with a misaligned tensor, then a bitwise comparison with the CPU
- * oracle (test infrastructure, linked only into this test).  Built and run by
- * tests/test_c_abi.py.  Prints "ok" on success. */
+ * buffers, three opt2s_step calls and two opt2s_step_max_unorm calls on a
+ * mixed fp32/fp16/bf16 AdEMAMix collection with a misaligned tensor, then a
+ * bitwise comparison with the CPU oracle (test infrastructure, linked only
+ * into this test).  Built and run by tests/test_c_abi.py.  Prints "ok" on
+ * success. */
 #include <stdio.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -13,6 +14,11 @@
 int oracle_step_f32(int algo, int dtype, int skip_zeros, float lr, float beta1, float beta2,
                     float beta3, float alpha, float eps, float weight_decay, int step,
                     void *param, const void *grad, float *state1, float *state2, int64_t n);
+int oracle_step_f32_max_unorm(int algo, int dtype, int skip_zeros, float lr, float beta1,
+                              float beta2, float beta3, float alpha, float eps,
+                              float weight_decay, float max_unorm, int step, void *param,
+                              const void *grad, float *state1, float *state2, int64_t n,
+                              float *scale_out);
 uint16_t oracle_f32_to_f16(float x);
 uint16_t oracle_f32_to_bf16(float x);
 
@@ -72,14 +78,23 @@ int main(void)
         rec[i].reserved = 0;
     }
     TensorListDesc d = {rec, T};
-    for (int step = 1; step <= 3; ++step) {
-        int st = opt2s_step(&d, &h, step, 0);
-        if (st != OPT2S_OK) { printf("opt2s_step: %s\n", opt2s_error_string(st)); return 1; }
+    const float max_unorm = 0.05f;           /* steps 4 and 5: bounded update norm */
+    for (int step = 1; step <= 5; ++step) {
+        int st = step <= 3 ? opt2s_step(&d, &h, step, 0)
+                           : opt2s_step_max_unorm(&d, &h, max_unorm, step, 0);
+        if (st != OPT2S_OK) { printf("step %d: %s\n", step, opt2s_error_string(st)); return 1; }
         for (int i = 0; i < T; ++i) {
             const int es = dt[i] == OPT2S_F32 ? 4 : 2;
-            oracle_step_f32(1, dt[i], 0, h.lr, h.beta1, h.beta2, h.beta3, h.alpha, h.eps,
-                            h.weight_decay, step, (char *)hp[i] + offset[i] * es,
-                            (const char *)hg[i] + offset[i] * es, hs1[i], hs2[i], n[i]);
+            if (step <= 3)
+                oracle_step_f32(1, dt[i], 0, h.lr, h.beta1, h.beta2, h.beta3, h.alpha, h.eps,
+                                h.weight_decay, step, (char *)hp[i] + offset[i] * es,
+                                (const char *)hg[i] + offset[i] * es, hs1[i], hs2[i], n[i]);
+            else
+                oracle_step_f32_max_unorm(1, dt[i], 0, h.lr, h.beta1, h.beta2, h.beta3, h.alpha,
+                                          h.eps, h.weight_decay, max_unorm, step,
+                                          (char *)hp[i] + offset[i] * es,
+                                          (const char *)hg[i] + offset[i] * es, hs1[i], hs2[i],
+                                          n[i], NULL);
         }
     }
     CK(cudaDeviceSynchronize());
