@@ -277,7 +277,9 @@ int64_t opt2s_noalloc_max_chunks(void);
  * scales, and the scaled update.  The tensor is read twice (once for the
  * sums, once for the update).  Plans are cached like opt2s_step's, each with
  * a workspace of 64 bytes per 2,048 elements plus 24 bytes per group and
- * 8 bytes per tensor and per chunk, freed by opt2s_release_cache().
+ * 8 bytes per tensor and per chunk, freed by opt2s_release_cache().  The
+ * workspace belongs to the collection's plan: like its params and states,
+ * two steps of the same collection must not overlap on the GPU.
  */
 int opt2s_step_max_unorm(const TensorListDesc *desc, const Hyper *hyper, float max_unorm,
                          int step, cudaStream_t stream);
