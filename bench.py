@@ -892,7 +892,8 @@ def main():
     ap.add_argument("--workload", default="large_f32",
                     choices=["large_f32", "transformer_bf16", "small_collection"])
     ap.add_argument("--numel", type=int, default=0,
-                    help="size of the large_f32 tensor (default 268,435,456)")
+                    help="size of the large_f32 tensor, and of the tensor of --mode max-unorm and "
+                         "--mode roofline-table (default 268,435,456)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-extras", action="store_true",
@@ -917,9 +918,12 @@ def main():
         from elementwise_optimizer_b200 import _build
         _build.build()
         torch.cuda.set_device(local_rank)
-        res = {"direct-cells": run_direct_cells, "eager-collection": run_eager_collection,
-               "shard-emulated": run_shard_emulated,
-               "roofline-table": run_roofline_table, "max-unorm": run_max_unorm}[args.mode]()
+        sized = {"roofline-table": run_roofline_table, "max-unorm": run_max_unorm}
+        if args.mode in sized and args.numel:
+            res = sized[args.mode](numel=args.numel)
+        else:
+            res = {"direct-cells": run_direct_cells, "eager-collection": run_eager_collection,
+                   "shard-emulated": run_shard_emulated, **sized}[args.mode]()
         res["env"] = environment()
         print(json.dumps(res), flush=True)
         return
