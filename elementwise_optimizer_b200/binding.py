@@ -112,6 +112,11 @@ EXPORTS = {
                                                   ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]),
     "opt2s_testing_validate": (ctypes.c_int, [ctypes.POINTER(TensorListDesc),
                                               ctypes.POINTER(Hyper), ctypes.c_int]),
+    "opt2s_testing_unorm_tables": (ctypes.c_int, [ctypes.POINTER(TensorListDesc), ctypes.c_int32,
+                                                  ctypes.c_int64, ctypes.POINTER(ctypes.c_uint32),
+                                                  ctypes.POINTER(ctypes.c_uint32),
+                                                  ctypes.POINTER(ctypes.c_uint32),
+                                                  ctypes.POINTER(ctypes.c_int64)]),
     "opt2s_testing_set_chunk_elems": (ctypes.c_int64, [ctypes.c_int64]),
     "opt2s_testing_set_launch": (ctypes.c_int, [ctypes.c_int, ctypes.c_int]),
     "opt2s_testing_default_chunk_elems": (ctypes.c_int64, []),
@@ -354,6 +359,24 @@ def testing_build_chunks(tl: TensorList, algo: str, chunk_elems: int = 0) -> lis
     check(L.opt2s_testing_build_chunks(ctypes.byref(tl.desc), ALGOS[algo], chunk_elems,
                                        arr, n.value, ctypes.byref(n)), "build_chunks")
     return [(c.tensor, c.start, c.len, c.dtype) for c in arr[:n.value]]
+
+
+def testing_unorm_tables(tl: TensorList, algo: str, chunk_elems: int = 0) -> dict:
+    """The host tables of the bounded-update-norm step for `tl` (see
+    opt2s_testing.h): block count, group ranges, first group per tensor and
+    each chunk's tensor."""
+    L = lib()
+    counts = (ctypes.c_int64 * 3)()
+    null = ctypes.POINTER(ctypes.c_uint32)()
+    check(L.opt2s_testing_unorm_tables(ctypes.byref(tl.desc), ALGOS[algo], int(chunk_elems),
+                                       null, null, null, counts), "testing_unorm_tables")
+    ranges = (ctypes.c_uint32 * max(1, 2 * counts[1]))()
+    first = (ctypes.c_uint32 * (tl.desc.count + 1))()
+    chunks = (ctypes.c_uint32 * max(1, counts[2]))()
+    check(L.opt2s_testing_unorm_tables(ctypes.byref(tl.desc), ALGOS[algo], int(chunk_elems),
+                                       ranges, first, chunks, counts), "testing_unorm_tables")
+    return {"nblocks": counts[0], "ranges": list(ranges[:2 * counts[1]]),
+            "first_group": list(first), "chunk_tensor": list(chunks[:counts[2]])}
 
 
 def testing_validate(tl: TensorList, hyper: Hyper, step: int) -> int:

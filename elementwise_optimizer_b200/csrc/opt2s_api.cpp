@@ -240,31 +240,50 @@ std::vector<ChunkRec> build_chunk_table(const TensorListDesc* d, int64_t chunk_e
 
 // Builds the bounded-update-norm workspace of `plan` for `desc` (host tables,
 // then one device allocation and three uploads).
-int unorm_workspace(const TensorListDesc* desc, int64_t chunk_elems, opt2s_plan* plan)
+// Host tables of the bounded-update-norm step for `desc` (the plan's chunks
+// have `chunk_elems` elements): the norm blocks, the group ranges (first and
+// end block of each group of kNormGroupBlocks consecutive blocks of one
+// tensor), each tensor's first group (count + 1 entries) and each chunk's
+// tensor.  The caller has checked that the block count fits in 32 bits.
+struct UnormTables {
+    std::vector<ChunkRec> blocks;
+    std::vector<uint32_t> ranges;
+    std::vector<uint32_t> first_group;
+    std::vector<uint32_t> chunk_tensor;
+};
+
+UnormTables unorm_tables(const TensorListDesc* desc, int64_t chunk_elems)
 {
     using opt2s::kNormBlockElems;
     using opt2s::kNormGroupBlocks;
-    if (count_chunks(desc, kNormBlockElems) > INT32_MAX) return OPT2S_ERR_TOO_LARGE;
-    std::vector<ChunkRec> blocks = build_chunk_table(desc, kNormBlockElems, false);
-    // groups of kNormGroupBlocks consecutive blocks of one tensor
-    std::vector<uint32_t> ranges;
-    std::vector<uint32_t> first_group(static_cast<size_t>(desc->count) + 1, 0);
+    UnormTables t;
+    t.blocks = build_chunk_table(desc, kNormBlockElems, false);
+    t.first_group.assign(static_cast<size_t>(desc->count) + 1, 0);
     uint32_t block0 = 0;
     for (int32_t i = 0; i < desc->count; ++i) {
         const uint32_t nb = static_cast<uint32_t>(
             (desc->tensors[i].numel + kNormBlockElems - 1) / kNormBlockElems);
         for (uint32_t b = 0; b < nb; b += kNormGroupBlocks) {
-            ranges.push_back(block0 + b);
-            ranges.push_back(block0 + std::min<uint32_t>(b + kNormGroupBlocks, nb));
+            t.ranges.push_back(block0 + b);
+            t.ranges.push_back(block0 + std::min<uint32_t>(b + kNormGroupBlocks, nb));
         }
         block0 += nb;
-        first_group[i + 1] = static_cast<uint32_t>(ranges.size() / 2);
+        t.first_group[i + 1] = static_cast<uint32_t>(t.ranges.size() / 2);
     }
-    std::vector<uint32_t> chunk_tensor;
-    chunk_tensor.reserve(static_cast<size_t>(plan->nchunks));
     for_each_chunk(desc, chunk_elems, [&](int32_t i, const opt2s_tensor&, int64_t, int64_t) {
-        chunk_tensor.push_back(static_cast<uint32_t>(i));
+        t.chunk_tensor.push_back(static_cast<uint32_t>(i));
     });
+    return t;
+}
+
+int unorm_workspace(const TensorListDesc* desc, int64_t chunk_elems, opt2s_plan* plan)
+{
+    if (count_chunks(desc, opt2s::kNormBlockElems) > INT32_MAX) return OPT2S_ERR_TOO_LARGE;
+    UnormTables tab = unorm_tables(desc, chunk_elems);
+    const std::vector<ChunkRec>& blocks = tab.blocks;
+    const std::vector<uint32_t>& ranges = tab.ranges;
+    const std::vector<uint32_t>& first_group = tab.first_group;
+    const std::vector<uint32_t>& chunk_tensor = tab.chunk_tensor;
     const size_t ngroups = ranges.size() / 2;
     // layout: blocks | partial | group ranges | group sums | first_group | scale | chunk_tensor
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
@@ -751,6 +770,25 @@ OPT2S_API int opt2s_testing_build_chunks(const TensorListDesc* desc, int32_t alg
     for_each_chunk(desc, ce, [&](int32_t i, const opt2s_tensor& t, int64_t s, int64_t len) {
         out[k++] = opt2s_testing_chunk{i, s, len, t.dtype, 0};
     });
+    return OPT2S_OK;
+}
+
+OPT2S_API int opt2s_testing_unorm_tables(const TensorListDesc* desc, int32_t algo, int64_t chunk_elems,
+                                         uint32_t* group_ranges, uint32_t* first_group,
+                                         uint32_t* chunk_tensor, int64_t* counts)
+{
+    if (!counts) return OPT2S_ERR_INVALID_ARG;
+    int st = validate_desc(desc, algo);
+    if (st != OPT2S_OK) return st;
+    if (count_chunks(desc, opt2s::kNormBlockElems) > INT32_MAX) return OPT2S_ERR_TOO_LARGE;
+    const int64_t ce = chunk_elems > 0 ? chunk_elems : opt2s::kDefaultChunkElems;
+    const UnormTables t = unorm_tables(desc, ce);
+    counts[0] = static_cast<int64_t>(t.blocks.size());
+    counts[1] = static_cast<int64_t>(t.ranges.size() / 2);
+    counts[2] = static_cast<int64_t>(t.chunk_tensor.size());
+    if (group_ranges) std::copy(t.ranges.begin(), t.ranges.end(), group_ranges);
+    if (first_group) std::copy(t.first_group.begin(), t.first_group.end(), first_group);
+    if (chunk_tensor) std::copy(t.chunk_tensor.begin(), t.chunk_tensor.end(), chunk_tensor);
     return OPT2S_OK;
 }
 

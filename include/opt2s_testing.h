@@ -74,6 +74,19 @@ int64_t opt2s_testing_default_chunk_elems(void);
  * fit in one wave (chunks <= resident_warps). */
 int64_t opt2s_testing_choose_chunk_elems(const TensorListDesc *desc, int64_t resident_warps);
 
+/* Host only: the tables the bounded-update-norm step (opt2s_step_max_unorm)
+ * builds for `desc` when the plan's chunks have `chunk_elems` elements (<= 0:
+ * the largest chunk length).  counts[0] = norm blocks (2,048 elements each,
+ * per tensor), counts[1] = groups, counts[2] = chunks.  Each non-null array
+ * receives, in descriptor order: group_ranges, 2 per group (first block, end
+ * block; a group is up to 64 consecutive blocks of one tensor); first_group,
+ * count + 1 entries (tensor t owns groups [first_group[t],
+ * first_group[t + 1])); chunk_tensor, the tensor of each chunk.  Call with
+ * null arrays first to size them.  Validates `desc` like opt2s_step. */
+int opt2s_testing_unorm_tables(const TensorListDesc *desc, int32_t algo, int64_t chunk_elems,
+                               uint32_t *group_ranges, uint32_t *first_group,
+                               uint32_t *chunk_tensor, int64_t *counts);
+
 /* Runs the step kernel's exact division by a constant in (0, 1] and the IEEE
  * division __fdiv_rn side by side on `n` seeded random operand pairs on the
  * current device (mode 0: x of every class; mode 1: x/d next to a binary32

@@ -14,7 +14,10 @@ against a plain restatement of its rule:
     minimises (waves of chunks over the resident warps) x (c / 32 + 8), the
     longest on ties, where a plan with 16-bit tensors takes 128 only when it
     fits in one wave;
-  * the shard partition: consecutive, 8-element aligned, covering the buffer.
+  * the shard partition: consecutive, 8-element aligned, covering the buffer;
+  * the bounded-update-norm tables: 2,048-element norm blocks per tensor,
+    groups of at most 64 consecutive blocks of one tensor covering each
+    tensor's blocks in order, and each chunk's tensor.
 
 Pointers are fake addresses: nothing is dereferenced.
 """
@@ -167,3 +170,27 @@ def test_shard_partition(numel, world):
         assert start % 8 == 0 or n == 0
         pos += n
     assert pos == numel
+
+
+@SETTINGS
+@given(collections(), st.sampled_from([0, 128, 256, 1000, 2048, 8192]))
+def test_norm_tables_group_each_tensors_blocks_in_order(coll, chunk):
+    sizes, dts, recs = coll
+    tl = B.TensorList(recs)
+    t = B.testing_unorm_tables(tl, "adam", chunk)
+    nb = [-(-n // 2048) for n in sizes]
+    assert t["nblocks"] == sum(nb)
+    ranges = list(zip(t["ranges"][0::2], t["ranges"][1::2]))
+    first = t["first_group"]
+    assert len(first) == len(sizes) + 1 and first[0] == 0 and first[-1] == len(ranges)
+    block0 = 0
+    for i, n in enumerate(nb):
+        mine = ranges[first[i]:first[i + 1]]
+        pos = block0
+        for lo, hi in mine:                    # contiguous, in order, 1..64 blocks each
+            assert lo == pos and 1 <= hi - lo <= 64
+            pos = hi
+        assert pos == block0 + n
+        block0 += n
+    chunks = B.testing_build_chunks(tl, "adam", chunk)
+    assert t["chunk_tensor"] == [c[0] for c in chunks]
