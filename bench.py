@@ -176,10 +176,10 @@ def environment():
     return env
 
 
-def traffic_for(kernel_key):
+def traffic_for(kernel_key, path=None):
     """ncu DRAM bytes per launch, if the committed capture is of the kernel
     sources as they are now (else None)."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    path = path or os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         rec = json.load(open(path)).get(kernel_key)
         if rec and rec.get("kernel_source_sha256") == kernel_source_sha256():

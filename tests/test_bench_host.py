@@ -1,0 +1,51 @@
+"""bench.py pieces that run without a GPU: the environment record every
+result carries, the CPU-baseline leg's shape, the traffic lookup keyed by the
+kernel sources, and the algorithmic byte counts the roofline divides by."""
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_environment_record():
+    env = bench.environment()
+    for key in ("torch", "cuda_runtime", "kernel_sources_sha256", "command", "driver", "nvcc"):
+        assert key in env
+    assert len(env["kernel_sources_sha256"]) == 64
+
+
+def test_cpu_baseline_reports_all_core_and_single_thread_figures():
+    w = bench.workload("large_f32")
+    r = bench.cpu_baseline(w, 0.5)
+    assert r["kind"] == "oracle" and r["unit"] == "elements/s"
+    assert r["cores"] == (os.cpu_count() or 1)
+    assert r["value"] > 0 and r["single_thread_value"] > 0
+    assert "single-threaded oracle" in r["sample"]
+
+
+def test_traffic_lookup_follows_the_kernel_sources(tmp_path):
+    key = "step_kernel/single_f32_n268435456_adam"
+    record = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
+    assert bench.traffic_for(key) in (None, record[key]["dram_bytes_per_launch"])
+    if record[key]["kernel_source_sha256"] == bench.kernel_source_sha256():
+        assert bench.traffic_for(key) == record[key]["dram_bytes_per_launch"]
+    stale = dict(record)
+    stale[key] = dict(record[key], kernel_source_sha256="0" * 64)
+    p = tmp_path / "dram_traffic.json"
+    p.write_text(json.dumps(stale))
+    assert bench.traffic_for(key, str(p)) is None          # other sources: no figure
+    assert bench.traffic_for("no/such/kernel") is None
+
+
+def test_algorithmic_bytes_per_element():
+    from elementwise_optimizer_b200 import synth
+    assert bench.algorithmic_bytes(synth.large_f32()) == 28 * 268_435_456
+    tr = synth.transformer_bf16()
+    assert bench.algorithmic_bytes(tr) == 30 * tr.numel
+    sc = synth.small_collection()
+    assert bench.algorithmic_bytes(sc) == sum(n * (28 if d == "f32" else 22)
+                                              for n, d in zip(sc.sizes, sc.dtypes))
