@@ -47,6 +47,9 @@
  *   - AdEMAMix state1 holds [m1(0..n) | m2(0..n)], 2*n floats.
  *   - fp16/bf16 params are widened exactly and narrowed with
  *     round-to-nearest-even; state is always fp32.
+ *   - max_unorm > 0 (oracle_step_f32_max_unorm): the tensor's update norm is
+ *     bounded by max_unorm times its weight norm, as written out above that
+ *     function; the pages name the option without its arithmetic.
  */
 #include <math.h>
 #include <stdint.h>
