@@ -143,13 +143,40 @@ class ClockSampler:
 KERNEL_SOURCES = ("opt2s_kernel.cu", "opt2s_internal.h", "opt2s_api.cpp")
 
 
+def strip_c_comments(text):
+    """C/C++ source without its comments, every run of whitespace made one
+    space: what the compiler sees, so that a comment edit does not count as a
+    kernel change.  String and character literals are kept as they are."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_sha256():
     """Hash of the sources that define the step kernel and its launch
-    configuration (chunk length, block width)."""
+    configuration (chunk length, block width), comments and whitespace
+    aside."""
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "elementwise_optimizer_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "elementwise_optimizer_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(strip_c_comments(f.read()).encode())
     return h.hexdigest()
 
 

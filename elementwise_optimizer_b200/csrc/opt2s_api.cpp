@@ -238,8 +238,6 @@ std::vector<ChunkRec> build_chunk_table(const TensorListDesc* d, int64_t chunk_e
     return out;
 }
 
-// Builds the bounded-update-norm workspace of `plan` for `desc` (host tables,
-// then one device allocation and three uploads).
 // Host tables of the bounded-update-norm step for `desc` (the plan's chunks
 // have `chunk_elems` elements): the norm blocks, the group ranges (first and
 // end block of each group of kNormGroupBlocks consecutive blocks of one
@@ -276,6 +274,8 @@ UnormTables unorm_tables(const TensorListDesc* desc, int64_t chunk_elems)
     return t;
 }
 
+// Builds the bounded-update-norm workspace of `plan` for `desc` (host tables,
+// then one device allocation and four uploads).
 int unorm_workspace(const TensorListDesc* desc, int64_t chunk_elems, opt2s_plan* plan)
 {
     if (count_chunks(desc, opt2s::kNormBlockElems) > INT32_MAX) return OPT2S_ERR_TOO_LARGE;

@@ -633,7 +633,7 @@ __global__ void advance_index_kernel(int* index, int table_len)
 }
 
 // ---------------------------------------------------------------------------
-// The step with bounded update norms (max_unorm > 0), three launches:
+// The step with bounded update norms (max_unorm > 0), four launches:
 //   1. unorm_partials_kernel: for every block of kNormBlockElems elements of
 //      a tensor (the host's norm table, fixed blocks whatever the plan's
 //      chunk length), the binary64 sums of u^2 (u = num/den, the update

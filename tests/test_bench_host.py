@@ -49,3 +49,11 @@ def test_algorithmic_bytes_per_element():
     sc = synth.small_collection()
     assert bench.algorithmic_bytes(sc) == sum(n * (28 if d == "f32" else 22)
                                               for n, d in zip(sc.sizes, sc.dtypes))
+
+
+def test_source_hash_ignores_comments_but_not_code():
+    src = 'int a = 1; // note\n/* block\n comment */ const char* s = "x//y/*z*/";\n'
+    assert bench.strip_c_comments(src) == bench.strip_c_comments(
+        'int a = 1;\n/* other words */ const char* s = "x//y/*z*/"; // more\n')
+    assert bench.strip_c_comments(src) != bench.strip_c_comments(src.replace("a = 1", "a = 2"))
+    assert '"x//y/*z*/"' in bench.strip_c_comments(src)
