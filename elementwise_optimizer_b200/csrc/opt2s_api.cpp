@@ -61,6 +61,11 @@ int cuda_fail(cudaError_t e)
     return OPT2S_ERR_CUDA;
 }
 
+using opt2s::elem_bytes;
+using opt2s::make_scalars;
+using opt2s::Range;
+using opt2s::validate_hyper;
+
 int block_threads_now(int algo, int only)
 {
     return g_block_threads > 0 ? g_block_threads : opt2s::default_block_threads(algo, only);
@@ -117,31 +122,9 @@ int64_t chunk_elems_for(const TensorListDesc* d, int32_t algo, int only)
     return choose_chunk_elems(d, warps);
 }
 
-int elem_bytes(int32_t dtype) { return dtype == OPT2S_F32 ? 4 : 2; }
-
 // ---------------------------------------------------------------------------
 // Validation (host only, no CUDA call)
 // ---------------------------------------------------------------------------
-
-int validate_hyper(const Hyper* h, int step)
-{
-    if (!h) return OPT2S_ERR_INVALID_ARG;
-    if (h->algo != OPT2S_ADAM && h->algo != OPT2S_ADEMAMIX) return OPT2S_ERR_INVALID_ARG;
-    if (h->skip_zeros != 0 && h->skip_zeros != 1) return OPT2S_ERR_INVALID_ARG;
-    if (step < 1) return OPT2S_ERR_INVALID_ARG;
-    auto unit = [](float b) { return std::isfinite(b) && b >= 0.0f && b < 1.0f; };
-    if (!std::isfinite(h->lr) || !unit(h->beta1) || !unit(h->beta2)) return OPT2S_ERR_INVALID_ARG;
-    if (!std::isfinite(h->eps) || h->eps < 0.0f) return OPT2S_ERR_INVALID_ARG;
-    if (!std::isfinite(h->weight_decay)) return OPT2S_ERR_INVALID_ARG;
-    if (h->algo == OPT2S_ADEMAMIX && (!unit(h->beta3) || !std::isfinite(h->alpha)))
-        return OPT2S_ERR_INVALID_ARG;
-    return OPT2S_OK;
-}
-
-struct Range {
-    uintptr_t lo, hi;   // [lo, hi)
-    bool written;
-};
 
 // Every record well formed, and no buffer that is written overlaps any other
 // buffer (two gradients may share memory: both are only read).
@@ -153,40 +136,13 @@ int validate_desc(const TensorListDesc* d, int32_t algo)
     if (d->count > 0 && !d->tensors) return OPT2S_ERR_INVALID_ARG;
     std::vector<Range> ranges;
     for (int32_t i = 0; i < d->count; ++i) {
-        const opt2s_tensor& t = d->tensors[i];
-        if (t.numel < 0 || t.reserved != 0) return OPT2S_ERR_INVALID_ARG;
-        if (t.dtype != OPT2S_F32 && t.dtype != OPT2S_F16 && t.dtype != OPT2S_BF16)
-            return OPT2S_ERR_INVALID_ARG;
-        if (t.numel == 0) continue;
-        if (t.numel > (int64_t(1) << 40)) return OPT2S_ERR_INVALID_ARG;
-        if (!t.param || !t.grad || !t.state1 || !t.state2) return OPT2S_ERR_INVALID_ARG;
-        const int es = elem_bytes(t.dtype);
-        const auto p = reinterpret_cast<uintptr_t>(t.param);
-        const auto g = reinterpret_cast<uintptr_t>(t.grad);
-        const auto s1 = reinterpret_cast<uintptr_t>(t.state1);
-        const auto s2 = reinterpret_cast<uintptr_t>(t.state2);
-        if (p % es || g % es || s1 % 4 || s2 % 4) return OPT2S_ERR_INVALID_ARG;
-        const uintptr_t n = static_cast<uintptr_t>(t.numel);
-        const uintptr_t s1_elems = algo == OPT2S_ADEMAMIX ? 2 * n : n;
-        ranges.push_back({p, p + n * es, true});
-        ranges.push_back({g, g + n * es, false});
-        ranges.push_back({s1, s1 + s1_elems * 4, true});
-        ranges.push_back({s2, s2 + n * 4, true});
+        Range r[4];
+        int n = 0;
+        const int st = opt2s::record_ranges(d->tensors[i], algo, r, &n);
+        if (st != OPT2S_OK) return st;
+        ranges.insert(ranges.end(), r, r + n);
     }
-    std::sort(ranges.begin(), ranges.end(),
-              [](const Range& a, const Range& b) { return a.lo < b.lo; });
-    // Sweep: compare each range with the furthest-reaching earlier range of
-    // each kind; any overlap involving a written range is an alias.
-    uintptr_t reach_w = 0, reach_any = 0;
-    bool have_w = false, have_any = false;
-    for (const Range& r : ranges) {
-        if (have_w && r.lo < reach_w) return OPT2S_ERR_ALIAS;
-        if (r.written && have_any && r.lo < reach_any) return OPT2S_ERR_ALIAS;
-        if (r.written) { reach_w = have_w ? std::max(reach_w, r.hi) : r.hi; have_w = true; }
-        reach_any = have_any ? std::max(reach_any, r.hi) : r.hi;
-        have_any = true;
-    }
-    return OPT2S_OK;
+    return opt2s::overlap_status(ranges.data(), ranges.size());
 }
 
 // ---------------------------------------------------------------------------
@@ -394,24 +350,6 @@ int plan_destroy(opt2s_plan* plan)
     }
     delete plan;
     return st;
-}
-
-StepScalars make_scalars(const Hyper* h, int step)
-{
-    StepScalars s;
-    s.lr = h->lr;
-    s.beta1 = h->beta1;
-    s.beta2 = h->beta2;
-    s.beta3 = h->beta3;
-    s.one_minus_beta1 = 1.0f - h->beta1;
-    s.one_minus_beta2 = 1.0f - h->beta2;
-    s.one_minus_beta3 = 1.0f - h->beta3;
-    s.alpha = h->alpha;
-    s.eps = h->eps;
-    s.bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(h->beta1), static_cast<double>(step)));
-    s.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(h->beta2), static_cast<double>(step)));
-    s.decay = static_cast<float>(1.0 - static_cast<double>(h->lr) * static_cast<double>(h->weight_decay));
-    return s;
 }
 
 int plan_step(const opt2s_plan* plan, const Hyper* h, int step, cudaStream_t stream)
@@ -687,16 +625,7 @@ OPT2S_API int opt2s_shard_step(const opt2s_shard_desc* d, const Hyper* hyper, in
         ranges.push_back({s1, s1 + (hyper->algo == OPT2S_ADEMAMIX ? 2 * k : k) * 4, true});
         ranges.push_back({s2, s2 + k * 4, true});
     }
-    std::sort(ranges.begin(), ranges.end(), [](const Range& a, const Range& b) { return a.lo < b.lo; });
-    uintptr_t reach_w = 0, reach_any = 0;
-    bool have_w = false, have_any = false;
-    for (const Range& r : ranges) {
-        if (have_w && r.lo < reach_w) return OPT2S_ERR_ALIAS;
-        if (r.written && have_any && r.lo < reach_any) return OPT2S_ERR_ALIAS;
-        if (r.written) { reach_w = have_w ? std::max(reach_w, r.hi) : r.hi; have_w = true; }
-        reach_any = have_any ? std::max(reach_any, r.hi) : r.hi;
-        have_any = true;
-    }
+    if ((st = opt2s::overlap_status(ranges.data(), ranges.size())) != OPT2S_OK) return st;
     if (len == 0) return OPT2S_OK;
     opt2s::ShardArgs a{};
     for (int q = 0; q < d->world; ++q) {
@@ -860,3 +789,11 @@ OPT2S_API int opt2s_testing_fail_allocs(int count)
 }
 
 OPT2S_API int64_t opt2s_testing_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+// ---------------------------------------------------------------------------
+// Shared with the other translation units (opt2s_internal.h)
+// ---------------------------------------------------------------------------
+
+int opt2s::record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+
+void opt2s::count_launches(int64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }

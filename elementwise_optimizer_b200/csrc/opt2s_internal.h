@@ -1,9 +1,14 @@
-// Internal declarations shared by the host API (opt2s_api.cpp) and the
-// kernel translation unit (opt2s_kernel.cu).  Not installed, not public.
+// Internal declarations shared by the host API (opt2s_api.cpp), the kernel
+// translation unit (opt2s_kernel.cu) and the no-allocation entry point
+// (opt2s_noalloc.cu).  Not installed, not public.
 #pragma once
 
+#include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cuda_runtime.h>
+
+#include "opt2s.h"
 
 namespace opt2s {
 
@@ -161,5 +166,111 @@ cudaError_t check_division(uint64_t seed, int64_t n, int mode, unsigned long lon
 // Number of blocks a launch of `nchunks` chunks uses on the current device.
 cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros, int only,
                      int block_threads, int max_blocks, int* grid);
+
+// ---------------------------------------------------------------------------
+// Host-side rules every entry point applies, in one place.  None of them
+// touches the heap, so the no-allocation entry point uses them too.
+// ---------------------------------------------------------------------------
+
+inline int elem_bytes(int32_t dtype) { return dtype == OPT2S_F32 ? 4 : 2; }
+
+// Hyper-parameters and step number of one call.
+inline int validate_hyper(const Hyper* h, int step)
+{
+    if (!h) return OPT2S_ERR_INVALID_ARG;
+    if (h->algo != OPT2S_ADAM && h->algo != OPT2S_ADEMAMIX) return OPT2S_ERR_INVALID_ARG;
+    if (h->skip_zeros != 0 && h->skip_zeros != 1) return OPT2S_ERR_INVALID_ARG;
+    if (step < 1) return OPT2S_ERR_INVALID_ARG;
+    auto unit = [](float b) { return std::isfinite(b) && b >= 0.0f && b < 1.0f; };
+    if (!std::isfinite(h->lr) || !unit(h->beta1) || !unit(h->beta2)) return OPT2S_ERR_INVALID_ARG;
+    if (!std::isfinite(h->eps) || h->eps < 0.0f) return OPT2S_ERR_INVALID_ARG;
+    if (!std::isfinite(h->weight_decay)) return OPT2S_ERR_INVALID_ARG;
+    if (h->algo == OPT2S_ADEMAMIX && (!unit(h->beta3) || !std::isfinite(h->alpha)))
+        return OPT2S_ERR_INVALID_ARG;
+    return OPT2S_OK;
+}
+
+// The per-step scalars: bias corrections and decay evaluated in double and
+// rounded to fp32 once, 1 - beta as fp32 subtractions.  The reciprocals of
+// the bias corrections are filled in at launch (fill_reciprocals).
+inline StepScalars make_scalars(const Hyper* h, int step)
+{
+    StepScalars s;
+    s.lr = h->lr;
+    s.beta1 = h->beta1;
+    s.beta2 = h->beta2;
+    s.beta3 = h->beta3;
+    s.one_minus_beta1 = 1.0f - h->beta1;
+    s.one_minus_beta2 = 1.0f - h->beta2;
+    s.one_minus_beta3 = 1.0f - h->beta3;
+    s.alpha = h->alpha;
+    s.eps = h->eps;
+    s.bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(h->beta1), static_cast<double>(step)));
+    s.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(h->beta2), static_cast<double>(step)));
+    s.decay = static_cast<float>(1.0 - static_cast<double>(h->lr) * static_cast<double>(h->weight_decay));
+    s.inv_bc1 = s.inv_bc2 = 0.0;
+    return s;
+}
+
+// An address range [lo, hi) of one buffer, and whether the step writes it.
+struct Range {
+    uintptr_t lo, hi;
+    bool written;
+};
+
+// Checks one record of a collection stepped with `algo` and writes the
+// ranges of its four buffers to out[0..3] (*n = 4), or *n = 0 for an empty
+// record.  Pointers need element alignment; AdEMAMix's state1 spans 2*numel
+// floats.
+inline int record_ranges(const opt2s_tensor& t, int32_t algo, Range* out, int* n)
+{
+    *n = 0;
+    if (t.numel < 0 || t.reserved != 0) return OPT2S_ERR_INVALID_ARG;
+    if (t.dtype != OPT2S_F32 && t.dtype != OPT2S_F16 && t.dtype != OPT2S_BF16)
+        return OPT2S_ERR_INVALID_ARG;
+    if (t.numel == 0) return OPT2S_OK;
+    if (t.numel > (int64_t(1) << 40)) return OPT2S_ERR_INVALID_ARG;
+    if (!t.param || !t.grad || !t.state1 || !t.state2) return OPT2S_ERR_INVALID_ARG;
+    const int es = elem_bytes(t.dtype);
+    const auto p = reinterpret_cast<uintptr_t>(t.param);
+    const auto g = reinterpret_cast<uintptr_t>(t.grad);
+    const auto s1 = reinterpret_cast<uintptr_t>(t.state1);
+    const auto s2 = reinterpret_cast<uintptr_t>(t.state2);
+    if (p % es || g % es || s1 % 4 || s2 % 4) return OPT2S_ERR_INVALID_ARG;
+    const uintptr_t k = static_cast<uintptr_t>(t.numel);
+    out[0] = {p, p + k * es, true};
+    out[1] = {g, g + k * es, false};
+    out[2] = {s1, s1 + (algo == OPT2S_ADEMAMIX ? 2 * k : k) * 4, true};
+    out[3] = {s2, s2 + k * 4, true};
+    *n = 4;
+    return OPT2S_OK;
+}
+
+// Sorts r[0..n) in place by start and reports OPT2S_ERR_ALIAS if a written
+// range overlaps any other range (two read-only ranges may overlap: several
+// tensors may share one gradient buffer).  Each range is compared with the
+// furthest-reaching earlier range of each kind.
+inline int overlap_status(Range* r, size_t n)
+{
+    std::sort(r, r + n, [](const Range& a, const Range& b) { return a.lo < b.lo; });
+    uintptr_t reach_w = 0, reach_any = 0;
+    bool have_w = false, have_any = false;
+    for (size_t i = 0; i < n; ++i) {
+        if (have_w && r[i].lo < reach_w) return OPT2S_ERR_ALIAS;
+        if (r[i].written && have_any && r[i].lo < reach_any) return OPT2S_ERR_ALIAS;
+        if (r[i].written) { reach_w = have_w ? std::max(reach_w, r[i].hi) : r[i].hi; have_w = true; }
+        reach_any = have_any ? std::max(reach_any, r[i].hi) : r[i].hi;
+        have_any = true;
+    }
+    return OPT2S_OK;
+}
+
+// Keeps `e` as this thread's last CUDA error (opt2s_last_cuda_error) and
+// returns OPT2S_ERR_CUDA.  Defined in opt2s_api.cpp.
+int record_cuda_error(cudaError_t e);
+
+// Adds n to the count of kernels this library has launched.  Defined in
+// opt2s_api.cpp.
+void count_launches(int64_t n);
 
 }  // namespace opt2s

@@ -28,9 +28,7 @@
 //     that first call before any stream capture begins.
 
 #include <algorithm>
-#include <cmath>
 #include <cstdint>
-#include <cstring>
 #include <mutex>
 
 #include <cuda_runtime.h>
@@ -56,89 +54,35 @@ static __device__ __align__(256) ChunkRec g_noalloc_table[kNoAllocMaxChunks];
 // Host-side staging of the table and of the ranges used by the overlap check,
 // also fixed-size; a mutex serializes calls from different host threads.
 ChunkRec g_host_table[kNoAllocMaxChunks];
-struct Range { uintptr_t lo, hi; bool written; };
-Range g_ranges[4 * kNoAllocMaxChunks];
+opt2s::Range g_ranges[4 * kNoAllocMaxChunks];
 
 std::mutex g_mu;
 void* g_table_ptr[kMaxDevices];   // device address of g_noalloc_table, per device
 
-int elem_bytes(int32_t dtype) { return dtype == OPT2S_F32 ? 4 : 2; }
-
-// Same rules as opt2s_step's validation, written without heap use.
-int check_hyper(const Hyper* h, int step)
-{
-    if (!h) return OPT2S_ERR_INVALID_ARG;
-    if (h->algo != OPT2S_ADAM && h->algo != OPT2S_ADEMAMIX) return OPT2S_ERR_INVALID_ARG;
-    if (h->skip_zeros != 0 && h->skip_zeros != 1) return OPT2S_ERR_INVALID_ARG;
-    if (step < 1) return OPT2S_ERR_INVALID_ARG;
-    auto unit = [](float b) { return std::isfinite(b) && b >= 0.0f && b < 1.0f; };
-    if (!std::isfinite(h->lr) || !unit(h->beta1) || !unit(h->beta2)) return OPT2S_ERR_INVALID_ARG;
-    if (!std::isfinite(h->eps) || h->eps < 0.0f) return OPT2S_ERR_INVALID_ARG;
-    if (!std::isfinite(h->weight_decay)) return OPT2S_ERR_INVALID_ARG;
-    if (h->algo == OPT2S_ADEMAMIX && (!unit(h->beta3) || !std::isfinite(h->alpha)))
-        return OPT2S_ERR_INVALID_ARG;
-    return OPT2S_OK;
-}
-
-// Validates every record and counts the chunks, filling g_ranges; returns a
-// status.  *nchunks receives the chunk count (only meaningful on success).
+// Validates every record with the same rules as opt2s_step (shared from
+// opt2s_internal.h), checks buffer overlaps through the fixed g_ranges and
+// counts the chunks; *nchunks receives the count on success.
 int check_desc(const TensorListDesc* d, int32_t algo, int64_t chunk_elems, int64_t* nchunks)
 {
     if (!d || d->count < 0 || (d->count > 0 && !d->tensors)) return OPT2S_ERR_INVALID_ARG;
-    int64_t chunks = 0, nr = 0;
+    int64_t chunks = 0;
+    size_t nr = 0;
     for (int32_t i = 0; i < d->count; ++i) {
-        const opt2s_tensor& t = d->tensors[i];
-        if (t.numel < 0 || t.reserved != 0) return OPT2S_ERR_INVALID_ARG;
-        if (t.dtype != OPT2S_F32 && t.dtype != OPT2S_F16 && t.dtype != OPT2S_BF16)
-            return OPT2S_ERR_INVALID_ARG;
-        if (t.numel == 0) continue;
-        if (t.numel > (int64_t(1) << 40)) return OPT2S_ERR_INVALID_ARG;
-        if (!t.param || !t.grad || !t.state1 || !t.state2) return OPT2S_ERR_INVALID_ARG;
-        chunks += (t.numel + chunk_elems - 1) / chunk_elems;
+        opt2s::Range r[4];
+        int n = 0;
+        const int st = opt2s::record_ranges(d->tensors[i], algo, r, &n);
+        if (st != OPT2S_OK) return st;
+        if (n == 0) continue;
+        // every non-empty record takes at least one chunk, so while the count
+        // stays within the table, its ranges fit in g_ranges
+        chunks += (d->tensors[i].numel + chunk_elems - 1) / chunk_elems;
         if (chunks > kNoAllocMaxChunks) return OPT2S_ERR_TOO_LARGE;
-        const int es = elem_bytes(t.dtype);
-        const auto p = reinterpret_cast<uintptr_t>(t.param);
-        const auto g = reinterpret_cast<uintptr_t>(t.grad);
-        const auto s1 = reinterpret_cast<uintptr_t>(t.state1);
-        const auto s2 = reinterpret_cast<uintptr_t>(t.state2);
-        if (p % es || g % es || s1 % 4 || s2 % 4) return OPT2S_ERR_INVALID_ARG;
-        const uintptr_t n = static_cast<uintptr_t>(t.numel);
-        g_ranges[nr++] = {p, p + n * es, true};
-        g_ranges[nr++] = {g, g + n * es, false};
-        g_ranges[nr++] = {s1, s1 + (algo == OPT2S_ADEMAMIX ? 2 * n : n) * 4, true};
-        g_ranges[nr++] = {s2, s2 + n * 4, true};
+        for (int k = 0; k < n; ++k) g_ranges[nr++] = r[k];
     }
-    std::sort(g_ranges, g_ranges + nr, [](const Range& a, const Range& b) { return a.lo < b.lo; });
-    uintptr_t reach_w = 0, reach_any = 0;
-    bool have_w = false, have_any = false;
-    for (int64_t k = 0; k < nr; ++k) {
-        const Range& r = g_ranges[k];
-        if (have_w && r.lo < reach_w) return OPT2S_ERR_ALIAS;
-        if (r.written && have_any && r.lo < reach_any) return OPT2S_ERR_ALIAS;
-        if (r.written) { reach_w = have_w ? std::max(reach_w, r.hi) : r.hi; have_w = true; }
-        reach_any = have_any ? std::max(reach_any, r.hi) : r.hi;
-        have_any = true;
-    }
+    const int st = opt2s::overlap_status(g_ranges, nr);
+    if (st != OPT2S_OK) return st;
     *nchunks = chunks;
     return OPT2S_OK;
-}
-
-StepScalars scalars(const Hyper* h, int step)
-{
-    StepScalars s;
-    s.lr = h->lr;
-    s.beta1 = h->beta1;
-    s.beta2 = h->beta2;
-    s.beta3 = h->beta3;
-    s.one_minus_beta1 = 1.0f - h->beta1;
-    s.one_minus_beta2 = 1.0f - h->beta2;
-    s.one_minus_beta3 = 1.0f - h->beta3;
-    s.alpha = h->alpha;
-    s.eps = h->eps;
-    s.bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(h->beta1), static_cast<double>(step)));
-    s.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(h->beta2), static_cast<double>(step)));
-    s.decay = static_cast<float>(1.0 - static_cast<double>(h->lr) * static_cast<double>(h->weight_decay));
-    return s;
 }
 
 }  // namespace
@@ -146,7 +90,7 @@ StepScalars scalars(const Hyper* h, int step)
 OPT2S_API int opt2s_step_noalloc(const TensorListDesc* desc, const Hyper* hyper, int step,
                                  cudaStream_t stream)
 {
-    int st = check_hyper(hyper, step);
+    int st = opt2s::validate_hyper(hyper, step);
     if (st != OPT2S_OK) return st;
     std::lock_guard<std::mutex> lock(g_mu);
     const int64_t ce = kNoAllocChunkElems;
@@ -155,18 +99,22 @@ OPT2S_API int opt2s_step_noalloc(const TensorListDesc* desc, const Hyper* hyper,
     if (nchunks == 0) return OPT2S_OK;
 
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return OPT2S_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return opt2s::record_cuda_error(e);
+    if (dev < 0 || dev >= kMaxDevices) return opt2s::record_cuda_error(cudaErrorInvalidDevice);
     if (!g_table_ptr[dev]) {
         // once per device, with that device current
         void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_table) != cudaSuccess || !ptr) return OPT2S_ERR_CUDA;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_table);
+        if (e != cudaSuccess) return opt2s::record_cuda_error(e);
+        if (!ptr) return opt2s::record_cuda_error(cudaErrorInvalidSymbol);
         g_table_ptr[dev] = ptr;
     }
 
     int64_t k = 0;
     for (int32_t i = 0; i < desc->count; ++i) {
         const opt2s_tensor& t = desc->tensors[i];
-        const int es = elem_bytes(t.dtype);
+        const int es = opt2s::elem_bytes(t.dtype);
         for (int64_t s = 0; s < t.numel; s += ce) {
             ChunkRec& r = g_host_table[k++];
             r.p = static_cast<char*>(t.param) + s * es;
@@ -179,12 +127,12 @@ OPT2S_API int opt2s_step_noalloc(const TensorListDesc* desc, const Hyper* hyper,
         }
     }
     auto* table = static_cast<ChunkRec*>(g_table_ptr[dev]);
-    if (cudaMemcpyAsync(table, g_host_table, sizeof(ChunkRec) * nchunks, cudaMemcpyHostToDevice,
-                        stream) != cudaSuccess)
-        return OPT2S_ERR_CUDA;
-    if (opt2s::launch_step(table, nchunks, hyper->algo, hyper->skip_zeros, -1, scalars(hyper, step),
-                           opt2s::kDefaultBlockThreads, 0, stream) != cudaSuccess)
-        return OPT2S_ERR_CUDA;
+    e = cudaMemcpyAsync(table, g_host_table, sizeof(ChunkRec) * nchunks, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return opt2s::record_cuda_error(e);
+    e = opt2s::launch_step(table, nchunks, hyper->algo, hyper->skip_zeros, -1,
+                           opt2s::make_scalars(hyper, step), opt2s::kDefaultBlockThreads, 0, stream);
+    if (e != cudaSuccess) return opt2s::record_cuda_error(e);
+    opt2s::count_launches(1);
     return OPT2S_OK;
 }
 

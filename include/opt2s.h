@@ -228,8 +228,8 @@ int opt2s_shard_step(const opt2s_shard_desc *desc, const Hyper *hyper, int step,
  *
  * It calls no cudaMalloc, cudaFree or allocating library routine and keeps
  * no plan.  Each call builds the chunk table in a fixed host array and
- * uploads it (cudaMemcpyAsync on `stream`, from pageable memory, so the call
- * waits for `stream`'s earlier work) into a fixed device array of
+ * uploads it with cudaMemcpyAsync on `stream` (the copy and the launch are
+ * ordered on `stream` like any other work there) into a fixed device array of
  * opt2s_noalloc_max_chunks() records (65,536 records = 3 MiB), which every
  * GPU that loads the library holds until the process exits.  A collection
  * needing more chunk records (8,192 elements per chunk; at least one per
@@ -239,7 +239,8 @@ int opt2s_shard_step(const opt2s_shard_desc *desc, const Hyper *hyper, int step,
  * whose work overlaps on the GPU (unordered streams) race on the array.
  * The first call on each device looks up the array's device address and
  * caches it; make that first call before any stream capture begins.
- * Calls from several host threads are serialized.
+ * Calls from several host threads are serialized.  Each successful call
+ * counts one kernel launch.  CUDA failures are kept in opt2s_last_cuda_error.
  */
 int opt2s_step_noalloc(const TensorListDesc *desc, const Hyper *hyper, int step,
                        cudaStream_t stream);

@@ -2,11 +2,13 @@
 allocate device memory (a runtime that owns every byte of device memory
 through its own pool, or a deployment whose footprint is fixed at start-up).
 
-It must give the same results as opt2s_step, within the tolerance the parity
-tests use (fp32 within 2 ulp, fp16/bf16 within 1 ulp of the storage type;
-in practice bitwise), on two calls in a row -- the second call reuses the
-fixed device table the first one left behind -- and it must reject a
-collection larger than its fixed table before doing any work.
+It runs the same kernel and arithmetic as opt2s_step with another launch
+geometry (fixed 8,192-element chunks, 128-thread blocks), and launch geometry
+must not change a bit of the result.  So on two calls in a row -- the second
+call reuses the fixed device table the first one left behind -- its results
+must equal the oracle's bit for bit and opt2s_step's bit for bit, each call
+must count exactly one launch, and a collection larger than its fixed table
+must be rejected before any work (no launch, no update).
 
 This file is collected last on purpose, and it holds no state of its own
 between tests, so it passes both alone in a fresh process and after the rest
@@ -18,7 +20,7 @@ import torch
 
 from elementwise_optimizer_b200 import binding as B
 from elementwise_optimizer_b200 import synth
-from tests.gpu_support import Harness, storage_bits, ulp_distance
+from tests.gpu_support import Harness, storage_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -43,22 +45,25 @@ def _workload(algo):
 
 @pytest.mark.parametrize("layout", ["separate", "packed"])
 @pytest.mark.parametrize("algo", ["adam", "ademamix"])
-def test_noalloc_matches_opt2s_step_on_two_calls(algo, layout):
+def test_noalloc_matches_oracle_and_opt2s_step_on_two_calls(algo, layout):
     w = _workload(algo)
-    a = Harness(w, layout=layout)          # stepped by opt2s_step_noalloc
+    a = Harness(w, layout=layout)          # stepped by opt2s_step_noalloc, checked against the oracle
     b = Harness(w, layout=layout)          # stepped by opt2s_step
     for t in (1, 2):
         a.load_grads(t)
         b.load_grads(t)
+        before = B.launch_count()
         B.opt2s_step_noalloc(a.tl, a.hyper, t)
+        assert B.launch_count() == before + 1
         B.opt2s_step(b.tl, b.hyper, t)
+        a.oracle_step(t)
         torch.cuda.synchronize()
-        for i, dt in enumerate(w.dtypes):
-            tol = 2 if dt == "f32" else 1
-            assert ulp_distance(storage_bits(a.params[i]), storage_bits(b.params[i]), dt).max() <= tol
-            assert ulp_distance(storage_bits(a.s1[i]), storage_bits(b.s1[i]), "f32").max() <= 2
-            assert ulp_distance(storage_bits(a.s2[i]), storage_bits(b.s2[i]), "f32").max() <= 2
-            assert np.array_equal(storage_bits(a.grads[i]), storage_bits(b.grads[i]))
+        assert a.max_ulps() == {"param": 0, "state1": 0, "state2": 0}, t
+        assert a.grads_unchanged()
+        for i in range(len(w.sizes)):
+            assert np.array_equal(storage_bits(a.params[i]), storage_bits(b.params[i]))
+            assert np.array_equal(storage_bits(a.s1[i]), storage_bits(b.s1[i]))
+            assert np.array_equal(storage_bits(a.s2[i]), storage_bits(b.s2[i]))
 
 
 def test_noalloc_rejects_a_collection_beyond_its_table():
