@@ -10,7 +10,8 @@ What it computes and where each step comes from is stated in the header of
 ``opt2s_oracle.c`` (bitsandbytes issue "Investigate a 256-thread SM103 path
 for small 32-bit optimizer tensors", sections "Problem", "Scope" and
 "Correctness oracle"; Kingma & Ba 2015 Algorithm 1; Loshchilov & Hutter 2019
-Algorithm 2; Pagliardini et al. 2024 Algorithm 1).
+Algorithm 2; Pagliardini et al. 2024 Algorithm 1; You et al. 2020 Algorithm 2
+for LAMB).
 
 Every function here was pinned by ``tests/test_oracle_pins.py`` against
 values fixed by something other than the oracle itself (library optimizers in
@@ -77,6 +78,9 @@ def _load():
     lib.oracle_step_f32_max_unorm.argtypes = [i32, i32, i32, f32, f32, f32, f32, f32,
                                               f32, f32, f32, i32, vp, vp, vp, vp, i64, vp]
     lib.oracle_step_f32_max_unorm.restype = i32
+    lib.oracle_step_f32_lamb.argtypes = [i32, i32, f32, f32, f32, f32, f32, i32,
+                                         vp, vp, vp, vp, i64, vp]
+    lib.oracle_step_f32_lamb.restype = i32
     lib.oracle_average_grads.argtypes = [i32, i32, vp, vp, i64]
     lib.oracle_average_grads.restype = i32
     lib.oracle_bias_correction.argtypes = [f32, i32]
@@ -151,6 +155,29 @@ def step_f32_max_unorm(param: np.ndarray, grad: np.ndarray, state1: np.ndarray,
     if rc != 0:
         raise ValueError(f"oracle_step_f32_max_unorm rejected its arguments ({rc})")
     return float(scale[0])
+
+
+def step_f32_lamb(param: np.ndarray, grad: np.ndarray, m: np.ndarray,
+                  v: np.ndarray, *, dtype: str, step: int, lr: float, beta1: float,
+                  beta2: float, eps: float, weight_decay: float = 0.0,
+                  skip_zeros: bool = False) -> float:
+    """One LAMB step (You et al. 2020, Algorithm 2) over one tensor, in place:
+    the Adam direction plus weight_decay * param, scaled by the trust ratio
+    ||param|| / ||direction||.  ``param``/``grad`` hold storage bits of
+    ``dtype``; ``m``, ``v`` are float32.  Returns the fp32 trust ratio."""
+    n = param.size
+    if grad.size != n or param.itemsize != _ITEMSIZE[dtype] or \
+            grad.itemsize != _ITEMSIZE[dtype]:
+        raise ValueError("param/grad size or item size mismatch")
+    if m.dtype != np.float32 or v.dtype != np.float32 or m.size != n or v.size != n:
+        raise ValueError("state arrays must be float32 of the param's size")
+    ratio = np.zeros(1, np.float32)
+    rc = _load().oracle_step_f32_lamb(
+        DTYPE[dtype], int(bool(skip_zeros)), lr, beta1, beta2, eps, weight_decay,
+        int(step), _ptr(param), _ptr(grad), _ptr(m), _ptr(v), n, _ptr(ratio))
+    if rc != 0:
+        raise ValueError(f"oracle_step_f32_lamb rejected its arguments ({rc})")
+    return float(ratio[0])
 
 
 def step_f32_fgrad(param: np.ndarray, grad: np.ndarray, state1: np.ndarray,

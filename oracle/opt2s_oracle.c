@@ -32,6 +32,9 @@
  *              Better, Faster, Older", 2024, Algorithm 1 (a second, slow EMA
  *              m2 with rate beta3, not bias-corrected, mixed in with weight
  *              alpha).
+ *   [LAMB]     You et al., "Large Batch Optimization for Deep Learning:
+ *              Training BERT in 76 minutes", ICLR 2020, Algorithm 2 (per-layer
+ *              trust ratio ||x|| / ||r + lambda x||).
  *   [IEEE754]  IEEE 754-2008, section 4.3.1 (roundTiesToEven) and 3.6
  *              (binary16 format); bfloat16 is the upper half of binary32.
  *
@@ -50,6 +53,8 @@
  *   - max_unorm > 0 (oracle_step_f32_max_unorm): the tensor's update norm is
  *     bounded by max_unorm times its weight norm, as written out above that
  *     function; the pages name the option without its arithmetic.
+ *   - LAMB (oracle_step_f32_lamb): You et al. 2020, Algorithm 2, per tensor,
+ *     with the readings written out above that function.
  */
 #include <math.h>
 #include <stdint.h>
@@ -414,6 +419,82 @@ int oracle_step_f32_max_unorm(int algo, int dtype, int skip_zeros,
         m[i] = mi;
         v[i] = vi;
         if (algo == OR_ADEMAMIX) m2[i] = m2i;
+    }
+
+    _mm_setcsr(csr);
+    return 0;
+}
+
+/*
+ * LAMB: the layer-wise adaptive step of You et al., "Large Batch Optimization
+ * for Deep Learning: Training BERT in 76 minutes", ICLR 2020, Algorithm 2,
+ * over one tensor (the "layer").  [issue] "Scope" keeps the two-state kernel
+ * "for max-unorm/LAMB use"; the pages do not write LAMB out, so the paper's
+ * Algorithm 2 is followed, with these readings:
+ *   u_i = num_i / den_i, the bias-corrected Adam direction of element i
+ *         exactly as in the plain fp32 step (Algorithm 2's r_t);
+ *   w_i = u_i + wd*p_i in fp32 (the weight decay lambda sits inside the
+ *         trust ratio, as in Algorithm 2, not the decay-first AdamW form);
+ *   W   = sqrt(sum_i w_i^2), P = sqrt(sum_i p_i^2) over the tensor, p the
+ *         stored param before the step, squares, sums and roots in binary64,
+ *         summed in index order;
+ *   r   = P/W rounded to fp32 once, if P > 0 and W > 0, else 1: the scaling
+ *         function phi is the identity (the paper's experiments), and a zero
+ *         norm (a zero-initialised tensor, or no update) takes ratio 1 so
+ *         that such a tensor still moves (the paper leaves 0/x and x/0 open);
+ *   p_i = p_i - lr*(r*w_i) in fp32; m and v exactly as in the plain step.
+ * skip_zeros: an element whose gradient is zero keeps p, m and v; its p_i
+ * counts in P and it adds nothing to W.  Adam moments only (algo 0).
+ * Returns 0, or -1 on an argument the definitions do not cover.
+ */
+int oracle_step_f32_lamb(int dtype, int skip_zeros, float lr, float beta1,
+                         float beta2, float eps, float weight_decay, int step,
+                         void *param, const void *grad, float *state1,
+                         float *state2, int64_t n, float *ratio_out)
+{
+    if (step < 1 || n < 0) return -1;
+    if (dtype != OR_F32 && dtype != OR_F16 && dtype != OR_BF16) return -1;
+
+    unsigned int csr = _mm_getcsr();
+    _mm_setcsr(csr & ~(0x8000u | 0x0040u));             /* FTZ and DAZ off */
+
+    const float bc1 = oracle_bias_correction(beta1, step);
+    const float bc2 = oracle_bias_correction(beta2, step);
+    const float one_minus_b1 = 1.0f - beta1;
+    const float one_minus_b2 = 1.0f - beta2;
+    float *m = state1;
+    float *v = state2;
+
+    /* pass 1: the norms of the weights and of the decayed direction */
+    double sw = 0.0, sp = 0.0;
+    for (int64_t i = 0; i < n; i++) {
+        float p = load_param(param, dtype, i);
+        sp += (double)p * (double)p;
+        float g = load_param(grad, dtype, i);
+        if (skip_zeros && g == 0.0f) continue;
+        float mi, m2i, vi, u;
+        element_direction(OR_ADAM, g, m[i], 0.0f, v[i], beta1, beta2, 0.0f, 0.0f, eps,
+                          bc1, bc2, one_minus_b1, one_minus_b2, 0.0f, &mi, &m2i, &vi, &u);
+        float w = u + weight_decay * p;
+        sw += (double)w * (double)w;
+    }
+    const double W = sqrt(sw), P = sqrt(sp);
+    const float ratio = (P > 0.0 && W > 0.0) ? (float)(P / W) : 1.0f;
+    if (ratio_out) *ratio_out = ratio;
+
+    /* pass 2: the update along w, scaled by the trust ratio */
+    for (int64_t i = 0; i < n; i++) {
+        float g = load_param(grad, dtype, i);
+        if (skip_zeros && g == 0.0f) continue;
+        float p = load_param(param, dtype, i);
+        float mi, m2i, vi, u;
+        element_direction(OR_ADAM, g, m[i], 0.0f, v[i], beta1, beta2, 0.0f, 0.0f, eps,
+                          bc1, bc2, one_minus_b1, one_minus_b2, 0.0f, &mi, &m2i, &vi, &u);
+        float w = u + weight_decay * p;
+        p = p - lr * (ratio * w);
+        store_param(param, dtype, i, p);
+        m[i] = mi;
+        v[i] = vi;
     }
 
     _mm_setcsr(csr);

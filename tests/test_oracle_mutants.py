@@ -58,6 +58,22 @@ MUTANTS = {
         "sp += (double)p * (double)p;\n        float g = load_param(grad, dtype, i);\n"
         "        if (skip_zeros && g == 0.0f) continue;\n",
         "sp += (double)p * (double)p;\n        float g = load_param(grad, dtype, i);\n"),
+    "lamb_ratio_inverted": ("(float)(P / W)", "(float)(W / P)"),
+    "lamb_zero_weight_ratio_zero": ("(P > 0.0 && W > 0.0) ? (float)(P / W) : 1.0f",
+                                    "(W > 0.0) ? (float)(P / W) : 1.0f"),
+    "lamb_norm_without_decay": ("float w = u + weight_decay * p;\n        sw +=",
+                                "float w = u;\n        sw +="),
+    "lamb_decay_sign_in_update": ("float w = u + weight_decay * p;\n        p = p - lr",
+                                  "float w = u - weight_decay * p;\n        p = p - lr"),
+    "lamb_decay_outside_ratio": ("p = p - lr * (ratio * w);",
+                                 "p = p - lr * (ratio * u) - lr * (weight_decay * p);"),
+    "lamb_ratio_dropped": ("p = p - lr * (ratio * w);", "p = p - lr * w;"),
+    "lamb_counts_skipped": (
+        "sp += (double)p * (double)p;\n        float g = load_param(grad, dtype, i);\n"
+        "        if (skip_zeros && g == 0.0f) continue;\n        float mi, m2i, vi, u;\n"
+        "        element_direction(OR_ADAM",
+        "sp += (double)p * (double)p;\n        float g = load_param(grad, dtype, i);\n"
+        "        float mi, m2i, vi, u;\n        element_direction(OR_ADAM"),
 }
 
 

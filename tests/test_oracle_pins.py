@@ -561,3 +561,133 @@ def test_max_unorm_must_be_positive(oracle_mod):
         with pytest.raises(ValueError):
             oracle_mod.step_f32_max_unorm(p, gr, s1, v, dtype="f32", algo="adam", step=1,
                                           max_unorm=mu, **UNORM_HYPER)
+
+
+# --------------------------------------------------------------------------
+# LAMB (You et al. 2020, Algorithm 2): per tensor, the Adam direction plus
+# lambda*p, scaled by the trust ratio ||p|| / ||direction + lambda*p||.
+# --------------------------------------------------------------------------
+
+LAMB_HYPER = dict(lr=0.01, beta1=0.9, beta2=0.999, eps=1e-6)
+
+
+def _lamb_state(seed, n, dtype):
+    p, gr, m, v = _random_state(seed, n, dtype, "adam")
+    return p, gr, m, v
+
+
+@pytest.mark.parametrize("p0,wd", [(0.5, 0.0), (-4.0, 0.5), (3.0, 0.1)])
+def test_lamb_step_one_closed_form(oracle_mod, p0, wd):
+    """Every element equal: p0 and g = 0.25 at t = 1 give every element the
+    same direction u = g/(|g| + eps) (m/bc1 = g and sqrt(v/bc2) = |g| in
+    exact arithmetic), so w = u + wd*p0 for all of them and the trust
+    ratio is |p0| / |w|: each element moves by lr*|p0| against the sign of w.
+    (p0 = -4 with wd = 0.5 gives w = -1: the decay term inside w decides the
+    direction.)"""
+    n = 4096
+    p = np.full(n, p0, np.float32)
+    g = np.full(n, 0.25, np.float32)
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    r = oracle_mod.step_f32_lamb(p, g, m, v, dtype="f32", step=1, weight_decay=wd, **LAMB_HYPER)
+    u = 0.25 / (0.25 + LAMB_HYPER["eps"])
+    w = u + wd * p0
+    want = p0 - LAMB_HYPER["lr"] * abs(p0) * math.copysign(1.0, w)
+    assert r == pytest.approx(abs(p0) / abs(w), rel=1e-6)
+    assert np.all(p == p[0])
+    assert abs(float(p[0]) - want) <= 8 * float(ulp32(want)), (float(p[0]), want)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("wd", [0.0, 0.01, 0.3])
+@pytest.mark.parametrize("t", [1, 10, 1000])
+def test_lamb_update_is_the_trust_ratio_times_the_decayed_direction(oracle_mod, dtype, wd, t):
+    """Against the float64 shadow: the Adam direction u of every element is
+    taken from the shadow step (pinned to torch.optim.Adam) run with lr = 1
+    and no decay, w = u + wd*p0 and the trust ratio ||p0|| / ||w|| in float64.
+    The oracle's applied update p1 - p0 must equal -lr*ratio*w elementwise up
+    to fp32 rounding, and its norm must be lr*||p0||; skipped elements do
+    not move and add nothing to ||w||; the moments are the plain step's."""
+    n = 20000
+    for skip in (False, True):
+        p, gr, m, v = _lamb_state(600 + t, n, dtype)
+        if skip:
+            gr[::3] = 0
+        pf = synth.from_storage(p, dtype).astype(np.float64)
+        gf = synth.from_storage(gr, dtype).astype(np.float64)
+        sh_p, sh_m, sh_v = pf.copy(), m.astype(np.float64), v.astype(np.float64)
+        h32 = {k: float(np.float32(x)) for k, x in LAMB_HYPER.items()}
+        oracle_mod.step_f64(sh_p, gf, sh_m, sh_v, algo="adam", step=t, lr=1.0,
+                            beta1=h32["beta1"], beta2=h32["beta2"], eps=h32["eps"],
+                            skip_zeros=skip)
+        u = pf - sh_p
+        w = u + float(np.float32(wd)) * pf
+        live = ~((gr.view(np.uint16 if dtype != "f32" else np.uint32) << 1) == 0) if skip else \
+            np.ones(n, bool)
+        w[~live] = 0.0
+        ratio = np.linalg.norm(pf) / np.linalg.norm(w)
+        q, m1, v1 = p.copy(), m.copy(), v.copy()
+        r = oracle_mod.step_f32_lamb(q, gr, m1, v1, dtype=dtype, step=t, weight_decay=wd,
+                                     skip_zeros=skip, **LAMB_HYPER)
+        assert r == pytest.approx(ratio, rel=1e-5)
+        d = synth.from_storage(q, dtype).astype(np.float64) - pf
+        want = -LAMB_HYPER["lr"] * ratio * w
+        # each element: fp32 rounding of w (relative to |u| + |wd p|), of the
+        # products and of the final subtraction (one ulp of p in storage)
+        quantum = np.spacing(np.abs(synth.from_storage(q, dtype)).astype(np.float32)).astype(np.float64)
+        if dtype == "bf16":
+            quantum = quantum * 2.0 ** 16
+        slack = (LAMB_HYPER["lr"] * ratio * (np.abs(u) + abs(wd) * np.abs(pf)) * 1e-5 + quantum)
+        assert np.all(np.abs(d - want) <= slack)
+        if dtype == "f32":
+            assert np.linalg.norm(d) == pytest.approx(LAMB_HYPER["lr"] * np.linalg.norm(pf), rel=1e-4)
+        assert np.array_equal(q[~live], p[~live])
+        plain_p, plain_m, plain_v = p.copy(), m.copy(), v.copy()
+        oracle_mod.step_f32(plain_p, gr, plain_m, plain_v, dtype=dtype, algo="adam", step=t,
+                            skip_zeros=skip, **LAMB_HYPER)
+        assert np.array_equal(m1, plain_m) and np.array_equal(v1, plain_v)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_lamb_zero_weights_take_ratio_one(oracle_mod, dtype):
+    """||p0|| = 0 takes trust ratio 1, so from p0 = 0 the LAMB step is
+    p1 = 0 - lr*u, bit for bit the plain Adam step from p0 = 0 without decay
+    (0*decay - lr*u)."""
+    n = 3000
+    _, gr, m, v = _lamb_state(700, n, dtype)
+    p = synth.to_storage(np.zeros(n, np.float32), dtype)
+    a = (p.copy(), m.copy(), v.copy())
+    b = (p.copy(), m.copy(), v.copy())
+    r = oracle_mod.step_f32_lamb(a[0], gr, a[1], a[2], dtype=dtype, step=5, weight_decay=0.2,
+                                 **LAMB_HYPER)
+    oracle_mod.step_f32(b[0], gr, b[1], b[2], dtype=dtype, algo="adam", step=5, **LAMB_HYPER)
+    assert r == 1.0
+    for x, y in zip(a, b):
+        assert np.array_equal(x.view(np.uint8), y.view(np.uint8))
+
+
+def test_lamb_zero_gradient_closed_forms(oracle_mod):
+    """From zero moments and g = 0: the direction is u = 0, so w = wd*p.
+    Without decay W = 0 and the ratio is 1, leaving p unchanged; with decay
+    W = wd*||p||, the ratio 1/wd, and every element becomes p*(1 - lr) up to
+    rounding."""
+    n = 5000
+    p, _, _, _ = _lamb_state(800, n, "f32")
+    g = np.zeros(n, np.float32)
+    q = p.copy()
+    r = oracle_mod.step_f32_lamb(q, g, np.zeros(n, np.float32), np.zeros(n, np.float32),
+                                 dtype="f32", step=3, weight_decay=0.0, **LAMB_HYPER)
+    assert r == 1.0 and np.array_equal(q, p)
+    q = p.copy()
+    wd = 0.25
+    r = oracle_mod.step_f32_lamb(q, g, np.zeros(n, np.float32), np.zeros(n, np.float32),
+                                 dtype="f32", step=3, weight_decay=wd, **LAMB_HYPER)
+    assert r == pytest.approx(1.0 / wd, rel=1e-6)
+    want = p.astype(np.float64) * (1.0 - LAMB_HYPER["lr"])
+    assert np.all(np.abs(q - want) <= 4 * ulp32(want))
+
+
+def test_lamb_rejects_step_zero(oracle_mod):
+    p, gr, m, v = _lamb_state(900, 16, "f32")
+    with pytest.raises(ValueError):
+        oracle_mod.step_f32_lamb(p, gr, m, v, dtype="f32", step=0, **LAMB_HYPER)
