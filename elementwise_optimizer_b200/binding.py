@@ -93,6 +93,8 @@ EXPORTS = {
     "opt2s_noalloc_max_chunks": (ctypes.c_int64, []),
     "opt2s_step_max_unorm": (ctypes.c_int, [ctypes.POINTER(TensorListDesc), ctypes.POINTER(Hyper),
                                             ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
+    "opt2s_step_lamb": (ctypes.c_int, [ctypes.POINTER(TensorListDesc), ctypes.POINTER(Hyper),
+                                       ctypes.c_int, ctypes.c_void_p]),
     "opt2s_fill_step_scalars": (ctypes.c_int, [ctypes.POINTER(Hyper), ctypes.c_int, ctypes.c_int,
                                                ctypes.c_void_p]),
     "opt2s_plan_step_table": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
@@ -266,6 +268,14 @@ def opt2s_step_max_unorm(tl: TensorList, hyper: Hyper, max_unorm: float, step: i
     check(lib().opt2s_step_max_unorm(ctypes.byref(tl.desc), ctypes.byref(hyper),
                                      float(max_unorm), int(step), _stream_handle(stream)),
           "opt2s_step_max_unorm")
+
+
+def opt2s_step_lamb(tl: TensorList, hyper: Hyper, step: int, stream=None) -> None:
+    """The LAMB step (You et al. 2020, Algorithm 2; Adam moments): per tensor,
+    the Adam direction plus weight_decay * param, scaled by the trust ratio
+    ||param|| / ||direction||; four launches on `stream`."""
+    check(lib().opt2s_step_lamb(ctypes.byref(tl.desc), ctypes.byref(hyper), int(step),
+                                _stream_handle(stream)), "opt2s_step_lamb")
 
 
 def noalloc_max_chunks() -> int:

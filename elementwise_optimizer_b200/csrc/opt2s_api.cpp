@@ -454,13 +454,17 @@ int cached_plan(const TensorListDesc* desc, int32_t algo, bool unorm, const opt2
     return OPT2S_OK;
 }
 
-int plan_step_max_unorm(const opt2s_plan* plan, const Hyper* h, float max_unorm, int step,
-                        cudaStream_t stream)
+// One step of a plan with per-tensor norms: the bounded update norm
+// (lamb == false, max_unorm > 0) or LAMB (lamb == true, Adam moments, the
+// weight decay inside the trust-ratio scaled update).
+int plan_step_normed(const opt2s_plan* plan, const Hyper* h, bool lamb, float max_unorm, int step,
+                     cudaStream_t stream)
 {
     if (!plan) return OPT2S_ERR_INVALID_ARG;
     int st = validate_hyper(h, step);
     if (st != OPT2S_OK) return st;
-    if (!std::isfinite(max_unorm) || !(max_unorm > 0.0f)) return OPT2S_ERR_INVALID_ARG;
+    if (lamb ? h->algo != OPT2S_ADAM : (!std::isfinite(max_unorm) || !(max_unorm > 0.0f)))
+        return OPT2S_ERR_INVALID_ARG;
     if (h->algo != plan->algo) return OPT2S_ERR_INVALID_ARG;
     if (plan->nchunks == 0) return OPT2S_OK;
     if (!plan->d_unorm) return OPT2S_ERR_INVALID_ARG;
@@ -471,13 +475,17 @@ int plan_step_max_unorm(const opt2s_plan* plan, const Hyper* h, float max_unorm,
     const int bt = block_threads_now(h->algo, -1);
     if (g_block_threads > 0) {   // forced geometry: must fit the kernel
         int widest = 0;
-        e = opt2s::max_block_threads_scaled(h->algo, h->skip_zeros, &widest);
+        e = opt2s::max_block_threads_scaled(h->algo, h->skip_zeros, lamb ? 1 : 0, &widest);
         if (e != cudaSuccess) return cuda_fail(e);
         if (bt > widest) return OPT2S_ERR_INVALID_ARG;
     }
-    e = opt2s::launch_step_max_unorm(plan->d_chunks, plan->nchunks, h->algo, h->skip_zeros,
-                                     make_scalars(h, step), plan->unorm, max_unorm, bt,
-                                     g_max_blocks, stream);
+    if (lamb)
+        e = opt2s::launch_step_lamb(plan->d_chunks, plan->nchunks, h->skip_zeros, make_scalars(h, step),
+                                    h->weight_decay, plan->unorm, bt, g_max_blocks, stream);
+    else
+        e = opt2s::launch_step_max_unorm(plan->d_chunks, plan->nchunks, h->algo, h->skip_zeros,
+                                         make_scalars(h, step), plan->unorm, max_unorm, bt,
+                                         g_max_blocks, stream);
     if (e != cudaSuccess) return cuda_fail(e);
     const int launched = (plan->unorm.nblocks > 0) + (plan->unorm.ngroups > 0) +
                          (plan->unorm.ntensors > 0) + 1;
@@ -515,7 +523,23 @@ OPT2S_API int opt2s_step_max_unorm(const TensorListDesc* desc, const Hyper* hype
     const opt2s_plan* plan = nullptr;
     st = cached_plan(desc, hyper->algo, true, &plan);
     if (st != OPT2S_OK || !plan) return st;
-    return plan_step_max_unorm(plan, hyper, max_unorm, step, stream);
+    return plan_step_normed(plan, hyper, false, max_unorm, step, stream);
+}
+
+OPT2S_API int opt2s_step_lamb(const TensorListDesc* desc, const Hyper* hyper, int step,
+                              cudaStream_t stream)
+{
+    int st = validate_hyper(hyper, step);
+    if (st != OPT2S_OK) return st;
+    if (hyper->algo != OPT2S_ADAM) return OPT2S_ERR_INVALID_ARG;
+    if (!desc || desc->count < 0 || (desc->count > 0 && !desc->tensors))
+        return OPT2S_ERR_INVALID_ARG;
+    if (desc->count == 0) return OPT2S_OK;
+    std::unique_lock<std::mutex> lock(g_cache_mu);
+    const opt2s_plan* plan = nullptr;
+    st = cached_plan(desc, hyper->algo, true, &plan);   // the max_unorm step's tables
+    if (st != OPT2S_OK || !plan) return st;
+    return plan_step_normed(plan, hyper, true, 0.0f, step, stream);
 }
 
 OPT2S_API int opt2s_plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out_plan)

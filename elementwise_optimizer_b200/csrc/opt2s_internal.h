@@ -135,8 +135,17 @@ cudaError_t launch_step_max_unorm(const ChunkRec* d_chunks, int64_t nchunks, int
                                   float max_unorm, int block_threads, int max_blocks,
                                   cudaStream_t stream);
 
-// Widest block the scaled step kernel can launch with.
-cudaError_t max_block_threads_scaled(int algo, int skip_zeros, int* out);
+// Launches the four kernels of the LAMB step (Adam moments) on `stream`: the
+// same tables and launches, with the sums of (u + weight_decay*p)^2, the
+// trust ratio ||p|| / ||u + weight_decay*p|| per tensor, and
+// p = p - lr*(ratio*(u + weight_decay*p)).
+cudaError_t launch_step_lamb(const ChunkRec* d_chunks, int64_t nchunks, int skip_zeros,
+                             const StepScalars& s, float weight_decay, const UnormArgs& u,
+                             int block_threads, int max_blocks, cudaStream_t stream);
+
+// Widest block the scaled step kernel (bounded norm, or LAMB when `lamb`)
+// can launch with.
+cudaError_t max_block_threads_scaled(int algo, int skip_zeros, int lamb, int* out);
 
 // Sets s->inv_bc1, s->inv_bc2 = RN64(1/bc1), RN64(1/bc2) (host).
 void fill_reciprocals(StepScalars* s);

@@ -75,11 +75,16 @@ __device__ __forceinline__ float div_by_constant(float x, double r)
 // The per-element update.  direction() moves the moments of one element (in
 // place) and returns its update direction u = num/den; m/bc1 and v/bc2 use
 // the exact constant division above, num/den is an IEEE division.  update()
-// then applies p = p*decay - lr*u.  With SKIP, an element whose gradient
-// compares equal to zero (+0 or -0) is left untouched (no decay either).
-// SCALED (the bounded-update-norm step): p = p*decay - lr*(scale*u), which for
-// scale = 1 is the same value.
+// then applies the step to p.  With SKIP, an element whose gradient compares
+// equal to zero (+0 or -0) is left untouched (no decay either).  MODE:
+//   kPlain   p = p*decay - lr*u
+//   kScaled  p = p*decay - lr*(scale*u)   (bounded update norm; scale = 1
+//                                          gives the plain value)
+//   kLamb    p = p - lr*(scale*w), w = u + wd*p   (LAMB: the weight decay
+//                                          inside the trust-ratio scaled step)
 // ---------------------------------------------------------------------------
+enum : int { kPlain = 0, kScaled = 1, kLamb = 2 };
+
 template <int ALGO>
 __device__ __forceinline__ float direction(float g, float& m, float& v, float& m2,
                                            const StepScalars& s)
@@ -96,13 +101,23 @@ __device__ __forceinline__ float direction(float g, float& m, float& v, float& m
     return __fdiv_rn(num, den);
 }
 
-template <int ALGO, bool SKIP, bool SCALED = false>
+// LAMB's decayed direction w = u + wd*p of an element.
+__device__ __forceinline__ float lamb_direction(float u, float p, float wd)
+{
+    return __fadd_rn(u, __fmul_rn(wd, p));
+}
+
+template <int ALGO, bool SKIP, int MODE = kPlain>
 __device__ __forceinline__ void update(float g, float& p, float& m, float& v,
-                                       float& m2, const StepScalars& s, float scale = 1.0f)
+                                       float& m2, const StepScalars& s, float scale = 1.0f,
+                                       float wd = 0.0f)
 {
     if (SKIP && g == 0.0f) return;
     const float u = direction<ALGO>(g, m, v, m2, s);
-    p = __fsub_rn(__fmul_rn(p, s.decay), __fmul_rn(s.lr, SCALED ? __fmul_rn(scale, u) : u));
+    if (MODE == kLamb)
+        p = __fsub_rn(p, __fmul_rn(s.lr, __fmul_rn(scale, lamb_direction(u, p, wd))));
+    else
+        p = __fsub_rn(__fmul_rn(p, s.decay), __fmul_rn(s.lr, MODE == kScaled ? __fmul_rn(scale, u) : u));
 }
 
 // ---------------------------------------------------------------------------
@@ -259,9 +274,10 @@ __device__ __forceinline__ void store_state(float* b, uint32_t i, const float (&
 // One element through the scalar path (chunk head, tail, or a chunk whose
 // arrays are not mutually 16-byte aligned).  A skipped element is not even
 // written back.
-template <int DT, int ALGO, bool SKIP, bool SCALED = false>
+template <int DT, int ALGO, bool SKIP, int MODE = kPlain>
 __device__ __forceinline__ void scalar_element(const ChunkRec& c, uint32_t i,
-                                               const StepScalars& s, float scale = 1.0f)
+                                               const StepScalars& s, float scale = 1.0f,
+                                               float wd = 0.0f)
 {
     using P = Param<DT>;
     const float g = P::load1(c.g, i);
@@ -271,7 +287,7 @@ __device__ __forceinline__ void scalar_element(const ChunkRec& c, uint32_t i,
     float v = ld_global(c.v + i);
     float m2 = 0.0f;
     if (ALGO == kAdEMAMix) m2 = ld_global(c.m2 + i);
-    update<ALGO, false, SCALED>(g, p, m, v, m2, s, scale);
+    update<ALGO, false, MODE>(g, p, m, v, m2, s, scale, wd);
     P::store1(c.p, i, p);
     st_global(c.m + i, m);
     st_global(c.v + i, v);
@@ -295,10 +311,10 @@ struct Aligned {
 // elements per iteration (two 16-byte vectors of fp32, or one of fp16/bf16),
 // so a warp iteration covers 256 contiguous elements of each array; the mixed
 // case moves one vector per lane per iteration.
-template <int DT, int ALGO, bool SKIP, bool ALL, bool SCALED = false>
+template <int DT, int ALGO, bool SKIP, bool ALL, int MODE = kPlain>
 __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars& s, int lane,
                                             uint32_t head, uint32_t nvec, Aligned al,
-                                            float scale = 1.0f)
+                                            float scale = 1.0f, float wd = 0.0f)
 {
     using P = Param<DT>;
     constexpr int V = P::kVec;
@@ -329,7 +345,7 @@ __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars
                 P::widen(praw[u], p);
 #pragma unroll
                 for (int j = 0; j < V; ++j)
-                    update<ALGO, SKIP, SCALED>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s, scale);
+                    update<ALGO, SKIP, MODE>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s, scale, wd);
                 P::store(c.p, e, P::narrow(p, praw[u], g, SKIP));
                 store_state_any<V>(c.m, e, ALL || al.m, m[u]);
                 store_state_any<V>(c.v, e, ALL || al.v, v[u]);
@@ -341,9 +357,9 @@ __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars
 
 // One chunk, processed by one warp: a scalar head up to the element at which
 // param is 16-byte aligned, the vector body, and a scalar tail.
-template <int DT, int ALGO, bool SKIP, bool SCALED = false>
+template <int DT, int ALGO, bool SKIP, int MODE = kPlain>
 __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& s, int lane,
-                                          float scale = 1.0f)
+                                          float scale = 1.0f, float wd = 0.0f)
 {
     using P = Param<DT>;
     constexpr int V = P::kVec;
@@ -355,16 +371,16 @@ __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& 
     const uint32_t body_end = head + nvec * V;
 
     for (uint32_t i = lane; i < head; i += 32)
-        scalar_element<DT, ALGO, SKIP, SCALED>(c, i, s, scale);
+        scalar_element<DT, ALGO, SKIP, MODE>(c, i, s, scale, wd);
     for (uint32_t i = body_end + lane; i < len; i += 32)
-        scalar_element<DT, ALGO, SKIP, SCALED>(c, i, s, scale);
+        scalar_element<DT, ALGO, SKIP, MODE>(c, i, s, scale, wd);
 
     const Aligned al{aligned16(c.g, head, P::kBytes), aligned16(c.m, head, 4),
                      aligned16(c.v, head, 4), ALGO != kAdEMAMix || aligned16(c.m2, head, 4)};
     if (al.all())
-        vector_body<DT, ALGO, SKIP, true, SCALED>(c, s, lane, head, nvec, al, scale);
+        vector_body<DT, ALGO, SKIP, true, MODE>(c, s, lane, head, nvec, al, scale, wd);
     else
-        vector_body<DT, ALGO, SKIP, false, SCALED>(c, s, lane, head, nvec, al, scale);
+        vector_body<DT, ALGO, SKIP, false, MODE>(c, s, lane, head, nvec, al, scale, wd);
 }
 
 // A short 16-bit chunk (its record's dtype carries kShortFlag), processed by
@@ -633,19 +649,26 @@ __global__ void advance_index_kernel(int* index, int table_len)
 }
 
 // ---------------------------------------------------------------------------
-// The step with bounded update norms (max_unorm > 0), four launches:
+// The steps with per-tensor norms, four launches each:
+//   * bounded update norm (max_unorm > 0): the norm of the update direction
+//     u is bounded by max_unorm times the weight norm;
+//   * LAMB (You et al. 2020, Algorithm 2): the decayed direction w = u + wd*p
+//     is scaled by the trust ratio ||p|| / ||w||.
+// The launches:
 //   1. unorm_partials_kernel: for every block of kNormBlockElems elements of
 //      a tensor (the host's norm table, fixed blocks whatever the plan's
-//      chunk length), the binary64 sums of u^2 (u = num/den, the update
-//      direction; 0 for an element skip_zeros leaves alone) and of p^2 (p
-//      the param before the step).  Nothing is written but the two sums;
+//      chunk length), the sums of d^2 (d = u, or w for LAMB; 0 for an element
+//      skip_zeros leaves alone) and of p^2 (p the param before the step).
+//      Nothing is written but the two sums;
 //   2. unorm_group_kernel: the sums of each group of kNormGroupBlocks
 //      consecutive blocks of a tensor (one warp per group);
-//      unorm_scale_kernel: per tensor, the sums of its groups, U = sqrt(su),
-//      P = sqrt(sp), and scale = max_unorm*P/U if U > max_unorm*P, else 1
-//      (binary64, rounded to fp32 once);
-//   3. step_kernel_scaled: the step over the plan's chunks with
-//      p = p*decay - lr*(scale*u), scale read through the chunk's tensor.
+//   3. unorm_scale_kernel: per tensor, the sums of its groups, D = sqrt(sd),
+//      P = sqrt(sp), and the scale (binary64, rounded to fp32 once):
+//      max_unorm*P/D if D > max_unorm*P, else 1; or for LAMB P/D if P > 0
+//      and D > 0, else 1;
+//   4. step_kernel_scaled: the step over the plan's chunks with
+//      p = p*decay - lr*(scale*u), or p = p - lr*(scale*w) for LAMB, the
+//      scale read through the chunk's tensor.
 // The element arithmetic is direction(), as in the plain step.  Every sum
 // has a fixed order: lane l of the warp that owns a block adds the block's
 // elements l, l + 32, l + 64, ... one after the other, the 32 lanes then
@@ -653,14 +676,57 @@ __global__ void advance_index_kernel(int* index, int table_len)
 // combined in fixed orders too; so the scale does not depend on the plan's
 // chunk length, the block width or the storage alignment.  Accesses are
 // element-wise and contiguous across the warp.
+//
+// Each lane accumulates its 64 squares of a block as a double-float: an
+// unevaluated sum hi + lo of two binary32 numbers.  The square of a binary32
+// x is exactly sq + err with sq = RN(x*x) and err = fma(x, x, -sq) (exact for
+// 2^-50 <= |x| <= 2^56: no underflow of err, and 64 squares stay below
+// 2^128), and hi + sq is split exactly into s + e by Knuth's TwoSum (Knuth,
+// TAOCP vol. 2, 4.2.2, Theorem B); only lo + (e + err) is rounded, which
+// errs by at most 2^-48 of the running sum.  Elements outside that range
+// are added to a binary64 sum instead.  The lane's total is hi + lo + that
+// sum in binary64, so the block's sum errs by at most about 2^-42 of itself,
+// far below the fp32 rounding of the scale.  All of it stays on the fp32
+// pipe: no float-to-double conversion per element.
 // ---------------------------------------------------------------------------
-template <int DT, int ALGO, bool SKIP>
+constexpr float kSquareLo = 0x1p-50f;   // |x| range whose square splits exactly
+constexpr float kSquareHi = 0x1p56f;
+
+struct SquareSum {
+    float hi = 0.0f, lo = 0.0f;
+    double wide = 0.0;   // squares of out-of-range values
+
+    __device__ __forceinline__ void add(float x)
+    {
+        const float ax = fabsf(x);
+        if (ax >= kSquareLo && ax <= kSquareHi) {
+            const float sq = __fmul_rn(x, x);
+            const float err = __fmaf_rn(x, x, -sq);
+            const float s = __fadd_rn(hi, sq);
+            const float bp = __fsub_rn(s, hi);
+            const float e = __fadd_rn(__fsub_rn(hi, __fsub_rn(s, bp)), __fsub_rn(sq, bp));
+            hi = s;
+            lo = __fadd_rn(lo, __fadd_rn(e, err));
+        } else if (x != 0.0f) {
+            const double xd = static_cast<double>(x);
+            wide = __fma_rn(xd, xd, wide);
+        }
+    }
+
+    __device__ __forceinline__ double total() const
+    {
+        return __dadd_rn(__dadd_rn(static_cast<double>(hi), static_cast<double>(lo)), wide);
+    }
+};
+
+template <int DT, int ALGO, bool SKIP, int MODE>
 __device__ __forceinline__ void norm_block(const ChunkRec& c, const StepScalars& s, int lane,
-                                           double& su, double& sp)
+                                           float wd, double& sd, double& sp)
 {
     using P = Param<DT>;
     constexpr int K = 8;
     const uint32_t len = c.len;
+    SquareSum ad, ap;
     for (uint32_t base = 0; base < len; base += 32 * K) {
         float g[K], p[K], m[K], v[K], m2[K];
 #pragma unroll
@@ -675,20 +741,19 @@ __device__ __forceinline__ void norm_block(const ChunkRec& c, const StepScalars&
                 if (ALGO == kAdEMAMix) m2[k] = ld_global(c.m2 + i);
             }
         }
-        // x*x of a binary32 x is exact in binary64, so one fused multiply-add
-        // gives the same sum as a multiply and an add, with one operation less
 #pragma unroll
         for (int k = 0; k < K; ++k) {
             if (base + lane + 32 * k < len) {
-                const double pd = static_cast<double>(p[k]);
-                sp = __fma_rn(pd, pd, sp);
+                ap.add(p[k]);
                 if (!(SKIP && g[k] == 0.0f)) {
-                    const double ud = static_cast<double>(direction<ALGO>(g[k], m[k], v[k], m2[k], s));
-                    su = __fma_rn(ud, ud, su);
+                    const float u = direction<ALGO>(g[k], m[k], v[k], m2[k], s);
+                    ad.add(MODE == kLamb ? lamb_direction(u, p[k], wd) : u);
                 }
             }
         }
     }
+    sd = ad.total();
+    sp = ap.total();
 }
 
 __device__ __forceinline__ void warp_tree_sum(double& a, double& b)
@@ -700,9 +765,9 @@ __device__ __forceinline__ void warp_tree_sum(double& a, double& b)
     }
 }
 
-template <int ALGO, bool SKIP>
+template <int ALGO, bool SKIP, int MODE>
 __global__ void unorm_partials_kernel(const ChunkRec* __restrict__ blocks, int nblocks,
-                                      StepScalars s, double2* __restrict__ partial)
+                                      StepScalars s, float wd, double2* __restrict__ partial)
 {
     const int lane = threadIdx.x & 31;
     const int warps_per_block = blockDim.x >> 5;
@@ -710,14 +775,14 @@ __global__ void unorm_partials_kernel(const ChunkRec* __restrict__ blocks, int n
     const int nwarps = gridDim.x * warps_per_block;
     for (int b = warp; b < nblocks; b += nwarps) {
         const ChunkRec rec = blocks[b];
-        double su = 0.0, sp = 0.0;
+        double sd = 0.0, sp = 0.0;
         switch (rec.dtype & ~kShortFlag) {
-        case kF32: norm_block<kF32, ALGO, SKIP>(rec, s, lane, su, sp); break;
-        case kF16: norm_block<kF16, ALGO, SKIP>(rec, s, lane, su, sp); break;
-        default: norm_block<kBF16, ALGO, SKIP>(rec, s, lane, su, sp); break;
+        case kF32: norm_block<kF32, ALGO, SKIP, MODE>(rec, s, lane, wd, sd, sp); break;
+        case kF16: norm_block<kF16, ALGO, SKIP, MODE>(rec, s, lane, wd, sd, sp); break;
+        default: norm_block<kBF16, ALGO, SKIP, MODE>(rec, s, lane, wd, sd, sp); break;
         }
-        warp_tree_sum(su, sp);
-        if (lane == 0) partial[b] = make_double2(su, sp);
+        warp_tree_sum(sd, sp);
+        if (lane == 0) partial[b] = make_double2(sd, sp);
     }
 }
 
@@ -734,14 +799,14 @@ __global__ void unorm_group_kernel(const double2* __restrict__ partial,
     const int nwarps = gridDim.x * warps_per_block;
     for (int q = blockIdx.x * warps_per_block + (threadIdx.x >> 5); q < ngroups; q += nwarps) {
         const uint2 r = range[q];
-        double su = 0.0, sp = 0.0;
+        double sd = 0.0, sp = 0.0;
         for (uint32_t b = r.x + lane; b < r.y; b += 32) {
             const double2 x = partial[b];
-            su = __dadd_rn(su, x.x);
+            sd = __dadd_rn(sd, x.x);
             sp = __dadd_rn(sp, x.y);
         }
-        warp_tree_sum(su, sp);
-        if (lane == 0) group_sum[q] = make_double2(su, sp);
+        warp_tree_sum(sd, sp);
+        if (lane == 0) group_sum[q] = make_double2(sd, sp);
     }
 }
 
@@ -752,16 +817,17 @@ __global__ void unorm_group_kernel(const double2* __restrict__ partial,
 // warps.  The order depends only on the tensor, not on the grid.
 constexpr int kScaleThreads = 1024;
 
+template <int MODE>
 __global__ void __launch_bounds__(kScaleThreads)
 unorm_scale_kernel(const double2* __restrict__ sums, const uint32_t* __restrict__ first,
                    int ntensors, float max_unorm, float* __restrict__ scale)
 {
     constexpr int kWarps = kScaleThreads / 32;
-    __shared__ double su_w[kWarps], sp_w[kWarps];
+    __shared__ double sd_w[kWarps], sp_w[kWarps];
     const int lane = threadIdx.x & 31;
     const int w = threadIdx.x >> 5;
     for (int t = blockIdx.x; t < ntensors; t += gridDim.x) {   // the same t for the whole CTA
-        double au[4] = {0.0, 0.0, 0.0, 0.0}, ap[4] = {0.0, 0.0, 0.0, 0.0};
+        double ad[4] = {0.0, 0.0, 0.0, 0.0}, ap[4] = {0.0, 0.0, 0.0, 0.0};
         const uint32_t end = first[t + 1];
         for (uint32_t b = first[t] + threadIdx.x; b < end; b += 4 * kScaleThreads) {
 #pragma unroll
@@ -769,34 +835,38 @@ unorm_scale_kernel(const double2* __restrict__ sums, const uint32_t* __restrict_
                 const uint32_t i = b + k * kScaleThreads;
                 if (i < end) {
                     const double2 x = sums[i];
-                    au[k] = __dadd_rn(au[k], x.x);
+                    ad[k] = __dadd_rn(ad[k], x.x);
                     ap[k] = __dadd_rn(ap[k], x.y);
                 }
             }
         }
-        double su = __dadd_rn(__dadd_rn(au[0], au[1]), __dadd_rn(au[2], au[3]));
+        double sd = __dadd_rn(__dadd_rn(ad[0], ad[1]), __dadd_rn(ad[2], ad[3]));
         double sp = __dadd_rn(__dadd_rn(ap[0], ap[1]), __dadd_rn(ap[2], ap[3]));
-        warp_tree_sum(su, sp);
-        if (lane == 0) { su_w[w] = su; sp_w[w] = sp; }
+        warp_tree_sum(sd, sp);
+        if (lane == 0) { sd_w[w] = sd; sp_w[w] = sp; }
         __syncthreads();
         if (w == 0) {
-            su = lane < kWarps ? su_w[lane] : 0.0;
+            sd = lane < kWarps ? sd_w[lane] : 0.0;
             sp = lane < kWarps ? sp_w[lane] : 0.0;
-            warp_tree_sum(su, sp);
+            warp_tree_sum(sd, sp);
             if (lane == 0) {
-                const double U = __dsqrt_rn(su), P = __dsqrt_rn(sp);
-                const double limit = __dmul_rn(static_cast<double>(max_unorm), P);
-                scale[t] = U > limit ? __double2float_rn(__ddiv_rn(limit, U)) : 1.0f;
+                const double D = __dsqrt_rn(sd), P = __dsqrt_rn(sp);
+                if (MODE == kLamb) {
+                    scale[t] = (P > 0.0 && D > 0.0) ? __double2float_rn(__ddiv_rn(P, D)) : 1.0f;
+                } else {
+                    const double limit = __dmul_rn(static_cast<double>(max_unorm), P);
+                    scale[t] = D > limit ? __double2float_rn(__ddiv_rn(limit, D)) : 1.0f;
+                }
             }
         }
         __syncthreads();   // the shared sums are reused by the next tensor
     }
 }
 
-template <int ALGO, bool SKIP>
+template <int ALGO, bool SKIP, int MODE>
 __global__ void step_kernel_scaled(const ChunkRec* __restrict__ chunks, int nchunks,
                                    StepScalars s, const uint32_t* __restrict__ chunk_tensor,
-                                   const float* __restrict__ scale)
+                                   const float* __restrict__ scale, float wd)
 {
     const int lane = threadIdx.x & 31;
     const int warps_per_block = blockDim.x >> 5;
@@ -806,9 +876,9 @@ __global__ void step_kernel_scaled(const ChunkRec* __restrict__ chunks, int nchu
         const ChunkRec rec = chunks[c];
         const float sc = scale[chunk_tensor[c]];
         switch (rec.dtype & ~kShortFlag) {
-        case kF32: run_chunk<kF32, ALGO, SKIP, true>(rec, s, lane, sc); break;
-        case kF16: run_chunk<kF16, ALGO, SKIP, true>(rec, s, lane, sc); break;
-        default: run_chunk<kBF16, ALGO, SKIP, true>(rec, s, lane, sc); break;
+        case kF32: run_chunk<kF32, ALGO, SKIP, MODE>(rec, s, lane, sc, wd); break;
+        case kF16: run_chunk<kF16, ALGO, SKIP, MODE>(rec, s, lane, sc, wd); break;
+        default: run_chunk<kBF16, ALGO, SKIP, MODE>(rec, s, lane, sc, wd); break;
         }
     }
 }
@@ -1083,19 +1153,19 @@ cudaError_t unorm_grid(const void* fn, int64_t warps_needed, int block_threads, 
     return cudaSuccess;
 }
 
-template <int ALGO, bool SKIP>
+template <int ALGO, bool SKIP, int MODE>
 cudaError_t launch_unorm_typed(const ChunkRec* d_chunks, int64_t nchunks, const StepScalars& sc,
-                               const UnormArgs& u, float max_unorm, int block_threads,
+                               const UnormArgs& u, float max_unorm, float wd, int block_threads,
                                int max_blocks, cudaStream_t stream)
 {
     constexpr int kNormThreads = 256;
     int grid = 0;
     cudaError_t e = cudaSuccess;
     if (u.nblocks > 0) {
-        const void* k1 = reinterpret_cast<const void*>(unorm_partials_kernel<ALGO, SKIP>);
+        const void* k1 = reinterpret_cast<const void*>(unorm_partials_kernel<ALGO, SKIP, MODE>);
         if ((e = unorm_grid(k1, u.nblocks, kNormThreads, &grid)) != cudaSuccess) return e;
-        unorm_partials_kernel<ALGO, SKIP><<<grid, kNormThreads, 0, stream>>>(
-            u.blocks, static_cast<int>(u.nblocks), sc, reinterpret_cast<double2*>(u.partial));
+        unorm_partials_kernel<ALGO, SKIP, MODE><<<grid, kNormThreads, 0, stream>>>(
+            u.blocks, static_cast<int>(u.nblocks), sc, wd, reinterpret_cast<double2*>(u.partial));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (u.ngroups > 0) {
@@ -1107,26 +1177,26 @@ cudaError_t launch_unorm_typed(const ChunkRec* d_chunks, int64_t nchunks, const 
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (u.ntensors > 0) {
-        const void* k2 = reinterpret_cast<const void*>(unorm_scale_kernel);
+        const void* k2 = reinterpret_cast<const void*>(unorm_scale_kernel<MODE>);
         // one CTA per tensor, up to the resident CTAs of the device
         if ((e = unorm_grid(k2, static_cast<int64_t>(u.ntensors) * (kScaleThreads / 32), kScaleThreads,
                             &grid)) != cudaSuccess)
             return e;
-        unorm_scale_kernel<<<grid, kScaleThreads, 0, stream>>>(
+        unorm_scale_kernel<MODE><<<grid, kScaleThreads, 0, stream>>>(
             reinterpret_cast<const double2*>(u.group_sum), u.first_group, u.ntensors, max_unorm,
             u.scale);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (nchunks > 0) {
-        const void* k3 = reinterpret_cast<const void*>(step_kernel_scaled<ALGO, SKIP>);
+        const void* k3 = reinterpret_cast<const void*>(step_kernel_scaled<ALGO, SKIP, MODE>);
         if (max_blocks > 0) {
             const int64_t need = (nchunks + block_threads / 32 - 1) / (block_threads / 32);
             grid = static_cast<int>(need < max_blocks ? need : max_blocks);
         } else if ((e = unorm_grid(k3, nchunks, block_threads, &grid)) != cudaSuccess) {
             return e;
         }
-        step_kernel_scaled<ALGO, SKIP><<<grid, block_threads, 0, stream>>>(
-            d_chunks, static_cast<int>(nchunks), sc, u.chunk_tensor, u.scale);
+        step_kernel_scaled<ALGO, SKIP, MODE><<<grid, block_threads, 0, stream>>>(
+            d_chunks, static_cast<int>(nchunks), sc, u.chunk_tensor, u.scale, wd);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -1142,24 +1212,39 @@ cudaError_t launch_step_max_unorm(const ChunkRec* d_chunks, int64_t nchunks, int
     StepScalars sc = s;
     fill_reciprocals(&sc);
     if (algo == kAdEMAMix)
-        return skip_zeros ? launch_unorm_typed<kAdEMAMix, true>(d_chunks, nchunks, sc, u, max_unorm,
-                                                                block_threads, max_blocks, stream)
-                          : launch_unorm_typed<kAdEMAMix, false>(d_chunks, nchunks, sc, u, max_unorm,
-                                                                 block_threads, max_blocks, stream);
-    return skip_zeros ? launch_unorm_typed<kAdam, true>(d_chunks, nchunks, sc, u, max_unorm,
-                                                        block_threads, max_blocks, stream)
-                      : launch_unorm_typed<kAdam, false>(d_chunks, nchunks, sc, u, max_unorm,
-                                                         block_threads, max_blocks, stream);
+        return skip_zeros ? launch_unorm_typed<kAdEMAMix, true, kScaled>(
+                                d_chunks, nchunks, sc, u, max_unorm, 0.0f, block_threads, max_blocks, stream)
+                          : launch_unorm_typed<kAdEMAMix, false, kScaled>(
+                                d_chunks, nchunks, sc, u, max_unorm, 0.0f, block_threads, max_blocks, stream);
+    return skip_zeros ? launch_unorm_typed<kAdam, true, kScaled>(
+                            d_chunks, nchunks, sc, u, max_unorm, 0.0f, block_threads, max_blocks, stream)
+                      : launch_unorm_typed<kAdam, false, kScaled>(
+                            d_chunks, nchunks, sc, u, max_unorm, 0.0f, block_threads, max_blocks, stream);
 }
 
-cudaError_t max_block_threads_scaled(int algo, int skip_zeros, int* out)
+cudaError_t launch_step_lamb(const ChunkRec* d_chunks, int64_t nchunks, int skip_zeros,
+                             const StepScalars& s, float weight_decay, const UnormArgs& u,
+                             int block_threads, int max_blocks, cudaStream_t stream)
+{
+    StepScalars sc = s;
+    fill_reciprocals(&sc);
+    return skip_zeros ? launch_unorm_typed<kAdam, true, kLamb>(d_chunks, nchunks, sc, u, 0.0f, weight_decay,
+                                                               block_threads, max_blocks, stream)
+                      : launch_unorm_typed<kAdam, false, kLamb>(d_chunks, nchunks, sc, u, 0.0f, weight_decay,
+                                                                block_threads, max_blocks, stream);
+}
+
+cudaError_t max_block_threads_scaled(int algo, int skip_zeros, int lamb, int* out)
 {
     cudaFuncAttributes attr{};
-    const void* fn = algo == kAdEMAMix
-        ? (skip_zeros ? reinterpret_cast<const void*>(step_kernel_scaled<kAdEMAMix, true>)
-                      : reinterpret_cast<const void*>(step_kernel_scaled<kAdEMAMix, false>))
-        : (skip_zeros ? reinterpret_cast<const void*>(step_kernel_scaled<kAdam, true>)
-                      : reinterpret_cast<const void*>(step_kernel_scaled<kAdam, false>));
+    const void* fn =
+        lamb ? (skip_zeros ? reinterpret_cast<const void*>(step_kernel_scaled<kAdam, true, kLamb>)
+                           : reinterpret_cast<const void*>(step_kernel_scaled<kAdam, false, kLamb>))
+        : algo == kAdEMAMix
+            ? (skip_zeros ? reinterpret_cast<const void*>(step_kernel_scaled<kAdEMAMix, true, kScaled>)
+                          : reinterpret_cast<const void*>(step_kernel_scaled<kAdEMAMix, false, kScaled>))
+            : (skip_zeros ? reinterpret_cast<const void*>(step_kernel_scaled<kAdam, true, kScaled>)
+                          : reinterpret_cast<const void*>(step_kernel_scaled<kAdam, false, kScaled>));
     cudaError_t e = cudaFuncGetAttributes(&attr, fn);
     if (e != cudaSuccess) return e;
     *out = attr.maxThreadsPerBlock / 32 * 32;

@@ -23,6 +23,12 @@ stepped through one record per parameter, and AdEMAMix keeps each
 parameter's [m1 | m2] together in the flat state.  It is not combined with
 capturable=True.
 
+lamb=True makes the step LAMB's (opt2s_step_lamb; You et al. 2020,
+Algorithm 2; Adam moments only): per parameter, the Adam direction plus
+weight_decay * param, scaled by the trust ratio ||param|| / ||direction||.
+Like max_unorm it takes four launches per group and step, keeps one record
+per parameter under flatten=True, and is not combined with capturable=True.
+
 capturable=True routes every step through opt2s_plan_step_table: the per-step
 scalars live in a device table and the step index in device memory, so
 ``step()`` may be captured in a CUDA graph and each replay performs the next
@@ -42,19 +48,23 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                  betas=(0.9, 0.999), eps: float = 1e-8, weight_decay: float = 0.0,
                  beta3: float = 0.9999, alpha: float = 5.0, skip_zeros: bool = False,
                  capturable: bool = False, table_len: int = 1024, flatten: bool = False,
-                 max_unorm: float = 0.0):
+                 max_unorm: float = 0.0, lamb: bool = False):
         if algo not in B.ALGOS:
             raise ValueError(f"algo must be one of {sorted(B.ALGOS)}")
         if not (0.0 <= max_unorm < float("inf")):
             raise ValueError("max_unorm must be finite and >= 0 (0 disables the bound)")
         if max_unorm > 0.0 and capturable:
             raise ValueError("max_unorm and capturable are not combined")
+        if lamb and (capturable or max_unorm > 0.0 or algo == "ademamix"):
+            raise ValueError("lamb takes Adam moments and is not combined with capturable "
+                             "or max_unorm")
         defaults = dict(lr=lr, betas=tuple(betas), eps=eps, weight_decay=weight_decay,
                         beta3=beta3, alpha=alpha, skip_zeros=skip_zeros)
         self.algo = "ademamix" if algo == "ademamix" else "adam"
         self.capturable = capturable
         self.table_len = int(table_len)
         self.max_unorm = float(max_unorm)
+        self.lamb = bool(lamb)
         super().__init__(params, defaults)
         self._group_cache = {}
         self._flat = None
@@ -80,9 +90,9 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                 fs1 = torch.zeros(2 * n if two else n, dtype=torch.float32, device=dev)
                 fs2 = torch.zeros(n, dtype=torch.float32, device=dev)
                 # per_param: one record per parameter (needed by the per-
-                # parameter norms of max_unorm); AdEMAMix then keeps each
-                # parameter's [m1 | m2] together, else all m1 before all m2
-                per_param = self.max_unorm > 0.0
+                # parameter norms of max_unorm and LAMB); AdEMAMix then keeps
+                # each parameter's [m1 | m2] together, else all m1 before all m2
+                per_param = self.max_unorm > 0.0 or self.lamb
                 off = 0
                 views = ([], [], [], [])
                 with torch.no_grad():
@@ -181,7 +191,9 @@ class TwoStateOptimizer(torch.optim.Optimizer):
         if self._flat is not None:
             for f in self._flat:
                 hyper = self._hyper(self.param_groups[f["group"]])
-                if "records" in f:
+                if "records" in f and self.lamb:
+                    B.opt2s_step_lamb(f["records"], hyper, f["step"] + 1)
+                elif "records" in f:
                     B.opt2s_step_max_unorm(f["records"], hyper, self.max_unorm, f["step"] + 1)
                 else:
                     f["plan"].step(hyper, f["step"] + 1)
@@ -194,6 +206,8 @@ class TwoStateOptimizer(torch.optim.Optimizer):
             if self.capturable:
                 data["plan"].step_table(group["skip_zeros"], data["table"].data_ptr(),
                                         self.table_len, data["index"].data_ptr())
+            elif self.lamb:
+                B.opt2s_step_lamb(data["tl"], self._hyper(group), data["step"] + 1)
             elif self.max_unorm > 0.0:
                 B.opt2s_step_max_unorm(data["tl"], self._hyper(group), self.max_unorm,
                                        data["step"] + 1)
@@ -244,3 +258,11 @@ class AdEMAMix32bit(TwoStateOptimizer):
         b1, b2, b3 = betas
         super().__init__(params, "ademamix", lr, (b1, b2), eps, weight_decay, beta3=b3,
                          alpha=alpha, **kw)
+
+
+class LAMB32bit(TwoStateOptimizer):
+    """LAMB (You et al. 2020, Algorithm 2) with fp32 state: the weight decay
+    sits inside the trust-ratio scaled update."""
+
+    def __init__(self, params, lr=1e-3, betas=(0.9, 0.999), eps=1e-6, weight_decay=1e-2, **kw):
+        super().__init__(params, "adam", lr, betas, eps, weight_decay, lamb=True, **kw)

@@ -285,6 +285,34 @@ int64_t opt2s_noalloc_max_chunks(void);
 int opt2s_step_max_unorm(const TensorListDesc *desc, const Hyper *hyper, float max_unorm,
                          int step, cudaStream_t stream);
 
+/*
+ * LAMB: the layer-wise adaptive step of You et al., "Large Batch Optimization
+ * for Deep Learning: Training BERT in 76 minutes", ICLR 2020, Algorithm 2,
+ * with each tensor of the collection as a layer.  The issue's section "Scope"
+ * keeps the two-state kernel for "max-unorm/LAMB use" without writing LAMB
+ * out; this library follows Algorithm 2 with the scaling function phi the
+ * identity:
+ *
+ *     u_i = num_i/den_i, the Adam direction of element i in the step above
+ *     w_i = u_i + weight_decay*p_i                  (fp32; 0 for an element
+ *                                                    skip_zeros leaves alone)
+ *     W   = sqrt(sum_i w_i^2),  P = sqrt(sum_i p_i^2), p before the step,
+ *           per tensor, in binary64
+ *     r   = P/W if P > 0 and W > 0, else 1 (binary64, rounded to fp32 once)
+ *     p_i = p_i - lr*(r*w_i), with m and v as in the step above.
+ *
+ * The weight decay is inside the trust-ratio scaled update (Algorithm 2),
+ * not applied first as in opt2s_step; bc1, bc2 as in opt2s_step.
+ * hyper->algo must be OPT2S_ADAM (else OPT2S_ERR_INVALID_ARG).  Sums have
+ * the fixed order of opt2s_step_max_unorm, so r does not depend on launch
+ * geometry or alignment.  Four launches on `stream`; the plans, tables and
+ * workspace are those of opt2s_step_max_unorm (shared cache entries), with
+ * the same rule that two steps of the same collection must not overlap on
+ * the GPU.  Other arguments and validation as opt2s_step.
+ */
+int opt2s_step_lamb(const TensorListDesc *desc, const Hyper *hyper, int step,
+                    cudaStream_t stream);
+
 /* Frees every cached plan of every device (waits for the devices first). */
 int opt2s_release_cache(void);
 

@@ -311,6 +311,34 @@ def test_max_unorm_step_without_device(L):
     assert e.value.status == -2
 
 
+def test_lamb_argument_checks(L):
+    """LAMB takes Adam moments: AdEMAMix is rejected, as are a bad step and
+    bad hyper-parameters, before any CUDA call."""
+    tl = B.TensorList(records([64]))
+    with pytest.raises(B.Opt2sError) as e:
+        B.opt2s_step_lamb(tl, B.make_hyper("ademamix", beta3=0.9, alpha=1.0), 1, stream=0)
+    assert e.value.status == -1
+    with pytest.raises(B.Opt2sError) as e:
+        B.opt2s_step_lamb(tl, H, 0, stream=0)
+    assert e.value.status == -1
+    with pytest.raises(B.Opt2sError) as e:
+        B.opt2s_step_lamb(tl, B.make_hyper("adam", eps=-1.0), 1, stream=0)
+    assert e.value.status == -1
+    B.opt2s_step_lamb(B.TensorList([]), H, 1, stream=0)   # empty: no-op
+
+
+@pytest.mark.skipif(_cuda_available(), reason="checks the no-device path")
+def test_lamb_step_without_device(L):
+    tl = B.TensorList(records([64, 3000], ["f32", "bf16"]))
+    with pytest.raises(B.Opt2sError) as e:
+        B.opt2s_step_lamb(tl, H, 1, stream=0)
+    assert e.value.status == -4                       # CUDA: no device
+    p, g, s1, s2, n, dt = records([64])[0]
+    with pytest.raises(B.Opt2sError) as e:            # argument errors still first
+        B.opt2s_step_lamb(B.TensorList([(p, g, s1, s1, n, dt)]), H, 1, stream=0)
+    assert e.value.status == -2
+
+
 def test_missing_library_fails_loudly(tmp_path):
     code = ("import elementwise_optimizer_b200.binding as b; b.LIB_PATH='/nonexistent/x.so'\n"
             "try:\n  b.lib()\nexcept RuntimeError as e:\n  print('RAISED', e)\n")
