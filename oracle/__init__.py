@@ -81,6 +81,13 @@ def _load():
     lib.oracle_step_f32_lamb.argtypes = [i32, i32, f32, f32, f32, f32, f32, i32,
                                          vp, vp, vp, vp, i64, vp]
     lib.oracle_step_f32_lamb.restype = i32
+    lib.oracle_quant_map.argtypes = [i32, vp]
+    lib.oracle_quant_map.restype = i32
+    lib.oracle_quantize.argtypes = [vp, f32]
+    lib.oracle_quantize.restype = i32
+    lib.oracle_step_8bit.argtypes = [i32, i32, i32, f32, f32, f32, f32, f32, f32, f32, i32,
+                                     vp, vp, vp, vp, vp, vp, i64]
+    lib.oracle_step_8bit.restype = i32
     lib.oracle_average_grads.argtypes = [i32, i32, vp, vp, i64]
     lib.oracle_average_grads.restype = i32
     lib.oracle_bias_correction.argtypes = [f32, i32]
@@ -178,6 +185,53 @@ def step_f32_lamb(param: np.ndarray, grad: np.ndarray, m: np.ndarray,
     if rc != 0:
         raise ValueError(f"oracle_step_f32_lamb rejected its arguments ({rc})")
     return float(ratio[0])
+
+
+BLOCK8 = 2048
+
+
+def quant_map(signed: bool) -> np.ndarray:
+    """The 256 values of the 8-bit state codes, ascending (signed: dynamic
+    tree quantization for first moments; unsigned: for the second moment)."""
+    out = np.empty(256, np.float32)
+    if _load().oracle_quant_map(int(bool(signed)), _ptr(out)) != 0:
+        raise ValueError("oracle_quant_map failed")
+    return out
+
+
+def quantize(qmap: np.ndarray, x) -> np.ndarray:
+    """Codes of the map values nearest to x (ties to the lower code)."""
+    qmap = np.ascontiguousarray(qmap, np.float32)
+    xs = np.atleast_1d(np.asarray(x, np.float32))
+    f = _load().oracle_quantize
+    return np.array([f(_ptr(qmap), float(v)) for v in xs], np.uint8)
+
+
+def step_8bit(param: np.ndarray, grad: np.ndarray, q1: np.ndarray, q2: np.ndarray,
+              absmax1: np.ndarray, absmax2: np.ndarray, *, dtype: str, algo: str,
+              step: int, lr: float, beta1: float, beta2: float, eps: float,
+              beta3: float = 0.0, alpha: float = 0.0, weight_decay: float = 0.0,
+              skip_zeros: bool = False) -> None:
+    """One step over one tensor with 8-bit blockwise state, in place.
+    q1: uint8 codes of m (n) or [m1 | m2] (2n); absmax1: float32 per block
+    (nb) or [m1 | m2] (2 nb); q2: codes of v (n); absmax2: per block (nb)."""
+    n = param.size
+    nb = (n + BLOCK8 - 1) // BLOCK8
+    two = algo == "ademamix"
+    if grad.size != n or param.itemsize != _ITEMSIZE[dtype] or grad.itemsize != _ITEMSIZE[dtype]:
+        raise ValueError("param/grad size or item size mismatch")
+    if q1.dtype != np.uint8 or q2.dtype != np.uint8 or q1.size != (2 * n if two else n) or \
+            q2.size != n:
+        raise ValueError("codes must be uint8 of the right length")
+    if absmax1.dtype != np.float32 or absmax2.dtype != np.float32 or \
+            absmax1.size != (2 * nb if two else nb) or absmax2.size != nb:
+        raise ValueError("absmax arrays must be float32 of the right length")
+    rc = _load().oracle_step_8bit(
+        ALGO[algo], DTYPE[dtype], int(bool(skip_zeros)), lr, beta1, beta2, beta3, alpha, eps,
+        weight_decay, int(step), _ptr(param), _ptr(grad), _ptr(q1), _ptr(q2), _ptr(absmax1),
+        _ptr(absmax2), n)
+    if rc != 0:
+        raise ValueError(f"oracle_step_8bit rejected its arguments ({rc})")
 
 
 def step_f32_fgrad(param: np.ndarray, grad: np.ndarray, state1: np.ndarray,

@@ -35,6 +35,12 @@
  *   [LAMB]     You et al., "Large Batch Optimization for Deep Learning:
  *              Training BERT in 76 minutes", ICLR 2020, Algorithm 2 (per-layer
  *              trust ratio ||x|| / ||r + lambda x||).
+ *   [8bit]     Dettmers, Lewis, Shleifer & Zettlemoyer, "8-bit Optimizers via
+ *              Block-wise Quantization", ICLR 2022, sections 2.1 (block-wise
+ *              absmax quantization, B = 2048), 2.2 (dynamic tree
+ *              quantization) and 2.3 (dynamic quantization of the unsigned
+ *              second state).  [issue] "Problem": tensors below
+ *              min_8bit_size = 4096 elements keep the 32-bit state.
  *   [IEEE754]  IEEE 754-2008, section 4.3.1 (roundTiesToEven) and 3.6
  *              (binary16 format); bfloat16 is the upper half of binary32.
  *
@@ -55,9 +61,12 @@
  *     function; the pages name the option without its arithmetic.
  *   - LAMB (oracle_step_f32_lamb): You et al. 2020, Algorithm 2, per tensor,
  *     with the readings written out above that function.
+ *   - 8-bit blockwise state (oracle_step_8bit): [8bit], with the map and
+ *     quantization readings written out above oracle_quant_map.
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 #include <xmmintrin.h>
 
@@ -495,6 +504,169 @@ int oracle_step_f32_lamb(int dtype, int skip_zeros, float lr, float beta1,
         store_param(param, dtype, i, p);
         m[i] = mi;
         v[i] = vi;
+    }
+
+    _mm_setcsr(csr);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* 8-bit blockwise state [8bit].                                              */
+/* ------------------------------------------------------------------------ */
+
+#define OR_BLOCK8 2048                                  /* [8bit] 2.1: block size B */
+
+/*
+ * The quantization maps of [8bit]: the 256 values a state code stands for,
+ * in ascending order, so that code c means the c-th smallest value.
+ *
+ * [8bit] 2.2 (dynamic tree quantization, for the signed first moments): a
+ * code is a sign bit, then E zero bits (the value's decimal exponent,
+ * 10^-E), then an indicator bit 1, then F = 6 - E bits f of a linear fraction
+ * in [0.1, 1].  [8bit] 2.3 (dynamic quantization, for the non-negative
+ * second moment): the sign bit becomes one more fraction bit, F = 7 - E.
+ * E runs over 0..6 in both (the 7 decades down to 10^-7 the paper gives).
+ * Readings where the paper leaves the detail open:
+ *   - the F fraction bits split [0.1, 1] into 2^F equal bins and f stands
+ *     for the midpoint of bin f: value = 10^-E * (0.1 + 0.9*(2f+1)/2^(F+1)),
+ *     which is N/D with N = 2^(F+1) + 9*(2f+1) and D = 10^(E+1) * 2^(F+1),
+ *     both exact binary32 integers, so one IEEE division rounds it once;
+ *   - the bits with no indicator (all zeros after the sign, or all zeros in
+ *     the unsigned code's first seven bits) give two patterns: one is 0, the
+ *     other stands for 1.0, so that the element a block is normalised by
+ *     (x = 1 after the division by the block's absmax) is stored exactly.
+ * Returns 0.
+ */
+static int cmp_float_asc(const void *a, const void *b)
+{
+    float x = *(const float *)a, y = *(const float *)b;
+    return (x > y) - (x < y);
+}
+
+int oracle_quant_map(int is_signed, float *map)
+{
+    int k = 0;
+    const int f0 = is_signed ? 6 : 7;                   /* fraction bits at E = 0 */
+    for (int E = 0; E <= 6; E++) {
+        const int F = f0 - E;
+        float D = (float)(1 << (F + 1));
+        for (int e = 0; e <= E; e++) D *= 10.0f;       /* exact: 10^(E+1) 2^(F+1) < 2^31 */
+        for (int f = 0; f < (1 << F); f++) {
+            const float N = (float)((1 << (F + 1)) + 9 * (2 * f + 1));
+            const float value = N / D;
+            map[k++] = value;
+            if (is_signed) map[k++] = -value;
+        }
+    }
+    map[k++] = 0.0f;
+    map[k++] = 1.0f;
+    qsort(map, (size_t)k, sizeof(float), cmp_float_asc);
+    return k == 256 ? 0 : -1;
+}
+
+/* [8bit] 2.1: the code of the map value nearest to x; the distances are
+ * compared exactly (x and the map are binary32, whose differences binary64
+ * holds exactly wherever two candidates are close), and an exact tie goes to
+ * the lower code.  A NaN x gets code 0. */
+int oracle_quantize(const float *map, float x)
+{
+    int best = 0;
+    double bd = fabs((double)x - (double)map[0]);
+    for (int j = 1; j < 256; j++) {
+        double d = fabs((double)x - (double)map[j]);
+        if (d < bd) { bd = d; best = j; }
+    }
+    return best;
+}
+
+static int zero_code(const float *map)
+{
+    for (int j = 0; j < 256; j++)
+        if (map[j] == 0.0f) return j;
+    return 0;
+}
+
+/* One block of one state quantity: values x[0..len) (fp32) -> codes and the
+ * block's absmax.  [8bit] 2.1: N = max |x_i|, code_i = nearest(x_i / N) with
+ * the division rounded to fp32; a block whose absmax is 0 stores the code of
+ * 0 everywhere.  NaNs do not raise the absmax. */
+static void quantize_block(const float *map, const float *x, int64_t len, uint8_t *codes,
+                           float *absmax)
+{
+    float amax = 0.0f;
+    for (int64_t i = 0; i < len; i++) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    const int zc = zero_code(map);
+    for (int64_t i = 0; i < len; i++)
+        codes[i] = (uint8_t)(amax > 0.0f ? oracle_quantize(map, x[i] / amax) : zc);
+    *absmax = amax;
+}
+
+/*
+ * One optimizer step over one tensor whose state is stored in 8 bits, block
+ * by block ([8bit] section 2: dequantize the state of a block to fp32,
+ * update, quantize the new state back with the block's new absmax).
+ *
+ * q1        Adam: codes of m (n bytes).  AdEMAMix: [m1 codes | m2 codes] (2n).
+ * absmax1   Adam: absmax of m per block (ceil(n/2048) floats).  AdEMAMix:
+ *           [m1 absmaxes | m2 absmaxes] (2*ceil(n/2048)).
+ * q2        codes of v (n bytes); absmax2: absmax of v per block.
+ * m and m2 use the signed map, v the unsigned one.  A block is elements
+ * [2048k, 2048(k+1)) of the tensor.  State starting at zero: every absmax 0
+ * (codes then do not matter).
+ *
+ * Per element: m = map_s[q1]*absmax (fp32 product), likewise v and m2; the
+ * update is the plain fp32 step's (the same order, decay first), on these
+ * values; p is stored as in the plain step.  With skip_zeros, an element
+ * whose gradient is zero keeps p and its dequantized m, v (m2), which are
+ * then quantized with the block's new absmax like the others.
+ * Returns 0, or -1 on an argument the definitions do not cover.
+ */
+int oracle_step_8bit(int algo, int dtype, int skip_zeros, float lr, float beta1,
+                     float beta2, float beta3, float alpha, float eps, float weight_decay,
+                     int step, void *param, const void *grad, uint8_t *q1, uint8_t *q2,
+                     float *absmax1, float *absmax2, int64_t n)
+{
+    if (step < 1 || n < 0) return -1;
+    if (algo != OR_ADAM && algo != OR_ADEMAMIX) return -1;
+    if (dtype != OR_F32 && dtype != OR_F16 && dtype != OR_BF16) return -1;
+
+    unsigned int csr = _mm_getcsr();
+    _mm_setcsr(csr & ~(0x8000u | 0x0040u));             /* FTZ and DAZ off */
+
+    float smap[256], umap[256];
+    oracle_quant_map(1, smap);
+    oracle_quant_map(0, umap);
+    const float bc1 = oracle_bias_correction(beta1, step);
+    const float bc2 = oracle_bias_correction(beta2, step);
+    const float decay = oracle_decay_factor(lr, weight_decay);
+    const float one_minus_b1 = 1.0f - beta1;
+    const float one_minus_b2 = 1.0f - beta2;
+    const float one_minus_b3 = 1.0f - beta3;
+    const int64_t nblocks = (n + OR_BLOCK8 - 1) / OR_BLOCK8;
+
+    float m[OR_BLOCK8], v[OR_BLOCK8], m2[OR_BLOCK8];
+    for (int64_t b = 0; b < nblocks; b++) {
+        const int64_t lo = b * OR_BLOCK8;
+        const int64_t len = (n - lo < OR_BLOCK8) ? n - lo : OR_BLOCK8;
+        for (int64_t k = 0; k < len; k++) {
+            const int64_t i = lo + k;
+            m[k] = smap[q1[i]] * absmax1[b];
+            v[k] = umap[q2[i]] * absmax2[b];
+            m2[k] = algo == OR_ADEMAMIX ? smap[q1[n + i]] * absmax1[nblocks + b] : 0.0f;
+            float g = load_param(grad, dtype, i);
+            if (skip_zeros && g == 0.0f) continue;
+            float p = load_param(param, dtype, i);
+            update_element(algo, g, &p, &m[k], &m2[k], &v[k], lr, beta1, beta2, beta3, alpha,
+                           eps, bc1, bc2, decay, one_minus_b1, one_minus_b2, one_minus_b3);
+            store_param(param, dtype, i, p);
+        }
+        quantize_block(smap, m, len, q1 + lo, &absmax1[b]);
+        quantize_block(umap, v, len, q2 + lo, &absmax2[b]);
+        if (algo == OR_ADEMAMIX)
+            quantize_block(smap, m2, len, q1 + n + lo, &absmax1[nblocks + b]);
     }
 
     _mm_setcsr(csr);

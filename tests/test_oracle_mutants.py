@@ -68,6 +68,17 @@ MUTANTS = {
     "lamb_decay_outside_ratio": ("p = p - lr * (ratio * w);",
                                  "p = p - lr * (ratio * u) - lr * (weight_decay * p);"),
     "lamb_ratio_dropped": ("p = p - lr * (ratio * w);", "p = p - lr * w;"),
+    "map_bin_edges_not_midpoints": ("(1 << (F + 1)) + 9 * (2 * f + 1)", "(1 << (F + 1)) + 9 * (2 * f)"),
+    "map_spare_is_minus_one": ("map[k++] = 1.0f;", "map[k++] = -1.0f;"),
+    "map_decades_base_two": ("for (int e = 0; e <= E; e++) D *= 10.0f;",
+                             "for (int e = 0; e <= E; e++) D *= 2.0f;"),
+    "quantize_ties_upward": ("if (d < bd) { bd = d; best = j; }", "if (d <= bd) { bd = d; best = j; }"),
+    "quantize_without_division": ("oracle_quantize(map, x[i] / amax)", "oracle_quantize(map, x[i])"),
+    "absmax_kept_from_last_step": ("    *absmax = amax;\n", "    (void)amax;\n"),
+    "block_size_1024": ("#define OR_BLOCK8 2048", "#define OR_BLOCK8 1024"),
+    "dequant_without_absmax": ("m[k] = smap[q1[i]] * absmax1[b];", "m[k] = smap[q1[i]];"),
+    "v_on_signed_map": ("v[k] = umap[q2[i]] * absmax2[b];", "v[k] = smap[q2[i]] * absmax2[b];"),
+    "m2_with_m1_absmax": ("smap[q1[n + i]] * absmax1[nblocks + b]", "smap[q1[n + i]] * absmax1[b]"),
     "lamb_counts_skipped": (
         "sp += (double)p * (double)p;\n        float g = load_param(grad, dtype, i);\n"
         "        if (skip_zeros && g == 0.0f) continue;\n        float mi, m2i, vi, u;\n"

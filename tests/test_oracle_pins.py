@@ -691,3 +691,232 @@ def test_lamb_rejects_step_zero(oracle_mod):
     p, gr, m, v = _lamb_state(900, 16, "f32")
     with pytest.raises(ValueError):
         oracle_mod.step_f32_lamb(p, gr, m, v, dtype="f32", step=0, **LAMB_HYPER)
+
+
+# --------------------------------------------------------------------------
+# 8-bit blockwise state (Dettmers, Lewis, Shleifer & Zettlemoyer, "8-bit
+# Optimizers via Block-wise Quantization", ICLR 2022, sections 2.1-2.3).
+# --------------------------------------------------------------------------
+
+from fractions import Fraction
+
+
+def _rn32(fr: Fraction) -> np.float32:
+    """The binary32 value nearest to the exact rational fr (ties to an even
+    significand), found by comparing exact distances to the neighbours."""
+    c = np.float32(float(fr))
+    cands = [c, np.nextafter(c, np.float32(np.inf)), np.nextafter(c, np.float32(-np.inf))]
+    best = min(cands, key=lambda x: (abs(Fraction(float(x)) - fr),
+                                     int(np.array(x).view(np.uint32)) & 1))
+    return np.float32(best)
+
+
+def _map_from_bits(signed: bool) -> np.ndarray:
+    """Every 8-bit pattern of the data type decoded from its fields, as the
+    paper describes them: [sign,] E zero bits (decimal exponent 10^-E), an
+    indicator bit 1, then F fraction bits f of a linear quantization of
+    [0.1, 1] (the midpoint of the f-th of 2^F equal bins).  Patterns without
+    an indicator are 0, except one spare pattern, read as 1.0."""
+    vals = []
+    body = 7 if signed else 8                      # bits after the sign
+    for pattern in range(256):
+        sign = -1 if (signed and pattern >> 7) else 1
+        bits = pattern & ((1 << body) - 1)
+        if bits == 0 or (not signed and bits == 1):   # no indicator among the 7 leading bits
+            vals.append(None)
+            continue
+        width = body if signed else body - 1            # the unsigned last bit is a fraction bit
+        lead = bits if signed else bits >> 1
+        E = width - lead.bit_length()                   # zero bits before the indicator
+        if E > 6:
+            vals.append(None)
+            continue
+        F = (body - 1 - E)                              # remaining bits after the indicator
+        f = bits & ((1 << F) - 1)
+        value = Fraction(1, 10 ** E) * (Fraction(1, 10) + Fraction(9, 10) * Fraction(2 * f + 1, 2 ** (F + 1)))
+        vals.append(sign * value)
+    exact = sorted(set(v for v in vals if v is not None))
+    assert len(exact) == 254, len(exact)
+    out = np.array([_rn32(v) for v in exact] + [np.float32(0.0), np.float32(1.0)], np.float32)
+    return np.sort(out)
+
+
+@pytest.mark.parametrize("signed", [True, False])
+def test_quant_map_is_the_papers_data_type(oracle_mod, signed):
+    want = _map_from_bits(signed)
+    got = oracle_mod.quant_map(signed)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    # structure: strictly ascending, 0 and 1 present, 2^F values per decade
+    assert np.all(np.diff(got.astype(np.float64)) > 0)
+    assert 0.0 in got and got[-1] == 1.0
+    pos = got[(got > 0) & (got < 1)].astype(np.float64)
+    for E in range(7):
+        F = (6 if signed else 7) - E
+        inside = pos[(pos >= 0.1 * 10.0 ** -E) & (pos < 10.0 ** -E)]
+        assert len(inside) == 2 ** F, (E, len(inside))
+        if len(inside) > 1:      # a linear fraction: equal steps of 0.9*10^-E/2^F
+            assert np.allclose(np.diff(inside), 0.9 * 10.0 ** -E / 2 ** F, rtol=1e-5)
+    if signed:                   # symmetric apart from the spare 1.0
+        assert got[127] == 0.0 and np.array_equal(got[:127], -got[128:255][::-1])
+    else:
+        assert got[0] == 0.0 and np.all(got >= 0)
+
+
+def _nearest_codes(qmap, x):
+    """Brute force: the index of the nearest map value (float64 distances,
+    first index on a tie, i.e. the lower code)."""
+    d = np.abs(x.astype(np.float64)[:, None] - qmap.astype(np.float64)[None, :])
+    return np.argmin(d, axis=1).astype(np.uint8)
+
+
+@pytest.mark.parametrize("signed", [True, False])
+def test_quantize_is_the_nearest_code(oracle_mod, signed):
+    qmap = oracle_mod.quant_map(signed)
+    g = np.random.Generator(np.random.Philox(31))
+    lo = -1.0 if signed else 0.0
+    xs = [g.uniform(lo, 1.0, 4000).astype(np.float32),
+          (np.sign(g.uniform(lo, 1.0, 4000)) * 10.0 ** g.uniform(-9, 0, 4000)).astype(np.float32),
+          qmap]
+    a, b = qmap[:-1].astype(np.float64), qmap[1:].astype(np.float64)
+    mid = ((a + b) / 2).astype(np.float32)
+    exact_ties = mid[mid.astype(np.float64) == (a + b) / 2]
+    assert exact_ties.size > 100
+    xs += [exact_ties, np.nextafter(mid, np.float32(2)), np.nextafter(mid, np.float32(-2)),
+           np.array([0.0, -0.0, 1.0, 1e-45, 1e-30, 5e-8], np.float32)]
+    if signed:
+        xs.append(np.array([-1.0, -1e-45], np.float32))
+    x = np.concatenate(xs)
+    assert np.array_equal(oracle_mod.quantize(qmap, x), _nearest_codes(qmap, x))
+    assert np.array_equal(oracle_mod.quantize(qmap, qmap), np.arange(256, dtype=np.uint8))
+    # every exact tie goes to the lower of its two codes
+    codes = oracle_mod.quantize(qmap, exact_ties)
+    assert np.all(qmap[codes] < exact_ties)
+
+
+def _block_quantize(qmap, x, block=2048):
+    """Reference block quantization: per block the absmax in float32, the
+    normalised values x/absmax (float32 division), brute-force nearest codes;
+    the code of 0 where the absmax is 0."""
+    n = x.size
+    nb = (n + block - 1) // block
+    codes = np.empty(n, np.uint8)
+    amax = np.zeros(nb, np.float32)
+    zc = int(np.nonzero(qmap == 0.0)[0][0])
+    for b in range(nb):
+        seg = x[b * block:(b + 1) * block]
+        a = np.float32(np.max(np.abs(seg))) if seg.size else np.float32(0)
+        amax[b] = a
+        if a > 0:
+            codes[b * block:(b + 1) * block] = _nearest_codes(qmap, (seg / a).astype(np.float32))
+        else:
+            codes[b * block:(b + 1) * block] = zc
+    return codes, amax
+
+
+def _dequant(qmap, codes, amax, block=2048):
+    return (qmap[codes] * np.repeat(amax, block)[:codes.size]).astype(np.float32)
+
+
+def _eightbit_reference(oracle_mod, algo, dtype, p, gr, q1, q2, a1, a2, step, hyper, skip):
+    """The 8-bit step composed from pinned parts: dequantize (map value times
+    block absmax), the plain fp32 oracle step (pinned to torch.optim), and the
+    reference block quantization above."""
+    smap, umap = oracle_mod.quant_map(True), oracle_mod.quant_map(False)
+    n = p.size
+    nb = (n + 2047) // 2048
+    m = _dequant(smap, q1[:n], a1[:nb])
+    v = _dequant(umap, q2, a2)
+    s1 = m
+    if algo == "ademamix":
+        s1 = np.concatenate([m, _dequant(smap, q1[n:], a1[nb:])])
+    p = p.copy()
+    oracle_mod.step_f32(p, gr, s1, v, dtype=dtype, algo=algo, step=step, skip_zeros=skip, **hyper)
+    c1, b1 = _block_quantize(smap, s1[:n])
+    c2, b2 = _block_quantize(umap, v)
+    if algo == "ademamix":
+        c3, b3 = _block_quantize(smap, s1[n:])
+        c1, b1 = np.concatenate([c1, c3]), np.concatenate([b1, b3])
+    return p, c1, c2, b1, b2
+
+
+EIGHT_HYPER = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, beta3=0.9999, alpha=5.0,
+                   weight_decay=0.01)
+
+
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("t", [1, 2, 10, 1000])
+def test_8bit_step_is_dequantize_update_quantize(oracle_mod, algo, dtype, t):
+    """Random 8-bit states (codes and block absmaxes; zero state at t = 1),
+    a ragged last block, with and without skip_zeros: param bits, codes and
+    absmaxes equal the composition of the pinned parts."""
+    n = 3 * 2048 + 777
+    nb = 4
+    two = algo == "ademamix"
+    g = np.random.Generator(np.random.Philox(900 + t))
+    for skip in (False, True):
+        p = synth.to_storage(g.standard_normal(n).astype(np.float32), dtype)
+        gr = synth.to_storage((g.standard_normal(n) * 10.0 ** g.uniform(-5, 0, n)).astype(np.float32),
+                              dtype)
+        if skip:
+            gr[::5] = 0
+        if t == 1:
+            q1 = np.zeros(2 * n if two else n, np.uint8)
+            q2 = np.zeros(n, np.uint8)
+            a1 = np.zeros(2 * nb if two else nb, np.float32)
+            a2 = np.zeros(nb, np.float32)
+        else:
+            q1 = g.integers(0, 256, 2 * n if two else n).astype(np.uint8)
+            q2 = g.integers(0, 256, n).astype(np.uint8)
+            a1 = (g.random(2 * nb if two else nb) * 1e-2).astype(np.float32)
+            a2 = (g.random(nb) * 1e-4).astype(np.float32)
+        want = _eightbit_reference(oracle_mod, algo, dtype, p, gr, q1, q2, a1, a2, t,
+                                   EIGHT_HYPER, skip)
+        got = [p.copy(), q1.copy(), q2.copy(), a1.copy(), a2.copy()]
+        oracle_mod.step_8bit(got[0], gr, got[1], got[2], got[3], got[4], dtype=dtype, algo=algo,
+                             step=t, skip_zeros=skip, **EIGHT_HYPER)
+        for k, (x, y) in enumerate(zip(got, want)):
+            assert np.array_equal(x.view(np.uint8), y.view(np.uint8)), (skip, k)
+
+
+@pytest.mark.parametrize("algo", ["adam", "ademamix"])
+def test_8bit_first_step_equals_the_32bit_step(oracle_mod, algo):
+    """From zero state the dequantized moments are exactly 0, so the first
+    8-bit update of the param is the 32-bit step's, bit for bit; and each
+    block's stored absmax is the largest |m| of the 32-bit step's moments in
+    that block."""
+    n = 5000
+    g = np.random.Generator(np.random.Philox(77))
+    p = g.standard_normal(n).astype(np.float32)
+    gr = (g.standard_normal(n) * 1e-2).astype(np.float32)
+    two = algo == "ademamix"
+    a = [p.copy(), np.zeros(2 * n if two else n, np.uint8), np.zeros(n, np.uint8),
+         np.zeros(6 if two else 3, np.float32), np.zeros(3, np.float32)]
+    oracle_mod.step_8bit(a[0], gr, a[1], a[2], a[3], a[4], dtype="f32", algo=algo, step=1,
+                         **EIGHT_HYPER)
+    b = [p.copy(), np.zeros(2 * n if two else n, np.float32), np.zeros(n, np.float32)]
+    oracle_mod.step_f32(b[0], gr, b[1], b[2], dtype="f32", algo=algo, step=1, **EIGHT_HYPER)
+    assert np.array_equal(a[0], b[0])
+    for blk in range(3):
+        sl = slice(2048 * blk, min(n, 2048 * (blk + 1)))
+        assert a[3][blk] == np.max(np.abs(b[1][:n][sl]))
+        assert a[4][blk] == np.max(b[2][sl])
+
+
+def test_8bit_zero_gradient_keeps_zero_state(oracle_mod):
+    """g = 0 everywhere from zero state without decay: the moments stay 0, every
+    absmax stays 0 and every code is the code of 0; the param is unchanged."""
+    n = 4097
+    p = np.linspace(-1, 1, n).astype(np.float32)
+    q1 = np.zeros(n, np.uint8)
+    q2 = np.zeros(n, np.uint8)
+    a1 = np.zeros(3, np.float32)
+    a2 = np.zeros(3, np.float32)
+    h = dict(EIGHT_HYPER, weight_decay=0.0)
+    q = p.copy()
+    oracle_mod.step_8bit(q, np.zeros(n, np.float32), q1, q2, a1, a2, dtype="f32", algo="adam",
+                         step=1, **h)
+    smap, umap = oracle_mod.quant_map(True), oracle_mod.quant_map(False)
+    assert np.array_equal(q, p)
+    assert np.all(a1 == 0) and np.all(a2 == 0)
+    assert np.all(smap[q1] == 0) and np.all(umap[q2] == 0)
