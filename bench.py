@@ -910,6 +910,125 @@ def run_max_unorm(numel=268_435_456, steps=50, warmup=10, max_unorm=1.0):
             "rows": rows}
 
 
+def eightbit_bytes_per_elem(algo, dt):
+    """Algorithmic bytes per element of the 8-bit-state step: param and grad
+    in their storage type, one byte per state quantity per element read and
+    written, and each 2,048-element block's fp32 absmax per quantity read and
+    written (8 bytes per quantity per block)."""
+    es = 4 if dt == "f32" else 2
+    q = 3 if algo == "ademamix" else 2
+    return 3 * es + 2 * q + 8 * q / 2048
+
+
+def run_eightbit(numel=268_435_456, steps=50, warmup=10):
+    """The 8-bit blockwise-state step (opt2s_step_8bit) on one tensor of
+    `numel` elements (fp32 Adam, bf16 AdEMAMix), timed beside the 32-bit step
+    on the same param/grad; and the mixed AdamW collection of the eager
+    protocol (2,000 tensors of 64..1,024 elements with fp32 state plus 64
+    tensors of 4,096..65,536 elements with 8-bit state) in one launch, L2
+    flushed before each step."""
+    import torch
+    from elementwise_optimizer_b200 import binding as B
+    from elementwise_optimizer_b200 import synth
+    dev = torch.device("cuda")
+    peak, kind = measured_peak()
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+    rows = []
+    for algo, dt in (("adam", "f32"), ("ademamix", "bf16")):
+        two = algo == "ademamix"
+        nb = (numel + 2047) // 2048
+        p = torch.randn(numel, device=dev).to(tdt[dt])
+        grads = [(torch.randn(numel, device=dev) * 1e-2).to(tdt[dt]) for _ in range(2)]
+        q1 = torch.zeros((2 if two else 1) * numel, dtype=torch.uint8, device=dev)
+        q2 = torch.zeros(numel, dtype=torch.uint8, device=dev)
+        a1 = torch.zeros((2 if two else 1) * nb, device=dev)
+        a2 = torch.zeros(nb, device=dev)
+        lists = [B.TensorList8.from_tensors([p], [g], [q1], [q2], [a1], [a2]) for g in grads]
+        h = B.make_hyper(algo, weight_decay=0.01, beta3=0.9999, alpha=5.0)
+        row = {"algo": algo, "dtype": dt, "state": "8-bit blockwise"}
+        ms = []
+        for t in range(1, warmup + 1):
+            B.opt2s_step_8bit(lists[t % 2], h, t)
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        ev[0].record()
+        for k in range(steps):
+            B.opt2s_step_8bit(lists[k % 2], h, warmup + 1 + k)
+            ev[k + 1].record()
+        torch.cuda.synchronize()
+        ms = sum(ev[k].elapsed_time(ev[k + 1]) for k in range(steps)) / steps
+        per = eightbit_bytes_per_elem(algo, dt)
+        gbs = per * numel / (ms / 1e3) / 1e9
+        row["eightbit"] = {"ms_mean": ms, "bytes_per_elem": per, "gbs": gbs, "frac": gbs / peak,
+                           "elements_per_s": numel / (ms / 1e3)}
+        del q1, q2, a1, a2, lists
+        s1 = torch.zeros((2 if two else 1) * numel, device=dev)
+        s2 = torch.zeros(numel, device=dev)
+        plain = [B.TensorList.from_tensors([p], [g], [s1], [s2]) for g in grads]
+        for t in range(1, warmup + 1):
+            B.opt2s_step(plain[t % 2], h, t)
+        torch.cuda.synchronize()
+        ev[0].record()
+        for k in range(steps):
+            B.opt2s_step(plain[k % 2], h, warmup + 1 + k)
+            ev[k + 1].record()
+        torch.cuda.synchronize()
+        ms32 = sum(ev[k].elapsed_time(ev[k + 1]) for k in range(steps)) / steps
+        row["fp32_state"] = {"ms_mean": ms32, "bytes_per_elem": BYTES_PER_ELEM[(algo, dt)],
+                             "frac": BYTES_PER_ELEM[(algo, dt)] * numel / (ms32 / 1e3) / 1e9 / peak}
+        row["time_ratio_8_over_32"] = ms / ms32
+        rows.append(row)
+        del p, grads, s1, s2, plain
+        B.opt2s_release_cache()
+        torch.cuda.empty_cache()
+    # the mixed collection
+    w = synth.small_collection()
+    sizes = list(w.sizes) + [4096 * (1 << (i % 5)) for i in range(64)]
+    dtypes = list(w.dtypes) + [("f32", "bf16", "f16")[i % 3] for i in range(64)]
+    gen = torch.Generator(device=dev).manual_seed(3)
+    ps, gs, s1s, s2s, a1s, a2s = [], [], [], [], [], []
+    for n, d in zip(sizes, dtypes):
+        ps.append(torch.randn(n, device=dev, generator=gen).to(tdt[d]))
+        gs.append((torch.randn(n, device=dev, generator=gen) * 1e-2).to(tdt[d]))
+        if B.state_bits_for(n) == 8:
+            s1s.append(torch.zeros(n, dtype=torch.uint8, device=dev))
+            s2s.append(torch.zeros(n, dtype=torch.uint8, device=dev))
+            a1s.append(torch.zeros((n + 2047) // 2048, device=dev))
+            a2s.append(torch.zeros((n + 2047) // 2048, device=dev))
+        else:
+            s1s.append(torch.zeros(n, device=dev))
+            s2s.append(torch.zeros(n, device=dev))
+            a1s.append(None)
+            a2s.append(None)
+    tl = B.TensorList8.from_tensors(ps, gs, s1s, s2s, a1s, a2s)
+    h = B.make_hyper("adam", weight_decay=0.01)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    for t in range(1, 6):
+        B.opt2s_step_8bit(tl, h, t)
+    torch.cuda.synchronize()
+    launches0 = B.launch_count()
+    times = []
+    for t in range(6, 206):
+        flush.fill_(float(t))
+        flush.sum()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        B.opt2s_step_8bit(tl, h, t)
+        b.record()
+        times.append((a, b))
+    torch.cuda.synchronize()
+    us = sorted(a.elapsed_time(b) * 1e3 for a, b in times)
+    n8 = sum(n for n in sizes if B.state_bits_for(n) == 8)
+    mixed = {"tensors": len(sizes), "numel": int(sum(sizes)), "numel_8bit": int(n8),
+             "tensors_8bit": sum(1 for n in sizes if B.state_bits_for(n) == 8),
+             "us_median": _pct(us, 0.5), "us_p10": _pct(us, 0.1), "us_p90": _pct(us, 0.9),
+             "launches_per_step": (B.launch_count() - launches0) / 200,
+             "l2": "flushed before each step (256 MB written, then read)"}
+    return {"mode": "eightbit", "numel": numel, "peak_gbs": peak, "peak_source": kind,
+            "rows": rows, "mixed_adamw_collection": mixed}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -926,7 +1045,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the small-collection, e2e and cpu_baseline legs")
     ap.add_argument("--mode", choices=["headline", "direct-cells", "eager-collection", "max-unorm",
-                                       "shard-emulated", "roofline-table"],
+                                       "shard-emulated", "roofline-table", "eightbit"],
                     default="headline",
                     help="headline: the one-line bench; the others follow the issue's "
                          "direct-cell and eager-collection protocol and print their tables")
@@ -945,7 +1064,8 @@ def main():
         from elementwise_optimizer_b200 import _build
         _build.build()
         torch.cuda.set_device(local_rank)
-        sized = {"roofline-table": run_roofline_table, "max-unorm": run_max_unorm}
+        sized = {"roofline-table": run_roofline_table, "max-unorm": run_max_unorm,
+                 "eightbit": run_eightbit}
         if args.mode in sized and args.numel:
             res = sized[args.mode](numel=args.numel)
         else:

@@ -19,10 +19,11 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libopt2s.so")
 
-SOURCES = [os.path.join(CSRC, "opt2s_kernel.cu"), os.path.join(CSRC, "opt2s_api.cpp"),
+SOURCES = [os.path.join(CSRC, "opt2s_kernel.cu"), os.path.join(CSRC, "opt2s_kernel8.cu"),
+           os.path.join(CSRC, "opt2s_api.cpp"), os.path.join(CSRC, "opt2s_api8.cpp"),
            os.path.join(CSRC, "opt2s_noalloc.cu")]
-HEADERS = [os.path.join(CSRC, "opt2s_internal.h"), os.path.join(INCLUDE, "opt2s.h"),
-           os.path.join(INCLUDE, "opt2s_testing.h")]
+HEADERS = [os.path.join(CSRC, "opt2s_internal.h"), os.path.join(CSRC, "opt2s_device.cuh"),
+           os.path.join(INCLUDE, "opt2s.h"), os.path.join(INCLUDE, "opt2s_testing.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-shared",

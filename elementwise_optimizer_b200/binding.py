@@ -72,6 +72,22 @@ class opt2s_shard_desc(ctypes.Structure):
                 ("state1", ctypes.c_void_p), ("state2", ctypes.c_void_p)]
 
 
+class opt2s_tensor8(ctypes.Structure):
+    _fields_ = [("param", ctypes.c_void_p), ("grad", ctypes.c_void_p),
+                ("state1", ctypes.c_void_p), ("state2", ctypes.c_void_p),
+                ("absmax1", ctypes.c_void_p), ("absmax2", ctypes.c_void_p),
+                ("numel", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("state_bits", ctypes.c_int32)]
+
+
+class TensorListDesc8(ctypes.Structure):
+    _fields_ = [("tensors", ctypes.POINTER(opt2s_tensor8)), ("count", ctypes.c_int32)]
+
+
+BLOCK8 = 2048
+MIN_8BIT_SIZE = 4096
+
+
 class opt2s_testing_chunk(ctypes.Structure):
     _fields_ = [("tensor", ctypes.c_int64), ("start", ctypes.c_int64),
                 ("len", ctypes.c_int64), ("dtype", ctypes.c_int32),
@@ -95,6 +111,9 @@ EXPORTS = {
                                             ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
     "opt2s_step_lamb": (ctypes.c_int, [ctypes.POINTER(TensorListDesc), ctypes.POINTER(Hyper),
                                        ctypes.c_int, ctypes.c_void_p]),
+    "opt2s_step_8bit": (ctypes.c_int, [ctypes.POINTER(TensorListDesc8), ctypes.POINTER(Hyper),
+                                       ctypes.c_int, ctypes.c_void_p]),
+    "opt2s_8bit_state_bits": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64]),
     "opt2s_fill_step_scalars": (ctypes.c_int, [ctypes.POINTER(Hyper), ctypes.c_int, ctypes.c_int,
                                                ctypes.c_void_p]),
     "opt2s_plan_step_table": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
@@ -212,6 +231,42 @@ class TensorList:
         return cls(recs)
 
 
+class TensorList8:
+    """A marshalled collection for the 8-bit-state step: records (param,
+    grad, state1, state2, absmax1, absmax2, numel, dtype_code, state_bits),
+    pointers as ints (absmax pointers 0 for 32-bit records)."""
+
+    def __init__(self, records: Sequence[tuple]):
+        n = len(records)
+        self._arr = (opt2s_tensor8 * max(n, 1))()
+        for i, (p, g, s1, s2, a1, a2, numel, dt, bits) in enumerate(records):
+            self._arr[i] = opt2s_tensor8(p, g, s1, s2, a1 or None, a2 or None, int(numel),
+                                         int(dt), int(bits))
+        self.desc = TensorListDesc8(ctypes.cast(self._arr, ctypes.POINTER(opt2s_tensor8)), n)
+        self.count = n
+
+    @classmethod
+    def from_tensors(cls, params, grads, state1, state2, absmax1, absmax2) -> "TensorList8":
+        """From torch tensors; a record is 8-bit when its state1 is uint8
+        (then absmax1/absmax2 are its fp32 block absmaxes), else 32-bit
+        (absmax entries None)."""
+        import torch
+        recs = []
+        for p, g, s1, s2, a1, a2 in zip(params, grads, state1, state2, absmax1, absmax2):
+            for t in (p, g, s1, s2) + tuple(x for x in (a1, a2) if x is not None):
+                if not t.is_contiguous():
+                    raise ValueError("tensors must be contiguous")
+            if g.dtype != p.dtype or g.numel() != p.numel():
+                raise ValueError("grad must match param in dtype and size")
+            eight = s1.dtype == torch.uint8
+            if eight != (a1 is not None and a2 is not None):
+                raise ValueError("8-bit records need both absmax tensors, 32-bit ones none")
+            recs.append((_ptr(p), _ptr(g), _ptr(s1), _ptr(s2), _ptr(a1) if eight else 0,
+                         _ptr(a2) if eight else 0, p.numel(), _torch_dtype_code(p),
+                         8 if eight else 32))
+        return cls(recs)
+
+
 def make_hyper(algo: str = "adam", lr: float = 1e-3, beta1: float = 0.9,
                beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
                beta3: float = 0.0, alpha: float = 0.0, skip_zeros: bool = False) -> Hyper:
@@ -276,6 +331,18 @@ def opt2s_step_lamb(tl: TensorList, hyper: Hyper, step: int, stream=None) -> Non
     ||param|| / ||direction||; four launches on `stream`."""
     check(lib().opt2s_step_lamb(ctypes.byref(tl.desc), ctypes.byref(hyper), int(step),
                                 _stream_handle(stream)), "opt2s_step_lamb")
+
+
+def opt2s_step_8bit(tl: "TensorList8", hyper: Hyper, step: int, stream=None) -> None:
+    """One step of a collection with 8-bit blockwise state (small tensors
+    with fp32 state in the same launch)."""
+    check(lib().opt2s_step_8bit(ctypes.byref(tl.desc), ctypes.byref(hyper), int(step),
+                                _stream_handle(stream)), "opt2s_step_8bit")
+
+
+def state_bits_for(numel: int, min_8bit_size: int = MIN_8BIT_SIZE) -> int:
+    """8 when a tensor of numel elements keeps 8-bit state, else 32."""
+    return int(lib().opt2s_8bit_state_bits(int(numel), int(min_8bit_size)))
 
 
 def noalloc_max_chunks() -> int:

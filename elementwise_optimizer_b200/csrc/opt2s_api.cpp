@@ -682,6 +682,7 @@ OPT2S_API int opt2s_release_cache(void)
         if (s != OPT2S_OK) st = s;
     }
     g_cache.clear();
+    opt2s::release_cache8();
     return st;
 }
 

@@ -147,6 +147,38 @@ cudaError_t launch_step_lamb(const ChunkRec* d_chunks, int64_t nchunks, int skip
 // can launch with.
 cudaError_t max_block_threads_scaled(int algo, int skip_zeros, int lamb, int* out);
 
+// The step with 8-bit blockwise state.  A tensor with 8-bit state is cut
+// into blocks of kBlock8Elems elements; each block is one record, stepped by
+// one CTA: its param and grad (storage dtype), its codes of m (q1), v (q2)
+// and, for AdEMAMix, m2 (q3), and the block's absmax of each (a1, a2, a3: one
+// float each), all offset to the block's first element.  Small tensors with
+// fp32 state are ChunkRec chunks of the same launch.
+constexpr int64_t kBlock8Elems = 2048;
+struct alignas(16) Block8Rec {
+    void* p;
+    const void* g;
+    uint8_t* q1;
+    uint8_t* q2;
+    uint8_t* q3;      // AdEMAMix: codes of m2; not read by Adam
+    float* a1;
+    float* a2;
+    float* a3;        // AdEMAMix: absmax of m2
+    uint32_t len;     // elements in the block, 1..kBlock8Elems
+    int32_t dtype;
+};
+static_assert(sizeof(Block8Rec) == 80, "Block8Rec layout");
+
+// Launches one 8-bit-state step on `stream`: `nblocks` block records and
+// `nchunks` 32-bit chunk records (device memory).  max_blocks <= 0: the
+// occupancy cap (resident CTAs per SM x SMs).
+cudaError_t launch_step8(const Block8Rec* d_blocks, int64_t nblocks, const ChunkRec* d_chunks,
+                         int64_t nchunks, int algo, int skip_zeros, const StepScalars& s,
+                         int max_blocks, cudaStream_t stream);
+
+// Frees the cached plans of the 8-bit-state step (opt2s_api8.cpp); called by
+// opt2s_release_cache.
+void release_cache8();
+
 // Sets s->inv_bc1, s->inv_bc2 = RN64(1/bc1), RN64(1/bc2) (host).
 void fill_reciprocals(StepScalars* s);
 

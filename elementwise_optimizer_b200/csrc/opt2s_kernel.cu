@@ -10,418 +10,18 @@
 // and no tensor-core work: it is bound by HBM bandwidth (28 bytes per element
 // for fp32 Adam, 36 for fp32 AdEMAMix).
 //
-// Arithmetic: the 32-bit two-state update of bitsandbytes issue "Investigate
-// a 256-thread SM103 path for small 32-bit optimizer tensors" (sections
-// "Problem", "Scope", "Correctness oracle"), with the standard Adam (Kingma &
-// Ba 2015, Algorithm 1), decoupled weight decay (Loshchilov & Hutter 2019,
-// Algorithm 2) and AdEMAMix (Pagliardini et al. 2024, Algorithm 1)
-// definitions.  Every operation is an explicit round-to-nearest intrinsic
-// (__fmul_rn / __fadd_rn / __fdiv_rn / __fsqrt_rn) or the exact constant
-// division below, none of which the compiler may contract into FMA, so the
-// result of an element equals the plain IEEE evaluation of the documented
-// order and never depends on which code
-// path (vector body, scalar head/tail), chunk, warp or block computed it: the
-// issue's "Correctness oracle" section requires that launch geometry must not
-// change optimizer arithmetic.
+// The element arithmetic and the chunk walkers live in opt2s_device.cuh.
+// Every element's result is the plain IEEE evaluation of the documented fp32
+// order whatever code path, chunk, warp or block computed it: the issue's
+// "Correctness oracle" section requires that launch geometry must not change
+// optimizer arithmetic.
 
 #include <mutex>
 
-#include <cuda_bf16.h>
-#include <cuda_fp16.h>
-#include <cuda_runtime.h>
-
-#include "opt2s_internal.h"
+#include "opt2s_device.cuh"
 
 namespace opt2s {
 namespace {
-
-// Global loads and stores with the default cache policy.  Every byte of a
-// step is touched once, but measured on B200 the default (evict-normal)
-// policy streams this read-modify-write pattern about 1% faster than the
-// evict-first hints of ld/st.global.cs.
-template <typename T>
-__device__ __forceinline__ T ld_global(const T* p) { return *p; }
-template <typename T>
-__device__ __forceinline__ void st_global(T* p, const T& v) { *p = v; }
-
-// ---------------------------------------------------------------------------
-// Exact division by a per-launch constant.
-//
-// For every binary32 x and every binary32 d with 0 < |d| <= 1 (the bias
-// corrections bc1, bc2 lie in (0, 1]), with r = RN64(1/d) the correctly
-// rounded binary64 reciprocal computed once per launch on the host:
-//            RN32( RN64(x * r) ) == RN32(x / d).
-// Why: RN64(x*r) = (x/d)(1+e) with |e| <= 2^-52 + 2^-106, so it suffices that
-// x/d is never within 2^-49 (relative) of a binary32 rounding boundary
-// unless it is a binary32 number itself (then |e| < half an ulp keeps it).
-// A boundary is M = Mi*2^k with Mi odd; x - d*M is a multiple of the smaller
-// of the units of x's last bit and of d*M's last bit, and d*M spans fewer
-// than 2^49 of the latter, so if x != d*M then |x/d - M| >= 2^-49 |M|.
-// x == d*M cannot happen: for normal-range boundaries Mi has 25 significant
-// bits while x has 24, and a subnormal-range boundary (an odd multiple of
-// 2^-150) times |d| <= 1 is never a multiple of 2^-149 as every binary32 x
-// is.  binary64 neither overflows nor underflows here, and 0, +-Inf and NaN
-// pass through the product unchanged.  (The exclusion argument used in the
-// analysis of double rounding; see Muller et al., Handbook of Floating-Point
-// Arithmetic, 2nd ed., ch. 4.)  A GPU test checks it against __fdiv_rn on
-// random operands of every class.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ float div_by_constant(float x, double r)
-{
-    return __double2float_rn(__dmul_rn(static_cast<double>(x), r));
-}
-
-// ---------------------------------------------------------------------------
-// The per-element update.  direction() moves the moments of one element (in
-// place) and returns its update direction u = num/den; m/bc1 and v/bc2 use
-// the exact constant division above, num/den is an IEEE division.  update()
-// then applies the step to p.  With SKIP, an element whose gradient compares
-// equal to zero (+0 or -0) is left untouched (no decay either).  MODE:
-//   kPlain   p = p*decay - lr*u
-//   kScaled  p = p*decay - lr*(scale*u)   (bounded update norm; scale = 1
-//                                          gives the plain value)
-//   kLamb    p = p - lr*(scale*w), w = u + wd*p   (LAMB: the weight decay
-//                                          inside the trust-ratio scaled step)
-// ---------------------------------------------------------------------------
-enum : int { kPlain = 0, kScaled = 1, kLamb = 2 };
-
-template <int ALGO>
-__device__ __forceinline__ float direction(float g, float& m, float& v, float& m2,
-                                           const StepScalars& s)
-{
-    m = __fadd_rn(__fmul_rn(s.beta1, m), __fmul_rn(s.one_minus_beta1, g));
-    v = __fadd_rn(__fmul_rn(s.beta2, v),
-                  __fmul_rn(__fmul_rn(s.one_minus_beta2, g), g));
-    float num = div_by_constant(m, s.inv_bc1);
-    if (ALGO == kAdEMAMix) {
-        m2 = __fadd_rn(__fmul_rn(s.beta3, m2), __fmul_rn(s.one_minus_beta3, g));
-        num = __fadd_rn(num, __fmul_rn(s.alpha, m2));
-    }
-    const float den = __fadd_rn(__fsqrt_rn(div_by_constant(v, s.inv_bc2)), s.eps);
-    return __fdiv_rn(num, den);
-}
-
-// LAMB's decayed direction w = u + wd*p of an element.
-__device__ __forceinline__ float lamb_direction(float u, float p, float wd)
-{
-    return __fadd_rn(u, __fmul_rn(wd, p));
-}
-
-template <int ALGO, bool SKIP, int MODE = kPlain>
-__device__ __forceinline__ void update(float g, float& p, float& m, float& v,
-                                       float& m2, const StepScalars& s, float scale = 1.0f,
-                                       float wd = 0.0f)
-{
-    if (SKIP && g == 0.0f) return;
-    const float u = direction<ALGO>(g, m, v, m2, s);
-    if (MODE == kLamb)
-        p = __fsub_rn(p, __fmul_rn(s.lr, __fmul_rn(scale, lamb_direction(u, p, wd))));
-    else
-        p = __fsub_rn(__fmul_rn(p, s.decay), __fmul_rn(s.lr, MODE == kScaled ? __fmul_rn(scale, u) : u));
-}
-
-// ---------------------------------------------------------------------------
-// Storage traits of param / grad.  kVec elements make one 16-byte access.
-// ---------------------------------------------------------------------------
-template <int DT> struct Param;
-
-template <> struct Param<kF32> {
-    static constexpr int kVec = 4;
-    static constexpr int kBytes = 4;
-    using Raw = float4;
-    __device__ static Raw load(const void* b, uint32_t i) {
-        return ld_global(reinterpret_cast<const float4*>(static_cast<const float*>(b) + i));
-    }
-    __device__ static void store(void* b, uint32_t i, const Raw& r) {
-        st_global(reinterpret_cast<float4*>(static_cast<float*>(b) + i), r);
-    }
-    __device__ static void widen(const Raw& r, float (&x)[4]) {
-        x[0] = r.x; x[1] = r.y; x[2] = r.z; x[3] = r.w;
-    }
-    __device__ static Raw narrow(const float (&x)[4], const Raw&, const float (&)[4], bool) {
-        // fp32: an untouched element already holds its loaded bits
-        return make_float4(x[0], x[1], x[2], x[3]);
-    }
-    __device__ static float load1(const void* b, uint32_t i) {
-        return ld_global(static_cast<const float*>(b) + i);
-    }
-    __device__ static void store1(void* b, uint32_t i, float x) {
-        st_global(static_cast<float*>(b) + i, x);
-    }
-    // kVec elements from an address that need not be 16-byte aligned
-    __device__ static Raw load_elems(const void* b, uint32_t i) {
-        const float* f = static_cast<const float*>(b) + i;
-        return make_float4(ld_global(f), ld_global(f + 1), ld_global(f + 2), ld_global(f + 3));
-    }
-};
-
-// Shared by the two 16-bit formats: only the conversions differ.
-template <typename H2, typename Cvt> struct Param16 {
-    static constexpr int kVec = 8;
-    static constexpr int kBytes = 2;
-    using Raw = uint4;
-    __device__ static Raw load(const void* b, uint32_t i) {
-        return ld_global(reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(b) + i));
-    }
-    __device__ static void store(void* b, uint32_t i, const Raw& r) {
-        st_global(reinterpret_cast<uint4*>(static_cast<unsigned short*>(b) + i), r);
-    }
-    __device__ static void widen(const Raw& r, float (&x)[8]) {
-        const H2* h = reinterpret_cast<const H2*>(&r);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 f = Cvt::to_float2(h[k]);
-            x[2 * k] = f.x;
-            x[2 * k + 1] = f.y;
-        }
-    }
-    // Round to nearest even; with `skip`, elements whose gradient is zero keep
-    // their original storage bits exactly (NaN payloads included).
-    __device__ static Raw narrow(const float (&x)[8], const Raw& orig,
-                                 const float (&g)[8], bool skip) {
-        Raw r;
-        H2* h = reinterpret_cast<H2*>(&r);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) h[k] = Cvt::from_float2(x[2 * k], x[2 * k + 1]);
-        if (skip) {
-            uint32_t* w = reinterpret_cast<uint32_t*>(&r);
-            const uint32_t* o = reinterpret_cast<const uint32_t*>(&orig);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t mask = 0xFFFFu << (16 * (j & 1));
-                if (g[j] == 0.0f) w[j >> 1] = (w[j >> 1] & ~mask) | (o[j >> 1] & mask);
-            }
-        }
-        return r;
-    }
-    __device__ static float load1(const void* b, uint32_t i) {
-        return Cvt::to_float(ld_global(static_cast<const unsigned short*>(b) + i));
-    }
-    // kVec elements from an address that need not be 16-byte aligned
-    __device__ static Raw load_elems(const void* b, uint32_t i) {
-        const unsigned short* h = static_cast<const unsigned short*>(b) + i;
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            w[k] = static_cast<uint32_t>(ld_global(h + 2 * k)) |
-                   (static_cast<uint32_t>(ld_global(h + 2 * k + 1)) << 16);
-        return make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    __device__ static void store1(void* b, uint32_t i, float x) {
-        st_global(static_cast<unsigned short*>(b) + i, Cvt::from_float(x));
-    }
-};
-
-struct CvtF16 {
-    __device__ static float2 to_float2(__half2 h) { return __half22float2(h); }
-    __device__ static __half2 from_float2(float a, float b) { return __floats2half2_rn(a, b); }
-    __device__ static float to_float(unsigned short u) { return __half2float(__ushort_as_half(u)); }
-    __device__ static unsigned short from_float(float x) { return __half_as_ushort(__float2half_rn(x)); }
-};
-
-struct CvtBF16 {
-    __device__ static float2 to_float2(__nv_bfloat162 h) { return __bfloat1622float2(h); }
-    __device__ static __nv_bfloat162 from_float2(float a, float b) { return __floats2bfloat162_rn(a, b); }
-    __device__ static float to_float(unsigned short u) { return __bfloat162float(__ushort_as_bfloat16(u)); }
-    __device__ static unsigned short from_float(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
-};
-
-template <> struct Param<kF16> : Param16<__half2, CvtF16> {};
-template <> struct Param<kBF16> : Param16<__nv_bfloat162, CvtBF16> {};
-
-// fp32 state: N elements as N/4 16-byte accesses.
-template <int N>
-__device__ __forceinline__ void load_state(const float* b, uint32_t i, float (&x)[N]) {
-#pragma unroll
-    for (int k = 0; k < N / 4; ++k) {
-        const float4 t = ld_global(reinterpret_cast<const float4*>(b + i) + k);
-        x[4 * k] = t.x; x[4 * k + 1] = t.y; x[4 * k + 2] = t.z; x[4 * k + 3] = t.w;
-    }
-}
-
-// fp32 state through 16-byte accesses when `vec`, else element by element.
-template <int N>
-__device__ __forceinline__ void load_state_any(const float* b, uint32_t i, bool vec, float (&x)[N]) {
-    if (vec) {
-        load_state<N>(b, i, x);
-    } else {
-#pragma unroll
-        for (int k = 0; k < N; ++k) x[k] = ld_global(b + i + k);
-    }
-}
-
-template <int N>
-__device__ __forceinline__ void store_state(float* b, uint32_t i, const float (&x)[N]);
-
-template <int N>
-__device__ __forceinline__ void store_state_any(float* b, uint32_t i, bool vec, const float (&x)[N]) {
-    if (vec) {
-        store_state<N>(b, i, x);
-    } else {
-#pragma unroll
-        for (int k = 0; k < N; ++k) st_global(b + i + k, x[k]);
-    }
-}
-
-template <int N>
-__device__ __forceinline__ void store_state(float* b, uint32_t i, const float (&x)[N]) {
-#pragma unroll
-    for (int k = 0; k < N / 4; ++k)
-        st_global(reinterpret_cast<float4*>(b + i) + k,
-               make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]));
-}
-
-// One element through the scalar path (chunk head, tail, or a chunk whose
-// arrays are not mutually 16-byte aligned).  A skipped element is not even
-// written back.
-template <int DT, int ALGO, bool SKIP, int MODE = kPlain>
-__device__ __forceinline__ void scalar_element(const ChunkRec& c, uint32_t i,
-                                               const StepScalars& s, float scale = 1.0f,
-                                               float wd = 0.0f)
-{
-    using P = Param<DT>;
-    const float g = P::load1(c.g, i);
-    if (SKIP && g == 0.0f) return;
-    float p = P::load1(c.p, i);
-    float m = ld_global(c.m + i);
-    float v = ld_global(c.v + i);
-    float m2 = 0.0f;
-    if (ALGO == kAdEMAMix) m2 = ld_global(c.m2 + i);
-    update<ALGO, false, MODE>(g, p, m, v, m2, s, scale, wd);
-    P::store1(c.p, i, p);
-    st_global(c.m + i, m);
-    st_global(c.v + i, v);
-    if (ALGO == kAdEMAMix) st_global(c.m2 + i, m2);
-}
-
-__device__ __forceinline__ bool aligned16(const void* q, uint32_t head, int bytes) {
-    return ((reinterpret_cast<uintptr_t>(q) + static_cast<uintptr_t>(head) * bytes) & 15u) == 0;
-}
-
-// Alignment of the arrays other than param at the vector body's start.
-struct Aligned {
-    bool g, m, v, m2;
-    __device__ bool all() const { return g && m && v && m2; }
-};
-
-// The vector body of a chunk: vectors [0, nvec) starting at element `head`,
-// at which param is 16-byte aligned.  ALL: every other array is aligned too
-// (the common case); otherwise each array uses 16-byte or element-wise
-// accesses according to its own flag.  In the aligned case every lane moves 8
-// elements per iteration (two 16-byte vectors of fp32, or one of fp16/bf16),
-// so a warp iteration covers 256 contiguous elements of each array; the mixed
-// case moves one vector per lane per iteration.
-template <int DT, int ALGO, bool SKIP, bool ALL, int MODE = kPlain>
-__device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars& s, int lane,
-                                            uint32_t head, uint32_t nvec, Aligned al,
-                                            float scale = 1.0f, float wd = 0.0f)
-{
-    using P = Param<DT>;
-    constexpr int V = P::kVec;
-    constexpr int U = ALL ? 8 / V : 1;   // the mixed path keeps fewer values live
-    for (uint32_t v0 = 0; v0 < nvec; v0 += 32 * U) {
-        typename P::Raw graw[U], praw[U];
-        float m[U][V], v[U][V], m2[U][V];
-        // all loads of the iteration first, so they are in flight together
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const uint32_t vi = v0 + u * 32 + lane;
-            if (vi < nvec) {
-                const uint32_t e = head + vi * V;
-                graw[u] = (ALL || al.g) ? P::load(c.g, e) : P::load_elems(c.g, e);
-                praw[u] = P::load(c.p, e);
-                load_state_any<V>(c.m, e, ALL || al.m, m[u]);
-                load_state_any<V>(c.v, e, ALL || al.v, v[u]);
-                if (ALGO == kAdEMAMix) load_state_any<V>(c.m2, e, ALL || al.m2, m2[u]);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const uint32_t vi = v0 + u * 32 + lane;
-            if (vi < nvec) {
-                const uint32_t e = head + vi * V;
-                float g[V], p[V];
-                P::widen(graw[u], g);
-                P::widen(praw[u], p);
-#pragma unroll
-                for (int j = 0; j < V; ++j)
-                    update<ALGO, SKIP, MODE>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s, scale, wd);
-                P::store(c.p, e, P::narrow(p, praw[u], g, SKIP));
-                store_state_any<V>(c.m, e, ALL || al.m, m[u]);
-                store_state_any<V>(c.v, e, ALL || al.v, v[u]);
-                if (ALGO == kAdEMAMix) store_state_any<V>(c.m2, e, ALL || al.m2, m2[u]);
-            }
-        }
-    }
-}
-
-// One chunk, processed by one warp: a scalar head up to the element at which
-// param is 16-byte aligned, the vector body, and a scalar tail.
-template <int DT, int ALGO, bool SKIP, int MODE = kPlain>
-__device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& s, int lane,
-                                          float scale = 1.0f, float wd = 0.0f)
-{
-    using P = Param<DT>;
-    constexpr int V = P::kVec;
-    const uint32_t len = c.len;
-    uint32_t head = static_cast<uint32_t>(
-        ((16u - (reinterpret_cast<uintptr_t>(c.p) & 15u)) & 15u) / P::kBytes);
-    if (head > len) head = len;
-    const uint32_t nvec = (len - head) / V;
-    const uint32_t body_end = head + nvec * V;
-
-    for (uint32_t i = lane; i < head; i += 32)
-        scalar_element<DT, ALGO, SKIP, MODE>(c, i, s, scale, wd);
-    for (uint32_t i = body_end + lane; i < len; i += 32)
-        scalar_element<DT, ALGO, SKIP, MODE>(c, i, s, scale, wd);
-
-    const Aligned al{aligned16(c.g, head, P::kBytes), aligned16(c.m, head, 4),
-                     aligned16(c.v, head, 4), ALGO != kAdEMAMix || aligned16(c.m2, head, 4)};
-    if (al.all())
-        vector_body<DT, ALGO, SKIP, true, MODE>(c, s, lane, head, nvec, al, scale, wd);
-    else
-        vector_body<DT, ALGO, SKIP, false, MODE>(c, s, lane, head, nvec, al, scale, wd);
-}
-
-// A short 16-bit chunk (its record's dtype carries kShortFlag), processed by
-// one warp with element-wise accesses: lane l takes elements l, l + 32, l + 64
-// and l + 96, so each access instruction is still contiguous across the warp,
-// and a lane updates at most 4 elements where one 16-byte vector would give it
-// 8.  All loads come first, then the updates and stores.  Same arithmetic as
-// the vector body; a skipped element is not written back.  Kept out of line,
-// with its arguments by value (no stack frame), so that the step kernel's
-// register count stays that of its vector path.
-template <int DT, int ALGO, bool SKIP>
-__device__ __noinline__ void short_chunk(const ChunkRec c, const StepScalars s, int lane)
-{
-    using P = Param<DT>;
-    constexpr int K = kShortChunkElems / 32;
-    const uint32_t len = c.len;
-    float g[K], p[K], m[K], v[K], m2[K];
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-        const uint32_t i = lane + 32 * k;
-        g[k] = p[k] = m[k] = v[k] = m2[k] = 0.0f;
-        if (i < len) {
-            g[k] = P::load1(c.g, i);
-            p[k] = P::load1(c.p, i);
-            m[k] = ld_global(c.m + i);
-            v[k] = ld_global(c.v + i);
-            if (ALGO == kAdEMAMix) m2[k] = ld_global(c.m2 + i);
-        }
-    }
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-        const uint32_t i = lane + 32 * k;
-        if (i < len && !(SKIP && g[k] == 0.0f)) {
-            update<ALGO, false>(g[k], p[k], m[k], v[k], m2[k], s);
-            P::store1(c.p, i, p[k]);
-            st_global(c.m + i, m[k]);
-            st_global(c.v + i, v[k]);
-            if (ALGO == kAdEMAMix) st_global(c.m2 + i, m2[k]);
-        }
-    }
-}
 
 // ---------------------------------------------------------------------------
 // The sharded step (reduce-scatter + update + all-gather in one kernel).

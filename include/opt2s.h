@@ -313,6 +313,80 @@ int opt2s_step_max_unorm(const TensorListDesc *desc, const Hyper *hyper, float m
 int opt2s_step_lamb(const TensorListDesc *desc, const Hyper *hyper, int step,
                     cudaStream_t stream);
 
+/*
+ * 8-bit blockwise optimizer state, for collections whose tensors of at least
+ * min_8bit_size elements keep their state in 8 bits and whose smaller tensors
+ * keep it in fp32 -- the routing the issue's section "Problem" describes for
+ * bitsandbytes' 8-bit Adam/AdamW/AdEMAMix (min_8bit_size = 4096 by default):
+ * the small bias/norm/adapter tensors take the 32-bit update.  Both kinds are
+ * stepped in ONE launch.
+ *
+ * The 8-bit format is that of Dettmers, Lewis, Shleifer & Zettlemoyer,
+ * "8-bit Optimizers via Block-wise Quantization", ICLR 2022: each state
+ * quantity of a tensor is cut into blocks of OPT2S_BLOCK8 = 2048 elements
+ * (section 2.1); a block keeps one fp32 absmax and one byte per element, the
+ * code of a value of a 256-entry map -- dynamic tree quantization for the
+ * signed m and m2 (section 2.2), dynamic quantization for the non-negative v
+ * (section 2.3).  Code c stands for the c-th smallest map value.  The maps:
+ * for E = 0..6 and F = 6 - E (signed) or 7 - E (unsigned), the values
+ * 10^-E * (0.1 + 0.9*(2f+1)/2^(F+1)), f = 0 .. 2^F - 1 (both signs in the
+ * signed map), each rounded to fp32 once, plus 0 and 1.0: 256 values each.
+ *
+ * Per 8-bit block and step: every element's m = map_s[code]*absmax (fp32
+ * product), likewise v (map_u) and m2; the update of opt2s_step on these
+ * values; then each quantity's new block absmax max|x| and new codes: the
+ * code of the map value nearest to x/absmax (fp32 division; an exact tie
+ * takes the lower code), or the code of 0 when the absmax is 0.  With
+ * skip_zeros an element whose gradient is zero keeps its param and its
+ * dequantized state, which is requantized with the block's new absmax.
+ * A 32-bit record is stepped exactly as opt2s_step steps it.
+ *
+ * Per record, by state_bits:
+ *   8:  state1  uint8 codes of m (numel bytes), AdEMAMix [m1 | m2] (2*numel)
+ *       state2  uint8 codes of v (numel bytes)
+ *       absmax1 fp32 absmax of m per block (nb = ceil(numel/2048) floats),
+ *               AdEMAMix [m1 absmaxes | m2 absmaxes] (2*nb)
+ *       absmax2 fp32 absmax of v per block (nb floats)
+ *       Zero state before step 1: every absmax 0 (the codes then do not
+ *       matter; zero-filling everything is fine).
+ *   32: state1, state2 fp32 as in opt2s_tensor; absmax1, absmax2 NULL.
+ * Pointers need element alignment (fp32 state and absmaxes: 4 bytes; codes:
+ * none); aligned full blocks take 16-byte and 8-byte accesses.
+ *
+ * opt2s_step_8bit: one step of the collection in one launch on `stream`, one
+ * CTA per 8-bit block, warps on the 32-bit tensors' chunks.  Plans (the
+ * block and chunk tables) are cached per device like opt2s_step's.
+ * Validation as opt2s_step, plus state_bits in {8, 32}, non-null absmax
+ * pointers exactly for 8-bit records, and no overlap of any written buffer
+ * (codes and absmaxes included) with another buffer.
+ */
+#define OPT2S_BLOCK8 2048
+#define OPT2S_MIN_8BIT_SIZE 4096
+
+typedef struct {
+    void *param;
+    const void *grad;
+    void *state1;
+    void *state2;
+    float *absmax1;
+    float *absmax2;
+    int64_t numel;
+    int32_t dtype;        /* opt2s_dtype of param and grad */
+    int32_t state_bits;   /* 8 or 32 */
+} opt2s_tensor8;
+
+typedef struct {
+    const opt2s_tensor8 *tensors;   /* HOST array of `count` records */
+    int32_t count;
+} TensorListDesc8;
+
+int opt2s_step_8bit(const TensorListDesc8 *desc, const Hyper *hyper, int step,
+                    cudaStream_t stream);
+
+/* The routing: 8 when numel >= min_8bit_size, else 32 (min_8bit_size <= 0
+ * means OPT2S_MIN_8BIT_SIZE). */
+int opt2s_8bit_state_bits(int64_t numel, int64_t min_8bit_size);
+
 /* Frees every cached plan of every device (waits for the devices first). */
 int opt2s_release_cache(void);
 

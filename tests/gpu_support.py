@@ -269,3 +269,130 @@ class Harness:
             if not np.array_equal(storage_bits(g), host_bits(self._h_g[i])):
                 return False
         return True
+
+
+class Harness8:
+    """A collection for the 8-bit-state step on the GPU and its host mirror.
+
+    Tensors of at least ``min_8bit_size`` elements keep 8-bit blockwise state
+    (uint8 codes of m [| m2] and v, fp32 absmax per 2,048-element block);
+    smaller ones keep fp32 state.  Everything starts at zero.  layout
+    'separate' gives each buffer its own allocation; 'packed' puts every
+    tensor's param/grad (per dtype), codes and fp32 state back to back in
+    shared buffers, so most of them start misaligned.  Direct-mode workloads
+    only (the host mirror holds every element).
+    """
+
+    def __init__(self, w: synth.Workload, device="cuda", min_8bit_size=4096, layout="separate"):
+        assert not w.ring
+        self.w = w
+        self.device = torch.device(device)
+        two = w.algo == "ademamix"
+        self.bits = [8 if n >= min_8bit_size else 32 for n in w.sizes]
+        self.nb = [(n + 2047) // 2048 for n in w.sizes]
+        n_t = len(w.sizes)
+        init = w.params_init()
+        dev = self.device
+
+        def alloc(sizes, dtype):
+            """Views of one buffer (packed) or separate tensors, zero-filled."""
+            if layout == "separate":
+                return [torch.zeros(max(k, 0), dtype=dtype, device=dev) for k in sizes]
+            buf = torch.zeros(sum(sizes) + 1, dtype=dtype, device=dev)
+            out, pos = [], 1 if dtype == torch.uint8 else 0      # codes start odd
+            for k in sizes:
+                out.append(buf[pos:pos + k])
+                pos += k
+            self._keep.append(buf)
+            return out
+
+        self._keep = []
+        # param / grad: packed per dtype through the 32-bit harness's helper
+        self.params, self.grads = [None] * n_t, [None] * n_t
+        for dt in sorted(set(w.dtypes)):
+            members = [i for i, d in enumerate(w.dtypes) if d == dt]
+            ps = alloc([w.sizes[i] for i in members], TORCH[dt])
+            gs = alloc([w.sizes[i] for i in members], TORCH[dt])
+            for k, i in enumerate(members):
+                self.params[i], self.grads[i] = ps[k], gs[k]
+        e8 = [i for i in range(n_t) if self.bits[i] == 8]
+        e32 = [i for i in range(n_t) if self.bits[i] == 32]
+        q1 = alloc([(2 if two else 1) * w.sizes[i] for i in e8], torch.uint8)
+        q2 = alloc([w.sizes[i] for i in e8], torch.uint8)
+        a1 = alloc([(2 if two else 1) * self.nb[i] for i in e8], torch.float32)
+        a2 = alloc([self.nb[i] for i in e8], torch.float32)
+        s1 = alloc([(2 if two else 1) * w.sizes[i] for i in e32], torch.float32)
+        s2 = alloc([w.sizes[i] for i in e32], torch.float32)
+        self.s1, self.s2, self.a1, self.a2 = [None] * n_t, [None] * n_t, [None] * n_t, [None] * n_t
+        for k, i in enumerate(e8):
+            self.s1[i], self.s2[i], self.a1[i], self.a2[i] = q1[k], q2[k], a1[k], a2[k]
+        for k, i in enumerate(e32):
+            self.s1[i], self.s2[i] = s1[k], s2[k]
+        self.h_p, self.h_s1, self.h_s2, self.h_a1, self.h_a2 = [], [], [], [], []
+        for i in range(n_t):
+            self.params[i].copy_(to_device_storage(init[i], w.dtypes[i], dev))
+            self.h_p.append(synth.to_storage(init[i], w.dtypes[i]))
+            n = w.sizes[i]
+            if self.bits[i] == 8:
+                self.h_s1.append(np.zeros((2 if two else 1) * n, np.uint8))
+                self.h_s2.append(np.zeros(n, np.uint8))
+                self.h_a1.append(np.zeros((2 if two else 1) * self.nb[i], np.float32))
+                self.h_a2.append(np.zeros(self.nb[i], np.float32))
+            else:
+                self.h_s1.append(np.zeros((2 if two else 1) * n, np.float32))
+                self.h_s2.append(np.zeros(n, np.float32))
+                self.h_a1.append(None)
+                self.h_a2.append(None)
+        self._h_g = None
+        self.tl = B.TensorList8.from_tensors(self.params, self.grads, self.s1, self.s2,
+                                             self.a1, self.a2)
+        self.hyper = B.make_hyper(w.algo, skip_zeros=w.skip_zeros, **w.hyper)
+        torch.cuda.synchronize(dev)
+
+    def load_grads(self, step):
+        vals = self.w.grads(step)
+        for i, (v, dt) in enumerate(zip(vals, self.w.dtypes)):
+            self.grads[i].copy_(to_device_storage(v, dt, self.device))
+        self._h_g = [synth.to_storage(v, d) for v, d in zip(vals, self.w.dtypes)]
+
+    def gpu_step(self, step, stream=None):
+        B.opt2s_step_8bit(self.tl, self.hyper, step, stream)
+
+    def oracle_step(self, step):
+        w = self.w
+        for i, dt in enumerate(w.dtypes):
+            if self.bits[i] == 8:
+                oracle.step_8bit(self.h_p[i], self._h_g[i], self.h_s1[i], self.h_s2[i],
+                                 self.h_a1[i], self.h_a2[i], dtype=dt, algo=w.algo, step=step,
+                                 skip_zeros=w.skip_zeros, **w.hyper)
+            else:
+                oracle.step_f32(self.h_p[i], self._h_g[i], self.h_s1[i], self.h_s2[i], dtype=dt,
+                                algo=w.algo, step=step, skip_zeros=w.skip_zeros, **w.hyper)
+
+    def step_both(self, step):
+        self.load_grads(step)
+        self.gpu_step(step)
+        self.oracle_step(step)
+
+    def mismatches(self):
+        """(tensor, quantity, count of differing elements) for every array
+        that differs from the host mirror bit for bit."""
+        torch.cuda.synchronize(self.device)
+        bad = []
+        for i in range(len(self.w.sizes)):
+            pairs = [("param", storage_bits(self.params[i]), host_bits(self.h_p[i]))]
+            if self.bits[i] == 8:
+                pairs += [("codes1", self.s1[i].cpu().numpy(), self.h_s1[i]),
+                          ("codes2", self.s2[i].cpu().numpy(), self.h_s2[i]),
+                          ("absmax1", storage_bits(self.a1[i]), host_bits(self.h_a1[i])),
+                          ("absmax2", storage_bits(self.a2[i]), host_bits(self.h_a2[i]))]
+            else:
+                pairs += [("state1", storage_bits(self.s1[i]), host_bits(self.h_s1[i])),
+                          ("state2", storage_bits(self.s2[i]), host_bits(self.h_s2[i]))]
+            for name, a, b in pairs:
+                if not np.array_equal(a, b):
+                    bad.append((i, name, int(np.count_nonzero(a != b))))
+        return bad
+
+    def grads_unchanged(self):
+        return all(np.array_equal(storage_bits(g), host_bits(h)) for g, h in zip(self.grads, self._h_g))

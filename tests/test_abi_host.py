@@ -339,6 +339,65 @@ def test_lamb_step_without_device(L):
     assert e.value.status == -2
 
 
+def _rec8(arena, n, dt="f32", bits=8, algo="adam"):
+    es = 4 if dt == "f32" else 2
+    two = 2 if algo == "ademamix" else 1
+    sb = 1 if bits == 8 else 4
+    nb = (n + 2047) // 2048
+    a1 = arena.alloc(4 * two * nb) if bits == 8 else 0
+    a2 = arena.alloc(4 * nb) if bits == 8 else 0
+    return (arena.alloc(n * es), arena.alloc(n * es), arena.alloc(two * n * sb), arena.alloc(n * sb),
+            a1, a2, n, B.DTYPES[dt], bits)
+
+
+def test_8bit_routing_and_argument_checks(L):
+    """Routing by min_8bit_size, and every record checked before any CUDA
+    call: state_bits in {8, 32}, absmax pointers exactly for 8-bit records,
+    and no overlap of written codes or absmaxes with another buffer."""
+    assert B.state_bits_for(4095) == 32 and B.state_bits_for(4096) == 8
+    assert B.state_bits_for(10, 8) == 8 and B.state_bits_for(7, 8) == 32
+    assert B.state_bits_for(4096, 0) == 8            # <= 0: the default threshold
+    ar = Arena()
+    good = _rec8(ar, 5000)
+    small = _rec8(ar, 100, bits=32)
+    cases = []
+    p, g, s1, s2, a1, a2, n, dt, bits = good
+    cases.append(((p, g, s1, s2, 0, a2, n, dt, 8), -1))        # missing absmax1
+    cases.append(((p, g, s1, s2, a1, a2, n, dt, 16), -1))      # bad state_bits
+    cases.append(((p, g, s1, s1, a1, a2, n, dt, 8), -2))       # codes of m and v overlap
+    cases.append(((p, g, s1, s2, a1, a1, n, dt, 8), -2))       # absmaxes overlap
+    cases.append(((p, g, s1, s2, a1, a2, n, 7, 8), -1))        # bad dtype
+    sp, sg, ss1, ss2, _, _, sn, sdt, _ = small
+    cases.append(((sp, sg, ss1, ss2, a1, 0, sn, sdt, 32), -1))  # absmax on a 32-bit record
+    cases.append(((sp, sg, ss1 + 2, ss2, 0, 0, sn, sdt, 32), -1))  # misaligned fp32 state
+    for rec, want in cases:
+        with pytest.raises(B.Opt2sError) as e:
+            B.opt2s_step_8bit(B.TensorList8([good if rec[0] != p else small, rec]), H, 1, stream=0)
+        assert e.value.status == want, rec
+    with pytest.raises(B.Opt2sError) as e:
+        B.opt2s_step_8bit(B.TensorList8([good]), H, 0, stream=0)
+    assert e.value.status == -1
+    B.opt2s_step_8bit(B.TensorList8([]), H, 1, stream=0)                         # empty: no-op
+    # AdEMAMix state1 holds [m1 | m2] codes (2n bytes) and 2 x blocks absmaxes
+    ar2 = Arena()
+    rec = _rec8(ar2, 4096, algo="ademamix")
+    q = list(rec)
+    q[3] = q[2] + 4096                  # v codes inside m2's half of state1
+    with pytest.raises(B.Opt2sError) as e:
+        B.opt2s_step_8bit(B.TensorList8([tuple(q)]), B.make_hyper("ademamix", beta3=0.9, alpha=1.0),
+                          1, stream=0)
+    assert e.value.status == -2
+
+
+@pytest.mark.skipif(_cuda_available(), reason="checks the no-device path")
+def test_8bit_step_without_device(L):
+    ar = Arena()
+    tl = B.TensorList8([_rec8(ar, 5000), _rec8(ar, 100, bits=32)])
+    with pytest.raises(B.Opt2sError) as e:
+        B.opt2s_step_8bit(tl, H, 1, stream=0)
+    assert e.value.status == -4                       # CUDA: no device
+
+
 def test_missing_library_fails_loudly(tmp_path):
     code = ("import elementwise_optimizer_b200.binding as b; b.LIB_PATH='/nonexistent/x.so'\n"
             "try:\n  b.lib()\nexcept RuntimeError as e:\n  print('RAISED', e)\n")
