@@ -8,12 +8,16 @@ tensors (for which it reads ``data_ptr()``, ``numel()`` and ``dtype``).
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from typing import Iterable, Sequence
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libopt2s.so")
+# the test build: the same kernels plus the forcing knobs, the fault
+# injection and the division check (tests only, through testing_library())
+TESTING_LIB_PATH = os.path.join(_PKG, "libopt2s_testing.so")
 
 OPT2S_F32, OPT2S_F16, OPT2S_BF16 = 0, 1, 2
 OPT2S_ADAM, OPT2S_ADEMAMIX = 0, 1
@@ -150,23 +154,64 @@ EXPORTS = {
     "opt2s_testing_max_block_threads": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32]),
 }
 
-_lib = None
+# exported by the test build only
+TESTING_ONLY = {"opt2s_testing_set_chunk_elems", "opt2s_testing_set_launch",
+                "opt2s_testing_fail_allocs", "opt2s_testing_check_division"}
+
+_libs = {}
+_use_testing = False
+
+
+def _load(path: str, testing: bool) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build the CUDA library first "
+            "(python -m elementwise_optimizer_b200._build); there is no CPU fallback")
+    L = ctypes.CDLL(path)
+    for name, (res, args) in EXPORTS.items():
+        if name in TESTING_ONLY and not testing:
+            continue
+        fn = getattr(L, name)
+        fn.restype, fn.argtypes = res, args
+    return L
 
 
 def lib() -> ctypes.CDLL:
-    """Load libopt2s.so (raises if it has not been built)."""
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(
-                f"{LIB_PATH} is missing: build the CUDA library first "
-                "(python -m elementwise_optimizer_b200._build); there is no CPU fallback")
-        L = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in EXPORTS.items():
-            fn = getattr(L, name)
-            fn.restype, fn.argtypes = res, args
-        _lib = L
-    return _lib
+    """The loaded library (raises if it has not been built): libopt2s.so, or
+    the test build inside ``testing_library()``."""
+    key = "testing" if _use_testing else "product"
+    if key not in _libs:
+        _libs[key] = _load(TESTING_LIB_PATH if _use_testing else LIB_PATH, _use_testing)
+    return _libs[key]
+
+
+@contextlib.contextmanager
+def testing_library():
+    """Route every call of this module to the test build of the library
+    (libopt2s_testing.so: the same kernels, plus the forcing knobs and the
+    fault injection).  Tests only; plans made inside stay bound to it.  On
+    exit the knobs are reset and its plan cache released."""
+    global _use_testing
+    prev = _use_testing
+    _use_testing = True
+    try:
+        yield lib()
+    finally:
+        try:
+            L = lib()
+            L.opt2s_testing_set_launch(0, 0)
+            L.opt2s_testing_set_chunk_elems(0)
+            L.opt2s_testing_fail_allocs(0)
+            L.opt2s_release_cache()
+        finally:
+            _use_testing = prev
+
+
+def _testing_lib() -> ctypes.CDLL:
+    if not _use_testing:
+        raise RuntimeError("forcing knobs and fault injection exist only in the test build: "
+                           "call them inside binding.testing_library()")
+    return lib()
 
 
 def _error_string(status: int) -> str:
@@ -176,9 +221,10 @@ def _error_string(status: int) -> str:
         return "?"
 
 
-def check(status: int, where: str) -> None:
+def check(status: int, where: str, L: ctypes.CDLL | None = None) -> None:
+    """Raise Opt2sError for a failed call (L: the library that made it)."""
     if status != OPT2S_OK:
-        raise Opt2sError(status, where, lib().opt2s_last_cuda_error())
+        raise Opt2sError(status, where, (L or lib()).opt2s_last_cuda_error())
 
 
 # ---------------------------------------------------------------------------
@@ -354,28 +400,29 @@ class Plan:
 
     def __init__(self, tl: TensorList, algo: str):
         self._h = ctypes.c_void_p()
+        self._L = lib()   # a plan belongs to the library that made it
         self.tl = tl  # keep the descriptor alive with the plan
-        check(lib().opt2s_plan_create(ctypes.byref(tl.desc), ALGOS[algo],
-                                      ctypes.byref(self._h)), "opt2s_plan_create")
+        check(self._L.opt2s_plan_create(ctypes.byref(tl.desc), ALGOS[algo],
+                                        ctypes.byref(self._h)), "opt2s_plan_create", self._L)
 
     @property
     def num_chunks(self) -> int:
-        return int(lib().opt2s_plan_num_chunks(self._h))
+        return int(self._L.opt2s_plan_num_chunks(self._h))
 
     def step(self, hyper: Hyper, step: int, stream=None) -> None:
-        check(lib().opt2s_plan_step(self._h, ctypes.byref(hyper), int(step),
-                                    _stream_handle(stream)), "opt2s_plan_step")
+        check(self._L.opt2s_plan_step(self._h, ctypes.byref(hyper), int(step),
+                                      _stream_handle(stream)), "opt2s_plan_step", self._L)
 
     def step_table(self, skip_zeros: bool, d_table: int, table_len: int, d_index: int,
                    stream=None) -> None:
         """opt2s_plan_step_table: the scalars come from d_table[*d_index]
         (device pointers), which the call then advances; capturable."""
-        check(lib().opt2s_plan_step_table(self._h, int(bool(skip_zeros)), d_table, int(table_len),
-                                          d_index, _stream_handle(stream)), "opt2s_plan_step_table")
+        check(self._L.opt2s_plan_step_table(self._h, int(bool(skip_zeros)), d_table, int(table_len),
+                                            d_index, _stream_handle(stream)), "opt2s_plan_step_table", self._L)
 
     def close(self) -> None:
         if self._h:
-            check(lib().opt2s_plan_destroy(self._h), "opt2s_plan_destroy")
+            check(self._L.opt2s_plan_destroy(self._h), "opt2s_plan_destroy", self._L)
             self._h = ctypes.c_void_p()
 
     def __del__(self):
@@ -424,7 +471,8 @@ def opt2s_release_cache() -> None:
 
 
 # ---------------------------------------------------------------------------
-# Validation scaffolding (include/opt2s_testing.h) -- tests only
+# Validation scaffolding (include/opt2s_testing.h) -- tests only.  The forcing
+# knobs, the fault injection and the division check need testing_library().
 # ---------------------------------------------------------------------------
 
 def testing_build_chunks(tl: TensorList, algo: str, chunk_elems: int = 0) -> list:
@@ -461,7 +509,7 @@ def testing_validate(tl: TensorList, hyper: Hyper, step: int) -> int:
 
 
 def testing_set_chunk_elems(n: int) -> int:
-    return int(lib().opt2s_testing_set_chunk_elems(int(n)))
+    return int(_testing_lib().opt2s_testing_set_chunk_elems(int(n)))
 
 
 def testing_max_block_threads(algo: str, skip_zeros: bool) -> int:
@@ -474,7 +522,8 @@ def testing_max_block_threads(algo: str, skip_zeros: bool) -> int:
 def testing_check_division(seed: int, n: int, mode: int) -> int:
     """Mismatches between the kernel's constant division and __fdiv_rn."""
     out = ctypes.c_int64()
-    check(lib().opt2s_testing_check_division(seed, n, mode, ctypes.byref(out)), "check_division")
+    check(_testing_lib().opt2s_testing_check_division(seed, n, mode, ctypes.byref(out)),
+          "check_division")
     return int(out.value)
 
 
@@ -483,7 +532,7 @@ def testing_choose_chunk_elems(tl: TensorList, resident_warps: int) -> int:
 
 
 def testing_fail_allocs(count: int) -> None:
-    check(lib().opt2s_testing_fail_allocs(int(count)), "testing_fail_allocs")
+    check(_testing_lib().opt2s_testing_fail_allocs(int(count)), "testing_fail_allocs")
 
 
 def launch_count() -> int:
@@ -492,4 +541,4 @@ def launch_count() -> int:
 
 
 def testing_set_launch(block_threads: int = 0, max_blocks: int = 0) -> None:
-    check(lib().opt2s_testing_set_launch(int(block_threads), int(max_blocks)), "set_launch")
+    check(_testing_lib().opt2s_testing_set_launch(int(block_threads), int(max_blocks)), "set_launch")

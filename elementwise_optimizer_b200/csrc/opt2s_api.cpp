@@ -49,11 +49,28 @@ namespace {
 
 thread_local int t_last_cuda_error = 0;
 
-int64_t g_chunk_elems = 0;     // testing override (0 = default)
-int g_block_threads = 0;       // testing override (0 = default)
-int g_max_blocks = 0;          // testing override (0 = occupancy cap)
 std::atomic<int64_t> g_launches{0};   // kernels launched by this library
-std::atomic<int> g_fail_allocs{0};    // testing: plan allocations to fail
+
+// Forcing knobs exist only in the test build of the library
+// (libopt2s_testing.so, compiled with OPT2S_TESTING); the product build has
+// the defaults as constants, so no caller can change its launch geometry.
+#ifdef OPT2S_TESTING
+int64_t g_chunk_elems = 0;     // forced chunk length (0 = chosen per plan)
+int g_block_threads = 0;       // forced threads per block (0 = default)
+int g_max_blocks = 0;          // forced cap on blocks (0 = occupancy cap)
+std::atomic<int> g_fail_allocs{0};    // plan allocations to fail
+
+bool injected_alloc_failure()
+{
+    return g_fail_allocs.load() > 0 && g_fail_allocs.fetch_sub(1) > 0;
+}
+#else
+constexpr int64_t g_chunk_elems = 0;
+constexpr int g_block_threads = 0;
+constexpr int g_max_blocks = 0;
+
+constexpr bool injected_alloc_failure() { return false; }
+#endif
 
 int cuda_fail(cudaError_t e)
 {
@@ -251,8 +268,8 @@ int unorm_workspace(const TensorListDesc* desc, int64_t chunk_elems, opt2s_plan*
     size_t total = 0;
     for (size_t x : sizes) total += x;
     cudaError_t e;
-    if (g_fail_allocs.load() > 0 && g_fail_allocs.fetch_sub(1) > 0)
-        e = cudaErrorMemoryAllocation;                // injected by the test scaffolding
+    if (injected_alloc_failure())
+        e = cudaErrorMemoryAllocation;                // injected by the test build
     else
         e = cudaMalloc(&plan->d_unorm, total);
     if (e != cudaSuccess) {
@@ -305,8 +322,8 @@ int plan_create(const TensorListDesc* desc, int32_t algo, opt2s_plan** out, bool
     if (!plan) return OPT2S_ERR_NO_MEMORY;
     if (!table.empty()) {
         const size_t bytes = table.size() * sizeof(ChunkRec);
-        if (g_fail_allocs.load() > 0 && g_fail_allocs.fetch_sub(1) > 0)
-            e = cudaErrorMemoryAllocation;            // injected by the test scaffolding
+        if (injected_alloc_failure())
+            e = cudaErrorMemoryAllocation;            // injected by the test build
         else
             e = cudaMalloc(&plan->d_chunks, bytes);
         if (e != cudaSuccess) {
@@ -498,6 +515,7 @@ int plan_step_normed(const opt2s_plan* plan, const Hyper* h, bool lamb, float ma
 OPT2S_API int opt2s_step(const TensorListDesc* desc, const Hyper* hyper, int step,
                          cudaStream_t stream)
 {
+    OPT2S_RANGE("opt2s_step");
     int st = validate_hyper(hyper, step);
     if (st != OPT2S_OK) return st;
     if (!desc || desc->count < 0 || (desc->count > 0 && !desc->tensors))
@@ -513,6 +531,7 @@ OPT2S_API int opt2s_step(const TensorListDesc* desc, const Hyper* hyper, int ste
 OPT2S_API int opt2s_step_max_unorm(const TensorListDesc* desc, const Hyper* hyper, float max_unorm,
                                    int step, cudaStream_t stream)
 {
+    OPT2S_RANGE("opt2s_step_max_unorm");
     int st = validate_hyper(hyper, step);
     if (st != OPT2S_OK) return st;
     if (!std::isfinite(max_unorm) || !(max_unorm > 0.0f)) return OPT2S_ERR_INVALID_ARG;
@@ -529,6 +548,7 @@ OPT2S_API int opt2s_step_max_unorm(const TensorListDesc* desc, const Hyper* hype
 OPT2S_API int opt2s_step_lamb(const TensorListDesc* desc, const Hyper* hyper, int step,
                               cudaStream_t stream)
 {
+    OPT2S_RANGE("opt2s_step_lamb");
     int st = validate_hyper(hyper, step);
     if (st != OPT2S_OK) return st;
     if (hyper->algo != OPT2S_ADAM) return OPT2S_ERR_INVALID_ARG;
@@ -552,6 +572,7 @@ OPT2S_API int opt2s_plan_create(const TensorListDesc* desc, int32_t algo, opt2s_
 OPT2S_API int opt2s_plan_step(const opt2s_plan* plan, const Hyper* hyper, int step,
                               cudaStream_t stream)
 {
+    OPT2S_RANGE("opt2s_plan_step");
     return plan_step(plan, hyper, step, stream);
 }
 
@@ -623,6 +644,7 @@ OPT2S_API int opt2s_shard_range(int64_t numel, int32_t world, int32_t rank, int6
 OPT2S_API int opt2s_shard_step(const opt2s_shard_desc* d, const Hyper* hyper, int step,
                                cudaStream_t stream)
 {
+    OPT2S_RANGE("opt2s_shard_step");
     int st = validate_hyper(hyper, step);
     if (st != OPT2S_OK) return st;
     if (!d || d->reserved != 0) return OPT2S_ERR_INVALID_ARG;
@@ -753,6 +775,39 @@ OPT2S_API int opt2s_testing_validate(const TensorListDesc* desc, const Hyper* hy
     return validate_desc(desc, hyper->algo);
 }
 
+OPT2S_API int64_t opt2s_testing_default_chunk_elems(void) { return opt2s::kDefaultChunkElems; }
+
+OPT2S_API int opt2s_testing_max_block_threads(int32_t algo, int32_t skip_zeros)
+{
+    if ((algo != OPT2S_ADAM && algo != OPT2S_ADEMAMIX) || (skip_zeros != 0 && skip_zeros != 1))
+        return OPT2S_ERR_INVALID_ARG;
+    int widest = 0;
+    cudaError_t e = opt2s::max_block_threads(algo, skip_zeros, -1, &widest);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return widest;
+}
+
+OPT2S_API int64_t opt2s_testing_choose_chunk_elems(const TensorListDesc* desc, int64_t resident_warps)
+{
+    if (!desc || desc->count < 0 || (desc->count > 0 && !desc->tensors)) return OPT2S_ERR_INVALID_ARG;
+    return choose_chunk_elems(desc, resident_warps);
+}
+
+OPT2S_API int64_t opt2s_testing_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+// ---------------------------------------------------------------------------
+// Shared with the other translation units (opt2s_internal.h)
+// ---------------------------------------------------------------------------
+
+int opt2s::record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+
+void opt2s::count_launches(int64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+#ifdef OPT2S_TESTING
+// ---------------------------------------------------------------------------
+// Forcing knobs, fault injection and the division check: test build only
+// ---------------------------------------------------------------------------
+
 OPT2S_API int64_t opt2s_testing_set_chunk_elems(int64_t chunk_elems)
 {
     const int64_t prev = g_chunk_elems;
@@ -771,16 +826,11 @@ OPT2S_API int opt2s_testing_set_launch(int block_threads, int max_blocks)
     return OPT2S_OK;
 }
 
-OPT2S_API int64_t opt2s_testing_default_chunk_elems(void) { return opt2s::kDefaultChunkElems; }
-
-OPT2S_API int opt2s_testing_max_block_threads(int32_t algo, int32_t skip_zeros)
+OPT2S_API int opt2s_testing_fail_allocs(int count)
 {
-    if ((algo != OPT2S_ADAM && algo != OPT2S_ADEMAMIX) || (skip_zeros != 0 && skip_zeros != 1))
-        return OPT2S_ERR_INVALID_ARG;
-    int widest = 0;
-    cudaError_t e = opt2s::max_block_threads(algo, skip_zeros, -1, &widest);
-    if (e != cudaSuccess) return cuda_fail(e);
-    return widest;
+    if (count < 0) return OPT2S_ERR_INVALID_ARG;
+    g_fail_allocs.store(count);
+    return OPT2S_OK;
 }
 
 OPT2S_API int opt2s_testing_check_division(uint64_t seed, int64_t n, int32_t mode,
@@ -799,26 +849,4 @@ OPT2S_API int opt2s_testing_check_division(uint64_t seed, int64_t n, int32_t mod
     *mismatches = static_cast<int64_t>(h);
     return OPT2S_OK;
 }
-
-OPT2S_API int64_t opt2s_testing_choose_chunk_elems(const TensorListDesc* desc, int64_t resident_warps)
-{
-    if (!desc || desc->count < 0 || (desc->count > 0 && !desc->tensors)) return OPT2S_ERR_INVALID_ARG;
-    return choose_chunk_elems(desc, resident_warps);
-}
-
-OPT2S_API int opt2s_testing_fail_allocs(int count)
-{
-    if (count < 0) return OPT2S_ERR_INVALID_ARG;
-    g_fail_allocs.store(count);
-    return OPT2S_OK;
-}
-
-OPT2S_API int64_t opt2s_testing_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
-
-// ---------------------------------------------------------------------------
-// Shared with the other translation units (opt2s_internal.h)
-// ---------------------------------------------------------------------------
-
-int opt2s::record_cuda_error(cudaError_t e) { return cuda_fail(e); }
-
-void opt2s::count_launches(int64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+#endif  // OPT2S_TESTING

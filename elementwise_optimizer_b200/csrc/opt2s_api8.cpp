@@ -203,6 +203,7 @@ bool same8(const Plan8& p, const TensorListDesc8* d)
 OPT2S_API int opt2s_step_8bit(const TensorListDesc8* desc, const Hyper* hyper, int step,
                               cudaStream_t stream)
 {
+    OPT2S_RANGE("opt2s_step_8bit");
     int st = opt2s::validate_hyper(hyper, step);
     if (st != OPT2S_OK) return st;
     if (!desc || desc->count < 0 || (desc->count > 0 && !desc->tensors)) return OPT2S_ERR_INVALID_ARG;

@@ -10,6 +10,24 @@
 
 #include "opt2s.h"
 
+// Optional NVTX ranges around the host side of each step entry point, for
+// timeline tools (build with -DOPT2S_NVTX; NVTX v3 is header-only and costs
+// nothing when no tool is attached).  Without the flag they compile away.
+#ifdef OPT2S_NVTX
+#include <nvtx3/nvToolsExt.h>
+namespace opt2s {
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+}  // namespace opt2s
+#define OPT2S_RANGE(name) ::opt2s::NvtxRange opt2s_nvtx_range_(name)
+#else
+#define OPT2S_RANGE(name) ((void)0)
+#endif
+
 namespace opt2s {
 
 enum : int { kF32 = 0, kF16 = 1, kBF16 = 2 };

@@ -90,6 +90,7 @@ int check_desc(const TensorListDesc* d, int32_t algo, int64_t chunk_elems, int64
 OPT2S_API int opt2s_step_noalloc(const TensorListDesc* desc, const Hyper* hyper, int step,
                                  cudaStream_t stream)
 {
+    OPT2S_RANGE("opt2s_step_noalloc");
     int st = opt2s::validate_hyper(hyper, step);
     if (st != OPT2S_OK) return st;
     std::lock_guard<std::mutex> lock(g_mu);

@@ -10,6 +10,14 @@
  * check the issue's "Correctness oracle" requirement that the launch geometry
  * must not change the optimizer arithmetic (results must be bitwise equal).
  *
+ * The host-only queries below are exported by the library.  The forcing
+ * knobs (opt2s_testing_set_chunk_elems, opt2s_testing_set_launch), the fault
+ * injection (opt2s_testing_fail_allocs) and the division check
+ * (opt2s_testing_check_division) exist only in the test build of the
+ * library, libopt2s_testing.so (the same kernels, compiled once and linked
+ * into both); the product libopt2s.so does not export them, and its launch
+ * geometry cannot be changed.
+ *
  * All knobs are process-wide, apply to plans created or launched afterwards,
  * and are not thread-safe against concurrent steps.
  */
@@ -47,12 +55,13 @@ int opt2s_testing_build_chunks(const TensorListDesc *desc, int32_t algo,
 int opt2s_testing_validate(const TensorListDesc *desc, const Hyper *hyper,
                            int step);
 
-/* Chunk length (elements, a positive multiple of 8) for plans created
- * afterwards; 0 restores the per-plan choice.  Returns the previous value. */
+/* Test build only.  Chunk length (elements, a positive multiple of 8) for
+ * plans created afterwards; 0 restores the per-plan choice.  Returns the
+ * previous value. */
 int64_t opt2s_testing_set_chunk_elems(int64_t chunk_elems);
 
-/* Threads per block (a multiple of 32 in [32, 1024]) and a cap on blocks per
- * launch (>= 1) for later launches; 0 restores each default.  A step whose
+/* Test build only.  Threads per block (a multiple of 32 in [32, 1024]) and a
+ * cap on blocks per launch (>= 1) for later launches; 0 restores each default.  A step whose
  * forced width exceeds opt2s_testing_max_block_threads() for its kernel
  * returns OPT2S_ERR_INVALID_ARG without launching. */
 int opt2s_testing_set_launch(int block_threads, int max_blocks);
@@ -87,15 +96,17 @@ int opt2s_testing_unorm_tables(const TensorListDesc *desc, int32_t algo, int64_t
                                uint32_t *group_ranges, uint32_t *first_group,
                                uint32_t *chunk_tensor, int64_t *counts);
 
-/* Runs the step kernel's exact division by a constant in (0, 1] and the IEEE
- * division __fdiv_rn side by side on `n` seeded random operand pairs on the
- * current device (mode 0: x of every class; mode 1: x/d next to a binary32
- * rounding boundary) and writes how many results differ (NaN equals NaN) to
- * *mismatches.  Synchronous; allocates a counter on the device. */
+/* Test build only.  Runs the step kernel's exact division by a constant in
+ * (0, 1] and the IEEE division __fdiv_rn side by side on `n` seeded random
+ * operand pairs on the current device (mode 0: x of every class; mode 1: x/d
+ * next to a binary32 rounding boundary) and writes how many results differ
+ * (NaN equals NaN) to *mismatches.  Synchronous; allocates a counter on the
+ * device. */
 int opt2s_testing_check_division(uint64_t seed, int64_t n, int32_t mode, int64_t *mismatches);
 
-/* Fault injection on the host: the next `count` device allocations of plan
- * creation fail as if the device were out of memory (OPT2S_ERR_NO_MEMORY). */
+/* Test build only.  Fault injection on the host: the next `count` device
+ * allocations of plan creation fail as if the device were out of memory
+ * (OPT2S_ERR_NO_MEMORY). */
 int opt2s_testing_fail_allocs(int count);
 
 /* Number of kernels this library has launched in this process. */

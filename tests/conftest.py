@@ -18,3 +18,13 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture
+def testing_lib():
+    """Run the test against the test build of the library (the same kernels
+    plus the forcing knobs and the fault injection); knobs are reset and the
+    build's plan cache released afterwards."""
+    from elementwise_optimizer_b200 import binding as B
+    with B.testing_library() as L:
+        yield L

@@ -38,16 +38,27 @@ def declared_functions():
     return names
 
 
+def _exported(path):
+    out = subprocess.run(["nm", "-D", "--defined-only", path], check=True,
+                         capture_output=True, text=True).stdout
+    return {l.split()[-1] for l in out.splitlines() if " T " in l and "opt2s_" in l}
+
+
 def test_exports_match_headers(L):
+    """The test build exports every function the headers declare; the
+    product exports all of them but the forcing knobs, the fault injection
+    and the division check, which exist only in the test build."""
     decl = declared_functions()
     assert "opt2s_step" in decl and "opt2s_plan_create" in decl
-    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], check=True,
-                         capture_output=True, text=True).stdout
-    exported = {l.split()[-1] for l in out.splitlines() if " T " in l and "opt2s_" in l}
-    assert exported == decl, (exported ^ decl)
-    for name in decl:
+    assert B.TESTING_ONLY <= decl
+    assert _exported(B.TESTING_LIB_PATH) == decl, (_exported(B.TESTING_LIB_PATH) ^ decl)
+    product = _exported(B.LIB_PATH)
+    assert product == decl - B.TESTING_ONLY, (product ^ (decl - B.TESTING_ONLY))
+    for name in decl - B.TESTING_ONLY:
         assert getattr(L, name) is not None
     assert set(B.EXPORTS) == decl
+    with pytest.raises(RuntimeError):         # knobs need the test build
+        B.testing_set_launch(0, 0)
 
 
 def test_struct_layout_matches_c(L):
@@ -246,6 +257,7 @@ def test_build_chunks_validates_first(L):
     assert e.value.status == -2
 
 
+@pytest.mark.usefixtures("testing_lib")
 def test_testing_knobs_validate(L):
     with pytest.raises(B.Opt2sError):
         B.testing_set_launch(33, 0)
@@ -520,3 +532,21 @@ def test_shard_step_validation(L):
     assert run(state1=params[0] + 64) == -2                        # state inside a param buffer
     assert run(state2=0) == -1
     assert L.opt2s_shard_step(None, ctypes.byref(h), 1, None) == -1
+
+
+def test_host_sources_compile_with_nvtx_ranges():
+    """The optional NVTX ranges (-DOPT2S_NVTX) compile in every host source
+    that marks a step entry point."""
+    import shutil
+    import subprocess
+    gxx = shutil.which("g++")
+    if gxx is None:
+        pytest.skip("no g++")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    csrc = os.path.join(root, "elementwise_optimizer_b200", "csrc")
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    for src in ("opt2s_api.cpp", "opt2s_api8.cpp"):
+        r = subprocess.run([gxx, "-std=c++17", "-fsyntax-only", "-DOPT2S_NVTX",
+                            "-I", os.path.join(root, "include"), "-I", csrc, "-I", cuda_inc,
+                            os.path.join(csrc, src)], capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr

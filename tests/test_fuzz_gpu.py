@@ -70,6 +70,7 @@ def draw_case(case):
     return w, layout, pad, first_step, steps, geometry, max_unorm
 
 
+@pytest.mark.usefixtures("testing_lib")
 @pytest.mark.parametrize("case", range(CASES))
 def test_random_collection_matches_oracle(case):
     w, layout, pad, first_step, steps, geometry, max_unorm = draw_case(case)

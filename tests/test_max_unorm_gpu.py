@@ -28,8 +28,6 @@ def _cuda():
     _build.build()
     B.lib()
     yield
-    B.testing_set_launch(0, 0)
-    B.testing_set_chunk_elems(0)
     B.opt2s_release_cache()
 
 
@@ -101,6 +99,7 @@ def _run(w, max_unorm, steps=2, layout="separate", pad=0, per_tensor=False):
     return _final(h)
 
 
+@pytest.mark.usefixtures("testing_lib")
 def test_geometry_and_alignment_do_not_change_the_result():
     """The norms are summed over fixed 2,048-element blocks in a fixed order,
     so neither the plan's chunk length, the block width, a per-tensor launch

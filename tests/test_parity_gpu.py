@@ -33,8 +33,6 @@ def _cuda():
     _build.build()
     B.lib()
     yield
-    B.testing_set_launch(0, 0)
-    B.testing_set_chunk_elems(0)
     B.opt2s_release_cache()
 
 
@@ -105,6 +103,7 @@ def test_boundary_sweep_1000_steps(algo, dtype, skip, wd):
     assert h.max_rel() <= 1e-5
 
 
+@pytest.mark.usefixtures("testing_lib")
 @pytest.mark.parametrize("mode", [0, 1])
 def test_constant_division_is_exact(mode):
     """The kernel divides by bc1, bc2 through a binary64 reciprocal; it must
@@ -164,6 +163,7 @@ def widest(w):
     return B.testing_max_block_threads(w.algo, w.skip_zeros)
 
 
+@pytest.mark.usefixtures("testing_lib")
 @pytest.mark.parametrize("block_threads,max_blocks,chunk", [
     (32, 0, 0), (64, 1, 0), (128, 3, 0), (384, 0, 0), ("widest", 0, 0), ("widest", 2, 0),
     (256, 0, 8), (256, 0, 64), (256, 0, 1000), (256, 5, 1 << 20)])
@@ -184,6 +184,7 @@ def test_geometry_does_not_change_arithmetic(block_threads, max_blocks, chunk):
     _assert_same(ref, got)
 
 
+@pytest.mark.usefixtures("testing_lib")
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
 def test_single_dtype_kernel_equals_the_generic_kernel(dtype):
     """A collection whose tensors all share one 16-bit dtype runs Adam on a
@@ -215,6 +216,7 @@ def test_single_dtype_kernel_equals_the_generic_kernel(dtype):
         _assert_same(uni, got)
 
 
+@pytest.mark.usefixtures("testing_lib")
 @pytest.mark.parametrize("skip", [False, True])
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("algo", ["adam", "ademamix"])
@@ -312,6 +314,7 @@ def test_misaligned_storage_matches_oracle():
     assert h.max_ulps() == {"param": 0, "state1": 0, "state2": 0}
 
 
+@pytest.mark.usefixtures("testing_lib")
 def test_ademamix_fp16_first_update_is_geometry_independent():
     """The case that failed the issue's bit-exact oracle (comment "NO-GO: the
     public AdEMAMix path fails the bit-exact oracle"): the first update of an
@@ -419,6 +422,7 @@ def test_resume_from_copied_state_is_bitwise():
     _assert_same(ref, _final_state(b))
 
 
+@pytest.mark.usefixtures("testing_lib")
 def test_too_wide_cta_is_rejected_without_launch():
     w = _geometry_workload()
     h = Harness(w)
