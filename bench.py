@@ -62,7 +62,7 @@ def workload(name, numel=0):
     if name == "large_f32" and numel:
         return synth.large_f32(numel)
     return {"large_f32": synth.large_f32, "transformer_bf16": synth.transformer_bf16,
-            "small_collection": synth.small_collection}[name]()
+            "small_collection": synth.small_collection, "single_small": synth.single_small}[name]()
 
 
 def algorithmic_bytes(w):
@@ -289,6 +289,107 @@ def small_collection_us(device, reps=200):
             "launches_per_step": launches / reps, "l2": "flushed before each step (256 MB written, then read)"}
 
 
+def single_small_us(device, reps=200):
+    """µs per step of the single 1,024-element fp32 tensor (Adam): per call
+    between CUDA events with L2 flushed before each step (as the collection),
+    and the device time per launch of 200 steps replayed from a CUDA graph
+    (no host dispatch between them)."""
+    import torch
+    from elementwise_optimizer_b200 import binding as B
+    w = workload("single_small")
+    d = make_device_workload(w, device, 1)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+    for t in range(1, 6):
+        B.opt2s_step(d["lists"][0], d["hyper"], t)
+    torch.cuda.synchronize()
+    times = []
+    launches0 = B.launch_count()
+    for t in range(6, 6 + reps):
+        flush.fill_(float(t))
+        flush.sum()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        B.opt2s_step(d["lists"][0], d["hyper"], t)
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize()
+    launches = B.launch_count() - launches0
+    us = sorted(a.elapsed_time(b) * 1e3 for a, b in times)
+    plan = B.Plan(d["lists"][0], w.algo)
+    plan.step(d["hyper"], 1000)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(reps):
+            plan.step(d["hyper"], 1000)
+    graph.replay()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    graph.replay()
+    b.record(stream)
+    b.synchronize()
+    graph_us = a.elapsed_time(b) * 1e3 / reps
+    del graph
+    plan.close()
+    q = lambda f: us[min(len(us) - 1, int(f * len(us)))]
+    nbytes = algorithmic_bytes(w)
+    return {"workload": w.name, "numel": w.numel, "us_per_step_median": q(0.5),
+            "us_per_step_p10": q(0.1), "us_per_step_p90": q(0.9),
+            "device_us_per_launch_graph": graph_us, "launches_per_step": launches / reps,
+            "algorithmic_bytes": nbytes,
+            "l2": "flushed before each timed step (256 MB written, then read); graph replay: L2 warm",
+            "bound": "launch latency (28,672 bytes a step)"}
+
+
+def transformer_measure(device, steps=10, warmup=3, e2e_steps=3):
+    """The 1.2 B-element bf16 AdEMAMix collection (24 layers, 240 tensors):
+    ms per step, GB/s and fraction of the HBM peak over `steps` steps (CUDA
+    events around each launch), plus the same metric end to end with host
+    buffers (pinned grads in, params out, one slice per tensor)."""
+    import torch
+    from elementwise_optimizer_b200 import binding as B
+    w = workload("transformer_bf16")
+    d = make_device_workload(w, device, 2)
+    stream = torch.cuda.current_stream()
+    step = 0
+    for _ in range(warmup):
+        step += 1
+        B.opt2s_step(d["lists"][step % 2], d["hyper"], step)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for k in range(steps):
+        step += 1
+        B.opt2s_step(d["lists"][step % 2], d["hyper"], step)
+        ev[k + 1].record(stream)
+    torch.cuda.synchronize()
+    per = [ev[k].elapsed_time(ev[k + 1]) for k in range(steps)]
+    mean_s = statistics.mean(per) / 1e3
+    peak, kind = measured_peak()
+    nbytes = algorithmic_bytes(w)
+    out = {"workload": w.name, "numel": w.numel, "tensors": len(w.sizes), "algo": w.algo,
+           "storage": "bf16", "state": "f32", "steps": steps,
+           "ms_per_step": statistics.mean(per), "ms_median": statistics.median(per),
+           "elements_per_s": w.numel / mean_s, "hbm_gbs": nbytes / mean_s / 1e9,
+           "roofline": {"bound": "hbm", "achieved": nbytes / mean_s / 1e9, "peak": peak,
+                        "unit": "GB/s", "frac": nbytes / mean_s / 1e9 / peak,
+                        "peak_source": kind, "algorithmic_bytes_per_launch": nbytes,
+                        "bytes_per_element": nbytes / w.numel},
+           "l2": f"inputs larger than L2 ({nbytes / 1e9:.1f} GB per step), no flush"}
+    if e2e_steps > 0:
+        try:
+            out["e2e"] = e2e_measure(w, d, device, e2e_steps)
+        except Exception as exc:  # reported, not hidden
+            out["e2e_error"] = repr(exc)
+    del d
+    torch.cuda.empty_cache()
+    return out
+
+
 def e2e_measure(w, d, device, steps, slices=8):
     """Same metric through the public call with host buffers: every step
     copies that step's gradient from pinned host memory to the device, runs
@@ -303,18 +404,17 @@ def e2e_measure(w, d, device, steps, slices=8):
     ranges = []                      # (tensor index, start, length) per slice
     for i, p in enumerate(params):
         n = p.numel()
-        k = max(1, min(slices, n // (1 << 20)))
+        # AdEMAMix keeps [m1 | m2] per tensor: a slice is then a whole tensor
+        k = 1 if w.algo == "ademamix" else max(1, min(slices, n // (1 << 20)))
         bounds = [n * j // k for j in range(k + 1)]
         ranges += [(i, bounds[j], bounds[j + 1] - bounds[j]) for j in range(k)]
     host_g = [g.cpu().pin_memory() for g in grads]
     host_p = [torch.empty(p.shape, dtype=p.dtype, pin_memory=True) for p in params]
     lists = []
     for i, a, n in ranges:
-        n1 = s1[i].numel() // params[i].numel()      # 1 (Adam) or 2 (AdEMAMix)
-        if n1 == 2:
-            raise NotImplementedError("sliced e2e supports one-moment state1 layouts")
+        n1 = s1[i].numel() // params[i].numel()      # 1 (Adam) or 2 (AdEMAMix: whole tensor)
         lists.append(B.TensorList.from_tensors([params[i][a:a + n]], [grads[i][a:a + n]],
-                                               [s1[i][a:a + n]], [s2[i][a:a + n]]))
+                                               [s1[i][n1 * a:n1 * (a + n)]], [s2[i][a:a + n]]))
     plans = [B.Plan(tl, w.algo) for tl in lists]     # one explicit plan per slice
     compute = torch.cuda.current_stream()
     h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
@@ -413,6 +513,7 @@ def run_ours(args, rank, world, local_rank):
     extras = {}
     if rank == 0 and world == 1 and not args.no_extras:
         extras["small_collection"] = small_collection_us(device)
+        extras["single_small"] = single_small_us(device)
     if not args.no_extras:
         # every rank streams its own host buffers; the line reports all ranks'
         # elements over the slowest rank's time.  A rank whose leg fails still
@@ -430,6 +531,12 @@ def run_ours(args, rank, world, local_rank):
             e2e["value"] = w.numel * world / (e2e_ms / 1e3)
             e2e["n_gpus"] = world
             extras["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_extras and args.workload == "large_f32":
+        # the largest configuration, measured after the headline's buffers
+        # are freed (1.2 B elements, 21.7 GB with two gradient buffers)
+        del d
+        torch.cuda.empty_cache()
+        extras["transformer_bf16"] = transformer_measure(device)
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
         cpu = cpu_baseline(w, args.cpu_seconds)

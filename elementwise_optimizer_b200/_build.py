@@ -31,7 +31,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libopt2s.so")
 TESTING_LIB = os.path.join(PKG, "libopt2s_testing.so")
 
-COMMON = ["opt2s_kernel.cu", "opt2s_kernel8.cu", "opt2s_noalloc.cu", "opt2s_api8.cpp"]
+COMMON = ["opt2s_kernel.cu", "opt2s_kernel8.cu", "opt2s_noalloc.cu", "opt2s_api8.cpp", "opt2s_ipc.cpp"]
 API = "opt2s_api.cpp"
 TESTING_ONLY = ["opt2s_testing.cu"]
 SOURCES = [os.path.join(CSRC, f) for f in COMMON + [API] + TESTING_ONLY]

@@ -92,6 +92,10 @@ BLOCK8 = 2048
 MIN_8BIT_SIZE = 4096
 
 
+class opt2s_ipc_handle(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_ubyte * 64)]
+
+
 class opt2s_testing_chunk(ctypes.Structure):
     _fields_ = [("tensor", ctypes.c_int64), ("start", ctypes.c_int64),
                 ("len", ctypes.c_int64), ("dtype", ctypes.c_int32),
@@ -127,6 +131,11 @@ EXPORTS = {
                                          ctypes.POINTER(ctypes.c_int64)]),
     "opt2s_shard_step": (ctypes.c_int, [ctypes.POINTER(opt2s_shard_desc), ctypes.POINTER(Hyper),
                                         ctypes.c_int, ctypes.c_void_p]),
+    "opt2s_ipc_export": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(opt2s_ipc_handle),
+                                        ctypes.POINTER(ctypes.c_int64)]),
+    "opt2s_ipc_open": (ctypes.c_int, [ctypes.POINTER(opt2s_ipc_handle), ctypes.c_int64,
+                                      ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_void_p)]),
+    "opt2s_ipc_close": (ctypes.c_int, [ctypes.c_void_p]),
     "opt2s_release_cache": (ctypes.c_int, []),
     "opt2s_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "opt2s_last_cuda_error": (ctypes.c_int, []),
@@ -464,6 +473,30 @@ def make_shard_desc(world: int, rank: int, numel: int, dtype: int, params, grads
 def opt2s_shard_step(desc: opt2s_shard_desc, hyper: Hyper, step: int, stream=None) -> None:
     check(lib().opt2s_shard_step(ctypes.byref(desc), ctypes.byref(hyper), int(step),
                                  _stream_handle(stream)), "opt2s_shard_step")
+
+
+def ipc_export(ptr) -> tuple:
+    """(handle bytes, offset) of the device allocation holding ``ptr`` (an
+    int address or a tensor), for another process's ipc_open."""
+    h = opt2s_ipc_handle()
+    off = ctypes.c_int64()
+    check(lib().opt2s_ipc_export(_ptr(ptr), ctypes.byref(h), ctypes.byref(off)), "opt2s_ipc_export")
+    return bytes(h.bytes), int(off.value)
+
+
+def ipc_open(handle: bytes, offset: int) -> tuple:
+    """Map another process's exported allocation: (base, address of its
+    buffer).  Unmap with ipc_close(base)."""
+    h = opt2s_ipc_handle()
+    ctypes.memmove(h.bytes, handle, 64)
+    base, ptr = ctypes.c_void_p(), ctypes.c_void_p()
+    check(lib().opt2s_ipc_open(ctypes.byref(h), int(offset), ctypes.byref(base), ctypes.byref(ptr)),
+          "opt2s_ipc_open")
+    return int(base.value), int(ptr.value)
+
+
+def ipc_close(base: int) -> None:
+    check(lib().opt2s_ipc_close(int(base)), "opt2s_ipc_close")
 
 
 def opt2s_release_cache() -> None:

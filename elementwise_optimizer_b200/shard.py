@@ -7,8 +7,10 @@ for the shard (rank order, fp32), updates it, and writes the new values into
 every rank's param buffer.  How the other ranks' buffers become addressable
 from this device is the caller's choice (CUDA IPC handles, symmetric memory,
 or peer access between devices driven by one process); the step only needs
-their addresses.  Order each step after all ranks' gradients are complete and
-before any rank reads its params again (a barrier on each side).
+their addresses.  ``PeerBuffers`` does it with CUDA IPC over a
+torch.distributed process group, one process per GPU.  Order each step after
+all ranks' gradients are complete and before any rank reads its params again
+(a barrier on each side).
 """
 from __future__ import annotations
 
@@ -21,6 +23,49 @@ def shard_range(numel: int, world: int, rank: int) -> tuple:
     """(start, length) of ``rank``'s shard; shards are disjoint, cover every
     element, differ in size by at most 8 and start at multiples of 8."""
     return B.opt2s_shard_range(numel, world, rank)
+
+
+class PeerBuffers:
+    """Every rank's flat param and grad buffers, addressable from this rank's
+    device: this rank's own tensors, and the other ranks' allocations mapped
+    through CUDA IPC (opt2s_ipc_export / opt2s_ipc_open; across GPUs the
+    mapping enables peer access, so the step's loads and stores cross
+    NVLink).  The handles travel with one all_gather_object over ``group``.
+    Call close() once no kernel uses the mappings any more."""
+
+    def __init__(self, param: torch.Tensor, grad: torch.Tensor, group=None):
+        import torch.distributed as dist
+        world = dist.get_world_size(group)
+        rank = dist.get_rank(group)
+        mine = (B.ipc_export(param), B.ipc_export(grad), param.numel(), str(param.dtype))
+        every = [None] * world
+        dist.all_gather_object(every, mine, group=group)
+        for q, (_, _, n, dt) in enumerate(every):
+            if n != param.numel() or dt != str(param.dtype):
+                raise ValueError(f"rank {q} holds {n} elements of {dt}; every rank must match")
+        self.params, self.grads = [], []
+        self._bases = []
+        opened = {}          # one mapping per exported allocation
+        for q, (ph, gh, _, _) in enumerate(every):
+            if q == rank:
+                self.params.append(param)
+                self.grads.append(grad)
+                continue
+            addr = []
+            for handle, offset in (ph, gh):
+                if handle not in opened:
+                    base, _ = B.ipc_open(handle, 0)
+                    opened[handle] = base
+                    self._bases.append(base)
+                addr.append(opened[handle] + offset)
+            self.params.append(addr[0])
+            self.grads.append(addr[1])
+        self._keep = (param, grad)
+
+    def close(self) -> None:
+        for base in self._bases:
+            B.ipc_close(base)
+        self._bases = []
 
 
 class ShardedStep:

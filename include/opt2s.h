@@ -215,6 +215,27 @@ typedef struct {
 
 int opt2s_shard_range(int64_t numel, int32_t world, int32_t rank, int64_t *start,
                       int64_t *len);
+
+/*
+ * Peer mappings for the sharded step between processes (one per GPU): CUDA
+ * IPC.  opt2s_ipc_export gives the handle of the device allocation that
+ * holds `ptr` and ptr's byte offset inside it; another process passes both to
+ * opt2s_ipc_open, which maps the allocation (enabling peer access on first
+ * use when it lives on another GPU of the node) and returns its base and the
+ * mapped address of the exporter's `ptr`.  opt2s_ipc_close(base) unmaps it
+ * (only after every kernel that uses the mapping has finished).  A handle
+ * is 64 opaque bytes; it is valid while the exporting allocation lives.
+ * Errors: OPT2S_ERR_INVALID_ARG for null arguments, OPT2S_ERR_CUDA (with
+ * opt2s_last_cuda_error) when the driver refuses, e.g. for an address that is
+ * not device memory or a handle opened in the process that exported it.
+ */
+typedef struct {
+    unsigned char bytes[64];
+} opt2s_ipc_handle;
+
+int opt2s_ipc_export(const void *ptr, opt2s_ipc_handle *handle, int64_t *offset);
+int opt2s_ipc_open(const opt2s_ipc_handle *handle, int64_t offset, void **base, void **ptr);
+int opt2s_ipc_close(void *base);
 int opt2s_shard_step(const opt2s_shard_desc *desc, const Hyper *hyper, int step,
                      cudaStream_t stream);
 
