@@ -29,6 +29,13 @@ weight_decay * param, scaled by the trust ratio ||param|| / ||direction||.
 Like max_unorm it takes four launches per group and step, keeps one record
 per parameter under flatten=True, and is not combined with capturable=True.
 
+Without flatten, each group's launch records (the tensors' addresses) are
+built once and reused while the group holds the same parameter and gradient
+tensor objects, checked by identity each step; zero_grad() therefore zeroes
+gradients in place by default (set_to_none=False), so that they stay the
+same tensors.  Reassigning a tensor's storage in place (``p.data = x``,
+``.set_()``) keeps the object and is not seen: call refresh() after it.
+
 capturable=True routes every step through opt2s_plan_step_table: the per-step
 scalars live in a device table and the step index in device memory, so
 ``step()`` may be captured in a CUDA graph and each replay performs the next
@@ -37,6 +44,8 @@ and call ``refill_step_table()`` between replays at least once every
 ``table_len`` steps (``steps_left()`` tells how many remain).
 """
 from __future__ import annotations
+
+import operator
 
 import torch
 
@@ -124,11 +133,38 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                     entry["plan"] = B.Plan(tl, self.algo)
                 self._flat.append(entry)
 
-    def zero_grad(self, set_to_none: bool = True):
+    def zero_grad(self, set_to_none: bool = False):
+        """Zero the gradients in place (one launch per device and dtype), so
+        that the cached launch records stay valid; set_to_none=True drops
+        them as torch.optim does (the next step then rebuilds the records)."""
         if self._flat is None:
-            return super().zero_grad(set_to_none)
+            if set_to_none:
+                return super().zero_grad(True)
+            grads = [p.grad for g in self.param_groups for p in g["params"] if p.grad is not None]
+            if grads:
+                torch._foreach_zero_(grads)
+            return None
         for f in self._flat:           # keep the views: gradients accumulate into them
             f["grad"].zero_()
+
+    def refresh(self) -> None:
+        """Forget the cached launch records (after ``p.data = x`` or another
+        in-place change of a tensor's storage)."""
+        self._sync_steps()
+        self._group_cache = {}
+
+    def _sync_steps(self) -> None:
+        for data in self._group_cache.values():
+            for st in data["states"]:
+                st["step"] = data["step"]
+
+    def state_dict(self):
+        self._sync_steps()
+        return super().state_dict()
+
+    def load_state_dict(self, state_dict) -> None:
+        super().load_state_dict(state_dict)
+        self._group_cache = {}
 
     # ---- per-group launch data ------------------------------------------
     def _hyper(self, group):
@@ -148,12 +184,24 @@ class TwoStateOptimizer(torch.optim.Optimizer):
         return st
 
     def _launch_data(self, gi, group):
+        params = group["params"]
+        grads = [p.grad for p in params]
+        cached = self._group_cache.get(gi)
+        if (cached is not None and len(params) == len(cached["all_params"])
+                and all(map(operator.is_, grads, cached["all_grads"]))
+                and all(map(operator.is_, params, cached["all_params"]))):
+            return cached      # the same tensors as last step: reuse the records
+        data = self._build_launch_data(gi, group, cached)
+        data["all_params"] = list(params)
+        data["all_grads"] = grads
+        return data
+
+    def _build_launch_data(self, gi, group, cached):
         ps = [p for p in group["params"] if p.grad is not None]
         for p in ps:
             if not p.is_cuda or not p.is_contiguous() or not p.grad.is_contiguous():
                 raise ValueError("parameters and gradients must be contiguous CUDA tensors")
         key = tuple((p.data_ptr(), p.grad.data_ptr(), p.numel()) for p in ps)
-        cached = self._group_cache.get(gi)
         if cached is not None and cached["key"] == key:
             return cached
         states = [self._state_of(p) for p in ps]
@@ -162,6 +210,8 @@ class TwoStateOptimizer(torch.optim.Optimizer):
         data = {"key": key, "params": ps, "tl": tl, "states": states, "step": 0}
         if cached is not None:
             data["step"] = cached["step"]
+            for st in cached["states"]:      # parameters that leave the group keep their count
+                st["step"] = cached["step"]
         elif states:
             data["step"] = states[0]["step"]
         if self.capturable:
@@ -213,9 +263,7 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                                        data["step"] + 1)
             else:
                 B.opt2s_step(data["tl"], self._hyper(group), data["step"] + 1)
-            data["step"] += 1
-            for s in data["states"]:
-                s["step"] = data["step"]
+            data["step"] += 1          # per-parameter counts are written by _sync_steps
         return loss
 
     def refill_step_table(self, next_step: int | None = None) -> None:
