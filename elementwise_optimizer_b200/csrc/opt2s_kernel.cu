@@ -277,46 +277,23 @@ __global__ void advance_index_kernel(int* index, int table_len)
 // chunk length, the block width or the storage alignment.  Accesses are
 // element-wise and contiguous across the warp.
 //
-// Each lane accumulates its 64 squares of a block as a double-float: an
-// unevaluated sum hi + lo of two binary32 numbers.  The square of a binary32
-// x is exactly sq + err with sq = RN(x*x) and err = fma(x, x, -sq) (exact for
-// 2^-50 <= |x| <= 2^56: no underflow of err, and 64 squares stay below
-// 2^128), and hi + sq is split exactly into s + e by Knuth's TwoSum (Knuth,
-// TAOCP vol. 2, 4.2.2, Theorem B); only lo + (e + err) is rounded, which
-// errs by at most 2^-48 of the running sum.  Elements outside that range
-// are added to a binary64 sum instead.  The lane's total is hi + lo + that
-// sum in binary64, so the block's sum errs by at most about 2^-42 of itself,
-// far below the fp32 rounding of the scale.  All of it stays on the fp32
-// pipe: no float-to-double conversion per element.
+// Each lane adds its squares in binary64: the square of a binary32 x is exact
+// in binary64, so one fused multiply-add gives the same sum as a multiply and
+// an add.  (A double-float lane sum -- two binary32 numbers, TwoProduct and
+// TwoSum on the fp32 pipe -- avoids the float-to-double conversions but
+// measured slower on B200: more instructions per element.)  The partials
+// kernel is limited to 64 registers per thread, 4 CTAs of 256 threads per
+// SM: the extra resident warps hide more of the load latency, and measured
+// faster than 3 CTAs at 80 registers.
 // ---------------------------------------------------------------------------
-constexpr float kSquareLo = 0x1p-50f;   // |x| range whose square splits exactly
-constexpr float kSquareHi = 0x1p56f;
-
 struct SquareSum {
-    float hi = 0.0f, lo = 0.0f;
-    double wide = 0.0;   // squares of out-of-range values
-
+    double s = 0.0;
     __device__ __forceinline__ void add(float x)
     {
-        const float ax = fabsf(x);
-        if (ax >= kSquareLo && ax <= kSquareHi) {
-            const float sq = __fmul_rn(x, x);
-            const float err = __fmaf_rn(x, x, -sq);
-            const float s = __fadd_rn(hi, sq);
-            const float bp = __fsub_rn(s, hi);
-            const float e = __fadd_rn(__fsub_rn(hi, __fsub_rn(s, bp)), __fsub_rn(sq, bp));
-            hi = s;
-            lo = __fadd_rn(lo, __fadd_rn(e, err));
-        } else if (x != 0.0f) {
-            const double xd = static_cast<double>(x);
-            wide = __fma_rn(xd, xd, wide);
-        }
+        const double xd = static_cast<double>(x);
+        s = __fma_rn(xd, xd, s);
     }
-
-    __device__ __forceinline__ double total() const
-    {
-        return __dadd_rn(__dadd_rn(static_cast<double>(hi), static_cast<double>(lo)), wide);
-    }
+    __device__ __forceinline__ double total() const { return s; }
 };
 
 template <int DT, int ALGO, bool SKIP, int MODE>
@@ -365,8 +342,10 @@ __device__ __forceinline__ void warp_tree_sum(double& a, double& b)
     }
 }
 
+constexpr int kNormThreads = 256;
+
 template <int ALGO, bool SKIP, int MODE>
-__global__ void unorm_partials_kernel(const ChunkRec* __restrict__ blocks, int nblocks,
+__global__ void __launch_bounds__(kNormThreads, 4) unorm_partials_kernel(const ChunkRec* __restrict__ blocks, int nblocks,
                                       StepScalars s, float wd, double2* __restrict__ partial)
 {
     const int lane = threadIdx.x & 31;
@@ -703,7 +682,6 @@ cudaError_t launch_unorm_typed(const ChunkRec* d_chunks, int64_t nchunks, const 
                                const UnormArgs& u, float max_unorm, float wd, int block_threads,
                                int max_blocks, cudaStream_t stream)
 {
-    constexpr int kNormThreads = 256;
     int grid = 0;
     cudaError_t e = cudaSuccess;
     if (u.nblocks > 0) {

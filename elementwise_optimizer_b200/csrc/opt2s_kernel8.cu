@@ -19,21 +19,40 @@
 // (with both signs for the signed map), plus 0 and 1.0.  Each value is
 // N/D with N = 2^(F+1) + 9*(2f+1) and D = 10^(E+1)*2^(F+1), exact binary32
 // integers, so one IEEE division gives it rounded once.  Every CTA builds the
-// two maps in shared memory at start, and the thresholds between neighbours:
-// T_j = the binary32 number at or below the exact midpoint of map[j] and
-// map[j+1] (binary64 holds the midpoint exactly).  For a binary32 x,
-// x > T_j exactly when x lies above that midpoint, so the number of
-// thresholds below x is the code of the nearest map value, an exact tie going
-// to the lower code.  A binary search over the 255 thresholds finds it.
+// two maps in shared memory at start.
 //
-// Per 8-bit block (one CTA of 256 threads, 8 consecutive elements a thread):
+// Quantization: the code of x = RN32(m / absmax) is the map value nearest to
+// x, an exact tie going to the lower code.  With T_j the binary32 number at
+// or below the exact midpoint of map[j] and map[j+1] (binary64 holds the
+// midpoint exactly), x > T_j exactly when x lies above that midpoint, so the
+// code is the number of thresholds below x.  Rather than search the 255
+// thresholds, each CTA tabulates them over the bits of x: |x| in [2^-23, 1]
+// falls in one of 24 binades x 128 slices (the exponent and the top 7
+// fraction bits); every slice is narrower than the gap between two
+// thresholds (the finest gap, 0.9/128 at the top of the unsigned map, is
+// above the widest slice, 2^-8), so a slice holds at most one threshold, and
+// its entry gives the code at the slice's bottom and that threshold: code =
+// base + (|x| > T).  Below 2^-23 the nearest value is 0 in both maps (their
+// first thresholds are 2.75e-7 and 1.6e-7).  The signed map is symmetric but
+// for its top value 1.0, so negative x use the positive table: the mirror of
+// code c is 254 - c (0 at least), one lower again when |x| is exactly a
+// midpoint (the tie then goes to the lower, more negative, code).
+// x itself is RN32(RN64(m * RN64(1/absmax))): for every quotient in the
+// binary32 normal range that is RN32(m/absmax) exactly (the binary64 product
+// errs by less than 2^-52, while a quotient that is not representable never
+// lies within 2^-49 of a binary32 rounding boundary; see div_by_constant in
+// opt2s_device.cuh), and below it both give the code of 0.
+//
+// Per 8-bit block (one CTA of 256 threads, 8 elements a thread; fp32 storage
+// takes elements 4t..4t+3 and 1024+4t..1024+4t+3, 16-bit storage 8t..8t+7, so
+// that every warp access is contiguous):
 //   1. dequantize: m = map_s[code]*absmax (fp32 product), v with map_u;
 //   2. the plain step's element update (opt2s_device.cuh), param stored;
 //   3. the block's new absmax of |m|, v (, |m2|): fmaxf over the thread's
 //      elements, the warp and the CTA's 8 warps (max is exact, so the order
 //      does not matter; NaNs are ignored);
-//   4. quantize: code of m/absmax (IEEE fp32 division), or the code of 0
-//      when the absmax is 0; thread 0 stores the new absmaxes.
+//   4. quantize each value with the block's new absmax, or store the code of
+//      0 when it is 0; thread 0 stores the new absmaxes.
 // With skip_zeros an element whose gradient is zero keeps its param and its
 // dequantized state, which is requantized with the block's new absmax.
 // Warps of a CTA walk the 32-bit chunks of small tensors exactly as the plain
@@ -50,11 +69,23 @@ constexpr int kB8Threads = 256;                  // one CTA per 8-bit block
 constexpr int kB8PerThread = kBlock8Elems / kB8Threads;
 static_assert(kB8PerThread == 8, "eight elements a thread");
 
-struct Maps {
-    float smap[256], umap[256];   // signed (m, m2) and unsigned (v) maps
-    float sthr[256], uthr[256];   // thresholds between neighbours (255 used)
-    float red[2][3][kB8Threads / 32];   // per-warp maxima, double-buffered
+constexpr int kSlices = 24 * 128;        // binades 2^-23 .. 2^0, 128 slices each
+constexpr uint32_t kZeroSigned = 127;   // code of 0 in the signed map
+constexpr uint32_t kZeroUnsigned = 0;   // and in the unsigned one
+
+// A slice of |x|: the code at its bottom, its threshold (+Inf if none) and
+// whether that threshold is an exact midpoint (bit 8 of `code`).
+struct QSlice {
+    float thr;
+    uint32_t code;
 };
+
+struct Maps {
+    float smap[256], umap[256];          // signed (m, m2) and unsigned (v) maps
+    QSlice stab[kSlices], utab[kSlices];  // quantization slices, |x| for the signed map
+    float red[2][3][kB8Threads / 32];    // per-warp maxima, double-buffered
+};
+constexpr size_t kMapsBytes = sizeof(Maps);
 
 // Value of map entry k before sorting: the k-th (value, sign) of the
 // construction above, in the order of E, f (and sign); k = 254 is 0 and
@@ -80,47 +111,95 @@ __device__ float map_value(bool is_signed, int k)
     return k == at ? 0.0f : 1.0f;
 }
 
-// Builds both maps and their thresholds in shared memory (all threads of the
-// CTA take part; ends with a barrier).  Sorting: the rank of a value is the
-// number of values below it (all 256 are distinct).
+// The threshold between map[j] and map[j + 1] (the binary32 number at or
+// below their exact midpoint) and whether the midpoint is exact.
+__device__ __forceinline__ float threshold(const float* map, int j, bool* exact)
+{
+    const double mid = __dmul_rn(__dadd_rn(static_cast<double>(map[j]), static_cast<double>(map[j + 1])), 0.5);
+    const float t = __double2float_rd(mid);
+    *exact = static_cast<double>(t) == mid;
+    return t;
+}
+
+// Number of thresholds of `map` at or below... strictly below `lo`, by a
+// binary search over the 255 thresholds (table building only).
+__device__ int codes_below(const float* map, float lo)
+{
+    int c = 0;
+    bool ex;
+    for (int step = 128; step >= 1; step >>= 1)
+        if (c + step - 1 < 255 && threshold(map, c + step - 1, &ex) < lo) c += step;
+    return c;
+}
+
+// Slice s of |x| for `map` (x >= 0): bottom code and its single threshold.
+__device__ QSlice make_slice(const float* map, int s)
+{
+    const int e = s >> 7, k = s & 127;
+    const uint32_t lo_bits = static_cast<uint32_t>(e + 127 - 23) << 23 | static_cast<uint32_t>(k) << 16;
+    const uint32_t hi_bits = lo_bits + (1u << 16);
+    const float lo = __uint_as_float(lo_bits), hi = __uint_as_float(hi_bits);
+    const int c = codes_below(map, lo);
+    QSlice q;
+    q.code = static_cast<uint32_t>(c);
+    q.thr = __int_as_float(0x7f800000);   // +Inf: no threshold in the slice
+    if (c < 255) {
+        bool exact = false;
+        const float t = threshold(map, c, &exact);
+        if (t < hi) {
+            q.thr = t;
+            q.code |= exact ? 0x100u : 0u;
+        }
+    }
+    return q;
+}
+
+// Builds both maps and their slice tables in shared memory (all threads of
+// the CTA take part; ends with a barrier).  Sorting: the rank of a value is
+// the number of values below it (all 256 are distinct).
 __device__ void build_maps(Maps& mp)
 {
     const int t = threadIdx.x;
     const float sv = map_value(true, t);
     const float uv = map_value(false, t);
-    mp.sthr[t] = sv;             // unsorted values, for the ranking
-    mp.uthr[t] = uv;
+    float* scratch = reinterpret_cast<float*>(mp.stab);   // unsorted values, for the ranking
+    scratch[t] = sv;
+    scratch[256 + t] = uv;
     __syncthreads();
     int rs = 0, ru = 0;
     for (int j = 0; j < 256; ++j) {
-        rs += mp.sthr[j] < sv;
-        ru += mp.uthr[j] < uv;
+        rs += scratch[j] < sv;
+        ru += scratch[256 + j] < uv;
     }
+    __syncthreads();
     mp.smap[rs] = sv;
     mp.umap[ru] = uv;
     __syncthreads();
-    if (t < 255) {
-        mp.sthr[t] = __double2float_rd(__dmul_rn(__dadd_rn(static_cast<double>(mp.smap[t]),
-                                                           static_cast<double>(mp.smap[t + 1])), 0.5));
-        mp.uthr[t] = __double2float_rd(__dmul_rn(__dadd_rn(static_cast<double>(mp.umap[t]),
-                                                           static_cast<double>(mp.umap[t + 1])), 0.5));
+    for (int s = t; s < kSlices; s += kB8Threads) {
+        mp.stab[s] = make_slice(mp.smap, s);
+        mp.utab[s] = make_slice(mp.umap, s);
     }
     __syncthreads();
 }
 
-// Code of the nearest map value: the number of thresholds below x.
-__device__ __forceinline__ uint32_t code_of(const float* thr, float x)
+// Code of the map value nearest to m/absmax (inv = RN64(1/absmax); absmax
+// > 0): the slice of |x| gives it, mirrored for negative x in the signed map.
+template <bool SIGNED>
+__device__ __forceinline__ uint32_t quantize(const QSlice* tab, float m, double inv)
 {
-    uint32_t c = 0;
-#pragma unroll
-    for (uint32_t step = 128; step >= 1; step >>= 1)
-        if (x > thr[c + step - 1]) c += step;
+    const float x = __double2float_rn(__dmul_rn(static_cast<double>(m), inv));
+    const uint32_t b = __float_as_uint(x);
+    const int e = static_cast<int>((b >> 23) & 0xFFu) - (127 - 23);
+    if (e < 0) return SIGNED ? kZeroSigned : kZeroUnsigned;   // |x| < 2^-23
+    if (e > 23) return 0u;                                     // NaN (|x| <= 1 otherwise)
+    const QSlice q = tab[(e << 7) | ((b >> 16) & 0x7Fu)];
+    const float a = fabsf(x);
+    uint32_t c = (q.code & 0xFFu) + (a > q.thr ? 1u : 0u);
+    if (SIGNED && (b >> 31)) {
+        const int k = 254 - static_cast<int>(c) - ((a == q.thr && (q.code & 0x100u)) ? 1 : 0);
+        c = k < 0 ? 0u : static_cast<uint32_t>(k);
+    }
     return c;
-}
-
-__device__ __forceinline__ uint32_t quantize(const float* thr, float x, float amax, uint32_t zero)
-{
-    return amax > 0.0f ? code_of(thr, __fdiv_rn(x, amax)) : zero;
 }
 
 __device__ __forceinline__ float warp_max(float x)
@@ -130,35 +209,66 @@ __device__ __forceinline__ float warp_max(float x)
     return x;
 }
 
-// Eight codes of a thread: one 8-byte access when `vec`, else byte by byte.
-__device__ __forceinline__ void load_codes(const uint8_t* q, uint32_t i, uint32_t len, bool vec,
+// Element j of run u of this thread (runs of V elements, one storage vector
+// each): fp32 (V = 4) takes 4t..4t+3 and 1024+4t..1024+4t+3, 16-bit (V = 8)
+// 8t..8t+7, so that each warp access is contiguous.
+template <int V>
+__device__ __forceinline__ uint32_t elem(int u, int j)
+{
+    return static_cast<uint32_t>(u * (kBlock8Elems * V / 8) + threadIdx.x * V + j);
+}
+
+// A thread's eight codes: one V-byte access per run when `vec`, else byte by
+// byte (0 past the end of the block).
+template <int V>
+__device__ __forceinline__ void load_codes(const uint8_t* q, uint32_t len, bool vec,
                                            uint32_t (&c)[kB8PerThread])
 {
-    if (vec) {
-        const uint2 w = *reinterpret_cast<const uint2*>(q + i);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            c[k] = (w.x >> (8 * k)) & 0xFFu;
-            c[4 + k] = (w.y >> (8 * k)) & 0xFFu;
+    for (int u = 0; u < 8 / V; ++u) {
+        const uint32_t e = elem<V>(u, 0);
+        if (vec) {
+            if (V == 8) {
+                const uint2 w = *reinterpret_cast<const uint2*>(q + e);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    c[k] = (w.x >> (8 * k)) & 0xFFu;
+                    c[4 + k] = (w.y >> (8 * k)) & 0xFFu;
+                }
+            } else {
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(q + e);
+#pragma unroll
+                for (int k = 0; k < V; ++k) c[u * V + k] = (w >> (8 * k)) & 0xFFu;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < V; ++k) c[u * V + k] = e + k < len ? q[e + k] : 0u;
         }
-    } else {
-#pragma unroll
-        for (int k = 0; k < kB8PerThread; ++k) c[k] = i + k < len ? q[i + k] : 0u;
     }
 }
 
-__device__ __forceinline__ void store_codes(uint8_t* q, uint32_t i, uint32_t len, bool vec,
+template <int V>
+__device__ __forceinline__ void store_codes(uint8_t* q, uint32_t len, bool vec,
                                             const uint32_t (&c)[kB8PerThread])
 {
-    if (vec) {
-        uint2 w;
-        w.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-        w.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-        *reinterpret_cast<uint2*>(q + i) = w;
-    } else {
 #pragma unroll
-        for (int k = 0; k < kB8PerThread; ++k)
-            if (i + k < len) q[i + k] = static_cast<uint8_t>(c[k]);
+    for (int u = 0; u < 8 / V; ++u) {
+        const uint32_t e = elem<V>(u, 0);
+        if (vec) {
+            if (V == 8) {
+                uint2 w;
+                w.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+                w.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+                *reinterpret_cast<uint2*>(q + e) = w;
+            } else {
+                *reinterpret_cast<uint32_t*>(q + e) = c[u * V] | (c[u * V + 1] << 8) |
+                                                      (c[u * V + 2] << 16) | (c[u * V + 3] << 24);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < V; ++k)
+                if (e + k < len) q[e + k] = static_cast<uint8_t>(c[u * V + k]);
+        }
     }
 }
 
@@ -175,30 +285,30 @@ __device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int b
 {
     using P = Param<DT>;
     constexpr int V = P::kVec;
+    constexpr int R = 8 / V;   // runs a thread
     const uint32_t len = b.len;
-    const uint32_t i0 = threadIdx.x * kB8PerThread;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // full, aligned blocks move 8 elements a thread in 16-byte (param, grad)
-    // and 8-byte (codes) accesses; others go element by element
+    // full, aligned blocks move a run in one 16-byte (param, grad) and one
+    // V-byte (codes) access; others go element by element
     const bool vec = len == static_cast<uint32_t>(kBlock8Elems) && al(b.p, 16) && al(b.g, 16) &&
-                     al(b.q1, 8) && al(b.q2, 8) && (ALGO != kAdEMAMix || al(b.q3, 8));
+                     al(b.q1, V) && al(b.q2, V) && (ALGO != kAdEMAMix || al(b.q3, V));
 
     const float a1 = b.a1[0], a2 = b.a2[0];
     const float a3 = ALGO == kAdEMAMix ? b.a3[0] : 0.0f;
     uint32_t c1[kB8PerThread], c2[kB8PerThread], c3[kB8PerThread];
-    load_codes(b.q1, i0, len, vec, c1);
-    load_codes(b.q2, i0, len, vec, c2);
-    if (ALGO == kAdEMAMix) load_codes(b.q3, i0, len, vec, c3);
+    load_codes<V>(b.q1, len, vec, c1);
+    load_codes<V>(b.q2, len, vec, c2);
+    if (ALGO == kAdEMAMix) load_codes<V>(b.q3, len, vec, c3);
     float g[kB8PerThread], p[kB8PerThread];
-    typename P::Raw praw[8 / V], graw[8 / V];
+    typename P::Raw praw[R], graw[R];
     if (vec) {
 #pragma unroll
-        for (int u = 0; u < 8 / V; ++u) {
-            graw[u] = P::load(b.g, i0 + u * V);
-            praw[u] = P::load(b.p, i0 + u * V);
+        for (int u = 0; u < R; ++u) {
+            graw[u] = P::load(b.g, elem<V>(u, 0));
+            praw[u] = P::load(b.p, elem<V>(u, 0));
         }
 #pragma unroll
-        for (int u = 0; u < 8 / V; ++u) {
+        for (int u = 0; u < R; ++u) {
             float x[V], y[V];
             P::widen(graw[u], x);
             P::widen(praw[u], y);
@@ -207,11 +317,13 @@ __device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int b
         }
     } else {
 #pragma unroll
-        for (int k = 0; k < kB8PerThread; ++k) {
-            const bool in = i0 + k < len;
-            g[k] = in ? P::load1(b.g, i0 + k) : 0.0f;
-            p[k] = in ? P::load1(b.p, i0 + k) : 0.0f;
-        }
+        for (int u = 0; u < R; ++u)
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                const uint32_t e = elem<V>(u, j);
+                g[u * V + j] = e < len ? P::load1(b.g, e) : 0.0f;
+                p[u * V + j] = e < len ? P::load1(b.p, e) : 0.0f;
+            }
     }
 
     float m[kB8PerThread], v[kB8PerThread], m2[kB8PerThread];
@@ -221,7 +333,7 @@ __device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int b
         m[k] = __fmul_rn(mp.smap[c1[k]], a1);
         v[k] = __fmul_rn(mp.umap[c2[k]], a2);
         m2[k] = ALGO == kAdEMAMix ? __fmul_rn(mp.smap[c3[k]], a3) : 0.0f;
-        if (i0 + k < len) {
+        if (elem<V>(k / V, k % V) < len) {
             update<ALGO, SKIP>(g[k], p[k], m[k], v[k], m2[k], s);
             x1 = fmaxf(x1, fabsf(m[k]));
             x2 = fmaxf(x2, fabsf(v[k]));
@@ -230,16 +342,20 @@ __device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int b
     }
     if (vec) {
 #pragma unroll
-        for (int u = 0; u < 8 / V; ++u) {
+        for (int u = 0; u < R; ++u) {
             float y[V], gg[V];
 #pragma unroll
             for (int j = 0; j < V; ++j) { y[j] = p[u * V + j]; gg[j] = g[u * V + j]; }
-            P::store(b.p, i0 + u * V, P::narrow(y, praw[u], gg, SKIP));
+            P::store(b.p, elem<V>(u, 0), P::narrow(y, praw[u], gg, SKIP));
         }
     } else {
 #pragma unroll
-        for (int k = 0; k < kB8PerThread; ++k)
-            if (i0 + k < len && !(SKIP && g[k] == 0.0f)) P::store1(b.p, i0 + k, p[k]);
+        for (int u = 0; u < R; ++u)
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                const uint32_t e = elem<V>(u, j);
+                if (e < len && !(SKIP && g[u * V + j] == 0.0f)) P::store1(b.p, e, p[u * V + j]);
+            }
     }
 
     // the block's new absmaxes
@@ -265,25 +381,31 @@ __device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int b
         b.a2[0] = n2;
         if (ALGO == kAdEMAMix) b.a3[0] = n3;
     }
+    // correctly rounded binary64 reciprocals of the new absmaxes
+    const double i1 = n1 > 0.0f ? __drcp_rn(static_cast<double>(n1)) : 0.0;
+    const double i2 = n2 > 0.0f ? __drcp_rn(static_cast<double>(n2)) : 0.0;
+    const double i3 = (ALGO == kAdEMAMix && n3 > 0.0f) ? __drcp_rn(static_cast<double>(n3)) : 0.0;
 #pragma unroll
     for (int k = 0; k < kB8PerThread; ++k) {
-        c1[k] = quantize(mp.sthr, m[k], n1, 127u);
-        c2[k] = quantize(mp.uthr, v[k], n2, 0u);
-        if (ALGO == kAdEMAMix) c3[k] = quantize(mp.sthr, m2[k], n3, 127u);
+        c1[k] = n1 > 0.0f ? quantize<true>(mp.stab, m[k], i1) : kZeroSigned;
+        c2[k] = n2 > 0.0f ? quantize<false>(mp.utab, v[k], i2) : kZeroUnsigned;
+        if (ALGO == kAdEMAMix) c3[k] = n3 > 0.0f ? quantize<true>(mp.stab, m2[k], i3) : kZeroSigned;
     }
-    store_codes(b.q1, i0, len, vec, c1);
-    store_codes(b.q2, i0, len, vec, c2);
-    if (ALGO == kAdEMAMix) store_codes(b.q3, i0, len, vec, c3);
+    store_codes<V>(b.q1, len, vec, c1);
+    store_codes<V>(b.q2, len, vec, c2);
+    if (ALGO == kAdEMAMix) store_codes<V>(b.q3, len, vec, c3);
 }
 
 // Work unit u < nblocks: 8-bit block u, by the whole CTA.  Otherwise unit u
 // holds the 32-bit chunks 8(u - nblocks) .. 8(u - nblocks) + 7, one a warp.
+// The maps and slice tables live in dynamic shared memory (kMapsBytes).
 template <int ALGO, bool SKIP>
 __global__ void __launch_bounds__(kB8Threads)
 step8_kernel(const Block8Rec* __restrict__ blocks, int nblocks, const ChunkRec* __restrict__ chunks,
              int nchunks, StepScalars s)
 {
-    __shared__ Maps mp;
+    extern __shared__ __align__(16) unsigned char smem8[];
+    Maps& mp = *reinterpret_cast<Maps*>(smem8);
     build_maps(mp);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int units = nblocks + (nchunks + kB8Threads / 32 - 1) / (kB8Threads / 32);
@@ -320,7 +442,7 @@ Kernel8Fn pick8(int algo, int skip)
 }
 
 constexpr int kMaxDevices8 = 64;
-int g_occ8[kMaxDevices8][4];   // resident CTAs per SM, per device and kernel
+int g_occ8[kMaxDevices8][4];   // resident CTAs per SM, per device and kernel (0: not set up)
 int g_sms8[kMaxDevices8];
 std::mutex g_occ8_mu;
 
@@ -333,32 +455,37 @@ cudaError_t launch_step8(const Block8Rec* d_blocks, int64_t nblocks, const Chunk
     const int64_t units = nblocks + (nchunks + kB8Threads / 32 - 1) / (kB8Threads / 32);
     if (units <= 0) return cudaSuccess;
     Kernel8Fn fn = pick8(algo, skip_zeros);
-    int cap = max_blocks;
-    if (cap <= 0) {
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e != cudaSuccess) return e;
-        if (dev < 0 || dev >= kMaxDevices8) return cudaErrorInvalidDevice;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices8) return cudaErrorInvalidDevice;
+    int cap = 0;
+    {
         std::lock_guard<std::mutex> lock(g_occ8_mu);
         const int k = (algo == kAdEMAMix ? 2 : 0) + (skip_zeros ? 1 : 0);
         if (g_occ8[dev][k] == 0) {
+            // the tables take more than the default 48 KB of shared memory
             int per_sm = 0, sms = 0;
-            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(kMapsBytes));
+            if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
             if (e == cudaSuccess)
-                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kB8Threads, 0);
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kB8Threads, kMapsBytes);
             if (e != cudaSuccess) return e;
             g_sms8[dev] = sms;
             g_occ8[dev][k] = per_sm < 1 ? 1 : per_sm;
         }
         cap = g_occ8[dev][k] * g_sms8[dev];
     }
+    if (max_blocks > 0) cap = max_blocks;
     const int grid = static_cast<int>(units < cap ? units : cap);
     StepScalars sc = s;
     fill_reciprocals(&sc);
     int nb = static_cast<int>(nblocks), nc = static_cast<int>(nchunks);
     void* args[] = {const_cast<Block8Rec**>(&d_blocks), &nb, const_cast<ChunkRec**>(&d_chunks), &nc, &sc};
-    return cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3(grid), dim3(kB8Threads), args, 0,
-                            stream);
+    return cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3(grid), dim3(kB8Threads), args,
+                            kMapsBytes, stream);
 }
 
 }  // namespace opt2s

@@ -150,17 +150,10 @@ class TwoStateOptimizer(torch.optim.Optimizer):
     def refresh(self) -> None:
         """Forget the cached launch records (after ``p.data = x`` or another
         in-place change of a tensor's storage)."""
-        self._sync_steps()
-        self._group_cache = {}
-
-    def _sync_steps(self) -> None:
         for data in self._group_cache.values():
             for st in data["states"]:
                 st["step"] = data["step"]
-
-    def state_dict(self):
-        self._sync_steps()
-        return super().state_dict()
+        self._group_cache = {}
 
     def load_state_dict(self, state_dict) -> None:
         super().load_state_dict(state_dict)
@@ -210,10 +203,17 @@ class TwoStateOptimizer(torch.optim.Optimizer):
         data = {"key": key, "params": ps, "tl": tl, "states": states, "step": 0}
         if cached is not None:
             data["step"] = cached["step"]
-            for st in cached["states"]:      # parameters that leave the group keep their count
-                st["step"] = cached["step"]
-        elif states:
-            data["step"] = states[0]["step"]
+            data["counter"] = cached["counter"]
+            current = {id(st) for st in states}
+            for st in cached["states"]:      # a parameter that leaves the group keeps its count
+                if id(st) not in current:
+                    st["step"] = cached["step"]
+        else:
+            data["step"] = int(states[0]["step"]) if states else 0
+            data["counter"] = torch.tensor(data["step"], dtype=torch.int64)
+        # every stepped parameter's state["step"] is the group's shared counter
+        for st in states:
+            st["step"] = data["counter"]
         if self.capturable:
             data["plan"] = B.Plan(tl, self.algo)
             dev = ps[0].device if ps else torch.device("cuda")
@@ -263,7 +263,8 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                                        data["step"] + 1)
             else:
                 B.opt2s_step(data["tl"], self._hyper(group), data["step"] + 1)
-            data["step"] += 1          # per-parameter counts are written by _sync_steps
+            data["step"] += 1
+            data["counter"].fill_(data["step"])   # the parameters' shared step count
         return loss
 
     def refill_step_table(self, next_step: int | None = None) -> None:
@@ -277,6 +278,7 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                 continue
             if next_step is not None:
                 data["step"] = next_step - 1
+                data["counter"].fill_(data["step"])
             self._refill(data, group)
 
     def steps_left(self) -> int:

@@ -2,11 +2,11 @@
 
 Per tensor, the oracle's oracle_step_f32_lamb takes the weight norm and the
 norm of the decayed direction w = u + weight_decay*p as plain binary64 sums
-in index order; the CUDA path sums in a fixed tree (double-float lane sums,
-binary64 above them).  The trust ratio is rounded to fp32, so the two agree
-bit for bit unless a ratio falls within about 2^-40 of an fp32 rounding
-boundary (never on these inputs): every case asserts 0 ulp on param, state1
-and state2, and untouched gradients.
+in index order; the CUDA path sums in a fixed tree of binary64 sums.  The
+trust ratio is rounded to fp32, so the two agree bit for bit unless a ratio
+falls within a few binary64 ulp of an fp32 rounding boundary (never on these
+inputs): every case asserts 0 ulp on param, state1 and state2, and untouched
+gradients.
 """
 import numpy as np
 import pytest
