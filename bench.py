@@ -140,7 +140,7 @@ class ClockSampler:
 # Our arm
 # ---------------------------------------------------------------------------
 
-KERNEL_SOURCES = ("opt2s_kernel.cu", "opt2s_internal.h", "opt2s_api.cpp")
+KERNEL_SOURCES = ("opt2s_kernel.cu", "opt2s_device.cuh", "opt2s_internal.h", "opt2s_api.cpp")
 
 
 def strip_c_comments(text):
@@ -203,14 +203,19 @@ def environment():
     return env
 
 
-def traffic_for(kernel_key, path=None):
-    """ncu DRAM bytes per launch, if the committed capture is of the kernel
-    sources as they are now (else None)."""
+def traffic_for(kernel_key, numel, path=None):
+    """ncu DRAM bytes (read + written) per launch of `numel` elements, if the
+    committed capture is of the kernel sources as they are now (else None).
+    The capture is of a small case of the same kernel (16,777,216 elements,
+    larger than L2, a few hundred MB on the device); the step moves a fixed
+    number of bytes per element, so the figure is scaled by the element
+    count."""
     path = path or os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         rec = json.load(open(path)).get(kernel_key)
         if rec and rec.get("kernel_source_sha256") == kernel_source_sha256():
-            return float(rec["dram_bytes_per_launch"])
+            per_launch = float(rec["dram_bytes_read_per_launch"]) + float(rec["dram_bytes_write_per_launch"])
+            return per_launch * numel / float(rec["captured_numel"])
     except Exception:
         pass
     return None
@@ -549,8 +554,8 @@ def run_ours(args, rank, world, local_rank):
     mean_launch_s = statistics.mean(per_launch_ms) / 1e3
     peak, peak_kind = measured_peak()
     achieved = algo_bytes / mean_launch_s / 1e9
-    kernel_key = f"step_kernel/{w.name}"
-    traffic = traffic_for(kernel_key)
+    kernel_key = f"step_kernel/{'+'.join(sorted(set(w.dtypes)))}_{w.algo}"
+    traffic = traffic_for(kernel_key, w.numel)
     dtype = sorted(set(w.dtypes))
     line = {
         "metric": METRIC,
@@ -581,6 +586,9 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
+                     "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of a "
+                                        "16,777,216-element launch of the same kernel sources, scaled by "
+                                        "elements (profiles/dram_traffic.json)") if traffic else None,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
                      "kernel": "opt2s step_kernel", "algorithmic_bytes_per_launch": algo_bytes},
     }

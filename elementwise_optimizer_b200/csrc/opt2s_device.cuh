@@ -302,14 +302,17 @@ struct Aligned {
 // elements per iteration (two 16-byte vectors of fp32, or one of fp16/bf16),
 // so a warp iteration covers 256 contiguous elements of each array; the mixed
 // case moves one vector per lane per iteration.
-template <int DT, int ALGO, bool SKIP, bool ALL, int MODE = kPlain>
+template <int DT, int ALGO, bool SKIP, bool ALL, int MODE = kPlain, int U16 = 1>
 __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars& s, int lane,
                                             uint32_t head, uint32_t nvec, Aligned al,
                                             float scale = 1.0f, float wd = 0.0f)
 {
     using P = Param<DT>;
     constexpr int V = P::kVec;
-    constexpr int U = ALL ? 8 / V : 1;   // the mixed path keeps fewer values live
+    // vectors a lane moves per iteration: 8 elements (U16 x 8 for 16-bit
+    // storage in the kernels specialised to one dtype); the mixed path keeps
+    // fewer values live
+    constexpr int U = ALL ? (V == 8 ? U16 : 8 / V) : 1;
     for (uint32_t v0 = 0; v0 < nvec; v0 += 32 * U) {
         typename P::Raw graw[U], praw[U];
         float m[U][V], v[U][V], m2[U][V];
@@ -348,7 +351,7 @@ __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars
 
 // One chunk, processed by one warp: a scalar head up to the element at which
 // param is 16-byte aligned, the vector body, and a scalar tail.
-template <int DT, int ALGO, bool SKIP, int MODE = kPlain>
+template <int DT, int ALGO, bool SKIP, int MODE = kPlain, int U16 = 1>
 __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& s, int lane,
                                           float scale = 1.0f, float wd = 0.0f)
 {
@@ -369,7 +372,7 @@ __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& 
     const Aligned al{aligned16(c.g, head, P::kBytes), aligned16(c.m, head, 4),
                      aligned16(c.v, head, 4), ALGO != kAdEMAMix || aligned16(c.m2, head, 4)};
     if (al.all())
-        vector_body<DT, ALGO, SKIP, true, MODE>(c, s, lane, head, nvec, al, scale, wd);
+        vector_body<DT, ALGO, SKIP, true, MODE, U16>(c, s, lane, head, nvec, al, scale, wd);
     else
         vector_body<DT, ALGO, SKIP, false, MODE>(c, s, lane, head, nvec, al, scale, wd);
 }

@@ -66,8 +66,9 @@ struct StepScalars {
 // Threads per block.  Adam's generic kernel (96 registers) fits 20 resident
 // warps per SM as 128-thread blocks (16 as 256-thread blocks); AdEMAMix's (120
 // registers) fits 16 warps either way and measured faster as 256-thread blocks;
-// Adam specialised to one 16-bit dtype (66-72 registers) measured fastest as
-// 256-thread blocks.  `only` is the dtype every chunk of a plan shares, or -1.
+// Adam specialised to one 16-bit dtype moves two 16-byte param vectors a lane
+// per iteration (about 104 registers) and measured fastest as 256-thread
+// blocks.  `only` is the dtype every chunk of a plan shares, or -1.
 constexpr int kAdamBlockThreads = 128;
 constexpr int kAdEMAMixBlockThreads = 256;
 constexpr int kSpecialisedBlockThreads = 256;

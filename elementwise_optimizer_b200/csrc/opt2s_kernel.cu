@@ -201,9 +201,11 @@ __device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, i
         const ChunkRec rec = chunks[c];
         const bool short16 = SHORT && (rec.dtype & kShortFlag) != 0;
         if (ONLY >= 0) {
+            // one 16-bit dtype: two 16-byte param vectors a lane per iteration
+            // (16 elements), the bytes in flight of the fp32 path
             constexpr int D = ONLY >= 0 ? ONLY : kF16;
             if (short16) short_chunk<D, ALGO, SKIP>(rec, s, lane);
-            else run_chunk<D, ALGO, SKIP>(rec, s, lane);
+            else run_chunk<D, ALGO, SKIP, kPlain, 2>(rec, s, lane);
         } else {
             switch (rec.dtype & ~kShortFlag) {
             case kF32: run_chunk<kF32, ALGO, SKIP>(rec, s, lane); break;

@@ -55,8 +55,9 @@
 //      0 when it is 0; thread 0 stores the new absmaxes.
 // With skip_zeros an element whose gradient is zero keeps its param and its
 // dequantized state, which is requantized with the block's new absmax.
-// Warps of a CTA walk the 32-bit chunks of small tensors exactly as the plain
-// step kernel does (the same device functions), eight chunks per work unit.
+// Warps of a CTA walk the 32-bit chunks of small tensors element by element
+// with the plain step's element routine (opt2s_device.cuh), eight chunks per
+// work unit.
 
 #include <mutex>
 
@@ -66,6 +67,14 @@ namespace opt2s {
 namespace {
 
 constexpr int kB8Threads = 256;                  // one CTA per 8-bit block
+#ifndef OPT2S_B8_MIN_CTAS
+#define OPT2S_B8_MIN_CTAS 3
+#endif
+#ifndef OPT2S_B8_PREFETCH
+#define OPT2S_B8_PREFETCH 1
+#endif
+constexpr int kB8MinCtas = OPT2S_B8_MIN_CTAS;   // resident CTAs per SM the registers must allow
+constexpr bool kPrefetchNext = OPT2S_B8_PREFETCH != 0;
 constexpr int kB8PerThread = kBlock8Elems / kB8Threads;
 static_assert(kB8PerThread == 8, "eight elements a thread");
 
@@ -218,57 +227,76 @@ __device__ __forceinline__ uint32_t elem(int u, int j)
     return static_cast<uint32_t>(u * (kBlock8Elems * V / 8) + threadIdx.x * V + j);
 }
 
-// A thread's eight codes: one V-byte access per run when `vec`, else byte by
-// byte (0 past the end of the block).
+// A thread's eight codes, packed four to a 32-bit word (word w holds the codes
+// of elements 4w .. 4w+3 of the thread, lowest byte first): one V-byte
+// access per run when `vec`, else byte by byte (0 past the end of the block).
 template <int V>
-__device__ __forceinline__ void load_codes(const uint8_t* q, uint32_t len, bool vec,
-                                           uint32_t (&c)[kB8PerThread])
+__device__ __forceinline__ void load_codes(const uint8_t* q, uint32_t len, bool vec, uint32_t (&w)[2])
 {
 #pragma unroll
     for (int u = 0; u < 8 / V; ++u) {
         const uint32_t e = elem<V>(u, 0);
         if (vec) {
             if (V == 8) {
-                const uint2 w = *reinterpret_cast<const uint2*>(q + e);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    c[k] = (w.x >> (8 * k)) & 0xFFu;
-                    c[4 + k] = (w.y >> (8 * k)) & 0xFFu;
-                }
+                const uint2 x = *reinterpret_cast<const uint2*>(q + e);
+                w[0] = x.x;
+                w[1] = x.y;
             } else {
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(q + e);
-#pragma unroll
-                for (int k = 0; k < V; ++k) c[u * V + k] = (w >> (8 * k)) & 0xFFu;
+                w[u] = *reinterpret_cast<const uint32_t*>(q + e);
             }
         } else {
 #pragma unroll
-            for (int k = 0; k < V; ++k) c[u * V + k] = e + k < len ? q[e + k] : 0u;
+            for (int h = 0; h < V / 4; ++h) {
+                uint32_t x = 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (e + 4 * h + k < len) x |= static_cast<uint32_t>(q[e + 4 * h + k]) << (8 * k);
+                w[u * (V / 4) + h] = x;
+            }
         }
     }
 }
 
+__device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[2], int k)
+{
+    return (w[k >> 2] >> (8 * (k & 3))) & 0xFFu;
+}
+
 template <int V>
-__device__ __forceinline__ void store_codes(uint8_t* q, uint32_t len, bool vec,
-                                            const uint32_t (&c)[kB8PerThread])
+__device__ __forceinline__ void store_codes(uint8_t* q, uint32_t len, bool vec, const uint32_t (&w)[2])
 {
 #pragma unroll
     for (int u = 0; u < 8 / V; ++u) {
         const uint32_t e = elem<V>(u, 0);
         if (vec) {
-            if (V == 8) {
-                uint2 w;
-                w.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-                w.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-                *reinterpret_cast<uint2*>(q + e) = w;
-            } else {
-                *reinterpret_cast<uint32_t*>(q + e) = c[u * V] | (c[u * V + 1] << 8) |
-                                                      (c[u * V + 2] << 16) | (c[u * V + 3] << 24);
-            }
+            if (V == 8)
+                *reinterpret_cast<uint2*>(q + e) = make_uint2(w[0], w[1]);
+            else
+                *reinterpret_cast<uint32_t*>(q + e) = w[u];
         } else {
 #pragma unroll
             for (int k = 0; k < V; ++k)
-                if (e + k < len) q[e + k] = static_cast<uint8_t>(c[u * V + k]);
+                if (e + k < len) q[e + k] = static_cast<uint8_t>(code_at(w, u * V + k));
         }
+    }
+}
+
+// Asks L2 for the lines of the next block this CTA will step (param, grad and
+// codes), so that its loads after this block's barrier find them there.
+template <int ALGO>
+__device__ __forceinline__ void prefetch_block(const Block8Rec& b, int es)
+{
+    const uint32_t t = threadIdx.x;
+    const uint32_t pg_lines = (b.len * es + 127) / 128, q_lines = (b.len + 127) / 128;
+    auto pf = [](const void* a) { asm volatile("prefetch.global.L2 [%0];" :: "l"(a)); };
+    for (uint32_t l = t; l < pg_lines; l += kB8Threads) {
+        pf(static_cast<const char*>(b.p) + 128 * l);
+        pf(static_cast<const char*>(b.g) + 128 * l);
+    }
+    if (t < q_lines) {
+        pf(b.q1 + 128 * t);
+        pf(b.q2 + 128 * t);
+        if (ALGO == kAdEMAMix) pf(b.q3 + 128 * t);
     }
 }
 
@@ -295,7 +323,7 @@ __device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int b
 
     const float a1 = b.a1[0], a2 = b.a2[0];
     const float a3 = ALGO == kAdEMAMix ? b.a3[0] : 0.0f;
-    uint32_t c1[kB8PerThread], c2[kB8PerThread], c3[kB8PerThread];
+    uint32_t c1[2], c2[2], c3[2];
     load_codes<V>(b.q1, len, vec, c1);
     load_codes<V>(b.q2, len, vec, c2);
     if (ALGO == kAdEMAMix) load_codes<V>(b.q3, len, vec, c3);
@@ -330,9 +358,9 @@ __device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int b
     float x1 = 0.0f, x2 = 0.0f, x3 = 0.0f;
 #pragma unroll
     for (int k = 0; k < kB8PerThread; ++k) {
-        m[k] = __fmul_rn(mp.smap[c1[k]], a1);
-        v[k] = __fmul_rn(mp.umap[c2[k]], a2);
-        m2[k] = ALGO == kAdEMAMix ? __fmul_rn(mp.smap[c3[k]], a3) : 0.0f;
+        m[k] = __fmul_rn(mp.smap[code_at(c1, k)], a1);
+        v[k] = __fmul_rn(mp.umap[code_at(c2, k)], a2);
+        m2[k] = ALGO == kAdEMAMix ? __fmul_rn(mp.smap[code_at(c3, k)], a3) : 0.0f;
         if (elem<V>(k / V, k % V) < len) {
             update<ALGO, SKIP>(g[k], p[k], m[k], v[k], m2[k], s);
             x1 = fmaxf(x1, fabsf(m[k]));
@@ -385,22 +413,35 @@ __device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int b
     const double i1 = n1 > 0.0f ? __drcp_rn(static_cast<double>(n1)) : 0.0;
     const double i2 = n2 > 0.0f ? __drcp_rn(static_cast<double>(n2)) : 0.0;
     const double i3 = (ALGO == kAdEMAMix && n3 > 0.0f) ? __drcp_rn(static_cast<double>(n3)) : 0.0;
+    c1[0] = c1[1] = c2[0] = c2[1] = c3[0] = c3[1] = 0u;
 #pragma unroll
     for (int k = 0; k < kB8PerThread; ++k) {
-        c1[k] = n1 > 0.0f ? quantize<true>(mp.stab, m[k], i1) : kZeroSigned;
-        c2[k] = n2 > 0.0f ? quantize<false>(mp.utab, v[k], i2) : kZeroUnsigned;
-        if (ALGO == kAdEMAMix) c3[k] = n3 > 0.0f ? quantize<true>(mp.stab, m2[k], i3) : kZeroSigned;
+        const int sh = 8 * (k & 3);
+        c1[k >> 2] |= (n1 > 0.0f ? quantize<true>(mp.stab, m[k], i1) : kZeroSigned) << sh;
+        c2[k >> 2] |= (n2 > 0.0f ? quantize<false>(mp.utab, v[k], i2) : kZeroUnsigned) << sh;
+        if (ALGO == kAdEMAMix)
+            c3[k >> 2] |= (n3 > 0.0f ? quantize<true>(mp.stab, m2[k], i3) : kZeroSigned) << sh;
     }
     store_codes<V>(b.q1, len, vec, c1);
     store_codes<V>(b.q2, len, vec, c2);
     if (ALGO == kAdEMAMix) store_codes<V>(b.q3, len, vec, c3);
 }
 
+// A 32-bit chunk (at most 256 elements of a small tensor) by one warp, element
+// by element: lane l takes elements l, l + 32, ... with the plain step's
+// element routine.  Its few registers leave the 8-bit block path the
+// kernel's register budget.
+template <int DT, int ALGO, bool SKIP>
+__device__ __forceinline__ void small_chunk(const ChunkRec& c, const StepScalars& s, int lane)
+{
+    for (uint32_t i = lane; i < c.len; i += 32) scalar_element<DT, ALGO, SKIP>(c, i, s);
+}
+
 // Work unit u < nblocks: 8-bit block u, by the whole CTA.  Otherwise unit u
 // holds the 32-bit chunks 8(u - nblocks) .. 8(u - nblocks) + 7, one a warp.
 // The maps and slice tables live in dynamic shared memory (kMapsBytes).
 template <int ALGO, bool SKIP>
-__global__ void __launch_bounds__(kB8Threads)
+__global__ void __launch_bounds__(kB8Threads, kB8MinCtas)
 step8_kernel(const Block8Rec* __restrict__ blocks, int nblocks, const ChunkRec* __restrict__ chunks,
              int nchunks, StepScalars s)
 {
@@ -413,6 +454,10 @@ step8_kernel(const Block8Rec* __restrict__ blocks, int nblocks, const ChunkRec* 
     for (int u = blockIdx.x; u < units; u += gridDim.x) {   // the same u for the whole CTA
         if (u < nblocks) {
             const Block8Rec b = blocks[u];
+            if (kPrefetchNext && u + static_cast<int>(gridDim.x) < nblocks) {
+                const Block8Rec nb = blocks[u + gridDim.x];
+                prefetch_block<ALGO>(nb, nb.dtype == kF32 ? 4 : 2);
+            }
             switch (b.dtype) {
             case kF32: block8<kF32, ALGO, SKIP>(b, s, mp, buf); break;
             case kF16: block8<kF16, ALGO, SKIP>(b, s, mp, buf); break;
@@ -424,9 +469,9 @@ step8_kernel(const Block8Rec* __restrict__ blocks, int nblocks, const ChunkRec* 
             if (c < nchunks) {
                 const ChunkRec rec = chunks[c];
                 switch (rec.dtype & ~kShortFlag) {
-                case kF32: run_chunk<kF32, ALGO, SKIP>(rec, s, lane); break;
-                case kF16: run_chunk<kF16, ALGO, SKIP>(rec, s, lane); break;
-                default: run_chunk<kBF16, ALGO, SKIP>(rec, s, lane); break;
+                case kF32: small_chunk<kF32, ALGO, SKIP>(rec, s, lane); break;
+                case kF16: small_chunk<kF16, ALGO, SKIP>(rec, s, lane); break;
+                default: small_chunk<kBF16, ALGO, SKIP>(rec, s, lane); break;
                 }
             }
         }

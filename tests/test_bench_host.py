@@ -5,6 +5,8 @@ import json
 import os
 import sys
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
@@ -28,17 +30,21 @@ def test_cpu_baseline_reports_all_core_and_single_thread_figures():
 
 
 def test_traffic_lookup_follows_the_kernel_sources(tmp_path):
-    key = "step_kernel/single_f32_n268435456_adam"
-    record = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
-    assert bench.traffic_for(key) in (None, record[key]["dram_bytes_per_launch"])
-    if record[key]["kernel_source_sha256"] == bench.kernel_source_sha256():
-        assert bench.traffic_for(key) == record[key]["dram_bytes_per_launch"]
-    stale = dict(record)
-    stale[key] = dict(record[key], kernel_source_sha256="0" * 64)
+    """The committed DRAM figure is used only for the kernel sources it was
+    captured from, and scaled from the captured element count."""
+    key = "step_kernel/f32_adam"
+    rec = {"kernel_source_sha256": bench.kernel_source_sha256(), "captured_numel": 16777216,
+           "dram_bytes_read_per_launch": 268.9e6, "dram_bytes_write_per_launch": 145.0e6}
     p = tmp_path / "dram_traffic.json"
-    p.write_text(json.dumps(stale))
-    assert bench.traffic_for(key, str(p)) is None          # other sources: no figure
-    assert bench.traffic_for("no/such/kernel") is None
+    p.write_text(json.dumps({key: rec}))
+    got = bench.traffic_for(key, 268435456, str(p))
+    assert got == pytest.approx((268.9e6 + 145.0e6) * 16)
+    p.write_text(json.dumps({key: dict(rec, kernel_source_sha256="0" * 64)}))
+    assert bench.traffic_for(key, 268435456, str(p)) is None     # other sources: no figure
+    assert bench.traffic_for("no/such/kernel", 1, str(p)) is None
+    committed = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
+    for k, r in committed.items():
+        assert "captured_numel" in r and r["captured_numel"] <= 1 << 26, k   # small-case captures only
 
 
 def test_algorithmic_bytes_per_element():
