@@ -30,6 +30,10 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libopt2s.so")
 TESTING_LIB = os.path.join(PKG, "libopt2s_testing.so")
+# the optimizer front end's marshalling helper (a PyTorch C++ extension)
+MARSHAL_SRC = os.path.join(PKG, "csrc", "opt2s_marshal.cpp")
+MARSHAL_DIR = os.path.join(PKG, "_build")
+MARSHAL_NAME = "opt2s_marshal"
 
 COMMON = ["opt2s_kernel.cu", "opt2s_kernel8.cu", "opt2s_noalloc.cu", "opt2s_api8.cpp", "opt2s_ipc.cpp"]
 API = "opt2s_api.cpp"
@@ -51,6 +55,8 @@ def nvcc() -> str:
 
 
 def stale() -> bool:
+    if not os.path.exists(marshal_path()) or os.path.getmtime(marshal_path()) < os.path.getmtime(MARSHAL_SRC):
+        return True
     for lib in (LIB, TESTING_LIB):
         if not os.path.exists(lib):
             return True
@@ -58,6 +64,26 @@ def stale() -> bool:
         if any(os.path.getmtime(f) > t for f in SOURCES + HEADERS):
             return True
     return False
+
+
+def marshal_path() -> str:
+    return os.path.join(MARSHAL_DIR, MARSHAL_NAME + ".so")
+
+
+def build_marshal(force: bool = False, verbose: bool = False) -> str:
+    """Compile the optimizer's marshalling extension in-tree (host C++ against
+    PyTorch's headers; no device code)."""
+    out = marshal_path()
+    header = os.path.join(INCLUDE, "opt2s.h")
+    if (not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(MARSHAL_SRC)
+            and os.path.getmtime(out) >= os.path.getmtime(header)):
+        return out
+    os.makedirs(MARSHAL_DIR, exist_ok=True)
+    from torch.utils import cpp_extension
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    cpp_extension.load(name=MARSHAL_NAME, sources=[MARSHAL_SRC], build_directory=MARSHAL_DIR,
+                       extra_cflags=["-O2"], extra_include_paths=[INCLUDE, cuda_inc], verbose=verbose)
+    return out
 
 
 def build(force: bool = False, verbose: bool = False, nvtx: bool = False) -> str:
@@ -92,6 +118,7 @@ def build(force: bool = False, verbose: bool = False, nvtx: bool = False) -> str
         for out, objs in links:
             subprocess.run([nvcc(), *ARCH, "-shared", "-o", out + ".tmp", *objs], check=True)
             os.replace(out + ".tmp", out)
+    build_marshal(force=force, verbose=verbose)
     return LIB
 
 

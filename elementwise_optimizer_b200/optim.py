@@ -30,11 +30,16 @@ Like max_unorm it takes four launches per group and step, keeps one record
 per parameter under flatten=True, and is not combined with capturable=True.
 
 Without flatten, each group's launch records (the tensors' addresses) are
-built once and reused while the group holds the same parameter and gradient
-tensor objects, checked by identity each step; zero_grad() therefore zeroes
-gradients in place by default (set_to_none=False), so that they stay the
-same tensors.  Reassigning a tensor's storage in place (``p.data = x``,
-``.set_()``) keeps the object and is not seen: call refresh() after it.
+built once and refreshed in place every step by a small C++ helper
+(csrc/opt2s_marshal.cpp) that reads the current parameter and gradient
+addresses; a group is rebuilt only when a gradient is missing or a tensor no
+longer fits its record.  zero_grad() zeroes gradients in place by default
+(set_to_none=False), so that their addresses, and the library's cached plan,
+stay the same.  Without the helper the records are reused while the tensors
+are the same objects (checked by identity); reassigning a tensor's storage in
+place (``p.data = x``) is then not seen: call refresh() after it.  A group
+shares one step count (one launch, one set of bias corrections): a parameter
+left out of a step, its gradient None, still counts that step.
 
 capturable=True routes every step through opt2s_plan_step_table: the per-step
 scalars live in a device table and the step index in device memory, so
@@ -45,11 +50,35 @@ and call ``refill_step_table()`` between replays at least once every
 """
 from __future__ import annotations
 
+import ctypes
+import importlib.machinery
+import importlib.util
 import operator
+import os
 
 import torch
 
 from . import binding as B
+
+_marshal = None
+
+
+def _marshal_module():
+    """The in-tree marshalling extension (csrc/opt2s_marshal.cpp, built by
+    _build.build), or None when it has not been built: the identity check in
+    Python then stands in for it (same results, more host time)."""
+    global _marshal
+    if _marshal is None:
+        from . import _build
+        path = _build.marshal_path()
+        _marshal = False
+        if os.path.exists(path):
+            loader = importlib.machinery.ExtensionFileLoader(_build.MARSHAL_NAME, path)
+            spec = importlib.util.spec_from_loader(_build.MARSHAL_NAME, loader)
+            mod = importlib.util.module_from_spec(spec)
+            loader.exec_module(mod)
+            _marshal = mod
+    return _marshal or None
 
 
 class TwoStateOptimizer(torch.optim.Optimizer):
@@ -178,15 +207,22 @@ class TwoStateOptimizer(torch.optim.Optimizer):
 
     def _launch_data(self, gi, group):
         params = group["params"]
-        grads = [p.grad for p in params]
         cached = self._group_cache.get(gi)
-        if (cached is not None and len(params) == len(cached["all_params"])
-                and all(map(operator.is_, grads, cached["all_grads"]))
-                and all(map(operator.is_, params, cached["all_params"]))):
-            return cached      # the same tensors as last step: reuse the records
+        if cached is not None and cached["dense"] and len(params) == len(cached["params"]):
+            marshal = _marshal_module()
+            if marshal is not None:
+                # every parameter has a record: refresh the addresses in place
+                rc = marshal.refresh_records(params, cached["records"], len(params))
+                if rc == 0 or (rc == 1 and not self.capturable):
+                    return cached
+            elif (all(map(operator.is_, [p.grad for p in params], cached["all_grads"]))
+                  and all(map(operator.is_, params, cached["params"]))):
+                return cached      # the same tensors as last step: reuse the records
         data = self._build_launch_data(gi, group, cached)
-        data["all_params"] = list(params)
-        data["all_grads"] = grads
+        data["all_grads"] = [p.grad for p in params]
+        data["dense"] = len(data["params"]) == len(params) and all(
+            map(operator.is_, data["params"], params))
+        data["records"] = ctypes.addressof(data["tl"]._arr)
         return data
 
     def _build_launch_data(self, gi, group, cached):
