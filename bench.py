@@ -395,6 +395,73 @@ def transformer_measure(device, steps=10, warmup=3, e2e_steps=3):
     return out
 
 
+def shard_measure(device, world, rank, numel=268_435_456, steps=10, warmup=3):
+    """The ZeRO-style sharded step across the N ranks of the run, over peer
+    memory: every rank holds the whole flat fp32 param buffer (the same
+    values) and its own gradient, maps the other ranks' buffers with CUDA IPC
+    (shard.PeerBuffers), and steps its shard with opt2s_shard_step -- the
+    rank-order gradient mean, the update and the param all-gather in one
+    kernel, its remote loads and stores crossing NVLink.  Each step sits
+    between two barriers; the time is the max over ranks of the CUDA-event
+    time between them.  Every rank takes the same collective steps on every
+    path: a rank that cannot set up reports it through one all-reduce, and
+    then no rank steps.  Its results are checked against the oracle by
+    tests/test_shard_ipc_gpu.py (two processes)."""
+    import torch
+    import torch.distributed as dist
+    from elementwise_optimizer_b200 import binding as B
+    from elementwise_optimizer_b200 import shard
+    peers, err = None, None
+    try:
+        gen = torch.Generator(device=device)
+        gen.manual_seed(0x0E0A0000 + 8)                 # the same params on every rank
+        param = torch.empty(numel, device=device)
+        param.normal_(0.0, 1.0, generator=gen)
+        gen.manual_seed(0x0E0A0000 + 9 + rank)          # each rank its own gradient
+        grad = torch.empty(numel, device=device)
+        grad.normal_(0.0, 1e-2, generator=gen)
+        peers = shard.PeerBuffers(param, grad)
+        st = shard.ShardedStep(peers.params, peers.grads, rank, "adam")
+        ok = 1
+    except Exception as exc:  # reported, not hidden
+        err, ok = repr(exc), 0
+    flag = torch.tensor([ok], dtype=torch.int32, device=device)
+    dist.all_reduce(flag, op=dist.ReduceOp.MIN)
+    if int(flag.item()) == 0:
+        if peers is not None:
+            peers.close()
+        return {"error": err or "another rank could not set up its peer mappings"}
+    h = B.make_hyper("adam")
+    times = []
+    for t in range(1, warmup + steps + 1):
+        dist.barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        st.step(h, t)
+        b.record()
+        torch.cuda.synchronize()
+        dist.barrier()
+        if t > warmup:
+            times.append(a.elapsed_time(b))
+    mean_ms = max_over_ranks(statistics.mean(times), device)
+    torch.cuda.synchronize()
+    dist.barrier()                                      # no rank unmaps while another steps
+    peers.close()
+    nbytes = (8 * world + 20) * numel
+    nvlink_per_rank = 8 * (world - 1) * numel // world  # remote gradient reads + param writes
+    return {"workload": f"flat fp32 Adam, {numel} elements sharded over {world} ranks",
+            "ms_per_step": mean_ms, "elements_per_s": numel / (mean_ms / 1e3),
+            "algorithmic_bytes_per_step": nbytes,
+            "gbs_all_ranks": nbytes / (mean_ms / 1e3) / 1e9,
+            "nvlink_bytes_per_rank": nvlink_per_rank,
+            "nvlink_gbs_per_rank": nvlink_per_rank / (mean_ms / 1e3) / 1e9,
+            "path": "CUDA IPC peer mappings; one opt2s_shard_step launch per rank per step "
+                    "(plain peer loads and stores, no TMA, no multicast), barriers on both sides",
+            "steps": steps}
+
+
 def e2e_measure(w, d, device, steps, slices=8):
     """Same metric through the public call with host buffers: every step
     copies that step's gradient from pinned host memory to the device, runs
@@ -536,6 +603,12 @@ def run_ours(args, rank, world, local_rank):
             e2e["value"] = w.numel * world / (e2e_ms / 1e3)
             e2e["n_gpus"] = world
             extras["e2e"] = e2e
+    if world > 1 and not args.no_extras:
+        # every rank runs it (same collective steps); rank 0 reports it
+        del d
+        torch.cuda.empty_cache()
+        d = None
+        extras["shard"] = shard_measure(device, world, rank)
     if rank == 0 and world == 1 and not args.no_extras and args.workload == "large_f32":
         # the largest configuration, measured after the headline's buffers
         # are freed (1.2 B elements, 21.7 GB with two gradient buffers)

@@ -26,22 +26,25 @@
 // or below the exact midpoint of map[j] and map[j+1] (binary64 holds the
 // midpoint exactly), x > T_j exactly when x lies above that midpoint, so the
 // code is the number of thresholds below x.  Rather than search the 255
-// thresholds, each CTA tabulates them over the bits of x: |x| in [2^-23, 1]
-// falls in one of 24 binades x 128 slices (the exponent and the top 7
-// fraction bits); every slice is narrower than the gap between two
-// thresholds (the finest gap, 0.9/128 at the top of the unsigned map, is
-// above the widest slice, 2^-8), so a slice holds at most one threshold, and
-// its entry gives the code at the slice's bottom and that threshold: code =
-// base + (|x| > T).  Below 2^-23 the nearest value is 0 in both maps (their
-// first thresholds are 2.75e-7 and 1.6e-7).  The signed map is symmetric but
-// for its top value 1.0, so negative x use the positive table: the mirror of
-// code c is 254 - c (0 at least), one lower again when |x| is exactly a
-// midpoint (the tie then goes to the lower, more negative, code).
-// x itself is RN32(RN64(m * RN64(1/absmax))): for every quotient in the
-// binary32 normal range that is RN32(m/absmax) exactly (the binary64 product
-// errs by less than 2^-52, while a quotient that is not representable never
-// lies within 2^-49 of a binary32 rounding boundary; see div_by_constant in
-// opt2s_device.cuh), and below it both give the code of 0.
+// thresholds, each CTA tabulates them over the bits of x: the exponent picks
+// a row (|x| below 2^-23, where the nearest value is 0 in both maps; one row
+// per binade up to 2^0; NaN), the top 7 fraction bits a slice of the row.
+// Every slice is narrower than the gap between two thresholds (the finest,
+// 0.9/128 at the top of the unsigned map, is above the widest slice, 2^-8),
+// so a slice holds at most one threshold, and its 4-byte entry holds the code
+// at the slice's low end in value order (16 bits) and the low 16 bits of that
+// threshold's magnitude (the rest of its bits are the slice's own): the code
+// is base + (low16(x) > t) for x >= 0, base + (low16(x) < t) for x < 0, with
+// t a value that never compares true when the slice has no threshold.  The
+// signed map has a table per sign.
+// x itself is first taken as RN32(m * RN32(1/absmax)), within 3 ulp of
+// RN32(m/absmax); only when that lies within 4 ulp of the slice's threshold or
+// of a slice boundary (about 12 cases in 65,536) is x recomputed exactly as
+// RN32(RN64(m * RN64(1/absmax))): for every quotient in the binary32 normal
+// range that is RN32(m/absmax) (the binary64 product errs by less than
+// 2^-52, while a quotient that is not representable never lies within 2^-49
+// of a binary32 rounding boundary; see div_by_constant in opt2s_device.cuh),
+// and below it both give the code of 0.
 //
 // Per 8-bit block (one CTA of 256 threads, 8 elements a thread; fp32 storage
 // takes elements 4t..4t+3 and 1024+4t..1024+4t+3, 16-bit storage 8t..8t+7, so
@@ -67,31 +70,24 @@ namespace opt2s {
 namespace {
 
 constexpr int kB8Threads = 256;                  // one CTA per 8-bit block
-#ifndef OPT2S_B8_MIN_CTAS
-#define OPT2S_B8_MIN_CTAS 3
-#endif
-#ifndef OPT2S_B8_PREFETCH
-#define OPT2S_B8_PREFETCH 1
-#endif
-constexpr int kB8MinCtas = OPT2S_B8_MIN_CTAS;   // resident CTAs per SM the registers must allow
-constexpr bool kPrefetchNext = OPT2S_B8_PREFETCH != 0;
+// Resident CTAs per SM the registers must allow: the kernel waits on loads
+// and on its barrier, so more resident CTAs measured faster (Adam: 4 CTAs at
+// 64 registers beat 3 at 80 and 2 at 128; AdEMAMix, with a third state,
+// measured best at 3).  Each CTA also prefetches its next block into L2.
+template <int ALGO>
+constexpr int kB8MinCtas = ALGO == kAdEMAMix ? 3 : 4;
 constexpr int kB8PerThread = kBlock8Elems / kB8Threads;
 static_assert(kB8PerThread == 8, "eight elements a thread");
 
-constexpr int kSlices = 24 * 128;        // binades 2^-23 .. 2^0, 128 slices each
-constexpr uint32_t kZeroSigned = 127;   // code of 0 in the signed map
-constexpr uint32_t kZeroUnsigned = 0;   // and in the unsigned one
-
-// A slice of |x|: the code at its bottom, its threshold (+Inf if none) and
-// whether that threshold is an exact midpoint (bit 8 of `code`).
-struct QSlice {
-    float thr;
-    uint32_t code;
-};
+constexpr int kRows = 26;                // |x| < 2^-23; 24 binades 2^-23 .. 2^0; NaN
+constexpr int kSlices = kRows * 128;     // 128 slices a row
+constexpr uint32_t kZeroSigned = 127;    // code of 0 in the signed map
+constexpr uint32_t kZeroUnsigned = 0;    // and in the unsigned one
 
 struct Maps {
     float smap[256], umap[256];          // signed (m, m2) and unsigned (v) maps
-    QSlice stab[kSlices], utab[kSlices];  // quantization slices, |x| for the signed map
+    uint32_t stab[2][kSlices];           // slices of the signed map, x >= 0 and x < 0
+    uint32_t utab[kSlices];              // slices of the unsigned map
     float red[2][3][kB8Threads / 32];    // per-warp maxima, double-buffered
 };
 constexpr size_t kMapsBytes = sizeof(Maps);
@@ -120,47 +116,57 @@ __device__ float map_value(bool is_signed, int k)
     return k == at ? 0.0f : 1.0f;
 }
 
-// The threshold between map[j] and map[j + 1] (the binary32 number at or
-// below their exact midpoint) and whether the midpoint is exact.
-__device__ __forceinline__ float threshold(const float* map, int j, bool* exact)
+// The threshold between map[j] and map[j + 1]: the binary32 number at or
+// below their exact midpoint.
+__device__ __forceinline__ float threshold(const float* map, int j)
 {
-    const double mid = __dmul_rn(__dadd_rn(static_cast<double>(map[j]), static_cast<double>(map[j + 1])), 0.5);
-    const float t = __double2float_rd(mid);
-    *exact = static_cast<double>(t) == mid;
-    return t;
+    return __double2float_rd(
+        __dmul_rn(__dadd_rn(static_cast<double>(map[j]), static_cast<double>(map[j + 1])), 0.5));
 }
 
-// Number of thresholds of `map` at or below... strictly below `lo`, by a
-// binary search over the 255 thresholds (table building only).
-__device__ int codes_below(const float* map, float lo)
+// Number of thresholds below x (strictly, or at or below with `or_equal`),
+// by a binary search over the 255 thresholds (table building only).
+__device__ int thresholds_below(const float* map, float x, bool or_equal)
 {
     int c = 0;
-    bool ex;
-    for (int step = 128; step >= 1; step >>= 1)
-        if (c + step - 1 < 255 && threshold(map, c + step - 1, &ex) < lo) c += step;
+    for (int step = 128; step >= 1; step >>= 1) {
+        if (c + step - 1 < 255) {
+            const float t = threshold(map, c + step - 1);
+            if (t < x || (or_equal && t == x)) c += step;
+        }
+    }
     return c;
 }
 
-// Slice s of |x| for `map` (x >= 0): bottom code and its single threshold.
-__device__ QSlice make_slice(const float* map, int s)
+// Entry of slice i for x of sign `neg` (table building only).
+__device__ uint32_t make_slice(const float* map, int i, bool neg)
 {
-    const int e = s >> 7, k = s & 127;
-    const uint32_t lo_bits = static_cast<uint32_t>(e + 127 - 23) << 23 | static_cast<uint32_t>(k) << 16;
-    const uint32_t hi_bits = lo_bits + (1u << 16);
-    const float lo = __uint_as_float(lo_bits), hi = __uint_as_float(hi_bits);
-    const int c = codes_below(map, lo);
-    QSlice q;
-    q.code = static_cast<uint32_t>(c);
-    q.thr = __int_as_float(0x7f800000);   // +Inf: no threshold in the slice
-    if (c < 255) {
-        bool exact = false;
-        const float t = threshold(map, c, &exact);
-        if (t < hi) {
-            q.thr = t;
-            q.code |= exact ? 0x100u : 0u;
+    const int r = i >> 7, k = i & 127;
+    const uint32_t never = neg ? 0u : 0xFFFFu;   // a low-16 compare that is never true
+    if (r == 0) return (neg ? kZeroSigned : (map[0] < 0.0f ? kZeroSigned : kZeroUnsigned)) << 16 | never;
+    if (r == kRows - 1) return 0u << 16 | never;   // NaN: code 0
+    const uint32_t lo_bits = static_cast<uint32_t>(r - 1 + 127 - 23) << 23 | static_cast<uint32_t>(k) << 16;
+    const float lo = __uint_as_float(lo_bits), hi = __uint_as_float(lo_bits + (1u << 16));
+    uint32_t base, t = never;
+    if (!neg) {
+        // x in [lo, hi): thresholds below lo always count; one may lie in [lo, hi)
+        const int c = thresholds_below(map, lo, false);
+        base = static_cast<uint32_t>(c);
+        if (c < 255) {
+            const float th = threshold(map, c);
+            if (th < hi) t = __float_as_uint(th) & 0xFFFFu;
+        }
+    } else {
+        // x in (-hi, -lo]: thresholds at or below -hi always count; one may lie
+        // in (-hi, -lo), counting when |x| < |threshold|
+        const int c = thresholds_below(map, -hi, true);
+        base = static_cast<uint32_t>(c);
+        if (c < 255) {
+            const float th = threshold(map, c);
+            if (th < -lo) t = __float_as_uint(-th) & 0xFFFFu;
         }
     }
-    return q;
+    return base << 16 | t;
 }
 
 // Builds both maps and their slice tables in shared memory (all threads of
@@ -171,7 +177,7 @@ __device__ void build_maps(Maps& mp)
     const int t = threadIdx.x;
     const float sv = map_value(true, t);
     const float uv = map_value(false, t);
-    float* scratch = reinterpret_cast<float*>(mp.stab);   // unsorted values, for the ranking
+    float* scratch = reinterpret_cast<float*>(mp.utab);   // unsorted values, for the ranking
     scratch[t] = sv;
     scratch[256 + t] = uv;
     __syncthreads();
@@ -184,31 +190,47 @@ __device__ void build_maps(Maps& mp)
     mp.smap[rs] = sv;
     mp.umap[ru] = uv;
     __syncthreads();
-    for (int s = t; s < kSlices; s += kB8Threads) {
-        mp.stab[s] = make_slice(mp.smap, s);
-        mp.utab[s] = make_slice(mp.umap, s);
+    for (int i = t; i < kSlices; i += kB8Threads) {
+        mp.stab[0][i] = make_slice(mp.smap, i, false);
+        mp.stab[1][i] = make_slice(mp.smap, i, true);
+        mp.utab[i] = make_slice(mp.umap, i, false);
     }
     __syncthreads();
 }
 
-// Code of the map value nearest to m/absmax (inv = RN64(1/absmax); absmax
-// > 0): the slice of |x| gives it, mirrored for negative x in the signed map.
+// The slice entry of x's bits b: (code at the slice's low end) << 16 | t.
 template <bool SIGNED>
-__device__ __forceinline__ uint32_t quantize(const QSlice* tab, float m, double inv)
+__device__ __forceinline__ uint32_t slice_of(const Maps& mp, uint32_t b)
 {
-    const float x = __double2float_rn(__dmul_rn(static_cast<double>(m), inv));
-    const uint32_t b = __float_as_uint(x);
-    const int e = static_cast<int>((b >> 23) & 0xFFu) - (127 - 23);
-    if (e < 0) return SIGNED ? kZeroSigned : kZeroUnsigned;   // |x| < 2^-23
-    if (e > 23) return 0u;                                     // NaN (|x| <= 1 otherwise)
-    const QSlice q = tab[(e << 7) | ((b >> 16) & 0x7Fu)];
-    const float a = fabsf(x);
-    uint32_t c = (q.code & 0xFFu) + (a > q.thr ? 1u : 0u);
-    if (SIGNED && (b >> 31)) {
-        const int k = 254 - static_cast<int>(c) - ((a == q.thr && (q.code & 0x100u)) ? 1 : 0);
-        c = k < 0 ? 0u : static_cast<uint32_t>(k);
+    int r = static_cast<int>((b >> 23) & 0xFFu) - (127 - 24);   // row: binade of 2^-23 is 1
+    r = r < 0 ? 0 : (r > kRows - 1 ? kRows - 1 : r);
+    const uint32_t i = static_cast<uint32_t>(r << 7) | ((b >> 16) & 0x7Fu);
+    return SIGNED ? mp.stab[b >> 31][i] : mp.utab[i];
+}
+
+__device__ __forceinline__ uint32_t code_in(uint32_t q, uint32_t b, bool neg)
+{
+    const uint32_t lo16 = b & 0xFFFFu, t = q & 0xFFFFu;
+    return (q >> 16) + (neg ? (lo16 < t ? 1u : 0u) : (lo16 > t ? 1u : 0u));
+}
+
+// Code of the map value nearest to m/absmax (absmax > 0; r32 = RN32(1/absmax),
+// r64 = RN64(1/absmax)).  The fast quotient RN32(m*r32) is within 3 ulp of
+// RN32(m/absmax); when it lies within 4 ulp of the slice's threshold or of a
+// slice boundary the exact quotient decides.
+template <bool SIGNED>
+__device__ __forceinline__ uint32_t quantize(const Maps& mp, float m, float r32, double r64)
+{
+    uint32_t b = __float_as_uint(__fmul_rn(m, r32));
+    uint32_t q = slice_of<SIGNED>(mp, b);
+    const uint32_t lo16 = b & 0xFFFFu, t = q & 0xFFFFu;
+    const uint32_t d = lo16 > t ? lo16 - t : t - lo16;
+    const bool real_thr = t != 0u && t != 0xFFFFu;
+    if (lo16 < 4u || lo16 > 0xFFFFu - 4u || (real_thr && d <= 4u)) {
+        b = __float_as_uint(__double2float_rn(__dmul_rn(static_cast<double>(m), r64)));
+        q = slice_of<SIGNED>(mp, b);
     }
-    return c;
+    return code_in(q, b, SIGNED && (b >> 31));
 }
 
 __device__ __forceinline__ float warp_max(float x)
@@ -409,18 +431,22 @@ __device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int b
         b.a2[0] = n2;
         if (ALGO == kAdEMAMix) b.a3[0] = n3;
     }
-    // correctly rounded binary64 reciprocals of the new absmaxes
+    // reciprocals of the new absmaxes: RN32 for the fast quotient, RN64 for
+    // the exact one
     const double i1 = n1 > 0.0f ? __drcp_rn(static_cast<double>(n1)) : 0.0;
     const double i2 = n2 > 0.0f ? __drcp_rn(static_cast<double>(n2)) : 0.0;
     const double i3 = (ALGO == kAdEMAMix && n3 > 0.0f) ? __drcp_rn(static_cast<double>(n3)) : 0.0;
+    const float f1 = n1 > 0.0f ? __frcp_rn(n1) : 0.0f;
+    const float f2 = n2 > 0.0f ? __frcp_rn(n2) : 0.0f;
+    const float f3 = (ALGO == kAdEMAMix && n3 > 0.0f) ? __frcp_rn(n3) : 0.0f;
     c1[0] = c1[1] = c2[0] = c2[1] = c3[0] = c3[1] = 0u;
 #pragma unroll
     for (int k = 0; k < kB8PerThread; ++k) {
         const int sh = 8 * (k & 3);
-        c1[k >> 2] |= (n1 > 0.0f ? quantize<true>(mp.stab, m[k], i1) : kZeroSigned) << sh;
-        c2[k >> 2] |= (n2 > 0.0f ? quantize<false>(mp.utab, v[k], i2) : kZeroUnsigned) << sh;
+        c1[k >> 2] |= (n1 > 0.0f ? quantize<true>(mp, m[k], f1, i1) : kZeroSigned) << sh;
+        c2[k >> 2] |= (n2 > 0.0f ? quantize<false>(mp, v[k], f2, i2) : kZeroUnsigned) << sh;
         if (ALGO == kAdEMAMix)
-            c3[k >> 2] |= (n3 > 0.0f ? quantize<true>(mp.stab, m2[k], i3) : kZeroSigned) << sh;
+            c3[k >> 2] |= (n3 > 0.0f ? quantize<true>(mp, m2[k], f3, i3) : kZeroSigned) << sh;
     }
     store_codes<V>(b.q1, len, vec, c1);
     store_codes<V>(b.q2, len, vec, c2);
@@ -441,7 +467,7 @@ __device__ __forceinline__ void small_chunk(const ChunkRec& c, const StepScalars
 // holds the 32-bit chunks 8(u - nblocks) .. 8(u - nblocks) + 7, one a warp.
 // The maps and slice tables live in dynamic shared memory (kMapsBytes).
 template <int ALGO, bool SKIP>
-__global__ void __launch_bounds__(kB8Threads, kB8MinCtas)
+__global__ void __launch_bounds__(kB8Threads, kB8MinCtas<ALGO>)
 step8_kernel(const Block8Rec* __restrict__ blocks, int nblocks, const ChunkRec* __restrict__ chunks,
              int nchunks, StepScalars s)
 {
@@ -454,7 +480,7 @@ step8_kernel(const Block8Rec* __restrict__ blocks, int nblocks, const ChunkRec* 
     for (int u = blockIdx.x; u < units; u += gridDim.x) {   // the same u for the whole CTA
         if (u < nblocks) {
             const Block8Rec b = blocks[u];
-            if (kPrefetchNext && u + static_cast<int>(gridDim.x) < nblocks) {
+            if (u + static_cast<int>(gridDim.x) < nblocks) {
                 const Block8Rec nb = blocks[u + gridDim.x];
                 prefetch_block<ALGO>(nb, nb.dtype == kF32 ? 4 : 2);
             }

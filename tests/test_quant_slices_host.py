@@ -1,79 +1,123 @@
-"""The 8-bit kernel's quantization by slices of |x|, checked on the CPU.
+"""The 8-bit kernel's quantization by slices of x, checked on the CPU.
 
 The kernel finds the code of the map value nearest to x without a search:
-|x| in [2^-23, 1] falls in one of 24 binades x 128 slices (the exponent and
-the top 7 fraction bits), each slice holds at most one threshold between
-neighbouring map values, and its entry gives the code at the slice's bottom
-plus one if |x| is above that threshold; negative x in the signed map use the
-mirror code 254 - c (one lower at an exact midpoint); |x| below 2^-23 takes
-the code of 0.  These tests rebuild that rule from the pinned oracle map and
-check its premises and its result against the oracle's brute-force nearest
-code, over random values, every threshold and its neighbours, and exact ties.
+the exponent of x picks a row (below 2^-23, where the nearest value is 0;
+one row per binade up to 2^0; NaN), the top 7 fraction bits a slice of the
+row; every slice holds at most one threshold between neighbouring map
+values, and its entry gives the code at the slice's low end (in value order)
+and the low 16 bits of that threshold's magnitude, compared with the low 16
+bits of x (greater for x >= 0, smaller for x < 0; a table per sign).  These
+tests rebuild that rule from the pinned oracle map and check its premises
+and its result against the oracle's brute-force nearest code, over random
+values, every threshold and its neighbours, and exact ties.  They also check
+the margin the kernel's fast quotient relies on: RN32(m * RN32(1/N)) is within
+3 ulp of RN32(m / N).
 """
 import numpy as np
 import pytest
+
+ROWS = 26
 
 
 def _thresholds(qmap):
     mid = (qmap[:-1].astype(np.float64) + qmap[1:].astype(np.float64)) / 2
     t = mid.astype(np.float32)
     t = np.where(t.astype(np.float64) > mid, np.nextafter(t, np.float32(-np.inf)), t)   # round down
-    return t.astype(np.float32), t.astype(np.float64) == mid
+    return t.astype(np.float32)
 
 
-def _slices(qmap):
-    thr, exact = _thresholds(qmap)
-    lo_bits = ((np.arange(24)[:, None] + 127 - 23) << 23 | (np.arange(128)[None, :] << 16)).reshape(-1)
-    lo = lo_bits.astype(np.uint32).view(np.float32)
-    hi = (lo_bits + (1 << 16)).astype(np.uint32).view(np.float32)
-    base = np.searchsorted(thr, lo, side="left")              # thresholds strictly below lo
-    inside = [(thr >= a) & (thr < b) for a, b in zip(lo, hi)]
-    return thr, exact, lo, hi, base, inside
+def _bits(x):
+    return int(np.float32(x).view(np.uint32))
 
 
-def _code(qmap, slices, x, signed):
-    thr, exact, lo, hi, base, inside = slices
+def _table(qmap, neg):
+    thr = _thresholds(qmap)
+    never = 0 if neg else 0xFFFF
+    zero = int(np.nonzero(qmap == 0)[0][0])
+    tab = []
+    for i in range(ROWS * 128):
+        r, k = divmod(i, 128)
+        if r == 0:
+            tab.append((zero << 16) | never)
+            continue
+        if r == ROWS - 1:
+            tab.append(never)
+            continue
+        lo_bits = ((r - 1 + 127 - 23) << 23) | (k << 16)
+        lo = np.uint32(lo_bits).view(np.float32)
+        hi = np.uint32(lo_bits + (1 << 16)).view(np.float32)
+        t = never
+        if not neg:
+            base = int(np.searchsorted(thr, lo, side="left"))        # thresholds < lo
+            if base < 255 and thr[base] < hi:
+                t = _bits(thr[base]) & 0xFFFF
+        else:
+            base = int(np.searchsorted(thr, -hi, side="right"))      # thresholds <= -hi
+            if base < 255 and thr[base] < -lo:
+                t = _bits(-thr[base]) & 0xFFFF
+        tab.append((base << 16) | t)
+    return tab
+
+
+def _inside_counts(qmap):
+    thr = _thresholds(qmap)
+    counts = []
+    for i in range(128, (ROWS - 1) * 128):
+        r, k = divmod(i, 128)
+        lo_bits = ((r - 1 + 127 - 23) << 23) | (k << 16)
+        lo = np.uint32(lo_bits).view(np.float32)
+        hi = np.uint32(lo_bits + (1 << 16)).view(np.float32)
+        counts.append(int(((thr >= lo) & (thr < hi)).sum()))
+        counts.append(int(((thr > -hi) & (thr < -lo)).sum()))
+    return counts
+
+
+def _code(tabs, x, signed):
     out = []
     for v in np.asarray(x, np.float32):
-        a = abs(float(v))
-        if a < 2.0 ** -23:
-            out.append(127 if signed else 0)
-            continue
-        bits = int(np.float32(a).view(np.uint32))
-        s = ((bits >> 23) - (127 - 23)) * 128 + ((bits >> 16) & 0x7F)
-        c = int(base[s])
-        t = thr[c] if c < 255 and thr[c] < hi[s] else np.float32(np.inf)
-        tie = c < 255 and thr[c] < hi[s] and bool(exact[c]) and a == float(t)
-        c += 1 if a > float(t) else 0
-        if signed and v < 0:
-            c = max(0, 254 - c - (1 if tie else 0))
-        out.append(c)
+        b = _bits(v)
+        r = min(max(((b >> 23) & 0xFF) - (127 - 24), 0), ROWS - 1)
+        i = (r << 7) | ((b >> 16) & 0x7F)
+        neg = signed and (b >> 31) == 1
+        q = tabs[1 if neg else 0][i]
+        lo16, t = b & 0xFFFF, q & 0xFFFF
+        out.append((q >> 16) + (int(lo16 < t) if neg else int(lo16 > t)))
     return np.array(out, np.uint8)
 
 
 @pytest.mark.parametrize("signed", [True, False])
 def test_every_slice_holds_at_most_one_threshold(oracle_mod, signed):
     qmap = oracle_mod.quant_map(signed)
-    *_, inside = _slices(qmap)
-    assert max(int(m.sum()) for m in inside) <= 1
-    thr, _ = _thresholds(qmap)
-    pos = thr[thr > 0]
-    assert pos.min() > 2.0 ** -23          # below 2^-23 the nearest value is 0
+    assert max(_inside_counts(qmap)) <= 1
+    thr = _thresholds(qmap)
+    assert np.abs(thr[thr != 0]).min() > 2.0 ** -23     # below 2^-23 the nearest value is 0
 
 
 @pytest.mark.parametrize("signed", [True, False])
 def test_slice_rule_gives_the_nearest_code(oracle_mod, signed):
     qmap = oracle_mod.quant_map(signed)
-    sl = _slices(qmap)
-    thr, exact = _thresholds(qmap)
+    tabs = (_table(qmap, False), _table(qmap, True))
+    thr = _thresholds(qmap)
     g = np.random.Generator(np.random.Philox(71))
     lo = -1.0 if signed else 0.0
     xs = [g.uniform(lo, 1.0, 3000), np.sign(g.uniform(lo, 1.0, 3000)) * 10.0 ** g.uniform(-9, 0, 3000),
           qmap, thr, np.nextafter(thr, np.float32(2)), np.nextafter(thr, np.float32(-2)),
-          np.array([0.0, 1.0, 2.0 ** -23, np.nextafter(np.float32(2.0 ** -23), np.float32(0))])]
+          np.array([0.0, 1.0, 2.0 ** -23, np.nextafter(np.float32(2.0 ** -23), np.float32(0)), np.nan])]
     if signed:
-        xs += [-thr, -np.nextafter(thr, np.float32(2)), -qmap, np.array([-1.0, -(2.0 ** -23)])]
+        xs += [-thr, -np.nextafter(thr, np.float32(2)), -qmap, np.array([-1.0, -(2.0 ** -23), -0.0])]
     x = np.concatenate([np.asarray(a, np.float64) for a in xs]).astype(np.float32)
-    x = x[(x >= -1) & (x <= 1)]
-    assert np.array_equal(_code(qmap, sl, x, signed), oracle_mod.quantize(qmap, x))
-    assert exact.sum() > 50                 # exact ties are among the cases
+    x = x[np.isnan(x) | ((x >= -1) & (x <= 1))]
+    assert np.array_equal(_code(tabs, x, signed), oracle_mod.quantize(qmap, x))
+
+
+def test_fast_quotient_is_within_three_ulp():
+    """RN32(m * RN32(1/N)) against RN32(m / N), for |m| <= N over many
+    magnitudes: at most 3 ulp of the exact quotient apart."""
+    g = np.random.Generator(np.random.Philox(73))
+    n = (10.0 ** g.uniform(-30, 30, 200_000)).astype(np.float32)
+    m = (n * g.uniform(-1, 1, n.size).astype(np.float32)).astype(np.float32)
+    exact = (m / n).astype(np.float32)
+    fast = (m * (np.float32(1) / n)).astype(np.float32)
+    ok = np.isfinite(fast) & (np.abs(exact) >= 2.0 ** -126)
+    ulp = np.spacing(np.abs(exact[ok])).astype(np.float64)
+    assert np.max(np.abs(fast[ok].astype(np.float64) - exact[ok].astype(np.float64)) / ulp) <= 3

@@ -123,3 +123,48 @@ def test_two_processes_step_their_shards_over_ipc(tmp_path, dtype, algo):
                for r in range(world)]
     assert results == ["ok"] * world, results
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+
+
+def _bench_rank(rank, world, port, out_dir):
+    import datetime
+    import json
+    import sys
+    import torch.distributed as dist
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dev = torch.device("cuda", rank % torch.cuda.device_count())
+    torch.cuda.set_device(dev)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        res = bench.shard_measure(dev, world, rank, numel=4_000_037, steps=3, warmup=1)
+        with open(os.path.join(out_dir, f"bench{rank}.json"), "w") as f:
+            json.dump(res, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_shard_leg_runs_across_processes(tmp_path):
+    """The bench's sharded-step leg (run at N > 1): peer mappings, barriers and
+    the max-over-ranks time, with two processes."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import json
+    import torch.multiprocessing as mp
+    from elementwise_optimizer_b200 import _build
+    _build.build()
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_bench_rank, args=(r, 2, port, str(tmp_path))) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    for r in range(2):
+        res = json.load(open(tmp_path / f"bench{r}.json"))
+        assert "error" not in res, res
+        assert res["ms_per_step"] > 0 and res["nvlink_bytes_per_rank"] == 8 * 4_000_037 // 2
