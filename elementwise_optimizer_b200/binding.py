@@ -161,6 +161,7 @@ EXPORTS = {
     "opt2s_testing_check_division": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int32,
                                                     ctypes.POINTER(ctypes.c_int64)]),
     "opt2s_testing_max_block_threads": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32]),
+    "opt2s_testing_quant_tables": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int64]),
 }
 
 # exported by the test build only
@@ -566,6 +567,21 @@ def testing_choose_chunk_elems(tl: TensorList, resident_warps: int) -> int:
 
 def testing_fail_allocs(count: int) -> None:
     check(_testing_lib().opt2s_testing_fail_allocs(int(count)), "testing_fail_allocs")
+
+
+QUANT_TABLE_WORDS = 512 + 3 * 26 * 128
+
+
+def testing_quant_tables():
+    """The 8-bit step's quantization tables as the library builds them:
+    (signed map, unsigned map, signed slices x >= 0, x < 0, unsigned slices)."""
+    import numpy as np
+    buf = (ctypes.c_uint32 * QUANT_TABLE_WORDS)()
+    check(lib().opt2s_testing_quant_tables(buf, QUANT_TABLE_WORDS), "testing_quant_tables")
+    a = np.frombuffer(bytes(buf), np.uint32).copy()
+    n = 26 * 128
+    return (a[:256].view(np.float32), a[256:512].view(np.float32), a[512:512 + n],
+            a[512 + n:512 + 2 * n], a[512 + 2 * n:])
 
 
 def launch_count() -> int:

@@ -11,6 +11,8 @@
 // block, one per 32-bit chunk -- and every later step is one launch that
 // reads them.
 
+#include <algorithm>
+#include <cmath>
 #include <cstring>
 #include <list>
 #include <mutex>
@@ -21,6 +23,7 @@
 
 #include "opt2s.h"
 #include "opt2s_internal.h"
+#include "opt2s_testing.h"
 
 #define OPT2S_API extern "C" __attribute__((visibility("default")))
 
@@ -90,13 +93,122 @@ int validate8(const TensorListDesc8* d, int32_t algo)
     return opt2s::overlap_status(ranges.data(), ranges.size());
 }
 
+// ---------------------------------------------------------------------------
+// Quantization tables (the layout is described in opt2s_internal.h)
+// ---------------------------------------------------------------------------
+
+// The 256 values of a map, ascending: for E = 0..6 and F = 6 - E (signed) or
+// 7 - E (unsigned) fraction bits, 10^-E * (0.1 + 0.9*(2f+1)/2^(F+1)) for
+// f = 0 .. 2^F - 1 (both signs when signed), plus 0 and 1.0 -- Dettmers et
+// al. 2022, sections 2.2 (dynamic tree quantization) and 2.3 (dynamic
+// quantization).  Each value is N/D with N = 2^(F+1) + 9*(2f+1) and
+// D = 10^(E+1)*2^(F+1), exact binary32 integers: one IEEE division.
+void quant_map(bool is_signed, float* out)
+{
+    int k = 0;
+    const int f0 = is_signed ? 6 : 7;
+    for (int E = 0; E <= 6; ++E) {
+        const int F = f0 - E;
+        float D = static_cast<float>(1 << (F + 1));
+        for (int e = 0; e <= E; ++e) D *= 10.0f;
+        for (int f = 0; f < (1 << F); ++f) {
+            const float v = static_cast<float>((1 << (F + 1)) + 9 * (2 * f + 1)) / D;
+            out[k++] = v;
+            if (is_signed) out[k++] = -v;
+        }
+    }
+    out[k++] = 0.0f;
+    out[k++] = 1.0f;
+    std::sort(out, out + k);
+}
+
+// The binary32 number at or below the exact midpoint of map[j] and map[j+1]
+// (binary64 holds the midpoint exactly).
+float threshold(const float* map, int j)
+{
+    const double mid = (static_cast<double>(map[j]) + static_cast<double>(map[j + 1])) * 0.5;
+    float t = static_cast<float>(mid);
+    if (static_cast<double>(t) > mid) t = std::nextafter(t, -INFINITY);
+    return t;
+}
+
+// Number of thresholds below x (or at or below it, with `or_equal`).
+int thresholds_below(const float* thr, float x, bool or_equal)
+{
+    return static_cast<int>(or_equal ? std::upper_bound(thr, thr + 255, x) - thr
+                                     : std::lower_bound(thr, thr + 255, x) - thr);
+}
+
+uint32_t bits_of(float x)
+{
+    uint32_t u;
+    std::memcpy(&u, &x, sizeof u);
+    return u;
+}
+
+float float_of(uint32_t u)
+{
+    float x;
+    std::memcpy(&x, &u, sizeof x);
+    return x;
+}
+
+// Slice i of the map with thresholds `thr`, for x of sign `neg`.
+uint32_t slice_entry(const float* thr, uint32_t zero_code, int i, bool neg)
+{
+    const int r = i >> 7, k = i & 127;
+    const uint32_t never = neg ? 0u : 0xFFFFu;   // a low-16 compare that never holds
+    if (r == 0) return zero_code << 16 | never;                      // |x| < 2^-23
+    if (r == opt2s::kQuantRows - 1) return never;                    // NaN: code 0
+    const uint32_t lo_bits = static_cast<uint32_t>(r - 1 + 127 - 23) << 23 | static_cast<uint32_t>(k) << 16;
+    const float lo = float_of(lo_bits), hi = float_of(lo_bits + (1u << 16));
+    uint32_t t = never;
+    int base;
+    if (!neg) {
+        // x in [lo, hi): thresholds below lo count; at most one lies in [lo, hi)
+        base = thresholds_below(thr, lo, false);
+        if (base < 255 && thr[base] < hi) t = bits_of(thr[base]) & 0xFFFFu;
+    } else {
+        // x in (-hi, -lo]: thresholds at or below -hi count; at most one lies
+        // in (-hi, -lo) and counts when |x| is below its magnitude
+        base = thresholds_below(thr, -hi, true);
+        if (base < 255 && thr[base] < -lo) t = bits_of(-thr[base]) & 0xFFFFu;
+    }
+    return static_cast<uint32_t>(base) << 16 | t;
+}
+
+}  // namespace
+
+void opt2s::build_quant_tables(uint32_t* out)
+{
+    float smap[256], umap[256], sthr[255], uthr[255];
+    quant_map(true, smap);
+    quant_map(false, umap);
+    for (int j = 0; j < 255; ++j) {
+        sthr[j] = threshold(smap, j);
+        uthr[j] = threshold(umap, j);
+    }
+    constexpr int kSlices = opt2s::kQuantRows * 128;
+    std::memcpy(out, smap, sizeof smap);
+    std::memcpy(out + 256, umap, sizeof umap);
+    for (int i = 0; i < kSlices; ++i) {
+        out[512 + i] = slice_entry(sthr, 127, i, false);
+        out[512 + kSlices + i] = slice_entry(sthr, 127, i, true);
+        out[512 + 2 * kSlices + i] = slice_entry(uthr, 0, i, false);
+    }
+}
+
+namespace {
+
 struct Plan8 {
     int device;
     int32_t algo;
     int64_t nblocks, nchunks;
-    void* d_mem;                 // Block8Rec[nblocks] then ChunkRec[nchunks]
+    void* d_mem;                 // quantization tables, Block8Rec[nblocks], ChunkRec[nchunks]
     std::vector<opt2s_tensor8> records;
 };
+
+constexpr size_t kTableBytes = opt2s::kQuantTableWords * sizeof(uint32_t);   // a multiple of 16
 
 // Tables of `d` (validated): one Block8Rec per 2,048-element block of every
 // 8-bit tensor, one ChunkRec per kChunk32 elements of every 32-bit tensor, in
@@ -154,21 +266,22 @@ int plan8_create(const TensorListDesc8* d, int32_t algo, int dev, Plan8** out)
                                           std::vector<opt2s_tensor8>(d->tensors, d->tensors + d->count)};
     if (!plan) return OPT2S_ERR_NO_MEMORY;
     const size_t bb = blocks.size() * sizeof(Block8Rec), cb = chunks.size() * sizeof(ChunkRec);
-    if (bb + cb > 0) {
-        cudaError_t e = cudaMalloc(&plan->d_mem, bb + cb);
-        if (e != cudaSuccess) {
-            delete plan;
-            if (e == cudaErrorMemoryAllocation) { opt2s::record_cuda_error(e); return OPT2S_ERR_NO_MEMORY; }
-            return opt2s::record_cuda_error(e);
-        }
-        if (bb) e = cudaMemcpy(plan->d_mem, blocks.data(), bb, cudaMemcpyHostToDevice);
-        if (e == cudaSuccess && cb)
-            e = cudaMemcpy(static_cast<char*>(plan->d_mem) + bb, chunks.data(), cb, cudaMemcpyHostToDevice);
-        if (e != cudaSuccess) {
-            cudaFree(plan->d_mem);
-            delete plan;
-            return opt2s::record_cuda_error(e);
-        }
+    std::vector<uint32_t> tables(opt2s::kQuantTableWords);
+    opt2s::build_quant_tables(tables.data());
+    cudaError_t e = cudaMalloc(&plan->d_mem, kTableBytes + bb + cb);
+    if (e != cudaSuccess) {
+        delete plan;
+        if (e == cudaErrorMemoryAllocation) { opt2s::record_cuda_error(e); return OPT2S_ERR_NO_MEMORY; }
+        return opt2s::record_cuda_error(e);
+    }
+    char* at = static_cast<char*>(plan->d_mem);
+    e = cudaMemcpy(at, tables.data(), kTableBytes, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && bb) e = cudaMemcpy(at + kTableBytes, blocks.data(), bb, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && cb) e = cudaMemcpy(at + kTableBytes + bb, chunks.data(), cb, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        cudaFree(plan->d_mem);
+        delete plan;
+        return opt2s::record_cuda_error(e);
     }
     *out = plan;
     return OPT2S_OK;
@@ -232,10 +345,11 @@ OPT2S_API int opt2s_step_8bit(const TensorListDesc8* desc, const Hyper* hyper, i
         }
     }
     if (plan->nblocks + plan->nchunks == 0) return OPT2S_OK;
-    const auto* d_blocks = static_cast<const Block8Rec*>(plan->d_mem);
-    const auto* d_chunks = reinterpret_cast<const ChunkRec*>(static_cast<const char*>(plan->d_mem) +
-                                                             plan->nblocks * sizeof(Block8Rec));
-    e = opt2s::launch_step8(d_blocks, plan->nblocks, d_chunks, plan->nchunks, hyper->algo,
+    const char* at = static_cast<const char*>(plan->d_mem);
+    const auto* d_tables = reinterpret_cast<const uint32_t*>(at);
+    const auto* d_blocks = reinterpret_cast<const Block8Rec*>(at + kTableBytes);
+    const auto* d_chunks = reinterpret_cast<const ChunkRec*>(at + kTableBytes + plan->nblocks * sizeof(Block8Rec));
+    e = opt2s::launch_step8(d_blocks, plan->nblocks, d_chunks, plan->nchunks, d_tables, hyper->algo,
                             hyper->skip_zeros, opt2s::make_scalars(hyper, step), 0, stream);
     if (e != cudaSuccess) return opt2s::record_cuda_error(e);
     opt2s::count_launches(1);
@@ -253,4 +367,11 @@ void opt2s::release_cache8()
     std::lock_guard<std::mutex> lock(g_cache8_mu);
     for (Plan8* p : g_cache8) plan8_destroy(p);
     g_cache8.clear();
+}
+
+OPT2S_API int opt2s_testing_quant_tables(uint32_t* out, int64_t cap)
+{
+    if (!out || cap < opt2s::kQuantTableWords) return OPT2S_ERR_INVALID_ARG;
+    opt2s::build_quant_tables(out);
+    return OPT2S_OK;
 }

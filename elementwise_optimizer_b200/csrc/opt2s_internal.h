@@ -187,12 +187,27 @@ struct alignas(16) Block8Rec {
 };
 static_assert(sizeof(Block8Rec) == 80, "Block8Rec layout");
 
-// Launches one 8-bit-state step on `stream`: `nblocks` block records and
-// `nchunks` 32-bit chunk records (device memory).  max_blocks <= 0: the
-// occupancy cap (resident CTAs per SM x SMs).
+// The quantization tables of the 8-bit step, as 32-bit words: the signed
+// and the unsigned map (256 binary32 values each, ascending), then the slice
+// entries (kQuantRows x 128 each) of the signed map for x >= 0 and for x < 0
+// and of the unsigned map.  A slice entry is (code at the slice's low end in
+// value order) << 16 | (low 16 bits of the magnitude of the one threshold
+// inside the slice, or a value whose compare never holds).  Built on the host
+// by build_quant_tables (opt2s_api8.cpp) and copied into every CTA's shared
+// memory.
+constexpr int kQuantRows = 26;
+constexpr int kQuantTableWords = 512 + 3 * kQuantRows * 128;
+
+// Fills `out` (kQuantTableWords words) with the tables above.
+void build_quant_tables(uint32_t* out);
+
+// Launches one 8-bit-state step on `stream`: `nblocks` block records,
+// `nchunks` 32-bit chunk records and the quantization tables (device memory,
+// 16-byte aligned).  max_blocks <= 0: the occupancy cap (resident CTAs per SM
+// x SMs).
 cudaError_t launch_step8(const Block8Rec* d_blocks, int64_t nblocks, const ChunkRec* d_chunks,
-                         int64_t nchunks, int algo, int skip_zeros, const StepScalars& s,
-                         int max_blocks, cudaStream_t stream);
+                         int64_t nchunks, const uint32_t* d_tables, int algo, int skip_zeros,
+                         const StepScalars& s, int max_blocks, cudaStream_t stream);
 
 // Frees the cached plans of the 8-bit-state step (opt2s_api8.cpp); called by
 // opt2s_release_cache.

@@ -18,8 +18,10 @@
 //     10^-E * (0.1 + 0.9*(2f + 1)/2^(F+1)),  f = 0 .. 2^F - 1
 // (with both signs for the signed map), plus 0 and 1.0.  Each value is
 // N/D with N = 2^(F+1) + 9*(2f+1) and D = 10^(E+1)*2^(F+1), exact binary32
-// integers, so one IEEE division gives it rounded once.  Every CTA builds the
-// two maps in shared memory at start.
+// integers, so one IEEE division gives it rounded once.  The host builds the
+// two maps and the slice tables below once per plan (opt2s_api8.cpp,
+// build_quant_tables) and uploads them with it; every CTA copies them into
+// shared memory at start.
 //
 // Quantization: the code of x = RN32(m / absmax) is the map value nearest to
 // x, an exact tie going to the lower code.  With T_j the binary32 number at
@@ -62,6 +64,7 @@
 // with the plain step's element routine (opt2s_device.cuh), eight chunks per
 // work unit.
 
+#include <cstddef>
 #include <mutex>
 
 #include "opt2s_device.cuh"
@@ -79,10 +82,10 @@ constexpr int kB8MinCtas = ALGO == kAdEMAMix ? 3 : 4;
 constexpr int kB8PerThread = kBlock8Elems / kB8Threads;
 static_assert(kB8PerThread == 8, "eight elements a thread");
 
-constexpr int kRows = 26;                // |x| < 2^-23; 24 binades 2^-23 .. 2^0; NaN
-constexpr int kSlices = kRows * 128;     // 128 slices a row
-constexpr uint32_t kZeroSigned = 127;    // code of 0 in the signed map
-constexpr uint32_t kZeroUnsigned = 0;    // and in the unsigned one
+constexpr int kRows = kQuantRows;         // |x| < 2^-23; 24 binades 2^-23 .. 2^0; NaN
+constexpr int kSlices = kRows * 128;      // 128 slices a row
+constexpr uint32_t kZeroSigned = 127;     // code of 0 in the signed map
+constexpr uint32_t kZeroUnsigned = 0;     // and in the unsigned one
 
 struct Maps {
     float smap[256], umap[256];          // signed (m, m2) and unsigned (v) maps
@@ -92,109 +95,17 @@ struct Maps {
 };
 constexpr size_t kMapsBytes = sizeof(Maps);
 
-// Value of map entry k before sorting: the k-th (value, sign) of the
-// construction above, in the order of E, f (and sign); k = 254 is 0 and
-// k = 255 is 1.0.
-__device__ float map_value(bool is_signed, int k)
-{
-    const int f0 = is_signed ? 6 : 7;
-    int at = 0;
-    for (int E = 0; E <= 6; ++E) {
-        const int F = f0 - E;
-        const int per = (1 << F) * (is_signed ? 2 : 1);
-        if (k < at + per) {
-            const int r = k - at;
-            const int f = is_signed ? r >> 1 : r;
-            float D = static_cast<float>(1 << (F + 1));
-            for (int e = 0; e <= E; ++e) D = __fmul_rn(D, 10.0f);
-            const float N = static_cast<float>((1 << (F + 1)) + 9 * (2 * f + 1));
-            const float v = __fdiv_rn(N, D);
-            return (is_signed && (r & 1)) ? -v : v;
-        }
-        at += per;
-    }
-    return k == at ? 0.0f : 1.0f;
-}
+// The tables as the host lays them out (QuantTables, opt2s_internal.h) are
+// the leading words of Maps; each CTA copies them in at start.
+static_assert(offsetof(Maps, smap) == 0 && offsetof(Maps, umap) == 256 * 4 &&
+                  offsetof(Maps, stab) == 512 * 4 && offsetof(Maps, utab) == (512 + 2 * kSlices) * 4,
+              "table layout");
+static_assert(kQuantTableWords == 512 + 3 * kSlices, "table size");
 
-// The threshold between map[j] and map[j + 1]: the binary32 number at or
-// below their exact midpoint.
-__device__ __forceinline__ float threshold(const float* map, int j)
+__device__ void load_maps(Maps& mp, const uint4* __restrict__ tables)
 {
-    return __double2float_rd(
-        __dmul_rn(__dadd_rn(static_cast<double>(map[j]), static_cast<double>(map[j + 1])), 0.5));
-}
-
-// Number of thresholds below x (strictly, or at or below with `or_equal`),
-// by a binary search over the 255 thresholds (table building only).
-__device__ int thresholds_below(const float* map, float x, bool or_equal)
-{
-    int c = 0;
-    for (int step = 128; step >= 1; step >>= 1) {
-        if (c + step - 1 < 255) {
-            const float t = threshold(map, c + step - 1);
-            if (t < x || (or_equal && t == x)) c += step;
-        }
-    }
-    return c;
-}
-
-// Entry of slice i for x of sign `neg` (table building only).
-__device__ uint32_t make_slice(const float* map, int i, bool neg)
-{
-    const int r = i >> 7, k = i & 127;
-    const uint32_t never = neg ? 0u : 0xFFFFu;   // a low-16 compare that is never true
-    if (r == 0) return (neg ? kZeroSigned : (map[0] < 0.0f ? kZeroSigned : kZeroUnsigned)) << 16 | never;
-    if (r == kRows - 1) return 0u << 16 | never;   // NaN: code 0
-    const uint32_t lo_bits = static_cast<uint32_t>(r - 1 + 127 - 23) << 23 | static_cast<uint32_t>(k) << 16;
-    const float lo = __uint_as_float(lo_bits), hi = __uint_as_float(lo_bits + (1u << 16));
-    uint32_t base, t = never;
-    if (!neg) {
-        // x in [lo, hi): thresholds below lo always count; one may lie in [lo, hi)
-        const int c = thresholds_below(map, lo, false);
-        base = static_cast<uint32_t>(c);
-        if (c < 255) {
-            const float th = threshold(map, c);
-            if (th < hi) t = __float_as_uint(th) & 0xFFFFu;
-        }
-    } else {
-        // x in (-hi, -lo]: thresholds at or below -hi always count; one may lie
-        // in (-hi, -lo), counting when |x| < |threshold|
-        const int c = thresholds_below(map, -hi, true);
-        base = static_cast<uint32_t>(c);
-        if (c < 255) {
-            const float th = threshold(map, c);
-            if (th < -lo) t = __float_as_uint(-th) & 0xFFFFu;
-        }
-    }
-    return base << 16 | t;
-}
-
-// Builds both maps and their slice tables in shared memory (all threads of
-// the CTA take part; ends with a barrier).  Sorting: the rank of a value is
-// the number of values below it (all 256 are distinct).
-__device__ void build_maps(Maps& mp)
-{
-    const int t = threadIdx.x;
-    const float sv = map_value(true, t);
-    const float uv = map_value(false, t);
-    float* scratch = reinterpret_cast<float*>(mp.utab);   // unsorted values, for the ranking
-    scratch[t] = sv;
-    scratch[256 + t] = uv;
-    __syncthreads();
-    int rs = 0, ru = 0;
-    for (int j = 0; j < 256; ++j) {
-        rs += scratch[j] < sv;
-        ru += scratch[256 + j] < uv;
-    }
-    __syncthreads();
-    mp.smap[rs] = sv;
-    mp.umap[ru] = uv;
-    __syncthreads();
-    for (int i = t; i < kSlices; i += kB8Threads) {
-        mp.stab[0][i] = make_slice(mp.smap, i, false);
-        mp.stab[1][i] = make_slice(mp.smap, i, true);
-        mp.utab[i] = make_slice(mp.umap, i, false);
-    }
+    uint4* dst = reinterpret_cast<uint4*>(&mp);
+    for (int i = threadIdx.x; i < kQuantTableWords / 4; i += kB8Threads) dst[i] = tables[i];
     __syncthreads();
 }
 
@@ -469,11 +380,11 @@ __device__ __forceinline__ void small_chunk(const ChunkRec& c, const StepScalars
 template <int ALGO, bool SKIP>
 __global__ void __launch_bounds__(kB8Threads, kB8MinCtas<ALGO>)
 step8_kernel(const Block8Rec* __restrict__ blocks, int nblocks, const ChunkRec* __restrict__ chunks,
-             int nchunks, StepScalars s)
+             int nchunks, const uint4* __restrict__ tables, StepScalars s)
 {
     extern __shared__ __align__(16) unsigned char smem8[];
     Maps& mp = *reinterpret_cast<Maps*>(smem8);
-    build_maps(mp);
+    load_maps(mp, tables);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int units = nblocks + (nchunks + kB8Threads / 32 - 1) / (kB8Threads / 32);
     int buf = 0;
@@ -504,7 +415,7 @@ step8_kernel(const Block8Rec* __restrict__ blocks, int nblocks, const ChunkRec* 
     }
 }
 
-using Kernel8Fn = void (*)(const Block8Rec*, int, const ChunkRec*, int, StepScalars);
+using Kernel8Fn = void (*)(const Block8Rec*, int, const ChunkRec*, int, const uint4*, StepScalars);
 
 Kernel8Fn pick8(int algo, int skip)
 {
@@ -520,8 +431,8 @@ std::mutex g_occ8_mu;
 }  // namespace
 
 cudaError_t launch_step8(const Block8Rec* d_blocks, int64_t nblocks, const ChunkRec* d_chunks,
-                         int64_t nchunks, int algo, int skip_zeros, const StepScalars& s,
-                         int max_blocks, cudaStream_t stream)
+                         int64_t nchunks, const uint32_t* d_tables, int algo, int skip_zeros,
+                         const StepScalars& s, int max_blocks, cudaStream_t stream)
 {
     const int64_t units = nblocks + (nchunks + kB8Threads / 32 - 1) / (kB8Threads / 32);
     if (units <= 0) return cudaSuccess;
@@ -554,7 +465,9 @@ cudaError_t launch_step8(const Block8Rec* d_blocks, int64_t nblocks, const Chunk
     StepScalars sc = s;
     fill_reciprocals(&sc);
     int nb = static_cast<int>(nblocks), nc = static_cast<int>(nchunks);
-    void* args[] = {const_cast<Block8Rec**>(&d_blocks), &nb, const_cast<ChunkRec**>(&d_chunks), &nc, &sc};
+    const uint4* tab = reinterpret_cast<const uint4*>(d_tables);
+    void* args[] = {const_cast<Block8Rec**>(&d_blocks), &nb, const_cast<ChunkRec**>(&d_chunks), &nc,
+                    const_cast<uint4**>(&tab), &sc};
     return cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3(grid), dim3(kB8Threads), args,
                             kMapsBytes, stream);
 }

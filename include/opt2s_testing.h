@@ -109,6 +109,12 @@ int opt2s_testing_check_division(uint64_t seed, int64_t n, int32_t mode, int64_t
  * (OPT2S_ERR_NO_MEMORY). */
 int opt2s_testing_fail_allocs(int count);
 
+/* Host only: the quantization tables the 8-bit step uploads with every plan
+ * (the signed and unsigned maps, then the slice entries; the layout is
+ * described in the library's internal header): `cap` >= 10,496 words.
+ * Lets the tests check the library's tables against the oracle's map. */
+int opt2s_testing_quant_tables(uint32_t *out, int64_t cap);
+
 /* Number of kernels this library has launched in this process. */
 int64_t opt2s_testing_launch_count(void);
 

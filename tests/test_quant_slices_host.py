@@ -121,3 +121,19 @@ def test_fast_quotient_is_within_three_ulp():
     ok = np.isfinite(fast) & (np.abs(exact) >= 2.0 ** -126)
     ulp = np.spacing(np.abs(exact[ok])).astype(np.float64)
     assert np.max(np.abs(fast[ok].astype(np.float64) - exact[ok].astype(np.float64)) / ulp) <= 3
+
+
+def test_library_tables_are_the_rule(oracle_mod):
+    """The tables the library uploads with every 8-bit plan (built on the
+    host, opt2s_api8.cpp) equal the pinned oracle maps and the slice rule
+    rebuilt here from them."""
+    from elementwise_optimizer_b200 import _build
+    from elementwise_optimizer_b200 import binding as B
+    _build.build()
+    smap, umap, spos, sneg, upos = B.testing_quant_tables()
+    qs, qu = oracle_mod.quant_map(True), oracle_mod.quant_map(False)
+    assert np.array_equal(smap.view(np.uint32), qs.view(np.uint32))
+    assert np.array_equal(umap.view(np.uint32), qu.view(np.uint32))
+    assert np.array_equal(spos, np.array(_table(qs, False), np.uint32))
+    assert np.array_equal(sneg, np.array(_table(qs, True), np.uint32))
+    assert np.array_equal(upos, np.array(_table(qu, False), np.uint32))
