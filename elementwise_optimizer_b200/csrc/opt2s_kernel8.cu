@@ -110,12 +110,14 @@ __device__ void load_maps(Maps& mp, const uint4* __restrict__ tables)
 }
 
 // The slice entry of x's bits b: (code at the slice's low end) << 16 | t.
+// The exponent and the top 7 fraction bits, bits 16..30 of b, number the
+// slices of all binades in order; clamping puts every |x| below 2^-23 in
+// slice 0 of the first row and every NaN in the last slice of the NaN row.
 template <bool SIGNED>
 __device__ __forceinline__ uint32_t slice_of(const Maps& mp, uint32_t b)
 {
-    int r = static_cast<int>((b >> 23) & 0xFFu) - (127 - 24);   // row: binade of 2^-23 is 1
-    r = r < 0 ? 0 : (r > kRows - 1 ? kRows - 1 : r);
-    const uint32_t i = static_cast<uint32_t>(r << 7) | ((b >> 16) & 0x7Fu);
+    int i = static_cast<int>((b >> 16) & 0x7FFFu) - (127 - 24) * 128;
+    i = min(max(i, 0), kSlices - 1);
     return SIGNED ? mp.stab[b >> 31][i] : mp.utab[i];
 }
 
@@ -127,17 +129,16 @@ __device__ __forceinline__ uint32_t code_in(uint32_t q, uint32_t b, bool neg)
 
 // Code of the map value nearest to m/absmax (absmax > 0; r32 = RN32(1/absmax),
 // r64 = RN64(1/absmax)).  The fast quotient RN32(m*r32) is within 3 ulp of
-// RN32(m/absmax); when it lies within 4 ulp of the slice's threshold or of a
-// slice boundary the exact quotient decides.
+// RN32(m/absmax); when its low 16 bits lie within 4 of the slice's threshold
+// or of a slice boundary, the exact quotient decides.  (A slice without a
+// threshold holds 0 or 0xFFFF there, which only adds boundary cases.)
 template <bool SIGNED>
 __device__ __forceinline__ uint32_t quantize(const Maps& mp, float m, float r32, double r64)
 {
     uint32_t b = __float_as_uint(__fmul_rn(m, r32));
     uint32_t q = slice_of<SIGNED>(mp, b);
-    const uint32_t lo16 = b & 0xFFFFu, t = q & 0xFFFFu;
-    const uint32_t d = lo16 > t ? lo16 - t : t - lo16;
-    const bool real_thr = t != 0u && t != 0xFFFFu;
-    if (lo16 < 4u || lo16 > 0xFFFFu - 4u || (real_thr && d <= 4u)) {
+    const uint32_t lo4 = (b & 0xFFFFu) + 4u;
+    if (lo4 - (q & 0xFFFFu) <= 8u || (lo4 & 0xFFFFu) < 8u) {
         b = __float_as_uint(__double2float_rn(__dmul_rn(static_cast<double>(m), r64)));
         q = slice_of<SIGNED>(mp, b);
     }
@@ -241,18 +242,18 @@ __device__ __forceinline__ bool al(const void* q, uint32_t bytes)
 // One 8-bit block by the whole CTA.  `buf` selects the half of the reduction
 // scratch this block uses (alternating between a CTA's blocks, so that no
 // second barrier is needed before the next block writes it).
-template <int DT, int ALGO, bool SKIP>
-__device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int buf)
+// FULL: a whole block of kBlock8Elems elements whose arrays are aligned for
+// the vector accesses (the common case, with no per-element bounds checks);
+// otherwise elements are accessed one by one and those past `len` skipped.
+template <int DT, int ALGO, bool SKIP, bool FULL>
+__device__ __forceinline__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int buf)
 {
     using P = Param<DT>;
     constexpr int V = P::kVec;
     constexpr int R = 8 / V;   // runs a thread
-    const uint32_t len = b.len;
+    const uint32_t len = FULL ? static_cast<uint32_t>(kBlock8Elems) : b.len;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // full, aligned blocks move a run in one 16-byte (param, grad) and one
-    // V-byte (codes) access; others go element by element
-    const bool vec = len == static_cast<uint32_t>(kBlock8Elems) && al(b.p, 16) && al(b.g, 16) &&
-                     al(b.q1, V) && al(b.q2, V) && (ALGO != kAdEMAMix || al(b.q3, V));
+    constexpr bool vec = FULL;
 
     const float a1 = b.a1[0], a2 = b.a2[0];
     const float a3 = ALGO == kAdEMAMix ? b.a3[0] : 0.0f;
@@ -294,7 +295,7 @@ __device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int b
         m[k] = __fmul_rn(mp.smap[code_at(c1, k)], a1);
         v[k] = __fmul_rn(mp.umap[code_at(c2, k)], a2);
         m2[k] = ALGO == kAdEMAMix ? __fmul_rn(mp.smap[code_at(c3, k)], a3) : 0.0f;
-        if (elem<V>(k / V, k % V) < len) {
+        if (FULL || elem<V>(k / V, k % V) < len) {
             update<ALGO, SKIP>(g[k], p[k], m[k], v[k], m2[k], s);
             x1 = fmaxf(x1, fabsf(m[k]));
             x2 = fmaxf(x2, fabsf(v[k]));
@@ -364,6 +365,24 @@ __device__ void block8(const Block8Rec& b, const StepScalars& s, Maps& mp, int b
     if (ALGO == kAdEMAMix) store_codes<V>(b.q3, len, vec, c3);
 }
 
+// A ragged or unaligned block, out of line so that it does not add to the
+// full-block path's registers.
+template <int DT, int ALGO, bool SKIP>
+__device__ __noinline__ void block8_part(const Block8Rec b, const StepScalars s, Maps& mp, int buf)
+{
+    block8<DT, ALGO, SKIP, false>(b, s, mp, buf);
+}
+
+template <int DT, int ALGO, bool SKIP>
+__device__ __forceinline__ void block8_any(const Block8Rec& b, const StepScalars& s, Maps& mp, int buf)
+{
+    constexpr int V = Param<DT>::kVec;
+    const bool full = b.len == static_cast<uint32_t>(kBlock8Elems) && al(b.p, 16) && al(b.g, 16) &&
+                      al(b.q1, V) && al(b.q2, V) && (ALGO != kAdEMAMix || al(b.q3, V));
+    if (full) block8<DT, ALGO, SKIP, true>(b, s, mp, buf);
+    else block8_part<DT, ALGO, SKIP>(b, s, mp, buf);
+}
+
 // A 32-bit chunk (at most 256 elements of a small tensor) by one warp, element
 // by element: lane l takes elements l, l + 32, ... with the plain step's
 // element routine.  Its few registers leave the 8-bit block path the
@@ -396,9 +415,9 @@ step8_kernel(const Block8Rec* __restrict__ blocks, int nblocks, const ChunkRec* 
                 prefetch_block<ALGO>(nb, nb.dtype == kF32 ? 4 : 2);
             }
             switch (b.dtype) {
-            case kF32: block8<kF32, ALGO, SKIP>(b, s, mp, buf); break;
-            case kF16: block8<kF16, ALGO, SKIP>(b, s, mp, buf); break;
-            default: block8<kBF16, ALGO, SKIP>(b, s, mp, buf); break;
+            case kF32: block8_any<kF32, ALGO, SKIP>(b, s, mp, buf); break;
+            case kF16: block8_any<kF16, ALGO, SKIP>(b, s, mp, buf); break;
+            default: block8_any<kBF16, ALGO, SKIP>(b, s, mp, buf); break;
             }
             buf ^= 1;
         } else {
