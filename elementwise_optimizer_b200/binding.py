@@ -63,7 +63,8 @@ class opt2s_step_scalars(ctypes.Structure):
     _fields_ = [(n, ctypes.c_float) for n in (
         "lr", "beta1", "beta2", "beta3", "one_minus_beta1", "one_minus_beta2",
         "one_minus_beta3", "alpha", "eps", "bc1", "bc2", "decay")] + [
-        ("inv_bc1", ctypes.c_double), ("inv_bc2", ctypes.c_double)]
+        ("inv_bc1", ctypes.c_double), ("inv_bc2", ctypes.c_double)] + [
+        (n, ctypes.c_float) for n in ("rcp_bc1_hi", "rcp_bc1_lo", "rcp_bc2_hi", "rcp_bc2_lo")]
 
 
 MAX_WORLD = 8

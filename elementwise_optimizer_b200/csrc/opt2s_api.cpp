@@ -584,6 +584,8 @@ static_assert(sizeof(opt2s_step_scalars) == sizeof(StepScalars), "scalar table l
 static_assert(offsetof(opt2s_step_scalars, decay) == offsetof(StepScalars, decay), "scalar table layout");
 static_assert(offsetof(opt2s_step_scalars, inv_bc1) == offsetof(StepScalars, inv_bc1), "scalar table layout");
 static_assert(offsetof(opt2s_step_scalars, inv_bc2) == offsetof(StepScalars, inv_bc2), "scalar table layout");
+static_assert(offsetof(opt2s_step_scalars, rcp_bc1_hi) == offsetof(StepScalars, rcp_bc1_hi), "scalar table layout");
+static_assert(offsetof(opt2s_step_scalars, rcp_bc2_lo) == offsetof(StepScalars, rcp_bc2_lo), "scalar table layout");
 
 OPT2S_API int opt2s_fill_step_scalars(const Hyper* hyper, int first_step, int count,
                                       opt2s_step_scalars* out)
@@ -836,7 +838,8 @@ OPT2S_API int opt2s_testing_fail_allocs(int count)
 OPT2S_API int opt2s_testing_check_division(uint64_t seed, int64_t n, int32_t mode,
                                            int64_t* mismatches)
 {
-    if (!mismatches || n < 0 || (mode != 0 && mode != 1)) return OPT2S_ERR_INVALID_ARG;
+    if (!mismatches || n < 0 || mode < 0 || mode > 2) return OPT2S_ERR_INVALID_ARG;
+    if (mode == 2 && n > (int64_t{1} << 20)) return OPT2S_ERR_INVALID_ARG;   // n * 2^32 operands
     unsigned long long* d_count = nullptr;
     cudaError_t e = cudaMalloc(&d_count, sizeof(*d_count));
     if (e != cudaSuccess) return cuda_fail(e);

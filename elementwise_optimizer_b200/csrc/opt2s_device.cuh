@@ -36,12 +36,11 @@ template <typename T>
 __device__ __forceinline__ void st_global(T* p, const T& v) { *p = v; }
 
 // ---------------------------------------------------------------------------
-// Exact division by a per-launch constant.
+// Exact division by a per-launch constant d, 2^-25 <= d <= 1 (the bias
+// corrections bc1, bc2), with r = RN64(1/d) and its fp32 split hi = RN32(r),
+// lo = RN32(r - hi) computed once per launch on the host.
 //
-// For every binary32 x and every binary32 d with 0 < |d| <= 1 (the bias
-// corrections bc1, bc2 lie in (0, 1]), with r = RN64(1/d) the correctly
-// rounded binary64 reciprocal computed once per launch on the host:
-//            RN32( RN64(x * r) ) == RN32(x / d).
+// Wide route, for every binary32 x:  RN32( RN64(x * r) ) == RN32(x / d).
 // Why: RN64(x*r) = (x/d)(1+e) with |e| <= 2^-52 + 2^-106, so it suffices that
 // x/d is never within 2^-49 (relative) of a binary32 rounding boundary
 // unless it is a binary32 number itself (then |e| < half an ulp keeps it).
@@ -54,12 +53,37 @@ __device__ __forceinline__ void st_global(T* p, const T& v) { *p = v; }
 // is.  binary64 neither overflows nor underflows here, and 0, +-Inf and NaN
 // pass through the product unchanged.  (The exclusion argument used in the
 // analysis of double rounding; see Muller et al., Handbook of Floating-Point
-// Arithmetic, 2nd ed., ch. 4.)  A GPU test checks it against __fdiv_rn on
-// random operands of every class.
+// Arithmetic, 2nd ed., ch. 4.)
+//
+// fp32 route, for 2^-40 <= |x| < 2^96 (everything else takes the wide route):
+//     q0 = RN32(x*hi + RN32(x*lo)),  rem = x - q0*d,  q = RN32(q0 + rem*hi).
+// hi + lo is 1/d to within 2^-47 (relative), so q0 is x/d to within half an
+// ulp plus 2^-46 relative: a faithful quotient.  The remainder of a faithful
+// quotient is a binary32 number, so one FMA computes it exactly (it is a
+// multiple of 2^-111 here: no underflow), and with hi the correctly rounded
+// reciprocal, RN32(q0 + rem*hi) is the correctly rounded quotient
+// (Markstein's theorem: P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990; also
+// Muller et al., ch. 4).  No step overflows or underflows in that range
+// (|x/d| < 2^121).  Four fp32 operations and an exponent test instead of two
+// float/double conversions and a binary64 product: the conversions run on
+// the narrow XU pipe, which limits the compute-heavy kernels.
+// GPU tests check both routes against __fdiv_rn: every binary32 x for a
+// sample of divisors, and random operands near rounding boundaries.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float div_by_constant(float x, double r)
+__device__ __forceinline__ float div_by_constant_wide(float x, double r)
 {
     return __double2float_rn(__dmul_rn(static_cast<double>(x), r));
+}
+
+__device__ __forceinline__ float div_by_constant(float x, float d, float hi, float lo, double r)
+{
+    // biased exponent of |x| in [87, 223): 2^-40 <= |x| < 2^96
+    const uint32_t e = __float_as_uint(x) & 0x7F800000u;
+    if (__builtin_expect(e - (87u << 23) >= (136u << 23), 0)) return div_by_constant_wide(x, r);
+    const float q0 = __fmaf_rn(x, hi, __fmul_rn(x, lo));
+    const float rem = __fmaf_rn(-q0, d, x);
+    return __fmaf_rn(rem, hi, q0);
 }
 
 // ---------------------------------------------------------------------------
@@ -83,12 +107,13 @@ __device__ __forceinline__ float direction(float g, float& m, float& v, float& m
     m = __fadd_rn(__fmul_rn(s.beta1, m), __fmul_rn(s.one_minus_beta1, g));
     v = __fadd_rn(__fmul_rn(s.beta2, v),
                   __fmul_rn(__fmul_rn(s.one_minus_beta2, g), g));
-    float num = div_by_constant(m, s.inv_bc1);
+    float num = div_by_constant(m, s.bc1, s.rcp_bc1_hi, s.rcp_bc1_lo, s.inv_bc1);
     if (ALGO == kAdEMAMix) {
         m2 = __fadd_rn(__fmul_rn(s.beta3, m2), __fmul_rn(s.one_minus_beta3, g));
         num = __fadd_rn(num, __fmul_rn(s.alpha, m2));
     }
-    const float den = __fadd_rn(__fsqrt_rn(div_by_constant(v, s.inv_bc2)), s.eps);
+    const float den = __fadd_rn(__fsqrt_rn(div_by_constant(v, s.bc2, s.rcp_bc2_hi, s.rcp_bc2_lo,
+                                                                   s.inv_bc2)), s.eps);
     return __fdiv_rn(num, den);
 }
 

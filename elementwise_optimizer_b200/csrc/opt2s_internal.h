@@ -57,10 +57,12 @@ struct StepScalars {
     float eps;
     float bc1, bc2;
     float decay;
-    // RN64(1/bc1), RN64(1/bc2): filled in by launch_step from bc1/bc2 (both
-    // in (0, 1]); the kernel divides by bc1, bc2 exactly through them (see
-    // div_by_constant in opt2s_kernel.cu)
+    // RN64(1/bc1), RN64(1/bc2), and each split into an fp32 pair
+    // (RN32(r), RN32(r - RN32(r))): filled in at launch from bc1/bc2 (both in
+    // [2^-25, 1]); the kernels divide by bc1, bc2 exactly through them (see
+    // div_by_constant in opt2s_device.cuh)
     double inv_bc1, inv_bc2;
+    float rcp_bc1_hi, rcp_bc1_lo, rcp_bc2_hi, rcp_bc2_lo;
 };
 
 // Threads per block.  Adam's generic kernel (96 registers) fits 20 resident
@@ -213,7 +215,8 @@ cudaError_t launch_step8(const Block8Rec* d_blocks, int64_t nblocks, const Chunk
 // opt2s_release_cache.
 void release_cache8();
 
-// Sets s->inv_bc1, s->inv_bc2 = RN64(1/bc1), RN64(1/bc2) (host).
+// Sets s->inv_bc1, s->inv_bc2 = RN64(1/bc1), RN64(1/bc2) and their fp32
+// splits rcp_bc*_hi = RN32(inv), rcp_bc*_lo = RN32(inv - hi) (host).
 void fill_reciprocals(StepScalars* s);
 
 // Launches one step whose scalars are d_table[*d_index] (device memory),
@@ -284,6 +287,7 @@ inline StepScalars make_scalars(const Hyper* h, int step)
     s.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(h->beta2), static_cast<double>(step)));
     s.decay = static_cast<float>(1.0 - static_cast<double>(h->lr) * static_cast<double>(h->weight_decay));
     s.inv_bc1 = s.inv_bc2 = 0.0;
+    s.rcp_bc1_hi = s.rcp_bc1_lo = s.rcp_bc2_hi = s.rcp_bc2_lo = 0.0f;
     return s;
 }
 

@@ -623,6 +623,11 @@ void fill_reciprocals(StepScalars* s)
 {
     s->inv_bc1 = 1.0 / static_cast<double>(s->bc1);
     s->inv_bc2 = 1.0 / static_cast<double>(s->bc2);
+    // inv - hi is exact in binary64 (the two agree to 24 bits)
+    s->rcp_bc1_hi = static_cast<float>(s->inv_bc1);
+    s->rcp_bc1_lo = static_cast<float>(s->inv_bc1 - static_cast<double>(s->rcp_bc1_hi));
+    s->rcp_bc2_hi = static_cast<float>(s->inv_bc2);
+    s->rcp_bc2_lo = static_cast<float>(s->inv_bc2 - static_cast<double>(s->rcp_bc2_hi));
 }
 
 cudaError_t launch_step_table(const ChunkRec* d_chunks, int64_t nchunks, int algo, int skip_zeros,

@@ -12,13 +12,17 @@ namespace opt2s {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Validation scaffolding: div_by_constant against __fdiv_rn on random operands.
-// Operands come from the SplitMix64 output function (Steele, Lea & Flood,
-// "Fast splittable pseudorandom number generators", OOPSLA 2014) applied to a
-// counter.  mode 0: x is a random bit pattern (every class: zeros, subnormals,
-// normals, infinities, NaNs).  mode 1: x = RN32(d * B) for B a random rounding
-// boundary, so x/d lies close to a boundary (the hard cases).  d is a random
-// binary32 in (0, 1] (subnormals included; d = 1 about once in 1,024 draws).
+// Validation scaffolding: div_by_constant against __fdiv_rn.  Operands come
+// from the SplitMix64 output function (Steele, Lea & Flood, "Fast splittable
+// pseudorandom number generators", OOPSLA 2014) applied to a counter.
+// Divisors lie in [2^-25, 1], the bias corrections' range: a random binade
+// and significand, with d = 1, powers of two and all-ones significands drawn
+// often.  The reciprocal and its fp32 split are formed as the host forms them.
+//   mode 0: n operands, x a random bit pattern (every class: zeros,
+//           subnormals, normals, infinities, NaNs);
+//   mode 1: n operands, x = RN32(d * B) for B a random rounding boundary, so
+//           that x/d lies close to a boundary (the hard cases);
+//   mode 2: n divisors, each with every one of the 2^32 binary32 x.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint64_t splitmix64(uint64_t z)
 {
@@ -28,35 +32,55 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t z)
     return z ^ (z >> 31);
 }
 
+__device__ __forceinline__ float draw_divisor(uint64_t h)
+{
+    uint32_t bits = (102u + static_cast<uint32_t>((h >> 32) % 25u)) << 23 |
+                    static_cast<uint32_t>(h & 0x7FFFFFu);          // [2^-25, 1)
+    if (((h >> 44) & 15u) == 0) bits &= 0xFF800000u;               // a power of two
+    if (((h >> 48) & 15u) == 0) bits |= 0x007FFFFFu;               // all-ones significand
+    if (((h >> 52) & 63u) == 0) bits = 0x3F800000u;                // d = 1
+    return __uint_as_float(bits);
+}
+
+__device__ __forceinline__ bool same_quotient(float x, float d)
+{
+    const double r = __drcp_rn(static_cast<double>(d));
+    const float hi = __double2float_rn(r);
+    const float lo = __double2float_rn(__dsub_rn(r, static_cast<double>(hi)));
+    const float a = div_by_constant(x, d, hi, lo, r);
+    const float b = __fdiv_rn(x, d);
+    return __float_as_uint(a) == __float_as_uint(b) || (isnan(a) && isnan(b));
+}
+
 __global__ void check_division_kernel(uint64_t seed, int64_t n, int mode,
                                       unsigned long long* mismatches)
 {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
-        const uint64_t h1 = splitmix64(seed + 3 * static_cast<uint64_t>(i));
-        const uint64_t h2 = splitmix64(seed + 3 * static_cast<uint64_t>(i) + 1);
-        uint32_t dbits = (static_cast<uint32_t>(h2 >> 32) % 127u) << 23 |
-                         static_cast<uint32_t>(h2 & 0x7FFFFFu);
-        if (dbits == 0) dbits = 1;
-        if ((h2 >> 54) == 0) dbits = 0x3F800000u;          // d = 1
-        const float d = __uint_as_float(dbits);
-        float x;
-        if (mode == 0) {
-            x = __uint_as_float(static_cast<uint32_t>(h1));
+    const int64_t total = mode == 2 ? (n << 32) : n;
+    unsigned long long bad = 0;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+        float x, d;
+        if (mode == 2) {
+            d = draw_divisor(splitmix64(seed + static_cast<uint64_t>(i >> 32)));
+            x = __uint_as_float(static_cast<uint32_t>(i));
         } else {
-            // a rounding boundary: the midpoint just above a random finite float
-            const uint64_t h3 = splitmix64(seed + 3 * static_cast<uint64_t>(i) + 2);
-            const float f = __uint_as_float(static_cast<uint32_t>(h3) & 0x7F7FFFFFu);
-            const double mid = 0.5 * (static_cast<double>(f) +
-                                      static_cast<double>(__uint_as_float(__float_as_uint(f) + 1)));
-            x = __double2float_rn(__dmul_rn(mid, static_cast<double>(d)));
-            if (h1 & 1) x = -x;
+            const uint64_t h1 = splitmix64(seed + 3 * static_cast<uint64_t>(i));
+            d = draw_divisor(splitmix64(seed + 3 * static_cast<uint64_t>(i) + 1));
+            if (mode == 0) {
+                x = __uint_as_float(static_cast<uint32_t>(h1));
+            } else {
+                // a rounding boundary: the midpoint just above a random finite float
+                const uint64_t h3 = splitmix64(seed + 3 * static_cast<uint64_t>(i) + 2);
+                const float f = __uint_as_float(static_cast<uint32_t>(h3) & 0x7F7FFFFFu);
+                const double mid = 0.5 * (static_cast<double>(f) +
+                                          static_cast<double>(__uint_as_float(__float_as_uint(f) + 1)));
+                x = __double2float_rn(__dmul_rn(mid, static_cast<double>(d)));
+                if (h1 & 1) x = -x;
+            }
         }
-        const float a = div_by_constant(x, __drcp_rn(static_cast<double>(d)));
-        const float b = __fdiv_rn(x, d);
-        const bool same = __float_as_uint(a) == __float_as_uint(b) || (isnan(a) && isnan(b));
-        if (!same) atomicAdd(mismatches, 1ull);
+        if (!same_quotient(x, d)) ++bad;
     }
+    if (bad) atomicAdd(mismatches, bad);
 }
 
 }  // namespace

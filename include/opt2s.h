@@ -168,6 +168,8 @@ typedef struct {
     float one_minus_beta1, one_minus_beta2, one_minus_beta3;
     float alpha, eps, bc1, bc2, decay;
     double inv_bc1, inv_bc2;    /* correctly rounded binary64 1/bc1, 1/bc2 */
+    float rcp_bc1_hi, rcp_bc1_lo;   /* fp32 split of inv_bc1: RN32(inv), RN32(inv - hi) */
+    float rcp_bc2_hi, rcp_bc2_lo;   /* and of inv_bc2 */
 } opt2s_step_scalars;
 
 int opt2s_fill_step_scalars(const Hyper *hyper, int first_step, int count,

@@ -97,11 +97,12 @@ int opt2s_testing_unorm_tables(const TensorListDesc *desc, int32_t algo, int64_t
                                uint32_t *chunk_tensor, int64_t *counts);
 
 /* Test build only.  Runs the step kernel's exact division by a constant in
- * (0, 1] and the IEEE division __fdiv_rn side by side on `n` seeded random
- * operand pairs on the current device (mode 0: x of every class; mode 1: x/d
- * next to a binary32 rounding boundary) and writes how many results differ
- * (NaN equals NaN) to *mismatches.  Synchronous; allocates a counter on the
- * device. */
+ * [2^-25, 1] and the IEEE division __fdiv_rn side by side on the current
+ * device: mode 0, `n` seeded random pairs with x of every class; mode 1, `n`
+ * pairs with x/d next to a binary32 rounding boundary; mode 2, `n` seeded
+ * divisors (n <= 2^20), each with all 2^32 binary32 x.  Writes how many
+ * results differ (NaN equals NaN) to *mismatches.  Synchronous; allocates a
+ * counter on the device. */
 int opt2s_testing_check_division(uint64_t seed, int64_t n, int32_t mode, int64_t *mismatches);
 
 /* Test build only.  Fault injection on the host: the next `count` device

@@ -71,8 +71,9 @@ def test_struct_layout_matches_c(L):
              offsetof(opt2s_tensor, dtype), sizeof(TensorListDesc), sizeof(Hyper),
              offsetof(Hyper, skip_zeros));
       printf("%zu %zu\n", sizeof(opt2s_testing_chunk), offsetof(opt2s_testing_chunk, dtype));
-      printf("%zu %zu %zu\n", sizeof(opt2s_step_scalars), offsetof(opt2s_step_scalars, decay),
-             offsetof(opt2s_step_scalars, inv_bc2));
+      printf("%zu %zu %zu %zu %zu\n", sizeof(opt2s_step_scalars), offsetof(opt2s_step_scalars, decay),
+             offsetof(opt2s_step_scalars, inv_bc2), offsetof(opt2s_step_scalars, rcp_bc1_hi),
+             offsetof(opt2s_step_scalars, rcp_bc2_lo));
       return 0;
     }"""
     with tempfile.TemporaryDirectory() as d:
@@ -90,7 +91,8 @@ def test_struct_layout_matches_c(L):
     assert b == [ctypes.sizeof(B.opt2s_testing_chunk), B.opt2s_testing_chunk.dtype.offset]
     c = list(map(int, lines[2].split()))
     assert c == [ctypes.sizeof(B.opt2s_step_scalars), B.opt2s_step_scalars.decay.offset,
-                 B.opt2s_step_scalars.inv_bc2.offset]
+                 B.opt2s_step_scalars.inv_bc2.offset, B.opt2s_step_scalars.rcp_bc1_hi.offset,
+                 B.opt2s_step_scalars.rcp_bc2_lo.offset]
 
 
 def test_abi_version(L):
@@ -440,6 +442,10 @@ def test_step_scalar_table_matches_the_definitions(L, oracle_mod):
         assert s.one_minus_beta1 == f32(1) - f32(0.9)
         assert s.one_minus_beta3 == f32(1) - f32(0.9999)
         assert s.inv_bc1 == 1.0 / float(f32(s.bc1)) and s.inv_bc2 == 1.0 / float(f32(s.bc2))
+        for inv, hi, lo in ((s.inv_bc1, s.rcp_bc1_hi, s.rcp_bc1_lo), (s.inv_bc2, s.rcp_bc2_hi, s.rcp_bc2_lo)):
+            assert hi == float(f32(inv)) and lo == float(f32(inv - hi))
+            # the pair carries the reciprocal to about 2^-48 relative
+            assert abs(hi + lo - inv) <= 2.0 ** -47 * inv
         assert (s.lr, s.alpha) == (f32(3e-3), f32(5.0))
 
 

@@ -106,11 +106,19 @@ def test_boundary_sweep_1000_steps(algo, dtype, skip, wd):
 @pytest.mark.usefixtures("testing_lib")
 @pytest.mark.parametrize("mode", [0, 1])
 def test_constant_division_is_exact(mode):
-    """The kernel divides by bc1, bc2 through a binary64 reciprocal; it must
-    equal IEEE division (__fdiv_rn) for every x and every divisor in (0, 1]:
+    """The kernel divides by bc1, bc2 through a precomputed reciprocal (an fp32
+    FMA correction, or binary64 outside |x| in [2^-40, 2^96)); it must equal
+    IEEE division (__fdiv_rn) for every x and every divisor in [2^-25, 1]:
     2^32 random pairs of every class (mode 0) and near rounding boundaries
     (mode 1)."""
     assert B.testing_check_division(0x0E0A0000 + mode, 1 << 32, mode) == 0
+
+
+@pytest.mark.usefixtures("testing_lib")
+def test_constant_division_every_dividend():
+    """The same against every one of the 2^32 binary32 dividends, for 96 seeded
+    divisors (powers of two, all-ones significands and d = 1 among them)."""
+    assert B.testing_check_division(0x0E0A0002, 96, 2) == 0
 
 
 # --------------------------------------------------------------------------
