@@ -444,7 +444,7 @@ class Plan:
 
 
 def fill_step_scalars(hyper: Hyper, first_step: int, count: int) -> bytes:
-    """opt2s_fill_step_scalars: the raw table of `count` steps (64 bytes each),
+    """opt2s_fill_step_scalars: the raw table of `count` steps (80 bytes each),
     ready to be copied to device memory."""
     arr = (opt2s_step_scalars * max(count, 1))()
     check(lib().opt2s_fill_step_scalars(ctypes.byref(hyper), int(first_step), int(count),

@@ -65,31 +65,53 @@ __device__ __forceinline__ void st_global(T* p, const T& v) { *p = v; }
 // (Markstein's theorem: P. Markstein, "Computation of elementary functions on
 // the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990; also
 // Muller et al., ch. 4).  No step overflows or underflows in that range
-// (|x/d| < 2^121).  Four fp32 operations and an exponent test instead of two
-// float/double conversions and a binary64 product: the conversions run on
-// the narrow XU pipe, which limits the compute-heavy kernels.
+// (|x/d| < 2^121).
+// Which route a kernel uses is a measured choice (both are exact): the
+// 32-bit step kernels and the norm pass are fastest with the binary64 route;
+// the 8-bit-state kernel, whose registers are tight, with the fp32 route
+// (the binary64 one then sits out of line, taken for out-of-range x only).
 // GPU tests check both routes against __fdiv_rn: every binary32 x for a
 // sample of divisors, and random operands near rounding boundaries.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float div_by_constant_wide(float x, double r)
+__device__ __forceinline__ float div_by_constant(float x, double r)
 {
     return __double2float_rn(__dmul_rn(static_cast<double>(x), r));
 }
 
-__device__ __forceinline__ float div_by_constant(float x, float d, float hi, float lo, double r)
+__device__ __noinline__ float div_by_constant_far(float x, double r)
+{
+    return div_by_constant(x, r);
+}
+
+__device__ __forceinline__ float div_by_constant_fma(float x, float d, float hi, float lo, double r)
 {
     // biased exponent of |x| in [87, 223): 2^-40 <= |x| < 2^96
     const uint32_t e = __float_as_uint(x) & 0x7F800000u;
-    if (__builtin_expect(e - (87u << 23) >= (136u << 23), 0)) return div_by_constant_wide(x, r);
+    if (__builtin_expect(e - (87u << 23) >= (136u << 23), 0)) return div_by_constant_far(x, r);
     const float q0 = __fmaf_rn(x, hi, __fmul_rn(x, lo));
     const float rem = __fmaf_rn(-q0, d, x);
     return __fmaf_rn(rem, hi, q0);
 }
 
+// m/bc1 and v/bc2 by the route FMA_DIV selects.
+template <bool FMA_DIV>
+__device__ __forceinline__ float div_bc1(float x, const StepScalars& s)
+{
+    return FMA_DIV ? div_by_constant_fma(x, s.bc1, s.rcp_bc1_hi, s.rcp_bc1_lo, s.inv_bc1)
+                   : div_by_constant(x, s.inv_bc1);
+}
+template <bool FMA_DIV>
+__device__ __forceinline__ float div_bc2(float x, const StepScalars& s)
+{
+    return FMA_DIV ? div_by_constant_fma(x, s.bc2, s.rcp_bc2_hi, s.rcp_bc2_lo, s.inv_bc2)
+                   : div_by_constant(x, s.inv_bc2);
+}
+
 // ---------------------------------------------------------------------------
 // The per-element update.  direction() moves the moments of one element (in
 // place) and returns its update direction u = num/den; m/bc1 and v/bc2 use
-// the exact constant division above, num/den is an IEEE division.  update()
+// the exact constant division above (FMA_DIV picks the route), num/den is an
+// IEEE division.  update()
 // then applies the step to p.  With SKIP, an element whose gradient compares
 // equal to zero (+0 or -0) is left untouched (no decay either).  MODE:
 //   kPlain   p = p*decay - lr*u
@@ -100,20 +122,19 @@ __device__ __forceinline__ float div_by_constant(float x, float d, float hi, flo
 // ---------------------------------------------------------------------------
 enum : int { kPlain = 0, kScaled = 1, kLamb = 2 };
 
-template <int ALGO>
+template <int ALGO, bool FMA_DIV = false>
 __device__ __forceinline__ float direction(float g, float& m, float& v, float& m2,
                                            const StepScalars& s)
 {
     m = __fadd_rn(__fmul_rn(s.beta1, m), __fmul_rn(s.one_minus_beta1, g));
     v = __fadd_rn(__fmul_rn(s.beta2, v),
                   __fmul_rn(__fmul_rn(s.one_minus_beta2, g), g));
-    float num = div_by_constant(m, s.bc1, s.rcp_bc1_hi, s.rcp_bc1_lo, s.inv_bc1);
+    float num = div_bc1<FMA_DIV>(m, s);
     if (ALGO == kAdEMAMix) {
         m2 = __fadd_rn(__fmul_rn(s.beta3, m2), __fmul_rn(s.one_minus_beta3, g));
         num = __fadd_rn(num, __fmul_rn(s.alpha, m2));
     }
-    const float den = __fadd_rn(__fsqrt_rn(div_by_constant(v, s.bc2, s.rcp_bc2_hi, s.rcp_bc2_lo,
-                                                                   s.inv_bc2)), s.eps);
+    const float den = __fadd_rn(__fsqrt_rn(div_bc2<FMA_DIV>(v, s)), s.eps);
     return __fdiv_rn(num, den);
 }
 
@@ -123,13 +144,13 @@ __device__ __forceinline__ float lamb_direction(float u, float p, float wd)
     return __fadd_rn(u, __fmul_rn(wd, p));
 }
 
-template <int ALGO, bool SKIP, int MODE = kPlain>
+template <int ALGO, bool SKIP, int MODE = kPlain, bool FMA_DIV = false>
 __device__ __forceinline__ void update(float g, float& p, float& m, float& v,
                                        float& m2, const StepScalars& s, float scale = 1.0f,
                                        float wd = 0.0f)
 {
     if (SKIP && g == 0.0f) return;
-    const float u = direction<ALGO>(g, m, v, m2, s);
+    const float u = direction<ALGO, FMA_DIV>(g, m, v, m2, s);
     if (MODE == kLamb)
         p = __fsub_rn(p, __fmul_rn(s.lr, __fmul_rn(scale, lamb_direction(u, p, wd))));
     else

@@ -52,7 +52,8 @@
 // takes elements 4t..4t+3 and 1024+4t..1024+4t+3, 16-bit storage 8t..8t+7, so
 // that every warp access is contiguous):
 //   1. dequantize: m = map_s[code]*absmax (fp32 product), v with map_u;
-//   2. the plain step's element update (opt2s_device.cuh), param stored;
+//   2. the plain step's element update (opt2s_device.cuh; its fp32 route for
+//      the bias-correction divisions), param stored;
 //   3. the block's new absmax of |m|, v (, |m2|): fmaxf over the thread's
 //      elements, the warp and the CTA's 8 warps (max is exact, so the order
 //      does not matter; NaNs are ignored);
@@ -296,7 +297,7 @@ __device__ __forceinline__ void block8(const Block8Rec& b, const StepScalars& s,
         v[k] = __fmul_rn(mp.umap[code_at(c2, k)], a2);
         m2[k] = ALGO == kAdEMAMix ? __fmul_rn(mp.smap[code_at(c3, k)], a3) : 0.0f;
         if (FULL || elem<V>(k / V, k % V) < len) {
-            update<ALGO, SKIP>(g[k], p[k], m[k], v[k], m2[k], s);
+            update<ALGO, SKIP, kPlain, true>(g[k], p[k], m[k], v[k], m2[k], s);
             x1 = fmaxf(x1, fabsf(m[k]));
             x2 = fmaxf(x2, fabsf(v[k]));
             if (ALGO == kAdEMAMix) x3 = fmaxf(x3, fabsf(m2[k]));

@@ -12,9 +12,10 @@ namespace opt2s {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Validation scaffolding: div_by_constant against __fdiv_rn.  Operands come
-// from the SplitMix64 output function (Steele, Lea & Flood, "Fast splittable
-// pseudorandom number generators", OOPSLA 2014) applied to a counter.
+// Validation scaffolding: both routes of the constant division against
+// __fdiv_rn.  Operands come from the SplitMix64 output function (Steele, Lea
+// & Flood, "Fast splittable pseudorandom number generators", OOPSLA 2014)
+// applied to a counter.
 // Divisors lie in [2^-25, 1], the bias corrections' range: a random binade
 // and significand, with d = 1, powers of two and all-ones significands drawn
 // often.  The reciprocal and its fp32 split are formed as the host forms them.
@@ -47,9 +48,11 @@ __device__ __forceinline__ bool same_quotient(float x, float d)
     const double r = __drcp_rn(static_cast<double>(d));
     const float hi = __double2float_rn(r);
     const float lo = __double2float_rn(__dsub_rn(r, static_cast<double>(hi)));
-    const float a = div_by_constant(x, d, hi, lo, r);
+    const float a = div_by_constant(x, r);                   // binary64 route
+    const float c = div_by_constant_fma(x, d, hi, lo, r);    // fp32 route
     const float b = __fdiv_rn(x, d);
-    return __float_as_uint(a) == __float_as_uint(b) || (isnan(a) && isnan(b));
+    auto same = [](float u, float w) { return __float_as_uint(u) == __float_as_uint(w) || (isnan(u) && isnan(w)); };
+    return same(a, b) && same(c, b);
 }
 
 __global__ void check_division_kernel(uint64_t seed, int64_t n, int mode,

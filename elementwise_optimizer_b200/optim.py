@@ -253,7 +253,8 @@ class TwoStateOptimizer(torch.optim.Optimizer):
         if self.capturable:
             data["plan"] = B.Plan(tl, self.algo)
             dev = ps[0].device if ps else torch.device("cuda")
-            data["table"] = torch.empty(self.table_len * 64, dtype=torch.uint8, device=dev)
+            data["table"] = torch.empty(self.table_len * ctypes.sizeof(B.opt2s_step_scalars),
+                                        dtype=torch.uint8, device=dev)
             data["index"] = torch.zeros(1, dtype=torch.int32, device=dev)
             self._refill(data, group)
         self._group_cache[gi] = data
