@@ -67,9 +67,10 @@ __device__ __forceinline__ void st_global(T* p, const T& v) { *p = v; }
 // Muller et al., ch. 4).  No step overflows or underflows in that range
 // (|x/d| < 2^121).
 // Which route a kernel uses is a measured choice (both are exact): the
-// 32-bit step kernels and the norm pass are fastest with the binary64 route;
-// the 8-bit-state kernel, whose registers are tight, with the fp32 route
-// (the binary64 one then sits out of line, taken for out-of-range x only).
+// binary64 route in the mixed-dtype and AdEMAMix step kernels and in the
+// norm pass; the fp32 route with an inline fallback in the Adam kernel
+// specialised to fp32 storage; the fp32 route with an out-of-line fallback in
+// the 8-bit-state kernel, whose registers are tight.
 // GPU tests check both routes against __fdiv_rn: every binary32 x for a
 // sample of divisors, and random operands near rounding boundaries.
 // ---------------------------------------------------------------------------
@@ -83,34 +84,43 @@ __device__ __noinline__ float div_by_constant_far(float x, double r)
     return div_by_constant(x, r);
 }
 
+// The fp32 route; FAR: the binary64 fallback out of line (a call taken for
+// out-of-range x only) rather than inline.
+template <bool FAR>
 __device__ __forceinline__ float div_by_constant_fma(float x, float d, float hi, float lo, double r)
 {
     // biased exponent of |x| in [87, 223): 2^-40 <= |x| < 2^96
     const uint32_t e = __float_as_uint(x) & 0x7F800000u;
-    if (__builtin_expect(e - (87u << 23) >= (136u << 23), 0)) return div_by_constant_far(x, r);
+    if (__builtin_expect(e - (87u << 23) >= (136u << 23), 0))
+        return FAR ? div_by_constant_far(x, r) : div_by_constant(x, r);
     const float q0 = __fmaf_rn(x, hi, __fmul_rn(x, lo));
     const float rem = __fmaf_rn(-q0, d, x);
     return __fmaf_rn(rem, hi, q0);
 }
 
-// m/bc1 and v/bc2 by the route FMA_DIV selects.
-template <bool FMA_DIV>
+// Routes of m/bc1 and v/bc2: the binary64 product, or the fp32 route with
+// its fallback inline or out of line.
+enum : int { kDivWide = 0, kDivFma = 1, kDivFmaFar = 2 };
+
+template <int ROUTE>
 __device__ __forceinline__ float div_bc1(float x, const StepScalars& s)
 {
-    return FMA_DIV ? div_by_constant_fma(x, s.bc1, s.rcp_bc1_hi, s.rcp_bc1_lo, s.inv_bc1)
-                   : div_by_constant(x, s.inv_bc1);
+    return ROUTE == kDivWide
+               ? div_by_constant(x, s.inv_bc1)
+               : div_by_constant_fma<ROUTE == kDivFmaFar>(x, s.bc1, s.rcp_bc1_hi, s.rcp_bc1_lo, s.inv_bc1);
 }
-template <bool FMA_DIV>
+template <int ROUTE>
 __device__ __forceinline__ float div_bc2(float x, const StepScalars& s)
 {
-    return FMA_DIV ? div_by_constant_fma(x, s.bc2, s.rcp_bc2_hi, s.rcp_bc2_lo, s.inv_bc2)
-                   : div_by_constant(x, s.inv_bc2);
+    return ROUTE == kDivWide
+               ? div_by_constant(x, s.inv_bc2)
+               : div_by_constant_fma<ROUTE == kDivFmaFar>(x, s.bc2, s.rcp_bc2_hi, s.rcp_bc2_lo, s.inv_bc2);
 }
 
 // ---------------------------------------------------------------------------
 // The per-element update.  direction() moves the moments of one element (in
 // place) and returns its update direction u = num/den; m/bc1 and v/bc2 use
-// the exact constant division above (FMA_DIV picks the route), num/den is an
+// the exact constant division above (ROUTE picks the route), num/den is an
 // IEEE division.  update()
 // then applies the step to p.  With SKIP, an element whose gradient compares
 // equal to zero (+0 or -0) is left untouched (no decay either).  MODE:
@@ -122,19 +132,19 @@ __device__ __forceinline__ float div_bc2(float x, const StepScalars& s)
 // ---------------------------------------------------------------------------
 enum : int { kPlain = 0, kScaled = 1, kLamb = 2 };
 
-template <int ALGO, bool FMA_DIV = false>
+template <int ALGO, int ROUTE = kDivWide>
 __device__ __forceinline__ float direction(float g, float& m, float& v, float& m2,
                                            const StepScalars& s)
 {
     m = __fadd_rn(__fmul_rn(s.beta1, m), __fmul_rn(s.one_minus_beta1, g));
     v = __fadd_rn(__fmul_rn(s.beta2, v),
                   __fmul_rn(__fmul_rn(s.one_minus_beta2, g), g));
-    float num = div_bc1<FMA_DIV>(m, s);
+    float num = div_bc1<ROUTE>(m, s);
     if (ALGO == kAdEMAMix) {
         m2 = __fadd_rn(__fmul_rn(s.beta3, m2), __fmul_rn(s.one_minus_beta3, g));
         num = __fadd_rn(num, __fmul_rn(s.alpha, m2));
     }
-    const float den = __fadd_rn(__fsqrt_rn(div_bc2<FMA_DIV>(v, s)), s.eps);
+    const float den = __fadd_rn(__fsqrt_rn(div_bc2<ROUTE>(v, s)), s.eps);
     return __fdiv_rn(num, den);
 }
 
@@ -144,13 +154,13 @@ __device__ __forceinline__ float lamb_direction(float u, float p, float wd)
     return __fadd_rn(u, __fmul_rn(wd, p));
 }
 
-template <int ALGO, bool SKIP, int MODE = kPlain, bool FMA_DIV = false>
+template <int ALGO, bool SKIP, int MODE = kPlain, int ROUTE = kDivWide>
 __device__ __forceinline__ void update(float g, float& p, float& m, float& v,
                                        float& m2, const StepScalars& s, float scale = 1.0f,
                                        float wd = 0.0f)
 {
     if (SKIP && g == 0.0f) return;
-    const float u = direction<ALGO, FMA_DIV>(g, m, v, m2, s);
+    const float u = direction<ALGO, ROUTE>(g, m, v, m2, s);
     if (MODE == kLamb)
         p = __fsub_rn(p, __fmul_rn(s.lr, __fmul_rn(scale, lamb_direction(u, p, wd))));
     else
@@ -311,7 +321,7 @@ __device__ __forceinline__ void store_state(float* b, uint32_t i, const float (&
 // One element through the scalar path (chunk head, tail, or a chunk whose
 // arrays are not mutually 16-byte aligned).  A skipped element is not even
 // written back.
-template <int DT, int ALGO, bool SKIP, int MODE = kPlain>
+template <int DT, int ALGO, bool SKIP, int MODE = kPlain, int ROUTE = kDivWide>
 __device__ __forceinline__ void scalar_element(const ChunkRec& c, uint32_t i,
                                                const StepScalars& s, float scale = 1.0f,
                                                float wd = 0.0f)
@@ -324,7 +334,7 @@ __device__ __forceinline__ void scalar_element(const ChunkRec& c, uint32_t i,
     float v = ld_global(c.v + i);
     float m2 = 0.0f;
     if (ALGO == kAdEMAMix) m2 = ld_global(c.m2 + i);
-    update<ALGO, false, MODE>(g, p, m, v, m2, s, scale, wd);
+    update<ALGO, false, MODE, ROUTE>(g, p, m, v, m2, s, scale, wd);
     P::store1(c.p, i, p);
     st_global(c.m + i, m);
     st_global(c.v + i, v);
@@ -348,7 +358,7 @@ struct Aligned {
 // elements per iteration (two 16-byte vectors of fp32, or one of fp16/bf16),
 // so a warp iteration covers 256 contiguous elements of each array; the mixed
 // case moves one vector per lane per iteration.
-template <int DT, int ALGO, bool SKIP, bool ALL, int MODE = kPlain, int U16 = 1>
+template <int DT, int ALGO, bool SKIP, bool ALL, int MODE = kPlain, int U16 = 1, int ROUTE = kDivWide>
 __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars& s, int lane,
                                             uint32_t head, uint32_t nvec, Aligned al,
                                             float scale = 1.0f, float wd = 0.0f)
@@ -385,7 +395,7 @@ __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars
                 P::widen(praw[u], p);
 #pragma unroll
                 for (int j = 0; j < V; ++j)
-                    update<ALGO, SKIP, MODE>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s, scale, wd);
+                    update<ALGO, SKIP, MODE, ROUTE>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s, scale, wd);
                 P::store(c.p, e, P::narrow(p, praw[u], g, SKIP));
                 store_state_any<V>(c.m, e, ALL || al.m, m[u]);
                 store_state_any<V>(c.v, e, ALL || al.v, v[u]);
@@ -397,7 +407,7 @@ __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars
 
 // One chunk, processed by one warp: a scalar head up to the element at which
 // param is 16-byte aligned, the vector body, and a scalar tail.
-template <int DT, int ALGO, bool SKIP, int MODE = kPlain, int U16 = 1>
+template <int DT, int ALGO, bool SKIP, int MODE = kPlain, int U16 = 1, int ROUTE = kDivWide>
 __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& s, int lane,
                                           float scale = 1.0f, float wd = 0.0f)
 {
@@ -411,16 +421,16 @@ __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& 
     const uint32_t body_end = head + nvec * V;
 
     for (uint32_t i = lane; i < head; i += 32)
-        scalar_element<DT, ALGO, SKIP, MODE>(c, i, s, scale, wd);
+        scalar_element<DT, ALGO, SKIP, MODE, ROUTE>(c, i, s, scale, wd);
     for (uint32_t i = body_end + lane; i < len; i += 32)
-        scalar_element<DT, ALGO, SKIP, MODE>(c, i, s, scale, wd);
+        scalar_element<DT, ALGO, SKIP, MODE, ROUTE>(c, i, s, scale, wd);
 
     const Aligned al{aligned16(c.g, head, P::kBytes), aligned16(c.m, head, 4),
                      aligned16(c.v, head, 4), ALGO != kAdEMAMix || aligned16(c.m2, head, 4)};
     if (al.all())
-        vector_body<DT, ALGO, SKIP, true, MODE, U16>(c, s, lane, head, nvec, al, scale, wd);
+        vector_body<DT, ALGO, SKIP, true, MODE, U16, ROUTE>(c, s, lane, head, nvec, al, scale, wd);
     else
-        vector_body<DT, ALGO, SKIP, false, MODE>(c, s, lane, head, nvec, al, scale, wd);
+        vector_body<DT, ALGO, SKIP, false, MODE, 1, ROUTE>(c, s, lane, head, nvec, al, scale, wd);
 }
 
 // A short 16-bit chunk (its record's dtype carries kShortFlag), processed by

@@ -189,6 +189,10 @@ ShardFn pick_shard(int algo, int skip, int world)
 // take the short-chunk path; otherwise they take the vector path, with the
 // same result (the table-driven kernel does so, which keeps its register
 // count at the plain kernel's).
+// The fp32-only body divides by the bias corrections with the fp32 route
+// (opt2s_device.cuh): measured about 1 % faster than the binary64 route on
+// the 268 M-element fp32 Adam step, where the mixed-dtype and AdEMAMix
+// bodies measured slower with it.
 template <int ALGO, bool SKIP, int ONLY, bool SHORT>
 __device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, int nchunks,
                                           const StepScalars& s)
@@ -200,10 +204,12 @@ __device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, i
     for (int c = warp; c < nchunks; c += nwarps) {
         const ChunkRec rec = chunks[c];
         const bool short16 = SHORT && (rec.dtype & kShortFlag) != 0;
-        if (ONLY >= 0) {
+        if (ONLY == kF32) {
+            run_chunk<kF32, ALGO, SKIP, kPlain, 1, kDivFma>(rec, s, lane);
+        } else if (ONLY >= 0) {
             // one 16-bit dtype: two 16-byte param vectors a lane per iteration
             // (16 elements), the bytes in flight of the fp32 path
-            constexpr int D = ONLY >= 0 ? ONLY : kF16;
+            constexpr int D = ONLY >= 0 && ONLY != kF32 ? ONLY : kF16;
             if (short16) short_chunk<D, ALGO, SKIP>(rec, s, lane);
             else run_chunk<D, ALGO, SKIP, kPlain, 2>(rec, s, lane);
         } else {
@@ -470,12 +476,13 @@ using TableKernelFn = void (*)(const ChunkRec*, int, const StepScalars*, const i
 template <int ALGO, bool SKIP>
 KernelFn pick_only(int only)
 {
+    if (only == kF32) return step_kernel<ALGO, SKIP, kF32>;
     if (only == kF16) return step_kernel<ALGO, SKIP, kF16>;
     if (only == kBF16) return step_kernel<ALGO, SKIP, kBF16>;
     return step_kernel<ALGO, SKIP, -1>;
 }
 
-// Specialised bodies exist for Adam over one 16-bit dtype (measured faster
+// Specialised bodies exist for Adam over one storage dtype (measured faster
 // there); every other combination uses the per-chunk dispatch.
 KernelFn pick(int algo, int skip, int only)
 {
@@ -486,6 +493,7 @@ KernelFn pick(int algo, int skip, int only)
 template <int ALGO, bool SKIP>
 TableKernelFn pick_table_only(int only)
 {
+    if (only == kF32) return step_kernel_table<ALGO, SKIP, kF32>;
     if (only == kF16) return step_kernel_table<ALGO, SKIP, kF16>;
     if (only == kBF16) return step_kernel_table<ALGO, SKIP, kBF16>;
     return step_kernel_table<ALGO, SKIP, -1>;
@@ -498,17 +506,18 @@ TableKernelFn pick_table(int algo, int skip, int only)
     return skip ? pick_table_only<kAdam, true>(only) : pick_table_only<kAdam, false>(only);
 }
 
+constexpr int kOnlyClasses = 4;   // generic, f16, bf16, f32
 int only_class(int algo, int only)
 {
     if (algo == kAdEMAMix) return 0;
-    return only == kF16 ? 1 : (only == kBF16 ? 2 : 0);
+    return only == kF16 ? 1 : (only == kBF16 ? 2 : (only == kF32 ? 3 : 0));
 }
 
 // Resident blocks per SM and SM count, cached per device (and kernel / block
 // size): device attributes are per device, not per process.
 constexpr int kMaxDevices = 64;
 struct OccEntry { int block_threads; int blocks_per_sm; };
-struct DeviceInfo { int sms; OccEntry occ[12][6]; };
+struct DeviceInfo { int sms; OccEntry occ[4 * kOnlyClasses][6]; };
 DeviceInfo g_info[kMaxDevices];
 bool g_info_ok[kMaxDevices];
 std::mutex g_info_mu;   // guards g_info / g_info_ok (host threads may launch concurrently)
@@ -544,7 +553,7 @@ cudaError_t grid_for(int64_t nchunks, int algo, int skip_zeros, int only, int bl
         std::lock_guard<std::mutex> lock(g_info_mu);
         DeviceInfo* info = nullptr;
         if ((e = device_info(dev, &info)) != cudaSuccess) return e;
-        const int k = ((algo == kAdEMAMix ? 2 : 0) + (skip_zeros ? 1 : 0)) * 3 + only_class(algo, only);
+        const int k = ((algo == kAdEMAMix ? 2 : 0) + (skip_zeros ? 1 : 0)) * kOnlyClasses + only_class(algo, only);
         int per_sm = 0;
         for (auto& x : info->occ[k])
             if (x.block_threads == block_threads) per_sm = x.blocks_per_sm;

@@ -297,7 +297,7 @@ __device__ __forceinline__ void block8(const Block8Rec& b, const StepScalars& s,
         v[k] = __fmul_rn(mp.umap[code_at(c2, k)], a2);
         m2[k] = ALGO == kAdEMAMix ? __fmul_rn(mp.smap[code_at(c3, k)], a3) : 0.0f;
         if (FULL || elem<V>(k / V, k % V) < len) {
-            update<ALGO, SKIP, kPlain, true>(g[k], p[k], m[k], v[k], m2[k], s);
+            update<ALGO, SKIP, kPlain, kDivFmaFar>(g[k], p[k], m[k], v[k], m2[k], s);
             x1 = fmaxf(x1, fabsf(m[k]));
             x2 = fmaxf(x2, fabsf(v[k]));
             if (ALGO == kAdEMAMix) x3 = fmaxf(x3, fabsf(m2[k]));

@@ -49,10 +49,11 @@ __device__ __forceinline__ bool same_quotient(float x, float d)
     const float hi = __double2float_rn(r);
     const float lo = __double2float_rn(__dsub_rn(r, static_cast<double>(hi)));
     const float a = div_by_constant(x, r);                   // binary64 route
-    const float c = div_by_constant_fma(x, d, hi, lo, r);    // fp32 route
+    const float c = div_by_constant_fma<false>(x, d, hi, lo, r);    // fp32 route
+    const float f = div_by_constant_fma<true>(x, d, hi, lo, r);     // same, fallback out of line
     const float b = __fdiv_rn(x, d);
     auto same = [](float u, float w) { return __float_as_uint(u) == __float_as_uint(w) || (isnan(u) && isnan(w)); };
-    return same(a, b) && same(c, b);
+    return same(a, b) && same(c, b) && same(f, b);
 }
 
 __global__ void check_division_kernel(uint64_t seed, int64_t n, int mode,
