@@ -70,23 +70,23 @@ struct StepScalars {
 // registers) fits 16 warps either way and measured faster as 256-thread blocks;
 // Adam specialised to one 16-bit dtype moves two 16-byte param vectors a lane
 // per iteration (about 104 registers) and measured fastest as 256-thread
-// blocks; Adam specialised to fp32 storage keeps the generic kernel's
-// 128-thread blocks.  `only` is the dtype every chunk of a plan shares, or -1.
+// blocks.  `only` is the dtype every chunk of a plan shares, or -1.
 constexpr int kAdamBlockThreads = 128;
 constexpr int kAdEMAMixBlockThreads = 256;
 constexpr int kSpecialisedBlockThreads = 256;
 constexpr int kDefaultBlockThreads = 128;      // the no-alloc entry point's width
-// Adam plans whose tensors share one storage dtype run a kernel specialised to
-// it; every other plan runs the per-chunk dispatch (-1).
+// Only Adam over one 16-bit dtype has a specialised kernel.  Kernels
+// specialised to fp32 storage (Adam, 78 registers) and to one dtype for
+// AdEMAMix (80-90 registers) were built and measured slower on 268 M-element
+// steps (4 % and 13 %): they fill more warp slots per SM, and these streaming
+// steps ran faster with fewer.
 inline int kernel_only(int algo, int uniform_dtype)
 {
-    return (algo == kAdam && (uniform_dtype == kF32 || uniform_dtype == kF16 || uniform_dtype == kBF16))
-               ? uniform_dtype
-               : -1;
+    return (algo == kAdam && (uniform_dtype == kF16 || uniform_dtype == kBF16)) ? uniform_dtype : -1;
 }
 inline int default_block_threads(int algo, int only)
 {
-    if (only == kF16 || only == kBF16) return kSpecialisedBlockThreads;
+    if (only >= 0) return kSpecialisedBlockThreads;
     return algo == kAdEMAMix ? kAdEMAMixBlockThreads : kAdamBlockThreads;
 }
 constexpr int64_t kDefaultChunkElems = 2048;   // largest chunk the plan builder picks

@@ -189,10 +189,6 @@ ShardFn pick_shard(int algo, int skip, int world)
 // take the short-chunk path; otherwise they take the vector path, with the
 // same result (the table-driven kernel does so, which keeps its register
 // count at the plain kernel's).
-// The fp32-only body divides by the bias corrections with the fp32 route
-// (opt2s_device.cuh): measured about 1 % faster than the binary64 route on
-// the 268 M-element fp32 Adam step, where the mixed-dtype and AdEMAMix
-// bodies measured slower with it.
 template <int ALGO, bool SKIP, int ONLY, bool SHORT>
 __device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, int nchunks,
                                           const StepScalars& s)
@@ -204,12 +200,10 @@ __device__ __forceinline__ void step_body(const ChunkRec* __restrict__ chunks, i
     for (int c = warp; c < nchunks; c += nwarps) {
         const ChunkRec rec = chunks[c];
         const bool short16 = SHORT && (rec.dtype & kShortFlag) != 0;
-        if (ONLY == kF32) {
-            run_chunk<kF32, ALGO, SKIP, kPlain, 1, kDivFma>(rec, s, lane);
-        } else if (ONLY >= 0) {
+        if (ONLY >= 0) {
             // one 16-bit dtype: two 16-byte param vectors a lane per iteration
             // (16 elements), the bytes in flight of the fp32 path
-            constexpr int D = ONLY >= 0 && ONLY != kF32 ? ONLY : kF16;
+            constexpr int D = ONLY >= 0 ? ONLY : kF16;
             if (short16) short_chunk<D, ALGO, SKIP>(rec, s, lane);
             else run_chunk<D, ALGO, SKIP, kPlain, 2>(rec, s, lane);
         } else {
@@ -278,12 +272,13 @@ __global__ void advance_index_kernel(int* index, int table_len)
 //      p = p*decay - lr*(scale*u), or p = p - lr*(scale*w) for LAMB, the
 //      scale read through the chunk's tensor.
 // The element arithmetic is direction(), as in the plain step.  Every sum
-// has a fixed order: lane l of the warp that owns a block adds the block's
-// elements l, l + 32, l + 64, ... one after the other, the 32 lanes then
-// combine in a fixed shuffle tree, a group's blocks and a tensor's groups are
-// combined in fixed orders too; so the scale does not depend on the plan's
-// chunk length, the block width or the storage alignment.  Accesses are
-// element-wise and contiguous across the warp.
+// has a fixed order: lane l of the warp that owns a block adds the elements
+// of its runs (V consecutive elements at V*l + 32*V*r, V = 4 for fp32 and 8
+// for 16-bit storage) in index order, the 32 lanes then combine in a fixed
+// shuffle tree, a group's blocks and a tensor's groups are combined in fixed
+// orders too; so the scale does not depend on the plan's chunk length, the
+// block width or the storage alignment.  Aligned blocks move each run with
+// one 16-byte access per array.
 //
 // Each lane adds its squares in binary64: the square of a binary32 x is exact
 // in binary64, so one fused multiply-add gives the same sum as a multiply and
@@ -304,31 +299,64 @@ struct SquareSum {
     __device__ __forceinline__ double total() const { return s; }
 };
 
+// One norm block by one warp.  Lane l owns the V-element runs starting at
+// V*l + 32*V*r (r = 0, 1, ...; V = the storage vector's elements: 4 for fp32,
+// 8 for 16-bit storage) and adds their elements in index order, run after
+// run.  When the block's arrays are 16-byte aligned a run is one vector
+// access per array; otherwise its elements are read one by one, in the same
+// lane assignment, so the sums do not depend on the alignment.
 template <int DT, int ALGO, bool SKIP, int MODE>
 __device__ __forceinline__ void norm_block(const ChunkRec& c, const StepScalars& s, int lane,
                                            float wd, double& sd, double& sp)
 {
     using P = Param<DT>;
-    constexpr int K = 8;
+    constexpr int V = P::kVec;
+    constexpr int R = 8 / V;              // runs a lane loads per iteration: 8 elements
+    constexpr int K = R * V;
     const uint32_t len = c.len;
+    const bool vec = aligned16(c.p, 0, P::kBytes) && aligned16(c.g, 0, P::kBytes) &&
+                     aligned16(c.m, 0, 4) && aligned16(c.v, 0, 4) &&
+                     (ALGO != kAdEMAMix || aligned16(c.m2, 0, 4));
     SquareSum ad, ap;
     for (uint32_t base = 0; base < len; base += 32 * K) {
         float g[K], p[K], m[K], v[K], m2[K];
 #pragma unroll
-        for (int k = 0; k < K; ++k) {
-            const uint32_t i = base + lane + 32 * k;
-            g[k] = p[k] = m[k] = v[k] = m2[k] = 0.0f;
-            if (i < len) {
-                g[k] = P::load1(c.g, i);
-                p[k] = P::load1(c.p, i);
-                m[k] = ld_global(c.m + i);
-                v[k] = ld_global(c.v + i);
-                if (ALGO == kAdEMAMix) m2[k] = ld_global(c.m2 + i);
+        for (int r = 0; r < R; ++r) {
+            const uint32_t e0 = base + (r * 32 + lane) * V;
+            if (vec && e0 + V <= len) {
+                float x[V], y[V], a[V], b[V], d[V];
+                P::widen(P::load(c.g, e0), x);
+                P::widen(P::load(c.p, e0), y);
+                load_state<V>(c.m, e0, a);
+                load_state<V>(c.v, e0, b);
+                if (ALGO == kAdEMAMix) load_state<V>(c.m2, e0, d);
+#pragma unroll
+                for (int j = 0; j < V; ++j) {
+                    g[r * V + j] = x[j];
+                    p[r * V + j] = y[j];
+                    m[r * V + j] = a[j];
+                    v[r * V + j] = b[j];
+                    m2[r * V + j] = ALGO == kAdEMAMix ? d[j] : 0.0f;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < V; ++j) {
+                    const uint32_t i = e0 + j;
+                    const int k = r * V + j;
+                    g[k] = p[k] = m[k] = v[k] = m2[k] = 0.0f;
+                    if (i < len) {
+                        g[k] = P::load1(c.g, i);
+                        p[k] = P::load1(c.p, i);
+                        m[k] = ld_global(c.m + i);
+                        v[k] = ld_global(c.v + i);
+                        if (ALGO == kAdEMAMix) m2[k] = ld_global(c.m2 + i);
+                    }
+                }
             }
         }
 #pragma unroll
         for (int k = 0; k < K; ++k) {
-            if (base + lane + 32 * k < len) {
+            if (base + ((k / V) * 32 + lane) * V + (k % V) < len) {
                 ap.add(p[k]);
                 if (!(SKIP && g[k] == 0.0f)) {
                     const float u = direction<ALGO>(g[k], m[k], v[k], m2[k], s);
@@ -476,13 +504,12 @@ using TableKernelFn = void (*)(const ChunkRec*, int, const StepScalars*, const i
 template <int ALGO, bool SKIP>
 KernelFn pick_only(int only)
 {
-    if (only == kF32) return step_kernel<ALGO, SKIP, kF32>;
     if (only == kF16) return step_kernel<ALGO, SKIP, kF16>;
     if (only == kBF16) return step_kernel<ALGO, SKIP, kBF16>;
     return step_kernel<ALGO, SKIP, -1>;
 }
 
-// Specialised bodies exist for Adam over one storage dtype (measured faster
+// Specialised bodies exist for Adam over one 16-bit dtype (measured faster
 // there); every other combination uses the per-chunk dispatch.
 KernelFn pick(int algo, int skip, int only)
 {
@@ -493,7 +520,6 @@ KernelFn pick(int algo, int skip, int only)
 template <int ALGO, bool SKIP>
 TableKernelFn pick_table_only(int only)
 {
-    if (only == kF32) return step_kernel_table<ALGO, SKIP, kF32>;
     if (only == kF16) return step_kernel_table<ALGO, SKIP, kF16>;
     if (only == kBF16) return step_kernel_table<ALGO, SKIP, kBF16>;
     return step_kernel_table<ALGO, SKIP, -1>;
@@ -506,11 +532,11 @@ TableKernelFn pick_table(int algo, int skip, int only)
     return skip ? pick_table_only<kAdam, true>(only) : pick_table_only<kAdam, false>(only);
 }
 
-constexpr int kOnlyClasses = 4;   // generic, f16, bf16, f32
+constexpr int kOnlyClasses = 3;   // generic, f16, bf16
 int only_class(int algo, int only)
 {
     if (algo == kAdEMAMix) return 0;
-    return only == kF16 ? 1 : (only == kBF16 ? 2 : (only == kF32 ? 3 : 0));
+    return only == kF16 ? 1 : (only == kBF16 ? 2 : 0);
 }
 
 // Resident blocks per SM and SM count, cached per device (and kernel / block
