@@ -24,8 +24,7 @@
 //     nothing has to start at zero.  Two calls whose work overlaps on the GPU
 //     (different streams, no ordering between them) race on the table;
 //   * the first call on each device looks up the table's device address
-//     (cudaGetSymbolAddress, with that device current) and caches it; make
-//     that first call before any stream capture begins.
+//     (cudaGetSymbolAddress, with that device current) and caches it.
 
 #include <algorithm>
 #include <cstdint>

@@ -260,8 +260,8 @@ int opt2s_shard_step(const opt2s_shard_desc *desc, const Hyper *hyper, int step,
  * All calls on a device share that array and leave the last call's table in
  * it; every call rewrites what it reads, so nothing must start at zero.  Calls
  * whose work overlaps on the GPU (unordered streams) race on the array.
- * The first call on each device looks up the array's device address and
- * caches it; make that first call before any stream capture begins.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it.
  * Calls from several host threads are serialized.  Each successful call
  * counts one kernel launch.  CUDA failures are kept in opt2s_last_cuda_error.
  */
