@@ -1053,9 +1053,10 @@ def run_roofline_table(numel=268_435_456, steps=50, warmup=10):
 def run_max_unorm(numel=268_435_456, steps=50, warmup=10, max_unorm=1.0):
     """The bounded-update-norm step (opt2s_step_max_unorm: norm sums, scales,
     scaled update) on one tensor of `numel` elements, timed beside the plain
-    step on the same buffers.  Its algorithmic bytes are the plain step's
-    plus one more read of every input (the norm pass reads g, p, m, v
-    [, m2] and writes nothing)."""
+    step on the same buffers, and for Adam the LAMB step (opt2s_step_lamb, the
+    same four launches).  Their algorithmic bytes are the plain step's plus
+    one more read of every input (the norm pass reads g, p, m, v [, m2] and
+    writes nothing)."""
     import torch
     from elementwise_optimizer_b200 import binding as B
     dev = torch.device("cuda")
@@ -1072,9 +1073,11 @@ def run_max_unorm(numel=268_435_456, steps=50, warmup=10, max_unorm=1.0):
         lists = [B.TensorList.from_tensors([p], [g], [s1], [s2]) for g in grads]
         h = B.make_hyper(algo, weight_decay=0.01, beta3=0.9999, alpha=5.0)
         row = {"algo": algo, "dtype": dt, "max_unorm": max_unorm}
-        for name, fn in (("plain", lambda k, t: B.opt2s_step(lists[k % 2], h, t)),
-                         ("max_unorm", lambda k, t: B.opt2s_step_max_unorm(lists[k % 2], h,
-                                                                            max_unorm, t))):
+        legs = [("plain", lambda k, t: B.opt2s_step(lists[k % 2], h, t)),
+                ("max_unorm", lambda k, t: B.opt2s_step_max_unorm(lists[k % 2], h, max_unorm, t))]
+        if algo == "adam":
+            legs.append(("lamb", lambda k, t: B.opt2s_step_lamb(lists[k % 2], h, t)))
+        for name, fn in legs:
             for t in range(1, warmup + 1):
                 fn(t, t)
             torch.cuda.synchronize()
@@ -1085,7 +1088,7 @@ def run_max_unorm(numel=268_435_456, steps=50, warmup=10, max_unorm=1.0):
                 ev[k + 1].record()
             torch.cuda.synchronize()
             ms = sum(ev[k].elapsed_time(ev[k + 1]) for k in range(steps)) / steps
-            per_elem = BYTES_PER_ELEM[(algo, dt)] + (read_bytes[(algo, dt)] if name == "max_unorm" else 0)
+            per_elem = BYTES_PER_ELEM[(algo, dt)] + (read_bytes[(algo, dt)] if name != "plain" else 0)
             gbs = per_elem * numel / (ms / 1e3) / 1e9
             row[name] = {"ms_mean": ms, "bytes_per_elem": per_elem, "gbs": gbs, "frac": gbs / peak}
         row["time_ratio"] = row["max_unorm"]["ms_mean"] / row["plain"]["ms_mean"]
