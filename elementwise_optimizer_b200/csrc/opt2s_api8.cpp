@@ -153,28 +153,34 @@ float float_of(uint32_t u)
     return x;
 }
 
-// Slice i of the map with thresholds `thr`, for x of sign `neg`.
+// Slice i of the map with thresholds `thr`, for x of sign `neg`: the code at
+// the slice's low end (in value order) in the high 16 bits, and in the low 16
+// a value c such that code(x) = (entry + l) >> 16 for l = the low 16 bits of
+// x's magnitude, complemented when x < 0.  With t the low 16 bits of the
+// slice's threshold magnitude: for x >= 0 the code is base + (l > t), and
+// c = 0xFFFF - t makes the carry out of the low half exactly (l > t); for
+// x < 0 it is base + (low16 < t) = base + (l > 0xFFFF - t), and c = t.  A
+// slice without a threshold has c = 0 (never a carry).
 uint32_t slice_entry(const float* thr, uint32_t zero_code, int i, bool neg)
 {
     const int r = i >> 7, k = i & 127;
-    const uint32_t never = neg ? 0u : 0xFFFFu;   // a low-16 compare that never holds
-    if (r == 0) return zero_code << 16 | never;                      // |x| < 2^-23
-    if (r == opt2s::kQuantRows - 1) return never;                    // NaN: code 0
+    if (r == 0) return zero_code << 16;                              // |x| < 2^-23
+    if (r == opt2s::kQuantRows - 1) return 0;                        // NaN: code 0
     const uint32_t lo_bits = static_cast<uint32_t>(r - 1 + 127 - 23) << 23 | static_cast<uint32_t>(k) << 16;
     const float lo = float_of(lo_bits), hi = float_of(lo_bits + (1u << 16));
-    uint32_t t = never;
+    uint32_t c = 0;
     int base;
     if (!neg) {
         // x in [lo, hi): thresholds below lo count; at most one lies in [lo, hi)
         base = thresholds_below(thr, lo, false);
-        if (base < 255 && thr[base] < hi) t = bits_of(thr[base]) & 0xFFFFu;
+        if (base < 255 && thr[base] < hi) c = 0xFFFFu - (bits_of(thr[base]) & 0xFFFFu);
     } else {
         // x in (-hi, -lo]: thresholds at or below -hi count; at most one lies
         // in (-hi, -lo) and counts when |x| is below its magnitude
         base = thresholds_below(thr, -hi, true);
-        if (base < 255 && thr[base] < -lo) t = bits_of(-thr[base]) & 0xFFFFu;
+        if (base < 255 && thr[base] < -lo) c = bits_of(-thr[base]) & 0xFFFFu;
     }
-    return static_cast<uint32_t>(base) << 16 | t;
+    return static_cast<uint32_t>(base) << 16 | c;
 }
 
 }  // namespace

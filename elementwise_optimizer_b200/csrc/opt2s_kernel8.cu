@@ -33,12 +33,14 @@
 // per binade up to 2^0; NaN), the top 7 fraction bits a slice of the row.
 // Every slice is narrower than the gap between two thresholds (the finest,
 // 0.9/128 at the top of the unsigned map, is above the widest slice, 2^-8),
-// so a slice holds at most one threshold, and its 4-byte entry holds the code
-// at the slice's low end in value order (16 bits) and the low 16 bits of that
-// threshold's magnitude (the rest of its bits are the slice's own): the code
-// is base + (low16(x) > t) for x >= 0, base + (low16(x) < t) for x < 0, with
-// t a value that never compares true when the slice has no threshold.  The
-// signed map has a table per sign.
+// so a slice holds at most one threshold; with t the low 16 bits of its
+// magnitude (the rest of its bits are the slice's own), the code is
+// base + (low16(x) > t) for x >= 0 and base + (low16(x) < t) for x < 0, base
+// the code at the slice's low end in value order.  The slice's 4-byte entry
+// holds base in its high half and, in its low half, 0xFFFF - t for x >= 0 or
+// t for x < 0 (0 without a threshold), so that with key = low16(x), or its
+// complement for x < 0, the code is (entry + key) >> 16: one addition whose
+// carry does the comparison.  The signed map has a table per sign.
 // x itself is first taken as RN32(m * RN32(1/absmax)), within 3 ulp of
 // RN32(m/absmax); only when that lies within 4 ulp of the slice's threshold or
 // of a slice boundary (about 12 cases in 65,536) is x recomputed exactly as
@@ -110,40 +112,45 @@ __device__ void load_maps(Maps& mp, const uint4* __restrict__ tables)
     __syncthreads();
 }
 
-// The slice entry of x's bits b: (code at the slice's low end) << 16 | t.
-// The exponent and the top 7 fraction bits, bits 16..30 of b, number the
-// slices of all binades in order; clamping puts every |x| below 2^-23 in
-// slice 0 of the first row and every NaN in the last slice of the NaN row.
+// The slice entry of x's bits b: (code at the slice's low end) << 16 | c
+// (opt2s_api8.cpp, slice_entry).  The exponent and the top 7 fraction bits,
+// bits 16..30 of b, number the slices of all binades in order; clamping puts
+// every |x| below 2^-23 in slice 0 of the first row and every NaN in the last
+// slice of the NaN row.
 template <bool SIGNED>
 __device__ __forceinline__ uint32_t slice_of(const Maps& mp, uint32_t b)
 {
-    int i = static_cast<int>((b >> 16) & 0x7FFFu) - (127 - 24) * 128;
-    i = min(max(i, 0), kSlices - 1);
+    const int i = __vimin_s32_relu(static_cast<int>((b >> 16) & 0x7FFFu) - (127 - 24) * 128, kSlices - 1);
     return SIGNED ? mp.stab[b >> 31][i] : mp.utab[i];
 }
 
-__device__ __forceinline__ uint32_t code_in(uint32_t q, uint32_t b, bool neg)
+// The low 16 bits of x's magnitude as the slice entries expect them: as they
+// are for x >= 0, complemented for x < 0 (signed map only).  The code is then
+// (entry + key) >> 16: the carry out of the low half adds the threshold.
+template <bool SIGNED>
+__device__ __forceinline__ uint32_t low_key(uint32_t b)
 {
-    const uint32_t lo16 = b & 0xFFFFu, t = q & 0xFFFFu;
-    return (q >> 16) + (neg ? (lo16 < t ? 1u : 0u) : (lo16 > t ? 1u : 0u));
+    return SIGNED ? (b ^ static_cast<uint32_t>(static_cast<int32_t>(b) >> 31)) & 0xFFFFu : b & 0xFFFFu;
 }
 
 // Code of the map value nearest to m/absmax (absmax > 0; r32 = RN32(1/absmax),
 // r64 = RN64(1/absmax)).  The fast quotient RN32(m*r32) is within 3 ulp of
-// RN32(m/absmax); when its low 16 bits lie within 4 of the slice's threshold
-// or of a slice boundary, the exact quotient decides.  (A slice without a
-// threshold holds 0 or 0xFFFF there, which only adds boundary cases.)
+// RN32(m/absmax); when its key lies within 4 of the slice's threshold or of a
+// slice boundary, the exact quotient decides.  With sum = entry + key,
+// (sum + 5) mod 2^16 <= 8 exactly when the key is within 4 of the threshold
+// (a slice without one only adds boundary cases).
 template <bool SIGNED>
 __device__ __forceinline__ uint32_t quantize(const Maps& mp, float m, float r32, double r64)
 {
     uint32_t b = __float_as_uint(__fmul_rn(m, r32));
-    uint32_t q = slice_of<SIGNED>(mp, b);
-    const uint32_t lo4 = (b & 0xFFFFu) + 4u;
-    if (lo4 - (q & 0xFFFFu) <= 8u || (lo4 & 0xFFFFu) < 8u) {
+    uint32_t key = low_key<SIGNED>(b);
+    uint32_t sum = slice_of<SIGNED>(mp, b) + key;
+    if (((sum + 5u) & 0xFFFFu) <= 8u || ((key + 4u) & 0xFFFFu) < 8u) {
         b = __float_as_uint(__double2float_rn(__dmul_rn(static_cast<double>(m), r64)));
-        q = slice_of<SIGNED>(mp, b);
+        key = low_key<SIGNED>(b);
+        sum = slice_of<SIGNED>(mp, b) + key;
     }
-    return code_in(q, b, SIGNED && (b >> 31));
+    return sum >> 16;
 }
 
 __device__ __forceinline__ float warp_max(float x)

@@ -4,9 +4,12 @@ The kernel finds the code of the map value nearest to x without a search:
 the exponent of x picks a row (below 2^-23, where the nearest value is 0;
 one row per binade up to 2^0; NaN), the top 7 fraction bits a slice of the
 row; every slice holds at most one threshold between neighbouring map
-values, and its entry gives the code at the slice's low end (in value order)
-and the low 16 bits of that threshold's magnitude, compared with the low 16
-bits of x (greater for x >= 0, smaller for x < 0; a table per sign).  These
+values, t the low 16 bits of its magnitude.  The code is the code at the
+slice's low end (in value order) plus (low16(x) > t) for x >= 0 or
+(low16(x) < t) for x < 0; the entry stores that base in its high half and
+0xFFFF - t (x >= 0) or t (x < 0) in its low half, so that the code is
+(entry + key) >> 16 with key = low16(x), complemented for x < 0 (a table per
+sign; 0 in the low half of a slice without a threshold).  These
 tests rebuild that rule from the pinned oracle map and check its premises
 and its result against the oracle's brute-force nearest code, over random
 values, every threshold and its neighbours, and exact ties.  They also check
@@ -32,30 +35,29 @@ def _bits(x):
 
 def _table(qmap, neg):
     thr = _thresholds(qmap)
-    never = 0 if neg else 0xFFFF
     zero = int(np.nonzero(qmap == 0)[0][0])
     tab = []
     for i in range(ROWS * 128):
         r, k = divmod(i, 128)
         if r == 0:
-            tab.append((zero << 16) | never)
+            tab.append(zero << 16)
             continue
         if r == ROWS - 1:
-            tab.append(never)
+            tab.append(0)
             continue
         lo_bits = ((r - 1 + 127 - 23) << 23) | (k << 16)
         lo = np.uint32(lo_bits).view(np.float32)
         hi = np.uint32(lo_bits + (1 << 16)).view(np.float32)
-        t = never
+        c = 0
         if not neg:
             base = int(np.searchsorted(thr, lo, side="left"))        # thresholds < lo
             if base < 255 and thr[base] < hi:
-                t = _bits(thr[base]) & 0xFFFF
+                c = 0xFFFF - (_bits(thr[base]) & 0xFFFF)
         else:
             base = int(np.searchsorted(thr, -hi, side="right"))      # thresholds <= -hi
             if base < 255 and thr[base] < -lo:
-                t = _bits(-thr[base]) & 0xFFFF
-        tab.append((base << 16) | t)
+                c = _bits(-thr[base]) & 0xFFFF
+        tab.append((base << 16) | c)
     return tab
 
 
@@ -80,8 +82,8 @@ def _code(tabs, x, signed):
         i = (r << 7) | ((b >> 16) & 0x7F)
         neg = signed and (b >> 31) == 1
         q = tabs[1 if neg else 0][i]
-        lo16, t = b & 0xFFFF, q & 0xFFFF
-        out.append((q >> 16) + (int(lo16 < t) if neg else int(lo16 > t)))
+        key = (b & 0xFFFF) ^ (0xFFFF if neg else 0)
+        out.append((q + key) >> 16)
     return np.array(out, np.uint8)
 
 
@@ -137,3 +139,51 @@ def test_library_tables_are_the_rule(oracle_mod):
     assert np.array_equal(spos, np.array(_table(qs, False), np.uint32))
     assert np.array_equal(sneg, np.array(_table(qs, True), np.uint32))
     assert np.array_equal(upos, np.array(_table(qu, False), np.uint32))
+
+
+def _device_code(tabs, m, n, signed):
+    """The kernel's decision, restated: the code of the fast quotient
+    RN32(m * RN32(1/n)) unless its key lies within 4 of the slice's threshold
+    or of a slice boundary, else the code of the exact quotient."""
+    fast = (m * (np.float32(1) / n)).astype(np.float32)
+    exact = (m.astype(np.float64) / n.astype(np.float64)).astype(np.float32)
+    out = []
+    for f, e in zip(fast, exact):
+        b = _bits(f)
+        r = min(max(((b >> 23) & 0xFF) - (127 - 24), 0), ROWS - 1)
+        neg = signed and (b >> 31) == 1
+        q = tabs[1 if neg else 0][(r << 7) | ((b >> 16) & 0x7F)]
+        key = (b & 0xFFFF) ^ (0xFFFF if neg else 0)
+        s = q + key
+        if ((s + 5) & 0xFFFF) <= 8 or ((key + 4) & 0xFFFF) < 8:
+            out.append(int(_code(tabs, np.array([e], np.float32), signed)[0]))
+        else:
+            out.append(s >> 16)
+    return np.array(out, np.uint8), exact
+
+
+@pytest.mark.parametrize("signed", [True, False])
+def test_fast_quotient_with_decision_test_gives_the_exact_code(oracle_mod, signed):
+    """Over random (m, absmax) pairs and pairs whose exact quotient lands on,
+    next to, or within a few ulp of every threshold, the kernel's fast path
+    with its decision test gives the nearest code of RN32(m / absmax)."""
+    qmap = oracle_mod.quant_map(signed)
+    tabs = (_table(qmap, False), _table(qmap, True))
+    thr = _thresholds(qmap)
+    g = np.random.Generator(np.random.Philox(79))
+    n = (10.0 ** g.uniform(-20, 20, 20_000)).astype(np.float32)
+    lo = -1.0 if signed else 0.0
+    m = (n * g.uniform(lo, 1, n.size).astype(np.float32)).astype(np.float32)
+    # quotients at the thresholds: m = RN32(T * n) for every threshold T (and its negative),
+    # then nudged by up to 3 ulp of m
+    t_all = np.concatenate([thr, -thr]) if signed else thr
+    nt = (10.0 ** g.uniform(-20, 20, t_all.size)).astype(np.float32)
+    mt = (t_all.astype(np.float64) * nt.astype(np.float64)).astype(np.float32)
+    steps = g.integers(-3, 4, mt.size)
+    mt = np.array([np.float32(x).view(np.int32) + int(k) for x, k in zip(mt, steps)], np.int32).view(np.float32)
+    m = np.concatenate([m, mt])
+    n = np.concatenate([n, nt])
+    keep = np.isfinite(m) & (np.abs(m) <= n)
+    m, n = m[keep], n[keep]
+    codes, exact = _device_code(tabs, m, n, signed)
+    assert np.array_equal(codes, oracle_mod.quantize(qmap, exact))
