@@ -199,9 +199,36 @@ __device__ __forceinline__ void load_codes(const uint8_t* q, uint32_t len, bool 
     }
 }
 
+// Byte k & 3 of word k >> 2, zero-extended (one byte permute).
 __device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[2], int k)
 {
-    return (w[k >> 2] >> (8 * (k & 3))) & 0xFFu;
+    return __byte_perm(w[k >> 2], 0u, 0x4440u | static_cast<uint32_t>(k & 3));
+}
+
+// Four codes (each < 256) packed into one word, c0 in the lowest byte.
+__device__ __forceinline__ uint32_t pack4(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3)
+{
+    return __byte_perm(__byte_perm(c0, c1, 0x0040u), __byte_perm(c2, c3, 0x0040u), 0x5410u);
+}
+
+// The codes of a thread's eight values x[] of one state, packed as the code
+// arrays store them (zero_code for all when the block's absmax is 0).
+template <bool SIGNED>
+__device__ __forceinline__ void quantize8(const Maps& mp, const float (&x)[kB8PerThread], float absmax,
+                                          uint32_t zero_code, uint32_t (&w)[2])
+{
+    if (absmax > 0.0f) {
+        // RN32 reciprocal for the fast quotient, RN64 for the exact one
+        const float r32 = __frcp_rn(absmax);
+        const double r64 = __drcp_rn(static_cast<double>(absmax));
+        uint32_t c[kB8PerThread];
+#pragma unroll
+        for (int k = 0; k < kB8PerThread; ++k) c[k] = quantize<SIGNED>(mp, x[k], r32, r64);
+        w[0] = pack4(c[0], c[1], c[2], c[3]);
+        w[1] = pack4(c[4], c[5], c[6], c[7]);
+    } else {
+        w[0] = w[1] = zero_code * 0x01010101u;
+    }
 }
 
 template <int V>
@@ -351,23 +378,9 @@ __device__ __forceinline__ void block8(const Block8Rec& b, const StepScalars& s,
         b.a2[0] = n2;
         if (ALGO == kAdEMAMix) b.a3[0] = n3;
     }
-    // reciprocals of the new absmaxes: RN32 for the fast quotient, RN64 for
-    // the exact one
-    const double i1 = n1 > 0.0f ? __drcp_rn(static_cast<double>(n1)) : 0.0;
-    const double i2 = n2 > 0.0f ? __drcp_rn(static_cast<double>(n2)) : 0.0;
-    const double i3 = (ALGO == kAdEMAMix && n3 > 0.0f) ? __drcp_rn(static_cast<double>(n3)) : 0.0;
-    const float f1 = n1 > 0.0f ? __frcp_rn(n1) : 0.0f;
-    const float f2 = n2 > 0.0f ? __frcp_rn(n2) : 0.0f;
-    const float f3 = (ALGO == kAdEMAMix && n3 > 0.0f) ? __frcp_rn(n3) : 0.0f;
-    c1[0] = c1[1] = c2[0] = c2[1] = c3[0] = c3[1] = 0u;
-#pragma unroll
-    for (int k = 0; k < kB8PerThread; ++k) {
-        const int sh = 8 * (k & 3);
-        c1[k >> 2] |= (n1 > 0.0f ? quantize<true>(mp, m[k], f1, i1) : kZeroSigned) << sh;
-        c2[k >> 2] |= (n2 > 0.0f ? quantize<false>(mp, v[k], f2, i2) : kZeroUnsigned) << sh;
-        if (ALGO == kAdEMAMix)
-            c3[k >> 2] |= (n3 > 0.0f ? quantize<true>(mp, m2[k], f3, i3) : kZeroSigned) << sh;
-    }
+    quantize8<true>(mp, m, n1, kZeroSigned, c1);
+    quantize8<false>(mp, v, n2, kZeroUnsigned, c2);
+    if (ALGO == kAdEMAMix) quantize8<true>(mp, m2, n3, kZeroSigned, c3);
     store_codes<V>(b.q1, len, vec, c1);
     store_codes<V>(b.q2, len, vec, c2);
     if (ALGO == kAdEMAMix) store_codes<V>(b.q3, len, vec, c3);
