@@ -57,8 +57,9 @@
 //   2. the plain step's element update (opt2s_device.cuh; its fp32 route for
 //      the bias-correction divisions), param stored;
 //   3. the block's new absmax of |m|, v (, |m2|): fmaxf over the thread's
-//      elements, the warp and the CTA's 8 warps (max is exact, so the order
-//      does not matter; NaNs are ignored);
+//      elements (NaNs are ignored), then an unsigned maximum of the bit
+//      patterns over the warp (one warp reduction) and the CTA's 8 warps
+//      (max is exact, so the order does not matter);
 //   4. quantize each value with the block's new absmax, or store the code of
 //      0 when it is 0; thread 0 stores the new absmaxes.
 // With skip_zeros an element whose gradient is zero keeps its param and its
@@ -94,7 +95,7 @@ struct Maps {
     float smap[256], umap[256];          // signed (m, m2) and unsigned (v) maps
     uint32_t stab[2][kSlices];           // slices of the signed map, x >= 0 and x < 0
     uint32_t utab[kSlices];              // slices of the unsigned map
-    float red[2][3][kB8Threads / 32];    // per-warp maxima, double-buffered
+    alignas(16) uint32_t red[2][3][kB8Threads / 32];   // per-warp maxima (bits), double-buffered
 };
 constexpr size_t kMapsBytes = sizeof(Maps);
 
@@ -153,11 +154,20 @@ __device__ __forceinline__ uint32_t quantize(const Maps& mp, float m, float r32,
     return sum >> 16;
 }
 
-__device__ __forceinline__ float warp_max(float x)
+// The maximum over the warp of a value that is >= +0 and not NaN: such
+// binary32 values order like their bit patterns as unsigned integers, so one
+// warp reduction on the bits gives it (the result as bits).
+__device__ __forceinline__ uint32_t warp_max_bits(float x)
 {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
-    return x;
+    return __reduce_max_sync(0xffffffffu, __float_as_uint(x));
+}
+
+// The maximum of the eight per-warp maxima (bits, as above) of one quantity.
+__device__ __forceinline__ float block_max(const uint32_t (&r)[kB8Threads / 32])
+{
+    const uint4 a = *reinterpret_cast<const uint4*>(&r[0]);
+    const uint4 b = *reinterpret_cast<const uint4*>(&r[4]);
+    return __uint_as_float(max(__vimax3_u32(a.x, a.y, a.z), __vimax3_u32(a.w, b.x, __vimax3_u32(b.y, b.z, b.w))));
 }
 
 // Element j of run u of this thread (runs of V elements, one storage vector
@@ -356,22 +366,17 @@ __device__ __forceinline__ void block8(const Block8Rec& b, const StepScalars& s,
     }
 
     // the block's new absmaxes
-    x1 = warp_max(x1);
-    x2 = warp_max(x2);
-    if (ALGO == kAdEMAMix) x3 = warp_max(x3);
+    // (x1, x2, x3 are >= +0 and never NaN: fmaxf from +0 skips NaN)
+    const uint32_t w1 = warp_max_bits(x1), w2 = warp_max_bits(x2);
+    const uint32_t w3 = ALGO == kAdEMAMix ? warp_max_bits(x3) : 0u;
     if (lane == 0) {
-        mp.red[buf][0][warp] = x1;
-        mp.red[buf][1][warp] = x2;
-        mp.red[buf][2][warp] = x3;
+        mp.red[buf][0][warp] = w1;
+        mp.red[buf][1][warp] = w2;
+        mp.red[buf][2][warp] = w3;
     }
     __syncthreads();
-    float n1 = 0.0f, n2 = 0.0f, n3 = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kB8Threads / 32; ++w) {
-        n1 = fmaxf(n1, mp.red[buf][0][w]);
-        n2 = fmaxf(n2, mp.red[buf][1][w]);
-        n3 = fmaxf(n3, mp.red[buf][2][w]);
-    }
+    const float n1 = block_max(mp.red[buf][0]), n2 = block_max(mp.red[buf][1]);
+    const float n3 = ALGO == kAdEMAMix ? block_max(mp.red[buf][2]) : 0.0f;
     // every thread has read the old absmaxes (before the barrier)
     if (threadIdx.x == 0) {
         b.a1[0] = n1;
