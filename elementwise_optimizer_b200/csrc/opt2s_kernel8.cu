@@ -79,10 +79,11 @@ namespace {
 constexpr int kB8Threads = 256;                  // one CTA per 8-bit block
 // Resident CTAs per SM the registers must allow: the kernel waits on loads
 // and on its barrier, so more resident CTAs measured faster (Adam: 4 CTAs at
-// 64 registers beat 3 at 80 and 2 at 128; AdEMAMix, with a third state,
-// measured best at 3).  Each CTA also prefetches its next block into L2.
+// 64 registers beat 3 at 80, 2 at 128 and 5 at 48, which spills; AdEMAMix, with
+// a third state, 4 at 64 registers and a few spilled bytes beat 3 at 80 by
+// 1 %).  Each CTA also prefetches its next block into L2.
 template <int ALGO>
-constexpr int kB8MinCtas = ALGO == kAdEMAMix ? 3 : 4;
+constexpr int kB8MinCtas = 4;
 constexpr int kB8PerThread = kBlock8Elems / kB8Threads;
 static_assert(kB8PerThread == 8, "eight elements a thread");
 
