@@ -118,12 +118,20 @@ __device__ void load_maps(Maps& mp, const uint4* __restrict__ tables)
 // (opt2s_api8.cpp, slice_entry).  The exponent and the top 7 fraction bits,
 // bits 16..30 of b, number the slices of all binades in order; clamping puts
 // every |x| below 2^-23 in slice 0 of the first row and every NaN in the last
-// slice of the NaN row.
+// slice of the NaN row.  The signed map's table follows the sign (the second
+// table for x < 0).  The unsigned map is indexed with the sign bit left in:
+// any x with it set (-0, -NaN; v is never negative otherwise) clamps to the
+// NaN row, whose code 0 is also the nearest code of every x <= 0 there.
 template <bool SIGNED>
 __device__ __forceinline__ uint32_t slice_of(const Maps& mp, uint32_t b)
 {
-    const int i = __vimin_s32_relu(static_cast<int>((b >> 16) & 0x7FFFu) - (127 - 24) * 128, kSlices - 1);
-    return SIGNED ? mp.stab[b >> 31][i] : mp.utab[i];
+    constexpr int kLow = (127 - 24) * 128;    // slice number of 2^-23
+    if (SIGNED) {
+        const int i = __vimin_s32_relu(static_cast<int>((b >> 16) & 0x7FFFu) - kLow, kSlices - 1);
+        const uint32_t other = static_cast<uint32_t>(static_cast<int32_t>(b) >> 31) & kSlices;
+        return (&mp.stab[0][0])[i + other];       // the two tables are contiguous
+    }
+    return mp.utab[__vimin_s32_relu(static_cast<int>(b >> 16) - kLow, kSlices - 1)];
 }
 
 // The low 16 bits of x's magnitude as the slice entries expect them: as they
@@ -135,19 +143,21 @@ __device__ __forceinline__ uint32_t low_key(uint32_t b)
     return SIGNED ? (b ^ static_cast<uint32_t>(static_cast<int32_t>(b) >> 31)) & 0xFFFFu : b & 0xFFFFu;
 }
 
-// Code of the map value nearest to m/absmax (absmax > 0; r32 = RN32(1/absmax),
-// r64 = RN64(1/absmax)).  The fast quotient RN32(m*r32) is within 3 ulp of
-// RN32(m/absmax); when its key lies within 4 of the slice's threshold or of a
-// slice boundary, the exact quotient decides.  With sum = entry + key,
+// Code of the map value nearest to m/absmax (absmax > 0, r32 = RN32(1/absmax)).
+// The fast quotient RN32(m*r32) is within 3 ulp of RN32(m/absmax); when its
+// key lies within 4 of the slice's threshold or of a slice boundary, the exact
+// quotient RN32(RN64(m * RN64(1/absmax))) decides (the binary64 reciprocal is
+// formed there, on that rare path only).  With sum = entry + key,
 // (sum + 5) mod 2^16 <= 8 exactly when the key is within 4 of the threshold
 // (a slice without one only adds boundary cases).
 template <bool SIGNED>
-__device__ __forceinline__ uint32_t quantize(const Maps& mp, float m, float r32, double r64)
+__device__ __forceinline__ uint32_t quantize(const Maps& mp, float m, float r32, float absmax)
 {
     uint32_t b = __float_as_uint(__fmul_rn(m, r32));
     uint32_t key = low_key<SIGNED>(b);
     uint32_t sum = slice_of<SIGNED>(mp, b) + key;
     if (((sum + 5u) & 0xFFFFu) <= 8u || ((key + 4u) & 0xFFFFu) < 8u) {
+        const double r64 = __drcp_rn(static_cast<double>(absmax));
         b = __float_as_uint(__double2float_rn(__dmul_rn(static_cast<double>(m), r64)));
         key = low_key<SIGNED>(b);
         sum = slice_of<SIGNED>(mp, b) + key;
@@ -229,12 +239,10 @@ __device__ __forceinline__ void quantize8(const Maps& mp, const float (&x)[kB8Pe
                                           uint32_t zero_code, uint32_t (&w)[2])
 {
     if (absmax > 0.0f) {
-        // RN32 reciprocal for the fast quotient, RN64 for the exact one
-        const float r32 = __frcp_rn(absmax);
-        const double r64 = __drcp_rn(static_cast<double>(absmax));
+        const float r32 = __frcp_rn(absmax);     // for the fast quotient
         uint32_t c[kB8PerThread];
 #pragma unroll
-        for (int k = 0; k < kB8PerThread; ++k) c[k] = quantize<SIGNED>(mp, x[k], r32, r64);
+        for (int k = 0; k < kB8PerThread; ++k) c[k] = quantize<SIGNED>(mp, x[k], r32, absmax);
         w[0] = pack4(c[0], c[1], c[2], c[3]);
         w[1] = pack4(c[4], c[5], c[6], c[7]);
     } else {

@@ -74,12 +74,19 @@ def _inside_counts(qmap):
     return counts
 
 
+def _slice(b, signed):
+    """The kernel's slice number of x's bits b: the exponent and the top 7
+    fraction bits, clamped to the table; the unsigned map keeps the sign bit
+    in, so any x with it set lands in the last (NaN) slice."""
+    top = (b >> 16) & 0x7FFF if signed else b >> 16
+    return min(max(top - (127 - 24) * 128, 0), ROWS * 128 - 1)
+
+
 def _code(tabs, x, signed):
     out = []
     for v in np.asarray(x, np.float32):
         b = _bits(v)
-        r = min(max(((b >> 23) & 0xFF) - (127 - 24), 0), ROWS - 1)
-        i = (r << 7) | ((b >> 16) & 0x7F)
+        i = _slice(b, signed)
         neg = signed and (b >> 31) == 1
         q = tabs[1 if neg else 0][i]
         key = (b & 0xFFFF) ^ (0xFFFF if neg else 0)
@@ -104,7 +111,8 @@ def test_slice_rule_gives_the_nearest_code(oracle_mod, signed):
     lo = -1.0 if signed else 0.0
     xs = [g.uniform(lo, 1.0, 3000), np.sign(g.uniform(lo, 1.0, 3000)) * 10.0 ** g.uniform(-9, 0, 3000),
           qmap, thr, np.nextafter(thr, np.float32(2)), np.nextafter(thr, np.float32(-2)),
-          np.array([0.0, 1.0, 2.0 ** -23, np.nextafter(np.float32(2.0 ** -23), np.float32(0)), np.nan])]
+          np.array([0.0, -0.0, 1.0, 2.0 ** -23, np.nextafter(np.float32(2.0 ** -23), np.float32(0)), np.nan,
+                    -np.nan])]
     if signed:
         xs += [-thr, -np.nextafter(thr, np.float32(2)), -qmap, np.array([-1.0, -(2.0 ** -23), -0.0])]
     x = np.concatenate([np.asarray(a, np.float64) for a in xs]).astype(np.float32)
@@ -150,9 +158,8 @@ def _device_code(tabs, m, n, signed):
     out = []
     for f, e in zip(fast, exact):
         b = _bits(f)
-        r = min(max(((b >> 23) & 0xFF) - (127 - 24), 0), ROWS - 1)
         neg = signed and (b >> 31) == 1
-        q = tabs[1 if neg else 0][(r << 7) | ((b >> 16) & 0x7F)]
+        q = tabs[1 if neg else 0][_slice(b, signed)]
         key = (b & 0xFFFF) ^ (0xFFFF if neg else 0)
         s = q + key
         if ((s + 5) & 0xFFFF) <= 8 or ((key + 4) & 0xFFFF) < 8:
