@@ -285,9 +285,10 @@ __global__ void advance_index_kernel(int* index, int table_len)
 // an add.  (A double-float lane sum -- two binary32 numbers, TwoProduct and
 // TwoSum on the fp32 pipe -- avoids the float-to-double conversions but
 // measured slower on B200: more instructions per element.)  The partials
-// kernel is limited to 64 registers per thread, 4 CTAs of 256 threads per
-// SM: the extra resident warps hide more of the load latency, and measured
-// faster than 3 CTAs at 80 registers.
+// kernel is limited to 64 registers per thread for Adam, 4 CTAs of 256
+// threads per SM: the extra resident warps hide more of the load latency,
+// and measured faster than 3 CTAs at 80 registers.  AdEMAMix, with a third
+// state array, spills at 64 and measured 0.6 % faster at 3 CTAs.
 // ---------------------------------------------------------------------------
 struct SquareSum {
     double s = 0.0;
@@ -381,7 +382,7 @@ __device__ __forceinline__ void warp_tree_sum(double& a, double& b)
 constexpr int kNormThreads = 256;
 
 template <int ALGO, bool SKIP, int MODE>
-__global__ void __launch_bounds__(kNormThreads, 4) unorm_partials_kernel(const ChunkRec* __restrict__ blocks, int nblocks,
+__global__ void __launch_bounds__(kNormThreads, ALGO == kAdEMAMix ? 3 : 4) unorm_partials_kernel(const ChunkRec* __restrict__ blocks, int nblocks,
                                       StepScalars s, float wd, double2* __restrict__ partial)
 {
     const int lane = threadIdx.x & 31;
