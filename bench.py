@@ -907,9 +907,10 @@ def run_direct_cells(rounds=7, samples=200, warmup=20):
 def run_eager_collection(rounds=7, steps=50, warmup=20):
     """optimizer.step() on a fixed collection: the 2,000 bias/norm/LoRA-like
     tensors (64..1,024 elements, fp32/bf16/fp16) plus 64 tensors of 4,096..
-    65,536 elements.  Wall time per step (host dispatch included, GPU drained
-    at the end of each batch); a captured CUDA graph of the same step as a
-    diagnostic control; torch.optim.AdamW(fused=True) for context."""
+    65,536 elements (the ones the 8-bit classes keep in 8-bit state).  Wall
+    time per step (host dispatch included, GPU drained at the end of each
+    batch); a captured CUDA graph of the same step as a diagnostic control;
+    torch.optim.AdamW(fused=True) for context."""
     import torch
     from elementwise_optimizer_b200 import optim, synth
     dev = torch.device("cuda")
@@ -944,6 +945,8 @@ def run_eager_collection(rounds=7, steps=50, warmup=20):
            "rounds": rounds, "steps_per_round": steps}
     for name, cls, kw in (("AdamW32bit", optim.AdamW32bit, {}),
                           ("AdEMAMix32bit", optim.AdEMAMix32bit, {}),
+                          ("AdamW8bit", optim.AdamW8bit, {}),
+                          ("AdEMAMix8bit", optim.AdEMAMix8bit, {}),
                           ("AdamW32bit_flatten", optim.AdamW32bit, dict(flatten=True)),
                           ("AdEMAMix32bit_flatten", optim.AdEMAMix32bit, dict(flatten=True))):
         res[name] = timed(cls(make(), lr=1e-4, **kw).step)

@@ -36,9 +36,11 @@ inline void* start_of(const c10::TensorImpl* t)
     return static_cast<char*>(t->storage().data_ptr().get()) + t->storage_offset() * t->itemsize();
 }
 
-// Whether a parameter and its gradient still fit record r: both defined,
-// dense, contiguous CUDA tensors of the record's element count and dtype.
-inline bool fits(const c10::TensorImpl* p, const c10::TensorImpl* g, const opt2s_tensor& r)
+// Whether a parameter and its gradient still fit record r (opt2s_tensor or
+// opt2s_tensor8): both defined, dense, contiguous CUDA tensors of the
+// record's element count and dtype.
+template <typename Rec>
+inline bool fits(const c10::TensorImpl* p, const c10::TensorImpl* g, const Rec& r)
 {
     return p->layout() == c10::kStrided && g->layout() == c10::kStrided &&
            p->is_cuda() && g->is_cuda() && p->is_contiguous() && g->is_contiguous() &&
@@ -55,18 +57,20 @@ inline const c10::TensorImpl* grad_of(const at::Tensor& p)
     return meta->grad_.unsafeGetTensorImpl();
 }
 
-// Refreshes the param and grad addresses of the `n` opt2s_tensor records at
-// address `records` from the tensors of `params` (record i <-> params[i]).
-// Returns 0 when no address changed, 1 when some did (the records now hold
-// the new ones), and -1 when a parameter has no gradient or no longer fits its
-// record (element count, storage dtype, contiguity, CUDA placement): the
-// caller then rebuilds its records.  The records are untouched on -1.
-// One pass checks every tensor and compares its addresses; only when an
-// address changed does a second pass, from the first change, write them.
-int64_t refresh_records(py::list params, uintptr_t records, int64_t n)
+// Refreshes the param and grad addresses of the `n` records (Rec:
+// opt2s_tensor or opt2s_tensor8) at address `records` from the tensors of
+// `params` (record i <-> params[i]).  Returns 0 when no address changed, 1
+// when some did (the records now hold the new ones), and -1 when a parameter
+// has no gradient or no longer fits its record (element count, storage
+// dtype, contiguity, CUDA placement): the caller then rebuilds its records.
+// The records are untouched on -1.  One pass checks every tensor and
+// compares its addresses; only when an address changed does a second pass,
+// from the first change, write them.
+template <typename Rec>
+int64_t refresh(py::list params, uintptr_t records, int64_t n)
 {
     if (static_cast<int64_t>(py::len(params)) != n) return -1;
-    auto* rec = reinterpret_cast<opt2s_tensor*>(records);
+    auto* rec = reinterpret_cast<Rec*>(records);
     PyObject* const* items = PySequence_Fast_ITEMS(params.ptr());
     int64_t first_change = -1;
     for (int64_t i = 0; i < n; ++i) {
@@ -87,10 +91,22 @@ int64_t refresh_records(py::list params, uintptr_t records, int64_t n)
     return 1;
 }
 
+int64_t refresh_records(py::list params, uintptr_t records, int64_t n)
+{
+    return refresh<opt2s_tensor>(params, records, n);
+}
+
+int64_t refresh_records8(py::list params, uintptr_t records, int64_t n)
+{
+    return refresh<opt2s_tensor8>(params, records, n);
+}
+
 }  // namespace
 
 PYBIND11_MODULE(TORCH_EXTENSION_NAME, m)
 {
     m.def("refresh_records", &refresh_records,
           "Refresh the param/grad addresses of opt2s_tensor records from a parameter list");
+    m.def("refresh_records8", &refresh_records8,
+          "Refresh the param/grad addresses of opt2s_tensor8 records from a parameter list");
 }

@@ -41,6 +41,15 @@ place (``p.data = x``) is then not seen: call refresh() after it.  A group
 shares one step count (one launch, one set of bias corrections): a parameter
 left out of a step, its gradient None, still counts that step.
 
+AdamW8bit, Adam8bit and AdEMAMix8bit keep 8-bit blockwise state
+(opt2s_step_8bit) for parameters of at least ``min_8bit_size`` elements and
+fp32 state for the smaller ones, one launch per group
+(TwoStateOptimizer8bit).
+
+load_state_dict keeps each state tensor's own dtype (fp32 moments of 16-bit
+parameters, uint8 codes), where torch.optim's loader alone would cast them to
+the parameter's dtype.
+
 capturable=True routes every step through opt2s_plan_step_table: the per-step
 scalars live in a device table and the step index in device memory, so
 ``step()`` may be captured in a CUDA graph and each replay performs the next
@@ -185,7 +194,22 @@ class TwoStateOptimizer(torch.optim.Optimizer):
         self._group_cache = {}
 
     def load_state_dict(self, state_dict) -> None:
+        """torch.optim's loader casts every floating-point state tensor to its
+        parameter's dtype; the state here keeps its own (fp32 moments, uint8
+        codes), so after it each tensor is copied again from the saved one,
+        dtype and bits kept, onto the parameter's device."""
         super().load_state_dict(state_dict)
+        from itertools import chain
+        saved_ids = chain.from_iterable(g["params"] for g in state_dict["param_groups"])
+        current = chain.from_iterable(g["params"] for g in self.param_groups)
+        for sid, p in zip(saved_ids, current):
+            saved = state_dict["state"].get(sid)
+            if not saved:
+                continue
+            st = self.state[p]
+            for k, v in saved.items():
+                if k != "step" and isinstance(v, torch.Tensor):
+                    st[k] = v.to(device=p.device, copy=True)
         self._group_cache = {}
 
     # ---- per-group launch data ------------------------------------------
@@ -212,7 +236,7 @@ class TwoStateOptimizer(torch.optim.Optimizer):
             marshal = _marshal_module()
             if marshal is not None:
                 # every parameter has a record: refresh the addresses in place
-                rc = marshal.refresh_records(params, cached["records"], len(params))
+                rc = getattr(marshal, self._refresh_fn)(params, cached["records"], len(params))
                 if rc == 0 or (rc == 1 and not self.capturable):
                     return cached
             elif (all(map(operator.is_, [p.grad for p in params], cached["all_grads"]))
@@ -234,8 +258,7 @@ class TwoStateOptimizer(torch.optim.Optimizer):
         if cached is not None and cached["key"] == key:
             return cached
         states = [self._state_of(p) for p in ps]
-        tl = B.TensorList.from_tensors(ps, [p.grad for p in ps], [s["state1"] for s in states],
-                                       [s["state2"] for s in states])
+        tl = self._records(ps, states)
         data = {"key": key, "params": ps, "tl": tl, "states": states, "step": 0}
         if cached is not None:
             data["step"] = cached["step"]
@@ -259,6 +282,13 @@ class TwoStateOptimizer(torch.optim.Optimizer):
             self._refill(data, group)
         self._group_cache[gi] = data
         return data
+
+    _refresh_fn = "refresh_records"     # the marshalling helper's refresh for these records
+
+    def _records(self, ps, states):
+        """The launch records of parameters ps with their states."""
+        return B.TensorList.from_tensors(ps, [p.grad for p in ps], [s["state1"] for s in states],
+                                         [s["state2"] for s in states])
 
     def _refill(self, data, group):
         first = data["step"] + 1
@@ -293,16 +323,20 @@ class TwoStateOptimizer(torch.optim.Optimizer):
             if self.capturable:
                 data["plan"].step_table(group["skip_zeros"], data["table"].data_ptr(),
                                         self.table_len, data["index"].data_ptr())
-            elif self.lamb:
-                B.opt2s_step_lamb(data["tl"], self._hyper(group), data["step"] + 1)
-            elif self.max_unorm > 0.0:
-                B.opt2s_step_max_unorm(data["tl"], self._hyper(group), self.max_unorm,
-                                       data["step"] + 1)
             else:
-                B.opt2s_step(data["tl"], self._hyper(group), data["step"] + 1)
+                self._launch(data["tl"], self._hyper(group), data["step"] + 1)
             data["step"] += 1
             data["counter"].fill_(data["step"])   # the parameters' shared step count
         return loss
+
+    def _launch(self, tl, hyper, step):
+        """One step of a group's records (not capturable)."""
+        if self.lamb:
+            B.opt2s_step_lamb(tl, hyper, step)
+        elif self.max_unorm > 0.0:
+            B.opt2s_step_max_unorm(tl, hyper, self.max_unorm, step)
+        else:
+            B.opt2s_step(tl, hyper, step)
 
     def refill_step_table(self, next_step: int | None = None) -> None:
         """Capturable mode: rewrite the device tables so that the next step
@@ -353,3 +387,73 @@ class LAMB32bit(TwoStateOptimizer):
 
     def __init__(self, params, lr=1e-3, betas=(0.9, 0.999), eps=1e-6, weight_decay=1e-2, **kw):
         super().__init__(params, "adam", lr, betas, eps, weight_decay, lamb=True, **kw)
+
+
+class TwoStateOptimizer8bit(TwoStateOptimizer):
+    """The two-state optimizer with 8-bit blockwise state (opt2s_step_8bit;
+    Dettmers, Lewis, Shleifer & Zettlemoyer, "8-bit Optimizers via Block-wise
+    Quantization", ICLR 2022).  A parameter of at least ``min_8bit_size``
+    elements keeps its state as one byte per element and quantity (uint8
+    codes: state1 = m, or [m1 | m2] for AdEMAMix; state2 = v) plus one fp32
+    absmax per 2,048-element block and quantity (absmax1, absmax2); a smaller
+    one keeps fp32 state as in the 32-bit classes.  Each parameter group is
+    one launch, mixed 8-bit and fp32 state included.  The state starts at
+    zero: the code of 0 (127 in the signed map of m and m2, 0 in the unsigned
+    map of v) with absmax 0.  Records are refreshed each step as in the
+    32-bit classes; flatten, capturable, max_unorm and LAMB are not offered
+    with 8-bit state."""
+
+    _refresh_fn = "refresh_records8"
+
+    def __init__(self, params, algo: str = "adamw", lr: float = 1e-3, betas=(0.9, 0.999),
+                 eps: float = 1e-8, weight_decay: float = 0.0, beta3: float = 0.9999,
+                 alpha: float = 5.0, skip_zeros: bool = False, min_8bit_size: int = B.MIN_8BIT_SIZE):
+        if int(min_8bit_size) < 1:
+            raise ValueError("min_8bit_size must be >= 1")
+        self.min_8bit_size = int(min_8bit_size)
+        super().__init__(params, algo, lr, betas, eps, weight_decay, beta3=beta3, alpha=alpha,
+                         skip_zeros=skip_zeros)
+
+    def _state_of(self, p):
+        st = self.state[p]
+        if "state1" not in st:
+            n = p.numel()
+            two = self.algo == "ademamix"
+            if B.state_bits_for(n, self.min_8bit_size) == 8:
+                nb = (n + B.BLOCK8 - 1) // B.BLOCK8
+                st["state1"] = torch.full((2 * n if two else n,), 127, dtype=torch.uint8, device=p.device)
+                st["state2"] = torch.zeros(n, dtype=torch.uint8, device=p.device)
+                st["absmax1"] = torch.zeros(2 * nb if two else nb, dtype=torch.float32, device=p.device)
+                st["absmax2"] = torch.zeros(nb, dtype=torch.float32, device=p.device)
+            else:
+                st["state1"] = torch.zeros(2 * n if two else n, dtype=torch.float32, device=p.device)
+                st["state2"] = torch.zeros(n, dtype=torch.float32, device=p.device)
+            st["step"] = 0
+        return st
+
+    def _records(self, ps, states):
+        return B.TensorList8.from_tensors(ps, [p.grad for p in ps], [s["state1"] for s in states],
+                                          [s["state2"] for s in states],
+                                          [s.get("absmax1") for s in states],
+                                          [s.get("absmax2") for s in states])
+
+    def _launch(self, tl, hyper, step):
+        B.opt2s_step_8bit(tl, hyper, step)
+
+
+class AdamW8bit(TwoStateOptimizer8bit):
+    def __init__(self, params, lr=1e-3, betas=(0.9, 0.999), eps=1e-8, weight_decay=1e-2, **kw):
+        super().__init__(params, "adamw", lr, betas, eps, weight_decay, **kw)
+
+
+class Adam8bit(TwoStateOptimizer8bit):
+    def __init__(self, params, lr=1e-3, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0, **kw):
+        super().__init__(params, "adam", lr, betas, eps, weight_decay, **kw)
+
+
+class AdEMAMix8bit(TwoStateOptimizer8bit):
+    def __init__(self, params, lr=1e-3, betas=(0.9, 0.999, 0.9999), alpha=5.0, eps=1e-8,
+                 weight_decay=1e-2, **kw):
+        b1, b2, b3 = betas
+        super().__init__(params, "ademamix", lr, (b1, b2), eps, weight_decay, beta3=b3,
+                         alpha=alpha, **kw)
