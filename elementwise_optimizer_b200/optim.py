@@ -48,7 +48,11 @@ fp32 state for the smaller ones, one launch per group
 
 load_state_dict keeps each state tensor's own dtype (fp32 moments of 16-bit
 parameters, uint8 codes), where torch.optim's loader alone would cast them to
-the parameter's dtype.
+the parameter's dtype; with flatten=True it copies the loaded state into the
+flat buffers the steps read.  The per-parameter state keys differ between
+the layouts (state1/state2 without flatten; exp_avg, exp_avg_sq and
+exp_avg_slow, views of the flat buffers, with it), so a state dict loads into
+an optimizer of the same layout.
 
 capturable=True routes every step through opt2s_plan_step_table: the per-step
 scalars live in a device table and the step index in device memory, so
@@ -142,6 +146,7 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                 per_param = self.max_unorm > 0.0 or self.lamb
                 off = 0
                 views = ([], [], [], [])
+                counter = torch.tensor(0, dtype=torch.int64)     # the entry's shared step count
                 with torch.no_grad():
                     for p in ps:
                         k = p.numel()
@@ -157,13 +162,16 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                         if two:
                             m2_at = m1_at + k if per_param else n + off
                             st["exp_avg_slow"] = fs1[m2_at:m2_at + k].view_as(p)
-                        st["step"] = 0
+                        st["step"] = counter
                         views[0].append(fp[off:off + k])
                         views[1].append(fg[off:off + k])
                         views[2].append(fs1[m1_at:m1_at + (2 * k if two else k)])
                         views[3].append(fs2[off:off + k])
                         off += k
-                entry = dict(group=gi, params=ps, param=fp, grad=fg, state1=fs1, state2=fs2, step=0)
+                entry = dict(group=gi, params=ps, param=fp, grad=fg, state1=fs1, state2=fs2, step=0,
+                             counter=counter,
+                             views=[{key: self.state[p][key] for key in self.state[p] if key != "step"}
+                                    for p in ps])
                 if per_param:
                     entry["records"] = B.TensorList.from_tensors(*views)
                 else:
@@ -210,6 +218,21 @@ class TwoStateOptimizer(torch.optim.Optimizer):
             for k, v in saved.items():
                 if k != "step" and isinstance(v, torch.Tensor):
                     st[k] = v.to(device=p.device, copy=True)
+        if self._flat is not None:
+            # the steps use the flat buffers: copy the loaded state into their
+            # views and put the views (and the entry's step count) back
+            with torch.no_grad():
+                for f in self._flat:
+                    for p, views in zip(f["params"], f["views"]):
+                        st = self.state[p]
+                        for key, view in views.items():
+                            if key in st:
+                                view.copy_(st[key].reshape(view.shape))
+                            st[key] = view
+                        if "step" in st:
+                            f["step"] = int(st["step"])
+                        st["step"] = f["counter"]
+                    f["counter"].fill_(f["step"])
         self._group_cache = {}
 
     # ---- per-group launch data ------------------------------------------
@@ -315,6 +338,7 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                 else:
                     f["plan"].step(hyper, f["step"] + 1)
                 f["step"] += 1
+                f["counter"].fill_(f["step"])
             return loss
         for gi, group in enumerate(self.param_groups):
             data = self._launch_data(gi, group)

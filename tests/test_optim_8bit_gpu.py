@@ -160,3 +160,40 @@ def test_state_dict_round_trip_keeps_state_bits(make):
         for k, v in opt.state[p].items():
             if isinstance(v, torch.Tensor) and k != "step":
                 assert torch.equal(v.view(torch.uint8), opt2.state[q][k].view(torch.uint8)), k
+
+
+@pytest.mark.parametrize("cls", [optim.AdamW32bit, optim.AdEMAMix32bit])
+def test_flat_layout_state_dict_round_trip(cls):
+    """With flatten=True the steps read the flat state buffers: a loaded
+    state must land in them (and in the step count), not only in the state
+    dict, so that the next step continues exactly."""
+    ps = _params(37)
+    opt = cls(ps, lr=3e-3, flatten=True)
+    gen = torch.Generator(device="cpu").manual_seed(11)
+
+    def grads_in_place(params, values=None):
+        out = []
+        for i, p in enumerate(params):
+            v = values[i] if values is not None else (torch.randn(p.shape, generator=gen) * 1e-2).to(p.dtype)
+            p.grad.copy_(v.cuda())              # flat layout: gradients stay views of one buffer
+            out.append(v)
+        return out
+
+    for _ in range(3):
+        grads_in_place(ps)
+        opt.step()
+    saved = copy.deepcopy(opt.state_dict())
+    qs = [torch.nn.Parameter(p.detach().clone()) for p in ps]
+    opt2 = cls(qs, lr=3e-3, flatten=True)
+    opt2.load_state_dict(saved)
+    vals = grads_in_place(ps)
+    grads_in_place(qs, vals)
+    opt.step()
+    opt2.step()
+    torch.cuda.synchronize()
+    for p, q in zip(ps, qs):
+        assert np.array_equal(_bits(p), _bits(q))
+        for k, v in opt.state[p].items():
+            if isinstance(v, torch.Tensor) and k != "step":
+                assert torch.equal(v, opt2.state[q][k]), k
+        assert int(opt2.state[q]["step"]) == 4
