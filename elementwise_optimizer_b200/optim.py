@@ -179,6 +179,31 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                     entry["plan"] = B.Plan(tl, self.algo)
                 self._flat.append(entry)
 
+    @staticmethod
+    def _check_flat_grads(f):
+        """The flat layout steps its gradient buffer, so every parameter's
+        .grad must still be its view into it.  Replacing the gradients (for
+        instance module.zero_grad(), which sets them to None by default, and
+        a backward that then makes new ones) would leave the buffer stale:
+        the first and last parameters of each buffer are checked (O(1) per
+        step) and the step refuses if either was replaced."""
+        fg = f["grad"]
+        base = fg.data_ptr()
+        end = base + fg.numel() * fg.element_size()
+        for p in (f["params"][0], f["params"][-1]):
+            g = p.grad
+            if g is None or not base <= g.data_ptr() < end:     # no other tensor lies in the buffer
+                raise RuntimeError(
+                    "flatten=True: a parameter's .grad is no longer its view of the flat gradient "
+                    "buffer (was it set to None, e.g. by module.zero_grad()?); use the optimizer's "
+                    "zero_grad(), which zeroes the views in place")
+
+    def add_param_group(self, param_group):
+        if getattr(self, "_flat", None) is not None:
+            raise ValueError("flatten=True lays out the groups given at construction; add groups "
+                             "before flattening, or use flatten=False")
+        super().add_param_group(param_group)
+
     def zero_grad(self, set_to_none: bool = False):
         """Zero the gradients in place (one launch per device and dtype), so
         that the cached launch records stay valid; set_to_none=True drops
@@ -330,6 +355,7 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                 loss = closure()
         if self._flat is not None:
             for f in self._flat:
+                self._check_flat_grads(f)
                 hyper = self._hyper(self.param_groups[f["group"]])
                 if "records" in f and self.lamb:
                     B.opt2s_step_lamb(f["records"], hyper, f["step"] + 1)

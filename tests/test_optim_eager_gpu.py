@@ -78,3 +78,22 @@ def test_eager_steps_follow_the_tensors(mode):
         st = opt.state[p]
         assert np.array_equal(st["state1"].cpu().numpy(), h["s1"])
         assert np.array_equal(st["state2"].cpu().numpy(), h["s2"])
+
+
+def test_flat_layout_refuses_replaced_gradients():
+    """flatten=True steps its flat gradient buffer; gradients set to None and
+    made anew by a backward would leave it stale, so the step refuses.  New
+    groups after flattening are refused too."""
+    ps = _params(23)
+    opt = optim.AdamW32bit(ps, lr=1e-3, flatten=True)
+    for p in ps:
+        p.grad.normal_()
+    opt.step()                                   # gradients are the flat views: fine
+    for p in ps:
+        p.grad = None                            # what module.zero_grad() does by default
+    for p in ps:
+        p.grad = torch.ones_like(p)              # a backward makes new tensors
+    with pytest.raises(RuntimeError):
+        opt.step()
+    with pytest.raises(ValueError):
+        opt.add_param_group({"params": [torch.nn.Parameter(torch.zeros(4, device="cuda"))]})
