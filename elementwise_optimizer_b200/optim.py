@@ -63,6 +63,7 @@ and call ``refill_step_table()`` between replays at least once every
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import importlib.machinery
 import importlib.util
@@ -92,6 +93,14 @@ def _marshal_module():
             loader.exec_module(mod)
             _marshal = mod
     return _marshal or None
+
+
+def _on_device(index):
+    """Makes CUDA device `index` current for a launch (nothing to do when it
+    already is): the library plans and launches on the current device."""
+    if index == torch._C._cuda_getDevice():
+        return contextlib.nullcontext()
+    return torch.cuda.device(index)
 
 
 class TwoStateOptimizer(torch.optim.Optimizer):
@@ -169,14 +178,15 @@ class TwoStateOptimizer(torch.optim.Optimizer):
                         views[3].append(fs2[off:off + k])
                         off += k
                 entry = dict(group=gi, params=ps, param=fp, grad=fg, state1=fs1, state2=fs2, step=0,
-                             counter=counter,
+                             counter=counter, device=dev.index,
                              views=[{key: self.state[p][key] for key in self.state[p] if key != "step"}
                                     for p in ps])
                 if per_param:
                     entry["records"] = B.TensorList.from_tensors(*views)
                 else:
                     tl = B.TensorList.from_tensors([fp], [fg], [fs1], [fs2])
-                    entry["plan"] = B.Plan(tl, self.algo)
+                    with _on_device(dev.index):
+                        entry["plan"] = B.Plan(tl, self.algo)
                 self._flat.append(entry)
 
     @staticmethod
@@ -302,12 +312,15 @@ class TwoStateOptimizer(torch.optim.Optimizer):
         for p in ps:
             if not p.is_cuda or not p.is_contiguous() or not p.grad.is_contiguous():
                 raise ValueError("parameters and gradients must be contiguous CUDA tensors")
+        if len({p.device for p in ps} | {p.grad.device for p in ps}) > 1:
+            raise ValueError("a parameter group's tensors and gradients must be on one CUDA device")
         key = tuple((p.data_ptr(), p.grad.data_ptr(), p.numel()) for p in ps)
         if cached is not None and cached["key"] == key:
             return cached
         states = [self._state_of(p) for p in ps]
         tl = self._records(ps, states)
-        data = {"key": key, "params": ps, "tl": tl, "states": states, "step": 0}
+        data = {"key": key, "params": ps, "tl": tl, "states": states, "step": 0,
+                "device": ps[0].device.index if ps else None}
         if cached is not None:
             data["step"] = cached["step"]
             data["counter"] = cached["counter"]
@@ -322,7 +335,8 @@ class TwoStateOptimizer(torch.optim.Optimizer):
         for st in states:
             st["step"] = data["counter"]
         if self.capturable:
-            data["plan"] = B.Plan(tl, self.algo)
+            with _on_device(data["device"] if ps else torch._C._cuda_getDevice()):
+                data["plan"] = B.Plan(tl, self.algo)
             dev = ps[0].device if ps else torch.device("cuda")
             data["table"] = torch.empty(self.table_len * ctypes.sizeof(B.opt2s_step_scalars),
                                         dtype=torch.uint8, device=dev)
@@ -357,12 +371,13 @@ class TwoStateOptimizer(torch.optim.Optimizer):
             for f in self._flat:
                 self._check_flat_grads(f)
                 hyper = self._hyper(self.param_groups[f["group"]])
-                if "records" in f and self.lamb:
-                    B.opt2s_step_lamb(f["records"], hyper, f["step"] + 1)
-                elif "records" in f:
-                    B.opt2s_step_max_unorm(f["records"], hyper, self.max_unorm, f["step"] + 1)
-                else:
-                    f["plan"].step(hyper, f["step"] + 1)
+                with _on_device(f["device"]):
+                    if "records" in f and self.lamb:
+                        B.opt2s_step_lamb(f["records"], hyper, f["step"] + 1)
+                    elif "records" in f:
+                        B.opt2s_step_max_unorm(f["records"], hyper, self.max_unorm, f["step"] + 1)
+                    else:
+                        f["plan"].step(hyper, f["step"] + 1)
                 f["step"] += 1
                 f["counter"].fill_(f["step"])
             return loss
@@ -370,11 +385,12 @@ class TwoStateOptimizer(torch.optim.Optimizer):
             data = self._launch_data(gi, group)
             if not data["params"]:
                 continue
-            if self.capturable:
-                data["plan"].step_table(group["skip_zeros"], data["table"].data_ptr(),
-                                        self.table_len, data["index"].data_ptr())
-            else:
-                self._launch(data["tl"], self._hyper(group), data["step"] + 1)
+            with _on_device(data["device"]):
+                if self.capturable:
+                    data["plan"].step_table(group["skip_zeros"], data["table"].data_ptr(),
+                                            self.table_len, data["index"].data_ptr())
+                else:
+                    self._launch(data["tl"], self._hyper(group), data["step"] + 1)
             data["step"] += 1
             data["counter"].fill_(data["step"])   # the parameters' shared step count
         return loss
