@@ -59,7 +59,9 @@ scalars live in a device table and the step index in device memory, so
 ``step()`` may be captured in a CUDA graph and each replay performs the next
 step.  Make one eager ``step()`` before capturing (it builds the launch plan),
 and call ``refill_step_table()`` between replays at least once every
-``table_len`` steps (``steps_left()`` tells how many remain).
+``table_len`` steps (``steps_left()`` tells how many remain); the table holds
+the hyper-parameters of the refill, so a change of ``lr`` or another group
+setting takes effect at the next refill.
 """
 from __future__ import annotations
 

@@ -67,7 +67,9 @@
 extern "C" {
 #endif
 
-#define OPT2S_ABI_VERSION 1
+/* 2: opt2s_step_scalars carries the fp32 splits of the bias-correction
+ * reciprocals (80 bytes a step, was 64). */
+#define OPT2S_ABI_VERSION 2
 
 /* Storage type of param and grad.  State is always fp32. */
 typedef enum { OPT2S_F32 = 0, OPT2S_F16 = 1, OPT2S_BF16 = 2 } opt2s_dtype;

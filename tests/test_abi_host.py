@@ -96,7 +96,7 @@ def test_struct_layout_matches_c(L):
 
 
 def test_abi_version(L):
-    assert L.opt2s_abi_version() == 1
+    assert L.opt2s_abi_version() == 2
 
 
 def test_error_strings(L):
