@@ -42,10 +42,11 @@
 // complement for x < 0, the code is (entry + key) >> 16: one addition whose
 // carry does the comparison.  The signed map has a table per sign.
 // x itself is first taken as RN32(m * RN32(1/absmax)), within 3 ulp of
-// RN32(m/absmax); only when that lies within 4 ulp of the slice's threshold or
-// of a slice boundary (about 12 cases in 65,536) is x recomputed exactly as
-// RN32(RN64(m * RN64(1/absmax))): for every quotient in the binary32 normal
-// range that is RN32(m/absmax) (the binary64 product errs by less than
+// RN32(m/absmax); only when that lies within 4 ulp of the slice's threshold, or
+// of an edge of a slice without one (about 9 cases in 65,536), is x
+// recomputed exactly as RN32(RN64(m * RN64(1/absmax))): for every quotient in
+// the binary32 normal range that is RN32(m/absmax) (the binary64 product errs
+// by less than
 // 2^-52, while a quotient that is not representable never lies within 2^-49
 // of a binary32 rounding boundary; see div_by_constant in opt2s_device.cuh),
 // and below it both give the code of 0.
@@ -145,18 +146,22 @@ __device__ __forceinline__ uint32_t low_key(uint32_t b)
 
 // Code of the map value nearest to m/absmax (absmax > 0, r32 = RN32(1/absmax)).
 // The fast quotient RN32(m*r32) is within 3 ulp of RN32(m/absmax); when its
-// key lies within 4 of the slice's threshold or of a slice boundary, the exact
-// quotient RN32(RN64(m * RN64(1/absmax))) decides (the binary64 reciprocal is
-// formed there, on that rare path only).  With sum = entry + key,
-// (sum + 5) mod 2^16 <= 8 exactly when the key is within 4 of the threshold
-// (a slice without one only adds boundary cases).
+// key lies within 4 of the slice's threshold, the exact quotient
+// RN32(RN64(m * RN64(1/absmax))) decides (the binary64 reciprocal is formed
+// there, on that rare path only).  With sum = entry + key, (sum + 5) mod 2^16
+// <= 8 exactly when the key is within 4 of the threshold (mod 2^16).  That
+// one test also covers a quotient near a slice boundary: in a slice without a
+// threshold (low half 0) it holds within 4 of either edge, and no slice that
+// holds a threshold has another one within 8 ulp beyond its edges (a property
+// of the two maps, checked on the host by the tests), so a fast quotient that
+// crosses an edge from such a slice crosses no threshold.
 template <bool SIGNED>
 __device__ __forceinline__ uint32_t quantize(const Maps& mp, float m, float r32, float absmax)
 {
     uint32_t b = __float_as_uint(__fmul_rn(m, r32));
     uint32_t key = low_key<SIGNED>(b);
     uint32_t sum = slice_of<SIGNED>(mp, b) + key;
-    if (((sum + 5u) & 0xFFFFu) <= 8u || ((key + 4u) & 0xFFFFu) < 8u) {
+    if (((sum + 5u) & 0xFFFFu) <= 8u) {
         const double r64 = __drcp_rn(static_cast<double>(absmax));
         b = __float_as_uint(__double2float_rn(__dmul_rn(static_cast<double>(m), r64)));
         key = low_key<SIGNED>(b);

@@ -152,7 +152,8 @@ def test_library_tables_are_the_rule(oracle_mod):
 def _device_code(tabs, m, n, signed):
     """The kernel's decision, restated: the code of the fast quotient
     RN32(m * RN32(1/n)) unless its key lies within 4 of the slice's threshold
-    or of a slice boundary, else the code of the exact quotient."""
+    (mod 2^16, so within 4 of either edge of a slice without one), else the
+    code of the exact quotient."""
     fast = (m * (np.float32(1) / n)).astype(np.float32)
     exact = (m.astype(np.float64) / n.astype(np.float64)).astype(np.float32)
     out = []
@@ -162,7 +163,7 @@ def _device_code(tabs, m, n, signed):
         q = tabs[1 if neg else 0][_slice(b, signed)]
         key = (b & 0xFFFF) ^ (0xFFFF if neg else 0)
         s = q + key
-        if ((s + 5) & 0xFFFF) <= 8 or ((key + 4) & 0xFFFF) < 8:
+        if ((s + 5) & 0xFFFF) <= 8:
             out.append(int(_code(tabs, np.array([e], np.float32), signed)[0]))
         else:
             out.append(s >> 16)
@@ -194,3 +195,65 @@ def test_fast_quotient_with_decision_test_gives_the_exact_code(oracle_mod, signe
     m, n = m[keep], n[keep]
     codes, exact = _device_code(tabs, m, n, signed)
     assert np.array_equal(codes, oracle_mod.quantize(qmap, exact))
+
+
+@pytest.mark.parametrize("signed", [True, False])
+def test_no_threshold_sits_near_an_edge_shared_with_another_threshold(oracle_mod, signed):
+    """The kernel needs no separate slice-boundary test because of two
+    properties of the maps: a threshold within 8 ulp of an edge of its slice
+    never faces a slice that holds a threshold across that edge (so a fast
+    quotient that crosses an edge from a slice holding a threshold crosses no
+    threshold), and every threshold lies more than 8 ulp above 2^-23, the edge
+    of the row of values whose code is that of 0."""
+    thr = _thresholds(oracle_mod.quant_map(signed))
+    for side in ((1, -1) if signed else (1,)):
+        mags = np.abs(thr[thr * side > 0]).astype(np.float32)
+        bits = mags.view(np.uint32).astype(np.int64)
+        slices = [_slice(int(b), True) for b in bits]
+        holders = set(slices)
+        for b, sl in zip(bits, slices):
+            low = int(b) & 0xFFFF
+            assert not (low <= 8 and sl - 1 in holders), (side, sl, low)
+            assert not (0x10000 - low <= 8 and sl + 1 in holders), (side, sl, low)
+        assert bits.min() > np.float32(2.0 ** -23).view(np.uint32) + 8
+
+
+def _codes_vec(tabs, bits, signed):
+    """The slice rule over an array of bit patterns (uint32), vectorised."""
+    bits = bits.astype(np.int64)
+    top = ((bits >> 16) & 0x7FFF) if signed else (bits >> 16)
+    idx = np.clip(top - (127 - 24) * 128, 0, ROWS * 128 - 1)
+    neg = ((bits >> 31) == 1) & signed
+    pos_t, neg_t = (np.array(t, np.int64) for t in tabs)
+    q = np.where(neg, neg_t[idx], pos_t[idx])
+    key = (bits & 0xFFFF) ^ np.where(neg, 0xFFFF, 0)
+    return q + key, key
+
+
+@pytest.mark.parametrize("signed", [True, False])
+def test_decision_test_around_every_edge_and_threshold(oracle_mod, signed):
+    """Every fast quotient within 3 ulp of an exact one, the exact one within
+    4 ulp of any slice edge or threshold of the map (both signs for the signed
+    map): the kernel's decision -- the fast quotient's code unless
+    (entry + key + 5) mod 2^16 <= 8, else the exact quotient's code -- gives
+    the exact quotient's nearest code."""
+    qmap = oracle_mod.quant_map(signed)
+    tabs = (_table(qmap, False), _table(qmap, True))
+    thr = _thresholds(qmap)
+    edges = np.arange((127 - 23) << 7, (127 << 7) + 1, dtype=np.int64) << 16     # every slice start, 2^-23 .. 1
+    anchors = np.concatenate([edges, np.abs(thr[thr != 0]).astype(np.float32).view(np.uint32).astype(np.int64)])
+    exact = (anchors[:, None] + np.arange(-4, 5)[None, :]).reshape(-1)
+    exact = exact[(exact > 0) & (exact <= np.float32(1.0).view(np.uint32))]
+    signs = (0, 1 << 31) if signed else (0,)
+    for sgn in signs:
+        e_bits = (exact | sgn).astype(np.uint32)
+        want = oracle_mod.quantize(qmap, e_bits.view(np.float32))
+        for d in range(-3, 4):
+            f_mag = np.clip(exact + d, 0, np.float32(1.0).view(np.uint32) + 3)
+            f_bits = (f_mag | sgn).astype(np.uint32)
+            s_f, _ = _codes_vec(tabs, f_bits, signed)
+            s_e, _ = _codes_vec(tabs, e_bits, signed)
+            redo = ((s_f + 5) & 0xFFFF) <= 8
+            got = np.where(redo, s_e >> 16, s_f >> 16).astype(np.uint8)
+            bad = np.nonzero(got != want)[0]
+            assert bad.size == 0, (sgn, d, e_bits[bad[:5]], f_bits[bad[:5]], got[bad[:5]], want[bad[:5]])
