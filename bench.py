@@ -395,6 +395,41 @@ def transformer_measure(device, steps=10, warmup=3, e2e_steps=3):
     return out
 
 
+def norm_steps_measure(w, d, steps=20, warmup=3, max_unorm=1.0):
+    """The bounded-update-norm step (max_unorm) and, for Adam, the LAMB step on
+    the headline's own buffers: ms per step (CUDA events around each step of
+    four launches), GB/s and fraction of the HBM peak against the plain step's
+    bytes plus one more read of every input."""
+    import torch
+    from elementwise_optimizer_b200 import binding as B
+    peak, kind = measured_peak()
+    nbuf = len(d["lists"])
+    legs = [("max_unorm", lambda k, t: B.opt2s_step_max_unorm(d["lists"][k % nbuf], d["hyper"], max_unorm, t))]
+    if w.algo == "adam":
+        legs.append(("lamb", lambda k, t: B.opt2s_step_lamb(d["lists"][k % nbuf], d["hyper"], t)))
+    per_elem = algorithmic_bytes(w) / w.numel + {"adam": 16, "ademamix": 20}[w.algo]
+    out = {"workload": w.name, "bytes_per_element": per_elem}
+    for name, fn in legs:
+        # warm-up steps touch every gradient buffer, so each descriptor's plan
+        # (with its norm tables) is built before the timed steps
+        nwarm = max(warmup, nbuf)
+        for t in range(1, nwarm + 1):
+            fn(t, t)
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        ev[0].record()
+        for k in range(steps):
+            fn(k, nwarm + 1 + k)
+            ev[k + 1].record()
+        torch.cuda.synchronize()
+        ms = statistics.mean(ev[k].elapsed_time(ev[k + 1]) for k in range(steps))
+        gbs = per_elem * w.numel / (ms / 1e3) / 1e9
+        out[name] = {"ms_per_step": ms, "launches_per_step": 4,
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                                  "frac": gbs / peak, "peak_source": kind}}
+    return out
+
+
 def shard_measure(device, world, rank, numel=268_435_456, steps=10, warmup=3):
     """The ZeRO-style sharded step across the N ranks of the run, over peer
     memory: every rank holds the whole flat fp32 param buffer (the same
@@ -610,11 +645,17 @@ def run_ours(args, rank, world, local_rank):
         d = None
         extras["shard"] = shard_measure(device, world, rank)
     if rank == 0 and world == 1 and not args.no_extras and args.workload == "large_f32":
-        # the largest configuration, measured after the headline's buffers
-        # are freed (1.2 B elements, 21.7 GB with two gradient buffers)
+        # the bounded-norm and LAMB steps on the same buffers, then the largest
+        # configuration after the headline's buffers are freed (1.2 B
+        # elements, 21.7 GB with two gradient buffers), then the 8-bit-state
+        # step (268 M fp32 Adam, 16 B/element) and its mixed collection
+        extras["norm_steps"] = norm_steps_measure(w, d)
         del d
         torch.cuda.empty_cache()
         extras["transformer_bf16"] = transformer_measure(device)
+        torch.cuda.empty_cache()
+        extras["eightbit"] = run_eightbit(steps=20, warmup=5, algos=(("adam", "f32"),))
+        extras["eightbit"].pop("env", None)
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
         cpu = cpu_baseline(w, args.cpu_seconds)
@@ -1114,13 +1155,13 @@ def eightbit_bytes_per_elem(algo, dt):
     return 3 * es + 2 * q + 8 * q / 2048
 
 
-def run_eightbit(numel=268_435_456, steps=50, warmup=10):
+def run_eightbit(numel=268_435_456, steps=50, warmup=10, algos=(("adam", "f32"), ("ademamix", "bf16"))):
     """The 8-bit blockwise-state step (opt2s_step_8bit) on one tensor of
-    `numel` elements (fp32 Adam, bf16 AdEMAMix), timed beside the 32-bit step
-    on the same param/grad; and the mixed AdamW collection of the eager
-    protocol (2,000 tensors of 64..1,024 elements with fp32 state plus 64
-    tensors of 4,096..65,536 elements with 8-bit state) in one launch, L2
-    flushed before each step."""
+    `numel` elements (by default fp32 Adam and bf16 AdEMAMix), timed beside
+    the 32-bit step on the same param/grad; and the mixed AdamW collection of
+    the eager protocol (2,000 tensors of 64..1,024 elements with fp32 state
+    plus 64 tensors of 4,096..65,536 elements with 8-bit state) in one
+    launch, L2 flushed before each step."""
     import torch
     from elementwise_optimizer_b200 import binding as B
     from elementwise_optimizer_b200 import synth
@@ -1128,7 +1169,7 @@ def run_eightbit(numel=268_435_456, steps=50, warmup=10):
     peak, kind = measured_peak()
     tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
     rows = []
-    for algo, dt in (("adam", "f32"), ("ademamix", "bf16")):
+    for algo, dt in algos:
         two = algo == "ademamix"
         nb = (numel + 2047) // 2048
         p = torch.randn(numel, device=dev).to(tdt[dt])
