@@ -46,10 +46,9 @@
 // of an edge of a slice without one (about 9 cases in 65,536), is x
 // recomputed exactly as RN32(RN64(m * RN64(1/absmax))): for every quotient in
 // the binary32 normal range that is RN32(m/absmax) (the binary64 product errs
-// by less than
-// 2^-52, while a quotient that is not representable never lies within 2^-49
-// of a binary32 rounding boundary; see div_by_constant in opt2s_device.cuh),
-// and below it both give the code of 0.
+// by less than 2^-52, while a quotient that is not representable never lies
+// within 2^-49 of a binary32 rounding boundary; see div_by_constant in
+// opt2s_device.cuh), and below it both give the code of 0.
 //
 // Per 8-bit block (one CTA of 256 threads, 8 elements a thread; fp32 storage
 // takes elements 4t..4t+3 and 1024+4t..1024+4t+3, 16-bit storage 8t..8t+7, so
@@ -65,9 +64,8 @@
 //      0 when it is 0; thread 0 stores the new absmaxes.
 // With skip_zeros an element whose gradient is zero keeps its param and its
 // dequantized state, which is requantized with the block's new absmax.
-// Warps of a CTA walk the 32-bit chunks of small tensors element by element
-// with the plain step's element routine (opt2s_device.cuh), eight chunks per
-// work unit.
+// Warps of a CTA walk the 32-bit chunks of small tensors element-wise with the
+// plain step's element update (opt2s_device.cuh), eight chunks per work unit.
 
 #include <cstddef>
 #include <mutex>
