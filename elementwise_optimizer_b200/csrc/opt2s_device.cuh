@@ -67,10 +67,13 @@ __device__ __forceinline__ void st_global(T* p, const T& v) { *p = v; }
 // Muller et al., ch. 4).  No step overflows or underflows in that range
 // (|x/d| < 2^121).
 // Which route a kernel uses is a measured choice (both are exact): the
-// binary64 route in the mixed-dtype and AdEMAMix step kernels and in the
-// norm pass; the fp32 route with an inline fallback in the Adam kernel
-// specialised to fp32 storage; the fp32 route with an out-of-line fallback in
-// the 8-bit-state kernel, whose registers are tight.
+// binary64 route element by element in the plain step kernels (kDivWide);
+// the fp32 route with one range test for a group of elements, and the
+// binary64 route for the whole group when any value is out of range
+// (update_group, kDivGroup), in the 8-bit-state kernel, the norm pass and
+// the scaled step.  A per-element range test cost those kernels more than the
+// route saved: its branch keeps the elements' dependent chains from
+// interleaving.
 // GPU tests check both routes against __fdiv_rn: every binary32 x for a
 // sample of divisors, and random operands near rounding boundaries.
 // ---------------------------------------------------------------------------
@@ -79,48 +82,32 @@ __device__ __forceinline__ float div_by_constant(float x, double r)
     return __double2float_rn(__dmul_rn(static_cast<double>(x), r));
 }
 
-__device__ __noinline__ float div_by_constant_far(float x, double r)
+// The fp32 route's range as one unsigned comparison: x is in range exactly
+// when fma_range_key(x) < kFmaRangeEnd (the biased exponent of |x| in
+// [87, 223), i.e. 2^-40 <= |x| < 2^96).  The maximum of several keys tests
+// several values at once.
+constexpr uint32_t kFmaRangeEnd = 136u << 23;
+__device__ __forceinline__ uint32_t fma_range_key(float x)
 {
-    return div_by_constant(x, r);
+    return (__float_as_uint(x) & 0x7F800000u) - (87u << 23);
 }
 
-// The fp32 route; FAR: the binary64 fallback out of line (a call taken for
-// out-of-range x only) rather than inline.
-template <bool FAR>
-__device__ __forceinline__ float div_by_constant_fma(float x, float d, float hi, float lo, double r)
+// The fp32 route's arithmetic, for x in its range.
+__device__ __forceinline__ float div_by_constant_in_range(float x, float d, float hi, float lo)
 {
-    // biased exponent of |x| in [87, 223): 2^-40 <= |x| < 2^96
-    const uint32_t e = __float_as_uint(x) & 0x7F800000u;
-    if (__builtin_expect(e - (87u << 23) >= (136u << 23), 0))
-        return FAR ? div_by_constant_far(x, r) : div_by_constant(x, r);
     const float q0 = __fmaf_rn(x, hi, __fmul_rn(x, lo));
     const float rem = __fmaf_rn(-q0, d, x);
     return __fmaf_rn(rem, hi, q0);
 }
 
-// Routes of m/bc1 and v/bc2: the binary64 product, or the fp32 route with
-// its fallback inline or out of line.
-enum : int { kDivWide = 0, kDivFma = 1, kDivFmaFar = 2 };
-
-template <int ROUTE>
-__device__ __forceinline__ float div_bc1(float x, const StepScalars& s)
-{
-    return ROUTE == kDivWide
-               ? div_by_constant(x, s.inv_bc1)
-               : div_by_constant_fma<ROUTE == kDivFmaFar>(x, s.bc1, s.rcp_bc1_hi, s.rcp_bc1_lo, s.inv_bc1);
-}
-template <int ROUTE>
-__device__ __forceinline__ float div_bc2(float x, const StepScalars& s)
-{
-    return ROUTE == kDivWide
-               ? div_by_constant(x, s.inv_bc2)
-               : div_by_constant_fma<ROUTE == kDivFmaFar>(x, s.bc2, s.rcp_bc2_hi, s.rcp_bc2_lo, s.inv_bc2);
-}
+// Routes of m/bc1 and v/bc2 in the vector walkers: the binary64 product
+// element by element, or the fp32 route a group at a time (update_group).
+enum : int { kDivWide = 0, kDivGroup = 1 };
 
 // ---------------------------------------------------------------------------
 // The per-element update.  direction() moves the moments of one element (in
 // place) and returns its update direction u = num/den; m/bc1 and v/bc2 use
-// the exact constant division above (ROUTE picks the route), num/den is an
+// the exact constant division above (the binary64 route), num/den is an
 // IEEE division.  update()
 // then applies the step to p.  With SKIP, an element whose gradient compares
 // equal to zero (+0 or -0) is left untouched (no decay either).  MODE:
@@ -132,20 +119,37 @@ __device__ __forceinline__ float div_bc2(float x, const StepScalars& s)
 // ---------------------------------------------------------------------------
 enum : int { kPlain = 0, kScaled = 1, kLamb = 2 };
 
-template <int ALGO, int ROUTE = kDivWide>
-__device__ __forceinline__ float direction(float g, float& m, float& v, float& m2,
-                                           const StepScalars& s)
+// The moments of one element, in place: m, v (and AdEMAMix's m2).
+template <int ALGO>
+__device__ __forceinline__ void moments(float g, float& m, float& v, float& m2, const StepScalars& s)
 {
     m = __fadd_rn(__fmul_rn(s.beta1, m), __fmul_rn(s.one_minus_beta1, g));
     v = __fadd_rn(__fmul_rn(s.beta2, v),
                   __fmul_rn(__fmul_rn(s.one_minus_beta2, g), g));
-    float num = div_bc1<ROUTE>(m, s);
-    if (ALGO == kAdEMAMix) {
-        m2 = __fadd_rn(__fmul_rn(s.beta3, m2), __fmul_rn(s.one_minus_beta3, g));
-        num = __fadd_rn(num, __fmul_rn(s.alpha, m2));
-    }
-    const float den = __fadd_rn(__fsqrt_rn(div_bc2<ROUTE>(v, s)), s.eps);
+    if (ALGO == kAdEMAMix) m2 = __fadd_rn(__fmul_rn(s.beta3, m2), __fmul_rn(s.one_minus_beta3, g));
+}
+
+// u = num/den from the bias-corrected moments mh = m/bc1 and vh = v/bc2.
+template <int ALGO>
+__device__ __forceinline__ float direction_of(float mh, float vh, float m2, const StepScalars& s)
+{
+    const float num = ALGO == kAdEMAMix ? __fadd_rn(mh, __fmul_rn(s.alpha, m2)) : mh;
+    const float den = __fadd_rn(__fsqrt_rn(vh), s.eps);
     return __fdiv_rn(num, den);
+}
+
+// The plain step's param update: p*decay - lr*u.
+__device__ __forceinline__ float plain_param(float p, float u, const StepScalars& s)
+{
+    return __fsub_rn(__fmul_rn(p, s.decay), __fmul_rn(s.lr, u));
+}
+
+template <int ALGO>
+__device__ __forceinline__ float direction(float g, float& m, float& v, float& m2,
+                                           const StepScalars& s)
+{
+    moments<ALGO>(g, m, v, m2, s);
+    return direction_of<ALGO>(div_by_constant(m, s.inv_bc1), div_by_constant(v, s.inv_bc2), m2, s);
 }
 
 // LAMB's decayed direction w = u + wd*p of an element.
@@ -154,17 +158,71 @@ __device__ __forceinline__ float lamb_direction(float u, float p, float wd)
     return __fadd_rn(u, __fmul_rn(wd, p));
 }
 
-template <int ALGO, bool SKIP, int MODE = kPlain, int ROUTE = kDivWide>
+// The param after the step, from its direction u (MODE as above).
+template <int MODE>
+__device__ __forceinline__ float param_after(float p, float u, const StepScalars& s, float scale,
+                                             float wd)
+{
+    if (MODE == kLamb) return __fsub_rn(p, __fmul_rn(s.lr, __fmul_rn(scale, lamb_direction(u, p, wd))));
+    return plain_param(p, MODE == kScaled ? __fmul_rn(scale, u) : u, s);
+}
+
+template <int ALGO, bool SKIP, int MODE = kPlain>
 __device__ __forceinline__ void update(float g, float& p, float& m, float& v,
                                        float& m2, const StepScalars& s, float scale = 1.0f,
                                        float wd = 0.0f)
 {
     if (SKIP && g == 0.0f) return;
-    const float u = direction<ALGO, ROUTE>(g, m, v, m2, s);
-    if (MODE == kLamb)
-        p = __fsub_rn(p, __fmul_rn(s.lr, __fmul_rn(scale, lamb_direction(u, p, wd))));
-    else
-        p = __fsub_rn(__fmul_rn(p, s.decay), __fmul_rn(s.lr, MODE == kScaled ? __fmul_rn(scale, u) : u));
+    const float u = direction<ALGO>(g, m, v, m2, s);
+    p = param_after<MODE>(p, u, s, scale, wd);
+}
+
+// update() on G of a thread's elements, O .. O+G-1 of its arrays, phase by
+// phase: the moments of all G, one range test for all their bias-correction
+// divisions (the fp32 route when every value is in its range, else the
+// binary64 route for all G: both are exact, so either gives the same
+// quotients), then the directions and the params.  No per-element branch
+// separates the elements' dependent chains, so they interleave.  With SKIP an
+// element whose gradient compares equal to zero keeps p, m, v and m2.
+template <int ALGO, bool SKIP, int MODE, int O, int G, int N>
+__device__ __forceinline__ void update_group(const float (&g)[N], float (&p)[N], float (&m)[N],
+                                             float (&v)[N], float (&m2)[N], const StepScalars& s,
+                                             float scale = 1.0f, float wd = 0.0f)
+{
+    static_assert(O + G <= N, "group inside the arrays");
+    float mn[G], vn[G], m2n[G], mh[G], vh[G];
+    uint32_t key = 0;
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+        mn[j] = m[O + j];
+        vn[j] = v[O + j];
+        m2n[j] = m2[O + j];
+        moments<ALGO>(g[O + j], mn[j], vn[j], m2n[j], s);
+        key = max(key, max(fma_range_key(mn[j]), fma_range_key(vn[j])));
+    }
+    if (__builtin_expect(key >= kFmaRangeEnd, 0)) {
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            mh[j] = div_by_constant(mn[j], s.inv_bc1);
+            vh[j] = div_by_constant(vn[j], s.inv_bc2);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            mh[j] = div_by_constant_in_range(mn[j], s.bc1, s.rcp_bc1_hi, s.rcp_bc1_lo);
+            vh[j] = div_by_constant_in_range(vn[j], s.bc2, s.rcp_bc2_hi, s.rcp_bc2_lo);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+        const float pn = param_after<MODE>(p[O + j], direction_of<ALGO>(mh[j], vh[j], m2n[j], s), s, scale, wd);
+        if (!SKIP || g[O + j] != 0.0f) {
+            p[O + j] = pn;
+            m[O + j] = mn[j];
+            v[O + j] = vn[j];
+            m2[O + j] = m2n[j];
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -321,7 +379,7 @@ __device__ __forceinline__ void store_state(float* b, uint32_t i, const float (&
 // One element through the scalar path (chunk head, tail, or a chunk whose
 // arrays are not mutually 16-byte aligned).  A skipped element is not even
 // written back.
-template <int DT, int ALGO, bool SKIP, int MODE = kPlain, int ROUTE = kDivWide>
+template <int DT, int ALGO, bool SKIP, int MODE = kPlain>
 __device__ __forceinline__ void scalar_element(const ChunkRec& c, uint32_t i,
                                                const StepScalars& s, float scale = 1.0f,
                                                float wd = 0.0f)
@@ -334,7 +392,7 @@ __device__ __forceinline__ void scalar_element(const ChunkRec& c, uint32_t i,
     float v = ld_global(c.v + i);
     float m2 = 0.0f;
     if (ALGO == kAdEMAMix) m2 = ld_global(c.m2 + i);
-    update<ALGO, false, MODE, ROUTE>(g, p, m, v, m2, s, scale, wd);
+    update<ALGO, false, MODE>(g, p, m, v, m2, s, scale, wd);
     P::store1(c.p, i, p);
     st_global(c.m + i, m);
     st_global(c.v + i, v);
@@ -393,9 +451,13 @@ __device__ __forceinline__ void vector_body(const ChunkRec& c, const StepScalars
                 float g[V], p[V];
                 P::widen(graw[u], g);
                 P::widen(praw[u], p);
+                if (ROUTE == kDivGroup) {
+                    update_group<ALGO, SKIP, MODE, 0, V, V>(g, p, m[u], v[u], m2[u], s, scale, wd);
+                } else {
 #pragma unroll
-                for (int j = 0; j < V; ++j)
-                    update<ALGO, SKIP, MODE, ROUTE>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s, scale, wd);
+                    for (int j = 0; j < V; ++j)
+                        update<ALGO, SKIP, MODE>(g[j], p[j], m[u][j], v[u][j], m2[u][j], s, scale, wd);
+                }
                 P::store(c.p, e, P::narrow(p, praw[u], g, SKIP));
                 store_state_any<V>(c.m, e, ALL || al.m, m[u]);
                 store_state_any<V>(c.v, e, ALL || al.v, v[u]);
@@ -421,9 +483,9 @@ __device__ __forceinline__ void run_chunk(const ChunkRec& c, const StepScalars& 
     const uint32_t body_end = head + nvec * V;
 
     for (uint32_t i = lane; i < head; i += 32)
-        scalar_element<DT, ALGO, SKIP, MODE, ROUTE>(c, i, s, scale, wd);
+        scalar_element<DT, ALGO, SKIP, MODE>(c, i, s, scale, wd);
     for (uint32_t i = body_end + lane; i < len; i += 32)
-        scalar_element<DT, ALGO, SKIP, MODE, ROUTE>(c, i, s, scale, wd);
+        scalar_element<DT, ALGO, SKIP, MODE>(c, i, s, scale, wd);
 
     const Aligned al{aligned16(c.g, head, P::kBytes), aligned16(c.m, head, 4),
                      aligned16(c.v, head, 4), ALGO != kAdEMAMix || aligned16(c.m2, head, 4)};

@@ -271,7 +271,12 @@ __global__ void advance_index_kernel(int* index, int table_len)
 //   4. step_kernel_scaled: the step over the plan's chunks with
 //      p = p*decay - lr*(scale*u), or p = p - lr*(scale*w) for LAMB, the
 //      scale read through the chunk's tensor.
-// The element arithmetic is direction(), as in the plain step.  Every sum
+// The element arithmetic is the plain step's (moments, the exact divisions by
+// bc1 and bc2, direction_of); the norm pass and the scaled step take the
+// divisions of a lane's elements with one range test (the fp32 route, or the
+// binary64 route for all when a value is out of its range; both exact), which
+// measured 3 % faster on the bounded-norm and LAMB steps than a test, or the
+// binary64 route, element by element.  Every sum
 // has a fixed order: lane l of the warp that owns a block adds the elements
 // of its runs (V consecutive elements at V*l + 32*V*r, V = 4 for fp32 and 8
 // for 16-bit storage) in index order, the 32 lanes then combine in a fixed
@@ -355,12 +360,35 @@ __device__ __forceinline__ void norm_block(const ChunkRec& c, const StepScalars&
                 }
             }
         }
+        // the moments of all K elements, then their bias-correction
+        // divisions with one range test (the fp32 route when every value is
+        // in its range, else the binary64 route for all: both are exact)
+        // and the directions
+        uint32_t key = 0;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            moments<ALGO>(g[k], m[k], v[k], m2[k], s);
+            key = max(key, max(fma_range_key(m[k]), fma_range_key(v[k])));
+        }
+        if (__builtin_expect(key >= kFmaRangeEnd, 0)) {
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                m[k] = div_by_constant(m[k], s.inv_bc1);
+                v[k] = div_by_constant(v[k], s.inv_bc2);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                m[k] = div_by_constant_in_range(m[k], s.bc1, s.rcp_bc1_hi, s.rcp_bc1_lo);
+                v[k] = div_by_constant_in_range(v[k], s.bc2, s.rcp_bc2_hi, s.rcp_bc2_lo);
+            }
+        }
 #pragma unroll
         for (int k = 0; k < K; ++k) {
             if (base + ((k / V) * 32 + lane) * V + (k % V) < len) {
                 ap.add(p[k]);
                 if (!(SKIP && g[k] == 0.0f)) {
-                    const float u = direction<ALGO>(g[k], m[k], v[k], m2[k], s);
+                    const float u = direction_of<ALGO>(m[k], v[k], m2[k], s);
                     ad.add(MODE == kLamb ? lamb_direction(u, p[k], wd) : u);
                 }
             }
@@ -479,6 +507,12 @@ unorm_scale_kernel(const double2* __restrict__ sums, const uint32_t* __restrict_
     }
 }
 
+// The scaled step's division route: a group at a time, except with
+// skip_zeros, whose per-element selects would take the kernel from 128 to 156
+// registers (AdEMAMix).
+template <bool SKIP>
+constexpr int kScaledRoute = SKIP ? kDivWide : kDivGroup;
+
 template <int ALGO, bool SKIP, int MODE>
 __global__ void step_kernel_scaled(const ChunkRec* __restrict__ chunks, int nchunks,
                                    StepScalars s, const uint32_t* __restrict__ chunk_tensor,
@@ -492,9 +526,9 @@ __global__ void step_kernel_scaled(const ChunkRec* __restrict__ chunks, int nchu
         const ChunkRec rec = chunks[c];
         const float sc = scale[chunk_tensor[c]];
         switch (rec.dtype & ~kShortFlag) {
-        case kF32: run_chunk<kF32, ALGO, SKIP, MODE>(rec, s, lane, sc, wd); break;
-        case kF16: run_chunk<kF16, ALGO, SKIP, MODE>(rec, s, lane, sc, wd); break;
-        default: run_chunk<kBF16, ALGO, SKIP, MODE>(rec, s, lane, sc, wd); break;
+        case kF32: run_chunk<kF32, ALGO, SKIP, MODE, 1, kScaledRoute<SKIP>>(rec, s, lane, sc, wd); break;
+        case kF16: run_chunk<kF16, ALGO, SKIP, MODE, 1, kScaledRoute<SKIP>>(rec, s, lane, sc, wd); break;
+        default: run_chunk<kBF16, ALGO, SKIP, MODE, 1, kScaledRoute<SKIP>>(rec, s, lane, sc, wd); break;
         }
     }
 }

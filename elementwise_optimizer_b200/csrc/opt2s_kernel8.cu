@@ -55,13 +55,15 @@
 // that every warp access is contiguous):
 //   1. dequantize: m = map_s[code]*absmax (fp32 product), v with map_u;
 //   2. the plain step's element update (opt2s_device.cuh; its fp32 route for
-//      the bias-correction divisions), param stored;
+//      the bias-correction divisions), a few elements at a time with one
+//      range test for their divisions (update_group), param stored;
 //   3. the block's new absmax of |m|, v (, |m2|): fmaxf over the thread's
 //      elements (NaNs are ignored), then an unsigned maximum of the bit
 //      patterns over the warp (one warp reduction) and the CTA's 8 warps
 //      (max is exact, so the order does not matter);
 //   4. quantize each value with the block's new absmax, or store the code of
-//      0 when it is 0; thread 0 stores the new absmaxes.
+//      0 when it is 0 (a thread's eight values of a state take one test for
+//      the rare exact quotients); thread 0 stores the new absmaxes.
 // With skip_zeros an element whose gradient is zero keeps its param and its
 // dequantized state, which is requantized with the block's new absmax.
 // Warps of a CTA walk the 32-bit chunks of small tensors element-wise with the
@@ -78,13 +80,22 @@ namespace {
 constexpr int kB8Threads = 256;                  // one CTA per 8-bit block
 // Resident CTAs per SM the registers must allow: the kernel waits on loads
 // and on its barrier, so more resident CTAs measured faster (Adam: 4 CTAs at
-// 64 registers beat 3 at 80, 2 at 128 and 5 at 48, which spills; AdEMAMix, with
-// a third state, 4 at 64 registers and a few spilled bytes beat 3 at 80 by
-// 1 %).  Each CTA also prefetches its next block into L2.
+// 64 registers beat 3 at 80, 2 at 128 and 5 at 48, which spills; with the
+// grouped update, 4 CTAs with a few spilled bytes still beat 3 without: Adam
+// 1.109 against 1.149 ms, AdEMAMix 1.403 against 1.439 at 268 M elements).
+// Each CTA also prefetches its next block into L2.
 template <int ALGO>
 constexpr int kB8MinCtas = 4;
 constexpr int kB8PerThread = kBlock8Elems / kB8Threads;
 static_assert(kB8PerThread == 8, "eight elements a thread");
+// Elements a thread updates together (update_group): measured at 268 M
+// elements against the element-by-element loop (1.280 / 1.656 ms for fp32
+// Adam / bf16 AdEMAMix): groups of 4 for Adam (1.109 ms; 8: 1.184), 8 for
+// AdEMAMix (1.403 ms; 4: 1.432), and 2 for AdEMAMix with skip_zeros, whose
+// selects cost registers (1.588 ms; 8 spills and takes 1.98, against 1.80
+// before).
+template <int ALGO, bool SKIP>
+constexpr int kGroup = ALGO == kAdEMAMix ? (SKIP ? 2 : 8) : 4;
 
 constexpr int kRows = kQuantRows;         // |x| < 2^-23; 24 binades 2^-23 .. 2^0; NaN
 constexpr int kSlices = kRows * 128;      // 128 slices a row
@@ -142,30 +153,36 @@ __device__ __forceinline__ uint32_t low_key(uint32_t b)
     return SIGNED ? (b ^ static_cast<uint32_t>(static_cast<int32_t>(b) >> 31)) & 0xFFFFu : b & 0xFFFFu;
 }
 
-// Code of the map value nearest to m/absmax (absmax > 0, r32 = RN32(1/absmax)).
-// The fast quotient RN32(m*r32) is within 3 ulp of RN32(m/absmax); when its
-// key lies within 4 of the slice's threshold, the exact quotient
-// RN32(RN64(m * RN64(1/absmax))) decides (the binary64 reciprocal is formed
-// there, on that rare path only).  With sum = entry + key, (sum + 5) mod 2^16
-// <= 8 exactly when the key is within 4 of the threshold (mod 2^16).  That
-// one test also covers a quotient near a slice boundary: in a slice without a
-// threshold (low half 0) it holds within 4 of either edge, and no slice that
-// holds a threshold has another one within 8 ulp beyond its edges (a property
-// of the two maps, checked on the host by the tests), so a fast quotient that
-// crosses an edge from such a slice crosses no threshold.
+// Quantization of one value m with absmax > 0, in two parts.  fast_sum
+// takes the fast quotient RN32(m*r32), r32 = RN32(1/absmax), within 3 ulp of
+// RN32(m/absmax), and returns sum = entry + key for it, whose high half is
+// then the code.  The code is certain unless the key lies within 4 of the
+// slice's threshold; with sum as above, (sum + 5) mod 2^16 <= 8 exactly then
+// (near_key).  That one test also covers a quotient near a slice boundary: in
+// a slice without a threshold (low half 0) it holds within 4 of either edge,
+// and no slice that holds a threshold has another one within 8 ulp beyond its
+// edges (a property of the two maps, checked on the host by the tests), so a
+// fast quotient that crosses an edge from such a slice crosses no threshold.
+// exact_sum gives the sum for the exact quotient RN32(RN64(m * RN64(1/absmax)))
+// (r64 = RN64(1/absmax)), for the values that near_key flags.
 template <bool SIGNED>
-__device__ __forceinline__ uint32_t quantize(const Maps& mp, float m, float r32, float absmax)
+__device__ __forceinline__ uint32_t sum_of_bits(const Maps& mp, uint32_t b)
 {
-    uint32_t b = __float_as_uint(__fmul_rn(m, r32));
-    uint32_t key = low_key<SIGNED>(b);
-    uint32_t sum = slice_of<SIGNED>(mp, b) + key;
-    if (((sum + 5u) & 0xFFFFu) <= 8u) {
-        const double r64 = __drcp_rn(static_cast<double>(absmax));
-        b = __float_as_uint(__double2float_rn(__dmul_rn(static_cast<double>(m), r64)));
-        key = low_key<SIGNED>(b);
-        sum = slice_of<SIGNED>(mp, b) + key;
-    }
-    return sum >> 16;
+    return slice_of<SIGNED>(mp, b) + low_key<SIGNED>(b);
+}
+template <bool SIGNED>
+__device__ __forceinline__ uint32_t fast_sum(const Maps& mp, float m, float r32)
+{
+    return sum_of_bits<SIGNED>(mp, __float_as_uint(__fmul_rn(m, r32)));
+}
+template <bool SIGNED>
+__device__ __forceinline__ uint32_t exact_sum(const Maps& mp, float m, double r64)
+{
+    return sum_of_bits<SIGNED>(mp, __float_as_uint(__double2float_rn(__dmul_rn(static_cast<double>(m), r64))));
+}
+__device__ __forceinline__ uint32_t near_key(uint32_t sum)
+{
+    return (sum + 5u) & 0xFFFFu;    // <= 8: the fast quotient does not decide
 }
 
 // The maximum over the warp of a value that is >= +0 and not NaN: such
@@ -237,17 +254,30 @@ __device__ __forceinline__ uint32_t pack4(uint32_t c0, uint32_t c1, uint32_t c2,
 
 // The codes of a thread's eight values x[] of one state, packed as the code
 // arrays store them (zero_code for all when the block's absmax is 0).
+// All eight fast quotients and table lookups come first, with one test for
+// the lot; the rare exact quotients (about 9 values in 65,536) follow in a
+// branch of their own, so that no per-value branch separates the lookups.
 template <bool SIGNED>
 __device__ __forceinline__ void quantize8(const Maps& mp, const float (&x)[kB8PerThread], float absmax,
                                           uint32_t zero_code, uint32_t (&w)[2])
 {
     if (absmax > 0.0f) {
         const float r32 = __frcp_rn(absmax);     // for the fast quotient
-        uint32_t c[kB8PerThread];
+        uint32_t sum[kB8PerThread];
+        uint32_t near = 0xFFFFu;
 #pragma unroll
-        for (int k = 0; k < kB8PerThread; ++k) c[k] = quantize<SIGNED>(mp, x[k], r32, absmax);
-        w[0] = pack4(c[0], c[1], c[2], c[3]);
-        w[1] = pack4(c[4], c[5], c[6], c[7]);
+        for (int k = 0; k < kB8PerThread; ++k) {
+            sum[k] = fast_sum<SIGNED>(mp, x[k], r32);
+            near = min(near, near_key(sum[k]));
+        }
+        if (__builtin_expect(near <= 8u, 0)) {
+            const double r64 = __drcp_rn(static_cast<double>(absmax));
+#pragma unroll
+            for (int k = 0; k < kB8PerThread; ++k)
+                if (near_key(sum[k]) <= 8u) sum[k] = exact_sum<SIGNED>(mp, x[k], r64);
+        }
+        w[0] = pack4(sum[0] >> 16, sum[1] >> 16, sum[2] >> 16, sum[3] >> 16);
+        w[1] = pack4(sum[4] >> 16, sum[5] >> 16, sum[6] >> 16, sum[7] >> 16);
     } else {
         w[0] = w[1] = zero_code * 0x01010101u;
     }
@@ -294,6 +324,17 @@ __device__ __forceinline__ void prefetch_block(const Block8Rec& b, int es)
 __device__ __forceinline__ bool al(const void* q, uint32_t bytes)
 {
     return (reinterpret_cast<uintptr_t>(q) & (bytes - 1)) == 0;
+}
+
+// All eight elements, G at a time.
+template <int ALGO, bool SKIP, int G, int O = 0>
+__device__ __forceinline__ void update_all(const float (&g)[kB8PerThread], float (&p)[kB8PerThread],
+                                           float (&m)[kB8PerThread], float (&v)[kB8PerThread],
+                                           float (&m2)[kB8PerThread], const StepScalars& s)
+{
+    static_assert(kB8PerThread % G == 0, "groups tile the thread's elements");
+    update_group<ALGO, SKIP, kPlain, O, G>(g, p, m, v, m2, s);
+    if constexpr (O + G < kB8PerThread) update_all<ALGO, SKIP, G, O + G>(g, p, m, v, m2, s);
 }
 
 // One 8-bit block by the whole CTA.  `buf` selects the half of the reduction
@@ -346,19 +387,23 @@ __device__ __forceinline__ void block8(const Block8Rec& b, const StepScalars& s,
     }
 
     float m[kB8PerThread], v[kB8PerThread], m2[kB8PerThread];
-    float x1 = 0.0f, x2 = 0.0f, x3 = 0.0f;
 #pragma unroll
     for (int k = 0; k < kB8PerThread; ++k) {
         m[k] = __fmul_rn(mp.smap[code_at(c1, k)], a1);
         v[k] = __fmul_rn(mp.umap[code_at(c2, k)], a2);
         m2[k] = ALGO == kAdEMAMix ? __fmul_rn(mp.smap[code_at(c3, k)], a3) : 0.0f;
+    }
+    // (elements past the end of a partial block are stepped too, from zero
+    // inputs, and then left out of the absmaxes and the stores)
+    update_all<ALGO, SKIP, kGroup<ALGO, SKIP>>(g, p, m, v, m2, s);
+    float x1 = 0.0f, x2 = 0.0f, x3 = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kB8PerThread; ++k)
         if (FULL || elem<V>(k / V, k % V) < len) {
-            update<ALGO, SKIP, kPlain, kDivFmaFar>(g[k], p[k], m[k], v[k], m2[k], s);
             x1 = fmaxf(x1, fabsf(m[k]));
             x2 = fmaxf(x2, fabsf(v[k]));
             if (ALGO == kAdEMAMix) x3 = fmaxf(x3, fabsf(m2[k]));
         }
-    }
     if (vec) {
 #pragma unroll
         for (int u = 0; u < R; ++u) {

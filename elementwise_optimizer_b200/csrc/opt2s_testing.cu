@@ -13,7 +13,7 @@ namespace {
 
 // ---------------------------------------------------------------------------
 // Validation scaffolding: both routes of the constant division against
-// __fdiv_rn.  Operands come from the SplitMix64 output function (Steele, Lea
+// __fdiv_rn (the fp32 route on the operands in its range).  Operands come from the SplitMix64 output function (Steele, Lea
 // & Flood, "Fast splittable pseudorandom number generators", OOPSLA 2014)
 // applied to a counter.
 // Divisors lie in [2^-25, 1], the bias corrections' range: a random binade
@@ -49,11 +49,12 @@ __device__ __forceinline__ bool same_quotient(float x, float d)
     const float hi = __double2float_rn(r);
     const float lo = __double2float_rn(__dsub_rn(r, static_cast<double>(hi)));
     const float a = div_by_constant(x, r);                   // binary64 route
-    const float c = div_by_constant_fma<false>(x, d, hi, lo, r);    // fp32 route
-    const float f = div_by_constant_fma<true>(x, d, hi, lo, r);     // same, fallback out of line
     const float b = __fdiv_rn(x, d);
     auto same = [](float u, float w) { return __float_as_uint(u) == __float_as_uint(w) || (isnan(u) && isnan(w)); };
-    return same(a, b) && same(c, b) && same(f, b);
+    // the fp32 route, for x in its range (a group with a value outside it
+    // takes the binary64 route)
+    const bool in_range = fma_range_key(x) < kFmaRangeEnd;
+    return same(a, b) && (!in_range || same(div_by_constant_in_range(x, d, hi, lo), b));
 }
 
 __global__ void check_division_kernel(uint64_t seed, int64_t n, int mode,
