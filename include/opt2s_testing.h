@@ -96,8 +96,9 @@ int opt2s_testing_unorm_tables(const TensorListDesc *desc, int32_t algo, int64_t
                                uint32_t *group_ranges, uint32_t *first_group,
                                uint32_t *chunk_tensor, int64_t *counts);
 
-/* Test build only.  Runs the step kernel's exact division by a constant in
- * [2^-25, 1] and the IEEE division __fdiv_rn side by side on the current
+/* Test build only.  Runs the kernels' exact division by a constant in
+ * [2^-25, 1] (the binary64 route for every x, and the fp32 route for the x in
+ * its range) and the IEEE division __fdiv_rn side by side on the current
  * device: mode 0, `n` seeded random pairs with x of every class; mode 1, `n`
  * pairs with x/d next to a binary32 rounding boundary; mode 2, `n` seeded
  * divisors (n <= 2^20), each with all 2^32 binary32 x.  Writes how many
