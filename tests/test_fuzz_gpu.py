@@ -7,9 +7,10 @@ specialised Adam kernel runs), the algorithm, skip_zeros, hyper-parameters
 (learning rate over four decades, beta1 including 0, weight decay on or off),
 the gradient recipe, the storage layout (separate allocations, packed back to
 back, or padded so that most tensors start misaligned), the starting step,
-for half the cases a forced chunk length and launch shape, and for a third of
+for half the cases a forced chunk length and launch shape, for a third of
 them a max_unorm bound (opt2s_step_max_unorm against the oracle's bounded
-step).  After every step, param, state1 and state2 must hold the oracle's
+step), and for some of the other Adam cases the LAMB step (opt2s_step_lamb
+against the oracle's).  After every step, param, state1 and state2 must hold the oracle's
 bits and the gradients must be untouched.
 """
 import numpy as np
@@ -67,13 +68,15 @@ def draw_case(case):
         geometry = (int(r.choice([32, 64, 128, 256])), int(r.choice([0, 1, 3, 7])),
                     int(r.choice([0, 8, 256, 1000, 4096])))
     max_unorm = float(np.float32(10 ** r.uniform(-2, 1))) if r.random() < 1 / 3 else 0.0
-    return w, layout, pad, first_step, steps, geometry, max_unorm
+    # LAMB takes Adam moments; drawn last, so the draws above are unchanged
+    lamb = algo == "adam" and max_unorm == 0.0 and r.random() < 0.4
+    return w, layout, pad, first_step, steps, geometry, max_unorm, lamb
 
 
 @pytest.mark.usefixtures("testing_lib")
 @pytest.mark.parametrize("case", range(CASES))
 def test_random_collection_matches_oracle(case):
-    w, layout, pad, first_step, steps, geometry, max_unorm = draw_case(case)
+    w, layout, pad, first_step, steps, geometry, max_unorm, lamb = draw_case(case)
     if geometry is not None:
         B.opt2s_release_cache()
         prev = B.testing_set_chunk_elems(geometry[2])
@@ -88,6 +91,13 @@ def test_random_collection_matches_oracle(case):
                     oracle.step_f32_max_unorm(h.h_p[i], h._h_g[i], h.h_s1[i], h.h_s2[i], dtype=dt,
                                               algo=w.algo, step=t, skip_zeros=w.skip_zeros,
                                               max_unorm=max_unorm, **w.hyper)
+            elif lamb:
+                h.load_grads(t)
+                B.opt2s_step_lamb(h.tl, h.hyper, t)
+                hy = {k: w.hyper[k] for k in ("lr", "beta1", "beta2", "eps", "weight_decay")}
+                for i, dt in enumerate(w.dtypes):
+                    oracle.step_f32_lamb(h.h_p[i], h._h_g[i], h.h_s1[i], h.h_s2[i], dtype=dt, step=t,
+                                         skip_zeros=w.skip_zeros, **hy)
             else:
                 h.step_both(t)
             worst = h.max_ulps()
