@@ -90,12 +90,12 @@ constexpr int kB8PerThread = kBlock8Elems / kB8Threads;
 static_assert(kB8PerThread == 8, "eight elements a thread");
 // Elements a thread updates together (update_group): measured at 268 M
 // elements against the element-by-element loop (1.280 / 1.656 ms for fp32
-// Adam / bf16 AdEMAMix): groups of 4 for Adam (1.109 ms; 8: 1.184), 8 for
-// AdEMAMix (1.403 ms; 4: 1.432), and 2 for AdEMAMix with skip_zeros, whose
-// selects cost registers (1.588 ms; 8 spills and takes 1.98, against 1.80
-// before).
+// Adam / bf16 AdEMAMix): groups of 4 for Adam (1.109 ms; 8: 1.184; 2: 1.134),
+// 8 for AdEMAMix (1.403 ms; 4: 1.432), and 2 with skip_zeros, whose selects
+// cost registers (Adam 1.146 ms, 4: 1.175, 8: 1.200; AdEMAMix 1.588 ms, 8
+// spills and takes 1.98, against 1.80 before).
 template <int ALGO, bool SKIP>
-constexpr int kGroup = ALGO == kAdEMAMix ? (SKIP ? 2 : 8) : 4;
+constexpr int kGroup = SKIP ? 2 : (ALGO == kAdEMAMix ? 8 : 4);
 
 constexpr int kRows = kQuantRows;         // |x| < 2^-23; 24 binades 2^-23 .. 2^0; NaN
 constexpr int kSlices = kRows * 128;      // 128 slices a row
