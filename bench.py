@@ -654,7 +654,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         extras["transformer_bf16"] = transformer_measure(device)
         torch.cuda.empty_cache()
-        extras["eightbit"] = run_eightbit(steps=20, warmup=5, algos=(("adam", "f32"),))
+        extras["eightbit"] = run_eightbit(steps=20, warmup=5, algos=(("adam", "f32"),), skip_zeros=False)
         extras["eightbit"].pop("env", None)
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
@@ -1155,13 +1155,15 @@ def eightbit_bytes_per_elem(algo, dt):
     return 3 * es + 2 * q + 8 * q / 2048
 
 
-def run_eightbit(numel=268_435_456, steps=50, warmup=10, algos=(("adam", "f32"), ("ademamix", "bf16"))):
+def run_eightbit(numel=268_435_456, steps=50, warmup=10, algos=(("adam", "f32"), ("ademamix", "bf16")),
+                 skip_zeros=True):
     """The 8-bit blockwise-state step (opt2s_step_8bit) on one tensor of
     `numel` elements (by default fp32 Adam and bf16 AdEMAMix), timed beside
-    the 32-bit step on the same param/grad; and the mixed AdamW collection of
-    the eager protocol (2,000 tensors of 64..1,024 elements with fp32 state
-    plus 64 tensors of 4,096..65,536 elements with 8-bit state) in one
-    launch, L2 flushed before each step."""
+    the 32-bit step on the same param/grad, and with skip_zeros (a third
+    gradient buffer with every seventh element zero) when `skip_zeros`; and
+    the mixed AdamW collection of the eager protocol (2,000 tensors of
+    64..1,024 elements with fp32 state plus 64 tensors of 4,096..65,536
+    elements with 8-bit state) in one launch, L2 flushed before each step."""
     import torch
     from elementwise_optimizer_b200 import binding as B
     from elementwise_optimizer_b200 import synth
@@ -1196,6 +1198,23 @@ def run_eightbit(numel=268_435_456, steps=50, warmup=10, algos=(("adam", "f32"),
         gbs = per * numel / (ms / 1e3) / 1e9
         row["eightbit"] = {"ms_mean": ms, "bytes_per_elem": per, "gbs": gbs, "frac": gbs / peak,
                            "elements_per_s": numel / (ms / 1e3)}
+        if skip_zeros:
+            gz = grads[0].clone()
+            gz[::7] = 0
+            lz = [lists[0], B.TensorList8.from_tensors([p], [gz], [q1], [q2], [a1], [a2])]
+            hz = B.make_hyper(algo, weight_decay=0.01, beta3=0.9999, alpha=5.0, skip_zeros=True)
+            t0 = warmup + steps
+            for t in range(1, warmup + 1):
+                B.opt2s_step_8bit(lz[t % 2], hz, t0 + t)
+            torch.cuda.synchronize()
+            ev[0].record()
+            for k in range(steps):
+                B.opt2s_step_8bit(lz[k % 2], hz, t0 + warmup + 1 + k)
+                ev[k + 1].record()
+            torch.cuda.synchronize()
+            msz = sum(ev[k].elapsed_time(ev[k + 1]) for k in range(steps)) / steps
+            row["eightbit_skip_zeros"] = {"ms_mean": msz, "grads": "alternately dense and every seventh zero"}
+            del gz, lz
         del q1, q2, a1, a2, lists
         s1 = torch.zeros((2 if two else 1) * numel, device=dev)
         s2 = torch.zeros(numel, device=dev)
