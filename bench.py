@@ -289,9 +289,28 @@ def small_collection_us(device, reps=200):
     us = sorted(a.elapsed_time(b) * 1e3 for a, b in times)
     launches = B.launch_count() - launches0
     q = lambda f: us[min(len(us) - 1, int(f * len(us)))]
+    # the protocol's floor: a one-element collection timed the same way (the
+    # events, the launch and cold data and instruction caches after the flush)
+    one = [torch.zeros(1, device=device) for _ in range(4)]
+    tl1 = B.TensorList.from_tensors([one[0]], [one[1]], [one[2]], [one[3]])
+    floor = []
+    for t in range(1, 6 + reps):
+        flush.fill_(float(t))
+        flush.sum()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        B.opt2s_step(tl1, d["hyper"], t)
+        b.record(stream)
+        if t > 5:
+            floor.append((a, b))
+    torch.cuda.synchronize()
+    fl = sorted(a.elapsed_time(b) * 1e3 for a, b in floor)
     return {"workload": w.name, "tensors": len(w.sizes), "numel": w.numel,
             "us_per_step_median": q(0.5), "us_per_step_p10": q(0.1), "us_per_step_p90": q(0.9),
-            "launches_per_step": launches / reps, "l2": "flushed before each step (256 MB written, then read)"}
+            "launches_per_step": launches / reps, "l2": "flushed before each step (256 MB written, then read)",
+            "protocol_floor_us_median": fl[len(fl) // 2],
+            "protocol_floor": "a one-element collection, same flush and events"}
 
 
 def single_small_us(device, reps=200):
